@@ -1,0 +1,211 @@
+"""Oracle for the quantized linear layer (test infrastructure only).
+
+Plain double-precision host C in ``bq_oracle.c``, wrapped here with ctypes
+and numpy for argument marshalling.  Only the tests, ``__graft_entry__.smoke``
+and the benchmark's CPU-baseline leg may import this package; the product
+path (``bit_quantized_linear_rmsnorm_b200``) never does, and the two share no
+code.  See ``bq_oracle.c`` for the page citations and the readings taken where
+the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# No fast-math and no contraction into fused multiply-add: every operation in
+# the oracle is one correctly rounded binary64 operation.
+CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math"]
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so with gcc if it is missing or older than its source."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+F64 = ctypes.c_double
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        sig = {
+            "bq_oracle_round_half_even": (F64, [F64]),
+            "bq_oracle_act_quant": (None, [P, I64, I64, F64, P, P, P, P, P]),
+            "bq_oracle_ternary_quant": (ctypes.c_int, [P, I64, I64, P, P, P]),
+            "bq_oracle_ternary_bake": (None, [P, F64, I64, P]),
+            "bq_oracle_ternary_pack": (None, [P, I64, I64, P]),
+            "bq_oracle_ternary_unpack": (I64, [P, I64, I64, P]),
+            "bq_oracle_int4_pack": (None, [P, I64, I64, P]),
+            "bq_oracle_int4_unpack": (None, [P, I64, I64, P]),
+            "bq_oracle_half_to_double": (F64, [ctypes.c_uint16]),
+            "bq_oracle_gemm_i8_pertoken": (I64, [P, I64, P, ctypes.c_int, I64, P, P, P, I64, I64, I64, P]),
+            "bq_oracle_bitlinear_from_codes": (None, [P, P, P, F64, P, I64, I64, I64, P, P]),
+            "bq_oracle_linear_w4_grouped": (None, [P, I64, I64, P, P, P, P, I64, I64, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(_lib, name)
+            fn.restype = res
+            fn.argtypes = args
+    return _lib
+
+
+def _c(a, dtype):
+    """Contiguous array of the given dtype (a copy only when needed)."""
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def round_half_even(v: float) -> float:
+    return lib().bq_oracle_round_half_even(float(v))
+
+
+def act_quant(x, eps: float = 1e-5, want_pre: bool = False, want_y: bool = False):
+    """RMSNorm + per-token absmax int8 quantization of x [M,K] (float32 values).
+
+    Returns dict with xq int8 [M,K], act_scale f64 [M], rowsum int64 [M] and,
+    when asked, the pre-rounding values ``pre`` and the normalised ``y``.
+    """
+    x = _c(x, np.float32)
+    M, K = x.shape
+    xq = np.empty((M, K), np.int8)
+    sc = np.empty(M, np.float64)
+    rs = np.empty(M, np.int64)
+    pre = np.empty((M, K), np.float64) if want_pre else None
+    y = np.empty((M, K), np.float64) if want_y else None
+    lib().bq_oracle_act_quant(_p(x), M, K, float(eps), _p(xq), _p(sc), _p(rs), _p(pre), _p(y))
+    out = {"xq": xq, "act_scale": sc, "rowsum": rs}
+    if want_pre:
+        out["pre"] = pre
+    if want_y:
+        out["y"] = y
+    return out
+
+
+def ternary_quant(w, want_pre: bool = False):
+    """Absmean ternary quantization with the bake rule; w float32 [N,K]."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    g = np.zeros(1, np.float64)
+    wq = np.empty((N, K), np.int8)
+    pre = np.empty((N, K), np.float64) if want_pre else None
+    baked = lib().bq_oracle_ternary_quant(_p(w), N, K, _p(g), _p(wq), _p(pre))
+    out = {"wq": wq, "gamma": float(g[0]), "already_ternary": bool(baked)}
+    if want_pre:
+        out["pre"] = pre
+    return out
+
+
+def ternary_bake(wq, gamma: float):
+    wq = _c(wq, np.int8)
+    out = np.empty(wq.shape, np.float32)
+    lib().bq_oracle_ternary_bake(_p(wq), float(gamma), wq.size, _p(out))
+    return out
+
+
+def ternary_pack(wq):
+    wq = _c(wq, np.int8)
+    N, K = wq.shape
+    assert K % 16 == 0
+    out = np.empty((N, K // 16), np.uint32)
+    lib().bq_oracle_ternary_pack(_p(wq), N, K, _p(out))
+    return out
+
+
+def ternary_unpack(packed, K: int):
+    packed = _c(packed, np.uint32)
+    N = packed.shape[0]
+    wq = np.empty((N, K), np.int8)
+    bad = lib().bq_oracle_ternary_unpack(_p(packed), N, K, _p(wq))
+    return wq, int(bad)
+
+
+def int4_pack(q):
+    q = _c(q, np.uint8)
+    rows, cols = q.shape
+    out = np.empty((rows, (cols + 7) // 8), np.uint32)
+    lib().bq_oracle_int4_pack(_p(q), rows, cols, _p(out))
+    return out
+
+
+def int4_unpack(packed, cols: int):
+    packed = _c(packed, np.uint32)
+    rows = packed.shape[0]
+    q = np.empty((rows, cols), np.uint8)
+    lib().bq_oracle_int4_unpack(_p(packed), rows, cols, _p(q))
+    return q
+
+
+def half_to_double(bits: int) -> float:
+    return lib().bq_oracle_half_to_double(int(bits) & 0xFFFF)
+
+
+def gemm_i8_pertoken(x, w, deq_scale, per_token_scale, bias=None, layout: int = 0):
+    """acc = x @ weight, out = acc * deqScale[n] * perTokenScale[m] (+ bias[n]).
+
+    x int8 [M,K]; w int8 [N,K] (layout 0) or [K,N] (layout 1).  Returns
+    (out f64 [M,N], number of accumulators outside int32).
+    """
+    x = _c(x, np.int8)
+    w = _c(w, np.int8)
+    M, K = x.shape
+    N = w.shape[0] if layout == 0 else w.shape[1]
+    deq = _c(deq_scale, np.float32)
+    pts = _c(per_token_scale, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((M, N), np.float64)
+    ovf = lib().bq_oracle_gemm_i8_pertoken(_p(x), K, _p(w), int(layout), w.shape[1], _p(deq), _p(pts),
+                                           _p(b), M, N, K, _p(out))
+    return out, int(ovf)
+
+
+def bitlinear_from_codes(xq, act_scale, wq, gamma: float, bias=None, want_acc: bool = False):
+    xq = _c(xq, np.int8)
+    wq = _c(wq, np.int8)
+    sc = _c(act_scale, np.float64)
+    M, K = xq.shape
+    N = wq.shape[0]
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((M, N), np.float64)
+    acc = np.empty((M, N), np.int64) if want_acc else None
+    lib().bq_oracle_bitlinear_from_codes(_p(xq), _p(sc), _p(wq), float(gamma), _p(b), M, N, K, _p(out), _p(acc))
+    return (out, acc) if want_acc else out
+
+
+def bitlinear(x, w, eps: float = 1e-5, bias=None):
+    """Whole BitLinear forward: act quant, ternary quant, integer linear, rescale."""
+    a = act_quant(x, eps)
+    t = ternary_quant(w)
+    out = bitlinear_from_codes(a["xq"], a["act_scale"], t["wq"], t["gamma"], bias)
+    return out, a, t
+
+
+def linear_w4_grouped(x, qweight, scales_f16_bits, qzeros, bias, group_size: int):
+    x = _c(x, np.float32)
+    M, K = x.shape
+    qw = _c(qweight, np.uint32)
+    N = qw.shape[0]
+    sc = _c(scales_f16_bits, np.uint16)
+    qz = _c(qzeros, np.uint32)
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((M, N), np.float64)
+    lib().bq_oracle_linear_w4_grouped(_p(x), M, K, _p(qw), _p(sc), _p(qz), _p(b), N, int(group_size), _p(out))
+    return out

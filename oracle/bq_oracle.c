@@ -1,0 +1,331 @@
+/*
+ * Oracle for the quantized linear layer: plain, slow, obviously correct host C.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the tests, the package's smoke check and the timed
+ * CPU baseline of the benchmark use it.  It shares no code, header, table or
+ * constant with the CUDA library; the two only meet through the seeded input
+ * generator, which holds none of the arithmetic below.
+ *
+ * Every routine works in double precision (IEEE binary64), uses no blocking,
+ * no reordering and no fused multiply-add (build with -ffp-contract=off), and
+ * follows the pages it cites step by step:
+ *
+ *   [BitLinear]  "Class BitLinear" (LLaMA-BitNet utils.py), class docstring
+ *                "Forward pass (training)" steps 1-5 and forward().
+ *   [common]     "Common Attention Utilities" (frankenstein-transformer
+ *                src.model.attention.common): activation_quant, weight_quant,
+ *                BitLinear.bake_ternary_weights.
+ *   [ATB]        "Per-token Quantization for Matmul" (Huawei CANN ATB):
+ *                Input / Output tables and the Example.
+ *   [linear_4bit] "vyre_libs/nn/linear/inner/linear_4bit/mod.rs" (docs.rs
+ *                vyre-libs 0.7.2): module doc, QuantizedLinear4BitSpec.
+ *
+ * Readings taken where the pages are silent (each is also listed in the
+ * design notes): RMSNorm puts eps inside the square root; the activation
+ * scale maps the row's absolute maximum to 127; absmax and absmean are
+ * clamped below at 1e-5; rounding is half-to-even; the ternary code is stored
+ * offset-binary (w+1) two bits per weight; INT4 nibbles are packed low-nibble
+ * first along the reduction axis; the INT4 affine form is s*(q - z).
+ *
+ * Pins: every function here is checked by the CPU test-suite against values
+ * the pages print (the ATB example), closed forms, invariants and library
+ * routines on special cases.  The BitLinear composition is pinned only
+ * through its steps plus closed-form special cases.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_ABSMAX_FLOOR 1e-5   /* absmax / absmean lower clamp            */
+#define ORACLE_ACT_QMAX 127.0      /* int8 activations scaled to +-127        */
+
+/* Round half to even, written out: floor, then compare the remainder. */
+double bq_oracle_round_half_even(double v)
+{
+    double f = floor(v);
+    double d = v - f; /* exact for |v| < 2^52 */
+    if (d > 0.5) return f + 1.0;
+    if (d < 0.5) return f;
+    return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+static double clampd(double v, double lo, double hi)
+{
+    return v < lo ? lo : (v > hi ? hi : v);
+}
+
+/*
+ * Per-token activation quantization after a parameter-free RMSNorm.
+ * [BitLinear] steps 1-2 (internal RMSNorm, 8-bit per-token quantization);
+ * [common] activation_quant (per-token scale over the last dimension into
+ * [-128, 127], round to integer).
+ *
+ *   r[m]        = sqrt( (1/K) sum_k x[m,k]^2 + eps )
+ *   y[m,k]      = x[m,k] / r[m]
+ *   a[m]        = max( max_k |y[m,k]|, 1e-5 )
+ *   pre[m,k]    = y[m,k] * 127 / a[m]              (pre-rounding value)
+ *   xq[m,k]     = clamp( round_half_even(pre), -128, 127 )
+ *   act_scale[m]= a[m] / 127                       (multiplied back in step 5)
+ *   rowsum[m]   = sum_k xq[m,k]
+ *
+ * x is read as float (bf16 inputs are passed widened, which is exact).
+ * Optional outputs (pre, y, rowsum) may be NULL.  Dense row-major [M,K].
+ */
+void bq_oracle_act_quant(const float *x, int64_t M, int64_t K, double eps,
+                         int8_t *xq, double *act_scale, int64_t *rowsum,
+                         double *pre, double *y_out)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *xr = x + m * K;
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) ss += (double)xr[k] * (double)xr[k];
+        double r = sqrt(ss / (double)K + eps);
+
+        double amax = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double y = (double)xr[k] / r;
+            if (y_out) y_out[m * K + k] = y;
+            if (fabs(y) > amax) amax = fabs(y);
+        }
+        double a = amax > ORACLE_ABSMAX_FLOOR ? amax : ORACLE_ABSMAX_FLOOR;
+
+        int64_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            double y = (double)xr[k] / r;
+            double v = y * ORACLE_ACT_QMAX / a;
+            if (pre) pre[m * K + k] = v;
+            double q = clampd(bq_oracle_round_half_even(v), -128.0, 127.0);
+            xq[m * K + k] = (int8_t)q;
+            sum += (int64_t)q;
+        }
+        act_scale[m] = a / ORACLE_ACT_QMAX;
+        if (rowsum) rowsum[m] = sum;
+    }
+}
+
+/*
+ * Absmean ternary weight quantization with the bake rule.
+ * [BitLinear] step 3 (ternary {-1,0,+1} via absmean); [common] weight_quant
+ * (scale by the inverse mean absolute value, round to the nearest integer in
+ * [-1, 1]) and bake_ternary_weights (a weight whose nonzero entries all equal
+ * +-max|w| is already ternary and is left as it is, so its scale is max|w|).
+ *
+ *   if some w != 0 and every nonzero |w| == max|w| = c:   gamma = c
+ *   else:  gamma = max( (1/(N K)) sum |w|, 1e-5 )
+ *   pre = w / gamma;   wq = clamp( round_half_even(pre), -1, 1 )
+ *
+ * Returns 1 when the bake rule applied, 0 otherwise.  pre may be NULL.
+ */
+int bq_oracle_ternary_quant(const float *w, int64_t N, int64_t K, double *gamma,
+                            int8_t *wq, double *pre)
+{
+    int64_t n_el = N * K;
+    double c = 0.0;
+    for (int64_t i = 0; i < n_el; ++i)
+        if (fabs((double)w[i]) > c) c = fabs((double)w[i]);
+
+    int already_ternary = c > 0.0;
+    for (int64_t i = 0; i < n_el && already_ternary; ++i) {
+        double aw = fabs((double)w[i]);
+        if (aw != 0.0 && aw != c) already_ternary = 0;
+    }
+
+    double g;
+    if (already_ternary) {
+        g = c;
+    } else {
+        double s = 0.0;
+        for (int64_t i = 0; i < n_el; ++i) s += fabs((double)w[i]);
+        g = s / (double)n_el;
+        if (g < ORACLE_ABSMAX_FLOOR) g = ORACLE_ABSMAX_FLOOR;
+    }
+    *gamma = g;
+
+    for (int64_t i = 0; i < n_el; ++i) {
+        double v = (double)w[i] / g;
+        if (pre) pre[i] = v;
+        wq[i] = (int8_t)clampd(bq_oracle_round_half_even(v), -1.0, 1.0);
+    }
+    return already_ternary;
+}
+
+/* bake(W) = wq * gamma, the weight that bake_ternary_weights stores. */
+void bq_oracle_ternary_bake(const int8_t *wq, double gamma, int64_t n_el, float *out)
+{
+    for (int64_t i = 0; i < n_el; ++i) out[i] = (float)((double)wq[i] * gamma);
+}
+
+/*
+ * Two-bit ternary packing (the pages fix no bit layout; this is the layout
+ * the library documents).  Row n of wq [N,K] becomes K/16 words; the code of
+ * element k = 16*w + 4*j + b is (wq + 1) in {0,1,2}, stored in bits
+ * [8*b + 2*j, 8*b + 2*j + 1] of word w.  K must be a multiple of 16.
+ */
+void bq_oracle_ternary_pack(const int8_t *wq, int64_t N, int64_t K, uint32_t *packed)
+{
+    int64_t words = K / 16;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t wi = 0; wi < words; ++wi) {
+            uint32_t word = 0;
+            for (int j = 0; j < 4; ++j)
+                for (int b = 0; b < 4; ++b) {
+                    int64_t k = 16 * wi + 4 * j + b;
+                    uint32_t code = (uint32_t)(wq[n * K + k] + 1);
+                    word |= code << (8 * b + 2 * j);
+                }
+            packed[n * words + wi] = word;
+        }
+}
+
+/* Inverse of bq_oracle_ternary_pack; returns the number of invalid codes (3). */
+int64_t bq_oracle_ternary_unpack(const uint32_t *packed, int64_t N, int64_t K, int8_t *wq)
+{
+    int64_t words = K / 16, bad = 0;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            int64_t wi = k / 16, j = (k % 16) / 4, b = k % 4;
+            uint32_t code = (packed[n * words + wi] >> (8 * b + 2 * j)) & 3u;
+            if (code == 3u) ++bad;
+            wq[n * K + k] = (int8_t)((int)code - 1);
+        }
+    return bad;
+}
+
+/*
+ * Nibble packing along the last axis, eight per 32-bit word ([linear_4bit]
+ * module doc: the kernel loads the packed u32 word and extracts the nibble
+ * for k).  Element c of a row sits in bits [4*(c%8), 4*(c%8)+3] of word c/8
+ * (low nibble first); a ragged last word is zero-padded.  Values must be
+ * 0..15.  Used for weights [N,K] and for zero-points [N,G].
+ */
+void bq_oracle_int4_pack(const uint8_t *q, int64_t rows, int64_t cols, uint32_t *packed)
+{
+    int64_t words = (cols + 7) / 8;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t wi = 0; wi < words; ++wi) {
+            uint32_t word = 0;
+            for (int j = 0; j < 8; ++j) {
+                int64_t c = 8 * wi + j;
+                if (c < cols) word |= ((uint32_t)q[r * cols + c] & 15u) << (4 * j);
+            }
+            packed[r * words + wi] = word;
+        }
+}
+
+void bq_oracle_int4_unpack(const uint32_t *packed, int64_t rows, int64_t cols, uint8_t *q)
+{
+    int64_t words = (cols + 7) / 8;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            q[r * cols + c] = (uint8_t)((packed[r * words + c / 8] >> (4 * (c % 8))) & 15u);
+}
+
+/*
+ * IEEE 754 binary16 bits to double, from the format's definition:
+ * sign, 5-bit exponent (bias 15), 10-bit fraction; exponent 0 is subnormal.
+ */
+double bq_oracle_half_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1, e = (h >> 10) & 31, f = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);
+    return sign ? -v : v;
+}
+
+/*
+ * Per-token W8A8 matmul with dequantization ([ATB] Input/Output tables and
+ * the Example, whose printed arithmetic fixes the formula):
+ *
+ *   acc[m,n] = sum_k x[m,k] * weight(k,n)          (exact, int64)
+ *   out[m,n] = (acc * deqScale[n]) * perTokenScale[m]  (+ bias[n])
+ *
+ * weight(k,n) = w[n*ldw + k] for layout 0 ([N,K], the nn.Linear layout,
+ * ATB transposeB = true) or w[k*ldw + n] for layout 1 ([K,N], the ATB
+ * default).  bias may be NULL.  out is dense [M,N].
+ * Returns the number of accumulators outside the int32 range (must be 0).
+ */
+int64_t bq_oracle_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w,
+                                   int layout, int64_t ldw, const float *deq_scale,
+                                   const float *per_token_scale, const float *bias,
+                                   int64_t M, int64_t N, int64_t K, double *out)
+{
+    int64_t overflow = 0;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t wv = layout == 0 ? w[n * ldw + k] : w[k * ldw + n];
+                acc += (int64_t)x[m * ldx + k] * wv;
+            }
+            if (acc > 2147483647LL || acc < -2147483648LL) ++overflow;
+            double v = ((double)acc * (double)deq_scale[n]) * (double)per_token_scale[m];
+            if (bias) v += (double)bias[n];
+            out[m * N + n] = v;
+        }
+    return overflow;
+}
+
+/*
+ * BitLinear steps 4-5 from the quantized operands ([BitLinear] forward:
+ * F.linear(x_q, w_q) then out * act_scale * w_scale):
+ *
+ *   out[m,n] = ((sum_k xq[m,k] * wq[n,k]) * act_scale[m]) * gamma  (+ bias[n])
+ *
+ * xq [M,K], wq [N,K] dense; bias may be NULL (the page disables it by
+ * default).  Also writes the exact integer accumulators when acc != NULL.
+ */
+void bq_oracle_bitlinear_from_codes(const int8_t *xq, const double *act_scale,
+                                    const int8_t *wq, double gamma, const float *bias,
+                                    int64_t M, int64_t N, int64_t K, double *out,
+                                    int64_t *acc_out)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += (int64_t)xq[m * K + k] * (int64_t)wq[n * K + k];
+            if (acc_out) acc_out[m * N + n] = acc;
+            double v = ((double)acc * act_scale[m]) * gamma;
+            if (bias) v += (double)bias[n];
+            out[m * N + n] = v;
+        }
+}
+
+/*
+ * Grouped affine INT4 linear ([linear_4bit] module doc: unpack-on-demand
+ * nibble extraction inside the k loop; grouped affine path with a scale and
+ * a zero-point per group, plus bias):
+ *
+ *   g = k / group_size
+ *   q = nibble k of row n of qweight [N, K/8];  z = nibble g of row n of
+ *   qzeros [N, ceil(G/8)];  s = scales[n, g] (binary16 bits)
+ *   out[m,n] = bias[n] + sum_k x[m,k] * s * (q - z)
+ *
+ * accumulated in double.  bias may be NULL.  out is dense [M,N].
+ */
+void bq_oracle_linear_w4_grouped(const float *x, int64_t M, int64_t K,
+                                 const uint32_t *qweight, const uint16_t *scales_f16,
+                                 const uint32_t *qzeros, const float *bias, int64_t N,
+                                 int64_t group_size, double *out)
+{
+    int64_t G = K / group_size;
+    int64_t wwords = K / 8, zwords = (G + 7) / 8;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double sum = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t g = k / group_size;
+                int q = (int)((qweight[n * wwords + k / 8] >> (4 * (k % 8))) & 15u);
+                int z = (int)((qzeros[n * zwords + g / 8] >> (4 * (g % 8))) & 15u);
+                double s = bq_oracle_half_to_double(scales_f16[n * G + g]);
+                sum += (double)x[m * K + k] * s * (double)(q - z);
+            }
+            out[m * N + n] = (bias ? (double)bias[n] : 0.0) + sum;
+        }
+}

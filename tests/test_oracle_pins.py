@@ -1,0 +1,305 @@
+"""Pins of the oracle to facts outside itself (CPU only).
+
+Each test checks the oracle against something it does not compute itself:
+values the pages print (the ATB worked example), closed forms, invariants the
+pages state, special cases that reduce to a library routine (numpy/torch in
+float64), and hand-worked golden words.  A plausible mistake in the oracle (a
+dropped eps, a wrong scale constant, a transposed operand, a wrong bit
+position, round-half-up instead of half-to-even) fails at least one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- rounding
+
+def test_round_half_even_ties():
+    cases = {0.5: 0.0, 1.5: 2.0, 2.5: 2.0, -0.5: 0.0, -1.5: -2.0, -2.5: -2.0,
+             126.5: 126.0, 127.5: 128.0, 0.49999999: 0.0, 0.50000001: 1.0, -3.7: -4.0}
+    for v, want in cases.items():
+        assert oracle.round_half_even(v) == want, v
+
+
+def test_round_half_even_matches_numpy_rint():
+    g = synth.rng(11)
+    v = np.concatenate([g.uniform(-300, 300, 2000), np.arange(-260, 260) + 0.5])
+    got = np.array([oracle.round_half_even(t) for t in v])
+    np.testing.assert_array_equal(got, np.rint(v))
+
+
+# ---------------------------------------------------------- activation quant
+
+def test_rmsnorm_matches_torch_rms_norm():
+    x = synth.normal_f32(synth.rng(1), (16, 300))
+    x[3] *= 1e-4  # a row where eps matters
+    eps = 1e-5
+    y = oracle.act_quant(x, eps, want_y=True)["y"]
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x).double(), (300,), eps=eps).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=0)
+
+
+def test_act_quant_invariants_random():
+    x = synth.normal_f32(synth.rng(2), (64, 512))
+    r = oracle.act_quant(x, 1e-5, want_pre=True)
+    xq, pre = r["xq"].astype(np.int64), r["pre"]
+    assert xq.min() >= -127 and xq.max() <= 127  # [-128,127] range; 127/absmax never reaches -128
+    am = np.argmax(np.abs(x), axis=1)
+    rows = np.arange(64)
+    np.testing.assert_array_equal(xq[rows, am], np.sign(x[rows, am]).astype(np.int64) * 127)
+    assert np.all(np.abs(xq - pre) <= 0.5 + 1e-12)  # rounding moves by at most half a step
+    np.testing.assert_array_equal(r["rowsum"], xq.sum(axis=1))
+    # dequantized value x_q * act_scale approximates the normalised y within half a step
+    y = oracle.act_quant(x, 1e-5, want_y=True)["y"]
+    assert np.all(np.abs(xq * r["act_scale"][:, None] - y) <= 0.5 * r["act_scale"][:, None] * (1 + 1e-12))
+
+
+def test_act_quant_codes_scale_invariant():
+    x = synth.normal_f32(synth.rng(3), (32, 256))
+    a = oracle.act_quant(x)["xq"]
+    b = oracle.act_quant(x * np.float32(8.0))["xq"]
+    c = oracle.act_quant(x * np.float32(0.25))["xq"]
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(a, c)
+
+
+@pytest.mark.parametrize("c", [1.0, -0.75, 3.0e-3, 250.0])
+def test_act_quant_constant_row_closed_form(c):
+    K, eps = 96, 1e-5
+    x = np.full((1, K), c, np.float32)
+    r = oracle.act_quant(x, eps)
+    cf = float(np.float32(c))
+    assert np.all(r["xq"] == (127 if c > 0 else -127))
+    want = 1.0 / (127.0 * math.sqrt(1.0 + eps / (cf * cf)))
+    assert r["act_scale"][0] == pytest.approx(want, rel=1e-14)
+
+
+def test_act_quant_one_hot_closed_form():
+    K, eps, j, c = 200, 1e-5, 37, -2.5
+    x = np.zeros((1, K), np.float32)
+    x[0, j] = c
+    r = oracle.act_quant(x, eps)
+    want_q = np.zeros(K, np.int8)
+    want_q[j] = -127
+    np.testing.assert_array_equal(r["xq"][0], want_q)
+    assert r["act_scale"][0] == pytest.approx(abs(c) / (127.0 * math.sqrt(c * c / K + eps)), rel=1e-14)
+    assert r["rowsum"][0] == -127
+
+
+def test_act_quant_zero_row():
+    r = oracle.act_quant(np.zeros((2, 64), np.float32))
+    assert np.all(r["xq"] == 0)
+    np.testing.assert_array_equal(r["act_scale"], np.full(2, 1e-5 / 127.0))
+
+
+# ------------------------------------------------------------ ternary quant
+
+def test_ternary_hand_cases(golden_dir):
+    d = _load(golden_dir, "ternary_hand_cases.json")
+    for case in d["cases"]:
+        w = np.array(case["w"], np.float32)
+        t = oracle.ternary_quant(w)
+        np.testing.assert_array_equal(t["wq"], np.array(case["wq"], np.int8), err_msg=case["name"])
+        assert t["already_ternary"] == case["already_ternary"], case["name"]
+        tol = case["gamma_rel_tol"]
+        assert abs(t["gamma"] - case["gamma"]) <= tol * case["gamma"], case["name"]
+
+
+def test_ternary_invariants_and_statistics():
+    sigma = 0.02
+    w = synth.normal_f32(synth.rng(4), (1024, 1024), sigma)
+    t = oracle.ternary_quant(w, want_pre=True)
+    assert set(np.unique(t["wq"]).tolist()) <= {-1, 0, 1}
+    # gamma -> sigma * sqrt(2/pi) for a normal weight; zero fraction -> erf(0.5/sqrt(pi))
+    assert t["gamma"] == pytest.approx(sigma * math.sqrt(2 / math.pi), rel=5e-3)
+    zero_frac = float(np.mean(t["wq"] == 0))
+    assert zero_frac == pytest.approx(math.erf(0.5 / math.sqrt(math.pi)), abs=3e-3)
+    # codes agree with sign and the 0.5 threshold of the pre-rounding value
+    pre = t["pre"]
+    want = np.where(pre > 0.5, 1, np.where(pre < -0.5, -1, 0))
+    np.testing.assert_array_equal(t["wq"], want)
+
+
+def test_ternary_bake_idempotent():
+    w = synth.normal_f32(synth.rng(5), (64, 128), 0.02)
+    t1 = oracle.ternary_quant(w)
+    baked = oracle.ternary_bake(t1["wq"], t1["gamma"])
+    t2 = oracle.ternary_quant(baked)
+    assert t2["already_ternary"]
+    np.testing.assert_array_equal(t2["wq"], t1["wq"])
+    assert t2["gamma"] == float(np.float32(t1["gamma"]))
+    np.testing.assert_array_equal(oracle.ternary_bake(t2["wq"], t2["gamma"]), baked)
+    # without the bake rule the scale would drift to gamma * (fraction nonzero)
+    nz = float(np.mean(t1["wq"] != 0))
+    assert abs(t2["gamma"] - t1["gamma"] * nz) > 0.1 * t1["gamma"]
+
+
+# ------------------------------------------------------------------ packing
+
+def test_ternary_pack_golden_words(golden_dir):
+    d = _load(golden_dir, "pack_words.json")
+    for case in d["ternary"]:
+        wq = np.array([case["wq"]], np.int8)
+        assert int(oracle.ternary_pack(wq)[0, 0]) == int(case["word"], 16)
+
+
+def test_ternary_pack_roundtrip():
+    g = synth.rng(6)
+    wq = g.integers(-1, 2, (37, 160)).astype(np.int8)
+    packed = oracle.ternary_pack(wq)
+    back, bad = oracle.ternary_unpack(packed, 160)
+    assert bad == 0
+    np.testing.assert_array_equal(back, wq)
+
+
+def test_int4_pack_golden_words(golden_dir):
+    d = _load(golden_dir, "pack_words.json")
+    for case in d["int4"]:
+        q = np.array([case["q"]], np.uint8)
+        assert int(oracle.int4_pack(q)[0, 0]) == int(case["word"], 16)
+
+
+def test_int4_pack_roundtrip():
+    q = synth.nibbles(synth.rng(7), (19, 77))
+    np.testing.assert_array_equal(oracle.int4_unpack(oracle.int4_pack(q), 77), q)
+
+
+def test_half_decode_matches_numpy_all_patterns():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    finite = np.isfinite(ref)
+    np.testing.assert_array_equal(got[finite], ref[finite])
+    assert np.all(np.isnan(got[np.isnan(ref)]))
+    assert np.all(got[np.isinf(ref)] == ref[np.isinf(ref)])
+
+
+# ------------------------------------------------------------------- W8A8
+
+def test_gemm_atb_worked_example(golden_dir):
+    d = _load(golden_dir, "atb_per_token_example.json")
+    x = np.array(d["x"], np.int8)
+    w = np.array(d["weight"], np.int8)  # [k, n]
+    out, ovf = oracle.gemm_i8_pertoken(x, w, np.array(d["deqScale"], np.float32),
+                                       np.array(d["perTokenScale"], np.float32), layout=1)
+    assert ovf == 0
+    np.testing.assert_array_equal(out, np.array(d["output"], np.float64))
+    # the same numbers with the weight in the nn.Linear [n, k] layout
+    out_nk, _ = oracle.gemm_i8_pertoken(x, w.T.copy(), np.array(d["deqScale"], np.float32),
+                                        np.array(d["perTokenScale"], np.float32), layout=0)
+    np.testing.assert_array_equal(out_nk, out)
+
+
+def test_gemm_unit_scales_is_integer_matmul():
+    g = synth.rng(8)
+    x, w = synth.int8_uniform(g, (23, 70)), synth.int8_uniform(g, (31, 70))
+    out, _ = oracle.gemm_i8_pertoken(x, w, np.ones(31, np.float32), np.ones(23, np.float32))
+    np.testing.assert_array_equal(out, (x.astype(np.int64) @ w.astype(np.int64).T).astype(np.float64))
+
+
+def test_gemm_scales_and_bias_match_numpy():
+    g = synth.rng(9)
+    x, w = synth.int8_uniform(g, (17, 45)), synth.int8_uniform(g, (29, 45))
+    deq, pts = synth.uniform_f32(g, (29,), 0.001, 0.01), synth.uniform_f32(g, (17,), 0.001, 0.01)
+    bias = synth.normal_f32(g, (29,), 0.1)
+    out, _ = oracle.gemm_i8_pertoken(x, w, deq, pts, bias)
+    acc = (x.astype(np.int64) @ w.astype(np.int64).T).astype(np.float64)
+    ref = pts.astype(np.float64)[:, None] * acc * deq.astype(np.float64)[None, :] + bias.astype(np.float64)
+    np.testing.assert_allclose(out, ref, rtol=1e-15, atol=1e-15)
+    # layout [K,N] with the transposed weight gives identical results
+    out_kn, _ = oracle.gemm_i8_pertoken(x, w.T.copy(), deq, pts, bias, layout=1)
+    np.testing.assert_array_equal(out_kn, out)
+
+
+def test_gemm_reports_int32_overflow():
+    # (-128)*(-128) = 2^14 per term: K = 2^17 terms reach 2^31, one past INT32_MAX
+    K = 131072
+    x = np.full((1, K), -128, np.int8)
+    w = np.full((1, K), -128, np.int8)
+    _, ovf = oracle.gemm_i8_pertoken(x, w, np.ones(1, np.float32), np.ones(1, np.float32))
+    assert ovf == 1
+    _, ovf = oracle.gemm_i8_pertoken(x[:, :K - 1], w[:, :K - 1], np.ones(1, np.float32), np.ones(1, np.float32))
+    assert ovf == 0
+
+
+# -------------------------------------------------------------- BitLinear
+
+def test_bitlinear_constant_weight_closed_form():
+    # every weight equal to c is already ternary: gamma = c, codes all +1, so
+    # out[m,n] = c * act_scale[m] * rowsum(x_q)[m]
+    x = synth.normal_f32(synth.rng(10), (5, 64))
+    w = np.full((7, 64), 0.03, np.float32)
+    out, a, t = oracle.bitlinear(x, w)
+    assert t["already_ternary"] and t["gamma"] == float(np.float32(0.03))
+    want = t["gamma"] * a["act_scale"] * a["rowsum"].astype(np.float64)
+    np.testing.assert_allclose(out, np.repeat(want[:, None], 7, axis=1), rtol=1e-15)
+
+
+def test_bitlinear_matches_integer_matmul_of_codes():
+    d = synth.bitlinear_tiny(0)
+    out, a, t = oracle.bitlinear(d["x"], d["w"], d["eps"])
+    acc = a["xq"].astype(np.int64) @ t["wq"].astype(np.int64).T
+    ref = acc.astype(np.float64) * a["act_scale"][:, None] * t["gamma"]
+    np.testing.assert_allclose(out, ref, rtol=1e-15)
+    # dequantized result approximates the float linear of the normalised input
+    y = oracle.act_quant(d["x"], d["eps"], want_y=True)["y"]
+    dense = y @ (t["wq"].astype(np.float64) * t["gamma"]).T
+    assert np.max(np.abs(out - dense)) < 0.05 * np.max(np.abs(dense))
+
+
+# ----------------------------------------------------------------- INT4
+
+def _w4_case(g, M, N, K, gs):
+    q = synth.nibbles(g, (N, K))
+    z = synth.nibbles(g, (N, K // gs))
+    s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+    b = synth.normal_f32(g, (N,), 0.01)
+    x = synth.normal_f32(g, (M, K))
+    return x, q, z, s, b
+
+
+def test_w4_matches_dequantized_matmul():
+    g = synth.rng(12)
+    for (M, N, K, gs) in [(3, 20, 256, 128), (2, 9, 192, 64), (1, 5, 64, 64), (4, 11, 96, 8)]:
+        x, q, z, s, b = _w4_case(g, M, N, K, gs)
+        out = oracle.linear_w4_grouped(x, oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), b, gs)
+        deq = np.repeat(s.astype(np.float64), gs, axis=1) * (q.astype(np.float64) - np.repeat(z, gs, axis=1))
+        ref = x.astype(np.float64) @ deq.T + b.astype(np.float64)
+        np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_w4_zero_point_equal_code_gives_bias():
+    g = synth.rng(13)
+    N, K, gs = 6, 128, 32
+    z = synth.nibbles(g, (N, K // gs))
+    q = np.repeat(z, gs, axis=1)
+    s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+    b = synth.normal_f32(g, (N,), 0.01)
+    out = oracle.linear_w4_grouped(synth.normal_f32(g, (3, K)), oracle.int4_pack(q), s.view(np.uint16),
+                                   oracle.int4_pack(z), b, gs)
+    np.testing.assert_array_equal(out, np.repeat(b.astype(np.float64)[None, :], 3, axis=0))
+
+
+def test_w4_one_hot_gathers_x():
+    g = synth.rng(14)
+    N, K, gs = 8, 64, 16
+    cols = g.integers(0, K, N)
+    q = np.zeros((N, K), np.uint8)
+    q[np.arange(N), cols] = 1
+    z = np.zeros((N, K // gs), np.uint8)
+    s = np.ones((N, K // gs), np.float16)
+    x = synth.normal_f32(g, (2, K))
+    out = oracle.linear_w4_grouped(x, oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), None, gs)
+    np.testing.assert_array_equal(out, x[:, cols].astype(np.float64))
