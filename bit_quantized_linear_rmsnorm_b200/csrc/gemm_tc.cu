@@ -1,0 +1,488 @@
+// Integer GEMMs on the sm_100a tensor cores (tcgen05.mma kind::i8) with a
+// fused dequantizing epilogue.
+//
+//  * W8A8 per-token ("Per-token Quantization for Matmul", Huawei CANN ATB:
+//    Input/Output tables and the Example):
+//        out[m,n] = (float(acc) * deqScale[n]) * perTokenScale[m] (+ bias[n])
+//    with the weight either [N][K] (K-major) or [K][N] (N-major operand).
+//  * W2A8 BitLinear prefill ("Class BitLinear", LLaMA-BitNet utils.py,
+//    forward steps 4-5): the weight arrives as 2-bit offset-binary codes;
+//    unpack warps expand each TMA-staged packed tile to u8 codes in the
+//    swizzled shared-memory layout the MMA reads, so no int8 copy of the
+//    weight ever exists in global memory.  acc(codes) - rowsum(xq) is the
+//    exact ternary accumulator:
+//        out[m,n] = (float(acc - rowsum[m]) * act_scale[m]) * gamma (+ bias[n])
+//
+// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
+//   warp 0      TMA producer: A tile (128 x 128 B) and B tile (256 x 128 B, or
+//               the 256 x 32 B packed tile) per stage, mbarrier tx-count.
+//   warp 1      MMA issuer: one thread issues 4 x tcgen05.mma (K = 32 each)
+//               per stage into a TMEM accumulator, commits to free the stage.
+//   warp 2      allocates / frees 512 TMEM columns (two 256-column
+//               accumulators, so the epilogue of tile t overlaps tile t+1).
+//   warps 4-7   epilogue: tcgen05.ld 32 columns at a time (warp w reads TMEM
+//               lanes 32*(w%4)..), scale in fp32, round once, stage through a
+//               64-byte-swizzled buffer, TMA store (out-of-range rows/cols are
+//               clipped by the TMA unit).
+//   warps 8-11  (W2A8 only) unpack 2-bit codes into the B stage.
+// Every mbarrier wait is bounded; on expiry the kernel records
+// BQ_ERR_TIMEOUT in the status word, drains its own async work and exits.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include "bq_common.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;  // K bytes per stage = one 128-byte swizzle row
+constexpr int UMMA_K = 32;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t A_BYTES = BM * BK;           // 16 KB
+constexpr uint32_t B_BYTES = BN * BK;           // 32 KB
+constexpr uint32_t P_BYTES = BN * (BK / 16) * 4;  // 8 KB packed 2-bit tile
+constexpr uint32_t STG_BYTES = BM * 64;         // 8 KB epilogue staging buffer
+
+template <bool PACKED>
+struct Cfg {
+    static constexpr int kStages = PACKED ? 3 : 4;
+    static constexpr int kThreads = PACKED ? 384 : 256;
+    static constexpr uint32_t OFF_A = 0;
+    static constexpr uint32_t OFF_B = OFF_A + kStages * A_BYTES;
+    static constexpr uint32_t OFF_P = OFF_B + kStages * B_BYTES;
+    static constexpr uint32_t OFF_STG = OFF_P + (PACKED ? kStages * P_BYTES : 0);
+    static constexpr uint32_t OFF_VEC = OFF_STG + 2 * STG_BYTES;   // colscale[BN], bias[BN]
+    static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * BN * 4;
+    // barriers: full[S], empty[S], bready[S], tfull[2], tempty[2], drain
+    static constexpr uint32_t NBAR = 3 * kStages + 5;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;      // tmem base, abort flag
+    static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;         // + alignment slack
+};
+
+struct GemmDev {
+    const float *colscale;
+    const float *rowscale;
+    const int32_t *rowcorr;
+    const float *bias;
+    int M, N, K;
+    uint32_t *status;
+};
+
+template <typename OutT>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Shared-memory descriptor of the N-major B tile (TMA box 128 N x 128 K,
+// 128-byte swizzle): K rows 128 bytes apart, 8-row groups 1024 bytes apart
+// (stride byte offset), the second 128-wide N half 16 KB further (leading
+// byte offset).
+__device__ __forceinline__ uint64_t smem_desc_mnmajor_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3fffu);
+    d |= static_cast<uint64_t>((BK * 128u) >> 4) << 16;  // leading byte offset: next 128-wide N block
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;        // stride byte offset: next 8 K rows
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
+template <bool PACKED, bool B_KN, typename OutT>
+__global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const GemmDev p) {
+    using C = Cfg<PACKED>;
+    constexpr int S = C::kStages;
+    constexpr int CC = 64 / static_cast<int>(sizeof(OutT));  // output columns per staging chunk
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+    auto bready = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    auto tfull = [&](int b) { return bar0 + 8u * (3 * S + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (3 * S + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    int *epi_fail = reinterpret_cast<int *>(smem + C::OFF_MISC + 8);
+    float *vcol = reinterpret_cast<float *>(smem + C::OFF_VEC);
+    float *vbias = vcol + BN;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int num_m = (p.M + BM - 1) / BM;
+    const int num_n = (p.N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int nkb = (p.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+            mbar_init(bready(s), 128);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *epi_fail = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmO);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------------ producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            const int m0 = (tile % num_m) * BM;
+            const int n0 = (tile / num_m) * BN;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t a_dst = sbase + C::OFF_A + stage * A_BYTES;
+                if constexpr (PACKED) {
+                    mbar_arrive_expect_tx(full(stage), A_BYTES + P_BYTES);
+                    tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
+                    tma_load_2d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * (BK / 16), n0, full(stage));
+                } else if constexpr (B_KN) {
+                    mbar_arrive_expect_tx(full(stage), A_BYTES + B_BYTES);
+                    tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
+                    const uint32_t b_dst = sbase + C::OFF_B + stage * B_BYTES;
+                    tma_load_2d(b_dst, &tmB, n0, kb * BK, full(stage));
+                    tma_load_2d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, full(stage));
+                } else {
+                    mbar_arrive_expect_tx(full(stage), A_BYTES + B_BYTES);
+                    tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
+                    tma_load_2d(sbase + C::OFF_B + stage * B_BYTES, &tmB, kb * BK, n0, full(stage));
+                }
+                ++issued;
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            // let the copies already issued land before the CTA goes away
+            for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i) {
+                const uint32_t bar = full(static_cast<int>(i % S));
+                const uint32_t par = static_cast<uint32_t>((i / S) & 1);
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(bar, par) && globaltimer_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_i8(BM, BN, true, !PACKED, B_KN);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+            const int abuf = t & 1;
+            const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
+            if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tbase + static_cast<uint32_t>(abuf * BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                    ok = false;
+                    break;
+                }
+                if constexpr (PACKED) {
+                    if (!mbar_wait(bready(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                tc_fence_after();
+                const uint32_t a_addr = sbase + C::OFF_A + stage * A_BYTES;
+                const uint32_t b_addr = sbase + C::OFF_B + stage * B_BYTES;
+#pragma unroll
+                for (int ks = 0; ks < BK / UMMA_K; ++ks) {
+                    const uint64_t ad = smem_desc_kmajor_sw128(a_addr + ks * UMMA_K);
+                    const uint64_t bd = B_KN ? smem_desc_mnmajor_sw128(b_addr + ks * UMMA_K * 128)
+                                             : smem_desc_kmajor_sw128(b_addr + ks * UMMA_K);
+                    tc_mma_i8(d_tmem, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                }
+                tc_commit(empty(stage));
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit(tfull(abuf));
+        }
+        if (!ok) {
+            // wait until every MMA issued so far has completed
+            tc_commit(drain);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp - 4;  // TMEM lane quarter
+        const int r = 32 * q + lane;
+        const int et = threadIdx.x - 128;  // 0..127
+        uint8_t *stg = smem + C::OFF_STG;
+        const float colscale_scalar = PACKED ? __ldg(p.colscale) : 0.0f;
+        uint32_t chunk_ctr = 0;
+        int t = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
+            const int m0 = (tile % num_m) * BM;
+            const int n0 = (tile / num_m) * BN;
+            const int abuf = t & 1;
+            const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
+
+            named_bar_sync(1, 128);  // previous tile finished reading vcol / vbias
+            for (int i = et; i < BN; i += 128) {
+                const int n = n0 + i;
+                vcol[i] = (!PACKED && n < p.N) ? __ldg(p.colscale + n) : 0.0f;
+                vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+            }
+            named_bar_sync(1, 128);
+
+            // The 128 epilogue threads take the same decision, so none is left
+            // alone at a named barrier: each waits (time-bounded only), then
+            // they agree through a shared flag.
+            const bool ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE);
+            if (!ok) {
+                atomicOr(epi_fail, 1);
+                *abort_flag = 1;
+            }
+            named_bar_sync(1, 128);
+            if (*reinterpret_cast<volatile int *>(epi_fail)) break;
+            tc_fence_after();
+            const int row = m0 + r;
+            const float rs = row < p.M ? __ldg(p.rowscale + row) : 0.0f;
+            const int corr = (p.rowcorr != nullptr && row < p.M) ? __ldg(p.rowcorr + row) : 0;
+
+#pragma unroll 1
+            for (int c32 = 0; c32 < BN / 32; ++c32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(abuf * BN + c32 * 32) +
+                                       (static_cast<uint32_t>(32 * q) << 16),
+                                   v);
+                tmem_wait_ld();
+                if (c32 == BN / 32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(tempty(abuf));
+                }
+                float f[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float a = static_cast<float>(static_cast<int>(v[j]) - corr);
+                    float o;
+                    if constexpr (PACKED)
+                        o = __fmul_rn(__fmul_rn(a, rs), colscale_scalar);
+                    else
+                        o = __fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs);
+                    f[j] = __fadd_rn(o, vbias[c32 * 32 + j]);
+                }
+                uint32_t w[32];
+                constexpr int kSub = sizeof(OutT) == 2 ? 1 : 2;  // 64-byte staging rows per 32 columns
+                if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w[j] = pack2<OutT>(f[2 * j], f[2 * j + 1]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(f[j]);
+                }
+#pragma unroll
+                for (int sc = 0; sc < kSub; ++sc) {
+                    const uint32_t sb = chunk_ctr & 1u;
+                    if (et == 0) bulk_wait_read<1>();
+                    named_bar_sync(1, 128);
+                    uint8_t *rowp = stg + sb * STG_BYTES + r * 64;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int pj = j ^ ((r >> 1) & 3);
+                        *reinterpret_cast<uint4 *>(rowp + pj * 16) =
+                            make_uint4(w[sc * 16 + 4 * j], w[sc * 16 + 4 * j + 1], w[sc * 16 + 4 * j + 2],
+                                       w[sc * 16 + 4 * j + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 128);
+                    if (et == 0) {
+                        tma_store_2d(&tmO, smem_u32(stg + sb * STG_BYTES), n0 + c32 * 32 + sc * CC, m0);
+                        bulk_commit();
+                    }
+                    ++chunk_ctr;
+                }
+            }
+        }
+        if (et == 0) bulk_wait_all();
+    } else if (PACKED && warp >= 8) {
+        // ------------------------------------------------------------ unpack 2-bit codes
+        const int ut = threadIdx.x - 256;  // 0..127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t *pk = reinterpret_cast<const uint32_t *>(smem + C::OFF_P + stage * P_BYTES);
+                uint8_t *bt = smem + C::OFF_B + stage * B_BYTES;
+#pragma unroll 4
+                for (int i = 0; i < (BN * 8) / 128; ++i) {
+                    const int idx = ut + 128 * i;
+                    const int n = idx >> 3, c = idx & 7;  // weight row, 16-element chunk of the 128-K slab
+                    const uint32_t u = pk[idx];
+                    const uint4 codes = make_uint4(u & 0x03030303u, (u >> 2) & 0x03030303u,
+                                                   (u >> 4) & 0x03030303u, (u >> 6) & 0x03030303u);
+                    *reinterpret_cast<uint4 *>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = codes;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(bready(stage));
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool PACKED, bool B_KN, typename OutT>
+bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+                   cudaStream_t s, const DevInfo &dev) {
+    using C = Cfg<PACKED>;
+    auto kern = gemm_tc_kernel<PACKED, B_KN, OutT>;
+    static bool attr_set[64] = {};  // once per device (also keeps later calls capture-safe)
+    if (!attr_set[dev.device]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
+            cudaSuccess)
+            return BQ_ERR_CUDA;
+        attr_set[dev.device] = true;
+    }
+    const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+    const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
+    GemmDev p;
+    p.colscale = g.colscale;
+    p.rowscale = g.rowscale;
+    p.rowcorr = g.rowcorr;
+    p.bias = g.bias;
+    p.M = static_cast<int>(g.M);
+    p.N = static_cast<int>(g.N);
+    p.K = static_cast<int>(g.K);
+    p.status = dev.status;
+    kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mO, p);
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+template <typename OutT>
+bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+                   cudaStream_t s, const DevInfo &dev) {
+    if (g.b_packed2) return launch_t<true, false, OutT>(g, mA, mB, mO, s, dev);
+    if (g.b_layout == BQ_W_KN) return launch_t<false, true, OutT>(g, mA, mB, mO, s, dev);
+    return launch_t<false, false, OutT>(g, mA, mB, mO, s, dev);
+}
+
+}  // namespace
+
+bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) {
+    CUtensorMap mA, mB, mO;
+    if (!make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.K, g.M, g.lda, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BQ_ERR_CUDA;
+    bool okB;
+    if (g.b_packed2)
+        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    else if (g.b_layout == BQ_W_KN)
+        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.N, g.K, g.ldb, 128, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+    else
+        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!okB) return BQ_ERR_CUDA;
+    CUtensorMapDataType odt = g.out_dtype == BQ_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                              : g.out_dtype == BQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const int esz = g.out_dtype == BQ_F32 ? 4 : 2;
+    if (!make_map(&mO, odt, g.out, g.N, g.M, g.ldo * esz, 64 / esz, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+        return BQ_ERR_CUDA;
+    switch (g.out_dtype) {
+        case BQ_F32:
+            return dispatch<float>(g, mA, mB, mO, s, dev);
+        case BQ_F16:
+            return dispatch<__half>(g, mA, mB, mO, s, dev);
+        default:
+            return dispatch<__nv_bfloat16>(g, mA, mB, mO, s, dev);
+    }
+}
+
+}  // namespace bq

@@ -1,0 +1,221 @@
+/*
+ * bq.h - C ABI of libbq.so, a B200 (sm_100a) implementation of the quantized
+ * linear layer: per-token int8 activation quantization after a
+ * parameter-free RMSNorm, ternary (absmean) or grouped affine INT4 weights,
+ * and integer matmuls with a fused dequantizing epilogue.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensor pointers are device pointers owned by the caller.  The library
+ *    never allocates, frees or synchronizes: scratch memory is the caller's
+ *    `workspace`, sized with bq_workspace_bytes().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) on the calling thread's current device.
+ *  - Matrices are row-major.  Leading dimensions (ld*) count elements.
+ *    Unless a call says otherwise, base pointers must be 16-byte aligned and
+ *    ld * element size must be a multiple of 16 bytes (TMA and vector-load
+ *    requirement); a violation returns BQ_ERR_MISALIGNED.
+ *  - Arguments are validated before anything is launched; an invalid call
+ *    returns a status != BQ_OK and leaves every output untouched.  M == 0 or
+ *    N == 0 is a valid empty call (BQ_OK, nothing launched); K must be >= 1.
+ *  - A CUDA error raised by a launch is returned as BQ_ERR_CUDA.
+ *  - Kernels bound every wait they perform.  A wait that runs out (it cannot
+ *    happen with a correct build) or an invalid value met inside a kernel
+ *    (a nibble > 15) is recorded in a per-device status word and the kernel
+ *    returns early; read and clear it with bq_device_status().
+ *  - Inputs must be finite.  Rounding is to nearest, ties to even.
+ *
+ * Data formats
+ * ------------
+ *  - Ternary weights (bq_weight_quant_ternary_pack, bq_bitlinear_w2a8):
+ *    uint32 wpacked[N][K/16].  Element k = 16*w + 4*j + b of row n has the
+ *    offset-binary code (w_q + 1) in {0,1,2} in bits [8b+2j, 8b+2j+1] of
+ *    word w, so (word >> 2j) & 0x03030303 yields the codes of k = 16w+4j+0..3
+ *    as four bytes.  One fp32 scale gamma per tensor.
+ *  - INT4 weights (bq_weight_pack_int4_grouped, bq_linear_w4_grouped):
+ *    uint32 qweight[N][K/8], element k of row n in bits [4*(k%8), 4*(k%8)+3]
+ *    of word k/8 (low nibble first); zero-points uint32 qzeros[N][ceil(G/8)]
+ *    packed the same way along the group axis (G = K / group_size, ragged
+ *    last word zero-padded); scales IEEE binary16 [N][G]; dequantized weight
+ *    w[n,k] = scale[n,g] * (q[n,k] - zero[n,g]) with g = k / group_size.
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *bq_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    BQ_OK = 0,
+    BQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad enum, value out of range */
+    BQ_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. no sm_100 device)   */
+    BQ_ERR_MISALIGNED = 3,  /* pointer / leading-dimension alignment rule broken   */
+    BQ_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required          */
+    BQ_ERR_CUDA = 5,        /* a CUDA runtime / driver call failed                 */
+    BQ_ERR_TIMEOUT = 6      /* (device status only) a bounded wait ran out         */
+} bq_status;
+
+typedef enum { BQ_F32 = 0, BQ_BF16 = 1, BQ_F16 = 2 } bq_dtype;
+
+typedef enum {
+    BQ_W_NK = 0, /* weight [N][K], K contiguous: nn.Linear layout (ATB transposeB = true) */
+    BQ_W_KN = 1  /* weight [K][N], N contiguous: the ATB operator's default layout        */
+} bq_wlayout;
+
+typedef enum {
+    BQ_OP_ACT_QUANT_INT8 = 0,
+    BQ_OP_WEIGHT_QUANT_TERNARY_PACK = 1,
+    BQ_OP_WEIGHT_PACK_INT4_GROUPED = 2,
+    BQ_OP_GEMM_I8_PERTOKEN = 3,
+    BQ_OP_BITLINEAR_W2A8 = 4,
+    BQ_OP_LINEAR_W4_GROUPED = 5
+} bq_op;
+
+/*
+ * Per-token int8 activation quantization after a parameter-free RMSNorm.
+ * Source: "Class BitLinear" (LLaMA-BitNet utils.py), forward steps 1-2, and
+ * "Common Attention Utilities" (frankenstein-transformer), activation_quant.
+ *
+ *   r[m] = sqrt(mean_k x[m,k]^2 + eps),  a[m] = max(max_k |x[m,k]| / r[m], 1e-5)
+ *   xq[m,k] = clamp(rne(x[m,k] / r[m] * 127 / a[m]), -128, 127)   (|xq| <= 127)
+ *   act_scale[m] = a[m] / 127,   rowsum[m] = sum_k xq[m,k]
+ *
+ * x: [M][ldx] of x_dtype BQ_F32 or BQ_BF16 (row base 16-byte aligned when
+ * ldx*size % 16 == 0; any K >= 1).  xq: int8 [M][ldq], 16-byte aligned,
+ * ldq % 16 == 0, ldq >= K.  act_scale: fp32 [M].  rowsum: int32 [M] or NULL.
+ */
+bq_status bq_act_quant_int8(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, int64_t ldx,
+                            float eps, int8_t *xq, int64_t ldq, float *act_scale, int32_t *rowsum,
+                            bq_stream_t stream);
+
+/*
+ * Absmean ternary quantization and 2-bit packing of a weight matrix.
+ * Source: "Common Attention Utilities", weight_quant and
+ * BitLinear.bake_ternary_weights; "Class BitLinear", forward step 3.
+ *
+ *   gamma = max|w| if w has a nonzero entry and every nonzero |w| equals
+ *           max|w| (already ternary: the bake rule keeps it unchanged);
+ *           otherwise max(mean|w|, 1e-5), the mean taken in fp64.
+ *   w_q = clamp(rne(w / gamma), -1, 1);  wpacked as in "Data formats".
+ *
+ * w: dense [N][K] of w_dtype BQ_F32 or BQ_BF16, 16-byte aligned; K % 16 == 0.
+ * wpacked: uint32 [N][K/16], 16-byte aligned.  w_scale: one fp32 on the
+ * device (written without a host round trip).  workspace: at least
+ * bq_workspace_bytes(BQ_OP_WEIGHT_QUANT_TERNARY_PACK, 0, N, K, 0) bytes,
+ * 256-byte aligned.  The result is deterministic (fixed reduction order).
+ */
+bq_status bq_weight_quant_ternary_pack(const void *w, bq_dtype w_dtype, int64_t N, int64_t K,
+                                       uint32_t *wpacked, float *w_scale, void *workspace,
+                                       size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Pack INT4 codes and zero-points into u32 words of eight nibbles.
+ * Source: "vyre_libs/nn/linear/inner/linear_4bit/mod.rs" (docs.rs vyre-libs),
+ * module doc (packed u32 weight, nibble extracted in the k loop) and
+ * QuantizedLinear4BitSpec (typed packed-word layout).
+ *
+ * q: uint8 [N][K] codes 0..15, K % 8 == 0.  zeros: uint8 [N][G] codes 0..15,
+ * G = K / group_size; group_size >= 1 divides K.  qweight: uint32 [N][K/8];
+ * qzeros: uint32 [N][ceil(G/8)].  All 4-byte aligned (q 8-byte aligned).
+ * A code > 15 is masked to its low nibble and flagged in the device status
+ * word as BQ_ERR_INVALID_ARG.
+ */
+bq_status bq_weight_pack_int4_grouped(const uint8_t *q, const uint8_t *zeros, int64_t N, int64_t K,
+                                      int64_t group_size, uint32_t *qweight, uint32_t *qzeros,
+                                      bq_stream_t stream);
+
+/*
+ * Per-token W8A8 matmul with a fused dequantizing epilogue.
+ * Source: "Per-token Quantization for Matmul" (Huawei CANN ATB), Input and
+ * Output tables and the Example (acc * deqScale[n] * perTokenScale[m]).
+ *
+ *   acc[m,n] = sum_k x[m,k] * w(k,n)   (exact int32; K <= 131071)
+ *   out[m,n] = (float(acc) * deq_scale[n]) * per_token_scale[m] (+ bias[n])
+ *
+ * x: int8 [M][ldx].  w: int8 [N][ldw] (BQ_W_NK) or [K][ldw] (BQ_W_KN).
+ * deq_scale: fp32 [N], 32-byte aligned (as the ATB page requires).
+ * per_token_scale: fp32 [M].  bias: fp32 [N] or NULL.  out: out_dtype
+ * (BQ_BF16, BQ_F16 or BQ_F32) [M][ldo], computed in fp32 and rounded once.
+ * Runs on the tcgen05 tensor cores; M, N and K tails are handled.
+ */
+bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_wlayout w_layout,
+                              int64_t ldw, const float *deq_scale, const float *per_token_scale,
+                              const float *bias, int64_t M, int64_t N, int64_t K, bq_dtype out_dtype,
+                              void *out, int64_t ldo, bq_stream_t stream);
+
+/*
+ * BitLinear forward with ternary weights and int8 activations (W1.58A8).
+ * Source: "Class BitLinear" (LLaMA-BitNet utils.py), forward steps 1-5.
+ *
+ *   (xq, act_scale, rowsum) = bq_act_quant_int8(x)   into the workspace
+ *   acc[m,n] = sum_k xq[m,k] * w_q[n,k]              (exact int32)
+ *   out[m,n] = (float(acc) * act_scale[m]) * gamma  (+ bias[n])
+ *
+ * x: dense [M][K] of x_dtype BQ_F32 or BQ_BF16; K % 16 == 0.  wpacked,
+ * w_scale: as written by bq_weight_quant_ternary_pack.  bias: fp32 [N] or
+ * NULL (the page disables it by default).  out: dense [M][N] of out_dtype.
+ * M <= 16 runs the bandwidth-bound decode kernel, larger M the tcgen05 GEMM
+ * that unpacks the 2-bit tiles in shared memory.  workspace: at least
+ * bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) bytes, 256-byte
+ * aligned; bq_bitlinear_workspace_layout() gives where xq [M][K] int8,
+ * act_scale fp32 [M] and rowsum int32 [M] sit, so they can be read back.
+ */
+bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t K,
+                            const uint32_t *wpacked, const float *w_scale, int64_t N,
+                            const float *bias, float eps, bq_dtype out_dtype, void *out,
+                            void *workspace, size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Grouped affine INT4 linear with fp32 activations.
+ * Source: "vyre_libs/nn/linear/inner/linear_4bit/mod.rs", module doc (fused
+ * unpack-on-demand; grouped affine path with scale and zero-point per group)
+ * and the grouped output drift tolerance constant.
+ *
+ *   out[m,n] = bias[n] + sum_k x[m,k] * scale[n,g] * (q[n,k] - zero[n,g])
+ *
+ * x: dense fp32 [M][K], K % 8 == 0, group_size % 8 == 0 and divides K.
+ * qweight, scales_f16, qzeros: as in "Data formats".  bias: fp32 [N] or NULL.
+ * out: dense fp32 [M][N].  Internally x is split per (token, group) into a
+ * 24-bit fixed-point value held as three byte planes so that the inner
+ * products are exact integer dot products; the representation error is below
+ * 1e-6 of the group's absolute maximum.  workspace: at least
+ * bq_workspace_bytes(BQ_OP_LINEAR_W4_GROUPED, M, N, K, group_size) bytes,
+ * 256-byte aligned.
+ */
+bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint32_t *qweight,
+                               const uint16_t *scales_f16, const uint32_t *qzeros,
+                               const float *bias, int64_t N, int64_t group_size, float *out,
+                               void *workspace, size_t workspace_bytes, bq_stream_t stream);
+
+/* Workspace bytes a call needs (0 for calls that need none). */
+size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t group_size);
+
+/* Byte offsets of xq [M][K], act_scale [M] and rowsum [M] inside the
+ * bq_bitlinear_w2a8 workspace. */
+void bq_bitlinear_workspace_layout(int64_t M, int64_t K, size_t *xq_offset, size_t *act_scale_offset,
+                                   size_t *rowsum_offset);
+
+/* Static description of a status code. */
+const char *bq_status_string(bq_status status);
+
+/*
+ * Synchronizes `stream`, then reads and clears the current device's status
+ * word.  Returns BQ_OK or the first error a kernel recorded; *detail (may be
+ * NULL) receives the raw word (bits 0-7 status, bits 8-31 the site).
+ */
+bq_status bq_device_status(bq_stream_t stream, uint32_t *detail);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int bq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

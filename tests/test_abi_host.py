@@ -1,0 +1,146 @@
+"""C-ABI checks that need no GPU: the library loads, exports every call the
+header declares, and rejects invalid arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_quantized_linear_rmsnorm_b200 as bq
+from bit_quantized_linear_rmsnorm_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return bq.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_six_calls():
+    names = _declared()
+    for n in ["bq_act_quant_int8", "bq_weight_quant_ternary_pack", "bq_weight_pack_int4_grouped",
+              "bq_gemm_i8_pertoken", "bq_bitlinear_w2a8", "bq_linear_w4_grouped"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in _declared():
+        assert hasattr(L, n), n
+    assert set(_declared()) <= set(bq.EXPORTED)
+
+
+def test_version_and_strings(L):
+    assert bq.bq_version() >= 100
+    assert bq.bq_status_string(bq.BQ_OK) == "ok"
+    assert "workspace" in bq.bq_status_string(bq.BQ_ERR_WORKSPACE)
+    assert bq.bq_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(L):
+    assert bq.bq_workspace_bytes(bq.BQ_OP_GEMM_I8_PERTOKEN, 4096, 4096, 4096) == 0
+    n = bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, 16, 11008, 4096)
+    xo, so, ro = bq.bq_bitlinear_workspace_layout(16, 4096)
+    assert xo == 0 and so >= 16 * 4096 and ro >= so + 16 * 4 and n >= ro + 16 * 4
+    assert so % 256 == 0 and ro % 256 == 0
+    assert bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4_GROUPED, 32, 14336, 4096, 128) >= 3 * 32 * 4096
+    assert bq.bq_workspace_bytes(bq.BQ_OP_WEIGHT_QUANT_TERNARY_PACK, 0, 4096, 4096) > 0
+    assert bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4_GROUPED, 1, 1, 128, 0) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)      # 64 KiB-aligned, never dereferenced
+ODD = ctypes.c_void_p(0x10001)
+
+
+def test_act_quant_rejects(L):
+    f = L.bq_act_quant_int8
+    assert f(None, bq.BQ_F32, 4, 64, 64, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, 7, 4, 64, 64, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F16, 4, 64, 64, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F32, 4, 0, 64, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F32, 4, 64, 32, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F32, 4, 64, 64, float("nan"), FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F32, 4, 64, 64, -1.0, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F32, 4, 64, 64, 1e-5, ODD, 64, FAKE, None, None) == bq.BQ_ERR_MISALIGNED
+    assert f(FAKE, bq.BQ_F32, 4, 64, 64, 1e-5, FAKE, 72, FAKE, None, None) == bq.BQ_ERR_MISALIGNED
+    # empty batch is a valid no-op
+    assert f(None, bq.BQ_F32, 0, 64, 64, 1e-5, None, 64, None, None, None) == bq.BQ_OK
+
+
+def test_ternary_pack_rejects(L):
+    f = L.bq_weight_quant_ternary_pack
+    assert f(FAKE, bq.BQ_F32, 8, 24, FAKE, FAKE, FAKE, 1 << 20, None) == bq.BQ_ERR_INVALID_ARG  # K % 16
+    assert f(FAKE, bq.BQ_F32, 8, 32, FAKE, FAKE, None, 0, None) == bq.BQ_ERR_WORKSPACE
+    assert f(FAKE, bq.BQ_F32, 8, 32, FAKE, FAKE, FAKE, 1, None) == bq.BQ_ERR_WORKSPACE
+    assert f(ODD, bq.BQ_F32, 8, 32, FAKE, FAKE, FAKE, 1 << 20, None) == bq.BQ_ERR_MISALIGNED
+    assert f(None, bq.BQ_F32, 0, 32, None, None, None, 0, None) == bq.BQ_OK
+
+
+def test_int4_pack_rejects(L):
+    f = L.bq_weight_pack_int4_grouped
+    assert f(FAKE, FAKE, 4, 12, 4, FAKE, FAKE, None) == bq.BQ_ERR_INVALID_ARG   # K % 8
+    assert f(FAKE, FAKE, 4, 64, 48, FAKE, FAKE, None) == bq.BQ_ERR_INVALID_ARG  # gs does not divide K
+    assert f(FAKE, FAKE, 4, 64, 0, FAKE, FAKE, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(ODD, FAKE, 4, 64, 16, FAKE, FAKE, None) == bq.BQ_ERR_MISALIGNED
+
+
+def _gemm(L, x=FAKE, ldx=64, w=FAKE, wl=0, ldw=64, deq=FAKE, pts=FAKE, bias=None, M=4, N=64, K=64, od=bq.BQ_BF16,
+          out=FAKE, ldo=64):
+    return L.bq_gemm_i8_pertoken(x, ldx, w, wl, ldw, deq, pts, bias, M, N, K, od, out, ldo, None)
+
+
+def test_gemm_rejects(L):
+    assert _gemm(L, K=0) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, K=131072, ldx=131072, ldw=131072) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, wl=5) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, od=9) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, ldx=32) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, ldo=32) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, x=None) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, deq=None) == bq.BQ_ERR_INVALID_ARG
+    assert _gemm(L, x=ODD) == bq.BQ_ERR_MISALIGNED
+    assert _gemm(L, ldx=72) == bq.BQ_ERR_MISALIGNED
+    assert _gemm(L, ldo=68) == bq.BQ_ERR_MISALIGNED          # 68 * 2 bytes is not a multiple of 16
+    assert _gemm(L, deq=ctypes.c_void_p(0x10010)) == bq.BQ_ERR_MISALIGNED  # deqScale 32-byte rule
+    assert _gemm(L, M=0) == bq.BQ_OK
+    assert _gemm(L, N=0, ldo=64) == bq.BQ_OK
+
+
+def test_bitlinear_rejects(L):
+    f = L.bq_bitlinear_w2a8
+    ok = dict(x=FAKE, xt=bq.BQ_BF16, M=32, K=128, wp=FAKE, ws_=FAKE, N=64, bias=None, eps=1e-5, od=bq.BQ_BF16,
+              out=FAKE, work=FAKE, nbytes=1 << 24)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["x"], a["xt"], a["M"], a["K"], a["wp"], a["ws_"], a["N"], a["bias"], a["eps"], a["od"], a["out"],
+                 a["work"], a["nbytes"], None)
+    assert call(K=40) == bq.BQ_ERR_INVALID_ARG
+    assert call(xt=bq.BQ_F16) == bq.BQ_ERR_INVALID_ARG
+    assert call(work=None) == bq.BQ_ERR_WORKSPACE
+    assert call(nbytes=16) == bq.BQ_ERR_WORKSPACE
+    assert call(work=ctypes.c_void_p(0x10040)) == bq.BQ_ERR_MISALIGNED
+    assert call(N=61) == bq.BQ_ERR_MISALIGNED     # tensor-core path stores whole 16-byte rows
+    assert call(K=144) == bq.BQ_ERR_MISALIGNED    # tensor-core path loads packed rows with TMA
+    assert call(M=0) == bq.BQ_OK
+
+
+def test_linear_w4_rejects(L):
+    f = L.bq_linear_w4_grouped
+
+    def call(M=1, K=256, gs=128, N=8, work=FAKE, nbytes=1 << 24, x=FAKE):
+        return f(x, M, K, FAKE, FAKE, FAKE, None, N, gs, FAKE, work, nbytes, None)
+    assert call(K=100) == bq.BQ_ERR_INVALID_ARG
+    assert call(gs=12) == bq.BQ_ERR_INVALID_ARG
+    assert call(gs=96) == bq.BQ_ERR_INVALID_ARG
+    assert call(K=65544, gs=8) == bq.BQ_ERR_INVALID_ARG
+    assert call(work=None) == bq.BQ_ERR_WORKSPACE
+    assert call(x=ODD) == bq.BQ_ERR_MISALIGNED
+    assert call(M=0) == bq.BQ_OK

@@ -1,0 +1,358 @@
+"""Parity of every C-ABI call with the oracle, on identical seeded inputs.
+
+Sizes span several tiles with ragged tails; the benchmark workloads run at
+full size (outputs compared on whole rows sampled by the oracle).  Integer
+results are bit-exact except codes whose exact pre-rounding value lies within
+1e-6 (relative) of a .5 boundary; dequantized outputs are within 1 bf16/fp16
+ulp or 1e-5 relative (fp32); grouped INT4 outputs within 1e-4*sqrt(K/128)
+absolute.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import bit_quantized_linear_rmsnorm_b200 as bq
+import oracle
+import synth
+from gpu_helpers import assert_codes, assert_out, bf16_dev, dev, host, padded, tie_band
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _ready():
+    from bit_quantized_linear_rmsnorm_b200 import _build
+    _build.build()
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    torch.cuda.init()
+    yield
+    st, detail = bq.bq_device_status()
+    assert st == bq.BQ_OK, f"device status word {detail:#x}"
+
+
+# ----------------------------------------------------------------- act quant
+
+def _check_act(x_f32, x_dev, eps, what):
+    xq, sc, rs = bq.bq_act_quant_int8(x_dev, eps)
+    torch.cuda.synchronize()
+    ref = oracle.act_quant(x_f32, eps, want_pre=True)
+    g_xq = host(xq)
+    assert_codes(g_xq, ref["xq"], ref["pre"], what)
+    np.testing.assert_allclose(host(sc), ref["act_scale"], rtol=1e-5, err_msg=what)
+    np.testing.assert_array_equal(host(rs), g_xq.astype(np.int64).sum(axis=1))
+    return g_xq
+
+
+@pytest.mark.parametrize("M,K,dtype", [(8, 256, "f32"), (37, 1000, "bf16"), (5, 4096, "bf16"),
+                                       (300, 4096, "bf16"), (3, 6000, "f32"), (64, 8200, "bf16"),
+                                       (1, 7, "f32"), (17, 33, "bf16")])
+def test_act_quant(M, K, dtype):
+    g = synth.rng((101, M, K))
+    x = synth.normal_f32(g, (M, K))
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(x)
+        x = synth.bf16_bits_to_f32(bits)
+        xd = bf16_dev(bits)
+    else:
+        xd = dev(x)
+    _check_act(x, xd, 1e-5, f"act_quant {M}x{K} {dtype}")
+
+
+def test_act_quant_special_rows():
+    K = 512
+    x = synth.normal_f32(synth.rng(102), (6, K))
+    x[0] = 0.0                 # zero row
+    x[1] = 0.75                # constant row
+    x[2] = 0.0
+    x[2, 100] = -3.0           # one-hot row
+    x[3] *= 1e-6               # tiny row: eps dominates the RMS
+    x[4, :] = np.float32(2.0 ** -20)
+    _check_act(x, dev(x), 1e-5, "special rows")
+    xq, sc, _ = bq.bq_act_quant_int8(dev(x), 1e-5)
+    assert np.all(host(xq)[0] == 0) and host(sc)[0] == pytest.approx(1e-5 / 127, rel=1e-6)
+    assert np.all(host(xq)[1] == 127)
+
+
+def test_act_quant_unaligned_rows_scalar_path():
+    M, K = 9, 300
+    x = synth.normal_f32(synth.rng(103), (M, K + 1))
+    xd = dev(x)[:, 1:]  # base 4 bytes off 16, stride 301 floats
+    _check_act(np.ascontiguousarray(x[:, 1:]), xd, 1e-5, "unaligned")
+
+
+def test_act_quant_outlier_channels_prefill_rows():
+    bits, xf = synth.bf16_activations(256, 4096, (5, 1), outlier_frac=0.01)
+    _check_act(xf, bf16_dev(bits), 1e-5, "outliers")
+
+
+# ------------------------------------------------------------ ternary pack
+
+def _check_ternary(w_f32, w_dev, what):
+    wp, ws = bq.bq_weight_quant_ternary_pack(w_dev)
+    torch.cuda.synchronize()
+    ref = oracle.ternary_quant(w_f32, want_pre=True)
+    gamma = float(host(ws)[0])
+    assert gamma == pytest.approx(ref["gamma"], rel=1e-6), what
+    K = w_f32.shape[1]
+    codes, bad = oracle.ternary_unpack(host(wp).view(np.uint32), K)
+    assert bad == 0, f"{what}: invalid 2-bit code"
+    assert_codes(codes, ref["wq"], ref["pre"] + 0.0, what)
+    if not tie_band(ref["pre"]).any():
+        np.testing.assert_array_equal(host(wp).view(np.uint32), oracle.ternary_pack(ref["wq"]))
+    return wp, ws, ref
+
+
+@pytest.mark.parametrize("N,K,dtype", [(128, 256, "f32"), (300, 512, "f32"), (64, 4096, "bf16"), (5, 16, "f32")])
+def test_ternary_pack(N, K, dtype):
+    w = synth.normal_f32(synth.rng((104, N, K)), (N, K), 0.02)
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(w)
+        _check_ternary(synth.bf16_bits_to_f32(bits), bf16_dev(bits), f"ternary {N}x{K} bf16")
+    else:
+        _check_ternary(w, dev(w), f"ternary {N}x{K}")
+
+
+def test_ternary_pack_full_decode_weight():
+    w = synth.bitlinear_weight(11008, 4096, 3)
+    _check_ternary(w, dev(w), "ternary 11008x4096")
+
+
+def test_ternary_pack_bake_rule_and_edges():
+    w = np.zeros((16, 64), np.float32)
+    _, ws, ref = _check_ternary(w, dev(w), "all zero")
+    assert float(host(ws)[0]) == pytest.approx(1e-5, rel=1e-6)
+    g = synth.rng(105)
+    w = (g.integers(-1, 2, (32, 64)) * 0.37).astype(np.float32)
+    _, ws, ref = _check_ternary(w, dev(w), "already ternary")
+    assert ref["already_ternary"] and float(host(ws)[0]) == np.float32(0.37)
+    # bake(W) packs to the same words and scale as W itself
+    w = synth.normal_f32(g, (48, 128), 0.02)
+    wp1, ws1, r1 = _check_ternary(w, dev(w), "master")
+    baked = oracle.ternary_bake(r1["wq"], r1["gamma"])
+    wp2, ws2, _ = _check_ternary(baked, dev(baked), "baked")
+    np.testing.assert_array_equal(host(wp1), host(wp2))
+    assert float(host(ws2)[0]) == pytest.approx(float(host(ws1)[0]), rel=1e-6)
+
+
+# --------------------------------------------------------------- INT4 pack
+
+@pytest.mark.parametrize("N,K,gs", [(14336, 4096, 128), (7, 192, 8), (3, 40, 8), (5, 64, 64)])
+def test_int4_pack(N, K, gs):
+    g = synth.rng((106, N, K))
+    q = synth.nibbles(g, (N, K))
+    z = synth.nibbles(g, (N, K // gs))
+    qw, qz = bq.bq_weight_pack_int4_grouped(dev(q), dev(z), gs)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(qw).view(np.uint32), oracle.int4_pack(q))
+    np.testing.assert_array_equal(host(qz).view(np.uint32), oracle.int4_pack(z))
+
+
+def test_int4_pack_flags_codes_above_15():
+    q = np.full((2, 16), 3, np.uint8)
+    q[1, 5] = 0x13
+    z = np.zeros((2, 2), np.uint8)
+    qw, _ = bq.bq_weight_pack_int4_grouped(dev(q), dev(z), 8)
+    st, detail = bq.bq_device_status()
+    assert st == bq.BQ_ERR_INVALID_ARG
+    assert (detail >> 8) == 16
+    assert bq.bq_device_status()[0] == bq.BQ_OK  # read-and-clear
+    q[1, 5] = 3
+    np.testing.assert_array_equal(host(qw).view(np.uint32), oracle.int4_pack(q))
+
+
+# ------------------------------------------------------------- W8A8 GEMM
+
+_TORCH_OUT = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
+
+
+def _gemm_case(M, N, K, layout, out, bias, seed):
+    d = synth.gemm_w8a8(M, N, K, seed)
+    w = d["w"] if layout == bq.BQ_W_NK else np.ascontiguousarray(d["w"].T)
+    b = synth.normal_f32(synth.rng((seed, 7)), (N,), 0.5) if bias else None
+    xd = padded(d["x"], 16)
+    wd = padded(w, 16)
+    deq = dev(d["deq_scale"])
+    pts = dev(d["per_token_scale"])
+    o = bq.bq_gemm_i8_pertoken(xd, wd, deq, pts, None if b is None else dev(b), w_layout=layout,
+                               out_dtype=_TORCH_OUT[out])
+    torch.cuda.synchronize()
+    ref, ovf = oracle.gemm_i8_pertoken(d["x"], w, d["deq_scale"], d["per_token_scale"], b, layout=layout)
+    assert ovf == 0
+    scale = None
+    if b is not None:
+        scale = np.abs(ref - b.astype(np.float64)) + np.abs(b.astype(np.float64))
+    assert_out(host(o), ref, _TORCH_OUT[out], f"gemm {M}x{N}x{K} layout {layout} {out}", scale=scale)
+
+
+def test_gemm_atb_worked_example(golden_dir):
+    import json
+    import os
+    with open(os.path.join(golden_dir, "atb_per_token_example.json")) as f:
+        ex = json.load(f)
+    x = np.array(ex["x"], np.int8)
+    w = np.array(ex["weight"], np.int8)  # [k, n]
+    for out in ("bf16", "f16", "f32"):
+        o = bq.bq_gemm_i8_pertoken(padded(x, 16), padded(w, 16), dev(np.array(ex["deqScale"], np.float32)),
+                                   dev(np.array(ex["perTokenScale"], np.float32)), w_layout=bq.BQ_W_KN,
+                                   out_dtype=_TORCH_OUT[out])
+        np.testing.assert_array_equal(host(o), np.array(ex["output"], np.float64))
+        o = bq.bq_gemm_i8_pertoken(padded(x, 16), padded(np.ascontiguousarray(w.T), 16),
+                                   dev(np.array(ex["deqScale"], np.float32)),
+                                   dev(np.array(ex["perTokenScale"], np.float32)), w_layout=bq.BQ_W_NK,
+                                   out_dtype=_TORCH_OUT[out])
+        np.testing.assert_array_equal(host(o), np.array(ex["output"], np.float64))
+
+
+@pytest.mark.parametrize("M,N,K,layout,out,bias", [
+    (300, 520, 400, bq.BQ_W_NK, "bf16", False),
+    (129, 257, 128, bq.BQ_W_NK, "f32", True),
+    (200, 384, 264, bq.BQ_W_KN, "f16", False),
+    (77, 200, 1000, bq.BQ_W_KN, "bf16", True),
+    (1, 8, 16, bq.BQ_W_NK, "bf16", False),
+    (513, 1030, 2048, bq.BQ_W_NK, "bf16", True),
+    (260, 2100, 96, bq.BQ_W_NK, "f32", False),
+])
+def test_gemm_ragged(M, N, K, layout, out, bias):
+    _gemm_case(M, N, K, layout, out, bias, seed=M + N + K)
+
+
+def test_gemm_full_size_sampled_rows():
+    d = synth.gemm_w8a8()
+    o = bq.bq_gemm_i8_pertoken(dev(d["x"]), dev(d["w"]), dev(d["deq_scale"]), dev(d["per_token_scale"]))
+    torch.cuda.synchronize()
+    rows = np.sort(synth.rng(107).choice(4096, 48, replace=False))
+    rows = np.concatenate([[0, 127, 128, 4095], rows])
+    ref, _ = oracle.gemm_i8_pertoken(d["x"][rows], d["w"], d["deq_scale"], d["per_token_scale"][rows])
+    assert_out(host(o)[rows], ref, torch.bfloat16, "gemm 4096^3 sampled rows")
+
+
+def test_gemm_closed_form_all_ones():
+    M, N, K = 200, 300, 1000
+    x = np.ones((M, K), np.int8)
+    w = np.ones((N, K), np.int8)
+    o = bq.bq_gemm_i8_pertoken(padded(x, 16), padded(w, 16), dev(np.ones(N, np.float32)),
+                               dev(np.ones(M, np.float32)), out_dtype=torch.float32)
+    np.testing.assert_array_equal(host(o), np.full((M, N), float(K)))
+
+
+# ------------------------------------------------------------- BitLinear
+
+def _bitlinear_check(x_f32, x_dev, w_f32, N, out, bias, what, rows=None):
+    """Runs the GPU pack + BitLinear, then checks the workspace codes and the
+    output against the oracle computed from the same inputs."""
+    eps = 1e-5
+    M, K = x_f32.shape
+    wp, ws_ = bq.bq_weight_quant_ternary_pack(dev(w_f32))
+    nbytes = bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, M, N, K)
+    work = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    b = None if bias is None else dev(bias)
+    o = bq.bq_bitlinear_w2a8(x_dev, wp, ws_, N, b, eps, _TORCH_OUT[out], workspace=work)
+    torch.cuda.synchronize()
+    xo, so, _ = bq.bq_bitlinear_workspace_layout(M, K)
+    g_xq = host(work[xo:xo + M * K].view(torch.int8).view(M, K))
+    g_sc = host(work[so:so + 4 * M].view(torch.float32))
+    sel = np.arange(M) if rows is None else rows
+    a = oracle.act_quant(x_f32[sel], eps, want_pre=True)
+    t = oracle.ternary_quant(w_f32, want_pre=True)
+    assert_codes(g_xq[sel], a["xq"], a["pre"], what + " xq")
+    np.testing.assert_allclose(g_sc[sel], a["act_scale"], rtol=1e-5)
+    ref = oracle.bitlinear_from_codes(a["xq"], a["act_scale"], t["wq"], t["gamma"], bias)
+    # codes in the tie band may round either way: widen by what they can move
+    xband = tie_band(a["pre"]).astype(np.float64)
+    wband = tie_band(t["pre"]).astype(np.float64)
+    extra = (xband @ np.abs(t["wq"]).T.astype(np.float64) + np.abs(a["xq"]).astype(np.float64) @ wband.T) \
+        * a["act_scale"][:, None] * t["gamma"]
+    scale = None
+    if bias is not None:
+        scale = np.abs(ref - bias.astype(np.float64)) + np.abs(bias.astype(np.float64))
+    assert_out(host(o)[sel], ref, _TORCH_OUT[out], what, extra=extra, scale=scale)
+
+
+def test_bitlinear_tiny_config():
+    d = synth.bitlinear_tiny(0)
+    _bitlinear_check(d["x"], dev(d["x"]), d["w"], 128, "f32", None, "bitlinear tiny")
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_bitlinear_decode_full_size(M):
+    d = synth.bitlinear_decode(M)
+    _bitlinear_check(d["x"], bf16_dev(d["x_bf16"]), d["w"], 11008, "bf16", None, f"decode M={M}")
+
+
+@pytest.mark.parametrize("M,N,K,out,bias", [(3, 100, 48, "f16", True), (7, 64, 4096, "f32", False),
+                                            (16, 72, 192, "bf16", True)])
+def test_bitlinear_decode_ragged(M, N, K, out, bias):
+    g = synth.rng((108, M, N, K))
+    x = synth.normal_f32(g, (M, K))
+    w = synth.normal_f32(g, (N, K), 0.02)
+    b = synth.normal_f32(g, (N,), 0.1) if bias else None
+    _bitlinear_check(x, dev(x), w, N, out, b, f"decode ragged {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K,out,bias", [(17, 256, 128, "bf16", False), (300, 520, 512, "bf16", True),
+                                            (129, 264, 640, "f32", False), (200, 1000, 1024, "f16", True)])
+def test_bitlinear_prefill_ragged(M, N, K, out, bias):
+    g = synth.rng((109, M, N, K))
+    bits, xf = synth.bf16_activations(M, K, (109, M), outlier_frac=0.01)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    b = synth.normal_f32(g, (N,), 0.1) if bias else None
+    _bitlinear_check(xf, bf16_dev(bits), w, N, out, b, f"prefill ragged {M}x{N}x{K}")
+
+
+def test_bitlinear_prefill_full_size_sampled_rows():
+    d = synth.bitlinear_prefill()
+    rows = np.sort(np.concatenate([[0, 1, 127, 128, 8191], synth.rng(110).choice(8192, 27, replace=False)]))
+    rows = np.unique(rows)
+    _bitlinear_check(d["x"], bf16_dev(d["x_bf16"]), d["w"], 4096, "bf16", None, "prefill 8192x4096x4096",
+                     rows=rows)
+
+
+# ------------------------------------------------------------- INT4 linear
+
+def _w4_check(M, N, K, gs, seed, rows=None, full=None):
+    if full is None:
+        g = synth.rng(seed)
+        q = synth.nibbles(g, (N, K))
+        z = synth.nibbles(g, (N, K // gs))
+        s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+        b = synth.normal_f32(g, (N,), 0.01)
+        x = synth.normal_f32(g, (M, K))
+    else:
+        q, z, s, b, x = full
+    qw, qz = bq.bq_weight_pack_int4_grouped(dev(q), dev(z), gs)
+    o = bq.bq_linear_w4_grouped(dev(x), qw, dev(s.view(np.int16)), qz, gs, dev(b))
+    torch.cuda.synchronize()
+    sel = np.arange(M) if rows is None else rows
+    ref = oracle.linear_w4_grouped(x[sel], oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), b, gs)
+    tol = 1e-4 * math.sqrt(K / 128)
+    err = np.abs(host(o)[sel] - ref)
+    assert err.max() <= tol, f"INT4 {M}x{N}x{K} g{gs}: max |err| {err.max():.3e} > {tol:.3e}"
+    return err.max()
+
+
+@pytest.mark.parametrize("M,N,K,gs", [(3, 100, 384, 64), (5, 33, 200, 8), (2, 7, 96, 96), (6, 300, 1024, 128),
+                                      (1, 64, 64, 32), (9, 129, 512, 256)])
+def test_linear_w4_ragged(M, N, K, gs):
+    _w4_check(M, N, K, gs, seed=(111, M, N, K))
+
+
+@pytest.mark.parametrize("M", [1, 32])
+def test_linear_w4_full_size(M):
+    w = synth.linear_w4_weights()
+    x = synth.linear_w4_activations(M)
+    rows = None if M == 1 else np.array([0, 5, 17, 31])
+    _w4_check(M, 14336, 4096, 128, None, rows=rows,
+              full=(w["q"], w["zeros"], w["scales_f16"], w["bias"], x))
+
+
+def test_linear_w4_zero_point_equals_code_gives_bias():
+    g = synth.rng(112)
+    N, K, gs = 40, 256, 64
+    z = synth.nibbles(g, (N, K // gs))
+    q = np.repeat(z, gs, axis=1)
+    s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+    b = synth.normal_f32(g, (N,), 0.01)
+    x = synth.normal_f32(g, (3, K))
+    _w4_check(3, N, K, gs, None, full=(q, z, s, b, x))
