@@ -28,7 +28,9 @@ EXPORTED = [
     "bq_act_quant_int8", "bq_weight_quant_ternary_pack", "bq_weight_pack_int4_grouped",
     "bq_gemm_i8_pertoken", "bq_bitlinear_w2a8", "bq_linear_w4_grouped", "bq_workspace_bytes",
     "bq_bitlinear_workspace_layout", "bq_status_string", "bq_device_status", "bq_version",
+    "bq_bitlinear_w2a8_noalloc",
 ]
+BQ_NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
 
 _DTYPE = {torch.float32: BQ_F32, torch.bfloat16: BQ_BF16, torch.float16: BQ_F16}
 
@@ -45,6 +47,7 @@ _SIGS = {
     "bq_gemm_i8_pertoken": (I32, [P, I64, P, I32, I64, P, P, P, I64, I64, I64, I32, P, I64, P]),
     "bq_bitlinear_w2a8": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P, SZ, P]),
     "bq_linear_w4_grouped": (I32, [P, I64, I64, P, P, P, P, I64, I64, P, P, SZ, P]),
+    "bq_bitlinear_w2a8_noalloc": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P]),
     "bq_workspace_bytes": (SZ, [I32, I64, I64, I64, I64]),
     "bq_bitlinear_workspace_layout": (None, [I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     "bq_status_string": (ctypes.c_char_p, [I32]),
@@ -218,4 +221,18 @@ def bq_linear_w4_grouped(x: torch.Tensor, qweight: torch.Tensor, scales_f16: tor
     st = lib().bq_linear_w4_grouped(_ptr(x), M, K, _ptr(qweight), _ptr(scales_f16), _ptr(qzeros), _ptr(bias), N,
                                     group_size, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check(st, "bq_linear_w4_grouped")
+    return out
+
+
+def bq_bitlinear_w2a8_noalloc(x: torch.Tensor, wpacked: torch.Tensor, w_scale: torch.Tensor, N: int, bias=None,
+                              eps: float = 1e-5, out_dtype=torch.bfloat16, out=None, stream=None):
+    """BitLinear forward that allocates nothing on the device beyond the output
+    given (or allocated here by torch when `out` is None): the library keeps
+    its scratch in a fixed static device array (see include/bq.h)."""
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    st = lib().bq_bitlinear_w2a8_noalloc(_ptr(x), _DTYPE[x.dtype], M, K, _ptr(wpacked), _ptr(w_scale), N, _ptr(bias),
+                                         float(eps), _DTYPE[out.dtype], _ptr(out), _stream(stream))
+    _check(st, "bq_bitlinear_w2a8_noalloc")
     return out

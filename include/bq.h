@@ -193,6 +193,36 @@ bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint3
                                const float *bias, int64_t N, int64_t group_size, float *out,
                                void *workspace, size_t workspace_bytes, bq_stream_t stream);
 
+/*
+ * BitLinear forward with the contract and results of bq_bitlinear_w2a8, for
+ * callers that cannot allocate device memory or hand over a workspace: a
+ * plugin or custom op whose host framework owns every device allocation and
+ * forbids cudaMalloc, or a latency-critical decode loop where an allocation
+ * would synchronize the device.  The pages have no counterpart of this entry
+ * point.
+ *
+ * The caller passes inputs and outputs as for bq_bitlinear_w2a8.  The scratch
+ * (int8 activations, per-token scales, row sums) lives in one static device
+ * array of BQ_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits.  A call whose scratch would exceed
+ * it (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) >
+ * BQ_NOALLOC_SCRATCH_BYTES, i.e. M*K above about 2 MB) returns
+ * BQ_ERR_WORKSPACE before launching anything.  The call never allocates
+ * (no cudaMalloc / cudaFree, no allocating library routine).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls on a device share the
+ * array and it keeps the last call's contents; each call writes all the
+ * scratch it reads, so nothing needs clearing, but calls that overlap on the
+ * GPU (unordered streams) race on it.
+ */
+#define BQ_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+bq_status bq_bitlinear_w2a8_noalloc(const void *x, bq_dtype x_dtype, int64_t M, int64_t K,
+                                    const uint32_t *wpacked, const float *w_scale, int64_t N,
+                                    const float *bias, float eps, bq_dtype out_dtype, void *out,
+                                    bq_stream_t stream);
+
 /* Workspace bytes a call needs (0 for calls that need none). */
 size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t group_size);
 
