@@ -55,6 +55,10 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-workloads", action="store_true", help="skip the secondary workloads")
+    p.add_argument("--workloads", default="decode,w4,prefill,tiny",
+                   help="comma list of secondary workloads: decode, w4, prefill, tiny")
+    p.add_argument("--workload-steps", type=int, default=200)
+    p.add_argument("--no-head", action="store_true", help="skip the headline GEMM (profiling runs only)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0 = calibrate to ~10 s)")
     return p.parse_args()
@@ -316,9 +320,27 @@ def workloads(args, pk):
     res = {}
     hbm = pk["hbm_gbs"]
     peak_int8 = 2.0 * pk["bf16_tflops"]
-    steps = 200
+    steps = args.workload_steps
+    want = set(args.workloads.split(","))
+    if "decode" in want:
+        _decode(res, steps, hbm)
+    if "w4" in want:
+        _w4(res, steps, hbm)
+    if "prefill" in want:
+        _prefill(res, max(steps // 4, 1), peak_int8)
+    if "tiny" in want:
+        _tiny(res, steps)
+    st, detail = bq.bq_device_status()
+    if st != bq.BQ_OK:
+        raise RuntimeError(f"device status {detail:#x} after the workloads")
+    return res
 
-    # BitLinear W1.58A8 decode, W [11008, 4096]
+
+def _decode(res, steps, hbm):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
     N, K = 11008, 4096
     w = torch.from_numpy(synth.bitlinear_weight(N, K, 3)).cuda()
     wp, wsc = bq.bq_weight_quant_ternary_pack(w)
@@ -342,6 +364,12 @@ def workloads(args, pk):
                                          "launches_per_step": 2, "config": f"x bf16 [{M},4096], W 2-bit [11008,4096]"}
     del wps
 
+
+def _w4(res, steps, hbm):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
     # Grouped affine INT4, 4096 -> 14336, g = 128
     N, K, gs = 14336, 4096, 128
     wq = synth.linear_w4_weights()
@@ -369,6 +397,12 @@ def workloads(args, pk):
                                   "config": f"x fp32 [{M},4096], INT4 [14336,4096] g128"}
     del sets
 
+
+def _prefill(res, steps, peak_int8):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
     # BitLinear prefill [8192, 4096] x [4096, 4096]
     d = synth.bitlinear_prefill()
     M, N, K = 8192, 4096, 4096
@@ -380,7 +414,7 @@ def workloads(args, pk):
     def step(i):
         bq.bq_bitlinear_w2a8(x, wp, wsc, N, None, 1e-5, torch.bfloat16, out=out, workspace=work)
 
-    ms, _ = graph_time(step, 50, 3)
+    ms, _ = graph_time(step, steps, 3)
     ops = 2.0 * M * N * K
     tops = ops / (ms * 1e-3) / 1e12
     res["bitlinear_prefill"] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(tops, 1),
@@ -388,6 +422,12 @@ def workloads(args, pk):
                                 "config": "x bf16 [8192,4096] (1% outlier channels), W 2-bit [4096,4096]; "
                                           "act quant + tcgen05 GEMM per step (160 MB moved > L2)"}
 
+
+def _tiny(res, steps):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
     # BitLinear tiny [8,256] x [128,256], fp32 out
     d = synth.bitlinear_tiny(0)
     x = torch.from_numpy(d["x"]).cuda()
@@ -398,12 +438,8 @@ def workloads(args, pk):
     def step(i):
         bq.bq_bitlinear_w2a8(x, wp, wsc, 128, None, 1e-5, torch.float32, out=out, workspace=work)
 
-    ms, _ = graph_time(step, 200, 3)
+    ms, _ = graph_time(step, steps, 3)
     res["bitlinear_tiny"] = {"us_per_step": round(ms * 1e3, 3), "config": "x fp32 [8,256], W [128,256]"}
-    st, detail = bq.bq_device_status()
-    if st != bq.BQ_OK:
-        raise RuntimeError(f"device status {detail:#x} after the workloads")
-    return res
 
 
 # ---------------------------------------------------------------------------
@@ -469,8 +505,13 @@ def main():
     import bit_quantized_linear_rmsnorm_b200 as bq
     bq.lib()
     pk = peaks()
-    head, d = headline(args, dist, pk)
     extra = {}
+    if args.no_head:
+        if rank == 0:
+            print(json.dumps({"workloads": workloads(args, pk)}), flush=True)
+        dist.close()
+        return
+    head, d = headline(args, dist, pk)
     if not args.no_workloads and rank == 0:
         extra = workloads(args, pk)
     base = None
