@@ -18,79 +18,14 @@
 // the exact x*127/max|x| by at most three fp32 roundings (<= 1.8e-7
 // relative).  |x*f| <= 127 * (1 + 2^-22) always rounds inside [-127, 127], so
 // the clamp of the definition never changes a value.
-#include <cuda_bf16.h>
-
-#include "bq_common.cuh"
 #include "bq_internal.h"
+#include "quant_common.cuh"
 
 namespace bq {
 namespace {
 
 constexpr int kWarpsPerBlock = 8;
 constexpr int kCacheChunks = 16;  // 16-byte chunks per lane kept in registers
-constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-
-template <typename In>
-struct Elt;
-template <>
-struct Elt<float> {
-    static constexpr int kPerChunk = 4;
-    __device__ static float get(const float *p, int64_t i) { return p[i]; }
-    __device__ static void unpack(const uint4 &v, float (&f)[4]) {
-        f[0] = __uint_as_float(v.x);
-        f[1] = __uint_as_float(v.y);
-        f[2] = __uint_as_float(v.z);
-        f[3] = __uint_as_float(v.w);
-    }
-};
-template <>
-struct Elt<__nv_bfloat16> {
-    static constexpr int kPerChunk = 8;
-    __device__ static float get(const __nv_bfloat16 *p, int64_t i) { return __bfloat162float(p[i]); }
-    __device__ static void unpack(const uint4 &v, float (&f)[8]) {
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-        }
-    }
-};
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ int warp_isum(int v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
-
-// Low byte of t holds the rounded code (two's complement).
-__device__ __forceinline__ uint32_t pack4(float t0, float t1, float t2, float t3) {
-    const uint32_t p01 = __byte_perm(__float_as_uint(t0), __float_as_uint(t1), 0x0040);
-    const uint32_t p23 = __byte_perm(__float_as_uint(t2), __float_as_uint(t3), 0x0040);
-    return __byte_perm(p01, p23, 0x5410);
-}
-
-// Row statistics -> the code factor f and the row's act_scale.
-__device__ __forceinline__ void row_factor(float ss, float amax, int64_t K, float eps, float &f,
-                                           float &act_scale) {
-    const float ms = __fdiv_rn(ss, static_cast<float>(K));
-    const float r = __fsqrt_rn(__fadd_rn(ms, eps));
-    const float inv_r = __fdiv_rn(1.0f, r);
-    const float a = fmaxf(__fmul_rn(amax, inv_r), 1e-5f);
-    const float qs = __fdiv_rn(127.0f, a);
-    f = __fmul_rn(inv_r, qs);
-    act_scale = __fdiv_rn(a, 127.0f);
-}
 
 // Vector path: row base and stride keep 16-byte alignment.
 template <typename In>
@@ -152,10 +87,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             ss0 = fmaf(xt, xt, ss0);
             amax = fmaxf(amax, fabsf(xt));
         }
-        const float ss = warp_sum(ss0 + ss1);
-        amax = warp_max(amax);
+        const float ss = warp_sum_f(ss0 + ss1);
+        amax = warp_max_f(amax);
         float f, scale;
-        row_factor(ss, amax, K, eps, f, scale);
+        quant_row_factor(ss, amax, K, eps, f, scale);
 
         int isum = 0;
         auto quant_chunk = [&](const uint4 &v, int64_t c) {
@@ -164,8 +99,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             uint32_t w[EPC / 4];
 #pragma unroll
             for (int j = 0; j < EPC / 4; ++j) {
-                w[j] = pack4(fmaf(e[4 * j], f, kMagic), fmaf(e[4 * j + 1], f, kMagic),
-                             fmaf(e[4 * j + 2], f, kMagic), fmaf(e[4 * j + 3], f, kMagic));
+                w[j] = pack_codes4(fmaf(e[4 * j], f, kRoundMagic), fmaf(e[4 * j + 1], f, kRoundMagic),
+                                   fmaf(e[4 * j + 2], f, kRoundMagic), fmaf(e[4 * j + 3], f, kRoundMagic));
                 isum = dp4a_ss(w[j], 0x01010101u, isum);
             }
             if constexpr (EPC == 8) {
@@ -184,12 +119,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             for (int64_t c = lane; c < nchunks; c += 32) quant_chunk(__ldg(xv + c), c);
         }
         if (tail0 + lane < K) {
-            const float t = fmaf(xt, f, kMagic);
-            const int code = static_cast<int>(__float_as_uint(t)) - 0x4B400000;
+            const int code = code_of(fmaf(xt, f, kRoundMagic));
             qr[tail0 + lane] = static_cast<int8_t>(code);
             isum += code;
         }
-        isum = warp_isum(isum);
+        isum = warp_sum_i(isum);
         if (lane == 0) {
             act_scale[m] = scale;
             if (rowsum) rowsum[m] = isum;
@@ -214,18 +148,17 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
             ss = fmaf(v, v, ss);
             amax = fmaxf(amax, fabsf(v));
         }
-        ss = warp_sum(ss);
-        amax = warp_max(amax);
+        ss = warp_sum_f(ss);
+        amax = warp_max_f(amax);
         float f, scale;
-        row_factor(ss, amax, K, eps, f, scale);
+        quant_row_factor(ss, amax, K, eps, f, scale);
         int isum = 0;
         for (int64_t k = lane; k < K; k += 32) {
-            const float t = fmaf(Elt<In>::get(xr, k), f, kMagic);
-            const int code = static_cast<int>(__float_as_uint(t)) - 0x4B400000;
+            const int code = code_of(fmaf(Elt<In>::get(xr, k), f, kRoundMagic));
             xq[m * ldq + k] = static_cast<int8_t>(code);
             isum += code;
         }
-        isum = warp_isum(isum);
+        isum = warp_sum_i(isum);
         if (lane == 0) {
             act_scale[m] = scale;
             if (rowsum) rowsum[m] = isum;

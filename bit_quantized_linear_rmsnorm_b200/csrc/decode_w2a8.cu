@@ -1,0 +1,405 @@
+// Fused BitLinear W1.58A8 decode (M <= 16 tokens): one launch per call.
+//
+// "Class BitLinear" (LLaMA-BitNet utils.py), forward steps 1-5, at inference
+// time (the page: specialised ternary kernels are only needed at inference):
+//   xq, act_scale = per-token int8 quantization of RMSNorm(x)
+//   acc[m,n] = sum_k xq[m,k] * w_q[n,k],   out = (float(acc) * act_scale[m]) * gamma (+ bias)
+//
+// Bandwidth-bound on the 2-bit weights.  One CTA per SM owns a contiguous
+// slice of output rows.  Thread 0 streams the slice's packed rows into a
+// shared-memory ring with cp.async.bulk (16 rows per stage, rows padded by 16
+// bytes so that fragment loads from different rows fall in different banks),
+// while every CTA quantizes the M activation rows itself into shared memory
+// (CTA 0 also writes them to the workspace).  Consumers:
+//   * M <= 2: one warp per weight row, one packed word (16 weights) per lane
+//     step, dp4a of the u8 codes with the s8 activations (for one token the
+//     activations sit in registers and the 2-bit fields are masked in place,
+//     so (word & (3 << 2j)) . x accumulates 4^j times the code dot product).
+//   * M >= 3: mma.sync m16n8k32 u8 x s8 over register fragments.  The packed
+//     layout puts the codes of k = 16w + 4j + b at bits [8b+2j, 8b+2j+1] of
+//     word w, so (word >> 2j) & 0x03030303 is exactly the A fragment of
+//     thread j of a quad (k = 4j..4j+3); the K range is split across the 16
+//     warps and the partial accumulators are reduced in shared memory.
+// The codes are offset binary (w_q + 1), so acc = dot(codes, xq) - rowsum.
+//
+// Programmatic dependent launch: the kernel lets the next kernel of the
+// stream start early and waits for the previous one (griddepcontrol.wait)
+// before its first global memory access.  Every mbarrier wait is bounded.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "bq_internal.h"
+#include "quant_common.cuh"
+
+namespace bq {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int CR = 16;             // weight rows per stage
+constexpr int kMaxKSteps = 16;     // k32 steps per warp in the mma path (K <= 8192)
+constexpr int kMaxWordsPerLane = 16;  // packed words per lane and row in the dp4a path (K <= 8192)
+
+struct DecodeArgs {
+    const void *x;
+    int M, K;
+    float eps;
+    const uint32_t *wpacked;
+    const float *w_scale;
+    const float *bias;
+    int N;
+    void *out;
+    int8_t *ws_xq;
+    float *ws_scale;
+    int32_t *ws_rowsum;
+    int rows_per_cta;
+    int stages;
+    uint32_t *status;
+};
+
+struct Layout {
+    uint32_t rs, xs, off_w, off_x, off_sc, off_rs, off_red, off_bar, off_flag, total;
+    __host__ __device__ Layout(int K, int MT, int S) {
+        rs = K / 4 + 16;
+        xs = K + 16;
+        off_w = 0;
+        off_x = off_w + S * CR * rs;
+        off_sc = off_x + MT * xs;
+        off_rs = off_sc + 4 * MT;
+        off_red = (off_rs + 4 * MT + 15) & ~15u;
+        off_bar = off_red + 2 * CR * 16 * 4;
+        off_flag = off_bar + 2 * S * 8;
+        total = off_flag + 16;
+    }
+};
+
+template <typename OutT>
+__device__ __forceinline__ OutT to_out(float v);
+template <>
+__device__ __forceinline__ float to_out<float>(float v) {
+    return v;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ __half to_out<__half>(float v) {
+    return __float2half_rn(v);
+}
+
+template <int MT, bool MMA, typename InT, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1) decode_w2a8_kernel(const DecodeArgs p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int S = p.stages;
+    const Layout L(p.K, MT, S);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int K = p.K, M = p.M;
+    const int words = K / 16;
+    const uint32_t rowbytes = static_cast<uint32_t>(K / 4);
+    const int n_begin = blockIdx.x * p.rows_per_cta;
+    const int n_end = min(p.N, n_begin + p.rows_per_cta);
+    const int rows = n_end - n_begin;
+    const int nchunks = (rows + CR - 1) / CR;
+    const uint32_t sbase = smem_u32(smem);
+    auto full = [&](int s) { return sbase + L.off_bar + 8u * s; };
+    auto empty = [&](int s) { return sbase + L.off_bar + 8u * (S + s); };
+    int8_t *xs = reinterpret_cast<int8_t *>(smem + L.off_x);
+    float *s_scale = reinterpret_cast<float *>(smem + L.off_sc);
+    int *s_rowsum = reinterpret_cast<int *>(smem + L.off_rs);
+    int *red = reinterpret_cast<int *>(smem + L.off_red);
+    int *fail = reinterpret_cast<int *>(smem + L.off_flag);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), kWarps);
+        }
+        *fail = 0;
+        fence_mbarrier_init();
+    }
+    for (int i = threadIdx.x; i < 2 * CR * 16; i += kThreads) red[i] = 0;
+    pdl_launch_dependents();
+    __syncthreads();
+    pdl_wait();  // previous grid complete and visible: global memory may be touched from here on
+
+    auto issue = [&](int c) {
+        const int stage = c % S;
+        const int rc = min(CR, rows - c * CR);
+        mbar_arrive_expect_tx(full(stage), rc * rowbytes);
+        for (int r = 0; r < rc; ++r)
+            bulk_load(sbase + L.off_w + (stage * CR + r) * L.rs,
+                      p.wpacked + static_cast<int64_t>(n_begin + c * CR + r) * words, rowbytes, full(stage));
+    };
+    int issued = 0;
+    if (threadIdx.x == 0) {
+        for (; issued < min(S, nchunks); ++issued) issue(issued);
+    }
+
+    // per-token activation quantization into shared memory (overlaps the weight stream)
+    for (int m = warp; m < M; m += kWarps) {
+        float sc;
+        int rsum;
+        warp_quant_row_vec<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps,
+                                xs + m * L.xs, blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr,
+                                sc, rsum);
+        if (lane == 0) {
+            s_scale[m] = sc;
+            s_rowsum[m] = rsum;
+            if (blockIdx.x == 0) {
+                p.ws_scale[m] = sc;
+                p.ws_rowsum[m] = rsum;
+            }
+        }
+    }
+    __syncthreads();
+    const float gamma = __ldg(p.w_scale);
+    OutT *out = static_cast<OutT *>(p.out);
+
+    // loop-invariant activation operands of this thread
+    constexpr int NT = (MT + 7) / 8;  // n8 tiles of the mma path
+    uint4 xr[MMA ? 1 : kMaxWordsPerLane];
+    uint32_t bf[MMA ? kMaxKSteps : 1][NT][2];
+    const int g = lane >> 2, t = lane & 3;
+    if constexpr (!MMA) {
+        if constexpr (MT == 1) {
+#pragma unroll
+            for (int j = 0; j < kMaxWordsPerLane; ++j) {
+                const int w = lane + 32 * j;
+                xr[j] = w < words ? *reinterpret_cast<const uint4 *>(xs + 16 * w) : make_uint4(0, 0, 0, 0);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kMaxKSteps; ++j) {
+            const int s = warp + kWarps * j;
+#pragma unroll
+            for (int tile = 0; tile < NT; ++tile) {
+                const int tok = tile * 8 + g;
+                const bool ok = s < K / 32 && tok < M;
+                bf[j][tile][0] = ok ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + 32 * s + 4 * t) : 0u;
+                bf[j][tile][1] = ok ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + 32 * s + 16 + 4 * t) : 0u;
+            }
+        }
+    }
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int stage = c % S;
+        const uint32_t phase = static_cast<uint32_t>(c / S) & 1u;
+        const int rc = min(CR, rows - c * CR);
+        // one decision for the whole CTA: every warp waits, then they agree
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_timed(full(stage), phase, p.status, SITE_DECODE_FULL);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok && lane == 0) atomicOr(fail, 1);
+        named_bar_sync(1, kThreads);
+        if (*reinterpret_cast<volatile int *>(fail)) break;
+        const uint8_t *wst = smem + L.off_w + stage * CR * L.rs;
+
+        if constexpr (!MMA) {
+            const int r = warp;
+            if (r < rc) {
+                const uint32_t *wr = reinterpret_cast<const uint32_t *>(wst + r * L.rs);
+                int acc[MT];
+                int acc4[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int m = 0; m < MT; ++m) acc[m] = 0;
+#pragma unroll
+                for (int j = 0; j < kMaxWordsPerLane; ++j) {
+                    const int w = lane + 32 * j;
+                    if (w < words) {
+                        const uint32_t u = wr[w];
+                        if constexpr (MT == 1) {
+                            acc4[0] = dp4a_us(u & 0x03030303u, xr[j].x, acc4[0]);
+                            acc4[1] = dp4a_us(u & 0x0c0c0c0cu, xr[j].y, acc4[1]);
+                            acc4[2] = dp4a_us(u & 0x30303030u, xr[j].z, acc4[2]);
+                            acc4[3] = dp4a_us(u & 0xc0c0c0c0u, xr[j].w, acc4[3]);
+                        } else {
+                            const uint32_t c0 = u & 0x03030303u, c1 = (u >> 2) & 0x03030303u;
+                            const uint32_t c2 = (u >> 4) & 0x03030303u, c3 = (u >> 6) & 0x03030303u;
+#pragma unroll
+                            for (int m = 0; m < MT; ++m) {
+                                if (m < M) {
+                                    const uint4 x4 = *reinterpret_cast<const uint4 *>(xs + m * L.xs + 16 * w);
+                                    int a = acc[m];
+                                    a = dp4a_us(c0, x4.x, a);
+                                    a = dp4a_us(c1, x4.y, a);
+                                    a = dp4a_us(c2, x4.z, a);
+                                    a = dp4a_us(c3, x4.w, a);
+                                    acc[m] = a;
+                                }
+                            }
+                        }
+                    }
+                }
+                if constexpr (MT == 1) acc[0] = acc4[0] + (acc4[1] >> 2) + (acc4[2] >> 4) + (acc4[3] >> 6);
+                const int n = n_begin + c * CR + r;
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m < M) {
+                        const int dot = warp_sum_i(acc[m]);
+                        if (lane == 0) {
+                            float v = __fmul_rn(__fmul_rn(static_cast<float>(dot - s_rowsum[m]), s_scale[m]), gamma);
+                            if (p.bias) v = __fadd_rn(v, __ldg(p.bias + n));
+                            out[static_cast<int64_t>(m) * p.N + n] = to_out<OutT>(v);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(stage));
+        } else {
+            int C[NT][4];
+#pragma unroll
+            for (int tile = 0; tile < NT; ++tile) C[tile][0] = C[tile][1] = C[tile][2] = C[tile][3] = 0;
+            const uint32_t *rg = reinterpret_cast<const uint32_t *>(wst + g * L.rs);
+            const uint32_t *rh = reinterpret_cast<const uint32_t *>(wst + (g + 8) * L.rs);
+#pragma unroll
+            for (int j = 0; j < kMaxKSteps; ++j) {
+                const int s = warp + kWarps * j;
+                if (s < K / 32) {
+                    const uint32_t sh = 2 * t;
+                    uint32_t a[4];
+                    a[0] = (rg[2 * s] >> sh) & 0x03030303u;
+                    a[1] = (rh[2 * s] >> sh) & 0x03030303u;
+                    a[2] = (rg[2 * s + 1] >> sh) & 0x03030303u;
+                    a[3] = (rh[2 * s + 1] >> sh) & 0x03030303u;
+#pragma unroll
+                    for (int tile = 0; tile < NT; ++tile) mma_u8s8_16832(C[tile], a, bf[j][tile][0], bf[j][tile][1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty(stage));  // this warp is done with the stage
+            int *rb = red + (c & 1) * CR * 16;
+#pragma unroll
+            for (int tile = 0; tile < NT; ++tile) {
+                const int col = tile * 8 + 2 * t;
+                atomicAdd(rb + g * 16 + col, C[tile][0]);
+                atomicAdd(rb + g * 16 + col + 1, C[tile][1]);
+                atomicAdd(rb + (g + 8) * 16 + col, C[tile][2]);
+                atomicAdd(rb + (g + 8) * 16 + col + 1, C[tile][3]);
+            }
+            named_bar_sync(1, kThreads);
+            const int tid = threadIdx.x;
+            if (tid < CR * 16) {
+                const int r = tid >> 4, m = tid & 15;
+                if (r < rc && m < M) {
+                    const int n = n_begin + c * CR + r;
+                    float v = __fmul_rn(__fmul_rn(static_cast<float>(rb[tid] - s_rowsum[m]), s_scale[m]), gamma);
+                    if (p.bias) v = __fadd_rn(v, __ldg(p.bias + n));
+                    out[static_cast<int64_t>(m) * p.N + n] = to_out<OutT>(v);
+                }
+                rb[tid] = 0;  // reused two stages later, after another CTA barrier
+            }
+        }
+
+        // refill the stage just released with chunk c + S
+        if (threadIdx.x == 0 && issued < nchunks) {
+            if (mbar_wait_timed(empty(stage), phase, p.status, SITE_DECODE_EMPTY)) {
+                issue(issued);
+                ++issued;
+            } else {
+                atomicOr(fail, 1);
+            }
+        }
+    }
+    // let every issued copy land before the CTA exits
+    if (threadIdx.x == 0) {
+        for (int c = max(0, issued - S); c < issued; ++c) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(full(c % S), static_cast<uint32_t>(c / S) & 1u) &&
+                   globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    }
+}
+
+template <int MT, bool MMA, typename InT, typename OutT>
+cudaError_t launch_t(const DecodeArgs &a, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
+    auto kern = decode_w2a8_kernel<MT, MMA, InT, OutT>;
+    static int attr_smem[64] = {};
+    if (smem > attr_smem[dev.device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_smem[dev.device] = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <typename InT, typename OutT>
+cudaError_t dispatch_m(const DecodeArgs &a, int MT, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
+    switch (MT) {
+        case 1:
+            return launch_t<1, false, InT, OutT>(a, smem, dev, s, grid);
+        case 2:
+            return launch_t<2, false, InT, OutT>(a, smem, dev, s, grid);
+        case 8:
+            return launch_t<8, true, InT, OutT>(a, smem, dev, s, grid);
+        default:
+            return launch_t<16, true, InT, OutT>(a, smem, dev, s, grid);
+    }
+}
+
+template <typename InT>
+cudaError_t dispatch_out(const DecodeArgs &a, bq_dtype ot, int MT, int smem, const DevInfo &dev, cudaStream_t s,
+                         int grid) {
+    switch (ot) {
+        case BQ_F32:
+            return dispatch_m<InT, float>(a, MT, smem, dev, s, grid);
+        case BQ_F16:
+            return dispatch_m<InT, __half>(a, MT, smem, dev, s, grid);
+        default:
+            return dispatch_m<InT, __nv_bfloat16>(a, MT, smem, dev, s, grid);
+    }
+}
+
+}  // namespace
+
+bool decode_w2a8_supported(const void *x, int64_t M, int64_t K) {
+    return M >= 1 && M <= 16 && K % 64 == 0 && K <= 8192 && reinterpret_cast<uintptr_t>(x) % 16 == 0;
+}
+
+cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
+                               const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
+                               int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,
+                               const DevInfo &dev) {
+    const int MT = M == 1 ? 1 : M == 2 ? 2 : M <= 8 ? 8 : 16;
+    const int rpc = static_cast<int>((N + dev.num_sms - 1) / dev.num_sms);
+    const int grid = static_cast<int>((N + rpc - 1) / rpc);
+    const int nchunks = (rpc + CR - 1) / CR;
+    const int budget = static_cast<int>(dev.max_smem_optin) - 1024;
+    int S = nchunks;
+    while (S > 2 && static_cast<int>(Layout(static_cast<int>(K), MT, S).total) > budget) --S;
+    if (static_cast<int>(Layout(static_cast<int>(K), MT, S).total) > budget) return cudaErrorInvalidConfiguration;
+    DecodeArgs a;
+    a.x = x;
+    a.M = static_cast<int>(M);
+    a.K = static_cast<int>(K);
+    a.eps = eps;
+    a.wpacked = wpacked;
+    a.w_scale = w_scale;
+    a.bias = bias;
+    a.N = static_cast<int>(N);
+    a.out = out;
+    a.ws_xq = ws_xq;
+    a.ws_scale = ws_scale;
+    a.ws_rowsum = ws_rowsum;
+    a.rows_per_cta = rpc;
+    a.stages = S;
+    a.status = dev.status;
+    const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, S).total);
+    if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(a, out_dtype, MT, smem, dev, s, grid);
+    return dispatch_out<float>(a, out_dtype, MT, smem, dev, s, grid);
+}
+
+}  // namespace bq
