@@ -58,7 +58,7 @@ struct DecodeArgs {
 };
 
 struct Layout {
-    uint32_t rs, xs, off_w, off_x, off_sc, off_rs, off_red, off_bar, off_flag, total;
+    uint32_t rs, xs, off_w, off_x, off_sc, off_rs, off_red, off_qred, off_bar, off_flag, total;
     __host__ __device__ Layout(int K, int MT, int S) {
         rs = K / 4 + 16;
         xs = K + 16;
@@ -67,7 +67,8 @@ struct Layout {
         off_sc = off_x + MT * xs;
         off_rs = off_sc + 4 * MT;
         off_red = (off_rs + 4 * MT + 15) & ~15u;
-        off_bar = off_red + 2 * CR * 16 * 4;
+        off_qred = off_red + 2 * CR * 16 * 4;
+        off_bar = off_qred + 3 * MT * kWarps * 4;  // [2][MT][warps] float sums/maxima + [MT][warps] int row sums
         off_flag = off_bar + 2 * S * 8;
         total = off_flag + 16;
     }
@@ -86,6 +87,115 @@ __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) {
 template <>
 __device__ __forceinline__ __half to_out<__half>(float v) {
     return __float2half_rn(v);
+}
+
+// The whole CTA quantizes the M activation rows: every thread issues its
+// 16-byte loads of all rows at once (two passes; the second hits L1/L2), the
+// per-row sums and maxima are reduced warp by warp and then across the 16
+// warps in a fixed order, with the same fp32 arithmetic as the standalone
+// quantization kernel (quant_common.cuh).
+template <int MT, typename InT>
+__device__ __forceinline__ void cta_quant_rows(const InT *__restrict__ x, int M, int K, float eps, int8_t *xs,
+                                               int xs_pitch, int8_t *ws_xq, float *s_scale, int *s_rowsum,
+                                               float *ws_scale, int32_t *ws_rowsum, float *redf, int *redi) {
+    constexpr int EPC = Elt<InT>::kPerChunk;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cpr = K / EPC;  // 16-byte chunks per row
+    float ss[MT], mx[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) ss[m] = mx[m] = 0.f;
+    for (int c = threadIdx.x; c < cpr; c += kThreads) {
+        uint4 v[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+            if (m < M) v[m] = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (m < M) {
+                float f[EPC];
+                Elt<InT>::unpack(v[m], f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) {
+                    ss[m] = fmaf(f[e], f[e], ss[m]);
+                    mx[m] = fmaxf(mx[m], fabsf(f[e]));
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        if (m < M) {
+            const float a = warp_sum_f(ss[m]), b = warp_max_f(mx[m]);
+            if (lane == 0) {
+                redf[m * kWarps + warp] = a;
+                redf[(MT + m) * kWarps + warp] = b;
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < M) {
+        const int m = threadIdx.x;
+        float a = 0.f, b = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+            a += redf[m * kWarps + w];
+            b = fmaxf(b, redf[(MT + m) * kWarps + w]);
+        }
+        float fac, sc;
+        quant_row_factor(a, b, K, eps, fac, sc);
+        redf[m * kWarps] = fac;  // reuse: the code factor of row m
+        s_scale[m] = sc;
+        if (ws_scale) ws_scale[m] = sc;
+    }
+    __syncthreads();
+    int isum[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) isum[m] = 0;
+    for (int c = threadIdx.x; c < cpr; c += kThreads) {
+        uint4 v[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+            if (m < M) v[m] = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            if (m < M) {
+                const float fac = redf[m * kWarps];
+                float e[EPC];
+                Elt<InT>::unpack(v[m], e);
+                uint32_t w[EPC / 4];
+#pragma unroll
+                for (int j = 0; j < EPC / 4; ++j) {
+                    w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
+                                       fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
+                    isum[m] = dp4a_ss(w[j], 0x01010101u, isum[m]);
+                }
+                int8_t *d0 = xs + m * xs_pitch + c * EPC;
+                int8_t *d1 = ws_xq ? ws_xq + static_cast<int64_t>(m) * K + c * EPC : nullptr;
+                if constexpr (EPC == 8) {
+                    *reinterpret_cast<uint2 *>(d0) = make_uint2(w[0], w[1]);
+                    if (d1) *reinterpret_cast<uint2 *>(d1) = make_uint2(w[0], w[1]);
+                } else {
+                    *reinterpret_cast<uint32_t *>(d0) = w[0];
+                    if (d1) *reinterpret_cast<uint32_t *>(d1) = w[0];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        if (m < M) {
+            const int v = warp_sum_i(isum[m]);
+            if (lane == 0) redi[m * kWarps + warp] = v;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < M) {
+        const int m = threadIdx.x;
+        int v = 0;
+        for (int w = 0; w < kWarps; ++w) v += redi[m * kWarps + w];
+        s_rowsum[m] = v;
+        if (ws_rowsum) ws_rowsum[m] = v;
+    }
+    __syncthreads();
 }
 
 template <int MT, bool MMA, typename InT, typename OutT>
@@ -137,22 +247,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_w2a8_kernel(const DecodeAr
     }
 
     // per-token activation quantization into shared memory (overlaps the weight stream)
-    for (int m = warp; m < M; m += kWarps) {
-        float sc;
-        int rsum;
-        warp_quant_row_vec<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps,
-                                xs + m * L.xs, blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr,
-                                sc, rsum);
-        if (lane == 0) {
-            s_scale[m] = sc;
-            s_rowsum[m] = rsum;
-            if (blockIdx.x == 0) {
-                p.ws_scale[m] = sc;
-                p.ws_rowsum[m] = rsum;
-            }
-        }
-    }
-    __syncthreads();
+    cta_quant_rows<MT, InT>(static_cast<const InT *>(p.x), M, K, p.eps, xs, L.xs,
+                            blockIdx.x == 0 ? p.ws_xq : nullptr, s_scale, s_rowsum,
+                            blockIdx.x == 0 ? p.ws_scale : nullptr, blockIdx.x == 0 ? p.ws_rowsum : nullptr,
+                            reinterpret_cast<float *>(smem + L.off_qred),
+                            reinterpret_cast<int *>(smem + L.off_qred) + 2 * MT * kWarps);
     const float gamma = __ldg(p.w_scale);
     OutT *out = static_cast<OutT *>(p.out);
 
