@@ -39,6 +39,7 @@ constexpr int kWarps = kThreads / 32;
 constexpr int CR = 16;             // weight rows per stage
 constexpr int kMaxKSteps = 16;     // k32 steps per warp in the mma path (K <= 8192)
 constexpr int kMaxWordsPerLane = 16;  // packed words per lane and row in the dp4a path (K <= 8192)
+constexpr int kRound = 5;          // chunks per reduction round of the mma path
 
 struct DecodeArgs {
     const void *x;
@@ -58,7 +59,7 @@ struct DecodeArgs {
 };
 
 struct Layout {
-    uint32_t rs, xs, off_w, off_x, off_sc, off_rs, off_red, off_qred, off_bar, off_flag, total;
+    uint32_t rs, xs, off_w, off_x, off_sc, off_rs, off_red, off_qred, off_bar, total;
     __host__ __device__ Layout(int K, int MT, int S) {
         rs = K / 4 + 16;
         xs = K + 16;
@@ -67,10 +68,9 @@ struct Layout {
         off_sc = off_x + MT * xs;
         off_rs = off_sc + 4 * MT;
         off_red = (off_rs + 4 * MT + 15) & ~15u;
-        off_qred = off_red + 2 * CR * 16 * 4;
-        off_bar = off_qred + 3 * MT * kWarps * 4;  // [2][MT][warps] float sums/maxima + [MT][warps] int row sums
-        off_flag = off_bar + 2 * S * 8;
-        total = off_flag + 16;
+        off_qred = off_red + kRound * CR * 16 * 4;
+        off_bar = off_qred + (3 * MT * kWarps + MT) * 4;  // [2][MT][warps] sums/maxima, [MT] factors, [MT][warps] row sums
+        total = off_bar + 2 * S * 8;
     }
 };
 
@@ -99,27 +99,43 @@ __device__ __forceinline__ void cta_quant_rows(const InT *__restrict__ x, int M,
                                                int xs_pitch, int8_t *ws_xq, float *s_scale, int *s_rowsum,
                                                float *ws_scale, int32_t *ws_rowsum, float *redf, int *redi) {
     constexpr int EPC = Elt<InT>::kPerChunk;
+    constexpr int CPT = MT <= 4 ? 4 : (MT <= 8 ? 2 : 1);  // cached 16-byte chunks per thread and row
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cpr = K / EPC;  // 16-byte chunks per row
+    const bool cached = cpr <= CPT * kThreads;
+    uint4 v[MT][CPT];
     float ss[MT], mx[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) ss[m] = mx[m] = 0.f;
-    for (int c = threadIdx.x; c < cpr; c += kThreads) {
-        uint4 v[MT];
+    auto stats = [&](const uint4 &q, int m) {
+        float f[EPC];
+        Elt<InT>::unpack(q, f);
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-            if (m < M) v[m] = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c);
+        for (int e = 0; e < EPC; ++e) {
+            ss[m] = fmaf(f[e], f[e], ss[m]);
+            mx[m] = fmaxf(mx[m], fabsf(f[e]));
+        }
+    };
+    if (cached) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if (m < M) {
-                float f[EPC];
-                Elt<InT>::unpack(v[m], f);
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + i * kThreads;
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) {
-                    ss[m] = fmaf(f[e], f[e], ss[m]);
-                    mx[m] = fmaxf(mx[m], fabsf(f[e]));
-                }
-            }
+            for (int m = 0; m < MT; ++m)
+                if (m < M && c < cpr) v[m][i] = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c);
+        }
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + i * kThreads;
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M && c < cpr) stats(v[m][i], m);
+        }
+    } else {
+        for (int c = threadIdx.x; c < cpr; c += kThreads) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M) stats(__ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c), m);
         }
     }
 #pragma unroll
@@ -142,7 +158,7 @@ __device__ __forceinline__ void cta_quant_rows(const InT *__restrict__ x, int M,
         }
         float fac, sc;
         quant_row_factor(a, b, K, eps, fac, sc);
-        redf[m * kWarps] = fac;  // reuse: the code factor of row m
+        redf[2 * MT * kWarps + m] = fac;
         s_scale[m] = sc;
         if (ws_scale) ws_scale[m] = sc;
     }
@@ -150,50 +166,56 @@ __device__ __forceinline__ void cta_quant_rows(const InT *__restrict__ x, int M,
     int isum[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) isum[m] = 0;
-    for (int c = threadIdx.x; c < cpr; c += kThreads) {
-        uint4 v[MT];
+    auto codes = [&](const uint4 &q, int m, int c) {
+        const float fac = redf[2 * MT * kWarps + m];
+        float e[EPC];
+        Elt<InT>::unpack(q, e);
+        uint32_t w[EPC / 4];
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-            if (m < M) v[m] = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c);
+        for (int j = 0; j < EPC / 4; ++j) {
+            w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
+                               fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
+            isum[m] = dp4a_ss(w[j], 0x01010101u, isum[m]);
+        }
+        int8_t *d0 = xs + m * xs_pitch + c * EPC;
+        int8_t *d1 = ws_xq ? ws_xq + static_cast<int64_t>(m) * K + c * EPC : nullptr;
+        if constexpr (EPC == 8) {
+            *reinterpret_cast<uint2 *>(d0) = make_uint2(w[0], w[1]);
+            if (d1) *reinterpret_cast<uint2 *>(d1) = make_uint2(w[0], w[1]);
+        } else {
+            *reinterpret_cast<uint32_t *>(d0) = w[0];
+            if (d1) *reinterpret_cast<uint32_t *>(d1) = w[0];
+        }
+    };
+    if (cached) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            if (m < M) {
-                const float fac = redf[m * kWarps];
-                float e[EPC];
-                Elt<InT>::unpack(v[m], e);
-                uint32_t w[EPC / 4];
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + i * kThreads;
 #pragma unroll
-                for (int j = 0; j < EPC / 4; ++j) {
-                    w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
-                                       fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
-                    isum[m] = dp4a_ss(w[j], 0x01010101u, isum[m]);
-                }
-                int8_t *d0 = xs + m * xs_pitch + c * EPC;
-                int8_t *d1 = ws_xq ? ws_xq + static_cast<int64_t>(m) * K + c * EPC : nullptr;
-                if constexpr (EPC == 8) {
-                    *reinterpret_cast<uint2 *>(d0) = make_uint2(w[0], w[1]);
-                    if (d1) *reinterpret_cast<uint2 *>(d1) = make_uint2(w[0], w[1]);
-                } else {
-                    *reinterpret_cast<uint32_t *>(d0) = w[0];
-                    if (d1) *reinterpret_cast<uint32_t *>(d1) = w[0];
-                }
-            }
+            for (int m = 0; m < MT; ++m)
+                if (m < M && c < cpr) codes(v[m][i], m, c);
+        }
+    } else {
+        for (int c = threadIdx.x; c < cpr; c += kThreads) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M) codes(__ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K) + c), m, c);
         }
     }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         if (m < M) {
-            const int v = warp_sum_i(isum[m]);
-            if (lane == 0) redi[m * kWarps + warp] = v;
+            const int q = warp_sum_i(isum[m]);
+            if (lane == 0) redi[m * kWarps + warp] = q;
         }
     }
     __syncthreads();
     if (threadIdx.x < M) {
         const int m = threadIdx.x;
-        int v = 0;
-        for (int w = 0; w < kWarps; ++w) v += redi[m * kWarps + w];
-        s_rowsum[m] = v;
-        if (ws_rowsum) ws_rowsum[m] = v;
+        int q = 0;
+        for (int w = 0; w < kWarps; ++w) q += redi[m * kWarps + w];
+        s_rowsum[m] = q;
+        if (ws_rowsum) ws_rowsum[m] = q;
     }
     __syncthreads();
 }
@@ -218,49 +240,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_w2a8_kernel(const DecodeAr
     float *s_scale = reinterpret_cast<float *>(smem + L.off_sc);
     int *s_rowsum = reinterpret_cast<int *>(smem + L.off_rs);
     int *red = reinterpret_cast<int *>(smem + L.off_red);
-    int *fail = reinterpret_cast<int *>(smem + L.off_flag);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), kWarps);
         }
-        *fail = 0;
         fence_mbarrier_init();
     }
-    for (int i = threadIdx.x; i < 2 * CR * 16; i += kThreads) red[i] = 0;
+    if constexpr (MMA)
+        for (int i = threadIdx.x; i < kRound * CR * 16; i += kThreads) red[i] = 0;
     pdl_launch_dependents();
     __syncthreads();
     pdl_wait();  // previous grid complete and visible: global memory may be touched from here on
 
-    auto issue = [&](int c) {
+    // Warp 0 streams the slice's packed rows: lane 0 arms each stage with its
+    // byte count, then the 32 lanes issue the row copies.
+    auto issue = [&](int c) {  // warp 0 only
         const int stage = c % S;
         const int rc = min(CR, rows - c * CR);
-        mbar_arrive_expect_tx(full(stage), rc * rowbytes);
-        for (int r = 0; r < rc; ++r)
+        if (lane == 0) mbar_arrive_expect_tx(full(stage), rc * rowbytes);
+        __syncwarp();
+        for (int r = lane; r < rc; r += 32)
             bulk_load(sbase + L.off_w + (stage * CR + r) * L.rs,
                       p.wpacked + static_cast<int64_t>(n_begin + c * CR + r) * words, rowbytes, full(stage));
     };
-    int issued = 0;
-    if (threadIdx.x == 0) {
-        for (; issued < min(S, nchunks); ++issued) issue(issued);
-    }
+    int issued = min(S, nchunks);
+    if (warp == 0)
+        for (int c = 0; c < issued; ++c) issue(c);
 
     // per-token activation quantization into shared memory (overlaps the weight stream)
     cta_quant_rows<MT, InT>(static_cast<const InT *>(p.x), M, K, p.eps, xs, L.xs,
                             blockIdx.x == 0 ? p.ws_xq : nullptr, s_scale, s_rowsum,
                             blockIdx.x == 0 ? p.ws_scale : nullptr, blockIdx.x == 0 ? p.ws_rowsum : nullptr,
                             reinterpret_cast<float *>(smem + L.off_qred),
-                            reinterpret_cast<int *>(smem + L.off_qred) + 2 * MT * kWarps);
+                            reinterpret_cast<int *>(smem + L.off_qred) + 2 * MT * kWarps + MT);
     const float gamma = __ldg(p.w_scale);
     OutT *out = static_cast<OutT *>(p.out);
 
-    // loop-invariant activation operands of this thread
-    constexpr int NT = (MT + 7) / 8;  // n8 tiles of the mma path
-    uint4 xr[MMA ? 1 : kMaxWordsPerLane];
-    uint32_t bf[MMA ? kMaxKSteps : 1][NT][2];
-    const int g = lane >> 2, t = lane & 3;
+    // Waits (bounded) for chunk c; warp-uniform result.
+    auto wait_chunk = [&](int c) -> bool {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_timed(full(c % S), static_cast<uint32_t>(c / S) & 1u, p.status, SITE_DECODE_FULL);
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    };
+    // Warp 0 refills the stage of chunk c with chunk c + S once every warp released it.
+    auto refill = [&](int c) {
+        if (warp == 0 && issued < nchunks) {
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_timed(empty(c % S), static_cast<uint32_t>(c / S) & 1u, p.status, SITE_DECODE_EMPTY);
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+                issue(issued);
+                ++issued;
+            }
+        }
+    };
+
     if constexpr (!MMA) {
+        // one weight row per warp and chunk: warp w owns row w of every chunk
+        uint4 xr[kMaxWordsPerLane];
         if constexpr (MT == 1) {
 #pragma unroll
             for (int j = 0; j < kMaxWordsPerLane; ++j) {
@@ -268,37 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_w2a8_kernel(const DecodeAr
                 xr[j] = w < words ? *reinterpret_cast<const uint4 *>(xs + 16 * w) : make_uint4(0, 0, 0, 0);
             }
         }
-    } else {
-#pragma unroll
-        for (int j = 0; j < kMaxKSteps; ++j) {
-            const int s = warp + kWarps * j;
-#pragma unroll
-            for (int tile = 0; tile < NT; ++tile) {
-                const int tok = tile * 8 + g;
-                const bool ok = s < K / 32 && tok < M;
-                bf[j][tile][0] = ok ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + 32 * s + 4 * t) : 0u;
-                bf[j][tile][1] = ok ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + 32 * s + 16 + 4 * t) : 0u;
-            }
-        }
-    }
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int stage = c % S;
-        const uint32_t phase = static_cast<uint32_t>(c / S) & 1u;
-        const int rc = min(CR, rows - c * CR);
-        // one decision for the whole CTA: every warp waits, then they agree
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_timed(full(stage), phase, p.status, SITE_DECODE_FULL);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok && lane == 0) atomicOr(fail, 1);
-        named_bar_sync(1, kThreads);
-        if (*reinterpret_cast<volatile int *>(fail)) break;
-        const uint8_t *wst = smem + L.off_w + stage * CR * L.rs;
-
-        if constexpr (!MMA) {
+        for (int c = 0; c < nchunks; ++c) {
+            if (!wait_chunk(c)) break;
+            const int stage = c % S;
+            const int rc = min(CR, rows - c * CR);
             const int r = warp;
             if (r < rc) {
-                const uint32_t *wr = reinterpret_cast<const uint32_t *>(wst + r * L.rs);
+                const uint32_t *wr = reinterpret_cast<const uint32_t *>(smem + L.off_w + (stage * CR + r) * L.rs);
                 int acc[MT];
                 int acc4[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -331,6 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_w2a8_kernel(const DecodeAr
                         }
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty(stage));  // the row has been read
                 if constexpr (MT == 1) acc[0] = acc4[0] + (acc4[1] >> 2) + (acc4[2] >> 4) + (acc4[3] >> 6);
                 const int n = n_begin + c * CR + r;
 #pragma unroll
@@ -344,66 +360,101 @@ __global__ void __launch_bounds__(kThreads, 1) decode_w2a8_kernel(const DecodeAr
                         }
                     }
                 }
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty(stage));
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty(stage));
-        } else {
-            int C[NT][4];
+            refill(c);
+        }
+    } else {
+        // K split across the 16 warps; each warp keeps one accumulator set per
+        // chunk of a round and the round ends with one shared-memory reduction.
+        constexpr int NT = (MT + 7) / 8;  // n8 tiles
+        const int g = lane >> 2, t = lane & 3;
+        uint32_t bf[kMaxKSteps][NT][2];
 #pragma unroll
-            for (int tile = 0; tile < NT; ++tile) C[tile][0] = C[tile][1] = C[tile][2] = C[tile][3] = 0;
-            const uint32_t *rg = reinterpret_cast<const uint32_t *>(wst + g * L.rs);
-            const uint32_t *rh = reinterpret_cast<const uint32_t *>(wst + (g + 8) * L.rs);
-#pragma unroll
-            for (int j = 0; j < kMaxKSteps; ++j) {
-                const int s = warp + kWarps * j;
-                if (s < K / 32) {
-                    const uint32_t sh = 2 * t;
-                    uint32_t a[4];
-                    a[0] = (rg[2 * s] >> sh) & 0x03030303u;
-                    a[1] = (rh[2 * s] >> sh) & 0x03030303u;
-                    a[2] = (rg[2 * s + 1] >> sh) & 0x03030303u;
-                    a[3] = (rh[2 * s + 1] >> sh) & 0x03030303u;
-#pragma unroll
-                    for (int tile = 0; tile < NT; ++tile) mma_u8s8_16832(C[tile], a, bf[j][tile][0], bf[j][tile][1]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty(stage));  // this warp is done with the stage
-            int *rb = red + (c & 1) * CR * 16;
+        for (int j = 0; j < kMaxKSteps; ++j) {
+            const int s = warp + kWarps * j;
 #pragma unroll
             for (int tile = 0; tile < NT; ++tile) {
-                const int col = tile * 8 + 2 * t;
-                atomicAdd(rb + g * 16 + col, C[tile][0]);
-                atomicAdd(rb + g * 16 + col + 1, C[tile][1]);
-                atomicAdd(rb + (g + 8) * 16 + col, C[tile][2]);
-                atomicAdd(rb + (g + 8) * 16 + col + 1, C[tile][3]);
+                const int tok = tile * 8 + g;
+                const bool ok = s < K / 32 && tok < M;
+                bf[j][tile][0] = ok ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + 32 * s + 4 * t) : 0u;
+                bf[j][tile][1] = ok ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + 32 * s + 16 + 4 * t) : 0u;
             }
-            named_bar_sync(1, kThreads);
-            const int tid = threadIdx.x;
-            if (tid < CR * 16) {
-                const int r = tid >> 4, m = tid & 15;
+        }
+        for (int c0 = 0; c0 < nchunks; c0 += kRound) {
+            const int cn = min(kRound, nchunks - c0);
+            int C[kRound][NT][4];
+#pragma unroll
+            for (int i = 0; i < kRound; ++i)
+#pragma unroll
+                for (int tile = 0; tile < NT; ++tile) C[i][tile][0] = C[i][tile][1] = C[i][tile][2] = C[i][tile][3] = 0;
+            bool ok = true;
+#pragma unroll
+            for (int i = 0; i < kRound; ++i) {
+                if (i < cn && ok) {
+                    const int c = c0 + i;
+                    ok = wait_chunk(c);
+                    if (ok) {
+                        const int stage = c % S;
+                        const uint8_t *wst = smem + L.off_w + stage * CR * L.rs;
+                        const uint32_t *rg = reinterpret_cast<const uint32_t *>(wst + g * L.rs);
+                        const uint32_t *rh = reinterpret_cast<const uint32_t *>(wst + (g + 8) * L.rs);
+#pragma unroll
+                        for (int j = 0; j < kMaxKSteps; ++j) {
+                            const int s = warp + kWarps * j;
+                            if (s < K / 32) {
+                                const uint32_t sh = 2 * t;
+                                uint32_t a[4];
+                                a[0] = (rg[2 * s] >> sh) & 0x03030303u;
+                                a[1] = (rh[2 * s] >> sh) & 0x03030303u;
+                                a[2] = (rg[2 * s + 1] >> sh) & 0x03030303u;
+                                a[3] = (rh[2 * s + 1] >> sh) & 0x03030303u;
+#pragma unroll
+                                for (int tile = 0; tile < NT; ++tile)
+                                    mma_u8s8_16832(C[i][tile], a, bf[j][tile][0], bf[j][tile][1]);
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(empty(stage));
+                        refill(c);
+                    }
+                }
+            }
+            // reduce the round across warps (every warp reaches this barrier)
+#pragma unroll
+            for (int i = 0; i < kRound; ++i) {
+                if (i < cn) {
+                    int *rb = red + i * CR * 16;
+#pragma unroll
+                    for (int tile = 0; tile < NT; ++tile) {
+                        const int col = tile * 8 + 2 * t;
+                        atomicAdd(rb + g * 16 + col, C[i][tile][0]);
+                        atomicAdd(rb + g * 16 + col + 1, C[i][tile][1]);
+                        atomicAdd(rb + (g + 8) * 16 + col, C[i][tile][2]);
+                        atomicAdd(rb + (g + 8) * 16 + col + 1, C[i][tile][3]);
+                    }
+                }
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < cn * CR * 16; e += kThreads) {
+                const int i = e / (CR * 16), r = (e / 16) % CR, m = e % 16;
+                const int c = c0 + i;
+                const int rc = min(CR, rows - c * CR);
                 if (r < rc && m < M) {
                     const int n = n_begin + c * CR + r;
-                    float v = __fmul_rn(__fmul_rn(static_cast<float>(rb[tid] - s_rowsum[m]), s_scale[m]), gamma);
+                    float v = __fmul_rn(__fmul_rn(static_cast<float>(red[e] - s_rowsum[m]), s_scale[m]), gamma);
                     if (p.bias) v = __fadd_rn(v, __ldg(p.bias + n));
                     out[static_cast<int64_t>(m) * p.N + n] = to_out<OutT>(v);
                 }
-                rb[tid] = 0;  // reused two stages later, after another CTA barrier
+                red[e] = 0;
             }
-        }
-
-        // refill the stage just released with chunk c + S
-        if (threadIdx.x == 0 && issued < nchunks) {
-            if (mbar_wait_timed(empty(stage), phase, p.status, SITE_DECODE_EMPTY)) {
-                issue(issued);
-                ++issued;
-            } else {
-                atomicOr(fail, 1);
-            }
+            __syncthreads();
         }
     }
     // let every issued copy land before the CTA exits
-    if (threadIdx.x == 0) {
+    if (warp == 0 && lane == 0) {
         for (int c = max(0, issued - S); c < issued; ++c) {
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(full(c % S), static_cast<uint32_t>(c / S) & 1u) &&
