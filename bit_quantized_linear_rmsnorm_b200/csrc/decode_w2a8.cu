@@ -63,14 +63,22 @@ struct Layout {
     __host__ __device__ Layout(int K, int MT, int S) {
         rs = K / 4 + 16;
         xs = K + 16;
+        // every region starts on a 16-byte boundary (bulk-copy targets, uint4
+        // accesses and the 8-byte mbarriers all rely on it)
         off_w = 0;
-        off_x = off_w + S * CR * rs;
-        off_sc = off_x + MT * xs;
-        off_rs = off_sc + 4 * MT;
-        off_red = (off_rs + 4 * MT + 15) & ~15u;
-        off_qred = off_red + kRound * CR * 16 * 4;
-        off_bar = off_qred + (3 * MT * kWarps + MT) * 4;  // [2][MT][warps] sums/maxima, [MT] factors, [MT][warps] row sums
+        off_x = a16(off_w + S * CR * rs);
+        off_sc = a16(off_x + MT * xs);
+        off_rs = a16(off_sc + 4 * MT);
+        off_red = a16(off_rs + 4 * MT);
+        off_qred = a16(off_red + kRound * CR * 16 * 4);
+        // [2][MT][warps] sums/maxima, [MT] code factors, [MT][warps] row sums
+        off_bar = a16(off_qred + (3 * MT * kWarps + MT) * 4);
         total = off_bar + 2 * S * 8;
+    }
+    __host__ __device__ static uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
+    __host__ bool aligned_ok() const {
+        return rs % 16 == 0 && xs % 16 == 0 && off_x % 16 == 0 && off_red % 16 == 0 && off_qred % 16 == 0 &&
+               off_bar % 8 == 0;
     }
 };
 
@@ -547,7 +555,9 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.rows_per_cta = rpc;
     a.stages = S;
     a.status = dev.status;
-    const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, S).total);
+    const Layout lay(static_cast<int>(K), MT, S);
+    if (!lay.aligned_ok()) return cudaErrorInvalidConfiguration;
+    const int smem = static_cast<int>(lay.total);
     if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(a, out_dtype, MT, smem, dev, s, grid);
     return dispatch_out<float>(a, out_dtype, MT, smem, dev, s, grid);
 }
