@@ -243,7 +243,7 @@ bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t 
     float *act_scale = reinterpret_cast<float *>(ws + sc_off);
     int32_t *rowsum = reinterpret_cast<int32_t *>(ws + rs_off);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (!gemm_path && decode_w2a8_supported(x, M, K))
+    if (!gemm_path && decode_w2a8_supported(x, M, N, K, dev))
         return from_cuda(launch_decode_w2a8(x, x_dtype, M, K, eps, wpacked, w_scale, bias, N, out_dtype, out, xq,
                                             act_scale, rowsum, s, dev));
     cudaError_t e = launch_act_quant(x, x_dtype, M, K, K, eps, xq, K, act_scale, rowsum, s, dev);

@@ -61,7 +61,7 @@ cudaError_t launch_gemv_w2a8(const int8_t *xq, int64_t ldq, const float *act_sca
 // Fused single-launch decode path (M <= 16) of the ternary linear: per-CTA
 // activation quantization + bulk-streamed packed weights.  Writes xq,
 // act_scale and rowsum to the workspace as well.
-bool decode_w2a8_supported(const void *x, int64_t M, int64_t K);
+bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const DevInfo &dev);
 cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
                                const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
                                int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,
