@@ -192,9 +192,14 @@ def graph_time(fn_for_step, steps: int, warmup: int, dist=None, clocks=None):
     with torch.cuda.graph(g, stream=s):
         for i in range(steps):
             fn_for_step(i)
-    # warm replay of the graph itself
-    g.replay()
-    s.synchronize()
+    # warm replays of the graph itself, for at least 50 ms so that the SM
+    # clocks have left their idle level before the timed replay
+    t_end = time.perf_counter() + 0.05
+    while True:
+        g.replay()
+        s.synchronize()
+        if time.perf_counter() >= t_end:
+            break
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
