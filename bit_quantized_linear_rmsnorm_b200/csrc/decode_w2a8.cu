@@ -5,30 +5,33 @@
 //   xq, act_scale = per-token int8 quantization of RMSNorm(x)
 //   acc[m,n] = sum_k xq[m,k] * w_q[n,k],   out = (float(acc) * act_scale[m]) * gamma (+ bias)
 //
-// Bandwidth-bound on the 2-bit weights.  One CTA per SM owns RB consecutive
-// output rows.  Its packed rows arrive in K slices: one 2-D TMA copy per
-// 128-byte slice of every row (box 32 words x RB rows, 128-byte swizzle), all
-// issued at once, each completing on its own mbarrier.  A handful of large
-// copies per CTA keeps the copy engine off the critical path; the swizzle
-// keeps the fragment loads below free of bank conflicts.  Meanwhile one warp
-// per token quantizes the activations (row held in registers, same fp32
-// arithmetic as the standalone kernel) into shared memory; CTA 0 also writes
-// them to the workspace.
-//   * M <= 2: warp w owns rows w, w+16, ...; per slice each lane takes one
-//     packed word (16 weights) of a row and runs dp4a of the u8 codes with the
-//     s8 activations (one token: activations in registers, 2-bit fields
-//     masked in place so (word & (3 << 2j)) . x accumulates 4^j times the code
-//     dot product).
+// Bandwidth-bound on the 2-bit weights.  One CTA owns RB consecutive output
+// rows; its packed rows are read in K slices (128 bytes of every row: one 2-D
+// TMA box of 32 words x RB rows, 128-byte swizzle, so fragment loads are free
+// of bank conflicts) through a ring of shared-memory stages.
+//
+// Overlap across calls.  A CTA is small enough (256 threads, <= 128
+// registers, a few slice stages) for two to share an SM, and each kernel
+// lets the next kernel of the stream launch at once (programmatic dependent
+// launch).  Before griddepcontrol.wait a CTA only prefetches its weight
+// slices into L2 -- nothing is consumed, so this is correct whatever the
+// previous kernel wrote -- and after the wait it reads them from L2.  So the
+// weight stream of call i+1 overlaps the tail of call i.
+//
+// After the wait, one warp per token quantizes the activations (row held in
+// registers, same fp32 arithmetic as the standalone kernel) into shared
+// memory; CTA 0 also writes them to the workspace.  Then:
+//   * M <= 2: warp w owns rows w, w+8, ...; per slice each lane takes one
+//     packed word (16 weights) of a row: dp4a of the u8 codes with the s8
+//     activations (one token: the 2-bit fields are masked in place, so
+//     (word & (3 << 2j)) . x accumulates 4^j times the code dot product).
 //   * M >= 3: mma.sync m16n8k32 u8 x s8.  The packed layout puts the codes of
 //     k = 16w + 4j + b at bits [8b+2j, 8b+2j+1] of word w, so
 //     (word >> 2j) & 0x03030303 is the A fragment of quad thread j; warp w
-//     takes k-step w of every slice for all 16-row blocks, and the partial
-//     accumulators are reduced across warps once, at the end.
+//     takes k-steps 2w and 2w+1 of every slice for all 16-row blocks, and
+//     the partial accumulators are reduced across warps once, at the end.
 // The codes are offset binary (w_q + 1), so acc = dot(codes, xq) - rowsum.
-//
-// Programmatic dependent launch: the kernel lets the next kernel of the
-// stream start early and waits for the previous one (griddepcontrol.wait)
-// before its first global memory access.  Every mbarrier wait is bounded.
+// Every mbarrier wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -39,13 +42,14 @@
 namespace bq {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kSliceWords = 32;               // 128 bytes of each packed row per slice
 constexpr int kMaxSlices = 16;                // K <= 8192
 constexpr int kMaxRB = 96;                    // rows per CTA
 constexpr int kMaxBlocks = kMaxRB / 16;       // 16-row blocks of the mma path
 constexpr int kMaxRowsPerWarp = kMaxRB / kWarps;
+constexpr int kStages = 4;                    // slice stages in shared memory
 
 struct DecodeArgs {
     const void *x;
@@ -63,17 +67,18 @@ struct DecodeArgs {
 };
 
 struct Layout {
-    uint32_t slice_bytes, nslices, xs, off_x, off_sc, off_rs, off_red, off_bar, total;
+    uint32_t slice_bytes, nslices, stages, xs, off_x, off_sc, off_rs, off_red, off_bar, total;
     __host__ __device__ Layout(int K, int MT, int rb) {
         nslices = static_cast<uint32_t>(K / (16 * kSliceWords));
+        stages = nslices < static_cast<uint32_t>(kStages) ? nslices : static_cast<uint32_t>(kStages);
         slice_bytes = (static_cast<uint32_t>(rb) * 128u + 1023u) & ~1023u;  // 1024-aligned for the swizzle
         xs = static_cast<uint32_t>(K) + 16u;                                 // padded token rows
-        off_x = nslices * slice_bytes;
+        off_x = stages * slice_bytes;
         off_sc = a16(off_x + MT * xs);
         off_rs = a16(off_sc + 4 * MT);
         off_red = a16(off_rs + 4 * MT);
-        off_bar = a16(off_red + kMaxRB * 16 * 4);
-        total = off_bar + 8 * nslices;
+        off_bar = a16(off_red + (MT > 2 ? kMaxRB * 16 * 4 : 0));
+        total = off_bar + 16 * stages;  // full[stages], empty[stages]
     }
     __host__ __device__ static uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
 };
@@ -167,56 +172,61 @@ __device__ __forceinline__ void warp_quant_token(const InT *__restrict__ xr, int
 }
 
 template <int MT, bool MMA, typename InT, typename OutT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     decode_w2a8_kernel(const __grid_constant__ CUtensorMap tmW, const DecodeArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = p.K, M = p.M;
     const Layout L(K, MT, p.rb);
-    const int ns = static_cast<int>(L.nslices);
+    const int ns = static_cast<int>(L.nslices), S = static_cast<int>(L.stages);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_begin = blockIdx.x * p.rb;
     const int rows = min(p.rb, p.N - n_begin);
     const uint32_t sbase = smem_u32(smem);
-    auto bar = [&](int s) { return sbase + L.off_bar + 8u * s; };
+    auto full = [&](int i) { return sbase + L.off_bar + 8u * i; };
+    auto empty = [&](int i) { return sbase + L.off_bar + 8u * (S + i); };
     int8_t *xs = reinterpret_cast<int8_t *>(smem + L.off_x);
     float *s_scale = reinterpret_cast<float *>(smem + L.off_sc);
     int *s_rowsum = reinterpret_cast<int *>(smem + L.off_rs);
     int *red = reinterpret_cast<int *>(smem + L.off_red);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < ns; ++s) mbar_init(bar(s), 1);
-        fence_mbarrier_init();
         tma_prefetch_desc(&tmW);
+        // pull this CTA's weights toward L2 while the previous grid finishes
+        for (int s = 0; s < ns; ++s) tma_prefetch_l2_2d(&tmW, s * kSliceWords, n_begin);
+        for (int i = 0; i < S; ++i) {
+            mbar_init(full(i), 1);
+            mbar_init(empty(i), kWarps);
+        }
+        fence_mbarrier_init();
     }
     if constexpr (MMA)
         for (int i = threadIdx.x; i < kMaxRB * 16; i += kThreads) red[i] = 0;
     pdl_launch_dependents();
     __syncthreads();
-    pdl_wait();  // previous grid complete and visible: global memory may be touched from here on
+    pdl_wait();  // previous grid complete and visible: data may be consumed from here on
 
-    // all K slices of this CTA's rows, one TMA copy each
-    if (threadIdx.x == 0) {
-        const uint32_t bytes = static_cast<uint32_t>(p.rb) * 128u;  // full box, rows past N read as zero
-        for (int s = 0; s < ns; ++s) {
-            mbar_arrive_expect_tx(bar(s), bytes);
-            tma_load_2d(sbase + s * L.slice_bytes, &tmW, s * kSliceWords, n_begin, bar(s));
-        }
-    }
+    const uint32_t slice_tx = static_cast<uint32_t>(p.rb) * 128u;  // full box; rows past N read as zero
+    auto load_slice = [&](int s) {  // one thread
+        const int st = s % S;
+        mbar_arrive_expect_tx(full(st), slice_tx);
+        tma_load_2d(sbase + st * L.slice_bytes, &tmW, s * kSliceWords, n_begin, full(st));
+    };
+    if (threadIdx.x == 0)
+        for (int s = 0; s < S; ++s) load_slice(s);
 
-    // per-token activation quantization (overlaps the weight stream)
-    if (warp < M) {
+    // per-token activation quantization
+    for (int m = warp; m < M; m += kWarps) {
         float sc;
         int rsum;
-        warp_quant_token<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(warp) * K, K, p.eps,
-                              xs + warp * L.xs, blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(warp) * K : nullptr,
-                              sc, rsum);
+        warp_quant_token<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps, xs + m * L.xs,
+                              blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr, sc, rsum);
         if (lane == 0) {
-            s_scale[warp] = sc;
-            s_rowsum[warp] = rsum;
+            s_scale[m] = sc;
+            s_rowsum[m] = rsum;
             if (blockIdx.x == 0) {
-                p.ws_scale[warp] = sc;
-                p.ws_rowsum[warp] = rsum;
+                p.ws_scale[m] = sc;
+                p.ws_rowsum[m] = rsum;
             }
         }
     }
@@ -224,21 +234,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float gamma = __ldg(p.w_scale);
     OutT *out = static_cast<OutT *>(p.out);
 
-    auto wait_slice = [&](int s) -> bool {  // warp-uniform
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait_timed(bar(s), 0, p.status, SITE_DECODE_FULL);
-        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    bool ok = true;
+    auto wait_full = [&](int s) -> bool {  // warp-uniform
+        bool good = true;
+        if (lane == 0) good = mbar_wait_timed(full(s % S), static_cast<uint32_t>(s / S) & 1u, p.status, SITE_DECODE_FULL);
+        return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+    };
+    auto release = [&](int s) {  // every warp, once per slice; thread 0 refills the stage
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty(s % S));
+        if (threadIdx.x == 0 && s + S < ns) {
+            if (mbar_wait_timed(empty(s % S), static_cast<uint32_t>(s / S) & 1u, p.status, SITE_DECODE_EMPTY))
+                load_slice(s + S);
+        }
     };
 
     if constexpr (!MMA) {
-        // rows r = warp + 16 i of this CTA; lane l takes word l of each slice
-        uint4 xr[kMaxSlices];
-        if constexpr (MT == 1) {
-#pragma unroll
-            for (int s = 0; s < kMaxSlices; ++s)
-                xr[s] = s < ns ? *reinterpret_cast<const uint4 *>(xs + 16 * (s * kSliceWords + lane))
-                               : make_uint4(0, 0, 0, 0);
-        }
+        // rows r = warp + 8 i of this CTA; lane l takes word l of each slice
         int acc[kMaxRowsPerWarp][MT];
         int acc4[kMaxRowsPerWarp][4];
 #pragma unroll
@@ -248,44 +260,41 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc4[i][j] = 0;
         }
-        bool ok = true;
+        for (int s = 0; s < ns && ok; ++s) {
+            ok = wait_full(s);
+            if (!ok) break;
+            const uint8_t *sl = smem + (s % S) * L.slice_bytes;
+            uint4 x4[MT];
 #pragma unroll
-        for (int s = 0; s < kMaxSlices; ++s) {
-            if (s < ns && ok) {
-                ok = wait_slice(s);
-                if (ok) {
-                    const uint8_t *sl = smem + s * L.slice_bytes;
+            for (int m = 0; m < MT; ++m)
+                x4[m] = m < M ? *reinterpret_cast<const uint4 *>(xs + m * L.xs + 16 * (s * kSliceWords + lane))
+                              : make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int i = 0; i < kMaxRowsPerWarp; ++i) {
-                        const int r = warp + kWarps * i;
-                        if (r < rows) {
-                            const uint32_t u = *reinterpret_cast<const uint32_t *>(sl + swz(r, lane));
-                            if constexpr (MT == 1) {
-                                acc4[i][0] = dp4a_us(u & 0x03030303u, xr[s].x, acc4[i][0]);
-                                acc4[i][1] = dp4a_us(u & 0x0c0c0c0cu, xr[s].y, acc4[i][1]);
-                                acc4[i][2] = dp4a_us(u & 0x30303030u, xr[s].z, acc4[i][2]);
-                                acc4[i][3] = dp4a_us(u & 0xc0c0c0c0u, xr[s].w, acc4[i][3]);
-                            } else {
-                                const uint32_t c0 = u & 0x03030303u, c1 = (u >> 2) & 0x03030303u;
-                                const uint32_t c2 = (u >> 4) & 0x03030303u, c3 = (u >> 6) & 0x03030303u;
+            for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+                const int r = warp + kWarps * i;
+                if (r < rows) {
+                    const uint32_t u = *reinterpret_cast<const uint32_t *>(sl + swz(r, lane));
+                    if constexpr (MT == 1) {
+                        acc4[i][0] = dp4a_us(u & 0x03030303u, x4[0].x, acc4[i][0]);
+                        acc4[i][1] = dp4a_us(u & 0x0c0c0c0cu, x4[0].y, acc4[i][1]);
+                        acc4[i][2] = dp4a_us(u & 0x30303030u, x4[0].z, acc4[i][2]);
+                        acc4[i][3] = dp4a_us(u & 0xc0c0c0c0u, x4[0].w, acc4[i][3]);
+                    } else {
+                        const uint32_t c0 = u & 0x03030303u, c1 = (u >> 2) & 0x03030303u;
+                        const uint32_t c2 = (u >> 4) & 0x03030303u, c3 = (u >> 6) & 0x03030303u;
 #pragma unroll
-                                for (int m = 0; m < MT; ++m) {
-                                    if (m < M) {
-                                        const uint4 x4 = *reinterpret_cast<const uint4 *>(
-                                            xs + m * L.xs + 16 * (s * kSliceWords + lane));
-                                        int a = acc[i][m];
-                                        a = dp4a_us(c0, x4.x, a);
-                                        a = dp4a_us(c1, x4.y, a);
-                                        a = dp4a_us(c2, x4.z, a);
-                                        a = dp4a_us(c3, x4.w, a);
-                                        acc[i][m] = a;
-                                    }
-                                }
-                            }
+                        for (int m = 0; m < MT; ++m) {
+                            int a = acc[i][m];
+                            a = dp4a_us(c0, x4[m].x, a);
+                            a = dp4a_us(c1, x4[m].y, a);
+                            a = dp4a_us(c2, x4[m].z, a);
+                            a = dp4a_us(c3, x4[m].w, a);
+                            acc[i][m] = a;
                         }
                     }
                 }
             }
+            release(s);
         }
         if (ok) {
 #pragma unroll
@@ -319,38 +328,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < kMaxBlocks; ++b)
 #pragma unroll
             for (int tile = 0; tile < NT; ++tile) C[b][tile][0] = C[b][tile][1] = C[b][tile][2] = C[b][tile][3] = 0;
-        bool ok = true;
+        for (int s = 0; s < ns && ok; ++s) {
+            ok = wait_full(s);
+            if (!ok) break;
+            const uint8_t *sl = smem + (s % S) * L.slice_bytes;
+            const uint32_t sh = 2 * t;
 #pragma unroll
-        for (int s = 0; s < kMaxSlices; ++s) {
-            if (s < ns && ok) {
-                // B fragments of k-step (s * 16 + warp): activations of tokens g (+8 per tile)
+            for (int h = 0; h < 2; ++h) {  // k-steps 2*warp + h of this slice
+                const int ks = 2 * warp + h;
+                const int k0 = 32 * (s * 16 + ks);
                 uint32_t bf[NT][2];
-                const int k0 = 32 * (s * 16 + warp);
 #pragma unroll
                 for (int tile = 0; tile < NT; ++tile) {
                     const int tok = tile * 8 + g;
                     bf[tile][0] = tok < M ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + k0 + 4 * t) : 0u;
                     bf[tile][1] = tok < M ? *reinterpret_cast<const uint32_t *>(xs + tok * L.xs + k0 + 16 + 4 * t) : 0u;
                 }
-                ok = wait_slice(s);
-                if (ok) {
-                    const uint8_t *sl = smem + s * L.slice_bytes;
-                    const uint32_t sh = 2 * t;
 #pragma unroll
-                    for (int b = 0; b < kMaxBlocks; ++b) {
-                        if (b < nblk) {
-                            const int rg = 16 * b + g, rh = rg + 8;
-                            uint32_t a[4];
-                            a[0] = (*reinterpret_cast<const uint32_t *>(sl + swz(rg, 2 * warp)) >> sh) & 0x03030303u;
-                            a[1] = (*reinterpret_cast<const uint32_t *>(sl + swz(rh, 2 * warp)) >> sh) & 0x03030303u;
-                            a[2] = (*reinterpret_cast<const uint32_t *>(sl + swz(rg, 2 * warp + 1)) >> sh) & 0x03030303u;
-                            a[3] = (*reinterpret_cast<const uint32_t *>(sl + swz(rh, 2 * warp + 1)) >> sh) & 0x03030303u;
+                for (int b = 0; b < kMaxBlocks; ++b) {
+                    if (b < nblk) {
+                        const int rg = 16 * b + g, rh = rg + 8;
+                        uint32_t a[4];
+                        a[0] = (*reinterpret_cast<const uint32_t *>(sl + swz(rg, 2 * ks)) >> sh) & 0x03030303u;
+                        a[1] = (*reinterpret_cast<const uint32_t *>(sl + swz(rh, 2 * ks)) >> sh) & 0x03030303u;
+                        a[2] = (*reinterpret_cast<const uint32_t *>(sl + swz(rg, 2 * ks + 1)) >> sh) & 0x03030303u;
+                        a[3] = (*reinterpret_cast<const uint32_t *>(sl + swz(rh, 2 * ks + 1)) >> sh) & 0x03030303u;
 #pragma unroll
-                            for (int tile = 0; tile < NT; ++tile) mma_u8s8_16832(C[b][tile], a, bf[tile][0], bf[tile][1]);
-                        }
+                        for (int tile = 0; tile < NT; ++tile) mma_u8s8_16832(C[b][tile], a, bf[tile][0], bf[tile][1]);
                     }
                 }
             }
+            release(s);
         }
         // reduce across warps (every warp reaches the barrier)
 #pragma unroll
@@ -380,11 +388,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     }
-    // every copy must have landed before the CTA exits
+    // every copy issued must have landed before the CTA exits
+    __syncthreads();
     if (threadIdx.x == 0) {
-        for (int s = 0; s < ns; ++s) {
+        for (int s = max(0, ns - S); s < ns; ++s) {
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(bar(s), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            while (!mbar_try_wait(full(s % S), static_cast<uint32_t>(s / S) & 1u) &&
+                   globaltimer_ns() - t0 < kWaitLimitNs) {
             }
         }
     }
