@@ -36,6 +36,8 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "bq_internal.h"
 #include "quant_common.cuh"
 
@@ -49,7 +51,6 @@ constexpr int kMaxSlices = 16;                // K <= 8192
 constexpr int kMaxRB = 96;                    // rows per CTA
 constexpr int kMaxBlocks = kMaxRB / 16;       // 16-row blocks of the mma path
 constexpr int kMaxRowsPerWarp = kMaxRB / kWarps;
-constexpr int kStages = 4;                    // slice stages in shared memory
 
 struct DecodeArgs {
     const void *x;
@@ -62,22 +63,24 @@ struct DecodeArgs {
     int8_t *ws_xq;
     float *ws_scale;
     int32_t *ws_rowsum;
-    int rb;  // rows per CTA (= TMA box rows)
+    int rb;      // rows per CTA (= TMA box rows)
+    int stages;  // shared-memory slice stages (all slices when they fit)
     uint32_t *status;
 };
 
 struct Layout {
-    uint32_t slice_bytes, nslices, stages, xs, off_x, off_sc, off_rs, off_red, off_bar, total;
-    __host__ __device__ Layout(int K, int MT, int rb) {
+    uint32_t slice_bytes, nslices, stages, xs, off_x, off_sc, off_rs, off_red, off_qred, off_bar, total;
+    __host__ __device__ Layout(int K, int MT, int rb, int max_stages) {
         nslices = static_cast<uint32_t>(K / (16 * kSliceWords));
-        stages = nslices < static_cast<uint32_t>(kStages) ? nslices : static_cast<uint32_t>(kStages);
+        stages = nslices < static_cast<uint32_t>(max_stages) ? nslices : static_cast<uint32_t>(max_stages);
         slice_bytes = (static_cast<uint32_t>(rb) * 128u + 1023u) & ~1023u;  // 1024-aligned for the swizzle
         xs = static_cast<uint32_t>(K) + 16u;                                 // padded token rows
         off_x = stages * slice_bytes;
         off_sc = a16(off_x + MT * xs);
         off_rs = a16(off_sc + 4 * MT);
         off_red = a16(off_rs + 4 * MT);
-        off_bar = a16(off_red + (MT > 2 ? kMaxRB * 16 * 4 : 0));
+        off_qred = a16(off_red + (MT > 2 ? kMaxRB * 16 * 4 : 0));
+        off_bar = a16(off_qred + 3 * kWarps * 2 * 4);  // cooperative prologue partials
         total = off_bar + 16 * stages;  // full[stages], empty[stages]
     }
     __host__ __device__ static uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
@@ -171,13 +174,118 @@ __device__ __forceinline__ void warp_quant_token(const InT *__restrict__ xr, int
     rowsum = warp_sum_i(isum);
 }
 
+// All warps quantize the (one or two) token rows together: warp w takes an
+// eighth of each row, partial sums and maxima meet in shared memory, and
+// every thread derives the same code factor from them.
+template <int MT, typename InT>
+__device__ __forceinline__ void cta_quant_small(const InT *__restrict__ x, int M, int K, float eps, int8_t *xs,
+                                                int xs_pitch, int8_t *ws_xq, float *s_scale, int *s_rowsum,
+                                                float *ws_scale, int32_t *ws_rowsum, float *q) {
+    constexpr int EPC = Elt<InT>::kPerChunk;
+    constexpr int CPL = 4;  // chunks per lane and row (K <= 4096 bf16 / 2048 fp32 fit in one pass)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nch = K / EPC;
+    const int per_warp = (nch + kWarps - 1) / kWarps;
+    const int c0 = warp * per_warp;
+    const int c1 = min(nch, c0 + per_warp);
+    float *q_ss = q, *q_mx = q + 2 * kWarps;
+    int *q_rs = reinterpret_cast<int *>(q + 4 * kWarps);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        if (m >= M) break;
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * K);
+        uint4 v[CPL];
+        const bool cached = c1 - c0 <= 32 * CPL;
+        float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+        auto stats = [&](const uint4 &u) {
+            float f[EPC];
+            Elt<InT>::unpack(u, f);
+#pragma unroll
+            for (int e = 0; e < EPC; e += 2) {
+                ss0 = fmaf(f[e], f[e], ss0);
+                ss1 = fmaf(f[e + 1], f[e + 1], ss1);
+                amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+            }
+        };
+        if (cached) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = c0 + lane + 32 * i;
+                if (c < c1) v[i] = __ldg(xv + c);
+            }
+#pragma unroll
+            for (int i = 0; i < CPL; ++i)
+                if (c0 + lane + 32 * i < c1) stats(v[i]);
+        } else {
+            for (int c = c0 + lane; c < c1; c += 32) stats(__ldg(xv + c));
+        }
+        const float a = warp_sum_f(ss0 + ss1), b = warp_max_f(amax);
+        if (lane == 0) {
+            q_ss[m * kWarps + warp] = a;
+            q_mx[m * kWarps + warp] = b;
+        }
+        __syncthreads();
+        float ss = 0.f, mx = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+            ss += q_ss[m * kWarps + w];
+            mx = fmaxf(mx, q_mx[m * kWarps + w]);
+        }
+        float fac, sc;
+        quant_row_factor(ss, mx, K, eps, fac, sc);
+        int isum = 0;
+        auto codes = [&](const uint4 &u, int c) {
+            float e[EPC];
+            Elt<InT>::unpack(u, e);
+            uint32_t w[EPC / 4];
+#pragma unroll
+            for (int j = 0; j < EPC / 4; ++j) {
+                w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
+                                   fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
+                isum = dp4a_ss(w[j], 0x01010101u, isum);
+            }
+            int8_t *d0 = xs + m * xs_pitch + c * EPC;
+            int8_t *d1 = ws_xq ? ws_xq + static_cast<int64_t>(m) * K + c * EPC : nullptr;
+            if constexpr (EPC == 8) {
+                *reinterpret_cast<uint2 *>(d0) = make_uint2(w[0], w[1]);
+                if (d1) *reinterpret_cast<uint2 *>(d1) = make_uint2(w[0], w[1]);
+            } else {
+                *reinterpret_cast<uint32_t *>(d0) = w[0];
+                if (d1) *reinterpret_cast<uint32_t *>(d1) = w[0];
+            }
+        };
+        if (cached) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = c0 + lane + 32 * i;
+                if (c < c1) codes(v[i], c);
+            }
+        } else {
+            for (int c = c0 + lane; c < c1; c += 32) codes(__ldg(xv + c), c);
+        }
+        const int r = warp_sum_i(isum);
+        if (lane == 0) q_rs[m * kWarps + warp] = r;
+        if (threadIdx.x == 0) {
+            s_scale[m] = sc;
+            if (ws_scale) ws_scale[m] = sc;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < M) {
+        const int m = threadIdx.x;
+        int r = 0;
+        for (int w = 0; w < kWarps; ++w) r += q_rs[m * kWarps + w];
+        s_rowsum[m] = r;
+        if (ws_rowsum) ws_rowsum[m] = r;
+    }
+}
+
 template <int MT, bool MMA, typename InT, typename OutT>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_w2a8_kernel(const __grid_constant__ CUtensorMap tmW, const DecodeArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = p.K, M = p.M;
-    const Layout L(K, MT, p.rb);
+    const Layout L(K, MT, p.rb, p.stages);
     const int ns = static_cast<int>(L.nslices), S = static_cast<int>(L.stages);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_begin = blockIdx.x * p.rb;
@@ -214,9 +322,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
     if (threadIdx.x == 0)
         for (int s = 0; s < S; ++s) load_slice(s);
+    const float gamma = __ldg(p.w_scale);
 
     // per-token activation quantization
-    for (int m = warp; m < M; m += kWarps) {
+    if constexpr (MT <= 2) {
+        cta_quant_small<MT, InT>(static_cast<const InT *>(p.x), M, K, p.eps, xs, L.xs,
+                                 blockIdx.x == 0 ? p.ws_xq : nullptr, s_scale, s_rowsum,
+                                 blockIdx.x == 0 ? p.ws_scale : nullptr, blockIdx.x == 0 ? p.ws_rowsum : nullptr,
+                                 reinterpret_cast<float *>(smem + L.off_qred));
+    } else for (int m = warp; m < M; m += kWarps) {
         float sc;
         int rsum;
         warp_quant_token<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps, xs + m * L.xs,
@@ -231,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
     __syncthreads();
-    const float gamma = __ldg(p.w_scale);
     OutT *out = static_cast<OutT *>(p.out);
 
     bool ok = true;
@@ -469,6 +582,20 @@ int rows_per_cta(int64_t N, const DevInfo &dev) {
 
 int mt_of(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 8 ? 8 : 16; }
 
+// Stages: every slice resident when two CTAs still fit on an SM, else the
+// largest ring that does (at least two stages).
+int stages_for(int64_t K, int MT, int rb, const DevInfo &dev) {
+    const int ns = static_cast<int>(K / (16 * kSliceWords));
+    const size_t per_sm = dev.max_smem_optin + 1024;  // an SM holds slightly more than one CTA may use
+    for (int st = ns; st >= 2; --st) {
+        const size_t need = Layout(static_cast<int>(K), MT, rb, st).total + 1024 + 1024;
+        if (2 * need <= per_sm) return st;
+    }
+    for (int st = ns; st >= 2; --st)
+        if (Layout(static_cast<int>(K), MT, rb, st).total + 1024 <= dev.max_smem_optin) return st;
+    return 0;
+}
+
 }  // namespace
 
 bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
@@ -476,8 +603,7 @@ bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const
         return false;
     const int rb = rows_per_cta(N, dev);
     if (rb > kMaxRB || rb < 1) return false;
-    const Layout lay(static_cast<int>(K), mt_of(M), rb);
-    return lay.total + 1024 <= dev.max_smem_optin;
+    return stages_for(K, mt_of(M), rb, dev) >= 2 || K / (16 * kSliceWords) == 1;
 }
 
 cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
@@ -511,8 +637,9 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.ws_scale = ws_scale;
     a.ws_rowsum = ws_rowsum;
     a.rb = rb;
+    a.stages = std::max(1, stages_for(K, MT, rb, dev));
     a.status = dev.status;
-    const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb).total) + 1024;
+    const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb, a.stages).total) + 1024;
     if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(map, a, out_dtype, MT, smem, dev, s, grid);
     return dispatch_out<float>(map, a, out_dtype, MT, smem, dev, s, grid);
 }
