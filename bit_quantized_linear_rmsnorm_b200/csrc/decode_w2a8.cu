@@ -6,21 +6,20 @@
 //   acc[m,n] = sum_k xq[m,k] * w_q[n,k],   out = (float(acc) * act_scale[m]) * gamma (+ bias)
 //
 // Bandwidth-bound on the 2-bit weights.  One CTA owns RB consecutive output
-// rows; its packed rows are read in K slices (128 bytes of every row: one 2-D
-// TMA box of 32 words x RB rows, 128-byte swizzle, so fragment loads are free
-// of bank conflicts) through a ring of shared-memory stages.
+// rows and copies them into shared memory with 16-byte cp.async (many copies
+// in flight per SM through the load/store path -- measured faster than 2-D
+// TMA boxes for this short HBM stream), laid out in 128-byte K slices of
+// every row with the 128-byte XOR swizzle (chunk c of row r at c ^ (r % 8))
+// so that the fragment loads below are free of bank conflicts.
 //
-// Overlap across calls.  A CTA is small enough (256 threads, <= 128
-// registers, a few slice stages) for two to share an SM, and each kernel
-// lets the next kernel of the stream launch at once (programmatic dependent
-// launch).  Before griddepcontrol.wait a CTA only prefetches its weight
-// slices into L2 -- nothing is consumed, so this is correct whatever the
-// previous kernel wrote -- and after the wait it reads them from L2.  So the
-// weight stream of call i+1 overlaps the tail of call i.
-//
-// After the wait, one warp per token quantizes the activations (row held in
-// registers, same fp32 arithmetic as the standalone kernel) into shared
-// memory; CTA 0 also writes them to the workspace.  Then:
+// Overlap across calls.  Each kernel lets the next kernel of the stream
+// launch at once (programmatic dependent launch); a CTA small enough to share
+// an SM (256 threads, <= 128 registers) starts while the previous call runs,
+// and before griddepcontrol.wait it only prefetches its weight lines into L2
+// -- nothing is consumed, so this is correct whatever the previous kernel
+// wrote.  After the wait it issues its weight copies, then quantizes the
+// activations while they are in flight (CTA 0 also writes xq, act_scale and
+// rowsum to the workspace), then:
 //   * M <= 2: warp w owns rows w, w+8, ...; per slice each lane takes one
 //     packed word (16 weights) of a row: dp4a of the u8 codes with the s8
 //     activations (one token: the 2-bit fields are masked in place, so
@@ -31,11 +30,8 @@
 //     takes k-steps 2w and 2w+1 of every slice for all 16-row blocks, and
 //     the partial accumulators are reduced across warps once, at the end.
 // The codes are offset binary (w_q + 1), so acc = dot(codes, xq) - rowsum.
-// Every mbarrier wait is bounded.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 
 #include "bq_internal.h"
@@ -47,6 +43,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kSliceWords = 32;               // 128 bytes of each packed row per slice
+constexpr int kChunksPerRow16 = 8;            // 16-byte chunks per row and slice
 constexpr int kMaxSlices = 16;                // K <= 8192
 constexpr int kMaxRB = 96;                    // rows per CTA
 constexpr int kMaxBlocks = kMaxRB / 16;       // 16-row blocks of the mma path
@@ -56,6 +53,7 @@ struct DecodeArgs {
     const void *x;
     int M, K;
     float eps;
+    const uint32_t *wpacked;
     const float *w_scale;
     const float *bias;
     int N;
@@ -63,25 +61,22 @@ struct DecodeArgs {
     int8_t *ws_xq;
     float *ws_scale;
     int32_t *ws_rowsum;
-    int rb;      // rows per CTA (= TMA box rows)
-    int stages;  // shared-memory slice stages (all slices when they fit)
+    int rb;  // rows per CTA
     uint32_t *status;
 };
 
 struct Layout {
-    uint32_t slice_bytes, nslices, stages, xs, off_x, off_sc, off_rs, off_red, off_qred, off_bar, total;
-    __host__ __device__ Layout(int K, int MT, int rb, int max_stages) {
+    uint32_t slice_bytes, nslices, xs, off_x, off_sc, off_rs, off_red, off_qred, total;
+    __host__ __device__ Layout(int K, int MT, int rb) {
         nslices = static_cast<uint32_t>(K / (16 * kSliceWords));
-        stages = nslices < static_cast<uint32_t>(max_stages) ? nslices : static_cast<uint32_t>(max_stages);
         slice_bytes = (static_cast<uint32_t>(rb) * 128u + 1023u) & ~1023u;  // 1024-aligned for the swizzle
         xs = static_cast<uint32_t>(K) + 16u;                                 // padded token rows
-        off_x = stages * slice_bytes;
+        off_x = nslices * slice_bytes;
         off_sc = a16(off_x + MT * xs);
         off_rs = a16(off_sc + 4 * MT);
         off_red = a16(off_rs + 4 * MT);
         off_qred = a16(off_red + (MT > 2 ? kMaxRB * 16 * 4 : 0));
-        off_bar = a16(off_qred + 3 * kWarps * 2 * 4);  // cooperative prologue partials
-        total = off_bar + 16 * stages;  // full[stages], empty[stages]
+        total = a16(off_qred + 3 * kWarps * 2 * 4);  // cooperative prologue partials
     }
     __host__ __device__ static uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
 };
@@ -281,86 +276,73 @@ __device__ __forceinline__ void cta_quant_small(const InT *__restrict__ x, int M
 
 template <int MT, bool MMA, typename InT, typename OutT>
 __global__ void __launch_bounds__(kThreads, 2)
-    decode_w2a8_kernel(const __grid_constant__ CUtensorMap tmW, const DecodeArgs p) {
+    decode_w2a8_kernel(const DecodeArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = p.K, M = p.M;
-    const Layout L(K, MT, p.rb, p.stages);
-    const int ns = static_cast<int>(L.nslices), S = static_cast<int>(L.stages);
+    const Layout L(K, MT, p.rb);
+    const int ns = static_cast<int>(L.nslices);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_begin = blockIdx.x * p.rb;
     const int rows = min(p.rb, p.N - n_begin);
     const uint32_t sbase = smem_u32(smem);
-    auto full = [&](int i) { return sbase + L.off_bar + 8u * i; };
-    auto empty = [&](int i) { return sbase + L.off_bar + 8u * (S + i); };
     int8_t *xs = reinterpret_cast<int8_t *>(smem + L.off_x);
     float *s_scale = reinterpret_cast<float *>(smem + L.off_sc);
     int *s_rowsum = reinterpret_cast<int *>(smem + L.off_rs);
     int *red = reinterpret_cast<int *>(smem + L.off_red);
+    const int words = K / 16;
+    const uint8_t *wbase = reinterpret_cast<const uint8_t *>(p.wpacked + static_cast<int64_t>(n_begin) * words);
+    const int row_bytes = K / 4;
 
-    if (threadIdx.x == 0) {
-        tma_prefetch_desc(&tmW);
-        // pull this CTA's weights toward L2 while the previous grid finishes
-        for (int s = 0; s < ns; ++s) tma_prefetch_l2_2d(&tmW, s * kSliceWords, n_begin);
-        for (int i = 0; i < S; ++i) {
-            mbar_init(full(i), 1);
-            mbar_init(empty(i), kWarps);
-        }
-        fence_mbarrier_init();
-    }
+    // pull this CTA's weight lines toward L2 while the previous grid finishes
+    for (int l = threadIdx.x; l < rows * (row_bytes / 128); l += kThreads)
+        prefetch_l2(wbase + static_cast<int64_t>(l) * 128);
     if constexpr (MMA)
         for (int i = threadIdx.x; i < kMaxRB * 16; i += kThreads) red[i] = 0;
     pdl_launch_dependents();
-    __syncthreads();
     pdl_wait();  // previous grid complete and visible: data may be consumed from here on
 
-    const uint32_t slice_tx = static_cast<uint32_t>(p.rb) * 128u;  // full box; rows past N read as zero
-    auto load_slice = [&](int s) {  // one thread
-        const int st = s % S;
-        mbar_arrive_expect_tx(full(st), slice_tx);
-        tma_load_2d(sbase + st * L.slice_bytes, &tmW, s * kSliceWords, n_begin, full(st));
-    };
-    if (threadIdx.x == 0)
-        for (int s = 0; s < S; ++s) load_slice(s);
+    // weight copies: 16-byte chunk q of row r -> slice q / 8, swizzled chunk (q % 8) ^ (r % 8)
+    {
+        const int cpr = row_bytes / 16;  // chunks per row
+        for (int j = threadIdx.x; j < p.rb * cpr; j += kThreads) {
+            const int r = j / cpr, q = j - r * cpr;
+            const int sl = q / kChunksPerRow16, c = q % kChunksPerRow16;
+            const uint32_t dst = sbase + sl * L.slice_bytes + r * 128 + ((c ^ (r & 7)) << 4);
+            const bool in = r < rows;
+            cp_async_16(dst, wbase + (in ? static_cast<int64_t>(r) * row_bytes + q * 16 : 0), in ? 16u : 0u);
+        }
+        cp_async_commit();
+    }
     const float gamma = __ldg(p.w_scale);
 
-    // per-token activation quantization
+    // per-token activation quantization (the weight copies are in flight)
     if constexpr (MT <= 2) {
         cta_quant_small<MT, InT>(static_cast<const InT *>(p.x), M, K, p.eps, xs, L.xs,
                                  blockIdx.x == 0 ? p.ws_xq : nullptr, s_scale, s_rowsum,
                                  blockIdx.x == 0 ? p.ws_scale : nullptr, blockIdx.x == 0 ? p.ws_rowsum : nullptr,
                                  reinterpret_cast<float *>(smem + L.off_qred));
-    } else for (int m = warp; m < M; m += kWarps) {
-        float sc;
-        int rsum;
-        warp_quant_token<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps, xs + m * L.xs,
-                              blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr, sc, rsum);
-        if (lane == 0) {
-            s_scale[m] = sc;
-            s_rowsum[m] = rsum;
-            if (blockIdx.x == 0) {
-                p.ws_scale[m] = sc;
-                p.ws_rowsum[m] = rsum;
+    } else {
+        for (int m = warp; m < M; m += kWarps) {
+            float sc;
+            int rsum;
+            warp_quant_token<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps,
+                                  xs + m * L.xs, blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr,
+                                  sc, rsum);
+            if (lane == 0) {
+                s_scale[m] = sc;
+                s_rowsum[m] = rsum;
+                if (blockIdx.x == 0) {
+                    p.ws_scale[m] = sc;
+                    p.ws_rowsum[m] = rsum;
+                }
             }
         }
     }
+    cp_async_wait_all();
     __syncthreads();
     OutT *out = static_cast<OutT *>(p.out);
 
-    bool ok = true;
-    auto wait_full = [&](int s) -> bool {  // warp-uniform
-        bool good = true;
-        if (lane == 0) good = mbar_wait_timed(full(s % S), static_cast<uint32_t>(s / S) & 1u, p.status, SITE_DECODE_FULL);
-        return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
-    };
-    auto release = [&](int s) {  // every warp, once per slice; thread 0 refills the stage
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty(s % S));
-        if (threadIdx.x == 0 && s + S < ns) {
-            if (mbar_wait_timed(empty(s % S), static_cast<uint32_t>(s / S) & 1u, p.status, SITE_DECODE_EMPTY))
-                load_slice(s + S);
-        }
-    };
 
     if constexpr (!MMA) {
         // rows r = warp + 8 i of this CTA; lane l takes word l of each slice
@@ -373,10 +355,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc4[i][j] = 0;
         }
-        for (int s = 0; s < ns && ok; ++s) {
-            ok = wait_full(s);
-            if (!ok) break;
-            const uint8_t *sl = smem + (s % S) * L.slice_bytes;
+        for (int s = 0; s < ns; ++s) {
+            const uint8_t *sl = smem + s * L.slice_bytes;
             uint4 x4[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m)
@@ -407,9 +387,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
             }
-            release(s);
         }
-        if (ok) {
+        {
 #pragma unroll
             for (int i = 0; i < kMaxRowsPerWarp; ++i) {
                 const int r = warp + kWarps * i;
@@ -441,10 +420,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int b = 0; b < kMaxBlocks; ++b)
 #pragma unroll
             for (int tile = 0; tile < NT; ++tile) C[b][tile][0] = C[b][tile][1] = C[b][tile][2] = C[b][tile][3] = 0;
-        for (int s = 0; s < ns && ok; ++s) {
-            ok = wait_full(s);
-            if (!ok) break;
-            const uint8_t *sl = smem + (s % S) * L.slice_bytes;
+        for (int s = 0; s < ns; ++s) {
+            const uint8_t *sl = smem + s * L.slice_bytes;
             const uint32_t sh = 2 * t;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // k-steps 2*warp + h of this slice
@@ -471,7 +448,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
             }
-            release(s);
         }
         // reduce across warps (every warp reaches the barrier)
 #pragma unroll
@@ -489,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
         __syncthreads();
-        if (ok) {
+        {
             for (int e = threadIdx.x; e < rows * 16; e += kThreads) {
                 const int r = e >> 4, m = e & 15;
                 if (m < M) {
@@ -501,33 +477,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
-    // every copy issued must have landed before the CTA exits
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int s = max(0, ns - S); s < ns; ++s) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(full(s % S), static_cast<uint32_t>(s / S) & 1u) &&
-                   globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
-        }
-    }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
 }
 
 template <int MT, bool MMA, typename InT, typename OutT>
-cudaError_t launch_t(const CUtensorMap &map, const DecodeArgs &a, int smem, const DevInfo &dev, cudaStream_t s,
-                     int grid) {
+cudaError_t launch_t(const DecodeArgs &a, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
     auto kern = decode_w2a8_kernel<MT, MMA, InT, OutT>;
     static int attr_smem[64] = {};
     if (smem > attr_smem[dev.device]) {
@@ -545,34 +498,33 @@ cudaError_t launch_t(const CUtensorMap &map, const DecodeArgs &a, int smem, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, map, a);
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <typename InT, typename OutT>
-cudaError_t dispatch_m(const CUtensorMap &map, const DecodeArgs &a, int MT, int smem, const DevInfo &dev,
-                       cudaStream_t s, int grid) {
+cudaError_t dispatch_m(const DecodeArgs &a, int MT, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
     switch (MT) {
         case 1:
-            return launch_t<1, false, InT, OutT>(map, a, smem, dev, s, grid);
+            return launch_t<1, false, InT, OutT>(a, smem, dev, s, grid);
         case 2:
-            return launch_t<2, false, InT, OutT>(map, a, smem, dev, s, grid);
+            return launch_t<2, false, InT, OutT>(a, smem, dev, s, grid);
         case 8:
-            return launch_t<8, true, InT, OutT>(map, a, smem, dev, s, grid);
+            return launch_t<8, true, InT, OutT>(a, smem, dev, s, grid);
         default:
-            return launch_t<16, true, InT, OutT>(map, a, smem, dev, s, grid);
+            return launch_t<16, true, InT, OutT>(a, smem, dev, s, grid);
     }
 }
 
 template <typename InT>
-cudaError_t dispatch_out(const CUtensorMap &map, const DecodeArgs &a, bq_dtype ot, int MT, int smem,
-                         const DevInfo &dev, cudaStream_t s, int grid) {
+cudaError_t dispatch_out(const DecodeArgs &a, bq_dtype ot, int MT, int smem, const DevInfo &dev, cudaStream_t s,
+                         int grid) {
     switch (ot) {
         case BQ_F32:
-            return dispatch_m<InT, float>(map, a, MT, smem, dev, s, grid);
+            return dispatch_m<InT, float>(a, MT, smem, dev, s, grid);
         case BQ_F16:
-            return dispatch_m<InT, __half>(map, a, MT, smem, dev, s, grid);
+            return dispatch_m<InT, __half>(a, MT, smem, dev, s, grid);
         default:
-            return dispatch_m<InT, __nv_bfloat16>(map, a, MT, smem, dev, s, grid);
+            return dispatch_m<InT, __nv_bfloat16>(a, MT, smem, dev, s, grid);
     }
 }
 
@@ -582,20 +534,6 @@ int rows_per_cta(int64_t N, const DevInfo &dev) {
 
 int mt_of(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 8 ? 8 : 16; }
 
-// Stages: every slice resident when two CTAs still fit on an SM, else the
-// largest ring that does (at least two stages).
-int stages_for(int64_t K, int MT, int rb, const DevInfo &dev) {
-    const int ns = static_cast<int>(K / (16 * kSliceWords));
-    const size_t per_sm = dev.max_smem_optin + 1024;  // an SM holds slightly more than one CTA may use
-    for (int st = ns; st >= 2; --st) {
-        const size_t need = Layout(static_cast<int>(K), MT, rb, st).total + 1024 + 1024;
-        if (2 * need <= per_sm) return st;
-    }
-    for (int st = ns; st >= 2; --st)
-        if (Layout(static_cast<int>(K), MT, rb, st).total + 1024 <= dev.max_smem_optin) return st;
-    return 0;
-}
-
 }  // namespace
 
 bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
@@ -603,7 +541,7 @@ bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const
         return false;
     const int rb = rows_per_cta(N, dev);
     if (rb > kMaxRB || rb < 1) return false;
-    return stages_for(K, mt_of(M), rb, dev) >= 2 || K / (16 * kSliceWords) == 1;
+    return Layout(static_cast<int>(K), mt_of(M), rb).total + 1024 <= dev.max_smem_optin;
 }
 
 cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
@@ -613,22 +551,12 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     const int MT = mt_of(M);
     const int rb = rows_per_cta(N, dev);
     const int grid = static_cast<int>((N + rb - 1) / rb);
-    auto fn = encode_fn();
-    if (fn == nullptr) return cudaErrorInvalidValue;
-    CUtensorMap map;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 4)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kSliceWords), static_cast<cuuint32_t>(rb)};
-    const cuuint32_t estr[2] = {1, 1};
-    if (fn(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(wpacked), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
     DecodeArgs a;
     a.x = x;
     a.M = static_cast<int>(M);
     a.K = static_cast<int>(K);
     a.eps = eps;
+    a.wpacked = wpacked;
     a.w_scale = w_scale;
     a.bias = bias;
     a.N = static_cast<int>(N);
@@ -637,11 +565,10 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.ws_scale = ws_scale;
     a.ws_rowsum = ws_rowsum;
     a.rb = rb;
-    a.stages = std::max(1, stages_for(K, MT, rb, dev));
     a.status = dev.status;
-    const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb, a.stages).total) + 1024;
-    if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(map, a, out_dtype, MT, smem, dev, s, grid);
-    return dispatch_out<float>(map, a, out_dtype, MT, smem, dev, s, grid);
+    const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb).total) + 1024;
+    if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(a, out_dtype, MT, smem, dev, s, grid);
+    return dispatch_out<float>(a, out_dtype, MT, smem, dev, s, grid);
 }
 
 }  // namespace bq
