@@ -479,6 +479,188 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
+// Register-streaming variant for one or two tokens: 512 threads, each loads
+// its 16-byte weight chunks j = t + 512 i of the CTA's rows (64 chunks per row
+// when K = 4096) straight into registers right after the dependency wait, so
+// every chunk of a thread covers the same 64-wide K range and needs the same
+// 64 activation bytes, held in registers.  dp4a per packed word; partial row
+// sums meet in shared memory.
+constexpr int kRegThreads = 512;
+constexpr int kRegChunks = 12;  // chunks per thread (rows per CTA * K/64 <= 512 * 12)
+
+template <int MT, typename InT, typename OutT>
+__global__ void __launch_bounds__(kRegThreads, 1) decode_w2a8_reg_kernel(const DecodeArgs p) {
+    __shared__ __align__(16) int8_t xs[2][8192 + 16];
+    __shared__ int rowacc[kMaxRB][2];
+    __shared__ float s_scale[2];
+    __shared__ int s_rowsum[2];
+    __shared__ float q[3 * 16 * 2];
+    const int K = p.K, M = p.M;
+    const int lane = threadIdx.x & 31;
+    const int n_begin = blockIdx.x * p.rb;
+    const int rows = min(p.rb, p.N - n_begin);
+    const int cpr = K / 64;  // 16-byte chunks per packed row
+    const uint4 *wv = reinterpret_cast<const uint4 *>(p.wpacked + static_cast<int64_t>(n_begin) * (K / 16));
+    const int total = rows * cpr;
+
+    // L2 prefetch of this CTA's weight lines before the dependency wait
+    for (int l = threadIdx.x; l < total / 8; l += kRegThreads) prefetch_l2(wv + 8 * l);
+    for (int i = threadIdx.x; i < kMaxRB * 2; i += kRegThreads) (&rowacc[0][0])[i] = 0;
+    pdl_launch_dependents();
+    pdl_wait();
+
+    uint4 w[kRegChunks];
+#pragma unroll
+    for (int i = 0; i < kRegChunks; ++i) {
+        const int j = threadIdx.x + kRegThreads * i;
+        w[i] = j < total ? __ldcs(wv + j) : make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
+    }
+    const float gamma = __ldg(p.w_scale);
+
+    // activations: the whole CTA quantizes the token rows (16 warps)
+    {
+        constexpr int EPC = Elt<InT>::kPerChunk;
+        const int warp = threadIdx.x >> 5;
+        const int nch = K / EPC;
+        for (int m = 0; m < M; ++m) {
+            const uint4 *xv = reinterpret_cast<const uint4 *>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K);
+            float ss = 0.f, mx = 0.f;
+            for (int c = threadIdx.x; c < nch; c += kRegThreads) {
+                float f[EPC];
+                Elt<InT>::unpack(__ldg(xv + c), f);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) {
+                    ss = fmaf(f[e], f[e], ss);
+                    mx = fmaxf(mx, fabsf(f[e]));
+                }
+            }
+            ss = warp_sum_f(ss);
+            mx = warp_max_f(mx);
+            if (lane == 0) {
+                q[m * 32 + warp] = ss;
+                q[m * 32 + 16 + warp] = mx;
+            }
+            __syncthreads();
+            float a = 0.f, b = 0.f;
+            for (int w2 = 0; w2 < 16; ++w2) {
+                a += q[m * 32 + w2];
+                b = fmaxf(b, q[m * 32 + 16 + w2]);
+            }
+            float fac, sc;
+            quant_row_factor(a, b, K, p.eps, fac, sc);
+            int isum = 0;
+            for (int c = threadIdx.x; c < nch; c += kRegThreads) {
+                float e[EPC];
+                Elt<InT>::unpack(__ldg(xv + c), e);
+                uint32_t wq[EPC / 4];
+#pragma unroll
+                for (int j = 0; j < EPC / 4; ++j) {
+                    wq[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
+                                        fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
+                    isum = dp4a_ss(wq[j], 0x01010101u, isum);
+                }
+                int8_t *ws = blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K + c * EPC : nullptr;
+                if constexpr (EPC == 8) {
+                    *reinterpret_cast<uint2 *>(&xs[m][c * 8]) = make_uint2(wq[0], wq[1]);
+                    if (ws) *reinterpret_cast<uint2 *>(ws) = make_uint2(wq[0], wq[1]);
+                } else {
+                    *reinterpret_cast<uint32_t *>(&xs[m][c * 4]) = wq[0];
+                    if (ws) *reinterpret_cast<uint32_t *>(ws) = wq[0];
+                }
+            }
+            isum = warp_sum_i(isum);
+            if (lane == 0) q[64 + m * 16 + warp] = __int_as_float(isum);
+            if (threadIdx.x == 0) {
+                s_scale[m] = sc;
+                if (blockIdx.x == 0) p.ws_scale[m] = sc;
+            }
+            __syncthreads();
+        }
+        if (threadIdx.x < M) {
+            int r = 0;
+            for (int w2 = 0; w2 < 16; ++w2) r += __float_as_int(q[64 + threadIdx.x * 16 + w2]);
+            s_rowsum[threadIdx.x] = r;
+            if (blockIdx.x == 0) p.ws_rowsum[threadIdx.x] = r;
+        }
+        __syncthreads();
+    }
+
+    // all chunks of this thread share the K range [64 q, 64 q + 64), q = t % cpr
+    const int qk = threadIdx.x % cpr;
+    uint4 xr[MT][4];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            xr[m][h] = m < M ? *reinterpret_cast<const uint4 *>(&xs[m][64 * qk + 16 * h]) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < kRegChunks; ++i) {
+        const int j = threadIdx.x + kRegThreads * i;
+        if (j < total) {
+            const int r = j / cpr;
+            const uint32_t wd[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m < M) {
+                    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {  // word h covers k = 64 qk + 16 h .. +16
+                        const uint4 xv4 = xr[m][h];
+                        a0 = dp4a_us(wd[h] & 0x03030303u, xv4.x, a0);
+                        a1 = dp4a_us(wd[h] & 0x0c0c0c0cu, xv4.y, a1);
+                        a2 = dp4a_us(wd[h] & 0x30303030u, xv4.z, a2);
+                        a3 = dp4a_us(wd[h] & 0xc0c0c0c0u, xv4.w, a3);
+                    }
+                    int v = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
+                    if (cpr >= 32) {  // the warp's 32 chunks belong to one row
+                        v = warp_sum_i(v);
+                        if (lane == 0) atomicAdd(&rowacc[r][m], v);
+                    } else {
+                        atomicAdd(&rowacc[r][m], v);
+                    }
+                }
+            }
+        }
+    }
+    __syncthreads();
+    OutT *out = static_cast<OutT *>(p.out);
+    for (int e = threadIdx.x; e < rows * M; e += kRegThreads) {
+        const int r = e / M, m = e % M;
+        const int n = n_begin + r;
+        float v = __fmul_rn(__fmul_rn(static_cast<float>(rowacc[r][m] - s_rowsum[m]), s_scale[m]), gamma);
+        if (p.bias) v = __fadd_rn(v, __ldg(p.bias + n));
+        out[static_cast<int64_t>(m) * p.N + n] = to_out<OutT>(v);
+    }
+}
+
+template <typename InT, typename OutT>
+cudaError_t launch_reg(const DecodeArgs &a, int MT, cudaStream_t s, int grid) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kRegThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (MT == 1) return cudaLaunchKernelEx(&cfg, decode_w2a8_reg_kernel<1, InT, OutT>, a);
+    return cudaLaunchKernelEx(&cfg, decode_w2a8_reg_kernel<2, InT, OutT>, a);
+}
+
+template <typename InT>
+cudaError_t launch_reg_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStream_t s, int grid) {
+    switch (ot) {
+        case BQ_F32:
+            return launch_reg<InT, float>(a, MT, s, grid);
+        case BQ_F16:
+            return launch_reg<InT, __half>(a, MT, s, grid);
+        default:
+            return launch_reg<InT, __nv_bfloat16>(a, MT, s, grid);
+    }
+}
+
 template <int MT, bool MMA, typename InT, typename OutT>
 cudaError_t launch_t(const DecodeArgs &a, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
     auto kern = decode_w2a8_kernel<MT, MMA, InT, OutT>;
@@ -566,6 +748,12 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.ws_rowsum = ws_rowsum;
     a.rb = rb;
     a.status = dev.status;
+    // (every chunk of a thread covers the same K range when K/64 divides 512)
+    if (M <= 2 && K <= 8192 && kRegThreads % (K / 64) == 0 &&
+        static_cast<int64_t>(rb) * (K / 64) <= kRegThreads * kRegChunks) {
+        if (xt == BQ_BF16) return launch_reg_out<__nv_bfloat16>(a, out_dtype, static_cast<int>(M), s, grid);
+        return launch_reg_out<float>(a, out_dtype, static_cast<int>(M), s, grid);
+    }
     const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb).total) + 1024;
     if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(a, out_dtype, MT, smem, dev, s, grid);
     return dispatch_out<float>(a, out_dtype, MT, smem, dev, s, grid);
