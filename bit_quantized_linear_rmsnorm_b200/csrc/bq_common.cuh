@@ -75,6 +75,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait that may suspend the thread (up to ~0.5 ms) until the phase
+// completes, instead of returning at once: fewer polling round trips.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(500000u)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up (records
 // BQ_ERR_TIMEOUT at `site` and returns false) after kWaitLimitNs, or as soon
 // as another role of the CTA has raised *abort.
@@ -82,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                                           uint32_t *status, uint32_t site) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (*abort) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             report(status, BQ_ERR_TIMEOUT, site);
@@ -98,7 +112,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ bool mbar_wait_timed(uint32_t bar, uint32_t parity, uint32_t *status, uint32_t site) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             report(status, BQ_ERR_TIMEOUT, site);
             return false;

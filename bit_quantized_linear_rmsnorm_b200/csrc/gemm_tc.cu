@@ -283,8 +283,12 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             // The 128 epilogue threads take the same decision, so none is left
             // alone at a named barrier: each waits (time-bounded only), then
             // they agree through a shared flag.
-            const bool ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE);
-            if (!ok) {
+            // one lane per warp waits (polling by 128 threads would take shared-
+            // memory bandwidth from the TMA and MMA), the warp follows it
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok && lane == 0) {
                 atomicOr(epi_fail, 1);
                 *abort_flag = 1;
             }
@@ -358,7 +362,9 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         bool ok = true;
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK)) {
+                bool got = true;
+                if (lane == 0) got = mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK);
+                if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
                     ok = false;
                     break;
                 }
