@@ -369,7 +369,7 @@ def _decode(res, steps, hbm):
         gbs = byts / (ms * 1e-3) / 1e9
         res[f"bitlinear_decode_M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
                                          "frac_hbm": round(gbs / hbm, 4), "algorithmic_bytes": byts,
-                                         "launches_per_step": 2, "config": f"x bf16 [{M},4096], W 2-bit [11008,4096]"}
+                                         "launches_per_step": 1, "config": f"x bf16 [{M},4096], W 2-bit [11008,4096]"}
     del wps
 
 

@@ -103,6 +103,20 @@ __device__ __forceinline__ uint32_t swz(int r, int w) {
            (static_cast<uint32_t>(w & 3) << 2);
 }
 
+// Rows of the CTA: the grid has one CTA per SM (or one per row when N is
+// smaller), and CTA b owns rows [b N / G, (b+1) N / G), so the ranges differ
+// by at most one row.  A grid of exactly one CTA per SM also keeps two CTAs of
+// the same call off one SM when consecutive calls overlap: each call's CTAs
+// can only take the slot that a CTA of the call before the previous one left.
+struct RowRange {
+    int begin, rows;
+};
+__device__ __forceinline__ RowRange row_range(int N) {
+    const int64_t b = blockIdx.x, G = gridDim.x;
+    const int n0 = static_cast<int>((b * N) / G), n1 = static_cast<int>(((b + 1) * N) / G);
+    return {n0, n1 - n0};
+}
+
 // One warp quantizes one token row (16-byte aligned, K % (16/sizeof(In)) == 0)
 // into shared memory (and the workspace when ws != nullptr).  Rows of up to
 // 512 chunks sit in registers, so their loads are all in flight at once.
@@ -283,8 +297,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const Layout L(K, MT, p.rb);
     const int ns = static_cast<int>(L.nslices);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_begin = blockIdx.x * p.rb;
-    const int rows = min(p.rb, p.N - n_begin);
+    const RowRange rr = row_range(p.N);
+    const int n_begin = rr.begin, rows = rr.rows;
     const uint32_t sbase = smem_u32(smem);
     int8_t *xs = reinterpret_cast<int8_t *>(smem + L.off_x);
     float *s_scale = reinterpret_cast<float *>(smem + L.off_sc);
@@ -479,79 +493,145 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-// Register-streaming variant for one or two tokens: 512 threads, each loads
-// its 16-byte weight chunks j = t + 512 i of the CTA's rows (64 chunks per row
-// when K = 4096) straight into registers right after the dependency wait, so
-// every chunk of a thread covers the same 64-wide K range and needs the same
-// 64 activation bytes, held in registers.  dp4a per packed word; partial row
-// sums meet in shared memory.
-constexpr int kRegThreads = 512;
-constexpr int kRegChunks = 12;  // chunks per thread (rows per CTA * K/64 <= 512 * 12)
+// Register-streaming variant for one token.  256 threads at most 128
+// registers each, so a CTA of the next call fits on the SM beside a running
+// one: it starts as soon as this call's CTAs have started (programmatic
+// dependent launch), prefetches its own weight lines into L2, and waits.
+// After the dependency wait each thread loads its activation chunks first
+// (they head the critical path: statistics -> code factor -> codes), then,
+// once its statistics are in shared memory, its weight chunks
+// j = t + 256 i (i < kStreamChunks) straight into registers.  With
+// 256 % (K/64) == 0 every chunk of a thread covers the same 64-wide K range
+// [64 q, 64 q + 64), q = t % (K/64), so it needs the same 64 activation bytes,
+// held in registers.  dp4a per packed word (the 2-bit fields are masked in
+// place: (word & (3 << 2j)) . x accumulates 4^j times the code dot product),
+// then the partial row sums of four chunks are reduced across the warp at
+// once (K/64 >= 32: the lanes of a warp share each chunk's row).
+constexpr int kStreamThreads = 256;
+constexpr int kStreamWarps = kStreamThreads / 32;
+constexpr int kStreamChunks = 20;      // weight chunks per thread (multiple of 4)
+constexpr int kStreamMaxRows = 160;    // rows per CTA
+constexpr int kStreamXPitch = 8192 + 16;
+
+template <int MT>
+struct StreamX {
+    static constexpr int kChunks = 4;  // activation chunks per thread and token
+};
+
+// Sum over the 32 lanes of four values at once: returns, in lanes 8c..8c+7,
+// the warp sum of value c (6 shuffles instead of 20).
+__device__ __forceinline__ int warp_sum4(int v0, int v1, int v2, int v3) {
+    const int lane = threadIdx.x & 31;
+    const bool h16 = lane & 16, h8 = lane & 8;
+    int k0 = h16 ? v2 : v0, k1 = h16 ? v3 : v1;
+    k0 += __shfl_xor_sync(0xffffffffu, h16 ? v0 : v2, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, h16 ? v1 : v3, 16);
+    int k = h8 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;
+}
+
+// Code dot product of one 16-byte chunk (64 weights) with its 64 activations.
+__device__ __forceinline__ int chunk_dot(const uint4 &w, const uint4 (&x)[4]) {
+    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {  // word h covers k = 64 q + 16 h .. + 16
+        a0 = dp4a_us(wd[h] & 0x03030303u, x[h].x, a0);
+        a1 = dp4a_us(wd[h] & 0x0c0c0c0cu, x[h].y, a1);
+        a2 = dp4a_us(wd[h] & 0x30303030u, x[h].z, a2);
+        a3 = dp4a_us(wd[h] & 0xc0c0c0c0u, x[h].w, a3);
+    }
+    return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
+}
 
 template <int MT, typename InT, typename OutT>
-__global__ void __launch_bounds__(kRegThreads, 1) decode_w2a8_reg_kernel(const DecodeArgs p) {
-    __shared__ __align__(16) int8_t xs[2][8192 + 16];
-    __shared__ int rowacc[kMaxRB][2];
-    __shared__ float s_scale[2];
-    __shared__ int s_rowsum[2];
-    __shared__ float q[3 * 16 * 2];
-    const int K = p.K, M = p.M;
-    const int lane = threadIdx.x & 31;
-    const int n_begin = blockIdx.x * p.rb;
-    const int rows = min(p.rb, p.N - n_begin);
+__global__ void __launch_bounds__(kStreamThreads, 2) decode_w2a8_stream_kernel(const DecodeArgs p) {
+    constexpr int EPC = Elt<InT>::kPerChunk;
+    constexpr int XC = StreamX<MT>::kChunks;
+    __shared__ __align__(16) int8_t xs[MT][kStreamXPitch];
+    __shared__ int rowacc[kStreamMaxRows][MT];
+    __shared__ float q_ss[MT][kStreamWarps], q_mx[MT][kStreamWarps];
+    __shared__ int q_rs[MT][kStreamWarps];
+    const int K = p.K;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const RowRange rr = row_range(p.N);
     const int cpr = K / 64;  // 16-byte chunks per packed row
-    const uint4 *wv = reinterpret_cast<const uint4 *>(p.wpacked + static_cast<int64_t>(n_begin) * (K / 16));
-    const int total = rows * cpr;
+    const uint4 *wv = reinterpret_cast<const uint4 *>(p.wpacked + static_cast<int64_t>(rr.begin) * (K / 16));
+    const int total = rr.rows * cpr;
 
     // L2 prefetch of this CTA's weight lines before the dependency wait
-    for (int l = threadIdx.x; l < total / 8; l += kRegThreads) prefetch_l2(wv + 8 * l);
-    for (int i = threadIdx.x; i < kMaxRB * 2; i += kRegThreads) (&rowacc[0][0])[i] = 0;
+    // (consumes nothing, so it is correct whatever the previous kernel wrote)
+    for (int l = threadIdx.x; l < total / 8; l += kStreamThreads) prefetch_l2(wv + 8 * l);
+    for (int i = threadIdx.x; i < kStreamMaxRows * MT; i += kStreamThreads) (&rowacc[0][0])[i] = 0;
     pdl_launch_dependents();
     pdl_wait();
 
-    uint4 w[kRegChunks];
+    // activations first
+    const int nch = K / EPC;
+    uint4 xc[MT][XC];
 #pragma unroll
-    for (int i = 0; i < kRegChunks; ++i) {
-        const int j = threadIdx.x + kRegThreads * i;
+    for (int m = 0; m < MT; ++m) {
+        const uint4 *xv = reinterpret_cast<const uint4 *>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K);
+#pragma unroll
+        for (int i = 0; i < XC; ++i) {
+            const int c = threadIdx.x + kStreamThreads * i;
+            xc[m][i] = c < nch ? __ldg(xv + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < XC; ++i) {
+            float f[EPC];
+            Elt<InT>::unpack(xc[m][i], f);
+#pragma unroll
+            for (int e = 0; e < EPC; e += 2) {
+                ss0 = fmaf(f[e], f[e], ss0);
+                ss1 = fmaf(f[e + 1], f[e + 1], ss1);
+                amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+            }
+        }
+        const float ss = warp_sum_f(ss0 + ss1), mx = warp_max_f(amax);
+        if (lane == 0) {
+            q_ss[m][warp] = ss;
+            q_mx[m][warp] = mx;
+        }
+    }
+
+    // then the weights (issued behind the activation loads)
+    uint4 w[kStreamChunks];
+#pragma unroll
+    for (int i = 0; i < kStreamChunks; ++i) {
+        const int j = threadIdx.x + kStreamThreads * i;
         w[i] = j < total ? __ldcs(wv + j) : make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);
     }
     const float gamma = __ldg(p.w_scale);
+    __syncthreads();
 
-    // activations: the whole CTA quantizes the token rows (16 warps)
-    {
-        constexpr int EPC = Elt<InT>::kPerChunk;
-        const int warp = threadIdx.x >> 5;
-        const int nch = K / EPC;
-        for (int m = 0; m < M; ++m) {
-            const uint4 *xv = reinterpret_cast<const uint4 *>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K);
-            float ss = 0.f, mx = 0.f;
-            for (int c = threadIdx.x; c < nch; c += kRegThreads) {
-                float f[EPC];
-                Elt<InT>::unpack(__ldg(xv + c), f);
+    // code factor of each token (every thread derives the same one), codes
+    float sc[MT];
 #pragma unroll
-                for (int e = 0; e < EPC; ++e) {
-                    ss = fmaf(f[e], f[e], ss);
-                    mx = fmaxf(mx, fabsf(f[e]));
-                }
-            }
-            ss = warp_sum_f(ss);
-            mx = warp_max_f(mx);
-            if (lane == 0) {
-                q[m * 32 + warp] = ss;
-                q[m * 32 + 16 + warp] = mx;
-            }
-            __syncthreads();
-            float a = 0.f, b = 0.f;
-            for (int w2 = 0; w2 < 16; ++w2) {
-                a += q[m * 32 + w2];
-                b = fmaxf(b, q[m * 32 + 16 + w2]);
-            }
-            float fac, sc;
-            quant_row_factor(a, b, K, p.eps, fac, sc);
-            int isum = 0;
-            for (int c = threadIdx.x; c < nch; c += kRegThreads) {
+    for (int m = 0; m < MT; ++m) {
+        float ss = 0.f, mx = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < kStreamWarps; ++w2) {
+            ss += q_ss[m][w2];
+            mx = fmaxf(mx, q_mx[m][w2]);
+        }
+        float fac;
+        quant_row_factor(ss, mx, K, p.eps, fac, sc[m]);
+        int isum = 0;
+#pragma unroll
+        for (int i = 0; i < XC; ++i) {
+            const int c = threadIdx.x + kStreamThreads * i;
+            if (c < nch) {
                 float e[EPC];
-                Elt<InT>::unpack(__ldg(xv + c), e);
+                Elt<InT>::unpack(xc[m][i], e);
                 uint32_t wq[EPC / 4];
 #pragma unroll
                 for (int j = 0; j < EPC / 4; ++j) {
@@ -568,76 +648,58 @@ __global__ void __launch_bounds__(kRegThreads, 1) decode_w2a8_reg_kernel(const D
                     if (ws) *reinterpret_cast<uint32_t *>(ws) = wq[0];
                 }
             }
-            isum = warp_sum_i(isum);
-            if (lane == 0) q[64 + m * 16 + warp] = __int_as_float(isum);
-            if (threadIdx.x == 0) {
-                s_scale[m] = sc;
-                if (blockIdx.x == 0) p.ws_scale[m] = sc;
-            }
-            __syncthreads();
         }
-        if (threadIdx.x < M) {
-            int r = 0;
-            for (int w2 = 0; w2 < 16; ++w2) r += __float_as_int(q[64 + threadIdx.x * 16 + w2]);
-            s_rowsum[threadIdx.x] = r;
-            if (blockIdx.x == 0) p.ws_rowsum[threadIdx.x] = r;
-        }
-        __syncthreads();
+        isum = warp_sum_i(isum);
+        if (lane == 0) q_rs[m][warp] = isum;
+        if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_scale[m] = sc[m];
     }
+    __syncthreads();
 
-    // all chunks of this thread share the K range [64 q, 64 q + 64), q = t % cpr
-    const int qk = threadIdx.x % cpr;
-    uint4 xr[MT][4];
+    // dot products: chunk i of this thread is row r0 + rstep * i
+    const int qk = threadIdx.x % cpr, r0 = threadIdx.x / cpr, rstep = kStreamThreads / cpr;
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
+    for (int m = 0; m < MT; ++m) {
+        uint4 xr[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h)
-            xr[m][h] = m < M ? *reinterpret_cast<const uint4 *>(&xs[m][64 * qk + 16 * h]) : make_uint4(0, 0, 0, 0);
+        for (int h = 0; h < 4; ++h) xr[h] = *reinterpret_cast<const uint4 *>(&xs[m][64 * qk + 16 * h]);
 #pragma unroll
-    for (int i = 0; i < kRegChunks; ++i) {
-        const int j = threadIdx.x + kRegThreads * i;
-        if (j < total) {
-            const int r = j / cpr;
-            const uint32_t wd[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m < M) {
-                    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {  // word h covers k = 64 qk + 16 h .. +16
-                        const uint4 xv4 = xr[m][h];
-                        a0 = dp4a_us(wd[h] & 0x03030303u, xv4.x, a0);
-                        a1 = dp4a_us(wd[h] & 0x0c0c0c0cu, xv4.y, a1);
-                        a2 = dp4a_us(wd[h] & 0x30303030u, xv4.z, a2);
-                        a3 = dp4a_us(wd[h] & 0xc0c0c0c0u, xv4.w, a3);
-                    }
-                    int v = a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
-                    if (cpr >= 32) {  // the warp's 32 chunks belong to one row
-                        v = warp_sum_i(v);
-                        if (lane == 0) atomicAdd(&rowacc[r][m], v);
-                    } else {
-                        atomicAdd(&rowacc[r][m], v);
-                    }
-                }
-            }
+        for (int g = 0; g < kStreamChunks / 4; ++g) {
+            const int k = warp_sum4(chunk_dot(w[4 * g], xr), chunk_dot(w[4 * g + 1], xr),
+                                    chunk_dot(w[4 * g + 2], xr), chunk_dot(w[4 * g + 3], xr));
+            const int r = r0 + rstep * (4 * g + (lane >> 3));
+            if ((lane & 7) == 0 && r < rr.rows) atomicAdd(&rowacc[r][m], k);
         }
     }
     __syncthreads();
+
+    // epilogue: out = ((acc - rowsum) * act_scale) * gamma (+ bias)
+    int rsum[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+        int r = 0;
+#pragma unroll
+        for (int w2 = 0; w2 < kStreamWarps; ++w2) r += q_rs[m][w2];
+        rsum[m] = r;
+        if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_rowsum[m] = r;
+    }
     OutT *out = static_cast<OutT *>(p.out);
-    for (int e = threadIdx.x; e < rows * M; e += kRegThreads) {
-        const int r = e / M, m = e % M;
-        const int n = n_begin + r;
-        float v = __fmul_rn(__fmul_rn(static_cast<float>(rowacc[r][m] - s_rowsum[m]), s_scale[m]), gamma);
-        if (p.bias) v = __fadd_rn(v, __ldg(p.bias + n));
-        out[static_cast<int64_t>(m) * p.N + n] = to_out<OutT>(v);
+    for (int r = threadIdx.x; r < rr.rows; r += kStreamThreads) {
+        const int n = rr.begin + r;
+        const float bias = p.bias ? __ldg(p.bias + n) : 0.f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float v = __fmul_rn(__fmul_rn(static_cast<float>(rowacc[r][m] - rsum[m]), sc[m]), gamma);
+            if (p.bias) v = __fadd_rn(v, bias);
+            out[static_cast<int64_t>(m) * p.N + n] = to_out<OutT>(v);
+        }
     }
 }
 
 template <typename InT, typename OutT>
-cudaError_t launch_reg(const DecodeArgs &a, int MT, cudaStream_t s, int grid) {
+cudaError_t launch_stream(const DecodeArgs &a, int MT, cudaStream_t s, int grid) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(kRegThreads);
+    cfg.blockDim = dim3(kStreamThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -645,19 +707,19 @@ cudaError_t launch_reg(const DecodeArgs &a, int MT, cudaStream_t s, int grid) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (MT == 1) return cudaLaunchKernelEx(&cfg, decode_w2a8_reg_kernel<1, InT, OutT>, a);
-    return cudaLaunchKernelEx(&cfg, decode_w2a8_reg_kernel<2, InT, OutT>, a);
+    (void)MT;  // one token (two would not fit the register budget)
+    return cudaLaunchKernelEx(&cfg, decode_w2a8_stream_kernel<1, InT, OutT>, a);
 }
 
 template <typename InT>
-cudaError_t launch_reg_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStream_t s, int grid) {
+cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStream_t s, int grid) {
     switch (ot) {
         case BQ_F32:
-            return launch_reg<InT, float>(a, MT, s, grid);
+            return launch_stream<InT, float>(a, MT, s, grid);
         case BQ_F16:
-            return launch_reg<InT, __half>(a, MT, s, grid);
+            return launch_stream<InT, __half>(a, MT, s, grid);
         default:
-            return launch_reg<InT, __nv_bfloat16>(a, MT, s, grid);
+            return launch_stream<InT, __nv_bfloat16>(a, MT, s, grid);
     }
 }
 
@@ -710,8 +772,24 @@ cudaError_t dispatch_out(const DecodeArgs &a, bq_dtype ot, int MT, int smem, con
     }
 }
 
+// One CTA per SM (fewer when N is smaller); the largest row range of a CTA.
+int grid_of(int64_t N, const DevInfo &dev) { return static_cast<int>(std::min<int64_t>(N, dev.num_sms)); }
 int rows_per_cta(int64_t N, const DevInfo &dev) {
-    return static_cast<int>((N + dev.num_sms - 1) / dev.num_sms);
+    const int64_t G = grid_of(N, dev);
+    return static_cast<int>((N + G - 1) / G);
+}
+
+// Shapes of the register-streaming kernel: one token, 256 % (K/64) == 0
+// with K/64 >= 32, the activation chunks of a thread cached in registers, and
+// every weight chunk of the CTA in flight at once.
+bool stream_supported(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev) {
+    if (M != 1 || K % 64 != 0 || K > kStreamXPitch - 16) return false;
+    const int64_t cpr = K / 64;
+    if (cpr < 32 || kStreamThreads % cpr != 0) return false;
+    const int64_t epc = xt == BQ_BF16 ? 8 : 4;
+    if (K / epc > static_cast<int64_t>(kStreamThreads) * StreamX<1>::kChunks) return false;
+    const int64_t rb = rows_per_cta(N, dev);
+    return rb <= kStreamMaxRows && rb * cpr <= static_cast<int64_t>(kStreamThreads) * kStreamChunks;
 }
 
 int mt_of(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 8 ? 8 : 16; }
@@ -732,7 +810,7 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
                                const DevInfo &dev) {
     const int MT = mt_of(M);
     const int rb = rows_per_cta(N, dev);
-    const int grid = static_cast<int>((N + rb - 1) / rb);
+    const int grid = grid_of(N, dev);
     DecodeArgs a;
     a.x = x;
     a.M = static_cast<int>(M);
@@ -748,11 +826,9 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.ws_rowsum = ws_rowsum;
     a.rb = rb;
     a.status = dev.status;
-    // (every chunk of a thread covers the same K range when K/64 divides 512)
-    if (M <= 2 && K <= 8192 && kRegThreads % (K / 64) == 0 &&
-        static_cast<int64_t>(rb) * (K / 64) <= kRegThreads * kRegChunks) {
-        if (xt == BQ_BF16) return launch_reg_out<__nv_bfloat16>(a, out_dtype, static_cast<int>(M), s, grid);
-        return launch_reg_out<float>(a, out_dtype, static_cast<int>(M), s, grid);
+    if (stream_supported(M, N, K, xt, dev)) {
+        if (xt == BQ_BF16) return launch_stream_out<__nv_bfloat16>(a, out_dtype, static_cast<int>(M), s, grid);
+        return launch_stream_out<float>(a, out_dtype, static_cast<int>(M), s, grid);
     }
     const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb).total) + 1024;
     if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(a, out_dtype, MT, smem, dev, s, grid);

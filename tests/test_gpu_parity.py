@@ -291,6 +291,25 @@ def test_bitlinear_decode_ragged(M, N, K, out, bias):
     _bitlinear_check(x, dev(x), w, N, out, b, f"decode ragged {M}x{N}x{K}")
 
 
+# one token: register-streaming kernel (fp32 and bf16 inputs, K = 2048 / 8192,
+# fewer rows than SMs); two tokens: shared-memory kernel with balanced rows
+@pytest.mark.parametrize("M,N,K,out,bias,xin", [(1, 300, 2048, "f32", True, "f32"), (1, 100, 4096, "f16", True, "bf16"),
+                                                (1, 5000, 8192, "bf16", False, "bf16"),
+                                                (2, 1000, 4096, "bf16", True, "bf16"),
+                                                (1, 11008, 4096, "f32", False, "f32")])
+def test_bitlinear_decode_stream_shapes(M, N, K, out, bias, xin):
+    g = synth.rng((110, M, N, K))
+    if xin == "bf16":
+        bits, x = synth.bf16_activations(M, K, (110, M, K))
+        x_dev = bf16_dev(bits)
+    else:
+        x = synth.normal_f32(g, (M, K))
+        x_dev = dev(x)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    b = synth.normal_f32(g, (N,), 0.1) if bias else None
+    _bitlinear_check(x, x_dev, w, N, out, b, f"decode stream {M}x{N}x{K} {xin}")
+
+
 @pytest.mark.parametrize("M,N,K,out,bias", [(17, 256, 128, "bf16", False), (300, 520, 512, "bf16", True),
                                             (129, 264, 640, "f32", False), (200, 1000, 1024, "f16", True)])
 def test_bitlinear_prefill_ragged(M, N, K, out, bias):
