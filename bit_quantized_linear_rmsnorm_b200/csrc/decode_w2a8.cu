@@ -63,6 +63,7 @@ struct DecodeArgs {
     int32_t *ws_rowsum;
     int rb;  // rows per CTA
     uint32_t *status;
+    bq_dtype out_dtype;
 };
 
 struct Layout {
@@ -723,6 +724,264 @@ cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStre
     }
 }
 
+// Register-streaming variant for 2..16 tokens on the mma.sync tensor path
+// (one m16n8k32 covers 16 rows x 32 K for eight tokens at once, where dp4a
+// would repeat the whole dot product per token).  Same launch shape as the
+// one-token kernel: 256 threads at most 128 registers, two CTAs per SM, one
+// CTA per SM per call, L2 prefetch before the dependency wait.
+//
+// Work unit = (16-row block rb, 256-wide K block kb); warp w takes the K
+// blocks kb = w + 8 c (c < KBW, K = 2048 KBW) of every row block.  Lane
+// (g = lane / 4, t = lane % 4) holds words 16 kb + 4 t .. + 3 of rows g and
+// g + 8 of the block (two 16-byte loads).  MMA (s, j) takes field j of words
+// 2 s and 2 s + 1 masked in place, (word & (3 << 2j)) = code * 4^j in each
+// byte, as the A fragment; its k-slots 4 t + b and 16 + 4 t + b hold the
+// codes of k = 16 (16 kb + 4 t + 2 s) + 4 j + b and of the next word, so the
+// matching B fragment of token g is bytes 4 j .. 4 j + 3 of the two 16-byte
+// activation chunks 16 kb + 4 t + 2 s and + 1.  The four fields accumulate in
+// four accumulators, combined as acc0 + acc1 / 4 + acc2 / 16 + acc3 / 64
+// (each acc_j is a multiple of 4^j, so the shifts are exact).
+constexpr int kMmaThreads = 256;
+constexpr int kMmaWarps = kMmaThreads / 32;
+constexpr int kMmaUnits = 10;  // units per warp held in registers
+
+// 16-byte chunk c of a token row sits at chunk c ^ (2 ((c >> 3) & 1)): the
+// B-fragment loads of lanes t = 0..3 (chunks 4 t + const) and of consecutive
+// tokens (row pitch K + 16 bytes) then fall in distinct bank groups.
+__device__ __forceinline__ int xchunk_swz(int c) { return c ^ (((c >> 3) & 1) << 1); }
+
+// One warp quantizes one token row into the swizzled shared-memory row `dst`
+// (and the workspace row `ws` when not null).  Rows of up to 512 chunks stay
+// in registers between the statistics and the codes; longer rows are read
+// twice.
+template <typename InT>
+__device__ __forceinline__ void warp_quant_token_swz(const InT *__restrict__ xr, int K, float eps, int8_t *dst,
+                                                     int8_t *ws, float &scale, int &rowsum) {
+    constexpr int EPC = Elt<InT>::kPerChunk;
+    constexpr int CPL = 16;
+    const int lane = threadIdx.x & 31;
+    const int nch = K / EPC;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(xr);
+    const bool cached = nch <= 32 * CPL;
+    float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+    uint4 c[CPL];
+    auto stats = [&](const uint4 &u) {
+        float f[EPC];
+        Elt<InT>::unpack(u, f);
+#pragma unroll
+        for (int e = 0; e < EPC; e += 2) {
+            ss0 = fmaf(f[e], f[e], ss0);
+            ss1 = fmaf(f[e + 1], f[e + 1], ss1);
+            amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+        }
+    };
+    if (cached) {
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int ch = lane + 32 * i;
+            c[i] = ch < nch ? __ldg(xv + ch) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) stats(c[i]);
+    } else {
+        for (int ch = lane; ch < nch; ch += 32) stats(__ldg(xv + ch));
+    }
+    const float ss = warp_sum_f(ss0 + ss1);
+    amax = warp_max_f(amax);
+    float fac;
+    quant_row_factor(ss, amax, K, eps, fac, scale);
+    int isum = 0;
+    auto codes = [&](const uint4 &u, int ch) {
+        float e[EPC];
+        Elt<InT>::unpack(u, e);
+        uint32_t w[EPC / 4];
+#pragma unroll
+        for (int j = 0; j < EPC / 4; ++j) {
+            w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
+                               fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
+            isum = dp4a_ss(w[j], 0x01010101u, isum);
+        }
+        const int o = ch * EPC;  // code byte offset
+        int8_t *d = dst + xchunk_swz(o >> 4) * 16 + (o & 15);
+        if constexpr (EPC == 8) {
+            *reinterpret_cast<uint2 *>(d) = make_uint2(w[0], w[1]);
+            if (ws) *reinterpret_cast<uint2 *>(ws + o) = make_uint2(w[0], w[1]);
+        } else {
+            *reinterpret_cast<uint32_t *>(d) = w[0];
+            if (ws) *reinterpret_cast<uint32_t *>(ws + o) = w[0];
+        }
+    };
+    if (cached) {
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            const int ch = lane + 32 * i;
+            if (ch < nch) codes(c[i], ch);
+        }
+    } else {
+        for (int ch = lane; ch < nch; ch += 32) codes(__ldg(xv + ch), ch);
+    }
+    rowsum = warp_sum_i(isum);
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_out(void *out, int64_t i, float v) {
+    static_cast<OutT *>(out)[i] = to_out<OutT>(v);
+}
+
+template <int MT, int KBW>
+struct MmaLayout {
+    static constexpr int kMaxRows = 16 * (kMmaUnits / KBW);
+    static __host__ __device__ int pitch(int K) { return K + 16; }
+    static __host__ __device__ int off_acc(int K) { return MT * pitch(K); }
+    static __host__ __device__ int off_scale(int K) { return off_acc(K) + kMaxRows * MT * 4; }
+    static __host__ __device__ int off_rowsum(int K) { return off_scale(K) + MT * 4; }
+    static __host__ __device__ int bytes(int K) { return off_rowsum(K) + MT * 4; }
+};
+
+template <int MT, int KBW, typename InT>
+__global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const DecodeArgs p) {
+    using L = MmaLayout<MT, KBW>;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int K = p.K, M = p.M;
+    const int xp = L::pitch(K);
+    int8_t *xs = reinterpret_cast<int8_t *>(smem);
+    int *rowacc = reinterpret_cast<int *>(smem + L::off_acc(K));
+    float *s_scale = reinterpret_cast<float *>(smem + L::off_scale(K));
+    int *s_rowsum = reinterpret_cast<int *>(smem + L::off_rowsum(K));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const RowRange rr = row_range(p.N);
+    const int wpr = K / 16;  // packed words per row
+    const uint32_t *wrow = p.wpacked + static_cast<int64_t>(rr.begin) * wpr;
+
+    for (int l = threadIdx.x; l < rr.rows * wpr / 32; l += kMmaThreads) prefetch_l2(wrow + 32 * l);
+    for (int i = threadIdx.x; i < L::kMaxRows * MT; i += kMmaThreads) rowacc[i] = 0;
+    pdl_launch_dependents();
+    pdl_wait();
+
+    // activations: warp w quantizes tokens w, w + 8 (codes stay out of registers)
+    for (int m = warp; m < M; m += kMmaWarps) {
+        float sc;
+        int rsum;
+        warp_quant_token_swz<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps,
+                                  xs + m * xp, blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr,
+                                  sc, rsum);
+        if (lane == 0) {
+            s_scale[m] = sc;
+            s_rowsum[m] = rsum;
+            if (blockIdx.x == 0) {
+                p.ws_scale[m] = sc;
+                p.ws_rowsum[m] = rsum;
+            }
+        }
+    }
+
+    // this warp's weight words (unit i: row block i / KBW, K block warp + 8 (i % KBW))
+    const int nrb = (rr.rows + 15) / 16;
+    uint4 wa[kMmaUnits], wb[kMmaUnits];
+#pragma unroll
+    for (int i = 0; i < kMmaUnits; ++i) {
+        const int rb = i / KBW, kb = warp + kMmaWarps * (i % KBW);
+        const int r0 = rb * 16 + g, r1 = r0 + 8;
+        const uint32_t *base = wrow + 16 * kb + 4 * t;
+        wa[i] = r0 < rr.rows ? __ldcs(reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(r0) * wpr))
+                             : make_uint4(0u, 0u, 0u, 0u);
+        wb[i] = r1 < rr.rows ? __ldcs(reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(r1) * wpr))
+                             : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const float gamma = __ldg(p.w_scale);
+    __syncthreads();
+
+    // token group h (tokens 8 h .. 8 h + 7) in the outer loop: one accumulator set live
+#pragma unroll
+    for (int h = 0; h < MT / 8; ++h) {
+        const int tok = g + 8 * h;
+        int racc[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < kMmaUnits; ++i) {
+            const int rb = i / KBW, kb = warp + kMmaWarps * (i % KBW);
+            if (rb < nrb) {
+                int acc[4][4] = {};
+#pragma unroll
+                for (int s = 0; s < 2; ++s) {
+                    uint4 bx0 = make_uint4(0u, 0u, 0u, 0u), bx1 = make_uint4(0u, 0u, 0u, 0u);
+                    if (tok < M) {
+                        const int c0 = 16 * kb + 4 * t + 2 * s;
+                        bx0 = *reinterpret_cast<const uint4 *>(xs + tok * xp + xchunk_swz(c0) * 16);
+                        bx1 = *reinterpret_cast<const uint4 *>(xs + tok * xp + xchunk_swz(c0 + 1) * 16);
+                    }
+                    const uint32_t w0 = s ? wa[i].z : wa[i].x, w1 = s ? wa[i].w : wa[i].y;
+                    const uint32_t v0 = s ? wb[i].z : wb[i].x, v1 = s ? wb[i].w : wb[i].y;
+                    const uint32_t b0[4] = {bx0.x, bx0.y, bx0.z, bx0.w}, b1[4] = {bx1.x, bx1.y, bx1.z, bx1.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t mk = 0x03030303u << (2 * j);
+                        const uint32_t a[4] = {w0 & mk, v0 & mk, w1 & mk, v1 & mk};
+                        mma_u8s8_16832(acc[j], a, b0[j], b1[j]);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) racc[c] += acc[0][c] + (acc[1][c] >> 2) + (acc[2][c] >> 4) + (acc[3][c] >> 6);
+                if (i % KBW == KBW - 1) {  // last K block of this row block: flush
+                    const int r0 = rb * 16 + g, r1 = r0 + 8;
+                    const int m0 = 2 * t + 8 * h, m1 = m0 + 1;
+                    if (r0 < rr.rows && m0 < M) atomicAdd(&rowacc[r0 * MT + m0], racc[0]);
+                    if (r0 < rr.rows && m1 < M) atomicAdd(&rowacc[r0 * MT + m1], racc[1]);
+                    if (r1 < rr.rows && m0 < M) atomicAdd(&rowacc[r1 * MT + m0], racc[2]);
+                    if (r1 < rr.rows && m1 < M) atomicAdd(&rowacc[r1 * MT + m1], racc[3]);
+                    racc[0] = racc[1] = racc[2] = racc[3] = 0;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // epilogue: out = ((acc - rowsum) * act_scale) * gamma (+ bias)
+    for (int e = threadIdx.x; e < rr.rows * M; e += kMmaThreads) {
+        const int r = e / M, m = e - r * M;
+        const int n = rr.begin + r;
+        float v = __fmul_rn(__fmul_rn(static_cast<float>(rowacc[r * MT + m] - s_rowsum[m]), s_scale[m]), gamma);
+        if (p.bias) v = __fadd_rn(v, __ldg(p.bias + n));
+        const int64_t o = static_cast<int64_t>(m) * p.N + n;
+        if (p.out_dtype == BQ_F32)
+            store_out<float>(p.out, o, v);
+        else if (p.out_dtype == BQ_F16)
+            store_out<__half>(p.out, o, v);
+        else
+            store_out<__nv_bfloat16>(p.out, o, v);
+    }
+}
+
+template <int MT, int KBW, typename InT>
+cudaError_t launch_mma_t(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
+    auto kern = decode_w2a8_mma_kernel<MT, KBW, InT>;
+    const int smem = MmaLayout<MT, KBW>::bytes(a.K);
+    static int attr_smem[64] = {};
+    if (smem > attr_smem[dev.device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_smem[dev.device] = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kMmaThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <typename InT>
+cudaError_t launch_mma(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
+    const bool two = a.M > 8;
+    if (a.K == 2048) return two ? launch_mma_t<16, 1, InT>(a, dev, s, grid) : launch_mma_t<8, 1, InT>(a, dev, s, grid);
+    return two ? launch_mma_t<16, 2, InT>(a, dev, s, grid) : launch_mma_t<8, 2, InT>(a, dev, s, grid);
+}
+
 template <int MT, bool MMA, typename InT, typename OutT>
 cudaError_t launch_t(const DecodeArgs &a, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
     auto kern = decode_w2a8_kernel<MT, MMA, InT, OutT>;
@@ -792,6 +1051,16 @@ bool stream_supported(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInf
     return rb <= kStreamMaxRows && rb * cpr <= static_cast<int64_t>(kStreamThreads) * kStreamChunks;
 }
 
+// Shapes of the mma.sync register-streaming kernel: 2..16 tokens, K = 2048 or
+// 4096, every unit of the CTA in registers, two CTAs per SM.
+bool mma_stream_supported(int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
+    if (M < 2 || M > 16 || (K != 2048 && K != 4096)) return false;
+    const int64_t max_rows = 16 * (kMmaUnits / (K / 2048));
+    const int smem = M > 8 ? MmaLayout<16, 1>::bytes(static_cast<int>(K)) : MmaLayout<8, 1>::bytes(static_cast<int>(K));
+    return rows_per_cta(N, dev) <= max_rows && 2 * static_cast<size_t>(smem + 1024) <= dev.max_smem_optin * 2 &&
+           static_cast<size_t>(smem) <= dev.max_smem_optin;
+}
+
 int mt_of(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 8 ? 8 : 16; }
 
 }  // namespace
@@ -826,6 +1095,11 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.ws_rowsum = ws_rowsum;
     a.rb = rb;
     a.status = dev.status;
+    a.out_dtype = out_dtype;
+    if (mma_stream_supported(M, N, K, dev)) {
+        if (xt == BQ_BF16) return launch_mma<__nv_bfloat16>(a, dev, s, grid);
+        return launch_mma<float>(a, dev, s, grid);
+    }
     if (stream_supported(M, N, K, xt, dev)) {
         if (xt == BQ_BF16) return launch_stream_out<__nv_bfloat16>(a, out_dtype, static_cast<int>(M), s, grid);
         return launch_stream_out<float>(a, out_dtype, static_cast<int>(M), s, grid);
