@@ -892,16 +892,20 @@ __global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const D
     const float gamma = __ldg(p.w_scale);
     __syncthreads();
 
-    // token group h (tokens 8 h .. 8 h + 7) in the outer loop: one accumulator set live
+    // token group h (tokens 8 h .. 8 h + 7) in the outer loop: one accumulator
+    // set live, kept across the KBW K blocks of a row block
 #pragma unroll
     for (int h = 0; h < MT / 8; ++h) {
         const int tok = g + 8 * h;
-        int racc[4] = {0, 0, 0, 0};
+        int acc[4][4];
 #pragma unroll
         for (int i = 0; i < kMmaUnits; ++i) {
             const int rb = i / KBW, kb = warp + kMmaWarps * (i % KBW);
+            if (i % KBW == 0) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
+            }
             if (rb < nrb) {
-                int acc[4][4] = {};
 #pragma unroll
                 for (int s = 0; s < 2; ++s) {
                     uint4 bx0 = make_uint4(0u, 0u, 0u, 0u), bx1 = make_uint4(0u, 0u, 0u, 0u);
@@ -920,16 +924,16 @@ __global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const D
                         mma_u8s8_16832(acc[j], a, b0[j], b1[j]);
                     }
                 }
+                if (i % KBW == KBW - 1) {  // last K block of this row block: combine and flush
+                    int v[4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) racc[c] += acc[0][c] + (acc[1][c] >> 2) + (acc[2][c] >> 4) + (acc[3][c] >> 6);
-                if (i % KBW == KBW - 1) {  // last K block of this row block: flush
+                    for (int c = 0; c < 4; ++c) v[c] = acc[0][c] + (acc[1][c] >> 2) + (acc[2][c] >> 4) + (acc[3][c] >> 6);
                     const int r0 = rb * 16 + g, r1 = r0 + 8;
                     const int m0 = 2 * t + 8 * h, m1 = m0 + 1;
-                    if (r0 < rr.rows && m0 < M) atomicAdd(&rowacc[r0 * MT + m0], racc[0]);
-                    if (r0 < rr.rows && m1 < M) atomicAdd(&rowacc[r0 * MT + m1], racc[1]);
-                    if (r1 < rr.rows && m0 < M) atomicAdd(&rowacc[r1 * MT + m0], racc[2]);
-                    if (r1 < rr.rows && m1 < M) atomicAdd(&rowacc[r1 * MT + m1], racc[3]);
-                    racc[0] = racc[1] = racc[2] = racc[3] = 0;
+                    if (r0 < rr.rows && m0 < M) atomicAdd(&rowacc[r0 * MT + m0], v[0]);
+                    if (r0 < rr.rows && m1 < M) atomicAdd(&rowacc[r0 * MT + m1], v[1]);
+                    if (r1 < rr.rows && m0 < M) atomicAdd(&rowacc[r1 * MT + m0], v[2]);
+                    if (r1 < rr.rows && m1 < M) atomicAdd(&rowacc[r1 * MT + m1], v[3]);
                 }
             }
         }

@@ -22,8 +22,11 @@
 // stored in that interleaved order so each matches one dp4a.
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "bq_common.cuh"
 #include "bq_internal.h"
+#include "quant_common.cuh"
 
 namespace bq {
 namespace {
@@ -272,6 +275,259 @@ cudaError_t launch_all(const uint32_t *qweight, const uint16_t *scales, const ui
     return cudaSuccess;
 }
 
+
+// ---------------------------------------------------------------------------
+// One-token decode kernel: a single launch that splits x into its 24-bit
+// planes in shared memory (every CTA, for all of K) and streams the packed
+// weights with a deep per-thread load pipeline.
+//
+// One CTA per SM (512 threads), CTA b owns rows [b N / G, (b+1) N / G).  With
+// CQ = K / 32 chunk columns (a chunk = 4 packed words = 32 weights, inside one
+// group), thread t always works on chunk column q = t % CQ, so the 96 bytes of
+// activation planes its chunks need stay in registers; its rows are
+// rg + RG i (rg = t / CQ, RG = 512 / CQ).  The chunks of a thread are loaded
+// kW4Ahead ahead of their use in a fully unrolled loop, so about 128 KB per
+// SM is in flight.  Per chunk: D_p = sum q * P_p by dp4a, then
+//   v = s[n,g] * sx[g] * (65536 D0 + 256 D1 + D2)  (- s z sx sumX once per group)
+// and the partial row sums of four chunks are reduced across the warp at once
+// (the lanes of a warp share each chunk's row when CQ >= 32).
+// ---------------------------------------------------------------------------
+constexpr int kW4Threads = 512;
+constexpr int kW4Warps = kW4Threads / 32;
+constexpr int kW4Chunks = 28;   // chunks per thread (rows per thread)
+constexpr int kW4Ahead = 16;    // loads in flight per thread
+constexpr int kW4MaxRows = 224;
+
+__device__ __forceinline__ float warp_fsum4(float v0, float v1, float v2, float v3) {
+    const int lane = threadIdx.x & 31;
+    const bool h16 = lane & 16, h8 = lane & 8;
+    float k0 = h16 ? v2 : v0, k1 = h16 ? v3 : v1;
+    k0 += __shfl_xor_sync(0xffffffffu, h16 ? v0 : v2, 16);
+    k1 += __shfl_xor_sync(0xffffffffu, h16 ? v1 : v3, 16);
+    float k = h8 ? k1 : k0;
+    k += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
+    k += __shfl_xor_sync(0xffffffffu, k, 4);
+    k += __shfl_xor_sync(0xffffffffu, k, 2);
+    k += __shfl_xor_sync(0xffffffffu, k, 1);
+    return k;
+}
+
+struct W4DecodeArgs {
+    const float *x;
+    const uint32_t *qweight;
+    const uint16_t *scales;
+    const uint32_t *qzeros;
+    const float *bias;
+    float *out;
+    int N, K, gs;
+};
+
+__global__ void __launch_bounds__(kW4Threads, 1) w4_decode_kernel(const W4DecodeArgs p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int K = p.K, gs = p.gs, G = K / gs, CQ = K / 32, RG = kW4Threads / CQ;
+    int8_t *planes = reinterpret_cast<int8_t *>(smem);                  // [3][K], perm8 order
+    float *s_sx = reinterpret_cast<float *>(smem + 3 * K);              // [G]
+    int *s_sumx = reinterpret_cast<int *>(s_sx + G);                    // [G]
+    float *s_part = reinterpret_cast<float *>(s_sumx + G);              // [kW4MaxRows][4]
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int64_t b = blockIdx.x, Gc = gridDim.x;
+    const int n0 = static_cast<int>((b * p.N) / Gc), rows = static_cast<int>(((b + 1) * p.N) / Gc) - n0;
+    const int q = t % CQ, rg = t / CQ;
+    const int g = q / (gs / 32);                  // group of this chunk column
+    const bool zlead = (q % (gs / 32)) == 0;      // first chunk of its group: adds the zero-point term
+    const int wrow = K / 8, zrow = (G + 7) / 8;
+    const uint4 *wq = reinterpret_cast<const uint4 *>(p.qweight + static_cast<int64_t>(n0) * wrow) + q;
+
+    pdl_launch_dependents();
+    pdl_wait();
+
+    // weight pipeline head: the first kW4Ahead chunks of this thread
+    uint4 w[kW4Ahead];
+    uint16_t sc[kW4Ahead];
+    uint32_t zw[kW4Ahead];
+#pragma unroll
+    for (int i = 0; i < kW4Ahead; ++i) {
+        const int r = rg + RG * i;
+        const bool in = r < rows;
+        w[i] = in ? __ldcs(wq + static_cast<int64_t>(r) * (wrow / 4)) : make_uint4(0u, 0u, 0u, 0u);
+        sc[i] = in ? __ldg(p.scales + static_cast<int64_t>(n0 + r) * G + g) : static_cast<uint16_t>(0);
+        zw[i] = (in && zlead) ? __ldg(p.qzeros + static_cast<int64_t>(n0 + r) * zrow + g / 8) : 0u;
+    }
+
+    // scales and zero-points of this CTA's rows -> shared memory (loads batched)
+    uint16_t *s_scale = reinterpret_cast<uint16_t *>(s_part + kW4MaxRows * (CQ / 32));   // [rows][G]
+    uint32_t *s_zero = reinterpret_cast<uint32_t *>(s_scale + ((kW4MaxRows * G + 1) & ~1));  // [rows][zrow]
+    {
+        const int ns = rows * G, nz = rows * zrow;
+        const uint16_t *sg = p.scales + static_cast<int64_t>(n0) * G;
+        const uint32_t *zg = p.qzeros + static_cast<int64_t>(n0) * zrow;
+        for (int base = 0; base < ns; base += 8 * kW4Threads) {
+            uint16_t v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = base + t + j * kW4Threads;
+                v[j] = i < ns ? __ldg(sg + i) : static_cast<uint16_t>(0);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = base + t + j * kW4Threads;
+                if (i < ns) s_scale[i] = v[j];
+            }
+        }
+        for (int i = t; i < nz; i += kW4Threads) s_zero[i] = __ldg(zg + i);
+    }
+
+    // activation planes: thread t splits elements EPT t .. EPT t + EPT - 1
+    // (EPT = K / 512, one group spans TPG = gs / EPT threads).  X = rne(x / sx),
+    // sx = max|x| / (2^23 - 1) per group, x / sx taken as x * (1 / sx): at
+    // most one more unit of error than the exact quotient.
+    {
+        const int EPT = K / kW4Threads, nv = EPT / 4, TPG = gs / EPT;
+        const float4 *x4 = reinterpret_cast<const float4 *>(p.x) + static_cast<int64_t>(t) * nv;
+        float4 xv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xv[j] = j < nv ? __ldg(x4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(xv[j].x), fabsf(xv[j].y)), fmaxf(fabsf(xv[j].z), fabsf(xv[j].w))));
+        for (int o = TPG / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float sx = __fdiv_rn(amax, 8388607.0f);
+        const float inv = amax > 0.f ? __fdiv_rn(1.0f, sx) : 0.f;
+        int sum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (j < nv) {
+                const float e4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    int X = __float2int_rn(__fmul_rn(e4[u], inv));
+                    X = max(-8388607, min(8388607, X));
+                    sum += X;
+                    const int k = EPT * t + 4 * j + u, jj = k & 7;
+                    const int pos = (k & ~7) + ((jj & 1) ? 4 + (jj >> 1) : (jj >> 1));
+                    planes[pos] = static_cast<int8_t>(X >> 16);
+                    planes[K + pos] = static_cast<int8_t>((X >> 8) & 255);
+                    planes[2 * K + pos] = static_cast<int8_t>(X & 255);
+                }
+            }
+        }
+        for (int o = TPG / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (t % TPG == 0) {
+            s_sx[(EPT * t) / gs] = sx;
+            s_sumx[(EPT * t) / gs] = sum;
+        }
+    }
+    __syncthreads();
+    uint4 xp[3][2];
+#pragma unroll
+    for (int pl = 0; pl < 3; ++pl)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) xp[pl][h] = *reinterpret_cast<const uint4 *>(planes + pl * K + 32 * q + 16 * h);
+    const float sxg = s_sx[g];
+    const float zterm = sxg * static_cast<float>(s_sumx[g]);
+
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < kW4Chunks; ++i) {
+        const int slot = i % kW4Ahead;
+        const int r = rg + RG * i;
+        float val = 0.f;
+        if (r < rows) {
+            const uint32_t wd[4] = {w[slot].x, w[slot].y, w[slot].z, w[slot].w};
+            int d0 = 0;
+            uint32_t d1 = 0u, d2 = 0u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // word j: elements 8 j .. 8 j + 7 of the chunk
+                const uint32_t lo = wd[j] & 0x0f0f0f0fu, hi = (wd[j] >> 4) & 0x0f0f0f0fu;
+                const uint4 &a = xp[0][j >> 1], &bq = xp[1][j >> 1], &c = xp[2][j >> 1];
+                const uint32_t p0l = (j & 1) ? a.z : a.x, p0h = (j & 1) ? a.w : a.y;
+                const uint32_t p1l = (j & 1) ? bq.z : bq.x, p1h = (j & 1) ? bq.w : bq.y;
+                const uint32_t p2l = (j & 1) ? c.z : c.x, p2h = (j & 1) ? c.w : c.y;
+                d0 = dp4a_us(hi, p0h, dp4a_us(lo, p0l, d0));
+                d1 = dp4a_uu(hi, p1h, dp4a_uu(lo, p1l, d1));
+                d2 = dp4a_uu(hi, p2h, dp4a_uu(lo, p2l, d2));
+            }
+            const float T = fmaf(65536.0f, static_cast<float>(d0),
+                                 fmaf(256.0f, static_cast<float>(d1), static_cast<float>(d2)));
+            const float s = __half2float(__ushort_as_half(s_scale[r * G + g]));
+            val = __fmul_rn(__fmul_rn(s, sxg), T);
+            if (zlead) {
+                const float z = static_cast<float>((s_zero[r * zrow + g / 8] >> (4 * (g % 8))) & 15u);
+                val = fmaf(-__fmul_rn(s, z), zterm, val);
+            }
+        }
+        // refill the slot
+        if (i + kW4Ahead < kW4Chunks) {
+            const int rn = rg + RG * (i + kW4Ahead);
+            w[slot] = rn < rows ? __ldcs(wq + static_cast<int64_t>(rn) * (wrow / 4)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        v[i & 3] = val;
+        if ((i & 3) == 3) {
+            const float k = warp_fsum4(v[0], v[1], v[2], v[3]);
+            const int rr = rg + RG * (i - 3 + (lane >> 3));
+            if ((lane & 7) == 0 && rr < rows) s_part[rr * (CQ / 32) + q / 32] = k;
+        }
+    }
+    __syncthreads();
+    for (int r = t; r < rows; r += kW4Threads) {
+        float acc = 0.f;
+        for (int j = 0; j < CQ / 32; ++j) acc += s_part[r * (CQ / 32) + j];
+        p.out[n0 + r] = (p.bias ? __ldg(p.bias + n0 + r) : 0.0f) + acc;
+    }
+}
+
+size_t w4_decode_smem(int K, int gs) {
+    const int G = K / gs, CQ = K / 32, zrow = (G + 7) / 8;
+    size_t b = static_cast<size_t>(3 * K) + 8u * G + 4u * kW4MaxRows * (CQ / 32);
+    b += 2u * ((kW4MaxRows * G + 1) & ~1) + 4u * kW4MaxRows * zrow;
+    return b;
+}
+
+bool w4_decode_supported(int64_t M, int64_t N, int64_t K, int64_t gs, const DevInfo &dev) {
+    if (M != 1 || gs % 32 != 0 || K % gs != 0 || K < 2048 || K > 8192 || (gs & (gs - 1)) != 0) return false;
+    if (gs / (K / kW4Threads) > 32) return false;  // a group spans at most one warp in the split
+    const int64_t CQ = K / 32;
+    if (kW4Threads % CQ != 0) return false;
+    const int64_t RG = kW4Threads / CQ, Gc = std::min<int64_t>(N, dev.num_sms);
+    const int64_t rb = (N + Gc - 1) / Gc;
+    if (rb > kW4Chunks * RG || rb > kW4MaxRows) return false;
+    return w4_decode_smem(static_cast<int>(K), static_cast<int>(gs)) <= dev.max_smem_optin;
+}
+
+cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight, const uint16_t *scales,
+                             const uint32_t *qzeros, const float *bias, int64_t N, int64_t gs, float *out,
+                             cudaStream_t s, const DevInfo &dev) {
+    W4DecodeArgs a;
+    a.x = x;
+    a.qweight = qweight;
+    a.scales = scales;
+    a.qzeros = qzeros;
+    a.bias = bias;
+    a.out = out;
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.gs = static_cast<int>(gs);
+    const int smem = static_cast<int>(w4_decode_smem(a.K, a.gs));
+    static int attr_smem[64] = {};
+    if (smem > 48 * 1024 && smem > attr_smem[dev.device]) {
+        cudaError_t e = cudaFuncSetAttribute(w4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        attr_smem[dev.device] = smem;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(N, dev.num_sms)));
+    cfg.blockDim = dim3(kW4Threads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, w4_decode_kernel, a);
+}
+
 }  // namespace
 
 size_t linear_w4_workspace_bytes(int64_t M, int64_t K, int64_t group_size) {
@@ -283,6 +539,9 @@ size_t linear_w4_workspace_bytes(int64_t M, int64_t K, int64_t group_size) {
 cudaError_t launch_linear_w4(const float *x, int64_t M, int64_t K, const uint32_t *qweight, const uint16_t *scales,
                              const uint32_t *qzeros, const float *bias, int64_t N, int64_t group_size, float *out,
                              void *ws_ptr, cudaStream_t s, const DevInfo &dev) {
+    if (w4_decode_supported(M, N, K, group_size, dev) && reinterpret_cast<uintptr_t>(qweight) % 16 == 0 &&
+        reinterpret_cast<uintptr_t>(x) % 16 == 0)
+        return launch_w4_decode(x, K, qweight, scales, qzeros, bias, N, group_size, out, s, dev);
     const int64_t G = K / group_size;
     const W4Workspace ws = carve(ws_ptr, M, K, G);
     int64_t grid = (M * G + 7) / 8;

@@ -344,7 +344,7 @@ def _w4_check(M, N, K, gs, seed, rows=None, full=None):
     else:
         q, z, s, b, x = full
     qw, qz = bq.bq_weight_pack_int4_grouped(dev(q), dev(z), gs)
-    o = bq.bq_linear_w4_grouped(dev(x), qw, dev(s.view(np.int16)), qz, gs, dev(b))
+    o = bq.bq_linear_w4_grouped(dev(x), qw, dev(s.view(np.int16)), qz, gs, None if b is None else dev(b))
     torch.cuda.synchronize()
     sel = np.arange(M) if rows is None else rows
     ref = oracle.linear_w4_grouped(x[sel], oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), b, gs)
@@ -358,6 +358,20 @@ def _w4_check(M, N, K, gs, seed, rows=None, full=None):
                                       (1, 64, 64, 32), (9, 129, 512, 256)])
 def test_linear_w4_ragged(M, N, K, gs):
     _w4_check(M, N, K, gs, seed=(111, M, N, K))
+
+
+# one token: the single-launch streaming kernel (K = 1024 .. 8192, groups of
+# 32 .. 256, more rows than SMs and fewer, with and without bias)
+@pytest.mark.parametrize("N,K,gs,bias", [(300, 2048, 64, True), (5000, 8192, 256, True), (100, 1024, 32, False),
+                                         (16000, 4096, 128, True), (7, 4096, 128, False)])
+def test_linear_w4_one_token(N, K, gs, bias):
+    g = synth.rng((113, N, K, gs))
+    q = synth.nibbles(g, (N, K))
+    z = synth.nibbles(g, (N, K // gs))
+    s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+    b = synth.normal_f32(g, (N,), 0.01) if bias else None
+    x = synth.normal_f32(g, (1, K))
+    _w4_check(1, N, K, gs, None, full=(q, z, s, b, x))
 
 
 @pytest.mark.parametrize("M", [1, 32])
