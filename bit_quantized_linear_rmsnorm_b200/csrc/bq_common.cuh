@@ -24,6 +24,8 @@ enum Site : uint32_t {
     SITE_DECODE_FULL = 8,
     SITE_DECODE_EMPTY = 9,
     SITE_INT4_PACK = 16,
+    SITE_W4_STAGE = 17,
+    SITE_W4_DRAIN = 18,
 };
 
 __device__ __forceinline__ void report(uint32_t *status, uint32_t code, uint32_t site) {
@@ -193,7 +195,38 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint3
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Arrives on mbarrier `bar` once every cp.async this thread issued so far has
+// landed (the arrival is counted in the barrier's initial count).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Waits until at most N of this thread's committed cp.async groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Same with a count known after unrolling (0..15; larger counts wait for all).
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+    switch (n) {
+        case 15: cp_async_wait_group<15>(); break;
+        case 14: cp_async_wait_group<14>(); break;
+        case 13: cp_async_wait_group<13>(); break;
+        case 12: cp_async_wait_group<12>(); break;
+        case 11: cp_async_wait_group<11>(); break;
+        case 10: cp_async_wait_group<10>(); break;
+        case 9: cp_async_wait_group<9>(); break;
+        case 8: cp_async_wait_group<8>(); break;
+        case 7: cp_async_wait_group<7>(); break;
+        case 6: cp_async_wait_group<6>(); break;
+        case 5: cp_async_wait_group<5>(); break;
+        case 4: cp_async_wait_group<4>(); break;
+        case 3: cp_async_wait_group<3>(); break;
+        case 2: cp_async_wait_group<2>(); break;
+        case 1: cp_async_wait_group<1>(); break;
+        default: cp_async_wait_group<0>(); break;
+    }
+}
 
 // Prefetch of one 128-byte line into L2 (consumes nothing).
 __device__ __forceinline__ void prefetch_l2(const void *p) {

@@ -277,40 +277,39 @@ cudaError_t launch_all(const uint32_t *qweight, const uint16_t *scales, const ui
 
 
 // ---------------------------------------------------------------------------
-// One-token decode kernel: a single launch that splits x into its 24-bit
-// planes in shared memory (every CTA, for all of K) and streams the packed
-// weights with a deep per-thread load pipeline.
+// One-token decode kernel on the mma.sync tensor path: a single launch that
+// splits x into 24-bit planes in shared memory (every CTA, for all of K) and
+// streams the CTA's packed weight rows into a ring of 16-row stages.  One
+// extra warp only issues those copies (16-byte cp.async through the load /
+// store path, measured faster per SM than bulk copies for this stream), and
+// refills a slot as soon as the 16 computing warps have released it (full /
+// empty mbarriers per slot), so the HBM stream keeps going while the other
+// warps split x and compute.
 //
-// One CTA per SM (512 threads), CTA b owns rows [b N / G, (b+1) N / G).  With
-// CQ = K / 32 chunk columns (a chunk = 4 packed words = 32 weights, inside one
-// group), thread t always works on chunk column q = t % CQ, so the 96 bytes of
-// activation planes its chunks need stay in registers; its rows are
-// rg + RG i (rg = t / CQ, RG = 512 / CQ).  The chunks of a thread are loaded
-// kW4Ahead ahead of their use in a fully unrolled loop, so about 128 KB per
-// SM is in flight.  Per chunk: D_p = sum q * P_p by dp4a, then
-//   v = s[n,g] * sx[g] * (65536 D0 + 256 D1 + D2)  (- s z sx sumX once per group)
-// and the partial row sums of four chunks are reduced across the warp at once
-// (the lanes of a warp share each chunk's row when CQ >= 32).
+// The planes use signed base-256 digits, X = 65536 P0 + 256 P1 + P2 with
+// P0, P1, P2 in [-128, 127] (|X| <= 8355711), so all three are s8 columns of
+// one B operand: one m16n8k32 (u8 weights x s8 planes) gives D0, D1 and D2 of
+// 16 rows in columns 0, 1, 2.
+//
+// A stage holds 16 rows at a pitch of K/2 + 64 bytes (the extra 64 bytes put
+// rows g and g + 1 in different bank groups).  Warp w takes the 128-weight
+// spans sp = w + 16 c (c < K / 2048) of every stage (one group each when
+// gs % 128 == 0).  Lane (g, t) reads words 4t .. 4t+3 of the span for rows g
+// and g + 8.  MMA pair e takes words 2e and 2e+1: the low nibbles
+// (word & 0x0f0f0f0f) as one A operand and the high nibbles masked in place
+// (word & 0xf0f0f0f0 = 16 q) as another, into two accumulators combined as
+// C_lo + C_hi / 16 (exact).  The k-slots of lane t map to the elements of words
+// 4t + 2e and 4t + 2e + 1, whose plane bytes (stored in the order 0,2,4,6,1,3,5,7
+// within each 8) are one 16-byte load: .x / .z feed the low-nibble MMA, .y / .w
+// the high-nibble one.
 // ---------------------------------------------------------------------------
-constexpr int kW4Threads = 512;
+constexpr int kW4Threads = 512;                 // computing threads
 constexpr int kW4Warps = kW4Threads / 32;
-constexpr int kW4Chunks = 28;   // chunks per thread (rows per thread)
-constexpr int kW4Ahead = 16;    // loads in flight per thread
-constexpr int kW4MaxRows = 224;
-
-__device__ __forceinline__ float warp_fsum4(float v0, float v1, float v2, float v3) {
-    const int lane = threadIdx.x & 31;
-    const bool h16 = lane & 16, h8 = lane & 8;
-    float k0 = h16 ? v2 : v0, k1 = h16 ? v3 : v1;
-    k0 += __shfl_xor_sync(0xffffffffu, h16 ? v0 : v2, 16);
-    k1 += __shfl_xor_sync(0xffffffffu, h16 ? v1 : v3, 16);
-    float k = h8 ? k1 : k0;
-    k += __shfl_xor_sync(0xffffffffu, h8 ? k0 : k1, 8);
-    k += __shfl_xor_sync(0xffffffffu, k, 4);
-    k += __shfl_xor_sync(0xffffffffu, k, 2);
-    k += __shfl_xor_sync(0xffffffffu, k, 1);
-    return k;
-}
+constexpr int kW4Streamers = 8;                  // warps that only stream the weights
+constexpr int kW4Block = kW4Threads + 32 * kW4Streamers;
+constexpr int kW4MaxRows = 128;
+constexpr int kW4MaxStages = 8;
+constexpr int kW4XMax = 8355711;  // 127 * (65536 + 256 + 1)
 
 struct W4DecodeArgs {
     const float *x;
@@ -319,80 +318,141 @@ struct W4DecodeArgs {
     const uint32_t *qzeros;
     const float *bias;
     float *out;
-    int N, K, gs;
+    int N, K, gs, nstg, rows_cap;
+    uint32_t *status;
 };
 
-__global__ void __launch_bounds__(kW4Threads, 1) w4_decode_kernel(const W4DecodeArgs p) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int K = p.K, gs = p.gs, G = K / gs, CQ = K / 32, RG = kW4Threads / CQ;
-    int8_t *planes = reinterpret_cast<int8_t *>(smem);                  // [3][K], perm8 order
-    float *s_sx = reinterpret_cast<float *>(smem + 3 * K);              // [G]
-    int *s_sumx = reinterpret_cast<int *>(s_sx + G);                    // [G]
-    float *s_part = reinterpret_cast<float *>(s_sumx + G);              // [kW4MaxRows][4]
+__device__ __forceinline__ int digit_s8(int v) { return ((v + 128) & 255) - 128; }
+
+// Shared-memory layout of the kernel (host and device).
+struct W4Layout {
+    int G, zrow, pitch;
+    uint32_t off_sx, off_sumx, off_part, off_tab, off_zero, off_bars, off_ring, total;
+    __host__ __device__ static uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
+    __host__ __device__ W4Layout(int K, int gs, int nstg, int rows_cap) {
+        G = K / gs;
+        zrow = (G + 7) / 8;
+        pitch = K / 2 + 64;
+        off_sx = a16(3u * K);
+        off_sumx = off_sx + 4u * G;
+        off_part = a16(off_sumx + 4u * G);
+        off_tab = a16(off_part + 4u * rows_cap * kW4Warps);
+        off_zero = a16(off_tab + 8u * rows_cap * G);
+        off_bars = a16(off_zero + 4u * rows_cap * zrow);
+        off_ring = (off_bars + 16u * kW4MaxStages + 127u) & ~127u;
+        total = off_ring + static_cast<uint32_t>(nstg) * 16u * pitch;
+    }
+};
+
+template <int SPW>  // spans per warp and stage: K / 2048
+__global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const W4DecodeArgs p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_abort;
+    const int K = p.K, gs = p.gs, nstg = p.nstg;
+    const W4Layout L(K, gs, nstg, p.rows_cap);
+    const int G = L.G, zrow = L.zrow, pitch = L.pitch;
+    int8_t *planes = reinterpret_cast<int8_t *>(smem);                  // [3][K], order 0,2,4,6,1,3,5,7
+    float *s_sx = reinterpret_cast<float *>(smem + L.off_sx);           // [G]
+    int *s_sumx = reinterpret_cast<int *>(smem + L.off_sumx);           // [G]
+    float *s_part = reinterpret_cast<float *>(smem + L.off_part);       // [rows][kW4Warps]
+    float2 *s_tab = reinterpret_cast<float2 *>(smem + L.off_tab);       // [rows][G]: s sx, s sx z sumX
+    uint32_t *s_zero = reinterpret_cast<uint32_t *>(smem + L.off_zero);    // [rows][zrow]
+    // full[s] at bars + 8 s (one arrival + the copy bytes), empty[s] at bars + 8 (kW4MaxStages + s)
+    const uint32_t bars = smem_u32(smem + L.off_bars), ring = smem_u32(smem + L.off_ring);
+    const uint32_t ebars = bars + 8u * kW4MaxStages;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int gq = lane >> 2, tq = lane & 3;
     const int64_t b = blockIdx.x, Gc = gridDim.x;
     const int n0 = static_cast<int>((b * p.N) / Gc), rows = static_cast<int>(((b + 1) * p.N) / Gc) - n0;
-    const int q = t % CQ, rg = t / CQ;
-    const int g = q / (gs / 32);                  // group of this chunk column
-    const bool zlead = (q % (gs / 32)) == 0;      // first chunk of its group: adds the zero-point term
-    const int wrow = K / 8, zrow = (G + 7) / 8;
-    const uint4 *wq = reinterpret_cast<const uint4 *>(p.qweight + static_cast<int64_t>(n0) * wrow) + q;
+    const int nst = (rows + 15) / 16;  // stages of this CTA
+    const uint32_t rowb = static_cast<uint32_t>(K / 2);  // packed bytes per row
+    const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(p.qweight) + static_cast<int64_t>(n0) * rowb;
 
+    if (t == 0) {
+        for (int s = 0; s < nstg; ++s) {
+            mbar_init(bars + 8 * s, 32 * kW4Streamers);  // one arrival per streaming lane
+            mbar_init(ebars + 8 * s, kW4Warps);
+        }
+        s_abort = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
     pdl_launch_dependents();
     pdl_wait();
 
-    // weight pipeline head: the first kW4Ahead chunks of this thread
-    uint4 w[kW4Ahead];
-    uint16_t sc[kW4Ahead];
-    uint32_t zw[kW4Ahead];
-#pragma unroll
-    for (int i = 0; i < kW4Ahead; ++i) {
-        const int r = rg + RG * i;
-        const bool in = r < rows;
-        w[i] = in ? __ldcs(wq + static_cast<int64_t>(r) * (wrow / 4)) : make_uint4(0u, 0u, 0u, 0u);
-        sc[i] = in ? __ldg(p.scales + static_cast<int64_t>(n0 + r) * G + g) : static_cast<uint16_t>(0);
-        zw[i] = (in && zlead) ? __ldg(p.qzeros + static_cast<int64_t>(n0 + r) * zrow + g / 8) : 0u;
+    // the streaming warp copies stage s (rows 16 s .. 16 s + 15) into ring slot
+    // s % nstg, each lane then arriving on the slot's full barrier once its
+    // own copies have landed
+    const int ppr_shift = __ffs(static_cast<int>(rowb / 16)) - 1;  // 16-byte pieces per row (a power of two)
+    const int sl = t - kW4Threads;  // lane among the streaming warps
+    auto issue = [&](int s) {
+        const int slot = s % nstg, r0 = 16 * s, nr = min(16, rows - r0);
+        const uint32_t dst = ring + static_cast<uint32_t>(slot) * 16u * pitch;
+        const int npc = nr << ppr_shift;
+        for (int i = sl; i < npc; i += 32 * kW4Streamers) {
+            const int j = i >> ppr_shift, c = i & ((1 << ppr_shift) - 1);
+            cp_async_16(dst + static_cast<uint32_t>(j) * pitch + 16u * c,
+                        wsrc + static_cast<int64_t>(r0 + j) * rowb + 16 * c, 16u);
+        }
+        cp_async_mbar_arrive_noinc(bars + 8 * slot);
+    };
+    if (warp >= kW4Warps) {  // the streaming warps
+        int s = 0;
+        for (; s < nst; ++s) {
+            const int slot = s % nstg;
+            if (s >= nstg) {  // the slot's previous stage must be released by every computing warp
+                bool ok = mbar_wait(ebars + 8 * slot, ((s / nstg) - 1) & 1, &s_abort, p.status, SITE_W4_STAGE);
+                if (!__all_sync(0xffffffffu, ok)) break;
+            }
+            issue(s);
+        }
+        cp_async_wait_all();  // (the copies land before the warp exits, whatever happened)
+        return;
     }
 
-    // scales and zero-points of this CTA's rows -> shared memory (loads batched)
-    uint16_t *s_scale = reinterpret_cast<uint16_t *>(s_part + kW4MaxRows * (CQ / 32));   // [rows][G]
-    uint32_t *s_zero = reinterpret_cast<uint32_t *>(s_scale + ((kW4MaxRows * G + 1) & ~1));  // [rows][zrow]
+    // activations, scales and zero-points (the weight stream is already running)
+    const int EPT = K / kW4Threads, nv = EPT / 4, TPG = gs / EPT;
+    float4 xv[4];
     {
-        const int ns = rows * G, nz = rows * zrow;
+        const float4 *x4 = reinterpret_cast<const float4 *>(p.x) + static_cast<int64_t>(t) * nv;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) xv[j] = j < nv ? __ldg(x4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int ns = rows * G;
+    uint16_t sv[16];
+    {
+        const int nz = rows * zrow;
         const uint16_t *sg = p.scales + static_cast<int64_t>(n0) * G;
         const uint32_t *zg = p.qzeros + static_cast<int64_t>(n0) * zrow;
-        for (int base = 0; base < ns; base += 8 * kW4Threads) {
-            uint16_t v[8];
+        uint32_t zv[2];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = base + t + j * kW4Threads;
-                v[j] = i < ns ? __ldg(sg + i) : static_cast<uint16_t>(0);
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int i = base + t + j * kW4Threads;
-                if (i < ns) s_scale[i] = v[j];
-            }
+        for (int j = 0; j < 16; ++j) {
+            const int i = t + j * kW4Threads;
+            sv[j] = i < ns ? __ldg(sg + i) : static_cast<uint16_t>(0);
         }
-        for (int i = t; i < nz; i += kW4Threads) s_zero[i] = __ldg(zg + i);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = t + j * kW4Threads;
+            zv[j] = i < nz ? __ldg(zg + i) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int i = t + j * kW4Threads;
+            if (i < nz) s_zero[i] = zv[j];
+        }
     }
 
     // activation planes: thread t splits elements EPT t .. EPT t + EPT - 1
-    // (EPT = K / 512, one group spans TPG = gs / EPT threads).  X = rne(x / sx),
-    // sx = max|x| / (2^23 - 1) per group, x / sx taken as x * (1 / sx): at
+    // (EPT = K / 512; a group spans TPG = gs / EPT threads).  X = rne(x / sx)
+    // with sx = max|x| / 8355711 per group, x / sx taken as x * (1 / sx): at
     // most one more unit of error than the exact quotient.
     {
-        const int EPT = K / kW4Threads, nv = EPT / 4, TPG = gs / EPT;
-        const float4 *x4 = reinterpret_cast<const float4 *>(p.x) + static_cast<int64_t>(t) * nv;
-        float4 xv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) xv[j] = j < nv ? __ldg(x4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
         float amax = 0.f;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             amax = fmaxf(amax, fmaxf(fmaxf(fabsf(xv[j].x), fabsf(xv[j].y)), fmaxf(fabsf(xv[j].z), fabsf(xv[j].w))));
         for (int o = TPG / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float sx = __fdiv_rn(amax, 8388607.0f);
+        const float sx = __fdiv_rn(amax, static_cast<float>(kW4XMax));
         const float inv = amax > 0.f ? __fdiv_rn(1.0f, sx) : 0.f;
         int sum = 0;
 #pragma unroll
@@ -402,13 +462,15 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4_decode_kernel(const W4Decode
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     int X = __float2int_rn(__fmul_rn(e4[u], inv));
-                    X = max(-8388607, min(8388607, X));
+                    X = max(-kW4XMax, min(kW4XMax, X));
                     sum += X;
+                    const int P2 = digit_s8(X), X1 = (X - P2) >> 8;
+                    const int P1 = digit_s8(X1), P0 = (X1 - P1) >> 8;
                     const int k = EPT * t + 4 * j + u, jj = k & 7;
                     const int pos = (k & ~7) + ((jj & 1) ? 4 + (jj >> 1) : (jj >> 1));
-                    planes[pos] = static_cast<int8_t>(X >> 16);
-                    planes[K + pos] = static_cast<int8_t>((X >> 8) & 255);
-                    planes[2 * K + pos] = static_cast<int8_t>(X & 255);
+                    planes[pos] = static_cast<int8_t>(P0);
+                    planes[K + pos] = static_cast<int8_t>(P1);
+                    planes[2 * K + pos] = static_cast<int8_t>(P2);
                 }
             }
         }
@@ -418,81 +480,109 @@ __global__ void __launch_bounds__(kW4Threads, 1) w4_decode_kernel(const W4Decode
             s_sumx[(EPT * t) / gs] = sum;
         }
     }
-    __syncthreads();
-    uint4 xp[3][2];
+    named_bar_sync(1, kW4Threads);
+    // per (row, group): s sx and s sx z sumX (G is a power of two)
+    const int g_shift = __ffs(G) - 1;
 #pragma unroll
-    for (int pl = 0; pl < 3; ++pl)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) xp[pl][h] = *reinterpret_cast<const uint4 *>(planes + pl * K + 32 * q + 16 * h);
-    const float sxg = s_sx[g];
-    const float zterm = sxg * static_cast<float>(s_sumx[g]);
-
-    float v[4];
-#pragma unroll
-    for (int i = 0; i < kW4Chunks; ++i) {
-        const int slot = i % kW4Ahead;
-        const int r = rg + RG * i;
-        float val = 0.f;
-        if (r < rows) {
-            const uint32_t wd[4] = {w[slot].x, w[slot].y, w[slot].z, w[slot].w};
-            int d0 = 0;
-            uint32_t d1 = 0u, d2 = 0u;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {  // word j: elements 8 j .. 8 j + 7 of the chunk
-                const uint32_t lo = wd[j] & 0x0f0f0f0fu, hi = (wd[j] >> 4) & 0x0f0f0f0fu;
-                const uint4 &a = xp[0][j >> 1], &bq = xp[1][j >> 1], &c = xp[2][j >> 1];
-                const uint32_t p0l = (j & 1) ? a.z : a.x, p0h = (j & 1) ? a.w : a.y;
-                const uint32_t p1l = (j & 1) ? bq.z : bq.x, p1h = (j & 1) ? bq.w : bq.y;
-                const uint32_t p2l = (j & 1) ? c.z : c.x, p2h = (j & 1) ? c.w : c.y;
-                d0 = dp4a_us(hi, p0h, dp4a_us(lo, p0l, d0));
-                d1 = dp4a_uu(hi, p1h, dp4a_uu(lo, p1l, d1));
-                d2 = dp4a_uu(hi, p2h, dp4a_uu(lo, p2l, d2));
-            }
-            const float T = fmaf(65536.0f, static_cast<float>(d0),
-                                 fmaf(256.0f, static_cast<float>(d1), static_cast<float>(d2)));
-            const float s = __half2float(__ushort_as_half(s_scale[r * G + g]));
-            val = __fmul_rn(__fmul_rn(s, sxg), T);
-            if (zlead) {
-                const float z = static_cast<float>((s_zero[r * zrow + g / 8] >> (4 * (g % 8))) & 15u);
-                val = fmaf(-__fmul_rn(s, z), zterm, val);
-            }
-        }
-        // refill the slot
-        if (i + kW4Ahead < kW4Chunks) {
-            const int rn = rg + RG * (i + kW4Ahead);
-            w[slot] = rn < rows ? __ldcs(wq + static_cast<int64_t>(rn) * (wrow / 4)) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        v[i & 3] = val;
-        if ((i & 3) == 3) {
-            const float k = warp_fsum4(v[0], v[1], v[2], v[3]);
-            const int rr = rg + RG * (i - 3 + (lane >> 3));
-            if ((lane & 7) == 0 && rr < rows) s_part[rr * (CQ / 32) + q / 32] = k;
+    for (int j = 0; j < 16; ++j) {
+        const int i = t + j * kW4Threads;
+        if (i < ns) {
+            const int r = i >> g_shift, grp = i & (G - 1);
+            const float fs = __fmul_rn(__half2float(__ushort_as_half(sv[j])), s_sx[grp]);
+            const float z = static_cast<float>((s_zero[r * zrow + grp / 8] >> (4 * (grp % 8))) & 15u);
+            s_tab[i] = make_float2(fs, __fmul_rn(__fmul_rn(fs, z), static_cast<float>(s_sumx[grp])));
         }
     }
-    __syncthreads();
+    named_bar_sync(1, kW4Threads);
+
+    const int SPG = gs / 128, spg_shift = __ffs(SPG) - 1;  // spans per group (a power of two)
+    for (int s = 0; s < nst; ++s) {
+        const int slot = s % nstg;
+        bool ok = mbar_wait(bars + 8 * slot, (s / nstg) & 1, &s_abort, p.status, SITE_W4_STAGE);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            const uint32_t sbase = ring + static_cast<uint32_t>(slot) * 16u * pitch;
+            const int r0 = 16 * s + gq, r1 = r0 + 8;
+            float acc0 = 0.f;  // row g (lane t = 0) or g + 8 (lane t = 2)
+#pragma unroll
+            for (int c = 0; c < SPW; ++c) {
+                const int sp = warp + kW4Warps * c;
+                uint4 wa, wb;
+                const uint32_t wad = sbase + static_cast<uint32_t>(gq) * pitch + 64u * sp + 16u * tq;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w) : "r"(wad));
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(wad + 8u * pitch));
+                uint4 bx[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+                if (gq < 3) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+                        bx[e] = *reinterpret_cast<const uint4 *>(planes + gq * K + 128 * sp + 32 * tq + 16 * e);
+                }
+                int clo[4] = {0, 0, 0, 0}, chi[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const uint32_t a0 = e ? wa.z : wa.x, a2 = e ? wa.w : wa.y;
+                    const uint32_t a1 = e ? wb.z : wb.x, a3 = e ? wb.w : wb.y;
+                    const uint32_t lo[4] = {a0 & 0x0f0f0f0fu, a1 & 0x0f0f0f0fu, a2 & 0x0f0f0f0fu, a3 & 0x0f0f0f0fu};
+                    const uint32_t hi[4] = {a0 & 0xf0f0f0f0u, a1 & 0xf0f0f0f0u, a2 & 0xf0f0f0f0u, a3 & 0xf0f0f0f0u};
+                    mma_u8s8_16832(clo, lo, bx[e].x, bx[e].z);
+                    mma_u8s8_16832(chi, hi, bx[e].y, bx[e].w);
+                }
+                int d[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) d[q] = clo[q] + (chi[q] >> 4);
+                // lane t = 0 finishes row g, lane t = 2 row g + 8 (D0, D1 in columns 0, 1 of
+                // lane t = 0, D2 in column 2 of lane t = 1)
+                const int e0 = __shfl_down_sync(0xffffffffu, d[0], 1);
+                const int e1 = __shfl_up_sync(0xffffffffu, d[2], 2), e2 = __shfl_up_sync(0xffffffffu, d[3], 2);
+                const int e3 = __shfl_up_sync(0xffffffffu, d[2], 1);
+                if ((tq & 1) == 0) {
+                    const int row = tq == 0 ? r0 : r1;
+                    const int D0 = tq == 0 ? d[0] : e1, D1 = tq == 0 ? d[1] : e2, D2 = tq == 0 ? e0 : e3;
+                    if (row < rows) {
+                        const float T = fmaf(65536.0f, static_cast<float>(D0),
+                                             fmaf(256.0f, static_cast<float>(D1), static_cast<float>(D2)));
+                        const float2 f = s_tab[row * G + (sp >> spg_shift)];
+                        acc0 += fmaf(f.x, T, (sp & (SPG - 1)) == 0 ? -f.y : 0.0f);
+                    }
+                }
+            }
+            if ((tq & 1) == 0) {
+                const int row = tq == 0 ? r0 : r1;
+                if (row < rows) s_part[row * kW4Warps + warp] = acc0;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ebars + 8 * slot);  // this warp is done with the slot
+    }
+    named_bar_sync(1, kW4Threads);
     for (int r = t; r < rows; r += kW4Threads) {
         float acc = 0.f;
-        for (int j = 0; j < CQ / 32; ++j) acc += s_part[r * (CQ / 32) + j];
+#pragma unroll
+        for (int w = 0; w < kW4Warps; ++w) acc += s_part[r * kW4Warps + w];
         p.out[n0 + r] = (p.bias ? __ldg(p.bias + n0 + r) : 0.0f) + acc;
     }
 }
 
-size_t w4_decode_smem(int K, int gs) {
-    const int G = K / gs, CQ = K / 32, zrow = (G + 7) / 8;
-    size_t b = static_cast<size_t>(3 * K) + 8u * G + 4u * kW4MaxRows * (CQ / 32);
-    b += 2u * ((kW4MaxRows * G + 1) & ~1) + 4u * kW4MaxRows * zrow;
-    return b;
+int w4_rows_cap(int64_t N, const DevInfo &dev) {
+    const int64_t Gc = std::min<int64_t>(N, dev.num_sms);
+    return static_cast<int>((N + Gc - 1) / Gc);
+}
+
+int w4_decode_stages(int K, int gs, int rows_cap, const DevInfo &dev) {
+    const W4Layout L0(K, gs, 0, rows_cap);
+    const int64_t room = static_cast<int64_t>(dev.max_smem_optin) - L0.total;
+    return static_cast<int>(std::min<int64_t>(kW4MaxStages, room / (16 * (K / 2 + 64))));
 }
 
 bool w4_decode_supported(int64_t M, int64_t N, int64_t K, int64_t gs, const DevInfo &dev) {
-    if (M != 1 || gs % 32 != 0 || K % gs != 0 || K < 2048 || K > 8192 || (gs & (gs - 1)) != 0) return false;
+    if (M != 1 || K % 2048 != 0 || K > 8192 || gs % 128 != 0 || K % gs != 0 || (gs & (gs - 1)) != 0) return false;
     if (gs / (K / kW4Threads) > 32) return false;  // a group spans at most one warp in the split
-    const int64_t CQ = K / 32;
-    if (kW4Threads % CQ != 0) return false;
-    const int64_t RG = kW4Threads / CQ, Gc = std::min<int64_t>(N, dev.num_sms);
-    const int64_t rb = (N + Gc - 1) / Gc;
-    if (rb > kW4Chunks * RG || rb > kW4MaxRows) return false;
-    return w4_decode_smem(static_cast<int>(K), static_cast<int>(gs)) <= dev.max_smem_optin;
+    const int64_t Gc = std::min<int64_t>(N, dev.num_sms), rb = (N + Gc - 1) / Gc, G = K / gs;
+    if (rb > kW4MaxRows) return false;
+    if (rb * G > 16 * kW4Threads || rb * ((G + 7) / 8) > 2 * kW4Threads) return false;  // scale / zero registers
+    return w4_decode_stages(static_cast<int>(K), static_cast<int>(gs), static_cast<int>(rb), dev) >= 2;
 }
 
 cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight, const uint16_t *scales,
@@ -508,16 +598,21 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
     a.N = static_cast<int>(N);
     a.K = static_cast<int>(K);
     a.gs = static_cast<int>(gs);
-    const int smem = static_cast<int>(w4_decode_smem(a.K, a.gs));
-    static int attr_smem[64] = {};
-    if (smem > 48 * 1024 && smem > attr_smem[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(w4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    a.rows_cap = w4_rows_cap(N, dev);
+    a.nstg = w4_decode_stages(a.K, a.gs, a.rows_cap, dev);
+    a.status = dev.status;
+    const int smem = static_cast<int>(W4Layout(a.K, a.gs, a.nstg, a.rows_cap).total);
+    auto kern = K == 2048 ? w4_decode_kernel<1> : K == 4096 ? w4_decode_kernel<2> : w4_decode_kernel<4>;
+    static int attr_smem[3][64] = {};
+    int &done = attr_smem[K == 2048 ? 0 : K == 4096 ? 1 : 2][dev.device];
+    if (smem > 48 * 1024 && smem > done) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        attr_smem[dev.device] = smem;
+        done = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(N, dev.num_sms)));
-    cfg.blockDim = dim3(kW4Threads);
+    cfg.blockDim = dim3(kW4Block);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -525,7 +620,7 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, w4_decode_kernel, a);
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace
