@@ -106,7 +106,7 @@ size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t gro
         }
         case BQ_OP_LINEAR_W4_GROUPED:
             if (group_size <= 0) return 0;
-            return linear_w4_workspace_bytes(M, K, group_size);
+            return linear_w4_workspace_bytes(M, N, K, group_size);
         default:
             return 0;
     }
@@ -280,7 +280,7 @@ bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint3
     if (M == 0 || N == 0) return BQ_OK;
     if (x == nullptr || qweight == nullptr || scales_f16 == nullptr || qzeros == nullptr || out == nullptr)
         return BQ_ERR_INVALID_ARG;
-    const size_t need = linear_w4_workspace_bytes(M, K, group_size);
+    const size_t need = linear_w4_workspace_bytes(M, N, K, group_size);
     if (workspace == nullptr || workspace_bytes < need) return BQ_ERR_WORKSPACE;
     if (!aligned(workspace, 256) || !aligned(x, 4) || !aligned(qweight, 4) || !aligned(scales_f16, 2) ||
         !aligned(qzeros, 4) || !aligned(bias, 4) || !aligned(out, 4))

@@ -68,7 +68,13 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
                                const DevInfo &dev);
 
 // Grouped INT4 linear.
-size_t linear_w4_workspace_bytes(int64_t M, int64_t K, int64_t group_size);
+size_t linear_w4_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group_size);
+// Multi-token path on the tensor cores (2..32 tokens, K % 1024 == 0, groups of 128k).
+bool w4_tc_supported(int64_t M, int64_t N, int64_t K, int64_t gs, const DevInfo &dev);
+size_t w4_tc_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_w4_tc(const float *x, int64_t M, int64_t K, const uint32_t *qweight, const uint16_t *scales,
+                         const uint32_t *qzeros, const float *bias, int64_t N, int64_t gs, float *out, void *ws,
+                         cudaStream_t s, const DevInfo &dev);
 cudaError_t launch_linear_w4(const float *x, int64_t M, int64_t K, const uint32_t *qweight,
                              const uint16_t *scales, const uint32_t *qzeros, const float *bias, int64_t N,
                              int64_t group_size, float *out, void *ws, cudaStream_t s, const DevInfo &dev);

@@ -625,10 +625,13 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
 
 }  // namespace
 
-size_t linear_w4_workspace_bytes(int64_t M, int64_t K, int64_t group_size) {
+size_t linear_w4_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group_size) {
     const int64_t G = K / group_size;
-    return align256(static_cast<size_t>(3 * M * K)) + align256(static_cast<size_t>(M * G) * 4) +
-           align256(static_cast<size_t>(M * G) * 4);
+    const size_t planes = align256(static_cast<size_t>(3 * M * K)) + align256(static_cast<size_t>(M * G) * 4) +
+                          align256(static_cast<size_t>(M * G) * 4);
+    // room for the tensor-core path whenever it may be taken (it depends on the device only through the grid)
+    const bool tc = M >= 2 && M <= 32 && K % 1024 == 0 && group_size % 128 == 0 && K % group_size == 0;
+    return tc ? std::max(planes, w4_tc_workspace_bytes(N, K)) : planes;
 }
 
 cudaError_t launch_linear_w4(const float *x, int64_t M, int64_t K, const uint32_t *qweight, const uint16_t *scales,
@@ -637,6 +640,9 @@ cudaError_t launch_linear_w4(const float *x, int64_t M, int64_t K, const uint32_
     if (w4_decode_supported(M, N, K, group_size, dev) && reinterpret_cast<uintptr_t>(qweight) % 16 == 0 &&
         reinterpret_cast<uintptr_t>(x) % 16 == 0)
         return launch_w4_decode(x, K, qweight, scales, qzeros, bias, N, group_size, out, s, dev);
+    if (w4_tc_supported(M, N, K, group_size, dev) && reinterpret_cast<uintptr_t>(qweight) % 16 == 0 &&
+        reinterpret_cast<uintptr_t>(x) % 16 == 0)
+        return launch_w4_tc(x, M, K, qweight, scales, qzeros, bias, N, group_size, out, ws_ptr, s, dev);
     const int64_t G = K / group_size;
     const W4Workspace ws = carve(ws_ptr, M, K, G);
     int64_t grid = (M * G + 7) / 8;

@@ -1,0 +1,432 @@
+// Multi-token grouped INT4 linear on the sm_100a tensor cores
+// ("vyre_libs/nn/linear/inner/linear_4bit/mod.rs" (docs.rs vyre-libs), module
+// doc: grouped affine INT4 linear, one scale and zero-point per group):
+//
+//   out[m,n] = bias[n] + sum_k x[m,k] * s[n,g] * (q[n,k] - z[n,g]),  g = k / gs
+//
+// Three launches (programmatic dependent launch between them):
+//  1. w4_planes_kernel: per token m, X = rne(x / sx) with sx = max|x| / 8355711
+//     over the whole row, written as signed base-256 digits P0, P1, P2
+//     (X = 65536 P0 + 256 P1 + P2, each digit in [-128, 127]).  Plane p of
+//     token m is row 32 p + m of a [96][K] int8 matrix (rows of absent tokens
+//     are zero).  The representation error is at most one unit of sx
+//     (x / sx taken as x * (1 / sx)), i.e. about max|x| * 1.2e-7.
+//  2. w4_tc_kernel: a CTA owns the rows of one row tile and one 1024-wide K
+//     slice.  Per 128-wide K block (one group when gs % 128 == 0) it computes
+//       D[n, 32 p + m] = sum_k (q[n,k] - z[n,g]) * P_p[m,k]
+//     with tcgen05.mma kind::i8 (M = 128 weight rows, N = 96, K = 32 per
+//     instruction, s8 x s8, 32-bit accumulators in TMEM): eight expander warps
+//     turn the packed codes minus the zero-point into s8 in a 128-byte-swizzled
+//     A stage (no dequantized weight reaches global memory); the plane slice
+//     (96 rows x 1024 B) stays resident in shared memory as B.  Per group the
+//     four epilogue warps read the three 32-column planes of their TMEM lane,
+//     T = 65536 D0 + 256 D1 + D2 (fp32), acc[m] += s[n,g] * T[m], and write one
+//     partial sum per (K slice, row, token).
+//  3. w4_reduce_kernel: out = bias + sx[m] * (sum of the K-slice partials,
+//     in slice order), so the result does not depend on scheduling.
+// Every mbarrier wait is bounded; on expiry the kernel records BQ_ERR_TIMEOUT
+// in the status word, drains its own async work and exits.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
+#include "bq_common.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+namespace {
+
+constexpr int kTcTok = 32;                 // token slots (columns per plane)
+constexpr int kTcCols = 3 * kTcTok;        // MMA N
+constexpr int kTcRows = 128;               // MMA M: weight rows per tile
+constexpr int kTcKB = 128;                 // K per stage (one 128-byte swizzle row)
+constexpr int kTcKS = 1024;                // K per CTA slice
+constexpr int kTcBlocks = kTcKS / kTcKB;   // K blocks per slice
+constexpr int kTcStages = 4;               // A stages
+constexpr int kTcMaxTiles = 4;             // row tiles of 128 per CTA
+constexpr int kTcXMax = 8355711;           // 127 * (65536 + 256 + 1)
+constexpr int kTcThreads = 448;            // warps 0-7 expand, 8-11 epilogue, 12 MMA, 13 TMEM
+constexpr uint32_t kTcABytes = kTcRows * kTcKB;       // 16 KB
+constexpr uint32_t kTcBBlock = kTcCols * kTcKB;       // 12 KB
+constexpr uint32_t kTcBBytes = kTcBBlock * kTcBlocks; // 96 KB
+constexpr uint32_t kTcTmemCols = 256;                 // two 96-column accumulators at 0 and 128
+
+struct TcLayout {
+    static constexpr uint32_t OFF_B = 0;
+    static constexpr uint32_t OFF_A = OFF_B + kTcBBytes;
+    static constexpr uint32_t OFF_BAR = OFF_A + kTcStages * kTcABytes;
+    // a_full[S], a_empty[S], t_full[2], t_empty[2], drain
+    static constexpr uint32_t NBAR = 2 * kTcStages + 5;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
+    static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;    // + alignment slack
+};
+
+__device__ __forceinline__ int tc_digit(int v) { return ((v + 128) & 255) - 128; }
+
+// ---------------------------------------------------------------------------
+// 1. activation planes, one CTA per token slot
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) w4_planes_kernel(const float *__restrict__ x, int M, int K,
+                                                       int8_t *__restrict__ planes, float *__restrict__ sx_out) {
+    __shared__ float red[8];
+    const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    pdl_launch_dependents();
+    pdl_wait();
+    int8_t *p0 = planes + static_cast<int64_t>(m) * K;
+    int8_t *p1 = planes + static_cast<int64_t>(kTcTok + m) * K;
+    int8_t *p2 = planes + static_cast<int64_t>(2 * kTcTok + m) * K;
+    if (m >= M) {  // absent token: zero planes
+        for (int k = 4 * t; k < K; k += 4 * 256) {
+            *reinterpret_cast<uint32_t *>(p0 + k) = 0u;
+            *reinterpret_cast<uint32_t *>(p1 + k) = 0u;
+            *reinterpret_cast<uint32_t *>(p2 + k) = 0u;
+        }
+        if (t == 0) sx_out[m] = 0.0f;
+        return;
+    }
+    const float4 *xr = reinterpret_cast<const float4 *>(x + static_cast<int64_t>(m) * K);
+    float amax = 0.f;
+    for (int i = t; i < K / 4; i += 256) {
+        const float4 v = __ldg(xr + i);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
+    const float sx = __fdiv_rn(amax, static_cast<float>(kTcXMax));
+    const float inv = amax > 0.f ? __fdiv_rn(1.0f, sx) : 0.f;
+    if (t == 0) sx_out[m] = sx;
+    for (int i = t; i < K / 4; i += 256) {
+        const float4 v = __ldg(xr + i);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            int X = __float2int_rn(__fmul_rn(e[u], inv));
+            X = max(-kTcXMax, min(kTcXMax, X));
+            const int d2 = tc_digit(X), X1 = (X - d2) >> 8;
+            const int d1 = tc_digit(X1), d0 = (X1 - d1) >> 8;
+            w0 |= (static_cast<uint32_t>(d0) & 255u) << (8 * u);
+            w1 |= (static_cast<uint32_t>(d1) & 255u) << (8 * u);
+            w2 |= (static_cast<uint32_t>(d2) & 255u) << (8 * u);
+        }
+        *reinterpret_cast<uint32_t *>(p0 + 4 * i) = w0;
+        *reinterpret_cast<uint32_t *>(p1 + 4 * i) = w1;
+        *reinterpret_cast<uint32_t *>(p2 + 4 * i) = w2;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. sum of the K-slice partials: out[m][n] = bias[n] + sx[m] * sum_s part[s][n][m]
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) w4_reduce_kernel(const float *__restrict__ part, const float *__restrict__ sx,
+                                                       const float *__restrict__ bias, int M, int N, int S,
+                                                       float *__restrict__ out) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int64_t total = static_cast<int64_t>(N) * M;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int n = static_cast<int>(i / M), m = static_cast<int>(i - static_cast<int64_t>(n) * M);
+        float acc = 0.f;
+        for (int s = 0; s < S; ++s) acc += part[(static_cast<int64_t>(s) * N + n) * kTcTok + m];
+        out[static_cast<int64_t>(m) * N + n] = (bias ? __ldg(bias + n) : 0.0f) + __fmul_rn(sx[m], acc);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2. tensor-core kernel
+// ---------------------------------------------------------------------------
+struct TcArgs {
+    const uint32_t *qweight;
+    const uint16_t *scales;
+    const uint32_t *qzeros;
+    const int8_t *planes;  // [96][K]
+    float *part;           // [S][N][32]
+    int N, K, gs, S, R;    // K slices, row tiles
+    uint32_t *status;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + TcLayout::OFF_BAR;
+    auto a_full = [&](int s) { return bar0 + 8u * s; };
+    auto a_empty = [&](int s) { return bar0 + 8u * (kTcStages + s); };
+    auto t_full = [&](int b) { return bar0 + 8u * (2 * kTcStages + b); };
+    auto t_empty = [&](int b) { return bar0 + 8u * (2 * kTcStages + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TcLayout::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcLayout::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rt = blockIdx.x / p.S, ks = blockIdx.x - rt * p.S;  // row tile, K slice
+    const int n0 = static_cast<int>((static_cast<int64_t>(rt) * p.N) / p.R);
+    const int rows = static_cast<int>((static_cast<int64_t>(rt + 1) * p.N) / p.R) - n0;
+    const int ntiles = (rows + kTcRows - 1) / kTcRows;  // <= kTcMaxTiles (host check)
+    const int nsteps = ntiles * kTcBlocks;
+    const int K = p.K, G = K / p.gs, zrow = (G + 7) / 8;
+    const int kbase = ks * kTcKS;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(a_full(s), 8);  // one arrival per expander warp
+            mbar_init(a_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(t_full(b), 1);
+            mbar_init(t_empty(b), 4);  // one arrival per epilogue warp
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == 13) {
+        tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    pdl_launch_dependents();
+    pdl_wait();  // the planes come from the previous launch
+
+    // resident B: the plane slice (96 rows x 1024 B) as 8 swizzled K blocks
+    for (int i = threadIdx.x; i < kTcCols * (kTcKS / 16); i += kTcThreads) {
+        const int r = i >> 6, c = i & 63, g = c >> 3, cc = c & 7;
+        cp_async_16(sbase + TcLayout::OFF_B + g * kTcBBlock + r * 128 + ((cc ^ (r & 7)) << 4),
+                    p.planes + static_cast<int64_t>(r) * K + kbase + 16 * c, 16u);
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp < 8) {
+        // ------------------------------------------------------------ expanders
+        // thread e: row e % 128 of the tile, K bytes 64 (e / 128) .. + 63 of the block
+        const int e = threadIdx.x, r_t = e & (kTcRows - 1), h = e >> 7;
+        constexpr int kPF = 8;  // steps fetched ahead
+        uint4 pa[kPF], pb[kPF];
+        uint32_t pz[kPF];
+        auto fetch = [&](int j, uint4 &a, uint4 &b, uint32_t &zw) {
+            const int t = j / kTcBlocks, g = j - t * kTcBlocks, r = t * kTcRows + r_t;
+            if (j < nsteps && r < rows) {
+                const int64_t n = n0 + r;
+                const uint4 *src =
+                    reinterpret_cast<const uint4 *>(p.qweight + n * (K / 8) + (kbase + g * kTcKB + 64 * h) / 8);
+                a = __ldcs(src);
+                b = __ldcs(src + 1);
+                const int grp = (kbase + g * kTcKB) / p.gs;
+                zw = __ldg(p.qzeros + n * zrow + grp / 8) >> (4 * (grp % 8));
+            } else {
+                a = b = make_uint4(0u, 0u, 0u, 0u);
+                zw = 0u;
+            }
+        };
+#pragma unroll
+        for (int i = 0; i < kPF; ++i) fetch(i, pa[i], pb[i], pz[i]);
+        bool ok = true;
+#pragma unroll
+        for (int j = 0; j < kTcMaxTiles * kTcBlocks; ++j) {
+            if (j < nsteps && ok) {
+                const int s = j % kTcStages, slot = j % kPF;
+                if (j >= kTcStages) {
+                    ok = mbar_wait(a_empty(s), static_cast<uint32_t>((j / kTcStages) - 1) & 1u, abort_flag, p.status,
+                                   SITE_W4_STAGE);
+                    ok = __all_sync(0xffffffffu, ok);
+                }
+                if (ok) {
+                    const int t = j / kTcBlocks;
+                    if (t * kTcRows + r_t < rows) {
+                        const uint32_t zrep = (pz[slot] & 15u) * 0x01010101u;
+                        const uint32_t wd[8] = {pa[slot].x, pa[slot].y, pa[slot].z, pa[slot].w,
+                                                pb[slot].x, pb[slot].y, pb[slot].z, pb[slot].w};
+                        uint32_t o[16];
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) {  // word w: elements 8 w .. 8 w + 7
+                            const uint32_t lo = wd[w] & 0x0f0f0f0fu, hi = (wd[w] >> 4) & 0x0f0f0f0fu;
+                            o[2 * w] = __vsub4(__byte_perm(lo, hi, 0x5140), zrep);
+                            o[2 * w + 1] = __vsub4(__byte_perm(lo, hi, 0x7362), zrep);
+                        }
+                        uint8_t *row = smem + TcLayout::OFF_A + s * kTcABytes + r_t * 128;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4 *>(row + (((4 * h + c) ^ (r_t & 7)) << 4)) =
+                                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                    }
+                    if (j + kPF < kTcMaxTiles * kTcBlocks) fetch(j + kPF, pa[slot], pb[slot], pz[slot]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(a_full(s));
+                }
+            }
+        }
+    } else if (warp == 12 && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_i8(kTcRows, kTcCols, true, true, false);
+        bool ok = true;
+        for (int j = 0; j < nsteps && ok; ++j) {
+            const int s = j % kTcStages, b = j & 1, g = j % kTcBlocks;
+            if (j >= 2 && !mbar_wait(t_empty(b), static_cast<uint32_t>((j >> 1) - 1) & 1u, abort_flag, p.status,
+                                     SITE_W4_STAGE)) {
+                ok = false;
+                break;
+            }
+            if (!mbar_wait(a_full(s), static_cast<uint32_t>(j / kTcStages) & 1u, abort_flag, p.status,
+                           SITE_W4_STAGE)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = sbase + TcLayout::OFF_A + s * kTcABytes;
+            const uint32_t b_addr = sbase + TcLayout::OFF_B + g * kTcBBlock;
+            const uint32_t d_tmem = tbase + static_cast<uint32_t>(b * 128);
+#pragma unroll
+            for (int kk = 0; kk < kTcKB / 32; ++kk)
+                tc_mma_i8(d_tmem, smem_desc_kmajor_sw128(a_addr + 32 * kk), smem_desc_kmajor_sw128(b_addr + 32 * kk),
+                          idesc, kk != 0 ? 1u : 0u);
+            tc_commit(a_empty(s));
+            tc_commit(t_full(b));
+        }
+        if (!ok) {  // wait until every MMA issued so far has completed
+            tc_commit(drain);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else if (warp >= 8 && warp < 12) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp - 8;  // TMEM lane quarter
+        const int r_in = 32 * q + lane;
+        float acc[kTcTok];
+        for (int j = 0; j < nsteps; ++j) {
+            const int t = j / kTcBlocks, g = j - t * kTcBlocks, b = j & 1;
+            const int r = t * kTcRows + r_in;
+            const bool valid = r < rows;
+            if (g == 0) {
+#pragma unroll
+                for (int i = 0; i < kTcTok; ++i) acc[i] = 0.f;
+            }
+            const int grp = (kbase + g * kTcKB) / p.gs;
+            const float sc =
+                valid ? __half2float(__ushort_as_half(__ldg(p.scales + static_cast<int64_t>(n0 + r) * G + grp))) : 0.f;
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(t_full(b), static_cast<uint32_t>(j >> 1) & 1u, abort_flag, p.status,
+                                          SITE_W4_STAGE);
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
+            tc_fence_after();
+            float T[kTcTok];
+            uint32_t v[32];
+            const uint32_t taddr = tbase + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(32 * q) << 16);
+            tmem_ld_32x32b_x32(taddr, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < kTcTok; ++i) T[i] = __fmul_rn(65536.0f, static_cast<float>(static_cast<int>(v[i])));
+            tmem_ld_32x32b_x32(taddr + 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < kTcTok; ++i) T[i] = fmaf(256.0f, static_cast<float>(static_cast<int>(v[i])), T[i]);
+            tmem_ld_32x32b_x32(taddr + 64, v);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(t_empty(b));
+#pragma unroll
+            for (int i = 0; i < kTcTok; ++i) acc[i] = fmaf(sc, __fadd_rn(T[i], static_cast<float>(static_cast<int>(v[i]))), acc[i]);
+            if (g == kTcBlocks - 1 && valid) {
+                float4 *dst = reinterpret_cast<float4 *>(p.part + (static_cast<int64_t>(ks) * p.N + n0 + r) * kTcTok);
+#pragma unroll
+                for (int i = 0; i < kTcTok / 4; ++i)
+                    dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 13) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTcTmemCols);
+    }
+}
+
+size_t a256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+int tc_slices(int64_t K) { return static_cast<int>(K / kTcKS); }
+
+int tc_row_tiles(int64_t N, int64_t K, const DevInfo &dev) {
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(N, dev.num_sms / tc_slices(K))));
+}
+
+template <typename KernT, typename... Args>
+cudaError_t launch_pdl(KernT kern, unsigned grid, unsigned block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+}  // namespace
+
+bool w4_tc_supported(int64_t M, int64_t N, int64_t K, int64_t gs, const DevInfo &dev) {
+    if (M < 2 || M > kTcTok || K % kTcKS != 0 || K > 16 * kTcKS || gs % kTcKB != 0 || K % gs != 0) return false;
+    const int64_t R = tc_row_tiles(N, K, dev);
+    if (R * tc_slices(K) > dev.num_sms) return false;  // one wave
+    if ((N + R - 1) / R > static_cast<int64_t>(kTcMaxTiles) * kTcRows) return false;
+    return TcLayout::SMEM <= dev.max_smem_optin;
+}
+
+size_t w4_tc_workspace_bytes(int64_t N, int64_t K) {
+    return a256(static_cast<size_t>(kTcCols) * K) + a256(4 * kTcTok) +
+           static_cast<size_t>(K / kTcKS) * N * kTcTok * 4;
+}
+
+cudaError_t launch_w4_tc(const float *x, int64_t M, int64_t K, const uint32_t *qweight, const uint16_t *scales,
+                         const uint32_t *qzeros, const float *bias, int64_t N, int64_t gs, float *out, void *ws,
+                         cudaStream_t s, const DevInfo &dev) {
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    int8_t *planes = reinterpret_cast<int8_t *>(w);
+    float *sx = reinterpret_cast<float *>(w + a256(static_cast<size_t>(kTcCols) * K));
+    float *part = reinterpret_cast<float *>(w + a256(static_cast<size_t>(kTcCols) * K) + a256(4 * kTcTok));
+    cudaError_t e = launch_pdl(w4_planes_kernel, kTcTok, 256, 0, s, x, static_cast<int>(M), static_cast<int>(K),
+                               planes, sx);
+    if (e != cudaSuccess) return e;
+    TcArgs a;
+    a.qweight = qweight;
+    a.scales = scales;
+    a.qzeros = qzeros;
+    a.planes = planes;
+    a.part = part;
+    a.N = static_cast<int>(N);
+    a.K = static_cast<int>(K);
+    a.gs = static_cast<int>(gs);
+    a.S = tc_slices(K);
+    a.R = tc_row_tiles(N, K, dev);
+    a.status = dev.status;
+    static bool attr_set[64] = {};
+    if (!attr_set[dev.device]) {
+        e = cudaFuncSetAttribute(w4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(TcLayout::SMEM));
+        if (e != cudaSuccess) return e;
+        attr_set[dev.device] = true;
+    }
+    e = launch_pdl(w4_tc_kernel, static_cast<unsigned>(a.R * a.S), kTcThreads, TcLayout::SMEM, s, a);
+    if (e != cudaSuccess) return e;
+    const int64_t total = N * M;
+    const unsigned rgrid = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, 4 * dev.num_sms));
+    return launch_pdl(w4_reduce_kernel, rgrid, 256, 0, s, static_cast<const float *>(part),
+                      static_cast<const float *>(sx), bias, static_cast<int>(M), static_cast<int>(N), a.S, out);
+}
+
+}  // namespace bq

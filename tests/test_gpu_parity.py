@@ -376,6 +376,31 @@ def test_linear_w4_one_token(N, K, gs, bias):
     _w4_check(1, N, K, gs, None, full=(q, z, s, b, x))
 
 
+# 2..32 tokens: the tensor-core path (planes prologue, tcgen05 kind::i8 with
+# the codes minus the zero-point expanded in shared memory, K-slice reduction)
+@pytest.mark.parametrize("M,N,K,gs,bias", [(2, 1000, 2048, 128, True), (32, 3000, 4096, 256, True),
+                                           (31, 640, 8192, 128, False), (4, 130, 1024, 128, True)])
+def test_linear_w4_tensor_core(M, N, K, gs, bias):
+    g = synth.rng((114, M, N, K, gs))
+    q = synth.nibbles(g, (N, K))
+    z = synth.nibbles(g, (N, K // gs))
+    s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+    b = synth.normal_f32(g, (N,), 0.01) if bias else None
+    x = synth.normal_f32(g, (M, K))
+    _w4_check(M, N, K, gs, None, full=(q, z, s, b, x))
+
+
+def test_linear_w4_tensor_core_zero_point_equals_code_gives_bias():
+    g = synth.rng(115)
+    N, K, gs = 200, 1024, 128
+    z = synth.nibbles(g, (N, K // gs))
+    q = np.repeat(z, gs, axis=1)
+    s = g.uniform(0.005, 0.02, (N, K // gs)).astype(np.float16)
+    b = synth.normal_f32(g, (N,), 0.01)
+    x = synth.normal_f32(g, (8, K))
+    _w4_check(8, N, K, gs, None, full=(q, z, s, b, x))
+
+
 @pytest.mark.parametrize("M", [1, 32])
 def test_linear_w4_full_size(M):
     w = synth.linear_w4_weights()
