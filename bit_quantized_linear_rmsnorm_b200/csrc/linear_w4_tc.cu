@@ -5,8 +5,9 @@
 //   out[m,n] = bias[n] + sum_k x[m,k] * s[n,g] * (q[n,k] - z[n,g]),  g = k / gs
 //
 // Three launches (programmatic dependent launch between them):
-//  1. w4_planes_kernel: per token m, X = rne(x / sx) with sx = max|x| / 8355711
-//     over the whole row, written as signed base-256 digits P0, P1, P2
+//  1. w4_planes_kernel: per token m and 1024-wide K slice s, X = rne(x / sx)
+//     with sx[m,s] = max|x| / 8355711 over the slice, written as signed
+//     base-256 digits P0, P1, P2
 //     (X = 65536 P0 + 256 P1 + P2, each digit in [-128, 127]).  Plane p of
 //     token m is row 32 p + m of a [96][K] int8 matrix (rows of absent tokens
 //     are zero).  The representation error is at most one unit of sx
@@ -19,11 +20,12 @@
 //     turn the packed codes minus the zero-point into s8 in a 128-byte-swizzled
 //     A stage (no dequantized weight reaches global memory); the plane slice
 //     (96 rows x 1024 B) stays resident in shared memory as B.  Per group the
-//     four epilogue warps read the three 32-column planes of their TMEM lane,
-//     T = 65536 D0 + 256 D1 + D2 (fp32), acc[m] += s[n,g] * T[m], and write one
-//     partial sum per (K slice, row, token).
-//  3. w4_reduce_kernel: out = bias + sx[m] * (sum of the K-slice partials,
-//     in slice order), so the result does not depend on scheduling.
+//     eight epilogue warps (two per TMEM lane quarter, 16 tokens each) read the
+//     three planes of their tokens, T = 65536 D0 + (256 D1 + D2) (the bracket in
+//     int32, T in fp32), acc[m] += s[n,g] * T[m], and write one partial sum per
+//     (K slice, token, row).  Four TMEM accumulators let the MMAs run ahead.
+//  3. w4_reduce_kernel: out = bias + sum over the K slices, in slice order, of
+//     sx[m,s] * partial, so the result does not depend on scheduling.
 // Every mbarrier wait is bounded; on expiry the kernel records BQ_ERR_TIMEOUT
 // in the status word, drains its own async work and exits.
 #include <cuda_fp16.h>
@@ -45,18 +47,24 @@ constexpr int kTcBlocks = kTcKS / kTcKB;   // K blocks per slice
 constexpr int kTcStages = 4;               // A stages
 constexpr int kTcMaxTiles = 4;             // row tiles of 128 per CTA
 constexpr int kTcXMax = 8355711;           // 127 * (65536 + 256 + 1)
-constexpr int kTcThreads = 448;            // warps 0-7 expand, 8-11 epilogue, 12 MMA, 13 TMEM
+constexpr int kTcThreads = 576;            // warps 0-7 expand, 8-15 epilogue, 16 MMA, 17 TMEM
+constexpr int kTcBufs = 4;                 // TMEM accumulators (96 columns each)
+constexpr int kTcRing = 6;                 // packed weight steps in flight per expander thread
 constexpr uint32_t kTcABytes = kTcRows * kTcKB;       // 16 KB
 constexpr uint32_t kTcBBlock = kTcCols * kTcKB;       // 12 KB
 constexpr uint32_t kTcBBytes = kTcBBlock * kTcBlocks; // 96 KB
-constexpr uint32_t kTcTmemCols = 256;                 // two 96-column accumulators at 0 and 128
+constexpr uint32_t kTcTmemCols = 512;                 // four 96-column accumulators at 0, 128, 256, 384
 
 struct TcLayout {
     static constexpr uint32_t OFF_B = 0;
     static constexpr uint32_t OFF_A = OFF_B + kTcBBytes;
-    static constexpr uint32_t OFF_BAR = OFF_A + kTcStages * kTcABytes;
-    // a_full[S], a_empty[S], t_full[2], t_empty[2], drain
-    static constexpr uint32_t NBAR = 2 * kTcStages + 5;
+    // packed weights: [kTcRing][2 rows][256 expander threads][16 B] (each thread its own pieces)
+    static constexpr uint32_t OFF_P = OFF_A + kTcStages * kTcABytes;
+    static constexpr uint32_t P_BYTES = kTcRing * 2 * 256 * 16;
+    static constexpr uint32_t OFF_Z = OFF_P + P_BYTES;  // zero-point word of each row for the slice
+    static constexpr uint32_t OFF_BAR = OFF_Z + kTcMaxTiles * kTcRows * 4;
+    // a_full[S], a_empty[S], t_full[B], t_empty[B], drain
+    static constexpr uint32_t NBAR = 2 * kTcStages + 2 * kTcBufs + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
     static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;    // + alignment slack
 };
@@ -64,32 +72,28 @@ struct TcLayout {
 __device__ __forceinline__ int tc_digit(int v) { return ((v + 128) & 255) - 128; }
 
 // ---------------------------------------------------------------------------
-// 1. activation planes, one CTA per token slot
+// 1. activation planes, one CTA per (token slot, K slice) (256 threads x 4 elements)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) w4_planes_kernel(const float *__restrict__ x, int M, int K,
                                                        int8_t *__restrict__ planes, float *__restrict__ sx_out) {
     __shared__ float red[8];
-    const int m = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int S = K / kTcKS;
+    const int m = blockIdx.x / S, s = blockIdx.x - m * S, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     pdl_launch_dependents();
     pdl_wait();
-    int8_t *p0 = planes + static_cast<int64_t>(m) * K;
-    int8_t *p1 = planes + static_cast<int64_t>(kTcTok + m) * K;
-    int8_t *p2 = planes + static_cast<int64_t>(2 * kTcTok + m) * K;
+    const int k = s * kTcKS + 4 * t;
+    int8_t *p0 = planes + static_cast<int64_t>(m) * K + k;
+    int8_t *p1 = planes + static_cast<int64_t>(kTcTok + m) * K + k;
+    int8_t *p2 = planes + static_cast<int64_t>(2 * kTcTok + m) * K + k;
     if (m >= M) {  // absent token: zero planes
-        for (int k = 4 * t; k < K; k += 4 * 256) {
-            *reinterpret_cast<uint32_t *>(p0 + k) = 0u;
-            *reinterpret_cast<uint32_t *>(p1 + k) = 0u;
-            *reinterpret_cast<uint32_t *>(p2 + k) = 0u;
-        }
-        if (t == 0) sx_out[m] = 0.0f;
+        *reinterpret_cast<uint32_t *>(p0) = 0u;
+        *reinterpret_cast<uint32_t *>(p1) = 0u;
+        *reinterpret_cast<uint32_t *>(p2) = 0u;
+        if (t == 0) sx_out[m * S + s] = 0.0f;
         return;
     }
-    const float4 *xr = reinterpret_cast<const float4 *>(x + static_cast<int64_t>(m) * K);
-    float amax = 0.f;
-    for (int i = t; i < K / 4; i += 256) {
-        const float4 v = __ldg(xr + i);
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-    }
+    const float4 v = __ldg(reinterpret_cast<const float4 *>(x + static_cast<int64_t>(m) * K + k));
+    float amax = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) red[warp] = amax;
@@ -99,29 +103,26 @@ __global__ void __launch_bounds__(256) w4_planes_kernel(const float *__restrict_
     for (int w = 0; w < 8; ++w) amax = fmaxf(amax, red[w]);
     const float sx = __fdiv_rn(amax, static_cast<float>(kTcXMax));
     const float inv = amax > 0.f ? __fdiv_rn(1.0f, sx) : 0.f;
-    if (t == 0) sx_out[m] = sx;
-    for (int i = t; i < K / 4; i += 256) {
-        const float4 v = __ldg(xr + i);
-        const float e[4] = {v.x, v.y, v.z, v.w};
-        uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
+    if (t == 0) sx_out[m * S + s] = sx;
+    const float e[4] = {v.x, v.y, v.z, v.w};
+    uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            int X = __float2int_rn(__fmul_rn(e[u], inv));
-            X = max(-kTcXMax, min(kTcXMax, X));
-            const int d2 = tc_digit(X), X1 = (X - d2) >> 8;
-            const int d1 = tc_digit(X1), d0 = (X1 - d1) >> 8;
-            w0 |= (static_cast<uint32_t>(d0) & 255u) << (8 * u);
-            w1 |= (static_cast<uint32_t>(d1) & 255u) << (8 * u);
-            w2 |= (static_cast<uint32_t>(d2) & 255u) << (8 * u);
-        }
-        *reinterpret_cast<uint32_t *>(p0 + 4 * i) = w0;
-        *reinterpret_cast<uint32_t *>(p1 + 4 * i) = w1;
-        *reinterpret_cast<uint32_t *>(p2 + 4 * i) = w2;
+    for (int u = 0; u < 4; ++u) {
+        int X = __float2int_rn(__fmul_rn(e[u], inv));
+        X = max(-kTcXMax, min(kTcXMax, X));
+        const int d2 = tc_digit(X), X1 = (X - d2) >> 8;
+        const int d1 = tc_digit(X1), d0 = (X1 - d1) >> 8;
+        w0 |= (static_cast<uint32_t>(d0) & 255u) << (8 * u);
+        w1 |= (static_cast<uint32_t>(d1) & 255u) << (8 * u);
+        w2 |= (static_cast<uint32_t>(d2) & 255u) << (8 * u);
     }
+    *reinterpret_cast<uint32_t *>(p0) = w0;
+    *reinterpret_cast<uint32_t *>(p1) = w1;
+    *reinterpret_cast<uint32_t *>(p2) = w2;
 }
 
 // ---------------------------------------------------------------------------
-// 3. sum of the K-slice partials: out[m][n] = bias[n] + sx[m] * sum_s part[s][n][m]
+// 3. out[m][n] = bias[n] + sum_s sx[m,s] * part[s][m][n]  (slices in order)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) w4_reduce_kernel(const float *__restrict__ part, const float *__restrict__ sx,
                                                        const float *__restrict__ bias, int M, int N, int S,
@@ -131,10 +132,11 @@ __global__ void __launch_bounds__(256) w4_reduce_kernel(const float *__restrict_
     const int64_t total = static_cast<int64_t>(N) * M;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int n = static_cast<int>(i / M), m = static_cast<int>(i - static_cast<int64_t>(n) * M);
+        const int m = static_cast<int>(i / N), n = static_cast<int>(i - static_cast<int64_t>(m) * N);
         float acc = 0.f;
-        for (int s = 0; s < S; ++s) acc += part[(static_cast<int64_t>(s) * N + n) * kTcTok + m];
-        out[static_cast<int64_t>(m) * N + n] = (bias ? __ldg(bias + n) : 0.0f) + __fmul_rn(sx[m], acc);
+        for (int s = 0; s < S; ++s)
+            acc = fmaf(sx[m * S + s], part[(static_cast<int64_t>(s) * kTcTok + m) * N + n], acc);
+        out[static_cast<int64_t>(m) * N + n] = (bias ? __ldg(bias + n) : 0.0f) + acc;
     }
 }
 
@@ -146,7 +148,7 @@ struct TcArgs {
     const uint16_t *scales;
     const uint32_t *qzeros;
     const int8_t *planes;  // [96][K]
-    float *part;           // [S][N][32]
+    float *part;           // [S][32][N]
     int N, K, gs, S, R;    // K slices, row tiles
     uint32_t *status;
 };
@@ -159,8 +161,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
     auto a_full = [&](int s) { return bar0 + 8u * s; };
     auto a_empty = [&](int s) { return bar0 + 8u * (kTcStages + s); };
     auto t_full = [&](int b) { return bar0 + 8u * (2 * kTcStages + b); };
-    auto t_empty = [&](int b) { return bar0 + 8u * (2 * kTcStages + 2 + b); };
-    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 4);
+    auto t_empty = [&](int b) { return bar0 + 8u * (2 * kTcStages + kTcBufs + b); };
+    const uint32_t drain = bar0 + 8u * (2 * kTcStages + 2 * kTcBufs);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TcLayout::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + TcLayout::OFF_MISC + 4);
 
@@ -178,15 +180,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
             mbar_init(a_full(s), 8);  // one arrival per expander warp
             mbar_init(a_empty(s), 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kTcBufs; ++b) {
             mbar_init(t_full(b), 1);
-            mbar_init(t_empty(b), 4);  // one arrival per epilogue warp
+            mbar_init(t_empty(b), 8);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (warp == 13) {
+    if (warp == 17) {
         tmem_alloc(smem_u32(tmem_slot), kTcTmemCols);
         tmem_relinquish();
         tc_fence_before();
@@ -200,6 +202,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         cp_async_16(sbase + TcLayout::OFF_B + g * kTcBBlock + r * 128 + ((cc ^ (r & 7)) << 4),
                     p.planes + static_cast<int64_t>(r) * K + kbase + 16 * c, 16u);
     }
+    {  // the zero-point word (8 nibbles) covering this slice's groups, per row
+        uint32_t *zs = reinterpret_cast<uint32_t *>(smem + TcLayout::OFF_Z);
+        const int zw = (kbase / p.gs) / 8;
+        for (int r = threadIdx.x; r < rows; r += kTcThreads) zs[r] = __ldg(p.qzeros + static_cast<int64_t>(n0 + r) * zrow + zw);
+    }
     cp_async_wait_all();
     fence_proxy_async_smem();
     __syncthreads();
@@ -208,76 +215,89 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
 
     if (warp < 8) {
         // ------------------------------------------------------------ expanders
-        // thread e: row e % 128 of the tile, K bytes 64 (e / 128) .. + 63 of the block
-        const int e = threadIdx.x, r_t = e & (kTcRows - 1), h = e >> 7;
-        constexpr int kPF = 8;  // steps fetched ahead
-        uint4 pa[kPF], pb[kPF];
-        uint32_t pz[kPF];
-        auto fetch = [&](int j, uint4 &a, uint4 &b, uint32_t &zw) {
-            const int t = j / kTcBlocks, g = j - t * kTcBlocks, r = t * kTcRows + r_t;
-            if (j < nsteps && r < rows) {
-                const int64_t n = n0 + r;
-                const uint4 *src =
-                    reinterpret_cast<const uint4 *>(p.qweight + n * (K / 8) + (kbase + g * kTcKB + 64 * h) / 8);
-                a = __ldcs(src);
-                b = __ldcs(src + 1);
-                const int grp = (kbase + g * kTcKB) / p.gs;
-                zw = __ldg(p.qzeros + n * zrow + grp / 8) >> (4 * (grp % 8));
-            } else {
-                a = b = make_uint4(0u, 0u, 0u, 0u);
-                zw = 0u;
+        // thread e: 16-byte piece pc = e % 4 (32 codes) of the block's 64 packed
+        // bytes, for rows rr = e / 4 and rr + 64 of the tile; four lanes cover a
+        // row's block, so every copy instruction reads whole 64-byte segments.
+        // The pieces are copied kTcRing steps ahead (cp.async into this
+        // thread's own ring slots, read back by the same thread).
+        const int e = threadIdx.x, pc = e & 3, rr = e >> 2;
+        const uint32_t *zs = reinterpret_cast<const uint32_t *>(smem + TcLayout::OFF_Z);
+        auto slot_addr = [&](int j, int half) {
+            return sbase + TcLayout::OFF_P + static_cast<uint32_t>((((j % kTcRing) * 2 + half) * 256 + e) * 16);
+        };
+        auto issue = [&](int j) {
+            const int t = j / kTcBlocks, g = j - t * kTcBlocks;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int r = t * kTcRows + rr + 64 * half;
+                const bool in = j < nsteps && r < rows;
+                const uint32_t *src = p.qweight + static_cast<int64_t>(n0 + (in ? r : 0)) * (K / 8) +
+                                      (kbase + g * kTcKB + 32 * pc) / 8;
+                cp_async_16(slot_addr(j, half), src, in ? 16u : 0u);
             }
+            cp_async_commit();
         };
 #pragma unroll
-        for (int i = 0; i < kPF; ++i) fetch(i, pa[i], pb[i], pz[i]);
+        for (int i = 0; i < kTcRing; ++i) issue(i);
+        // expand one row's piece: codes minus the zero-point as s8, two 16-byte chunks
+        auto expand = [&](uint8_t *row, int r_t, const uint4 &w, uint32_t zw) {
+            const uint32_t zrep = (zw & 15u) * 0x01010101u;
+            const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+            uint32_t o[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {  // word k: codes 8 k .. 8 k + 7 of the piece
+                const uint32_t lo = wd[k] & 0x0f0f0f0fu, hi = (wd[k] >> 4) & 0x0f0f0f0fu;
+                o[2 * k] = __vsub4(__byte_perm(lo, hi, 0x5140), zrep);
+                o[2 * k + 1] = __vsub4(__byte_perm(lo, hi, 0x7362), zrep);
+            }
+            *reinterpret_cast<uint4 *>(row + (((2 * pc) ^ (r_t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(row + (((2 * pc + 1) ^ (r_t & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        };
         bool ok = true;
 #pragma unroll
         for (int j = 0; j < kTcMaxTiles * kTcBlocks; ++j) {
             if (j < nsteps && ok) {
-                const int s = j % kTcStages, slot = j % kPF;
+                const int s = j % kTcStages;
                 if (j >= kTcStages) {
-                    ok = mbar_wait(a_empty(s), static_cast<uint32_t>((j / kTcStages) - 1) & 1u, abort_flag, p.status,
+                    ok = mbar_wait_spin(a_empty(s), static_cast<uint32_t>((j / kTcStages) - 1) & 1u, abort_flag, p.status,
                                    SITE_W4_STAGE);
                     ok = __all_sync(0xffffffffu, ok);
                 }
                 if (ok) {
-                    const int t = j / kTcBlocks;
-                    if (t * kTcRows + r_t < rows) {
-                        const uint32_t zrep = (pz[slot] & 15u) * 0x01010101u;
-                        const uint32_t wd[8] = {pa[slot].x, pa[slot].y, pa[slot].z, pa[slot].w,
-                                                pb[slot].x, pb[slot].y, pb[slot].z, pb[slot].w};
-                        uint32_t o[16];
-#pragma unroll
-                        for (int w = 0; w < 8; ++w) {  // word w: elements 8 w .. 8 w + 7
-                            const uint32_t lo = wd[w] & 0x0f0f0f0fu, hi = (wd[w] >> 4) & 0x0f0f0f0fu;
-                            o[2 * w] = __vsub4(__byte_perm(lo, hi, 0x5140), zrep);
-                            o[2 * w + 1] = __vsub4(__byte_perm(lo, hi, 0x7362), zrep);
-                        }
-                        uint8_t *row = smem + TcLayout::OFF_A + s * kTcABytes + r_t * 128;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            *reinterpret_cast<uint4 *>(row + (((4 * h + c) ^ (r_t & 7)) << 4)) =
-                                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-                    }
-                    if (j + kPF < kTcMaxTiles * kTcBlocks) fetch(j + kPF, pa[slot], pb[slot], pz[slot]);
+                    const int t = j / kTcBlocks, g = j - t * kTcBlocks;
+                    // this step's copies have landed (at most kTcRing - 1 later groups pending)
+                    cp_async_wait_pending(min(kTcRing, kTcMaxTiles * kTcBlocks - j) - 1);
+                    uint4 wa, wb;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w) : "r"(slot_addr(j, 0)));
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(slot_addr(j, 1)));
+                    const int zsh = 4 * (((kbase + g * kTcKB) / p.gs) % 8);
+                    uint8_t *stage = smem + TcLayout::OFF_A + s * kTcABytes;
+                    if (t * kTcRows + rr < rows) expand(stage + rr * 128, rr, wa, zs[t * kTcRows + rr] >> zsh);
+                    if (t * kTcRows + rr + 64 < rows)
+                        expand(stage + (rr + 64) * 128, rr + 64, wb, zs[t * kTcRows + rr + 64] >> zsh);
+                    // the slot's pieces are in registers: refill it
+                    if (j + kTcRing < kTcMaxTiles * kTcBlocks) issue(j + kTcRing);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(a_full(s));
                 }
             }
         }
-    } else if (warp == 12 && lane == 0) {
+        cp_async_wait_all();  // (copies issued past the last step land before the CTA exits)
+    } else if (warp == 16 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = idesc_i8(kTcRows, kTcCols, true, true, false);
         bool ok = true;
         for (int j = 0; j < nsteps && ok; ++j) {
-            const int s = j % kTcStages, b = j & 1, g = j % kTcBlocks;
-            if (j >= 2 && !mbar_wait(t_empty(b), static_cast<uint32_t>((j >> 1) - 1) & 1u, abort_flag, p.status,
-                                     SITE_W4_STAGE)) {
+            const int s = j % kTcStages, b = j % kTcBufs, g = j % kTcBlocks;
+            if (j >= kTcBufs && !mbar_wait_spin(t_empty(b), static_cast<uint32_t>((j / kTcBufs) - 1) & 1u, abort_flag,
+                                           p.status, SITE_W4_STAGE)) {
                 ok = false;
                 break;
             }
-            if (!mbar_wait(a_full(s), static_cast<uint32_t>(j / kTcStages) & 1u, abort_flag, p.status,
+            if (!mbar_wait_spin(a_full(s), static_cast<uint32_t>(j / kTcStages) & 1u, abort_flag, p.status,
                            SITE_W4_STAGE)) {
                 ok = false;
                 break;
@@ -299,56 +319,55 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
             while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
             }
         }
-    } else if (warp >= 8 && warp < 12) {
+    } else if (warp >= 8 && warp < 16) {
         // ------------------------------------------------------------ epilogue
-        const int q = warp - 8;  // TMEM lane quarter
+        const int q = warp & 3;          // TMEM lane quarter
+        const int th = (warp - 8) >> 2;  // tokens 16 th .. 16 th + 15
         const int r_in = 32 * q + lane;
-        float acc[kTcTok];
+        float acc[16];
         for (int j = 0; j < nsteps; ++j) {
-            const int t = j / kTcBlocks, g = j - t * kTcBlocks, b = j & 1;
+            const int t = j / kTcBlocks, g = j - t * kTcBlocks, b = j % kTcBufs;
             const int r = t * kTcRows + r_in;
             const bool valid = r < rows;
             if (g == 0) {
 #pragma unroll
-                for (int i = 0; i < kTcTok; ++i) acc[i] = 0.f;
+                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
             }
             const int grp = (kbase + g * kTcKB) / p.gs;
             const float sc =
                 valid ? __half2float(__ushort_as_half(__ldg(p.scales + static_cast<int64_t>(n0 + r) * G + grp))) : 0.f;
             bool ok = true;
-            if (lane == 0) ok = mbar_wait(t_full(b), static_cast<uint32_t>(j >> 1) & 1u, abort_flag, p.status,
-                                          SITE_W4_STAGE);
+            if (lane == 0)
+                ok = mbar_wait_spin(t_full(b), static_cast<uint32_t>(j / kTcBufs) & 1u, abort_flag, p.status,
+                               SITE_W4_STAGE);
             if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
             tc_fence_after();
-            float T[kTcTok];
-            uint32_t v[32];
-            const uint32_t taddr = tbase + static_cast<uint32_t>(b * 128) + (static_cast<uint32_t>(32 * q) << 16);
-            tmem_ld_32x32b_x32(taddr, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < kTcTok; ++i) T[i] = __fmul_rn(65536.0f, static_cast<float>(static_cast<int>(v[i])));
-            tmem_ld_32x32b_x32(taddr + 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < kTcTok; ++i) T[i] = fmaf(256.0f, static_cast<float>(static_cast<int>(v[i])), T[i]);
-            tmem_ld_32x32b_x32(taddr + 64, v);
+            uint32_t d0[16], d1[16], d2[16];
+            const uint32_t taddr = tbase + static_cast<uint32_t>(b * 128 + 16 * th) +
+                                   (static_cast<uint32_t>(32 * q) << 16);
+            tmem_ld_32x32b_x16(taddr, d0);
+            tmem_ld_32x32b_x16(taddr + kTcTok, d1);
+            tmem_ld_32x32b_x16(taddr + 2 * kTcTok, d2);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(t_empty(b));
 #pragma unroll
-            for (int i = 0; i < kTcTok; ++i) acc[i] = fmaf(sc, __fadd_rn(T[i], static_cast<float>(static_cast<int>(v[i]))), acc[i]);
+            for (int i = 0; i < 16; ++i) {
+                const int e = 256 * static_cast<int>(d1[i]) + static_cast<int>(d2[i]);  // |e| < 2^26
+                const float T = fmaf(65536.0f, static_cast<float>(static_cast<int>(d0[i])), static_cast<float>(e));
+                acc[i] = fmaf(sc, T, acc[i]);
+            }
             if (g == kTcBlocks - 1 && valid) {
-                float4 *dst = reinterpret_cast<float4 *>(p.part + (static_cast<int64_t>(ks) * p.N + n0 + r) * kTcTok);
+                float *dst = p.part + (static_cast<int64_t>(ks) * kTcTok + 16 * th) * p.N + n0 + r;
 #pragma unroll
-                for (int i = 0; i < kTcTok / 4; ++i)
-                    dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                for (int i = 0; i < 16; ++i) dst[static_cast<int64_t>(i) * p.N] = acc[i];
             }
         }
     }
 
     __syncthreads();
-    if (warp == 13) {
+    if (warp == 17) {
         tc_fence_after();
         tmem_dealloc(tbase, kTcTmemCols);
     }
@@ -388,7 +407,7 @@ bool w4_tc_supported(int64_t M, int64_t N, int64_t K, int64_t gs, const DevInfo 
 }
 
 size_t w4_tc_workspace_bytes(int64_t N, int64_t K) {
-    return a256(static_cast<size_t>(kTcCols) * K) + a256(4 * kTcTok) +
+    return a256(static_cast<size_t>(kTcCols) * K) + a256(4 * kTcTok * (K / kTcKS)) +
            static_cast<size_t>(K / kTcKS) * N * kTcTok * 4;
 }
 
@@ -398,9 +417,10 @@ cudaError_t launch_w4_tc(const float *x, int64_t M, int64_t K, const uint32_t *q
     uint8_t *w = static_cast<uint8_t *>(ws);
     int8_t *planes = reinterpret_cast<int8_t *>(w);
     float *sx = reinterpret_cast<float *>(w + a256(static_cast<size_t>(kTcCols) * K));
-    float *part = reinterpret_cast<float *>(w + a256(static_cast<size_t>(kTcCols) * K) + a256(4 * kTcTok));
-    cudaError_t e = launch_pdl(w4_planes_kernel, kTcTok, 256, 0, s, x, static_cast<int>(M), static_cast<int>(K),
-                               planes, sx);
+    float *part = reinterpret_cast<float *>(w + a256(static_cast<size_t>(kTcCols) * K) +
+                                            a256(4 * kTcTok * static_cast<size_t>(K / kTcKS)));
+    cudaError_t e = launch_pdl(w4_planes_kernel, static_cast<unsigned>(kTcTok * (K / kTcKS)), 256, 0, s, x,
+                               static_cast<int>(M), static_cast<int>(K), planes, sx);
     if (e != cudaSuccess) return e;
     TcArgs a;
     a.qweight = qweight;
