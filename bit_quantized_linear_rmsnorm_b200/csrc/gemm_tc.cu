@@ -24,7 +24,7 @@
 //               lanes 32*(w%4)..), scale in fp32, round once, stage through a
 //               64-byte-swizzled buffer, TMA store (out-of-range rows/cols are
 //               clipped by the TMA unit).
-//   warps 8-11  (W2A8 only) unpack 2-bit codes into the B stage.
+//   warps 8-15  (W2A8 only) unpack 2-bit codes into the B stage.
 // Every mbarrier wait is bounded; on expiry the kernel records
 // BQ_ERR_TIMEOUT in the status word, drains its own async work and exits.
 #include <cuda_bf16.h>
@@ -51,7 +51,8 @@ constexpr uint32_t STG_BYTES = BM * 64;         // 8 KB epilogue staging buffer
 template <bool PACKED>
 struct Cfg {
     static constexpr int kStages = PACKED ? 3 : 4;
-    static constexpr int kThreads = PACKED ? 384 : 256;
+    static constexpr int kUnpack = 256;  // unpack threads (W2A8)
+    static constexpr int kThreads = PACKED ? 256 + kUnpack : 256;
     static constexpr uint32_t OFF_A = 0;
     static constexpr uint32_t OFF_B = OFF_A + kStages * A_BYTES;
     static constexpr uint32_t OFF_P = OFF_B + kStages * B_BYTES;
@@ -135,7 +136,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 1);
-            mbar_init(bready(s), 128);
+            mbar_init(bready(s), C::kUnpack);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         if (et == 0) bulk_wait_all();
     } else if (PACKED && warp >= 8) {
         // ------------------------------------------------------------ unpack 2-bit codes
-        const int ut = threadIdx.x - 256;  // 0..127
+        const int ut = threadIdx.x - 256;  // 0 .. C::kUnpack - 1
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -371,8 +372,8 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                 const uint32_t *pk = reinterpret_cast<const uint32_t *>(smem + C::OFF_P + stage * P_BYTES);
                 uint8_t *bt = smem + C::OFF_B + stage * B_BYTES;
 #pragma unroll 4
-                for (int i = 0; i < (BN * 8) / 128; ++i) {
-                    const int idx = ut + 128 * i;
+                for (int i = 0; i < (BN * 8) / C::kUnpack; ++i) {
+                    const int idx = ut + C::kUnpack * i;
                     const int n = idx >> 3, c = idx & 7;  // weight row, 16-element chunk of the 128-K slab
                     const uint32_t u = pk[idx];
                     const uint4 codes = make_uint4(u & 0x03030303u, (u >> 2) & 0x03030303u,
