@@ -46,8 +46,8 @@ L2_COPIES = 8
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the
 # kernel source it was taken on; stale once the source changes.
 NCU_TRAFFIC = {
-    # profiles/gemm_w8a8_4096.md: 33.6128 MB read + 2.8987 MB written
-    ("gemm_w8a8_4096", "2e3763eb04762ca5"): 36511488,
+    # profiles/gemm_w8a8_4096.md: 33.608192 MB read + 2.481920 MB written
+    ("gemm_w8a8_4096", "71341f98e9f8e223"): 36090112,
 }
 
 
@@ -257,13 +257,18 @@ def headline(args, dist, pk):
     st, detail = bq.bq_device_status()
     if st != bq.BQ_OK:
         raise RuntimeError(f"device status {detail:#x} after the timed region")
-    peak_int8 = 2.0 * pk["bf16_tflops"]  # int8 dense = 2x bf16 dense (nominal 4.5 vs 2.25 PF)
+    # int8 dense = 2x bf16 dense (nominal 4.5 vs 2.25 PF); a timed region of more than 0.2 s
+    # runs under the power cap, which the sustained bf16 figure describes
+    sustained = ms_total >= 200.0
+    bf16_peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    peak_int8 = 2.0 * bf16_peak
     src = source_hash("gemm_tc.cu", "bq_common.cuh")
     traffic = NCU_TRAFFIC.get(("gemm_w8a8_4096", src))
     roof = {"bound": "tensor", "achieved": round(tops_rank, 2), "peak": round(peak_int8, 1), "unit": "TFLOP/s",
             "frac": round(tops_rank / peak_int8, 4), "traffic": traffic,
             "kernel": "gemm_tc_kernel<W8A8, K-major B, bf16 out>",
-            "peak_note": f"{pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (nominal int8/bf16 ratio); "
+            "peak_note": f"{pk['source']} bf16 {'sustained' if sustained else 'burst'} {bf16_peak} TFLOP/s x 2 "
+                         f"(nominal int8/bf16 ratio; timed region {ms_total:.0f} ms); "
                          "int8 ops counted like flops, 2 per multiply-add",
             "algorithmic_bytes_per_launch": 2 * 4096 * 4096 + 4096 * 4096 * 2 + 2 * 4096 * 4}
     # end to end through the public API with host buffers
