@@ -21,6 +21,7 @@
 // 0,2,4,6 and ((word >> 4) & 0x0f0f0f0f) those of 1,3,5,7; the planes are
 // stored in that interleaved order so each matches one dp4a.
 #include <cuda_fp16.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 
@@ -277,163 +278,173 @@ cudaError_t launch_all(const uint32_t *qweight, const uint16_t *scales, const ui
 
 
 // ---------------------------------------------------------------------------
-// One-token decode kernel on the mma.sync tensor path: a single launch that
-// splits x into 24-bit planes in shared memory (every CTA, for all of K) and
-// streams the CTA's packed weight rows into a ring of 16-row stages.  One
-// extra warp only issues those copies (16-byte cp.async through the load /
-// store path, measured faster per SM than bulk copies for this stream), and
-// refills a slot as soon as the 16 computing warps have released it (full /
-// empty mbarriers per slot), so the HBM stream keeps going while the other
-// warps split x and compute.
+// One-token decode kernel on the mma.sync tensor path: a single launch.  One
+// CTA per SM takes a range of 8-row boxes of the packed weights; one thread of
+// a producer warp streams them with TMA into a ring of box slots (a 3-D tensor
+// view of the rows, {128 bytes, 8 rows, K/256 column pairs}, 128-byte
+// swizzle: one copy moves 8 x K/2 bytes), and 16 computing warps consume them
+// while the next boxes are in flight.  After the dependency wait the
+// computing warps also split x into 24-bit planes (each warp keeps the plane
+// fragments of its own spans in registers), fold scale and activation scale
+// into one factor per (row, group) and sum each row's zero-point terms once.
 //
 // The planes use signed base-256 digits, X = 65536 P0 + 256 P1 + P2 with
 // P0, P1, P2 in [-128, 127] (|X| <= 8355711), so all three are s8 columns of
 // one B operand: one m16n8k32 (u8 weights x s8 planes) gives D0, D1 and D2 of
 // 16 rows in columns 0, 1, 2.
 //
-// A stage holds 16 rows at a pitch of K/2 + 64 bytes (the extra 64 bytes put
-// rows g and g + 1 in different bank groups).  Warp w takes the 128-weight
-// spans sp = w + 16 c (c < K / 2048) of every stage (one group each when
-// gs % 128 == 0).  Lane (g, t) reads words 4t .. 4t+3 of the span for rows g
-// and g + 8.  MMA pair e takes words 2e and 2e+1: the low nibbles
-// (word & 0x0f0f0f0f) as one A operand and the high nibbles masked in place
-// (word & 0xf0f0f0f0 = 16 q) as another, into two accumulators combined as
-// C_lo + C_hi / 16 (exact).  The k-slots of lane t map to the elements of words
-// 4t + 2e and 4t + 2e + 1, whose plane bytes (stored in the order 0,2,4,6,1,3,5,7
-// within each 8) are one 16-byte load: .x / .z feed the low-nibble MMA, .y / .w
-// the high-nibble one.
+// Work unit = (two boxes = 16 rows, one 128-weight span).  Warp w takes the
+// spans sp = w + 16 c (c < K / 2048).  MMA row g (0..7) is row sigma(g) of
+// the first box and MMA row g + 8 row sigma(g) of the second, with
+// sigma(g) = (g >> 1) | 4 (g & 1): the lanes that share a shared-memory phase
+// then read rows whose swizzle differs in bit 2, i.e. opposite halves of the
+// 128-byte line, so the fragment loads are free of bank conflicts.  Lane
+// (g, t) reads words 4t .. 4t+3 of the span for both of its rows.  MMA pair e
+// takes words 2e and 2e+1: the low nibbles (word & 0x0f0f0f0f) as one A
+// operand and the high nibbles masked in place (word & 0xf0f0f0f0 = 16 q) as
+// another, into two accumulators combined as C_lo + C_hi / 16 (exact).  The
+// k-slots of lane t map to the elements of words 4t + 2e and 4t + 2e + 1,
+// whose plane bytes (stored in the order 0,2,4,6,1,3,5,7 within each 8) are
+// one 16-byte load: .x / .z feed the low-nibble MMA, .y / .w the high one.
+//
+//   out[n] = bias[n] + sum_g s[n,g] sx[g] T[n,g] - sum_g s[n,g] sx[g] z[n,g] sumX[g]
+//
+// with T[n,g] = sum_{k in g} q[n,k] X[k] = 65536 D0 + 256 D1 + D2.
 // ---------------------------------------------------------------------------
-constexpr int kW4Threads = 512;                 // computing threads
+constexpr int kW4Threads = 512;  // computing threads
 constexpr int kW4Warps = kW4Threads / 32;
-constexpr int kW4Streamers = 8;                  // warps that only stream the weights
-constexpr int kW4Block = kW4Threads + 32 * kW4Streamers;
+constexpr int kW4Block = kW4Threads + 32;  // + the producer warp
 constexpr int kW4MaxRows = 128;
-constexpr int kW4MaxStages = 8;
+constexpr int kW4MaxSlots = 12;
+constexpr int kW4MinSlots = 4;
 constexpr int kW4XMax = 8355711;  // 127 * (65536 + 256 + 1)
 
 struct W4DecodeArgs {
     const float *x;
-    const uint32_t *qweight;
     const uint16_t *scales;
     const uint32_t *qzeros;
     const float *bias;
     float *out;
-    int N, K, gs, nstg, rows_cap;
+    int N, K, gs, nslots, rows_cap, nbox;  // nbox: 8-row boxes of the whole matrix
     uint32_t *status;
 };
 
 __device__ __forceinline__ int digit_s8(int v) { return ((v + 128) & 255) - 128; }
 
-// Shared-memory layout of the kernel (host and device).
+// float(v) for |v| < 2^22 on the FMA pipe: v added to the mantissa of 1.5 * 2^23
+// gives 1.5 * 2^23 + v exactly, then the offset is subtracted (both exact).
+// One 16-row x 128-weight inner product stays below 15 * 128 * 128 < 2^18.
+__device__ __forceinline__ float exact_float(int v) { return __int_as_float(0x4B400000 + v) - 12582912.0f; }
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory layout of the kernel (host and device), from a 1024-byte
+// aligned base: the ring first (one box per slot, K/2 bytes per row).  The
+// per-(row, group) factors are stored group-major with an odd row stride rs,
+// so the lanes of one row block (consecutive rows) and the lanes of one row
+// (consecutive groups) both hit distinct banks.
 struct W4Layout {
-    int G, zrow, pitch;
-    uint32_t off_sx, off_sumx, off_part, off_tab, off_zero, off_bars, off_ring, total;
+    int G, zrow, rs;
+    uint32_t slot, off_planes, off_sx, off_sumx, off_part, off_tab, off_zero, off_bars, total;
     __host__ __device__ static uint32_t a16(uint32_t v) { return (v + 15u) & ~15u; }
-    __host__ __device__ W4Layout(int K, int gs, int nstg, int rows_cap) {
+    __host__ __device__ W4Layout(int K, int gs, int nslots, int rows_cap) {
         G = K / gs;
         zrow = (G + 7) / 8;
-        pitch = K / 2 + 64;
-        off_sx = a16(3u * K);
+        rs = rows_cap | 1;
+        slot = 8u * static_cast<uint32_t>(K / 2);
+        off_planes = slot * static_cast<uint32_t>(nslots);
+        off_sx = a16(off_planes + 3u * K);
         off_sumx = off_sx + 4u * G;
         off_part = a16(off_sumx + 4u * G);
         off_tab = a16(off_part + 4u * rows_cap * kW4Warps);
-        off_zero = a16(off_tab + 8u * rows_cap * G);
-        off_bars = a16(off_zero + 4u * rows_cap * zrow);
-        off_ring = (off_bars + 16u * kW4MaxStages + 127u) & ~127u;
-        total = off_ring + static_cast<uint32_t>(nstg) * 16u * pitch;
+        off_zero = a16(off_tab + 8u * rs * G);
+        off_bars = (off_zero + 4u * rows_cap * zrow + 7u) & ~7u;
+        total = off_bars + 16u * kW4MaxSlots + 1024u;  // + alignment slack of the base
     }
 };
 
-template <int SPW>  // spans per warp and stage: K / 2048
-__global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const W4DecodeArgs p) {
-    extern __shared__ __align__(128) uint8_t smem[];
+template <int SPW>  // spans per warp: K / 2048
+__global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_constant__ CUtensorMap wmap,
+                                                                const W4DecodeArgs p) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     __shared__ int s_abort;
-    const int K = p.K, gs = p.gs, nstg = p.nstg;
-    const W4Layout L(K, gs, nstg, p.rows_cap);
-    const int G = L.G, zrow = L.zrow, pitch = L.pitch;
-    int8_t *planes = reinterpret_cast<int8_t *>(smem);                  // [3][K], order 0,2,4,6,1,3,5,7
-    float *s_sx = reinterpret_cast<float *>(smem + L.off_sx);           // [G]
-    int *s_sumx = reinterpret_cast<int *>(smem + L.off_sumx);           // [G]
-    float *s_part = reinterpret_cast<float *>(smem + L.off_part);       // [rows][kW4Warps]
-    float2 *s_tab = reinterpret_cast<float2 *>(smem + L.off_tab);       // [rows][G]: s sx, s sx z sumX
-    uint32_t *s_zero = reinterpret_cast<uint32_t *>(smem + L.off_zero);    // [rows][zrow]
-    // full[s] at bars + 8 s (one arrival + the copy bytes), empty[s] at bars + 8 (kW4MaxStages + s)
-    const uint32_t bars = smem_u32(smem + L.off_bars), ring = smem_u32(smem + L.off_ring);
-    const uint32_t ebars = bars + 8u * kW4MaxStages;
+    const int K = p.K, gs = p.gs, NS = p.nslots;
+    const W4Layout L(K, gs, NS, p.rows_cap);
+    const int G = L.G, zrow = L.zrow, rs = L.rs;
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t ring = smem_u32(smem);
+    int8_t *planes = reinterpret_cast<int8_t *>(smem + L.off_planes);    // [3][K], order 0,2,4,6,1,3,5,7
+    float *s_sx = reinterpret_cast<float *>(smem + L.off_sx);             // [G]
+    float *s_sumx = reinterpret_cast<float *>(smem + L.off_sumx);         // [G]: sum of X
+    float *s_part = reinterpret_cast<float *>(smem + L.off_part);         // [kW4Warps][rows_cap]
+    float2 *s_tab = reinterpret_cast<float2 *>(smem + L.off_tab);         // [G][rs]: s sx, s sx z sumX
+    uint32_t *s_zero = reinterpret_cast<uint32_t *>(smem + L.off_zero);   // [rows][zrow]
+    const uint32_t fbar = smem_u32(smem + L.off_bars), ebar = fbar + 8u * kW4MaxSlots;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int gq = lane >> 2, tq = lane & 3;
+    // boxes [j0, j1) of the matrix; rows n0 .. n0 + rows - 1
     const int64_t b = blockIdx.x, Gc = gridDim.x;
-    const int n0 = static_cast<int>((b * p.N) / Gc), rows = static_cast<int>(((b + 1) * p.N) / Gc) - n0;
-    const int nst = (rows + 15) / 16;  // stages of this CTA
-    const uint32_t rowb = static_cast<uint32_t>(K / 2);  // packed bytes per row
-    const uint8_t *wsrc = reinterpret_cast<const uint8_t *>(p.qweight) + static_cast<int64_t>(n0) * rowb;
+    const int j0 = static_cast<int>((b * p.nbox) / Gc), j1 = static_cast<int>(((b + 1) * p.nbox) / Gc);
+    const int nb = j1 - j0, n0 = 8 * j0, rows = min(8 * j1, p.N) - n0;
 
     if (t == 0) {
-        for (int s = 0; s < nstg; ++s) {
-            mbar_init(bars + 8 * s, 32 * kW4Streamers);  // one arrival per streaming lane
-            mbar_init(ebars + 8 * s, kW4Warps);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(fbar + 8 * s, 1);
+            mbar_init(ebar + 8 * s, kW4Warps);
         }
         s_abort = 0;
         fence_mbarrier_init();
     }
+    if (warp == kW4Warps && lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(&wmap) : "memory");
     __syncthreads();
     pdl_launch_dependents();
     pdl_wait();
 
-    // the streaming warp copies stage s (rows 16 s .. 16 s + 15) into ring slot
-    // s % nstg, each lane then arriving on the slot's full barrier once its
-    // own copies have landed
-    const int ppr_shift = __ffs(static_cast<int>(rowb / 16)) - 1;  // 16-byte pieces per row (a power of two)
-    const int sl = t - kW4Threads;  // lane among the streaming warps
-    auto issue = [&](int s) {
-        const int slot = s % nstg, r0 = 16 * s, nr = min(16, rows - r0);
-        const uint32_t dst = ring + static_cast<uint32_t>(slot) * 16u * pitch;
-        const int npc = nr << ppr_shift;
-        for (int i = sl; i < npc; i += 32 * kW4Streamers) {
-            const int j = i >> ppr_shift, c = i & ((1 << ppr_shift) - 1);
-            cp_async_16(dst + static_cast<uint32_t>(j) * pitch + 16u * c,
-                        wsrc + static_cast<int64_t>(r0 + j) * rowb + 16 * c, 16u);
-        }
-        cp_async_mbar_arrive_noinc(bars + 8 * slot);
-    };
-    if (warp >= kW4Warps) {  // the streaming warps
-        int s = 0;
-        for (; s < nst; ++s) {
-            const int slot = s % nstg;
-            if (s >= nstg) {  // the slot's previous stage must be released by every computing warp
-                bool ok = mbar_wait(ebars + 8 * slot, ((s / nstg) - 1) & 1, &s_abort, p.status, SITE_W4_STAGE);
-                if (!__all_sync(0xffffffffu, ok)) break;
+    if (warp == kW4Warps) {  // producer: box i of this CTA into slot i % NS
+        if (lane == 0) {
+            int i = 0;
+            for (; i < nb; ++i) {
+                const int slot = i % NS;
+                if (i >= NS && !mbar_wait(ebar + 8 * slot, ((i / NS) - 1) & 1, &s_abort, p.status, SITE_W4_STAGE))
+                    break;
+                mbar_arrive_expect_tx(fbar + 8 * slot, L.slot);
+                tma_load_3d(ring + static_cast<uint32_t>(slot) * L.slot, &wmap, 0, n0 + 8 * i, 0, fbar + 8 * slot);
             }
-            issue(s);
+            // the copies in flight land before the CTA exits, whatever happened
+            for (int k = max(0, i - NS); k < i; ++k)
+                mbar_wait_timed(fbar + 8 * (k % NS), (k / NS) & 1, p.status, SITE_W4_DRAIN);
         }
-        cp_async_wait_all();  // (the copies land before the warp exits, whatever happened)
         return;
     }
 
-    // activations, scales and zero-points (the weight stream is already running)
-    const int EPT = K / kW4Threads, nv = EPT / 4, TPG = gs / EPT;
-    float4 xv[4];
+    // activations, zero-points and scales (the weight stream is already running)
+    const int ns = rows * G, nz = rows * zrow;
+    const int sgo = n0 * G, zgo = n0 * zrow;
+    float4 xv[SPW];  // EPT = K / 512 = 4 SPW elements of x per thread
     {
-        const float4 *x4 = reinterpret_cast<const float4 *>(p.x) + static_cast<int64_t>(t) * nv;
+        const float4 *x4 = reinterpret_cast<const float4 *>(p.x) + static_cast<int64_t>(t) * SPW;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) xv[j] = j < nv ? __ldg(x4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < SPW; ++j) xv[j] = __ldg(x4 + j);
     }
-    const int ns = rows * G;
-    uint16_t sv[16];
-    {
-        const int nz = rows * zrow;
-        const uint16_t *sg = p.scales + static_cast<int64_t>(n0) * G;
-        const uint32_t *zg = p.qzeros + static_cast<int64_t>(n0) * zrow;
-        uint32_t zv[2];
+    uint16_t sv[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int i = t + j * kW4Threads;
-            sv[j] = i < ns ? __ldg(sg + i) : static_cast<uint16_t>(0);
-        }
+    for (int j = 0; j < 8; ++j) {
+        const int i = t + j * kW4Threads;
+        sv[j] = i < ns ? __ldg(p.scales + sgo + i) : static_cast<uint16_t>(0);
+    }
+    {
+        uint32_t zv[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int i = t + j * kW4Threads;
-            zv[j] = i < nz ? __ldg(zg + i) : 0u;
+            zv[j] = i < nz ? __ldg(p.qzeros + zgo + i) : 0u;
         }
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -442,83 +453,138 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const W4DecodeAr
         }
     }
 
-    // activation planes: thread t splits elements EPT t .. EPT t + EPT - 1
-    // (EPT = K / 512; a group spans TPG = gs / EPT threads).  X = rne(x / sx)
-    // with sx = max|x| / 8355711 per group, x / sx taken as x * (1 / sx): at
-    // most one more unit of error than the exact quotient.
+    // activation planes: thread t splits elements EPT t .. EPT t + EPT - 1 (a
+    // group spans TPG = gs / EPT threads).  X = rne(x / sx) with
+    // sx = max|x| / 8355711 per group, x / sx taken as x * (1 / sx): at most
+    // one more unit of error than the exact quotient.
     {
+        constexpr int EPT = 4 * SPW;
+        const int TPG = gs / EPT;
         float amax = 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < SPW; ++j)
             amax = fmaxf(amax, fmaxf(fmaxf(fabsf(xv[j].x), fabsf(xv[j].y)), fmaxf(fabsf(xv[j].z), fabsf(xv[j].w))));
         for (int o = TPG / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         const float sx = __fdiv_rn(amax, static_cast<float>(kW4XMax));
         const float inv = amax > 0.f ? __fdiv_rn(1.0f, sx) : 0.f;
         int sum = 0;
+        // byte e of this thread's run lands at position perm8(e) of its 8-chunk:
+        // word 2 (e / 8) + (e & 1), byte (e & 7) / 2
+        constexpr int NW = EPT / 4 < 2 ? 2 : EPT / 4;  // (half a chunk still touches both of its words)
+        uint32_t pw[3][NW];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (j < nv) {
-                const float e4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+        for (int w = 0; w < NW; ++w) pw[0][w] = pw[1][w] = pw[2][w] = 0u;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    int X = __float2int_rn(__fmul_rn(e4[u], inv));
-                    X = max(-kW4XMax, min(kW4XMax, X));
-                    sum += X;
-                    const int P2 = digit_s8(X), X1 = (X - P2) >> 8;
-                    const int P1 = digit_s8(X1), P0 = (X1 - P1) >> 8;
-                    const int k = EPT * t + 4 * j + u, jj = k & 7;
-                    const int pos = (k & ~7) + ((jj & 1) ? 4 + (jj >> 1) : (jj >> 1));
-                    planes[pos] = static_cast<int8_t>(P0);
-                    planes[K + pos] = static_cast<int8_t>(P1);
-                    planes[2 * K + pos] = static_cast<int8_t>(P2);
-                }
+        for (int j = 0; j < SPW; ++j) {
+            const float e4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                int X = __float2int_rn(__fmul_rn(e4[u], inv));
+                X = max(-kW4XMax, min(kW4XMax, X));
+                sum += X;
+                const int P2 = digit_s8(X), X1 = (X - P2) >> 8;
+                const int P1 = digit_s8(X1), P0 = (X1 - P1) >> 8;
+                const int e = 4 * j + u, w = 2 * (e >> 3) + (e & 1), sh = 8 * ((e & 7) >> 1);
+                pw[0][w] |= (static_cast<uint32_t>(P0) & 255u) << sh;
+                pw[1][w] |= (static_cast<uint32_t>(P1) & 255u) << sh;
+                pw[2][w] |= (static_cast<uint32_t>(P2) & 255u) << sh;
+            }
+        }
+        if (EPT >= 8) {  // whole 8-chunks: two words per chunk and plane
+#pragma unroll
+            for (int q = 0; q < 3; ++q)
+#pragma unroll
+                for (int w = 0; w < EPT / 4; w += 2)
+                    *reinterpret_cast<uint2 *>(planes + q * K + EPT * t + 4 * w) = make_uint2(pw[q][w], pw[q][w + 1]);
+        } else {  // half a chunk: elements 0..3 or 4..7 of it, i.e. bytes 0,1 of both words or bytes 2,3
+            const int base = (EPT * t) & ~7, hb = ((EPT * t) & 7) ? 2 : 0;
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                planes[q * K + base + hb] = static_cast<int8_t>(pw[q][0] & 255u);
+                planes[q * K + base + hb + 1] = static_cast<int8_t>((pw[q][0] >> 8) & 255u);
+                planes[q * K + base + 4 + hb] = static_cast<int8_t>(pw[q][1] & 255u);
+                planes[q * K + base + 4 + hb + 1] = static_cast<int8_t>((pw[q][1] >> 8) & 255u);
             }
         }
         for (int o = TPG / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
         if (t % TPG == 0) {
             s_sx[(EPT * t) / gs] = sx;
-            s_sumx[(EPT * t) / gs] = sum;
-        }
-    }
-    named_bar_sync(1, kW4Threads);
-    // per (row, group): s sx and s sx z sumX (G is a power of two)
-    const int g_shift = __ffs(G) - 1;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const int i = t + j * kW4Threads;
-        if (i < ns) {
-            const int r = i >> g_shift, grp = i & (G - 1);
-            const float fs = __fmul_rn(__half2float(__ushort_as_half(sv[j])), s_sx[grp]);
-            const float z = static_cast<float>((s_zero[r * zrow + grp / 8] >> (4 * (grp % 8))) & 15u);
-            s_tab[i] = make_float2(fs, __fmul_rn(__fmul_rn(fs, z), static_cast<float>(s_sumx[grp])));
+            s_sumx[(EPT * t) / gs] = static_cast<float>(sum);
         }
     }
     named_bar_sync(1, kW4Threads);
 
+    // per (row, group): s sx and s sx z sumX (G is a power of two)
+    const int g_shift = __ffs(G) - 1;
+    auto tab_items = [&](int base, const uint16_t(&v)[8]) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + t + j * kW4Threads;
+            if (i < ns) {
+                const int r = i >> g_shift, grp = i & (G - 1);
+                const float fs = __fmul_rn(__half2float(__ushort_as_half(v[j])), s_sx[grp]);
+                const float z = exact_float(static_cast<int>((s_zero[r * zrow + grp / 8] >> (4 * (grp % 8))) & 15u));
+                s_tab[grp * rs + r] = make_float2(fs, __fmul_rn(__fmul_rn(fs, z), s_sumx[grp]));
+            }
+        }
+    };
+    tab_items(0, sv);
+    for (int base = 8 * kW4Threads; base < ns; base += 8 * kW4Threads) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + t + j * kW4Threads;
+            sv[j] = i < ns ? __ldg(p.scales + sgo + i) : static_cast<uint16_t>(0);
+        }
+        tab_items(base, sv);
+    }
+    // this warp's plane fragments (the same for every row block)
+    uint4 bx[SPW][2];
+#pragma unroll
+    for (int c = 0; c < SPW; ++c) {
+        const int sp = warp + kW4Warps * c;
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+            bx[c][e] = gq < 3 ? *reinterpret_cast<const uint4 *>(planes + gq * K + 128 * sp + 32 * tq + 16 * e)
+                              : make_uint4(0u, 0u, 0u, 0u);
+    }
+    named_bar_sync(1, kW4Threads);
+
+    // C columns: lane t = 0 holds D0, D1 of MMA rows g and g + 8, lane t = 1
+    // holds D2 (column 2) of both.  Each accumulates its share of
+    // s sx T = s sx (65536 D0 + 256 D1) + s sx D2 (lane t = 0 also subtracts
+    // the zero-point term once per group); the two shares meet once per block.
     const int SPG = gs / 128, spg_shift = __ffs(SPG) - 1;  // spans per group (a power of two)
-    for (int s = 0; s < nst; ++s) {
-        const int slot = s % nstg;
-        bool ok = mbar_wait(bars + 8 * slot, (s / nstg) & 1, &s_abort, p.status, SITE_W4_STAGE);
+    const int sg = (gq >> 1) | ((gq & 1) << 2);             // sigma(g): row of the box
+    // byte offset of this lane's 16 bytes of span sp within a box: column pair
+    // sp / 2 (1 KB each), row sg (128 bytes), 16-byte chunk (4 (sp & 1) + t) ^ sg
+    auto frag_off = [&](int sp) -> uint32_t {
+        return static_cast<uint32_t>((sp >> 1) * 1024 + sg * 128 + ((((sp & 1) << 2) + tq) ^ sg) * 16);
+    };
+    const int nrb = (nb + 1) / 2;
+    int s0 = 0;        // slot of box 2 rb
+    uint32_t ph0 = 0;  // and the parity of its phase
+    for (int rb = 0; rb < nrb; ++rb) {
+        const bool has1 = 2 * rb + 1 < nb;
+        const int s1 = s0 + 1 == NS ? 0 : s0 + 1;
+        const uint32_t ph1 = s0 + 1 == NS ? ph0 ^ 1u : ph0;
+        bool ok = mbar_wait(fbar + 8 * s0, ph0, &s_abort, p.status, SITE_W4_STAGE);
+        if (has1) ok = ok && mbar_wait(fbar + 8 * s1, ph1, &s_abort, p.status, SITE_W4_STAGE);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
-            const uint32_t sbase = ring + static_cast<uint32_t>(slot) * 16u * pitch;
-            const int r0 = 16 * s + gq, r1 = r0 + 8;
-            float acc0 = 0.f;  // row g (lane t = 0) or g + 8 (lane t = 2)
+            const uint32_t b0 = ring + static_cast<uint32_t>(s0) * L.slot;
+            const uint32_t b1 = ring + static_cast<uint32_t>(s1) * L.slot;
+            const int r0 = 16 * rb + sg, r1 = r0 + 8;  // this lane's rows (MMA rows g, g + 8)
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
             for (int c = 0; c < SPW; ++c) {
                 const int sp = warp + kW4Warps * c;
-                uint4 wa, wb;
-                const uint32_t wad = sbase + static_cast<uint32_t>(gq) * pitch + 64u * sp + 16u * tq;
+                const uint32_t off = frag_off(sp);
+                uint4 wa, wb = make_uint4(0u, 0u, 0u, 0u);
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w) : "r"(wad));
-                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(wad + 8u * pitch));
-                uint4 bx[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-                if (gq < 3) {
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-                        bx[e] = *reinterpret_cast<const uint4 *>(planes + gq * K + 128 * sp + 32 * tq + 16 * e);
-                }
+                             : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w) : "r"(b0 + off));
+                if (has1)
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(b1 + off));
                 int clo[4] = {0, 0, 0, 0}, chi[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
@@ -526,71 +592,102 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const W4DecodeAr
                     const uint32_t a1 = e ? wb.z : wb.x, a3 = e ? wb.w : wb.y;
                     const uint32_t lo[4] = {a0 & 0x0f0f0f0fu, a1 & 0x0f0f0f0fu, a2 & 0x0f0f0f0fu, a3 & 0x0f0f0f0fu};
                     const uint32_t hi[4] = {a0 & 0xf0f0f0f0u, a1 & 0xf0f0f0f0u, a2 & 0xf0f0f0f0u, a3 & 0xf0f0f0f0u};
-                    mma_u8s8_16832(clo, lo, bx[e].x, bx[e].z);
-                    mma_u8s8_16832(chi, hi, bx[e].y, bx[e].w);
+                    mma_u8s8_16832(clo, lo, bx[c][e].x, bx[c][e].z);
+                    mma_u8s8_16832(chi, hi, bx[c][e].y, bx[c][e].w);
                 }
-                int d[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) d[q] = clo[q] + (chi[q] >> 4);
-                // lane t = 0 finishes row g, lane t = 2 row g + 8 (D0, D1 in columns 0, 1 of
-                // lane t = 0, D2 in column 2 of lane t = 1)
-                const int e0 = __shfl_down_sync(0xffffffffu, d[0], 1);
-                const int e1 = __shfl_up_sync(0xffffffffu, d[2], 2), e2 = __shfl_up_sync(0xffffffffu, d[3], 2);
-                const int e3 = __shfl_up_sync(0xffffffffu, d[2], 1);
-                if ((tq & 1) == 0) {
-                    const int row = tq == 0 ? r0 : r1;
-                    const int D0 = tq == 0 ? d[0] : e1, D1 = tq == 0 ? d[1] : e2, D2 = tq == 0 ? e0 : e3;
-                    if (row < rows) {
-                        const float T = fmaf(65536.0f, static_cast<float>(D0),
-                                             fmaf(256.0f, static_cast<float>(D1), static_cast<float>(D2)));
-                        const float2 f = s_tab[row * G + (sp >> spg_shift)];
-                        acc0 += fmaf(f.x, T, (sp & (SPG - 1)) == 0 ? -f.y : 0.0f);
+                if (tq < 2) {
+                    const int grp = sp >> spg_shift;
+                    const float2 f0 = r0 < rows ? s_tab[grp * rs + r0] : make_float2(0.f, 0.f);
+                    const float2 f1 = r1 < rows ? s_tab[grp * rs + r1] : make_float2(0.f, 0.f);
+                    const float z = (sp & (SPG - 1)) == 0 ? 1.0f : 0.0f;  // zero-point term once per group
+                    const float d0 = exact_float(clo[0] + (chi[0] >> 4));
+                    const float d1 = exact_float(clo[1] + (chi[1] >> 4));
+                    const float d2 = exact_float(clo[2] + (chi[2] >> 4));
+                    const float d3 = exact_float(clo[3] + (chi[3] >> 4));
+                    if (tq == 0) {  // 65536 D0 + 256 D1 of rows g, g + 8, minus the zero-point terms
+                        acc0 = fmaf(f0.x, fmaf(65536.0f, d0, 256.0f * d1), fmaf(-z, f0.y, acc0));
+                        acc1 = fmaf(f1.x, fmaf(65536.0f, d2, 256.0f * d3), fmaf(-z, f1.y, acc1));
+                    } else {  // D2 of rows g, g + 8
+                        acc0 = fmaf(f0.x, d0, acc0);
+                        acc1 = fmaf(f1.x, d2, acc1);
                     }
                 }
             }
-            if ((tq & 1) == 0) {
-                const int row = tq == 0 ? r0 : r1;
-                if (row < rows) s_part[row * kW4Warps + warp] = acc0;
+            acc0 += __shfl_down_sync(0xffffffffu, acc0, 1);
+            acc1 += __shfl_down_sync(0xffffffffu, acc1, 1);
+            if (tq == 0) {
+                if (r0 < rows) s_part[warp * p.rows_cap + r0] = acc0;
+                if (r1 < rows) s_part[warp * p.rows_cap + r1] = acc1;
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(ebars + 8 * slot);  // this warp is done with the slot
+        if (lane == 0) {  // this warp is done with both slots
+            mbar_arrive(ebar + 8 * s0);
+            if (has1) mbar_arrive(ebar + 8 * s1);
+        }
+        s0 = s1 + 1 == NS ? 0 : s1 + 1;
+        ph0 = s1 + 1 == NS ? ph1 ^ 1u : ph1;
     }
     named_bar_sync(1, kW4Threads);
     for (int r = t; r < rows; r += kW4Threads) {
         float acc = 0.f;
 #pragma unroll
-        for (int w = 0; w < kW4Warps; ++w) acc += s_part[r * kW4Warps + w];
+        for (int w = 0; w < kW4Warps; ++w) acc += s_part[w * p.rows_cap + r];
         p.out[n0 + r] = (p.bias ? __ldg(p.bias + n0 + r) : 0.0f) + acc;
     }
 }
 
-int w4_rows_cap(int64_t N, const DevInfo &dev) {
-    const int64_t Gc = std::min<int64_t>(N, dev.num_sms);
-    return static_cast<int>((N + Gc - 1) / Gc);
+PFN_cuTensorMapEncodeTiled_v12000 w4_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
 }
 
-int w4_decode_stages(int K, int gs, int rows_cap, const DevInfo &dev) {
+int w4_boxes(int64_t N) { return static_cast<int>((N + 7) / 8); }
+
+int w4_rows_cap(int64_t N, const DevInfo &dev) {
+    const int64_t nb = w4_boxes(N), Gc = std::min<int64_t>(nb, dev.num_sms);
+    return static_cast<int>(8 * ((nb + Gc - 1) / Gc));
+}
+
+int w4_decode_slots(int K, int gs, int rows_cap, const DevInfo &dev) {
     const W4Layout L0(K, gs, 0, rows_cap);
-    const int64_t room = static_cast<int64_t>(dev.max_smem_optin) - L0.total;
-    return static_cast<int>(std::min<int64_t>(kW4MaxStages, room / (16 * (K / 2 + 64))));
+    const int64_t room = static_cast<int64_t>(dev.max_smem_optin) - 1024 - L0.total;  // (static shared memory)
+    const int64_t n = std::min<int64_t>(kW4MaxSlots, room / L0.slot);
+    return n < kW4MinSlots ? 0 : static_cast<int>(n);
 }
 
 bool w4_decode_supported(int64_t M, int64_t N, int64_t K, int64_t gs, const DevInfo &dev) {
     if (M != 1 || K % 2048 != 0 || K > 8192 || gs % 128 != 0 || K % gs != 0 || (gs & (gs - 1)) != 0) return false;
-    if (gs / (K / kW4Threads) > 32) return false;  // a group spans at most one warp in the split
-    const int64_t Gc = std::min<int64_t>(N, dev.num_sms), rb = (N + Gc - 1) / Gc, G = K / gs;
-    if (rb > kW4MaxRows) return false;
-    if (rb * G > 16 * kW4Threads || rb * ((G + 7) / 8) > 2 * kW4Threads) return false;  // scale / zero registers
-    return w4_decode_stages(static_cast<int>(K), static_cast<int>(gs), static_cast<int>(rb), dev) >= 2;
+    if (gs > K / 16) return false;  // a group spans at most one warp in the split of x
+    if (w4_rows_cap(N, dev) > kW4MaxRows || w4_encode_fn() == nullptr) return false;
+    return w4_decode_slots(static_cast<int>(K), static_cast<int>(gs), w4_rows_cap(N, dev), dev) > 0;
 }
 
 cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight, const uint16_t *scales,
                              const uint32_t *qzeros, const float *bias, int64_t N, int64_t gs, float *out,
                              cudaStream_t s, const DevInfo &dev) {
+    // the packed rows as {128-byte column pairs of 16 u64, rows, column pairs}
+    CUtensorMap map;
+    {
+        const cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K / 256)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
+        const cuuint32_t box[3] = {16, 8, static_cast<cuuint32_t>(K / 256)};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        const CUresult r = w4_encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<uint32_t *>(qweight),
+                                          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     W4DecodeArgs a;
     a.x = x;
-    a.qweight = qweight;
     a.scales = scales;
     a.qzeros = qzeros;
     a.bias = bias;
@@ -599,9 +696,10 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
     a.K = static_cast<int>(K);
     a.gs = static_cast<int>(gs);
     a.rows_cap = w4_rows_cap(N, dev);
-    a.nstg = w4_decode_stages(a.K, a.gs, a.rows_cap, dev);
+    a.nslots = w4_decode_slots(a.K, a.gs, a.rows_cap, dev);
+    a.nbox = w4_boxes(N);
     a.status = dev.status;
-    const int smem = static_cast<int>(W4Layout(a.K, a.gs, a.nstg, a.rows_cap).total);
+    const int smem = static_cast<int>(W4Layout(a.K, a.gs, a.nslots, a.rows_cap).total);
     auto kern = K == 2048 ? w4_decode_kernel<1> : K == 4096 ? w4_decode_kernel<2> : w4_decode_kernel<4>;
     static int attr_smem[3][64] = {};
     int &done = attr_smem[K == 2048 ? 0 : K == 4096 ? 1 : 2][dev.device];
@@ -611,7 +709,7 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
         done = smem;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(N, dev.num_sms)));
+    cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(a.nbox, dev.num_sms)));
     cfg.blockDim = dim3(kW4Block);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = s;
@@ -620,7 +718,7 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    return cudaLaunchKernelEx(&cfg, kern, map, a);
 }
 
 }  // namespace

@@ -360,12 +360,15 @@ def test_linear_w4_ragged(M, N, K, gs):
     _w4_check(M, N, K, gs, seed=(111, M, N, K))
 
 
-# one token: the single-launch mma.sync streaming kernel (K = 2048 .. 8192,
-# groups of 128 / 256, more rows than SMs and fewer, with and without bias),
-# and shapes it leaves to the general path (groups of 32 / 64, K = 1024)
+# one token: the single-launch TMA-fed mma.sync kernel (K = 2048 .. 8192,
+# groups of 128 / 256, more 8-row boxes than SMs and fewer, row counts that
+# end inside a box, with and without bias), and shapes it leaves to the
+# general path (groups of 32 / 64, K = 1024)
 @pytest.mark.parametrize("N,K,gs,bias", [(300, 2048, 64, True), (5000, 8192, 256, True), (100, 1024, 32, False),
                                          (900, 2048, 128, True), (3000, 8192, 128, False),
-                                         (16000, 4096, 128, True), (7, 4096, 128, False)])
+                                         (16000, 4096, 128, True), (7, 4096, 128, False),
+                                         (14336, 4096, 128, True), (1001, 4096, 256, False),
+                                         (2301, 2048, 128, False)])
 def test_linear_w4_one_token(N, K, gs, bias):
     g = synth.rng((113, N, K, gs))
     q = synth.nibbles(g, (N, K))
