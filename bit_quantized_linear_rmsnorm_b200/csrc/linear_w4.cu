@@ -336,6 +336,11 @@ __device__ __forceinline__ int digit_s8(int v) { return ((v + 128) & 255) - 128;
 // One 16-row x 128-weight inner product stays below 15 * 128 * 128 < 2^18.
 __device__ __forceinline__ float exact_float(int v) { return __int_as_float(0x4B400000 + v) - 12582912.0f; }
 
+// Arrival on named barrier `id` without waiting (the producer waits on it).
+__device__ __forceinline__ void w4_bar_arrive(uint32_t id, uint32_t threads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
                                             uint32_t bar) {
     asm volatile(
@@ -357,7 +362,7 @@ struct W4Layout {
     __host__ __device__ W4Layout(int K, int gs, int nslots, int rows_cap) {
         G = K / gs;
         zrow = (G + 7) / 8;
-        rs = rows_cap | 1;
+        rs = (rows_cap + 8) | 1;  // (a row block may reach 8 rows past the last box)
         slot = 8u * static_cast<uint32_t>(K / 2);
         off_planes = slot * static_cast<uint32_t>(nslots);
         off_sx = a16(off_planes + 3u * K);
@@ -408,6 +413,9 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
     pdl_wait();
 
     if (warp == kW4Warps) {  // producer: box i of this CTA into slot i % NS
+        // the small loads of x, scales and zero-points enter the memory system
+        // ahead of the weight stream (they head the computing warps' critical path)
+        named_bar_sync(2, kW4Block);
         if (lane == 0) {
             int i = 0;
             for (; i < nb; ++i) {
@@ -446,6 +454,7 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
             const int i = t + j * kW4Threads;
             zv[j] = i < nz ? __ldg(p.qzeros + zgo + i) : 0u;
         }
+        w4_bar_arrive(2, kW4Block);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int i = t + j * kW4Threads;
@@ -579,12 +588,13 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
             for (int c = 0; c < SPW; ++c) {
                 const int sp = warp + kW4Warps * c;
                 const uint32_t off = frag_off(sp);
-                uint4 wa, wb = make_uint4(0u, 0u, 0u, 0u);
+                // (without a second box, the other slot's stale bytes only reach rows
+                // past the end, whose sums are never stored)
+                uint4 wa, wb;
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w) : "r"(b0 + off));
-                if (has1)
-                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(b1 + off));
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(b1 + off));
                 int clo[4] = {0, 0, 0, 0}, chi[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
@@ -595,23 +605,18 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
                     mma_u8s8_16832(clo, lo, bx[c][e].x, bx[c][e].z);
                     mma_u8s8_16832(chi, hi, bx[c][e].y, bx[c][e].w);
                 }
-                if (tq < 2) {
-                    const int grp = sp >> spg_shift;
-                    const float2 f0 = r0 < rows ? s_tab[grp * rs + r0] : make_float2(0.f, 0.f);
-                    const float2 f1 = r1 < rows ? s_tab[grp * rs + r1] : make_float2(0.f, 0.f);
-                    const float z = (sp & (SPG - 1)) == 0 ? 1.0f : 0.0f;  // zero-point term once per group
-                    const float d0 = exact_float(clo[0] + (chi[0] >> 4));
-                    const float d1 = exact_float(clo[1] + (chi[1] >> 4));
-                    const float d2 = exact_float(clo[2] + (chi[2] >> 4));
-                    const float d3 = exact_float(clo[3] + (chi[3] >> 4));
-                    if (tq == 0) {  // 65536 D0 + 256 D1 of rows g, g + 8, minus the zero-point terms
-                        acc0 = fmaf(f0.x, fmaf(65536.0f, d0, 256.0f * d1), fmaf(-z, f0.y, acc0));
-                        acc1 = fmaf(f1.x, fmaf(65536.0f, d2, 256.0f * d3), fmaf(-z, f1.y, acc1));
-                    } else {  // D2 of rows g, g + 8
-                        acc0 = fmaf(f0.x, d0, acc0);
-                        acc1 = fmaf(f1.x, d2, acc1);
-                    }
-                }
+                // every lane takes the same steps (no divergence): lane t = 0 adds
+                // 65536 D0 + 256 D1 and subtracts the zero-point term once per group,
+                // lane t = 1 adds D2; lanes t = 2, 3 hold zero columns
+                const int grp = sp >> spg_shift;
+                const float2 f0 = s_tab[grp * rs + r0], f1 = s_tab[grp * rs + r1];
+                const float zt = tq == 0 && (sp & (SPG - 1)) == 0 ? 1.0f : 0.0f;
+                const float d0 = exact_float(clo[0] + (chi[0] >> 4)), d1 = exact_float(clo[1] + (chi[1] >> 4));
+                const float d2 = exact_float(clo[2] + (chi[2] >> 4)), d3 = exact_float(clo[3] + (chi[3] >> 4));
+                const float u0 = tq == 0 ? fmaf(65536.0f, d0, 256.0f * d1) : d0;
+                const float u1 = tq == 0 ? fmaf(65536.0f, d2, 256.0f * d3) : d2;
+                acc0 = fmaf(f0.x, u0, fmaf(-zt, f0.y, acc0));
+                acc1 = fmaf(f1.x, u1, fmaf(-zt, f1.y, acc1));
             }
             acc0 += __shfl_down_sync(0xffffffffu, acc0, 1);
             acc1 += __shfl_down_sync(0xffffffffu, acc1, 1);

@@ -66,10 +66,17 @@ struct TcLayout {
     // a_full[S], a_empty[S], t_full[B], t_empty[B], drain
     static constexpr uint32_t NBAR = 2 * kTcStages + 2 * kTcBufs + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
-    static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;    // + alignment slack
+    static constexpr uint32_t OFF_GT = OFF_MISC + 16;         // per K block: group index, zero-point shift
+    static constexpr uint32_t SMEM = OFF_GT + 8 * kTcBlocks + 1024;  // + alignment slack
 };
 
 __device__ __forceinline__ int tc_digit(int v) { return ((v + 128) & 255) - 128; }
+
+// float(v) for |v| < 2^22 on the FMA pipe (v added to the mantissa of
+// 1.5 * 2^23, then the offset subtracted; both steps exact).  A 128-deep
+// inner product of codes minus zero-point (|.| <= 15) and plane digits
+// (|.| <= 128) stays below 2^18.
+__device__ __forceinline__ float tc_exact_float(int v) { return __int_as_float(0x4B400000 + v) - 12582912.0f; }
 
 // ---------------------------------------------------------------------------
 // 1. activation planes, one CTA per (token slot, K slice) (256 threads x 4 elements)
@@ -206,6 +213,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         uint32_t *zs = reinterpret_cast<uint32_t *>(smem + TcLayout::OFF_Z);
         const int zw = (kbase / p.gs) / 8;
         for (int r = threadIdx.x; r < rows; r += kTcThreads) zs[r] = __ldg(p.qzeros + static_cast<int64_t>(n0 + r) * zrow + zw);
+        int *gt = reinterpret_cast<int *>(smem + TcLayout::OFF_GT);  // (no division in the step loops)
+        if (threadIdx.x < kTcBlocks) {
+            const int grp = (kbase + kTcKB * static_cast<int>(threadIdx.x)) / p.gs;
+            gt[threadIdx.x] = grp;
+            gt[kTcBlocks + threadIdx.x] = 4 * (grp % 8);
+        }
     }
     cp_async_wait_all();
     fence_proxy_async_smem();
@@ -222,6 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         // thread's own ring slots, read back by the same thread).
         const int e = threadIdx.x, pc = e & 3, rr = e >> 2;
         const uint32_t *zs = reinterpret_cast<const uint32_t *>(smem + TcLayout::OFF_Z);
+        const int *zshift = reinterpret_cast<const int *>(smem + TcLayout::OFF_GT) + kTcBlocks;
         auto slot_addr = [&](int j, int half) {
             return sbase + TcLayout::OFF_P + static_cast<uint32_t>((((j % kTcRing) * 2 + half) * 256 + e) * 16);
         };
@@ -239,16 +253,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         };
 #pragma unroll
         for (int i = 0; i < kTcRing; ++i) issue(i);
-        // expand one row's piece: codes minus the zero-point as s8, two 16-byte chunks
+        // expand one row's piece: codes minus the zero-point as s8, two 16-byte
+        // chunks.  Per byte, q + (128 - z) lies in [113, 143] (no carry into the
+        // next byte), and flipping bit 7 leaves q - z in two's complement.
         auto expand = [&](uint8_t *row, int r_t, const uint4 &w, uint32_t zw) {
-            const uint32_t zrep = (zw & 15u) * 0x01010101u;
+            const uint32_t zoff = 0x80808080u - (zw & 15u) * 0x01010101u;
             const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
             uint32_t o[8];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {  // word k: codes 8 k .. 8 k + 7 of the piece
                 const uint32_t lo = wd[k] & 0x0f0f0f0fu, hi = (wd[k] >> 4) & 0x0f0f0f0fu;
-                o[2 * k] = __vsub4(__byte_perm(lo, hi, 0x5140), zrep);
-                o[2 * k + 1] = __vsub4(__byte_perm(lo, hi, 0x7362), zrep);
+                o[2 * k] = (__byte_perm(lo, hi, 0x5140) + zoff) ^ 0x80808080u;
+                o[2 * k + 1] = (__byte_perm(lo, hi, 0x7362) + zoff) ^ 0x80808080u;
             }
             *reinterpret_cast<uint4 *>(row + (((2 * pc) ^ (r_t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
             *reinterpret_cast<uint4 *>(row + (((2 * pc + 1) ^ (r_t & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
@@ -272,7 +288,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
                                  : "=r"(wa.x), "=r"(wa.y), "=r"(wa.z), "=r"(wa.w) : "r"(slot_addr(j, 0)));
                     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                                  : "=r"(wb.x), "=r"(wb.y), "=r"(wb.z), "=r"(wb.w) : "r"(slot_addr(j, 1)));
-                    const int zsh = 4 * (((kbase + g * kTcKB) / p.gs) % 8);
+                    const int zsh = zshift[g];
                     uint8_t *stage = smem + TcLayout::OFF_A + s * kTcABytes;
                     if (t * kTcRows + rr < rows) expand(stage + rr * 128, rr, wa, zs[t * kTcRows + rr] >> zsh);
                     if (t * kTcRows + rr + 64 < rows)
@@ -324,6 +340,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         const int q = warp & 3;          // TMEM lane quarter
         const int th = (warp - 8) >> 2;  // tokens 16 th .. 16 th + 15
         const int r_in = 32 * q + lane;
+        const int *grp_of = reinterpret_cast<const int *>(smem + TcLayout::OFF_GT);
+        // the scale of step j is loaded during step j - 1
+        auto scale_of = [&](int j) -> uint16_t {
+            const int t = j / kTcBlocks, g = j - t * kTcBlocks, r = t * kTcRows + r_in;
+            return j < nsteps && r < rows ? __ldg(p.scales + static_cast<int64_t>(n0 + r) * G + grp_of[g])
+                                          : static_cast<uint16_t>(0);
+        };
+        uint16_t sc_next = scale_of(0);
         float acc[16];
         for (int j = 0; j < nsteps; ++j) {
             const int t = j / kTcBlocks, g = j - t * kTcBlocks, b = j % kTcBufs;
@@ -333,9 +357,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[i] = 0.f;
             }
-            const int grp = (kbase + g * kTcKB) / p.gs;
-            const float sc =
-                valid ? __half2float(__ushort_as_half(__ldg(p.scales + static_cast<int64_t>(n0 + r) * G + grp))) : 0.f;
+            const float sc = __half2float(__ushort_as_half(sc_next));
+            sc_next = scale_of(j + 1);
             bool ok = true;
             if (lane == 0)
                 ok = mbar_wait_spin(t_full(b), static_cast<uint32_t>(j / kTcBufs) & 1u, abort_flag, p.status,
@@ -354,8 +377,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
             if (lane == 0) mbar_arrive(t_empty(b));
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int e = 256 * static_cast<int>(d1[i]) + static_cast<int>(d2[i]);  // |e| < 2^26
-                const float T = fmaf(65536.0f, static_cast<float>(static_cast<int>(d0[i])), static_cast<float>(e));
+                const float T = fmaf(65536.0f, tc_exact_float(static_cast<int>(d0[i])),
+                                     fmaf(256.0f, tc_exact_float(static_cast<int>(d1[i])),
+                                          tc_exact_float(static_cast<int>(d2[i]))));
                 acc[i] = fmaf(sc, T, acc[i]);
             }
             if (g == kTcBlocks - 1 && valid) {
