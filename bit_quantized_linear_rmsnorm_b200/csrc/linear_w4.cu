@@ -284,12 +284,12 @@ cudaError_t launch_all(const uint32_t *qweight, const uint16_t *scales, const ui
 // view of the rows, {128 bytes, 8 rows, K/256 column pairs}, 128-byte
 // swizzle: one copy moves 8 x K/2 bytes), and 16 computing warps consume them
 // while the next boxes are in flight.  After the dependency wait the
-// computing warps also split x into 24-bit planes (each warp keeps the plane
-// fragments of its own spans in registers), fold scale and activation scale
-// into one factor per (row, group) and sum each row's zero-point terms once.
+// computing warps also split x into 23-bit planes (each warp keeps the plane
+// fragments of its own spans in registers) and fold scale and activation
+// scale into one pair of factors per (row, group).
 //
 // The planes use signed base-256 digits, X = 65536 P0 + 256 P1 + P2 with
-// P0, P1, P2 in [-128, 127] (|X| <= 8355711), so all three are s8 columns of
+// P0 in [-64, 64] and P1, P2 in [-128, 127] (|X| <= 2^22 - 1), so all three are s8 columns of
 // one B operand: one m16n8k32 (u8 weights x s8 planes) gives D0, D1 and D2 of
 // 16 rows in columns 0, 1, 2.
 //
@@ -317,7 +317,7 @@ constexpr int kW4Block = kW4Threads + 32;  // + the producer warp
 constexpr int kW4MaxRows = 128;
 constexpr int kW4MaxSlots = 12;
 constexpr int kW4MinSlots = 4;
-constexpr int kW4XMax = 8355711;  // 127 * (65536 + 256 + 1)
+constexpr int kW4XMax = 4194303;  // 2^22 - 1: |X| stays in the exact range of the rounding FMA
 
 struct W4DecodeArgs {
     const float *x;
@@ -335,6 +335,15 @@ __device__ __forceinline__ int digit_s8(int v) { return ((v + 128) & 255) - 128;
 // gives 1.5 * 2^23 + v exactly, then the offset is subtracted (both exact).
 // One 16-row x 128-weight inner product stays below 15 * 128 * 128 < 2^18.
 __device__ __forceinline__ float exact_float(int v) { return __int_as_float(0x4B400000 + v) - 12582912.0f; }
+
+// mbar_wait with the polling loop out of line (keeps the consumers' loop body
+// small: the phase has usually completed by the time it is checked).
+__device__ __noinline__ bool w4_wait_slow(uint32_t bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+    return mbar_wait(bar, parity, abort, status, SITE_W4_STAGE);
+}
+__device__ __forceinline__ bool w4_wait(uint32_t bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+    return mbar_try_wait(bar, parity) || w4_wait_slow(bar, parity, abort, status);
+}
 
 // Arrival on named barrier `id` without waiting (the producer waits on it).
 __device__ __forceinline__ void w4_bar_arrive(uint32_t id, uint32_t threads) {
@@ -447,6 +456,8 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
         const int i = t + j * kW4Threads;
         sv[j] = i < ns ? __ldg(p.scales + sgo + i) : static_cast<uint16_t>(0);
     }
+    // the bias of row t (rows <= 128 < threads), added at the very end
+    const float bias_t = p.bias && t < rows ? __ldg(p.bias + n0 + t) : 0.0f;
     {
         uint32_t zv[2];
 #pragma unroll
@@ -464,8 +475,11 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
 
     // activation planes: thread t splits elements EPT t .. EPT t + EPT - 1 (a
     // group spans TPG = gs / EPT threads).  X = rne(x / sx) with
-    // sx = max|x| / 8355711 per group, x / sx taken as x * (1 / sx): at most
-    // one more unit of error than the exact quotient.
+    // sx = max|x| / (2^22 - 1) per group, x / sx taken as x * (1 / sx) and
+    // rounded by one FMA that adds 1.5 * 2^23 (exact while |x / sx| <= 2^22):
+    // at most one more unit of error than the exact quotient, on the FMA pipe.
+    // The digits are bytes of X: P2 = X (mod 256) as a signed byte,
+    // X1 = (X + 128) >> 8, P1 = X1 (mod 256), P0 = (X1 + 128) >> 8.
     {
         constexpr int EPT = 4 * SPW;
         const int TPG = gs / EPT;
@@ -477,42 +491,42 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
         const float sx = __fdiv_rn(amax, static_cast<float>(kW4XMax));
         const float inv = amax > 0.f ? __fdiv_rn(1.0f, sx) : 0.f;
         int sum = 0;
-        // byte e of this thread's run lands at position perm8(e) of its 8-chunk:
-        // word 2 (e / 8) + (e & 1), byte (e & 7) / 2
-        constexpr int NW = EPT / 4 < 2 ? 2 : EPT / 4;  // (half a chunk still touches both of its words)
-        uint32_t pw[3][NW];
-#pragma unroll
-        for (int w = 0; w < NW; ++w) pw[0][w] = pw[1][w] = pw[2][w] = 0u;
+        int xd[3][EPT];  // per element: X, X1, X0 (their low bytes are P2, P1, P0)
 #pragma unroll
         for (int j = 0; j < SPW; ++j) {
             const float e4[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                int X = __float2int_rn(__fmul_rn(e4[u], inv));
+                int X = __float_as_int(fmaf(e4[u], inv, 12582912.0f)) - 0x4B400000;
                 X = max(-kW4XMax, min(kW4XMax, X));
                 sum += X;
-                const int P2 = digit_s8(X), X1 = (X - P2) >> 8;
-                const int P1 = digit_s8(X1), P0 = (X1 - P1) >> 8;
-                const int e = 4 * j + u, w = 2 * (e >> 3) + (e & 1), sh = 8 * ((e & 7) >> 1);
-                pw[0][w] |= (static_cast<uint32_t>(P0) & 255u) << sh;
-                pw[1][w] |= (static_cast<uint32_t>(P1) & 255u) << sh;
-                pw[2][w] |= (static_cast<uint32_t>(P2) & 255u) << sh;
+                const int X1 = (X + 128) >> 8;
+                xd[2][4 * j + u] = X;
+                xd[1][4 * j + u] = X1;
+                xd[0][4 * j + u] = (X1 + 128) >> 8;
             }
         }
-        if (EPT >= 8) {  // whole 8-chunks: two words per chunk and plane
+        // low bytes of four values -> one word
+        auto pack4 = [](int a, int b, int c, int d) -> uint32_t {
+            return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+        };
+        if (EPT >= 8) {  // whole 8-chunks: even elements (positions 0..3), odd (4..7)
 #pragma unroll
             for (int q = 0; q < 3; ++q)
 #pragma unroll
-                for (int w = 0; w < EPT / 4; w += 2)
-                    *reinterpret_cast<uint2 *>(planes + q * K + EPT * t + 4 * w) = make_uint2(pw[q][w], pw[q][w + 1]);
-        } else {  // half a chunk: elements 0..3 or 4..7 of it, i.e. bytes 0,1 of both words or bytes 2,3
+                for (int h = 0; h < EPT / 8; ++h) {
+                    const int *v = xd[q] + 8 * h;
+                    *reinterpret_cast<uint2 *>(planes + q * K + EPT * t + 8 * h) =
+                        make_uint2(pack4(v[0], v[2], v[4], v[6]), pack4(v[1], v[3], v[5], v[7]));
+                }
+        } else {  // half a chunk: elements 0..3 or 4..7 of it, at positions hb, hb + 1, 4 + hb, 5 + hb
             const int base = (EPT * t) & ~7, hb = ((EPT * t) & 7) ? 2 : 0;
 #pragma unroll
             for (int q = 0; q < 3; ++q) {
-                planes[q * K + base + hb] = static_cast<int8_t>(pw[q][0] & 255u);
-                planes[q * K + base + hb + 1] = static_cast<int8_t>((pw[q][0] >> 8) & 255u);
-                planes[q * K + base + 4 + hb] = static_cast<int8_t>(pw[q][1] & 255u);
-                planes[q * K + base + 4 + hb + 1] = static_cast<int8_t>((pw[q][1] >> 8) & 255u);
+                planes[q * K + base + hb] = static_cast<int8_t>(xd[q][0]);
+                planes[q * K + base + hb + 1] = static_cast<int8_t>(xd[q][2]);
+                planes[q * K + base + 4 + hb] = static_cast<int8_t>(xd[q][1]);
+                planes[q * K + base + 4 + hb + 1] = static_cast<int8_t>(xd[q][3]);
             }
         }
         for (int o = TPG / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -576,8 +590,8 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
         const bool has1 = 2 * rb + 1 < nb;
         const int s1 = s0 + 1 == NS ? 0 : s0 + 1;
         const uint32_t ph1 = s0 + 1 == NS ? ph0 ^ 1u : ph0;
-        bool ok = mbar_wait(fbar + 8 * s0, ph0, &s_abort, p.status, SITE_W4_STAGE);
-        if (has1) ok = ok && mbar_wait(fbar + 8 * s1, ph1, &s_abort, p.status, SITE_W4_STAGE);
+        bool ok = w4_wait(fbar + 8 * s0, ph0, &s_abort, p.status);
+        if (has1) ok = ok && w4_wait(fbar + 8 * s1, ph1, &s_abort, p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             const uint32_t b0 = ring + static_cast<uint32_t>(s0) * L.slot;
@@ -634,11 +648,11 @@ __global__ void __launch_bounds__(kW4Block, 1) w4_decode_kernel(const __grid_con
         ph0 = s1 + 1 == NS ? ph1 ^ 1u : ph1;
     }
     named_bar_sync(1, kW4Threads);
-    for (int r = t; r < rows; r += kW4Threads) {
+    if (t < rows) {
         float acc = 0.f;
 #pragma unroll
-        for (int w = 0; w < kW4Warps; ++w) acc += s_part[w * p.rows_cap + r];
-        p.out[n0 + r] = (p.bias ? __ldg(p.bias + n0 + r) : 0.0f) + acc;
+        for (int w = 0; w < kW4Warps; ++w) acc += s_part[w * p.rows_cap + t];
+        p.out[n0 + t] = bias_t + acc;
     }
 }
 
