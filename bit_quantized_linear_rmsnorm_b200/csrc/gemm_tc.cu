@@ -101,10 +101,31 @@ __device__ __forceinline__ uint64_t smem_desc_mnmajor_sw128(uint32_t saddr) {
     return d;
 }
 
+// Work items of the persistent schedule (CTA b takes items b, b + G, ...): the
+// full waves of 128 x 256 tiles, then, when the last wave would leave at
+// least half of the CTAs idle, each of its tiles as two 128 x 128 halves, so
+// the busiest CTAs end half a tile earlier.
+struct Items {
+    int num_m, big, count;
+    __device__ Items(int num_tiles, int num_m_, int G, bool allow) : num_m(num_m_) {
+        const int full = (num_tiles / G) * G, left = num_tiles - full;
+        const bool split = allow && left > 0 && 2 * left <= G;
+        big = split ? full : num_tiles;
+        count = split ? full + 2 * left : num_tiles;
+    }
+    __device__ void tile(int item, int &m0, int &n0, bool &half) const {
+        const int t = item < big ? item : big + ((item - big) >> 1);
+        m0 = (t % num_m) * BM;
+        n0 = (t / num_m) * BN + (item < big ? 0 : ((item - big) & 1) * (BN / 2));
+        half = item >= big;
+    }
+};
+
 template <bool PACKED, bool B_KN, typename OutT>
 __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmO, const GemmDev p) {
+                   const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmO,
+                   const GemmDev p) {
     using C = Cfg<PACKED>;
     constexpr int S = C::kStages;
     constexpr int CC = 64 / static_cast<int>(sizeof(OutT));  // output columns per staging chunk
@@ -131,6 +152,8 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
     const int num_n = (p.N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
     const int nkb = (p.K + BK - 1) / BK;
+    // (the 2-bit path keeps whole tiles: its unpack warps expand the full B tile)
+    const Items items(num_tiles, num_m, static_cast<int>(gridDim.x), !PACKED);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -148,6 +171,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         fence_mbarrier_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmBh);
         tma_prefetch_desc(&tmO);
     }
     if (warp == 2) {
@@ -165,9 +189,11 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         uint32_t phase = 0;
         int64_t issued = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-            const int m0 = (tile % num_m) * BM;
-            const int n0 = (tile / num_m) * BN;
+        for (int item = blockIdx.x; item < items.count && ok; item += gridDim.x) {
+            int m0, n0;
+            bool half;
+            items.tile(item, m0, n0, half);
+            const uint32_t b_bytes = half ? B_BYTES / 2 : B_BYTES;
             for (int kb = 0; kb < nkb; ++kb) {
                 if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
                     ok = false;
@@ -179,15 +205,15 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                     tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
                     tma_load_2d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * (BK / 16), n0, full(stage));
                 } else if constexpr (B_KN) {
-                    mbar_arrive_expect_tx(full(stage), A_BYTES + B_BYTES);
+                    mbar_arrive_expect_tx(full(stage), A_BYTES + b_bytes);
                     tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
                     const uint32_t b_dst = sbase + C::OFF_B + stage * B_BYTES;
                     tma_load_2d(b_dst, &tmB, n0, kb * BK, full(stage));
-                    tma_load_2d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, full(stage));
+                    if (!half) tma_load_2d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, full(stage));
                 } else {
-                    mbar_arrive_expect_tx(full(stage), A_BYTES + B_BYTES);
+                    mbar_arrive_expect_tx(full(stage), A_BYTES + b_bytes);
                     tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
-                    tma_load_2d(sbase + C::OFF_B + stage * B_BYTES, &tmB, kb * BK, n0, full(stage));
+                    tma_load_2d(sbase + C::OFF_B + stage * B_BYTES, half ? &tmBh : &tmB, kb * BK, n0, full(stage));
                 }
                 ++issued;
                 if (++stage == S) {
@@ -209,11 +235,13 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = idesc_i8(BM, BN, true, !PACKED, B_KN);
+        constexpr uint32_t idesc_half = idesc_i8(BM, BN / 2, true, !PACKED, B_KN);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         int t = 0;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++t) {
+        for (int item = blockIdx.x; item < items.count && ok; item += gridDim.x, ++t) {
+            const uint32_t id = item < items.big ? idesc : idesc_half;
             const int abuf = t & 1;
             const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
             if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA)) {
@@ -241,7 +269,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                     const uint64_t ad = smem_desc_kmajor_sw128(a_addr + ks * UMMA_K);
                     const uint64_t bd = B_KN ? smem_desc_mnmajor_sw128(b_addr + ks * UMMA_K * 128)
                                              : smem_desc_kmajor_sw128(b_addr + ks * UMMA_K);
-                    tc_mma_i8(d_tmem, ad, bd, idesc, (kb | ks) != 0 ? 1u : 0u);
+                    tc_mma_i8(d_tmem, ad, bd, id, (kb | ks) != 0 ? 1u : 0u);
                 }
                 tc_commit(empty(stage));
                 if (++stage == S) {
@@ -267,9 +295,11 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         const float colscale_scalar = PACKED ? __ldg(p.colscale) : 0.0f;
         uint32_t chunk_ctr = 0;
         int t = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++t) {
-            const int m0 = (tile % num_m) * BM;
-            const int n0 = (tile / num_m) * BN;
+        for (int item = blockIdx.x; item < items.count; item += gridDim.x, ++t) {
+            int m0, n0;
+            bool half;
+            items.tile(item, m0, n0, half);
+            const int nc32 = half ? BN / 64 : BN / 32;  // 32-column chunks of this item
             const int abuf = t & 1;
             const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
 
@@ -301,13 +331,13 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             const int corr = (p.rowcorr != nullptr && row < p.M) ? __ldg(p.rowcorr + row) : 0;
 
 #pragma unroll 1
-            for (int c32 = 0; c32 < BN / 32; ++c32) {
+            for (int c32 = 0; c32 < nc32; ++c32) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(abuf * BN + c32 * 32) +
                                        (static_cast<uint32_t>(32 * q) << 16),
                                    v);
                 tmem_wait_ld();
-                if (c32 == BN / 32 - 1) {
+                if (c32 == nc32 - 1) {
                     tc_fence_before();
                     mbar_arrive(tempty(abuf));
                 }
@@ -361,7 +391,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        for (int item = blockIdx.x; item < items.count && ok; item += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb) {
                 bool got = true;
                 if (lane == 0) got = mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK);
@@ -427,7 +457,8 @@ bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64
 }
 
 template <bool PACKED, bool B_KN, typename OutT>
-bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
+                   const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
     using C = Cfg<PACKED>;
     auto kern = gemm_tc_kernel<PACKED, B_KN, OutT>;
@@ -449,22 +480,23 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
     p.N = static_cast<int>(g.N);
     p.K = static_cast<int>(g.K);
     p.status = dev.status;
-    kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mO, p);
+    kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mBh, mO, p);
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 template <typename OutT>
-bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
+                   const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
-    if (g.b_packed2) return launch_t<true, false, OutT>(g, mA, mB, mO, s, dev);
-    if (g.b_layout == BQ_W_KN) return launch_t<false, true, OutT>(g, mA, mB, mO, s, dev);
-    return launch_t<false, false, OutT>(g, mA, mB, mO, s, dev);
+    if (g.b_packed2) return launch_t<true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    if (g.b_layout == BQ_W_KN) return launch_t<false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
+    return launch_t<false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
 }
 
 }  // namespace
 
 bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) {
-    CUtensorMap mA, mB, mO;
+    CUtensorMap mA, mB, mBh, mO;
     if (!make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.K, g.M, g.lda, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return BQ_ERR_CUDA;
     bool okB;
@@ -476,6 +508,11 @@ bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) 
     else
         okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!okB) return BQ_ERR_CUDA;
+    // K-major weights: a 128-row box too, for the half tiles of a last partial wave
+    mBh = mB;
+    if (!g.b_packed2 && g.b_layout != BQ_W_KN &&
+        !make_map(&mBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BQ_ERR_CUDA;
     CUtensorMapDataType odt = g.out_dtype == BQ_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                               : g.out_dtype == BQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                       : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -484,11 +521,11 @@ bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) 
         return BQ_ERR_CUDA;
     switch (g.out_dtype) {
         case BQ_F32:
-            return dispatch<float>(g, mA, mB, mO, s, dev);
+            return dispatch<float>(g, mA, mB, mBh, mO, s, dev);
         case BQ_F16:
-            return dispatch<__half>(g, mA, mB, mO, s, dev);
+            return dispatch<__half>(g, mA, mB, mBh, mO, s, dev);
         default:
-            return dispatch<__nv_bfloat16>(g, mA, mB, mO, s, dev);
+            return dispatch<__nv_bfloat16>(g, mA, mB, mBh, mO, s, dev);
     }
 }
 

@@ -213,6 +213,10 @@ def test_gemm_atb_worked_example(golden_dir):
     (1, 8, 16, bq.BQ_W_NK, "bf16", False),
     (513, 1030, 2048, bq.BQ_W_NK, "bf16", True),
     (260, 2100, 96, bq.BQ_W_NK, "f32", False),
+    # more tiles than SMs with a short last wave: its tiles run as 128 x 128 halves
+    (1024, 5000, 64, bq.BQ_W_NK, "bf16", True),
+    (1100, 4400, 96, bq.BQ_W_KN, "f32", False),
+    (2000, 2560, 48, bq.BQ_W_NK, "f16", False),
 ])
 def test_gemm_ragged(M, N, K, layout, out, bias):
     _gemm_case(M, N, K, layout, out, bias, seed=M + N + K)
