@@ -46,8 +46,8 @@ L2_COPIES = 8
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the
 # kernel source it was taken on; stale once the source changes.
 NCU_TRAFFIC = {
-    # profiles/gemm_w8a8_4096.md: 33.608960 MB read + 2.566656 MB written
-    ("gemm_w8a8_4096", "46b247143e71f56c"): 36175616,
+    # profiles/gemm_w8a8_4096.md: 33.611008 MB read + 3.005952 MB written
+    ("gemm_w8a8_4096", "5c6842e83ac89bdf"): 36616960,
 }
 
 
@@ -266,7 +266,7 @@ def headline(args, dist, pk):
     traffic = NCU_TRAFFIC.get(("gemm_w8a8_4096", src))
     roof = {"bound": "tensor", "achieved": round(tops_rank, 2), "peak": round(peak_int8, 1), "unit": "TFLOP/s",
             "frac": round(tops_rank / peak_int8, 4), "traffic": traffic,
-            "kernel": "gemm_tc_kernel<W8A8, K-major B, bf16 out>",
+            "kernel": "gemm_pair_kernel<bf16 out> (W8A8, K-major B, CTA pairs, tcgen05 cta_group::2)",
             "peak_note": f"{pk['source']} bf16 {'sustained' if sustained else 'burst'} {bf16_peak} TFLOP/s x 2 "
                          f"(nominal int8/bf16 ratio; timed region {ms_total:.0f} ms); "
                          "int8 ops counted like flops, 2 per multiply-add",

@@ -428,6 +428,351 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// Pair kernel (W8A8 with K-major weights, large problems): clusters of two
+// CTAs on two SMs share one tcgen05.mma.cta_group::2 per 32 K of a 256 x 256
+// output tile.  CTA rank r stages its own 128 rows of A (rows m0 + 128 r) and
+// its half of B (rows n0 + 128 r), so each SM moves half of the B tile
+// through TMA and shared memory; the MMA of the leader (rank 0) reads both
+// CTAs' stages and writes each CTA's 128 rows x 256 columns into that CTA's
+// tensor memory.
+//   warp 0      TMA producer (both CTAs): waits for its own stage to be free,
+//               loads A and B with the pair form of the tensor copy, whose
+//               completion bytes count on the leader's full barrier (the
+//               leader's producer announces the bytes of both CTAs).
+//   warp 1      MMA issuer (leader only): 4 x tcgen05.mma.cta_group::2 per
+//               stage; the commit arrives on the stage's empty barrier in both
+//               CTAs.
+//   warp 2      allocates / frees 512 TMEM columns in both CTAs together.
+//   warps 4-7   epilogue (both CTAs): as in the single-CTA kernel, on the
+//               CTA's own rows; all 256 epilogue threads of the pair release
+//               an accumulator on the leader's barrier.
+// A short last wave runs as 256 x 128 halves (each CTA 64 rows of B).
+// Every wait is bounded; both CTAs always reach the closing cluster barrier.
+// ---------------------------------------------------------------------------
+namespace pairk {
+constexpr int kStages = 6;
+constexpr uint32_t PA_BYTES = 128 * BK;  // own 128 rows of A
+constexpr uint32_t PB_BYTES = 128 * BK;  // own half of a 256-wide B tile
+constexpr uint32_t OFF_A = 0;
+constexpr uint32_t OFF_B = OFF_A + kStages * PA_BYTES;
+constexpr uint32_t OFF_STG = OFF_B + kStages * PB_BYTES;
+constexpr uint32_t OFF_VEC = OFF_STG + 2 * STG_BYTES;  // colscale[BN], bias[BN]
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * BN * 4;
+// full[S], empty[S], tfull[2], tempty[2], drain
+constexpr uint32_t NBAR = 2 * kStages + 5;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, epilogue failure
+constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;
+}  // namespace pairk
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared::cluster address of the object at CTA-local address `addr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// Tensor copy into this CTA's shared memory whose completion counts on the
+// barrier at cluster address `bar` (the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                                 uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrives (once) on the barrier at CTA-local address `bar` in both CTAs of the
+// pair when the MMAs issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+template <typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmO,
+                     const GemmDev p) {
+    using namespace pairk;
+    constexpr int S = kStages;
+    constexpr int CC = 64 / static_cast<int>(sizeof(OutT));
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + OFF_BAR;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+    auto tfull = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (2 * S + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    int *epi_fail = reinterpret_cast<int *>(smem + OFF_MISC + 8);
+    float *vcol = reinterpret_cast<float *>(smem + OFF_VEC);
+    float *vbias = vcol + BN;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int num_m = (p.M + 2 * BM - 1) / (2 * BM);  // 256-row tiles
+    const int num_n = (p.N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int nkb = (p.K + BK - 1) / BK;
+    const int cl = static_cast<int>(blockIdx.x >> 1), ncl = static_cast<int>(gridDim.x >> 1);
+    // items as in the single-CTA schedule, over pairs and 256 x 256 tiles
+    const int full_w = (num_tiles / ncl) * ncl, left = num_tiles - full_w;
+    const bool split = left > 0 && 2 * left <= ncl;
+    const int big = split ? full_w : num_tiles, count = split ? full_w + 2 * left : num_tiles;
+    auto tile_of = [&](int item, int &m0, int &n0, bool &half) {
+        const int t = item < big ? item : big + ((item - big) >> 1);
+        m0 = (t % num_m) * 2 * BM;
+        n0 = (t / num_m) * BN + (item < big ? 0 : ((item - big) & 1) * (BN / 2));
+        half = item >= big;
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull(b), 1);
+            mbar_init(tempty(b), 256);  // the epilogue threads of both CTAs (leader's barrier)
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *epi_fail = 0;
+        fence_mbarrier_init();
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmBh);
+        tma_prefetch_desc(&tmO);
+    }
+    if (warp == 2) {
+        tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish_pair();
+        tc_fence_before();
+    }
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers initialized before any remote arrival
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        int stage = 0;
+        uint32_t phase = 0;
+        int64_t issued = 0;
+        bool ok = true;
+        for (int item = cl; item < count && ok; item += ncl) {
+            int m0, n0;
+            bool half;
+            tile_of(item, m0, n0, half);
+            const uint32_t b_bytes = half ? PB_BYTES / 2 : PB_BYTES;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
+                    ok = false;
+                    break;
+                }
+                if (leader) mbar_arrive_expect_tx(full(stage), 2u * (PA_BYTES + b_bytes));
+                const uint32_t lbar = cluster_addr(full(stage), 0);
+                tma_load_2d_pair(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank), lbar);
+                tma_load_2d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK,
+                                 n0 + (half ? BN / 4 : BN / 2) * static_cast<int>(rank), lbar);
+                ++issued;
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && leader) {
+            // the leader's full barriers count both CTAs' copies: let them land
+            for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i) {
+                const uint32_t bar = full(static_cast<int>(i % S));
+                const uint32_t par = static_cast<uint32_t>((i / S) & 1);
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(bar, par) && globaltimer_ns() - t0 < kWaitLimitNs) {
+                }
+            }
+        }
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        constexpr uint32_t idesc = idesc_i8(2 * BM, BN, true, true, false);
+        constexpr uint32_t idesc_half = idesc_i8(2 * BM, BN / 2, true, true, false);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        int t = 0;
+        for (int item = cl; item < count && ok; item += ncl, ++t) {
+            const uint32_t id = item < big ? idesc : idesc_half;
+            const int abuf = t & 1;
+            const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
+            if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tbase + static_cast<uint32_t>(abuf * BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = sbase + OFF_A + stage * PA_BYTES;
+                const uint32_t b_addr = sbase + OFF_B + stage * PB_BYTES;
+#pragma unroll
+                for (int ks = 0; ks < BK / UMMA_K; ++ks)
+                    tc_mma_i8_pair(d_tmem, smem_desc_kmajor_sw128(a_addr + ks * UMMA_K),
+                                   smem_desc_kmajor_sw128(b_addr + ks * UMMA_K), id, (kb | ks) != 0 ? 1u : 0u);
+                tc_commit_pair(empty(stage));
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (ok) tc_commit_pair(tfull(abuf));
+        }
+        if (!ok) {
+            tc_commit_pair(drain);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int q = warp - 4;
+        const int r = 32 * q + lane;
+        const int et = threadIdx.x - 128;
+        uint8_t *stg = smem + OFF_STG;
+        uint32_t chunk_ctr = 0;
+        int t = 0;
+        for (int item = cl; item < count; item += ncl, ++t) {
+            int m0, n0;
+            bool half;
+            tile_of(item, m0, n0, half);
+            const int mr = m0 + BM * static_cast<int>(rank);  // this CTA's first row
+            const int nc32 = half ? BN / 64 : BN / 32;
+            const int abuf = t & 1;
+            const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
+
+            named_bar_sync(1, 128);
+            for (int i = et; i < BN; i += 128) {
+                const int n = n0 + i;
+                vcol[i] = n < p.N ? __ldg(p.colscale + n) : 0.0f;
+                vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+            }
+            named_bar_sync(1, 128);
+
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok && lane == 0) {
+                atomicOr(epi_fail, 1);
+                *abort_flag = 1;
+            }
+            named_bar_sync(1, 128);
+            if (*reinterpret_cast<volatile int *>(epi_fail)) break;
+            tc_fence_after();
+            const int row = mr + r;
+            const float rs = row < p.M ? __ldg(p.rowscale + row) : 0.0f;
+
+#pragma unroll 1
+            for (int c32 = 0; c32 < nc32; ++c32) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tbase + static_cast<uint32_t>(abuf * BN + c32 * 32) +
+                                       (static_cast<uint32_t>(32 * q) << 16),
+                                   v);
+                tmem_wait_ld();
+                if (c32 == nc32 - 1) {
+                    tc_fence_before();
+                    mbar_arrive_remote(cluster_addr(tempty(abuf), 0));
+                }
+                float f[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float a = static_cast<float>(static_cast<int>(v[j]));
+                    f[j] = __fadd_rn(__fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs), vbias[c32 * 32 + j]);
+                }
+                uint32_t w[32];
+                constexpr int kSub = sizeof(OutT) == 2 ? 1 : 2;
+                if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w[j] = pack2<OutT>(f[2 * j], f[2 * j + 1]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(f[j]);
+                }
+#pragma unroll
+                for (int sc = 0; sc < kSub; ++sc) {
+                    const uint32_t sb = chunk_ctr & 1u;
+                    if (et == 0) bulk_wait_read<1>();
+                    named_bar_sync(1, 128);
+                    uint8_t *rowp = stg + sb * STG_BYTES + r * 64;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int pj = j ^ ((r >> 1) & 3);
+                        *reinterpret_cast<uint4 *>(rowp + pj * 16) =
+                            make_uint4(w[sc * 16 + 4 * j], w[sc * 16 + 4 * j + 1], w[sc * 16 + 4 * j + 2],
+                                       w[sc * 16 + 4 * j + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 128);
+                    if (et == 0) {
+                        tma_store_2d(&tmO, smem_u32(stg + sb * STG_BYTES), n0 + c32 * 32 + sc * CC, mr);
+                        bulk_commit();
+                    }
+                    ++chunk_ctr;
+                }
+            }
+        }
+        if (et == 0) bulk_wait_all();
+    }
+
+    __syncthreads();
+    cluster_sync_all();  // no remote arrival or MMA of the pair is left in flight
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc_pair(tbase, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Host side: tensor maps and launch
 // ---------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -485,10 +830,52 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
 }
 
 template <typename OutT>
+bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB128, const CUtensorMap &mB64,
+                      const CUtensorMap &mO, cudaStream_t s, const DevInfo &dev) {
+    auto kern = gemm_pair_kernel<OutT>;
+    static bool attr_set[64] = {};  // once per device (also keeps later calls capture-safe)
+    if (!attr_set[dev.device]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pairk::SMEM)) !=
+            cudaSuccess)
+            return BQ_ERR_CUDA;
+        attr_set[dev.device] = true;
+    }
+    const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN);
+    const int64_t pairs = std::min<int64_t>(tiles, dev.num_sms / 2);
+    GemmDev p;
+    p.colscale = g.colscale;
+    p.rowscale = g.rowscale;
+    p.rowcorr = nullptr;
+    p.bias = g.bias;
+    p.M = static_cast<int>(g.M);
+    p.N = static_cast<int>(g.N);
+    p.K = static_cast<int>(g.K);
+    p.status = dev.status;
+    kern<<<static_cast<unsigned>(2 * pairs), 256, pairk::SMEM, s>>>(mA, mB128, mB64, mO, p);
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+// The pair kernel takes W8A8 products with K-major weights that fill at least
+// one wave of CTA pairs with 256 x 256 tiles.
+bool use_pair(const GemmArgs &g, const DevInfo &dev) {
+    if (g.b_packed2 || g.b_layout == BQ_W_KN || dev.num_sms < 2) return false;
+    const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN);
+    return tiles >= dev.num_sms / 2;
+}
+
+template <typename OutT>
 bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
                    const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
     if (g.b_packed2) return launch_t<true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    if (use_pair(g, dev)) {
+        // per CTA of a pair: 128-row boxes of B (half of a 256-wide tile), 64-row boxes for half tiles
+        CUtensorMap mBq;
+        if (!make_map(&mBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 4,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+            return BQ_ERR_CUDA;
+        return launch_pair<OutT>(g, mA, mBh, mBq, mO, s, dev);
+    }
     if (g.b_layout == BQ_W_KN) return launch_t<false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
     return launch_t<false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
 }

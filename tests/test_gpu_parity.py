@@ -217,6 +217,10 @@ def test_gemm_atb_worked_example(golden_dir):
     (1024, 5000, 64, bq.BQ_W_NK, "bf16", True),
     (1100, 4400, 96, bq.BQ_W_KN, "f32", False),
     (2000, 2560, 48, bq.BQ_W_NK, "f16", False),
+    # enough 256 x 256 tiles for a wave of CTA pairs (tcgen05 cta_group::2), with and without half tiles
+    (2500, 4600, 64, bq.BQ_W_NK, "bf16", True),
+    (1536, 4864, 48, bq.BQ_W_NK, "f32", False),
+    (2048, 2560, 80, bq.BQ_W_NK, "f16", True),
 ])
 def test_gemm_ragged(M, N, K, layout, out, bias):
     _gemm_case(M, N, K, layout, out, bias, seed=M + N + K)
