@@ -447,22 +447,31 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
 //               CTA's own rows; all 256 epilogue threads of the pair release
 //               an accumulator on the leader's barrier.
 // A short last wave runs as 256 x 128 halves (each CTA 64 rows of B).
+// W2A8 (PACKED): each CTA loads A and its half of the packed 2-bit codes with
+// plain tensor copies on its own full barrier; its unpack warps (8-15)
+// expand only that half into the B stage and arrive on the leader's bready
+// barrier, which is what the MMA waits for (both CTAs' stages complete).
 // Every wait is bounded; both CTAs always reach the closing cluster barrier.
 // ---------------------------------------------------------------------------
-namespace pairk {
-constexpr int kStages = 6;
-constexpr uint32_t PA_BYTES = 128 * BK;  // own 128 rows of A
-constexpr uint32_t PB_BYTES = 128 * BK;  // own half of a 256-wide B tile
-constexpr uint32_t OFF_A = 0;
-constexpr uint32_t OFF_B = OFF_A + kStages * PA_BYTES;
-constexpr uint32_t OFF_STG = OFF_B + kStages * PB_BYTES;
-constexpr uint32_t OFF_VEC = OFF_STG + 2 * STG_BYTES;  // colscale[BN], bias[BN]
-constexpr uint32_t OFF_BAR = OFF_VEC + 2 * BN * 4;
-// full[S], empty[S], tfull[2], tempty[2], drain
-constexpr uint32_t NBAR = 2 * kStages + 5;
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, epilogue failure
-constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;
-}  // namespace pairk
+constexpr uint32_t PA_BYTES = 128 * BK;              // own 128 rows of A
+constexpr uint32_t PB_BYTES = 128 * BK;              // own half of a 256-wide B tile
+constexpr uint32_t PP_BYTES = 128 * (BK / 16) * 4;   // its packed 2-bit form
+template <bool PACKED>
+struct PairCfg {
+    static constexpr int kStages = PACKED ? 5 : 6;
+    static constexpr int kUnpack = 256;  // unpack threads (W2A8)
+    static constexpr int kThreads = PACKED ? 256 + kUnpack : 256;
+    static constexpr uint32_t OFF_A = 0;
+    static constexpr uint32_t OFF_B = OFF_A + kStages * PA_BYTES;
+    static constexpr uint32_t OFF_P = OFF_B + kStages * PB_BYTES;
+    static constexpr uint32_t OFF_STG = OFF_P + (PACKED ? kStages * PP_BYTES : 0);
+    static constexpr uint32_t OFF_VEC = OFF_STG + 2 * STG_BYTES;  // colscale[BN], bias[BN]
+    static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * BN * 4;
+    // full[S], empty[S], bready[S], tfull[2], tempty[2], drain
+    static constexpr uint32_t NBAR = 3 * kStages + 5;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, epilogue failure
+    static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;
+};
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -478,8 +487,9 @@ __device__ __forceinline__ uint32_t cluster_addr(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
+// Arrival (default release semantics) on the barrier at cluster address `caddr`.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
 }
 // Tensor copy into this CTA's shared memory whose completion counts on the
 // barrier at cluster address `bar` (the leader's).
@@ -520,13 +530,15 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-template <typename OutT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+template <bool PACKED, typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmO,
                      const GemmDev p) {
-    using namespace pairk;
-    constexpr int S = kStages;
+    using C = PairCfg<PACKED>;
+    constexpr int S = C::kStages;
+    constexpr uint32_t OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_P = C::OFF_P, OFF_STG = C::OFF_STG;
+    constexpr uint32_t OFF_VEC = C::OFF_VEC, OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC;
     constexpr int CC = 64 / static_cast<int>(sizeof(OutT));
 
     extern __shared__ uint8_t smem_raw[];
@@ -535,9 +547,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     const uint32_t bar0 = sbase + OFF_BAR;
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (S + s); };
-    auto tfull = [&](int b) { return bar0 + 8u * (2 * S + b); };
-    auto tempty = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
-    const uint32_t drain = bar0 + 8u * (2 * S + 4);
+    auto bready = [&](int s) { return bar0 + 8u * (2 * S + s); };
+    auto tfull = [&](int b) { return bar0 + 8u * (3 * S + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (3 * S + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
     int *epi_fail = reinterpret_cast<int *>(smem + OFF_MISC + 8);
@@ -568,6 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 1);
+            mbar_init(bready(s), 2 * C::kUnpack / 32);  // the unpack warps of both CTAs (leader's barrier)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
@@ -603,16 +617,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             bool half;
             tile_of(item, m0, n0, half);
             const uint32_t b_bytes = half ? PB_BYTES / 2 : PB_BYTES;
+            const int nb0 = n0 + (half ? BN / 4 : BN / 2) * static_cast<int>(rank);  // this CTA's B rows
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
+                if (!mbar_wait_spin(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
                     ok = false;
                     break;
                 }
-                if (leader) mbar_arrive_expect_tx(full(stage), 2u * (PA_BYTES + b_bytes));
-                const uint32_t lbar = cluster_addr(full(stage), 0);
-                tma_load_2d_pair(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank), lbar);
-                tma_load_2d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK,
-                                 n0 + (half ? BN / 4 : BN / 2) * static_cast<int>(rank), lbar);
+                if constexpr (PACKED) {  // own barrier: this CTA's unpack warps wait on it
+                    const uint32_t p_bytes = half ? PP_BYTES / 2 : PP_BYTES;
+                    mbar_arrive_expect_tx(full(stage), PA_BYTES + p_bytes);
+                    tma_load_2d(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
+                                full(stage));
+                    tma_load_2d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * (BK / 16), nb0,
+                                full(stage));
+                } else {  // the leader's barrier counts both CTAs' copies
+                    if (leader) mbar_arrive_expect_tx(full(stage), 2u * (PA_BYTES + b_bytes));
+                    const uint32_t lbar = cluster_addr(full(stage), 0);
+                    tma_load_2d_pair(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
+                                     lbar);
+                    tma_load_2d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK, nb0, lbar);
+                }
                 ++issued;
                 if (++stage == S) {
                     stage = 0;
@@ -620,8 +644,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 }
             }
         }
-        if (!ok && leader) {
-            // the leader's full barriers count both CTAs' copies: let them land
+        if (!ok && (leader || PACKED)) {
+            // let the copies this full barrier counts land (both CTAs' on the leader without 2-bit codes)
             for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i) {
                 const uint32_t bar = full(static_cast<int>(i % S));
                 const uint32_t par = static_cast<uint32_t>((i / S) & 1);
@@ -632,8 +656,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         }
     } else if (warp == 1 && lane == 0 && leader) {
         // ------------------------------------------------------------ MMA issuer (leader)
-        constexpr uint32_t idesc = idesc_i8(2 * BM, BN, true, true, false);
-        constexpr uint32_t idesc_half = idesc_i8(2 * BM, BN / 2, true, true, false);
+        constexpr uint32_t idesc = idesc_i8(2 * BM, BN, true, !PACKED, false);
+        constexpr uint32_t idesc_half = idesc_i8(2 * BM, BN / 2, true, !PACKED, false);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -649,7 +673,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             tc_fence_after();
             const uint32_t d_tmem = tbase + static_cast<uint32_t>(abuf * BN);
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                // (polled: the last arrival is often the peer CTA's)
+                if (!mbar_wait_spin(PACKED ? bready(stage) : full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
                     ok = false;
                     break;
                 }
@@ -680,6 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         const int r = 32 * q + lane;
         const int et = threadIdx.x - 128;
         uint8_t *stg = smem + OFF_STG;
+        const float colscale_scalar = PACKED ? __ldg(p.colscale) : 0.0f;
         uint32_t chunk_ctr = 0;
         int t = 0;
         for (int item = cl; item < count; item += ncl, ++t) {
@@ -694,7 +720,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             named_bar_sync(1, 128);
             for (int i = et; i < BN; i += 128) {
                 const int n = n0 + i;
-                vcol[i] = n < p.N ? __ldg(p.colscale + n) : 0.0f;
+                vcol[i] = (!PACKED && n < p.N) ? __ldg(p.colscale + n) : 0.0f;
                 vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
             }
             named_bar_sync(1, 128);
@@ -711,6 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             tc_fence_after();
             const int row = mr + r;
             const float rs = row < p.M ? __ldg(p.rowscale + row) : 0.0f;
+            const int corr = (PACKED && row < p.M) ? __ldg(p.rowcorr + row) : 0;
 
 #pragma unroll 1
             for (int c32 = 0; c32 < nc32; ++c32) {
@@ -726,8 +753,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 float f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float a = static_cast<float>(static_cast<int>(v[j]));
-                    f[j] = __fadd_rn(__fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs), vbias[c32 * 32 + j]);
+                    const float a = static_cast<float>(static_cast<int>(v[j]) - corr);
+                    const float o = PACKED ? __fmul_rn(__fmul_rn(a, rs), colscale_scalar)
+                                           : __fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs);
+                    f[j] = __fadd_rn(o, vbias[c32 * 32 + j]);
                 }
                 uint32_t w[32];
                 constexpr int kSub = sizeof(OutT) == 2 ? 1 : 2;
@@ -762,6 +791,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             }
         }
         if (et == 0) bulk_wait_all();
+    } else if (PACKED && warp >= 8) {
+        // ------------------------------------------------------------ unpack own half of B (both CTAs)
+        const int ut = threadIdx.x - 256;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int item = cl; item < count && ok; item += ncl) {
+            const int words = (item < big ? 128 : 64) * (BK / 16);  // packed words of this CTA's rows
+            for (int kb = 0; kb < nkb; ++kb) {
+                bool got = true;
+                if (lane == 0) got = mbar_wait_spin(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK);
+                if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t *pk = reinterpret_cast<const uint32_t *>(smem + OFF_P + stage * PP_BYTES);
+                uint8_t *bt = smem + OFF_B + stage * PB_BYTES;
+#pragma unroll 2
+                for (int idx = ut; idx < words; idx += C::kUnpack) {
+                    const int n = idx >> 3, c = idx & 7;  // weight row, 16-element chunk of the 128-K slab
+                    const uint32_t u = pk[idx];
+                    const uint4 codes = make_uint4(u & 0x03030303u, (u >> 2) & 0x03030303u,
+                                                   (u >> 4) & 0x03030303u, (u >> 6) & 0x03030303u);
+                    *reinterpret_cast<uint4 *>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = codes;
+                }
+                // every lane orders its stores before the tensor core's reads, then the
+                // warp's arrival on the leader releases them
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(cluster_addr(bready(stage), 0));
+                if (++stage == S) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
     }
 
     __syncthreads();
@@ -829,13 +894,14 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-template <typename OutT>
+template <bool PACKED, typename OutT>
 bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB128, const CUtensorMap &mB64,
                       const CUtensorMap &mO, cudaStream_t s, const DevInfo &dev) {
-    auto kern = gemm_pair_kernel<OutT>;
+    using C = PairCfg<PACKED>;
+    auto kern = gemm_pair_kernel<PACKED, OutT>;
     static bool attr_set[64] = {};  // once per device (also keeps later calls capture-safe)
     if (!attr_set[dev.device]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(pairk::SMEM)) !=
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
             cudaSuccess)
             return BQ_ERR_CUDA;
         attr_set[dev.device] = true;
@@ -845,20 +911,20 @@ bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMa
     GemmDev p;
     p.colscale = g.colscale;
     p.rowscale = g.rowscale;
-    p.rowcorr = nullptr;
+    p.rowcorr = g.rowcorr;
     p.bias = g.bias;
     p.M = static_cast<int>(g.M);
     p.N = static_cast<int>(g.N);
     p.K = static_cast<int>(g.K);
     p.status = dev.status;
-    kern<<<static_cast<unsigned>(2 * pairs), 256, pairk::SMEM, s>>>(mA, mB128, mB64, mO, p);
+    kern<<<static_cast<unsigned>(2 * pairs), C::kThreads, C::SMEM, s>>>(mA, mB128, mB64, mO, p);
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-// The pair kernel takes W8A8 products with K-major weights that fill at least
-// one wave of CTA pairs with 256 x 256 tiles.
+// The pair kernel takes products with K-major (or 2-bit packed) weights that
+// fill at least one wave of CTA pairs with 256 x 256 tiles.
 bool use_pair(const GemmArgs &g, const DevInfo &dev) {
-    if (g.b_packed2 || g.b_layout == BQ_W_KN || dev.num_sms < 2) return false;
+    if ((!g.b_packed2 && g.b_layout == BQ_W_KN) || dev.num_sms < 2) return false;
     const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN);
     return tiles >= dev.num_sms / 2;
 }
@@ -867,6 +933,16 @@ template <typename OutT>
 bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
                    const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
+    if (g.b_packed2 && use_pair(g, dev)) {
+        // per CTA of a pair: its half of the packed tile (128 rows), 64 rows for half tiles
+        CUtensorMap mP128, mP64;
+        if (!make_map(&mP128, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN / 2,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !make_map(&mP64, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN / 4,
+                      CU_TENSOR_MAP_SWIZZLE_NONE))
+            return BQ_ERR_CUDA;
+        return launch_pair<true, OutT>(g, mA, mP128, mP64, mO, s, dev);
+    }
     if (g.b_packed2) return launch_t<true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
     if (use_pair(g, dev)) {
         // per CTA of a pair: 128-row boxes of B (half of a 256-wide tile), 64-row boxes for half tiles
@@ -874,7 +950,7 @@ bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
         if (!make_map(&mBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 4,
                       CU_TENSOR_MAP_SWIZZLE_128B))
             return BQ_ERR_CUDA;
-        return launch_pair<OutT>(g, mA, mBh, mBq, mO, s, dev);
+        return launch_pair<false, OutT>(g, mA, mBh, mBq, mO, s, dev);
     }
     if (g.b_layout == BQ_W_KN) return launch_t<false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
     return launch_t<false, false, OutT>(g, mA, mB, mBh, mO, s, dev);

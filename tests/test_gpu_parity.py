@@ -322,7 +322,9 @@ def test_bitlinear_decode_stream_shapes(M, N, K, out, bias, xin):
 
 
 @pytest.mark.parametrize("M,N,K,out,bias", [(17, 256, 128, "bf16", False), (300, 520, 512, "bf16", True),
-                                            (129, 264, 640, "f32", False), (200, 1000, 1024, "f16", True)])
+                                            (129, 264, 640, "f32", False), (200, 1000, 1024, "f16", True),
+                                            # CTA-pair path, with and without half tiles in the last wave
+                                            (2500, 4600, 128, "bf16", True), (1536, 4864, 256, "f32", False)])
 def test_bitlinear_prefill_ragged(M, N, K, out, bias):
     g = synth.rng((109, M, N, K))
     bits, xf = synth.bf16_activations(M, K, (109, M), outlier_frac=0.01)
