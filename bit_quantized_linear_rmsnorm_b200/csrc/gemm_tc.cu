@@ -13,7 +13,12 @@
 //    exact ternary accumulator:
 //        out[m,n] = (float(acc - rowsum[m]) * act_scale[m]) * gamma (+ bias[n])
 //
-// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
+// Two kernels share the roles below.  Large products with K-major (or
+// packed) weights run on clusters of two CTAs (gemm_pair_kernel, 256 x 256
+// tiles per pair, tcgen05 cta_group::2; described at its definition); the
+// rest on single CTAs (gemm_tc_kernel).
+//
+// Single-CTA structure (one CTA per SM, persistent over 128 x 256 output tiles):
 //   warp 0      TMA producer: A tile (128 x 128 B) and B tile (256 x 128 B, or
 //               the 256 x 32 B packed tile) per stage, mbarrier tx-count.
 //   warp 1      MMA issuer: one thread issues 4 x tcgen05.mma (K = 32 each)
