@@ -18,6 +18,8 @@
 // the exact x*127/max|x| by at most three fp32 roundings (<= 1.8e-7
 // relative).  |x*f| <= 127 * (1 + 2^-22) always rounds inside [-127, 127], so
 // the clamp of the definition never changes a value.
+#include <algorithm>
+
 #include "bq_internal.h"
 #include "quant_common.cuh"
 
@@ -131,6 +133,100 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     }
 }
 
+// Block-per-row path for many rows (M of at least four CTAs per SM): a CTA of
+// 128 threads takes rows b, b + G, ...; thread t holds chunks t + 128 j
+// (j < CPT) of the row, so every load and store instruction of a warp covers
+// contiguous bytes, and it loads the chunks of its next row before reducing
+// and writing the current one (two rows in flight per CTA).  The rows spread
+// evenly over all CTAs, where one warp per row leaves a partial last wave of
+// rows.  Same arithmetic as the warp-per-row path.
+constexpr int kRowThreads = 128;
+template <typename In, int CPT>
+__global__ void __launch_bounds__(kRowThreads)
+    act_quant_row_kernel(const In *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float eps,
+                         int8_t *__restrict__ xq, int64_t ldq, float *__restrict__ act_scale,
+                         int32_t *__restrict__ rowsum) {
+    constexpr int EPC = Elt<In>::kPerChunk;
+    __shared__ float s_ss[kRowThreads / 32], s_mx[kRowThreads / 32];
+    __shared__ int s_rs[kRowThreads / 32];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int nchunks = static_cast<int>(K / EPC);  // K % EPC == 0 on this path
+    uint4 cur[CPT], nxt[CPT];
+    auto load_row = [&](int64_t m, uint4 (&dst)[CPT]) {
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x + m * ldx);
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + kRowThreads * j;
+            dst[j] = (m < M && c < nchunks) ? __ldcs(xv + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    int64_t m = blockIdx.x;
+    load_row(m, cur);
+    for (; m < M; m += gridDim.x) {
+        load_row(m + gridDim.x, nxt);
+        float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            float f[EPC];
+            Elt<In>::unpack(cur[j], f);
+#pragma unroll
+            for (int e = 0; e < EPC; e += 2) {
+                ss0 = fmaf(f[e], f[e], ss0);
+                ss1 = fmaf(f[e + 1], f[e + 1], ss1);
+                amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+            }
+        }
+        const float wss = warp_sum_f(ss0 + ss1), wmx = warp_max_f(amax);
+        if (lane == 0) {
+            s_ss[warp] = wss;
+            s_mx[warp] = wmx;
+        }
+        __syncthreads();
+        float ss = 0.f, mx = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRowThreads / 32; ++w) {
+            ss += s_ss[w];
+            mx = fmaxf(mx, s_mx[w]);
+        }
+        float f, scale;
+        quant_row_factor(ss, mx, K, eps, f, scale);
+        int8_t *qr = xq + m * ldq;
+        int isum = 0;
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) {
+            const int c = t + kRowThreads * j;
+            if (c < nchunks) {
+                float e[EPC];
+                Elt<In>::unpack(cur[j], e);
+                uint32_t w[EPC / 4];
+#pragma unroll
+                for (int q = 0; q < EPC / 4; ++q) {
+                    w[q] = pack_codes4(fmaf(e[4 * q], f, kRoundMagic), fmaf(e[4 * q + 1], f, kRoundMagic),
+                                       fmaf(e[4 * q + 2], f, kRoundMagic), fmaf(e[4 * q + 3], f, kRoundMagic));
+                    isum = dp4a_ss(w[q], 0x01010101u, isum);
+                }
+                if constexpr (EPC == 8) {
+                    *reinterpret_cast<uint2 *>(qr + c * 8) = make_uint2(w[0], w[1]);
+                } else {
+                    *reinterpret_cast<uint32_t *>(qr + c * 4) = w[0];
+                }
+            }
+        }
+        isum = warp_sum_i(isum);
+        if (lane == 0) s_rs[warp] = isum;
+        __syncthreads();
+        if (t == 0) {
+            int r = 0;
+#pragma unroll
+            for (int w = 0; w < kRowThreads / 32; ++w) r += s_rs[w];
+            act_scale[m] = scale;
+            if (rowsum) rowsum[m] = r;
+        }
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) cur[j] = nxt[j];
+    }
+}
+
 // Scalar path for rows without 16-byte alignment: two passes over x.
 template <typename In>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
@@ -174,6 +270,20 @@ cudaError_t launch_typed(const In *x, int64_t M, int64_t K, int64_t ldx, float e
     const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
     const bool vec = (reinterpret_cast<uintptr_t>(x) % 16 == 0) &&
                      ((ldx * static_cast<int64_t>(sizeof(In))) % 16 == 0);
+    constexpr int EPC = Elt<In>::kPerChunk;
+    const int64_t nch = K / EPC;
+    const int64_t rgrid = std::min<int64_t>(M, static_cast<int64_t>(dev.num_sms) * 12);
+    const bool rows_path = vec && K % EPC == 0 && nch <= 8 * kRowThreads && M >= 4 * dev.num_sms &&
+                           reinterpret_cast<uintptr_t>(xq) % 8 == 0 && ldq % 8 == 0;
+    if (rows_path) {
+        const int cpt = static_cast<int>((nch + kRowThreads - 1) / kRowThreads);
+        auto kern = cpt <= 1   ? act_quant_row_kernel<In, 1>
+                    : cpt <= 2 ? act_quant_row_kernel<In, 2>
+                    : cpt <= 4 ? act_quant_row_kernel<In, 4>
+                               : act_quant_row_kernel<In, 8>;
+        kern<<<static_cast<unsigned>(rgrid), kRowThreads, 0, s>>>(x, M, K, ldx, eps, xq, ldq, act_scale, rowsum);
+        return cudaGetLastError();
+    }
     if (vec)
         act_quant_vec_kernel<In><<<grid, kWarpsPerBlock * 32, 0, s>>>(x, M, K, ldx, eps, xq, ldq, act_scale,
                                                                        rowsum);

@@ -47,7 +47,10 @@ def _check_act(x_f32, x_dev, eps, what):
 
 @pytest.mark.parametrize("M,K,dtype", [(8, 256, "f32"), (37, 1000, "bf16"), (5, 4096, "bf16"),
                                        (300, 4096, "bf16"), (3, 6000, "f32"), (64, 8200, "bf16"),
-                                       (1, 7, "f32"), (17, 33, "bf16")])
+                                       (1, 7, "f32"), (17, 33, "bf16"),
+                                       # many rows: one CTA per row at a time (chunk counts 1..8 per thread)
+                                       (1300, 4096, "bf16"), (700, 4096, "f32"), (2000, 512, "bf16"),
+                                       (650, 1000, "f32"), (900, 8192, "bf16")])
 def test_act_quant(M, K, dtype):
     g = synth.rng((101, M, K))
     x = synth.normal_f32(g, (M, K))
