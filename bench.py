@@ -17,12 +17,17 @@ under "workloads", each against its own roofline.
 
 Multi-GPU: every rank runs an independent replica (the layer needs no
 exchange); the time is the max over ranks and `value` sums the work of all
-ranks.  `--impl reference` times the oracle (plain C, one host core) on a
-bounded sample of the same workload instead.
+ranks.  `--impl reference` times the oracle (plain C, row-parallel threads on
+all host cores) on a bounded sample of the same workload instead.
+
+`cpu_baseline` times the oracle, as it stands, on all host cores for every
+workload of the set (threads split the output rows; each thread runs the
+plain scalar oracle on its rows), on bounded row samples.
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import datetime
 import hashlib
 import json
@@ -44,11 +49,14 @@ L2_COPIES = 8
 
 # DRAM traffic of one launch of the headline kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the
-# kernel source it was taken on; stale once the source changes.
+# kernel source it was taken on; stale once the source changes.  The capture
+# flushes caches before the launch, not after it, so bf16 output still held in
+# L2 when the kernel ends is not counted as written.
 NCU_TRAFFIC = {
-    # profiles/gemm_w8a8_4096.md: 33.620992 MB read + 3.274240 MB written
+    # the ncu capture of the 4096^3 launch: 33.620992 MB read + 3.274240 MB written
     ("gemm_w8a8_4096", "83d85f51941e8ecf"): 36895232,
 }
+CPU_BUDGET_S = 4.0  # oracle wall time per workload in the CPU baseline
 
 
 def parse_args():
@@ -63,7 +71,8 @@ def parse_args():
     p.add_argument("--workload-steps", type=int, default=200)
     p.add_argument("--no-head", action="store_true", help="skip the headline GEMM (profiling runs only)")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows (0 = calibrate to ~10 s)")
+    p.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows of the headline (0 = calibrate)")
+    p.add_argument("--cpu-budget", type=float, default=CPU_BUDGET_S, help="oracle seconds per workload")
     return p.parse_args()
 
 
@@ -86,56 +95,118 @@ def source_hash(*names):
     return h.hexdigest()[:16]
 
 
-class Clocks:
-    """nvidia-smi sampled every 200 ms while the timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+def gpu_id(device: int) -> str:
+    """nvidia-smi -i argument naming the physical GPU behind torch device
+    `device` (its PCI bus id; torch's index is relative to CUDA_VISIBLE_DEVICES)."""
+    import torch
+    props = torch.cuda.get_device_properties(device)
+    dom, bus, dv = (getattr(props, a, None) for a in ("pci_domain_id", "pci_bus_id", "pci_device_id"))
+    if None not in (dom, bus, dv):
+        return f"{dom:08X}:{bus:02X}:{dv:02X}.0"
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    if vis:
+        entries = [e.strip() for e in vis.split(",") if e.strip()]
+        if device < len(entries):
+            return entries[device]
+    return str(device)
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+
+class Clocks:
+    """SM clock, power and clock-event reasons of the GPU, sampled every few
+    milliseconds (NVML, read-only queries) from a background thread while the
+    warm-up replays and the timed region run; nvidia-smi at 200 ms where NVML
+    is unavailable.  Every sample is taken under load (back-to-back replays)."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, device: int, period_s: float = 0.002):
+        self.device = device
+        self.period = period_s
+        self.samples = []  # (t, sm_mhz, max_mhz, reason bits)
+        self.marks = {}
+        self._stop = None
+        self._thread = None
+        self._smi = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        gid = gpu_id(self.device)
+        if ":" in gid:
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(gid)
+        if gid.startswith("GPU-"):
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(gid)
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(gid))
 
     def __enter__(self):
+        import threading
+        self.samples = []
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-i", str(self.gpu), "-lms", "200"], stdout=subprocess.PIPE,
-                                         stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-        time.sleep(0.25)
+            nv, h = self._handle()
+        except Exception:
+            nv = None
+        if nv is None:
+            try:
+                self._smi = subprocess.Popen(
+                    ["nvidia-smi", "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                     "--format=csv,noheader,nounits", "-i", gpu_id(self.device), "-lms", "200"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                self._smi = None
+            return self
+        self._stop = threading.Event()
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.perf_counter(), float(sm), float(mx), int(rs)))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
+    def mark(self, name: str):
+        self.marks[name] = time.perf_counter()
+
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            time.sleep(0.25)
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._smi is not None:
+            self._smi.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                out, _ = self._smi.communicate(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self._smi.kill()
+                out, _ = self._smi.communicate()
+            now = time.perf_counter()
+            for ln in out.splitlines():
+                parts = [x.strip() for x in ln.split(",")]
+                try:
+                    self.samples.append((now, float(parts[0]), float(parts[1]), int(parts[2], 16)))
+                except (ValueError, IndexError):
+                    continue
+        return False
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [x[1] for x in self.samples]
+        bits = 0
+        for x in self.samples:
+            bits |= x[3]
+        t0, t1 = self.marks.get("timed_start"), self.marks.get("timed_end")
+        inside = [x[1] for x in self.samples if t0 is not None and t1 is not None and t0 <= x[0] <= t1]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[2] for x in self.samples),
+                "reasons": sorted(n for n, b in self.REASONS if bits & b), "samples": len(sm),
+                "samples_in_timed_region": len(inside),
+                "sm_mhz_in_timed_region": statistics.median(inside) if inside else None,
+                "source": "nvml" if self._smi is None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -149,14 +220,18 @@ def dist_setup():
 
 
 class Dist:
-    def __init__(self, world, rank, local):
+    """Replica plumbing: a barrier and a max over ranks (NCCL on GPUs; gloo
+    on CPU for the host-side tests).  No collective touches the data path."""
+
+    def __init__(self, world, rank, local, backend: str = "nccl", timeout_s: int = 120):
         import torch
         self.world, self.rank, self.local = world, rank, local
+        self.backend = backend
         self.pg = None
         if world > 1:
             import torch.distributed as td
-            td.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                  device_id=torch.device("cuda", local))
+            kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+            td.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
             self.pg = td
 
     def barrier(self):
@@ -167,7 +242,7 @@ class Dist:
         if self.pg is None:
             return v
         import torch
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        t = torch.tensor([v], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
@@ -179,9 +254,20 @@ class Dist:
 # ---------------------------------------------------------------------------
 # timing helpers
 # ---------------------------------------------------------------------------
-def graph_time(fn_for_step, steps: int, warmup: int, dist=None, clocks=None):
+def aggregate(units_per_rank: float, ms_rank: float, dist) -> tuple:
+    """Whole-job throughput of independent replicas: the units all ranks
+    processed over the slowest rank's time.  Returns (units per second, max ms)."""
+    ms_max = dist.max(ms_rank)
+    return units_per_rank * dist.world / (ms_max * 1e-3), ms_max
+
+
+def graph_time(fn_for_step, steps: int, warmup: int, dist=None, clocks=None, sustain_s: float = 0.0):
     """Captures `steps` calls fn_for_step(i) in one CUDA graph and times one
-    replay with events on the capturing stream.  Returns ms per step."""
+    replay with events on the capturing stream.  Returns (ms per step, ms of
+    the replay, sustained ms per step or None).  `clocks` samples the GPU over
+    the warm replays and the timed replay.  With sustain_s > 0 the graph is
+    then replayed back to back for that long, under the power cap, and timed
+    as a whole (the sustained figure)."""
     import torch
     s = torch.cuda.Stream()
     with torch.cuda.stream(s):
@@ -194,37 +280,51 @@ def graph_time(fn_for_step, steps: int, warmup: int, dist=None, clocks=None):
             fn_for_step(i)
     # warm replays of the graph itself, for at least 50 ms so that the SM
     # clocks have left their idle level before the timed replay
-    t_end = time.perf_counter() + 0.05
-    while True:
-        g.replay()
-        s.synchronize()
-        if time.perf_counter() >= t_end:
-            break
+    def replays(seconds):
+        t_end = time.perf_counter() + seconds
+        n = 0
+        while True:
+            g.replay()
+            n += 1
+            s.synchronize()
+            if time.perf_counter() >= t_end:
+                return n
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ctx = clocks if clocks is not None else _Null()
-    with ctx:
+    if clocks is not None:
+        clocks.__enter__()
+    try:
+        replays(0.05)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        if clocks is not None:
+            clocks.mark("timed_start")
         with torch.cuda.stream(s):
             e0.record(s)
             g.replay()
             e1.record(s)
         s.synchronize()
-    torch.cuda.synchronize()
+        if clocks is not None:
+            clocks.mark("timed_end")
+        torch.cuda.synchronize()
+    finally:
+        if clocks is not None:
+            clocks.__exit__(None, None, None)
     if dist is not None:
         dist.barrier()
     ms = e0.elapsed_time(e1)
+    sustained = None
+    if sustain_s > 0:
+        reps = max(1, int(sustain_s / max(ms * 1e-3, 1e-6)))
+        with torch.cuda.stream(s):
+            e0.record(s)
+            for _ in range(reps):
+                g.replay()
+            e1.record(s)
+        s.synchronize()
+        sustained = e0.elapsed_time(e1) / (reps * steps)
     del g
-    return ms / steps, ms
-
-
-class _Null:
-    def __enter__(self):
-        return self
-
-    def __exit__(self, *a):
-        return False
+    return ms / steps, ms, sustained
 
 
 # ---------------------------------------------------------------------------
@@ -249,11 +349,11 @@ def headline(args, dist, pk):
         bq.bq_gemm_i8_pertoken(xs[j], ws[j], deq, pts, out=outs[j])
 
     clocks = Clocks(torch.cuda.current_device())
-    ms_step, ms_total = graph_time(step, args.steps, args.warmup, dist, clocks)
-    ms_step_max = dist.max(ms_step)
+    ms_step, ms_total, ms_sust = graph_time(step, args.steps, args.warmup, dist, clocks, sustain_s=1.5)
     ops = 2.0 * HEAD["M"] * HEAD["N"] * HEAD["K"]
     tops_rank = ops / (ms_step * 1e-3) / 1e12
-    value = ops * dist.world / (ms_step_max * 1e-3) / 1e12
+    ops_per_s, ms_step_max = aggregate(ops, ms_step, dist)
+    value = ops_per_s / 1e12
     st, detail = bq.bq_device_status()
     if st != bq.BQ_OK:
         raise RuntimeError(f"device status {detail:#x} after the timed region")
@@ -266,11 +366,20 @@ def headline(args, dist, pk):
     traffic = NCU_TRAFFIC.get(("gemm_w8a8_4096", src))
     roof = {"bound": "tensor", "achieved": round(tops_rank, 2), "peak": round(peak_int8, 1), "unit": "TFLOP/s",
             "frac": round(tops_rank / peak_int8, 4), "traffic": traffic,
+            "traffic_note": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch; the write count "
+                            "misses the bf16 output still in L2 when the kernel ends",
             "kernel": "gemm_pair_kernel<bf16 out> (W8A8, K-major B, CTA pairs, tcgen05 cta_group::2)",
             "peak_note": f"{pk['source']} bf16 {'sustained' if sustained else 'burst'} {bf16_peak} TFLOP/s x 2 "
                          f"(nominal int8/bf16 ratio; timed region {ms_total:.0f} ms); "
                          "int8 ops counted like flops, 2 per multiply-add",
             "algorithmic_bytes_per_launch": 2 * 4096 * 4096 + 4096 * 4096 * 2 + 2 * 4096 * 4}
+    if ms_sust is not None:
+        sust_tops = ops / (ms_sust * 1e-3) / 1e12
+        sust_peak = 2.0 * pk["bf16_tflops_sustained"]
+        roof["sustained"] = {"us_per_step": round(ms_sust * 1e3, 3), "achieved": round(sust_tops, 2),
+                             "peak": round(sust_peak, 1), "frac": round(sust_tops / sust_peak, 4),
+                             "note": "the same graph replayed back to back for 1.5 s (power-capped clocks), "
+                                     "against the sustained bf16 figure x 2"}
     # end to end through the public API with host buffers
     e2e = headline_e2e(args, d, dist)
     return {"value": value, "ms_per_step": ms_step_max, "roofline": roof, "clocks": clocks.summary(), "e2e": e2e,
@@ -369,7 +478,7 @@ def _decode(res, steps, hbm):
         def step(i, x=x, out=out, work=work):
             bq.bq_bitlinear_w2a8(x, wps[i % copies], wsc, N, None, 1e-5, torch.bfloat16, out=out, workspace=work)
 
-        ms, _ = graph_time(step, steps, 3)
+        ms, _, _ = graph_time(step, steps, 3)
         byts = N * K // 4 + 4 + 2 * M * K + 2 * M * N
         gbs = byts / (ms * 1e-3) / 1e9
         res[f"bitlinear_decode_M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
@@ -402,7 +511,7 @@ def _w4(res, steps, hbm):
             a, b, c = sets[i % copies]
             bq.bq_linear_w4_grouped(x, a, b, c, gs, bias, out=out, workspace=work)
 
-        ms, _ = graph_time(step, steps, 3)
+        ms, _, _ = graph_time(step, steps, 3)
         byts = N * K // 2 + N * (K // gs) * 2 + N * ((K // gs + 7) // 8) * 4 + 4 * N + 4 * M * K + 4 * M * N
         gbs = byts / (ms * 1e-3) / 1e9
         res[f"linear_w4_M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
@@ -428,7 +537,7 @@ def _prefill(res, steps, peak_int8, hbm):
     def step(i):
         bq.bq_bitlinear_w2a8(x, wp, wsc, N, None, 1e-5, torch.bfloat16, out=out, workspace=work)
 
-    ms, _ = graph_time(step, steps, 3)
+    ms, _, _ = graph_time(step, steps, 3)
     ops = 2.0 * M * N * K
     tops = ops / (ms * 1e-3) / 1e12
     # the activation quantization alone, to split the step (three copies of x so
@@ -441,7 +550,7 @@ def _prefill(res, steps, peak_int8, hbm):
     def aq(i):
         bq.bq_act_quant_int8(xs[i % 3], 1e-5, xq=xq, act_scale=sc, rowsum=rs)
 
-    ms_aq, _ = graph_time(aq, steps, 3)
+    ms_aq, _, _ = graph_time(aq, steps, 3)
     aq_bytes = 2 * M * K + M * K + 8 * M
     gemm_ms = max(ms - ms_aq, 1e-9)
     res["bitlinear_prefill"] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(tops, 1),
@@ -470,31 +579,148 @@ def _tiny(res, steps):
     def step(i):
         bq.bq_bitlinear_w2a8(x, wp, wsc, 128, None, 1e-5, torch.float32, out=out, workspace=work)
 
-    ms, _ = graph_time(step, steps, 3)
+    ms, _, _ = graph_time(step, steps, 3)
     res["bitlinear_tiny"] = {"us_per_step": round(ms * 1e3, 3), "config": "x fp32 [8,256], W [128,256]"}
 
 
 # ---------------------------------------------------------------------------
-# CPU baseline: the oracle on a bounded sample of the headline workload
+# CPU baseline: the oracle on all host cores, every workload of the set
 # ---------------------------------------------------------------------------
-def oracle_sample(d, rows: int):
-    import oracle
-    sel = np.arange(rows)
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _ranges(n: int, parts: int):
+    parts = max(1, min(parts, n))
+    step, extra = divmod(n, parts)
+    lo = 0
+    for i in range(parts):
+        hi = lo + step + (1 if i < extra else 0)
+        yield lo, hi
+        lo = hi
+
+
+def run_rows(fn, n: int, threads: int) -> float:
+    """Wall time of fn(lo, hi) over rows [0, n) split across `threads` threads.
+    The oracle's C routines run without the GIL (ctypes releases it), so the
+    threads run in parallel; each runs the plain oracle on its own rows."""
     t0 = time.perf_counter()
-    oracle.gemm_i8_pertoken(d["x"][sel], d["w"], d["deq_scale"], d["per_token_scale"][sel])
+    if threads <= 1:
+        fn(0, n)
+    else:
+        with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+            for f in [ex.submit(fn, lo, hi) for lo, hi in _ranges(n, threads)]:
+                f.result()
     return time.perf_counter() - t0
 
 
-def cpu_baseline(d, rows: int = 0):
+def sample_rows(fn, total: int, threads: int, budget_s: float, probe: int = 0) -> tuple:
+    """Rows of a bounded sample (whole multiples of the thread count, capped at
+    `total`) sized so fn over them takes about budget_s on `threads` threads.
+    Returns (rows, seconds) of the timed sample (when the whole workload fits,
+    the mean over repeated runs of it)."""
+    probe = probe or min(total, threads)
+    while True:
+        t = run_rows(fn, probe, threads)
+        if t >= 0.1 * budget_s or probe >= total:
+            break
+        probe = min(total, probe * 4)
+    if probe >= total:
+        # the whole workload fits the budget: repeat it for a stable mean
+        reps = max(1, min(50, int(0.5 * budget_s / max(t, 1e-6))))
+        if reps > 1:
+            t = sum(run_rows(fn, total, threads) for _ in range(reps)) / reps
+        return total, t
+    per_round = t / max(1, -(-probe // threads))  # seconds per row per thread
+    rows = int(budget_s / max(per_round, 1e-9)) * threads
+    rows = max(threads, min(total, rows))
+    return rows, run_rows(fn, rows, threads)
+
+
+def _head_fn(d):
     import oracle
+
+    def fn(lo, hi):
+        oracle.gemm_i8_pertoken(d["x"][lo:hi], d["w"], d["deq_scale"], d["per_token_scale"][lo:hi])
+    return fn
+
+
+def cpu_baseline(d, args, pk) -> dict:
+    """The oracle, as it stands, on the host cores for every workload; the
+    headline's figure is the line's cpu_baseline.value."""
+    import oracle
+    import synth
     oracle.build()
-    if rows <= 0:
-        t = oracle_sample(d, 2)
-        rows = int(max(2, min(4096, round(2 * 10.0 / max(t, 1e-6)))))
-    t = oracle_sample(d, rows)
-    ops = 2.0 * rows * HEAD["N"] * HEAD["K"]
-    return {"value": round(ops / t / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} of 4096 rows of the 4096^3 W8A8 GEMM (all 4096 columns), {t:.1f} s, one thread"}
+    cores = host_cores()
+    budget = args.cpu_budget
+    res = {}
+    # W8A8 GEMM 4096^3: rows of x
+    M, N, K = HEAD["M"], HEAD["N"], HEAD["K"]
+    if args.cpu_rows > 0:
+        rows = min(M, args.cpu_rows)
+        t = run_rows(_head_fn(d), rows, cores)
+    else:
+        rows, t = sample_rows(_head_fn(d), M, cores, budget)
+    res["gemm_w8a8_4096"] = {"value": round(2.0 * rows * N * K / t / 1e12, 6), "unit": "TOPS", "cores": cores,
+                             "sample": f"{rows} of {M} rows (all {N} columns), {t:.2f} s"}
+    # BitLinear prefill 8192 x 4096 x 4096: act quant + integer linear on rows of x (weights quantized beforehand)
+    dp = synth.bitlinear_prefill()
+    tq = oracle.ternary_quant(dp["w"])
+
+    def prefill(lo, hi):
+        a = oracle.act_quant(dp["x"][lo:hi], dp["eps"])
+        oracle.bitlinear_from_codes(a["xq"], a["act_scale"], tq["wq"], tq["gamma"])
+    rows, t = sample_rows(prefill, 8192, cores, budget)
+    res["bitlinear_prefill"] = {"value": round(2.0 * rows * 4096 * 4096 / t / 1e12, 6), "unit": "TOPS",
+                                "cores": cores, "sample": f"{rows} of 8192 rows (all 4096 columns), {t:.2f} s"}
+    # BitLinear decode, M in {1, 4, 16}: act quant of the tokens + integer linear over weight rows
+    wd = synth.bitlinear_weight(11008, 4096, 3)
+    td = oracle.ternary_quant(wd)
+    for Md in (1, 4, 16):
+        dd = synth.bitlinear_decode(Md)
+        a = oracle.act_quant(dd["x"], dd["eps"])
+
+        def decode(lo, hi, a=a, dd=dd):
+            aa = oracle.act_quant(dd["x"], dd["eps"]) if lo == 0 else a
+            oracle.bitlinear_from_codes(aa["xq"], aa["act_scale"], td["wq"][lo:hi], td["gamma"])
+        rows, t = sample_rows(decode, 11008, cores, budget / 3)
+        byts = (11008 * 4096 // 4 + 4 + 2 * Md * 4096 + 2 * Md * 11008) * rows / 11008
+        res[f"bitlinear_decode_M{Md}"] = {"value": round(byts / t / 1e9, 4), "unit": "GB/s", "cores": cores,
+                                          "sample": f"{rows} of 11008 weight rows, {t:.3f} s (bytes of the GPU "
+                                                    "call's packed weights, scaled to the rows)"}
+    # grouped INT4, M in {1, 32}: over weight rows
+    w4 = synth.linear_w4_weights()
+    qw, qz = oracle.int4_pack(w4["q"]), oracle.int4_pack(w4["zeros"])
+    sb = w4["scales_f16"].view(np.uint16)
+    Nw, Kw, gs = 14336, 4096, 128
+    for Mw in (1, 32):
+        xw = synth.linear_w4_activations(Mw)
+
+        def w4f(lo, hi, xw=xw):
+            oracle.linear_w4_grouped(xw, qw[lo:hi], sb[lo:hi], qz[lo:hi], w4["bias"][lo:hi], gs)
+        rows, t = sample_rows(w4f, Nw, cores, budget / 2)
+        byts = (Nw * Kw // 2 + Nw * (Kw // gs) * 2 + Nw * 4 * 4 + 4 * Nw + 4 * Mw * Kw + 4 * Mw * Nw) * rows / Nw
+        res[f"linear_w4_M{Mw}"] = {"value": round(byts / t / 1e9, 4), "unit": "GB/s", "cores": cores,
+                                   "sample": f"{rows} of {Nw} weight rows, {t:.3f} s (bytes of the GPU call, "
+                                             "scaled to the rows)"}
+    # BitLinear tiny 8 x 256 -> 128: whole forward from pre-quantized weights, one thread
+    dt = synth.bitlinear_tiny(0)
+    tt = oracle.ternary_quant(dt["w"])
+    reps = 200
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        a = oracle.act_quant(dt["x"], dt["eps"])
+        oracle.bitlinear_from_codes(a["xq"], a["act_scale"], tt["wq"], tt["gamma"])
+    t = (time.perf_counter() - t0) / reps
+    res["bitlinear_tiny"] = {"value": round(t * 1e6, 2), "unit": "us per call", "cores": 1,
+                             "sample": f"whole workload, mean of {reps} calls"}
+    head = res["gemm_w8a8_4096"]
+    return {"value": head["value"], "unit": "TOPS", "cores": cores, "kind": "oracle", "host_cores": os.cpu_count(),
+            "sample": f"W8A8 4096^3: {head['sample']}, plain C oracle on row-parallel threads",
+            "workloads": res}
 
 
 def reference_arm(args):
@@ -505,18 +731,28 @@ def reference_arm(args):
     import synth
     oracle.build()
     d = synth.gemm_w8a8(**HEAD)
-    rows = max(1, args.cpu_rows or 4)
+    cores = host_cores()
+    fn = _head_fn(d)
+    if args.cpu_rows > 0:
+        rows = args.cpu_rows
+    else:
+        # rows per step sized so that warm-up plus timed steps take about a minute
+        t1 = run_rows(fn, cores, cores)
+        rows = max(1, int(60.0 / max(args.steps + args.warmup, 1) / max(t1, 1e-6)) * cores)
+        rows = min(rows, HEAD["M"])
     for _ in range(args.warmup):
-        oracle_sample(d, rows)
-    t = sum(oracle_sample(d, rows) for _ in range(args.steps))
+        run_rows(fn, rows, cores)
+    t = sum(run_rows(fn, rows, cores) for _ in range(args.steps))
     ops = 2.0 * rows * HEAD["N"] * HEAD["K"] * args.steps
     value = ops / t / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
             "config": {"workload": HEAD_WORKLOAD, **HEAD, "sample_rows_per_step": rows},
-            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows} rows x 4096 columns per step, plain C double/int64 loops"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+                             "host_cores": os.cpu_count(),
+                             "sample": f"{rows} rows x 4096 columns per step, plain C double/int64 loops on "
+                                       f"{cores} row-parallel threads"},
             "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -548,7 +784,7 @@ def main():
         extra = workloads(args, pk)
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        base = cpu_baseline(d, args.cpu_rows)
+        base = cpu_baseline(d, args, pk)
     if rank == 0:
         line = {"metric": METRIC, "value": round(head["value"], 2), "unit": "TOPS", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(head["ms_per_step"], 5),

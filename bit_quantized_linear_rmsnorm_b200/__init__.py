@@ -28,8 +28,10 @@ EXPORTED = [
     "bq_act_quant_int8", "bq_weight_quant_ternary_pack", "bq_weight_pack_int4_grouped",
     "bq_gemm_i8_pertoken", "bq_bitlinear_w2a8", "bq_linear_w4_grouped", "bq_workspace_bytes",
     "bq_bitlinear_workspace_layout", "bq_status_string", "bq_device_status", "bq_version",
-    "bq_bitlinear_w2a8_noalloc",
+    "bq_bitlinear_w2a8_noalloc", "bq_bitlinear_w2a8_path", "bq_diag_gemm_withheld_arrival",
 ]
+(BQ_PATH_DECODE_STREAM, BQ_PATH_DECODE_MMA, BQ_PATH_DECODE_SMEM, BQ_PATH_ACT_QUANT_GEMV, BQ_PATH_TC_SINGLE,
+ BQ_PATH_TC_PAIR) = range(1, 7)
 BQ_NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
 
 _DTYPE = {torch.float32: BQ_F32, torch.bfloat16: BQ_BF16, torch.float16: BQ_F16}
@@ -48,6 +50,8 @@ _SIGS = {
     "bq_bitlinear_w2a8": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P, SZ, P]),
     "bq_linear_w4_grouped": (I32, [P, I64, I64, P, P, P, P, I64, I64, P, P, SZ, P]),
     "bq_bitlinear_w2a8_noalloc": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P]),
+    "bq_bitlinear_w2a8_path": (I32, [P, I32, I64, I64, I64, ctypes.POINTER(I32)]),
+    "bq_diag_gemm_withheld_arrival": (I32, [P, P, P, P, P, ctypes.c_uint64, P]),
     "bq_workspace_bytes": (SZ, [I32, I64, I64, I64, I64]),
     "bq_bitlinear_workspace_layout": (None, [I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     "bq_status_string": (ctypes.c_char_p, [I32]),
@@ -236,3 +240,12 @@ def bq_bitlinear_w2a8_noalloc(x: torch.Tensor, wpacked: torch.Tensor, w_scale: t
                                          float(eps), _DTYPE[out.dtype], _ptr(out), _stream(stream))
     _check(st, "bq_bitlinear_w2a8_noalloc")
     return out
+
+
+def bq_bitlinear_w2a8_path(x: torch.Tensor, N: int) -> int:
+    """Which kernels bq_bitlinear_w2a8 runs for x [M,K] and N outputs (a BQ_PATH_* value)."""
+    M, K = x.shape
+    path = I32(0)
+    st = lib().bq_bitlinear_w2a8_path(_ptr(x), _DTYPE[x.dtype], M, N, K, ctypes.byref(path))
+    _check(st, "bq_bitlinear_w2a8_path")
+    return path.value

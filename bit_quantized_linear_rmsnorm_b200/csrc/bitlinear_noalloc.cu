@@ -17,28 +17,27 @@
 // (different streams, no ordering between them) race on the array.
 #include <mutex>
 
-#include "../../include/bq.h"
-#include <cuda_runtime.h>
+#include "bq_internal.h"
 
 namespace {
 
 static __device__ __align__(256) uint8_t bq_noalloc_scratch[BQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-uint8_t *g_scratch[kMaxDevices] = {};
+uint8_t *g_scratch[bq::kMaxDevices] = {};
+uint64_t g_ctx[bq::kMaxDevices] = {};
 
 // In host code `bq_noalloc_scratch` names a host-side stand-in, not device
-// memory: the device address is looked up once per device, with that device
-// current, and cached.
-bq_status scratch_of_current_device(uint8_t **out) {
-    int d = -1;
-    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return BQ_ERR_CUDA;
+// memory: the device address is looked up once per device context, with that
+// device current, and cached against the context's identity.
+bq_status scratch_of(const bq::DevInfo &dev, uint8_t **out) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (g_scratch[d] == nullptr) {
+    const int d = dev.device;
+    if (g_scratch[d] == nullptr || g_ctx[d] != dev.ctx) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, bq_noalloc_scratch) != cudaSuccess || p == nullptr) return BQ_ERR_CUDA;
         g_scratch[d] = static_cast<uint8_t *>(p);
+        g_ctx[d] = dev.ctx;
     }
     *out = g_scratch[d];
     return BQ_OK;
@@ -50,11 +49,17 @@ extern "C" bq_status bq_bitlinear_w2a8_noalloc(const void *x, bq_dtype x_dtype, 
                                                const uint32_t *wpacked, const float *w_scale, int64_t N,
                                                const float *bias, float eps, bq_dtype out_dtype, void *out,
                                                bq_stream_t stream) {
-    if (M < 0 || N < 0 || K < 1) return BQ_ERR_INVALID_ARG;
-    const size_t need = bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0);
-    if (need > static_cast<size_t>(BQ_NOALLOC_SCRATCH_BYTES)) return BQ_ERR_WORKSPACE;
+    // the same argument checks as bq_bitlinear_w2a8, before anything else
+    bool empty = false;
+    bq_status st = bq::bitlinear_check_args(x, x_dtype, M, K, wpacked, w_scale, N, bias, eps, out_dtype, out, &empty);
+    if (st != BQ_OK || empty) return st;
+    if (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) > static_cast<size_t>(BQ_NOALLOC_SCRATCH_BYTES))
+        return BQ_ERR_WORKSPACE;
+    bq::DevInfo dev;
+    st = bq::current_device(&dev);
+    if (st != BQ_OK) return st;
     uint8_t *scratch = nullptr;
-    const bq_status st = scratch_of_current_device(&scratch);
+    st = scratch_of(dev, &scratch);
     if (st != BQ_OK) return st;
     return bq_bitlinear_w2a8(x, x_dtype, M, K, wpacked, w_scale, N, bias, eps, out_dtype, out, scratch,
                              static_cast<size_t>(BQ_NOALLOC_SCRATCH_BYTES), stream);

@@ -12,18 +12,46 @@
 __device__ uint32_t bq_dev_status_word = 0;
 
 namespace bq {
+
+uint64_t current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext *);
+    using GetId = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 1;
+    return static_cast<uint64_t>(id) + 2;
+}
+
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 DevInfo g_dev[kMaxDevices];
+
+}  // namespace
 
 bq_status current_device(DevInfo *out) {
     int d = -1;
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return BQ_ERR_CUDA;
+    uint64_t ctx = current_context_id();
     std::lock_guard<std::mutex> lk(g_mu);
     DevInfo &di = g_dev[d];
-    if (di.device != d) {
+    if (di.device != d || di.ctx != ctx) {
         DevInfo n;
         n.device = d;
         if (cudaDeviceGetAttribute(&n.num_sms, cudaDevAttrMultiProcessorCount, d) != cudaSuccess ||
@@ -34,9 +62,11 @@ bq_status current_device(DevInfo *out) {
         if (cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, d) != cudaSuccess)
             return BQ_ERR_CUDA;
         n.max_smem_optin = static_cast<size_t>(smem);
+        // (the lookup makes the device's primary context current if it was not)
         void *sym = nullptr;
         if (cudaGetSymbolAddress(&sym, bq_dev_status_word) != cudaSuccess) return BQ_ERR_CUDA;
         n.status = static_cast<uint32_t *>(sym);
+        n.ctx = ctx == 1 ? current_context_id() : ctx;
         di = n;
     }
     *out = di;
@@ -44,6 +74,8 @@ bq_status current_device(DevInfo *out) {
     if (di.cc_major != 10 || di.cc_minor != 0) return BQ_ERR_UNSUPPORTED;
     return BQ_OK;
 }
+
+namespace {
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -56,16 +88,57 @@ constexpr int64_t kMaxDim = 2147483647LL;  // tile indices are 32-bit
 constexpr int64_t kMaxKW4 = 65536;         // activation planes staged in shared memory
 constexpr int kGemvMaxM = 16;
 
-void bitlinear_layout(int64_t M, int64_t K, size_t *xq, size_t *sc, size_t *rs, size_t *total) {
-    *xq = 0;
-    *sc = align256(static_cast<size_t>(M) * static_cast<size_t>(K));
-    *rs = *sc + align256(static_cast<size_t>(M) * 4);
-    *total = *rs + align256(static_cast<size_t>(M) * 4);
+// Workspace of bq_bitlinear_w2a8: xq [M][K], act_scale [M], rowsum [M]; for
+// more than 16 tokens also, where the tensor-core path needs them, the packed
+// weight rows re-pitched to a multiple of 64 codes (the tensor copy wants
+// 16-byte row strides) and an output staging buffer with rows padded to 8
+// elements of up to 4 bytes.
+struct BitlinearLayout {
+    size_t xq, scale, rowsum, wpad, opad, total;
+};
+BitlinearLayout bitlinear_layout(int64_t M, int64_t N, int64_t K) {
+    BitlinearLayout l;
+    l.xq = 0;
+    l.scale = align256(static_cast<size_t>(M) * static_cast<size_t>(K));
+    l.rowsum = l.scale + align256(static_cast<size_t>(M) * 4);
+    l.wpad = l.rowsum + align256(static_cast<size_t>(M) * 4);
+    l.opad = l.wpad;
+    if (M > kGemvMaxM && K % 64 != 0)
+        l.opad += align256(static_cast<size_t>(N) * static_cast<size_t>((K + 63) / 64 * 4) * 4);
+    l.total = l.opad;
+    if (M > kGemvMaxM && N % 8 != 0) l.total += align256(static_cast<size_t>(M) * static_cast<size_t>((N + 7) / 8 * 8) * 4);
+    return l;
 }
 
 inline bq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA; }
 
+// Which kernels a BitLinear call of this shape runs (a bq_bitlinear_path).
+int bitlinear_path(const void *x, bq_dtype x_dtype, int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
+    if (M > kGemvMaxM) return gemm_uses_pair(true, BQ_W_NK, M, N, dev) ? BQ_PATH_TC_PAIR : BQ_PATH_TC_SINGLE;
+    if (decode_w2a8_supported(x, M, N, K, dev)) return decode_w2a8_kind(M, N, K, x_dtype, dev);
+    return BQ_PATH_ACT_QUANT_GEMV;
+}
+
 }  // namespace
+
+bq_status bitlinear_check_args(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const uint32_t *wpacked,
+                               const float *w_scale, int64_t N, const float *bias, float eps, bq_dtype out_dtype,
+                               void *out, bool *empty) {
+    *empty = false;
+    if (!act_dtype_ok(x_dtype) || !out_dtype_ok(out_dtype) || M < 0 || N < 0 || K < 1 || K > kMaxK ||
+        K % 16 != 0 || M > kMaxDim || N > kMaxDim || !std::isfinite(eps) || eps < 0.0f)
+        return BQ_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) {
+        *empty = true;
+        return BQ_OK;
+    }
+    if (x == nullptr || wpacked == nullptr || w_scale == nullptr || out == nullptr) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(wpacked, 16) || !aligned(out, 16) || !aligned(w_scale, 4) ||
+        !aligned(bias, 4))
+        return BQ_ERR_MISALIGNED;
+    return BQ_OK;
+}
+
 }  // namespace bq
 
 using namespace bq;
@@ -99,11 +172,8 @@ size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t gro
     switch (op) {
         case BQ_OP_WEIGHT_QUANT_TERNARY_PACK:
             return ternary_pack_workspace_bytes(N, K);
-        case BQ_OP_BITLINEAR_W2A8: {
-            size_t a, b, c, t;
-            bitlinear_layout(M, K, &a, &b, &c, &t);
-            return t;
-        }
+        case BQ_OP_BITLINEAR_W2A8:
+            return bitlinear_layout(M, N, K).total;
         case BQ_OP_LINEAR_W4_GROUPED:
             if (group_size <= 0) return 0;
             return linear_w4_workspace_bytes(M, N, K, group_size);
@@ -114,11 +184,10 @@ size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t gro
 
 void bq_bitlinear_workspace_layout(int64_t M, int64_t K, size_t *xq_offset, size_t *act_scale_offset,
                                    size_t *rowsum_offset) {
-    size_t a, b, c, t;
-    bitlinear_layout(M, K, &a, &b, &c, &t);
-    if (xq_offset) *xq_offset = a;
-    if (act_scale_offset) *act_scale_offset = b;
-    if (rowsum_offset) *rowsum_offset = c;
+    const BitlinearLayout l = bitlinear_layout(M, 0, K);
+    if (xq_offset) *xq_offset = l.xq;
+    if (act_scale_offset) *act_scale_offset = l.scale;
+    if (rowsum_offset) *rowsum_offset = l.rowsum;
 }
 
 bq_status bq_device_status(bq_stream_t stream, uint32_t *detail) {
@@ -221,41 +290,48 @@ bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_
 bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const uint32_t *wpacked,
                             const float *w_scale, int64_t N, const float *bias, float eps, bq_dtype out_dtype,
                             void *out, void *workspace, size_t workspace_bytes, bq_stream_t stream) {
-    if (!act_dtype_ok(x_dtype) || !out_dtype_ok(out_dtype) || M < 0 || N < 0 || K < 1 || K > kMaxK ||
-        K % 16 != 0 || M > kMaxDim || N > kMaxDim || !std::isfinite(eps) || eps < 0.0f)
-        return BQ_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return BQ_OK;
-    if (x == nullptr || wpacked == nullptr || w_scale == nullptr || out == nullptr) return BQ_ERR_INVALID_ARG;
-    size_t xq_off, sc_off, rs_off, need;
-    bitlinear_layout(M, K, &xq_off, &sc_off, &rs_off, &need);
-    if (workspace == nullptr || workspace_bytes < need) return BQ_ERR_WORKSPACE;
-    if (!aligned(workspace, 256) || !aligned(x, esize(x_dtype)) || !aligned(wpacked, 16) || !aligned(out, 16) ||
-        !aligned(w_scale, 4) || !aligned(bias, 4))
-        return BQ_ERR_MISALIGNED;
-    const bool gemm_path = M > kGemvMaxM;
-    // the tensor-core path stores rows of out and loads packed rows with TMA
-    if (gemm_path && ((N * esize(out_dtype)) % 16 != 0 || K % 64 != 0)) return BQ_ERR_MISALIGNED;
+    bool empty = false;
+    bq_status st = bitlinear_check_args(x, x_dtype, M, K, wpacked, w_scale, N, bias, eps, out_dtype, out, &empty);
+    if (st != BQ_OK || empty) return st;
+    const BitlinearLayout l = bitlinear_layout(M, N, K);
+    if (workspace == nullptr || workspace_bytes < l.total) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
     DevInfo dev;
-    const bq_status st = current_device(&dev);
+    st = current_device(&dev);
     if (st != BQ_OK) return st;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    int8_t *xq = reinterpret_cast<int8_t *>(ws + xq_off);
-    float *act_scale = reinterpret_cast<float *>(ws + sc_off);
-    int32_t *rowsum = reinterpret_cast<int32_t *>(ws + rs_off);
+    int8_t *xq = reinterpret_cast<int8_t *>(ws + l.xq);
+    float *act_scale = reinterpret_cast<float *>(ws + l.scale);
+    int32_t *rowsum = reinterpret_cast<int32_t *>(ws + l.rowsum);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (!gemm_path && decode_w2a8_supported(x, M, N, K, dev))
+    const int path = bitlinear_path(x, x_dtype, M, N, K, dev);
+    if (path == BQ_PATH_DECODE_STREAM || path == BQ_PATH_DECODE_MMA || path == BQ_PATH_DECODE_SMEM)
         return from_cuda(launch_decode_w2a8(x, x_dtype, M, K, eps, wpacked, w_scale, bias, N, out_dtype, out, xq,
                                             act_scale, rowsum, s, dev));
     cudaError_t e = launch_act_quant(x, x_dtype, M, K, K, eps, xq, K, act_scale, rowsum, s, dev);
     if (e != cudaSuccess) return BQ_ERR_CUDA;
-    if (!gemm_path)
+    if (path == BQ_PATH_ACT_QUANT_GEMV)
         return from_cuda(
             launch_gemv_w2a8(xq, K, act_scale, rowsum, wpacked, w_scale, bias, M, N, K, out_dtype, out, s, dev));
+    // tensor-core path: its tensor copies need 16-byte row pitches, so packed
+    // rows of K % 64 != 0 codes are re-pitched into the workspace first, and
+    // output rows of N * size % 16 != 0 bytes are staged there and copied out
+    const uint32_t *wrows = wpacked;
+    int64_t ldb = K / 16;
+    if (K % 64 != 0) {
+        uint32_t *wpad = reinterpret_cast<uint32_t *>(ws + l.wpad);
+        ldb = (K + 63) / 64 * 4;
+        e = cudaMemcpy2DAsync(wpad, static_cast<size_t>(ldb) * 4, wpacked, static_cast<size_t>(K / 16) * 4,
+                              static_cast<size_t>(K / 16) * 4, static_cast<size_t>(N), cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return BQ_ERR_CUDA;
+        wrows = wpad;
+    }
+    const bool stage_out = (N * esize(out_dtype)) % 16 != 0;
     GemmArgs g;
     g.a = xq;
     g.lda = K;
-    g.b = wpacked;
-    g.ldb = K / 16;
+    g.b = wrows;
+    g.ldb = ldb;
     g.b_packed2 = true;
     g.colscale = w_scale;
     g.rowscale = act_scale;
@@ -265,9 +341,56 @@ bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t 
     g.N = N;
     g.K = K;
     g.out_dtype = out_dtype;
-    g.out = out;
-    g.ldo = N;
-    return launch_gemm_tc(g, s, dev);
+    g.out = stage_out ? static_cast<void *>(ws + l.opad) : out;
+    g.ldo = stage_out ? (N + 7) / 8 * 8 : N;
+    st = launch_gemm_tc(g, s, dev);
+    if (st != BQ_OK || !stage_out) return st;
+    const size_t row = static_cast<size_t>(N) * esize(out_dtype);
+    return from_cuda(cudaMemcpy2DAsync(out, row, g.out, static_cast<size_t>(g.ldo) * esize(out_dtype), row,
+                                       static_cast<size_t>(M), cudaMemcpyDeviceToDevice, s));
+}
+
+bq_status bq_bitlinear_w2a8_path(const void *x, bq_dtype x_dtype, int64_t M, int64_t N, int64_t K, int *path) {
+    if (path == nullptr || !act_dtype_ok(x_dtype) || M < 1 || N < 1 || K < 1 || K % 16 != 0 || K > kMaxK ||
+        M > kMaxDim || N > kMaxDim)
+        return BQ_ERR_INVALID_ARG;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    *path = bitlinear_path(x, x_dtype, M, N, K, dev);
+    return BQ_OK;
+}
+
+bq_status bq_diag_gemm_withheld_arrival(const int8_t *x, const int8_t *w, const float *deq_scale,
+                                        const float *per_token_scale, void *out_bf16, uint64_t wait_limit_ns,
+                                        bq_stream_t stream) {
+    if (x == nullptr || w == nullptr || deq_scale == nullptr || per_token_scale == nullptr || out_bf16 == nullptr ||
+        wait_limit_ns < 100000ull || wait_limit_ns > 2000000000ull)
+        return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(out_bf16, 16) || !aligned(deq_scale, 32) ||
+        !aligned(per_token_scale, 4))
+        return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    // one 128 x 256 tile (a single CTA), two 128-wide K blocks: the second is withheld
+    GemmArgs g;
+    g.a = x;
+    g.lda = 256;
+    g.b = w;
+    g.ldb = 256;
+    g.colscale = deq_scale;
+    g.rowscale = per_token_scale;
+    g.M = 128;
+    g.N = 256;
+    g.K = 256;
+    g.out_dtype = BQ_BF16;
+    g.out = out_bf16;
+    g.ldo = 256;
+    g.wait_ns = wait_limit_ns;
+    g.withhold_kb = 1;
+    if (gemm_uses_pair(false, BQ_W_NK, g.M, g.N, dev)) return BQ_ERR_UNSUPPORTED;  // (a one-tile grid never pairs)
+    return launch_gemm_tc(g, static_cast<cudaStream_t>(stream), dev);
 }
 
 bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint32_t *qweight,

@@ -21,8 +21,6 @@ enum Site : uint32_t {
     SITE_GEMM_EPILOGUE = 3,
     SITE_GEMM_UNPACK = 4,
     SITE_GEMM_DRAIN = 5,
-    SITE_DECODE_FULL = 8,
-    SITE_DECODE_EMPTY = 9,
     SITE_INT4_PACK = 16,
     SITE_W4_STAGE = 17,
     SITE_W4_DRAIN = 18,
@@ -92,15 +90,16 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 
 // Waits for the phase with the given parity to complete.  Gives up (records
-// BQ_ERR_TIMEOUT at `site` and returns false) after kWaitLimitNs, or as soon
-// as another role of the CTA has raised *abort.
+// BQ_ERR_TIMEOUT at `site` and returns false) after `limit_ns` (kWaitLimitNs
+// unless the kernel takes its limit as an argument), or as soon as another
+// role of the CTA has raised *abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          uint32_t *status, uint32_t site) {
+                                          uint32_t *status, uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_sleep(bar, parity)) {
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report(status, BQ_ERR_TIMEOUT, site);
             *abort = 1;
             return false;
@@ -112,12 +111,12 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Same, polling without a suspend hint (for fine-grained hand-offs where a
 // suspended warp would wake up late).
 __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int *abort,
-                                               uint32_t *status, uint32_t site) {
+                                               uint32_t *status, uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report(status, BQ_ERR_TIMEOUT, site);
             *abort = 1;
             return false;
@@ -128,16 +127,24 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, vo
 
 // Time-bounded wait that ignores the abort flag (for groups of threads that
 // must take one common decision afterwards).
-__device__ __forceinline__ bool mbar_wait_timed(uint32_t bar, uint32_t parity, uint32_t *status, uint32_t site) {
+__device__ __forceinline__ bool mbar_wait_timed(uint32_t bar, uint32_t parity, uint32_t *status, uint32_t site,
+                                                uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_sleep(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             report(status, BQ_ERR_TIMEOUT, site);
             return false;
         }
     }
     return true;
+}
+
+// Bounded wait that records nothing (draining after another wait gave up).
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < limit_ns) {
+    }
 }
 
 // ----------------------------------------------------------------------------

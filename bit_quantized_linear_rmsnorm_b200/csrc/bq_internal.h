@@ -5,19 +5,61 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/bq.h"
 
 namespace bq {
 
+constexpr int kMaxDevices = 64;
+
 struct DevInfo {
     int device = -1;
+    uint64_t ctx = 0;            // identity of the device's current context (never 0 once known)
     int num_sms = 0;
     int cc_major = 0, cc_minor = 0;
     size_t max_smem_optin = 0;
     uint32_t *status = nullptr;  // device address of the status word
 };
+
+// Identity of the calling thread's current CUDA context (its driver-assigned
+// unique id, + 1 so that it is never 0); 1 when no context is current or the
+// driver entry points are unavailable.  Per-device state that a context owns
+// (symbol addresses, kernel attributes) is cached against this value, so a
+// context destroyed and re-created (cudaDeviceReset) is noticed.
+uint64_t current_context_id();
+
+// Opt-in to `bytes` of dynamic shared memory for kernel `kern`, once per
+// context and only when it grows (the attribute belongs to the context).
+struct SmemOptIn {
+    std::mutex mu;
+    uint64_t ctx[kMaxDevices] = {};
+    size_t bytes[kMaxDevices] = {};
+};
+inline cudaError_t smem_opt_in(SmemOptIn &c, const DevInfo &dev, const void *kern, size_t bytes) {
+    std::lock_guard<std::mutex> lk(c.mu);
+    const int d = dev.device;
+    if (c.ctx[d] == dev.ctx && bytes <= c.bytes[d]) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (e != cudaSuccess) return e;
+    if (c.ctx[d] != dev.ctx) c.bytes[d] = 0;
+    c.ctx[d] = dev.ctx;
+    if (bytes > c.bytes[d]) c.bytes[d] = bytes;
+    return cudaSuccess;
+}
+
+// The calling thread's current device, with its cached properties
+// (refreshed when the device's context changes).  BQ_ERR_UNSUPPORTED unless
+// it is an sm_100 device.
+bq_status current_device(DevInfo *out);
+
+// Every check of bq_bitlinear_w2a8 except the workspace ones; *empty is set
+// for a valid call with M == 0 or N == 0 (nothing to launch).
+bq_status bitlinear_check_args(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const uint32_t *wpacked,
+                               const float *w_scale, int64_t N, const float *bias, float eps, bq_dtype out_dtype,
+                               void *out, bool *empty);
 
 cudaError_t launch_act_quant(const void *x, bq_dtype xt, int64_t M, int64_t K, int64_t ldx, float eps,
                              int8_t *xq, int64_t ldq, float *act_scale, int32_t *rowsum, cudaStream_t s,
@@ -49,8 +91,12 @@ struct GemmArgs {
     bq_dtype out_dtype = BQ_BF16;
     void *out = nullptr;
     int64_t ldo = 0;
+    uint64_t wait_ns = 2000000000ull;  // limit of the kernel's bounded waits
+    int withhold_kb = -1;              // failure-detection check only (single-CTA kernel)
 };
 bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev);
+// Whether launch_gemm_tc runs a product of this shape on CTA pairs.
+bool gemm_uses_pair(bool packed, bq_wlayout b_layout, int64_t M, int64_t N, const DevInfo &dev);
 
 // Decode path (M <= 16) of the ternary linear: reads the packed weights once.
 cudaError_t launch_gemv_w2a8(const int8_t *xq, int64_t ldq, const float *act_scale, const int32_t *rowsum,
@@ -62,6 +108,9 @@ cudaError_t launch_gemv_w2a8(const int8_t *xq, int64_t ldq, const float *act_sca
 // activation quantization + bulk-streamed packed weights.  Writes xq,
 // act_scale and rowsum to the workspace as well.
 bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const DevInfo &dev);
+// Which decode kernel launch_decode_w2a8 runs for a supported shape
+// (BQ_PATH_DECODE_STREAM, BQ_PATH_DECODE_MMA or BQ_PATH_DECODE_SMEM).
+int decode_w2a8_kind(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev);
 cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
                                const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
                                int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,

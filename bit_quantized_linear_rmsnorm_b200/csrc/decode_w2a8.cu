@@ -960,12 +960,9 @@ template <int MT, int KBW, typename InT>
 cudaError_t launch_mma_t(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
     auto kern = decode_w2a8_mma_kernel<MT, KBW, InT>;
     const int smem = MmaLayout<MT, KBW>::bytes(a.K);
-    static int attr_smem[64] = {};
-    if (smem > attr_smem[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_smem[dev.device] = smem;
-    }
+    static SmemOptIn opt_in;
+    const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kMmaThreads);
@@ -989,12 +986,9 @@ cudaError_t launch_mma(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, 
 template <int MT, bool MMA, typename InT, typename OutT>
 cudaError_t launch_t(const DecodeArgs &a, int smem, const DevInfo &dev, cudaStream_t s, int grid) {
     auto kern = decode_w2a8_kernel<MT, MMA, InT, OutT>;
-    static int attr_smem[64] = {};
-    if (smem > attr_smem[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        attr_smem[dev.device] = smem;
-    }
+    static SmemOptIn opt_in;
+    const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kThreads);
@@ -1077,6 +1071,12 @@ bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const
     return Layout(static_cast<int>(K), mt_of(M), rb).total + 1024 <= dev.max_smem_optin;
 }
 
+int decode_w2a8_kind(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev) {
+    if (mma_stream_supported(M, N, K, dev)) return BQ_PATH_DECODE_MMA;
+    if (stream_supported(M, N, K, xt, dev)) return BQ_PATH_DECODE_STREAM;
+    return BQ_PATH_DECODE_SMEM;
+}
+
 cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
                                const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
                                int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,
@@ -1100,11 +1100,12 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.rb = rb;
     a.status = dev.status;
     a.out_dtype = out_dtype;
-    if (mma_stream_supported(M, N, K, dev)) {
+    const int kind = decode_w2a8_kind(M, N, K, xt, dev);
+    if (kind == BQ_PATH_DECODE_MMA) {
         if (xt == BQ_BF16) return launch_mma<__nv_bfloat16>(a, dev, s, grid);
         return launch_mma<float>(a, dev, s, grid);
     }
-    if (stream_supported(M, N, K, xt, dev)) {
+    if (kind == BQ_PATH_DECODE_STREAM) {
         if (xt == BQ_BF16) return launch_stream_out<__nv_bfloat16>(a, out_dtype, static_cast<int>(M), s, grid);
         return launch_stream_out<float>(a, out_dtype, static_cast<int>(M), s, grid);
     }

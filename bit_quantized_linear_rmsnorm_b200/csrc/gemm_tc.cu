@@ -77,6 +77,8 @@ struct GemmDev {
     const float *bias;
     int M, N, K;
     uint32_t *status;
+    uint64_t wait_ns;  // limit of every bounded wait
+    int withhold_kb;   // (failure-detection check only) K block of the first tile whose copies are never issued
 };
 
 template <typename OutT>
@@ -200,12 +202,14 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             items.tile(item, m0, n0, half);
             const uint32_t b_bytes = half ? B_BYTES / 2 : B_BYTES;
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
+                if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER, p.wait_ns)) {
                     ok = false;
                     break;
                 }
                 const uint32_t a_dst = sbase + C::OFF_A + stage * A_BYTES;
-                if constexpr (PACKED) {
+                if (kb == p.withhold_kb && item == static_cast<int>(blockIdx.x)) {
+                    // failure-detection check: this stage's barrier never completes
+                } else if constexpr (PACKED) {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + P_BYTES);
                     tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
                     tma_load_2d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * (BK / 16), n0, full(stage));
@@ -227,16 +231,11 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                 }
             }
         }
-        if (!ok) {
-            // let the copies already issued land before the CTA goes away
-            for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i) {
-                const uint32_t bar = full(static_cast<int>(i % S));
-                const uint32_t par = static_cast<uint32_t>((i / S) & 1);
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(bar, par) && globaltimer_ns() - t0 < kWaitLimitNs) {
-                }
-            }
-        }
+        // let the copies already issued land before the CTA can go away: at
+        // once when the MMA consumed them, bounded when another role gave up
+        // (a withheld block's barrier runs to the limit)
+        for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i)
+            mbar_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1), p.wait_ns);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
         constexpr uint32_t idesc = idesc_i8(BM, BN, true, !PACKED, B_KN);
@@ -249,19 +248,19 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             const uint32_t id = item < items.big ? idesc : idesc_half;
             const int abuf = t & 1;
             const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
-            if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA)) {
+            if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA, p.wait_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t d_tmem = tbase + static_cast<uint32_t>(abuf * BN);
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                if (!mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA, p.wait_ns)) {
                     ok = false;
                     break;
                 }
                 if constexpr (PACKED) {
-                    if (!mbar_wait(bready(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                    if (!mbar_wait(bready(stage), phase, abort_flag, p.status, SITE_GEMM_MMA, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -287,9 +286,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         if (!ok) {
             // wait until every MMA issued so far has completed
             tc_commit(drain);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
+            mbar_drain(drain, 0, p.wait_ns);
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ epilogue
@@ -322,7 +319,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             // one lane per warp waits (polling by 128 threads would take shared-
             // memory bandwidth from the TMA and MMA), the warp follows it
             bool ok = true;
-            if (lane == 0) ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE);
+            if (lane == 0) ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE, p.wait_ns);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok && lane == 0) {
                 atomicOr(epi_fail, 1);
@@ -399,7 +396,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         for (int item = blockIdx.x; item < items.count && ok; item += gridDim.x) {
             for (int kb = 0; kb < nkb; ++kb) {
                 bool got = true;
-                if (lane == 0) got = mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK);
+                if (lane == 0) got = mbar_wait(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK, p.wait_ns);
                 if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
                     ok = false;
                     break;
@@ -624,7 +621,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             const uint32_t b_bytes = half ? PB_BYTES / 2 : PB_BYTES;
             const int nb0 = n0 + (half ? BN / 4 : BN / 2) * static_cast<int>(rank);  // this CTA's B rows
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait_spin(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER)) {
+                if (!mbar_wait_spin(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -652,11 +649,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         if (!ok && (leader || PACKED)) {
             // let the copies this full barrier counts land (both CTAs' on the leader without 2-bit codes)
             for (int64_t i = issued > S ? issued - S : 0; i < issued; ++i) {
-                const uint32_t bar = full(static_cast<int>(i % S));
-                const uint32_t par = static_cast<uint32_t>((i / S) & 1);
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(bar, par) && globaltimer_ns() - t0 < kWaitLimitNs) {
-                }
+                mbar_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1), p.wait_ns);
             }
         }
     } else if (warp == 1 && lane == 0 && leader) {
@@ -671,7 +664,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             const uint32_t id = item < big ? idesc : idesc_half;
             const int abuf = t & 1;
             const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
-            if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA)) {
+            if (!mbar_wait(tempty(abuf), aphase ^ 1u, abort_flag, p.status, SITE_GEMM_MMA, p.wait_ns)) {
                 ok = false;
                 break;
             }
@@ -679,7 +672,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             const uint32_t d_tmem = tbase + static_cast<uint32_t>(abuf * BN);
             for (int kb = 0; kb < nkb; ++kb) {
                 // (polled: the last arrival is often the peer CTA's)
-                if (!mbar_wait_spin(PACKED ? bready(stage) : full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA)) {
+                if (!mbar_wait_spin(PACKED ? bready(stage) : full(stage), phase, abort_flag, p.status, SITE_GEMM_MMA, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -700,9 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         }
         if (!ok) {
             tc_commit_pair(drain);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
+            mbar_drain(drain, 0, p.wait_ns);
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ epilogue (both CTAs)
@@ -731,7 +722,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             named_bar_sync(1, 128);
 
             bool ok = true;
-            if (lane == 0) ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE);
+            if (lane == 0) ok = mbar_wait_timed(tfull(abuf), aphase, p.status, SITE_GEMM_EPILOGUE, p.wait_ns);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok && lane == 0) {
                 atomicOr(epi_fail, 1);
@@ -806,7 +797,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             const int words = (item < big ? 128 : 64) * (BK / 16);  // packed words of this CTA's rows
             for (int kb = 0; kb < nkb; ++kb) {
                 bool got = true;
-                if (lane == 0) got = mbar_wait_spin(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK);
+                if (lane == 0) got = mbar_wait_spin(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK, p.wait_ns);
                 if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
                     ok = false;
                     break;
@@ -877,13 +868,9 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
                    cudaStream_t s, const DevInfo &dev) {
     using C = Cfg<PACKED>;
     auto kern = gemm_tc_kernel<PACKED, B_KN, OutT>;
-    static bool attr_set[64] = {};  // once per device (also keeps later calls capture-safe)
-    if (!attr_set[dev.device]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
-            cudaSuccess)
-            return BQ_ERR_CUDA;
-        attr_set[dev.device] = true;
-    }
+    static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
+    if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
+        return BQ_ERR_CUDA;
     const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
     GemmDev p;
@@ -895,6 +882,8 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
     p.N = static_cast<int>(g.N);
     p.K = static_cast<int>(g.K);
     p.status = dev.status;
+    p.wait_ns = g.wait_ns;
+    p.withhold_kb = g.withhold_kb;
     kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mBh, mO, p);
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
@@ -904,13 +893,9 @@ bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMa
                       const CUtensorMap &mO, cudaStream_t s, const DevInfo &dev) {
     using C = PairCfg<PACKED>;
     auto kern = gemm_pair_kernel<PACKED, OutT>;
-    static bool attr_set[64] = {};  // once per device (also keeps later calls capture-safe)
-    if (!attr_set[dev.device]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
-            cudaSuccess)
-            return BQ_ERR_CUDA;
-        attr_set[dev.device] = true;
-    }
+    static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
+    if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
+        return BQ_ERR_CUDA;
     const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN);
     const int64_t pairs = std::min<int64_t>(tiles, dev.num_sms / 2);
     GemmDev p;
@@ -922,17 +907,15 @@ bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMa
     p.N = static_cast<int>(g.N);
     p.K = static_cast<int>(g.K);
     p.status = dev.status;
+    p.wait_ns = g.wait_ns;
+    p.withhold_kb = -1;  // (the check runs on a single CTA)
     kern<<<static_cast<unsigned>(2 * pairs), C::kThreads, C::SMEM, s>>>(mA, mB128, mB64, mO, p);
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 // The pair kernel takes products with K-major (or 2-bit packed) weights that
 // fill at least one wave of CTA pairs with 256 x 256 tiles.
-bool use_pair(const GemmArgs &g, const DevInfo &dev) {
-    if ((!g.b_packed2 && g.b_layout == BQ_W_KN) || dev.num_sms < 2) return false;
-    const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN);
-    return tiles >= dev.num_sms / 2;
-}
+bool use_pair(const GemmArgs &g, const DevInfo &dev) { return gemm_uses_pair(g.b_packed2, g.b_layout, g.M, g.N, dev); }
 
 template <typename OutT>
 bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
@@ -962,6 +945,12 @@ bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
 }
 
 }  // namespace
+
+bool gemm_uses_pair(bool packed, bq_wlayout b_layout, int64_t M, int64_t N, const DevInfo &dev) {
+    if ((!packed && b_layout == BQ_W_KN) || dev.num_sms < 2) return false;
+    const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+    return tiles >= dev.num_sms / 2;
+}
 
 bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) {
     CUtensorMap mA, mB, mBh, mO;

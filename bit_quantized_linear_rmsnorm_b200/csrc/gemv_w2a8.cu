@@ -191,12 +191,10 @@ cudaError_t launch_mt(const int8_t *xq, int64_t ldq, const float *act_scale, con
                       int64_t K, OutT *out, cudaStream_t s, const DevInfo &dev) {
     const size_t smem = static_cast<size_t>(M) * static_cast<size_t>(K);
     auto kern = gemv_w2a8_kernel<MT, OutT>;
-    static size_t attr_smem[64] = {};  // largest opt-in set so far, per device
-    if (smem > 48 * 1024 && smem > attr_smem[dev.device]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+    static SmemOptIn opt_in;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), smem);
         if (e != cudaSuccess) return e;
-        attr_smem[dev.device] = smem;
     }
     const int64_t rows_per_block = static_cast<int64_t>(kWarps) * kRows;
     int64_t grid = (N + rows_per_block - 1) / rows_per_block;

@@ -236,12 +236,10 @@ cudaError_t launch_pass(const uint32_t *qweight, const uint16_t *scales, const u
                         cudaStream_t s, const DevInfo &dev) {
     const size_t smem = static_cast<size_t>(3 * MT) * static_cast<size_t>(K);
     auto kern = w4_linear_dp4a_kernel<MT, VEC>;
-    static size_t attr_smem[64] = {};  // largest opt-in set so far, per device
-    if (smem > 48 * 1024 && smem > attr_smem[dev.device]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    static SmemOptIn opt_in;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), smem);
         if (e != cudaSuccess) return e;
-        attr_smem[dev.device] = smem;
     }
     int64_t grid = (N + kWarps - 1) / kWarps;
     const int64_t cap = static_cast<int64_t>(dev.num_sms) * 8;
@@ -720,12 +718,11 @@ cudaError_t launch_w4_decode(const float *x, int64_t K, const uint32_t *qweight,
     a.status = dev.status;
     const int smem = static_cast<int>(W4Layout(a.K, a.gs, a.nslots, a.rows_cap).total);
     auto kern = K == 2048 ? w4_decode_kernel<1> : K == 4096 ? w4_decode_kernel<2> : w4_decode_kernel<4>;
-    static int attr_smem[3][64] = {};
-    int &done = attr_smem[K == 2048 ? 0 : K == 4096 ? 1 : 2][dev.device];
-    if (smem > 48 * 1024 && smem > done) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static SmemOptIn opt_in[3];
+    if (smem > 48 * 1024) {
+        const cudaError_t e = smem_opt_in(opt_in[K == 2048 ? 0 : K == 4096 ? 1 : 2], dev,
+                                          reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
         if (e != cudaSuccess) return e;
-        done = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(a.nbox, dev.num_sms)));

@@ -331,9 +331,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         }
         if (!ok) {  // wait until every MMA issued so far has completed
             tc_commit(drain);
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-            }
+            mbar_drain(drain, 0, kWaitLimitNs);
         }
     } else if (warp >= 8 && warp < 16) {
         // ------------------------------------------------------------ epilogue
@@ -458,13 +456,9 @@ cudaError_t launch_w4_tc(const float *x, int64_t M, int64_t K, const uint32_t *q
     a.S = tc_slices(K);
     a.R = tc_row_tiles(N, K, dev);
     a.status = dev.status;
-    static bool attr_set[64] = {};
-    if (!attr_set[dev.device]) {
-        e = cudaFuncSetAttribute(w4_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(TcLayout::SMEM));
-        if (e != cudaSuccess) return e;
-        attr_set[dev.device] = true;
-    }
+    static SmemOptIn opt_in;
+    e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(w4_tc_kernel), static_cast<size_t>(TcLayout::SMEM));
+    if (e != cudaSuccess) return e;
     e = launch_pdl(w4_tc_kernel, static_cast<unsigned>(a.R * a.S), kTcThreads, TcLayout::SMEM, s, a);
     if (e != cudaSuccess) return e;
     const int64_t total = N * M;

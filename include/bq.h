@@ -24,6 +24,10 @@
  *    (a nibble > 15) is recorded in a per-device status word and the kernel
  *    returns early; read and clear it with bq_device_status().
  *  - Inputs must be finite.  Rounding is to nearest, ties to even.
+ *  - Per-device state (the status word's and the static scratch's device
+ *    addresses, kernel shared-memory opt-ins) is cached against the device's
+ *    current context and looked up again when that context changes (e.g.
+ *    after cudaDeviceReset); calls racing with a reset are not supported.
  *
  * Data formats
  * ------------
@@ -157,19 +161,39 @@ bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_
  *   acc[m,n] = sum_k xq[m,k] * w_q[n,k]              (exact int32)
  *   out[m,n] = (float(acc) * act_scale[m]) * gamma  (+ bias[n])
  *
- * x: dense [M][K] of x_dtype BQ_F32 or BQ_BF16; K % 16 == 0.  wpacked,
- * w_scale: as written by bq_weight_quant_ternary_pack.  bias: fp32 [N] or
- * NULL (the page disables it by default).  out: dense [M][N] of out_dtype.
- * M <= 16 runs the bandwidth-bound decode kernel, larger M the tcgen05 GEMM
- * that unpacks the 2-bit tiles in shared memory.  workspace: at least
- * bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) bytes, 256-byte
- * aligned; bq_bitlinear_workspace_layout() gives where xq [M][K] int8,
- * act_scale fp32 [M] and rowsum int32 [M] sit, so they can be read back.
+ * x: dense [M][K] of x_dtype BQ_F32 or BQ_BF16; K % 16 == 0, any N.
+ * wpacked, w_scale: as written by bq_weight_quant_ternary_pack.  bias: fp32
+ * [N] or NULL (the page disables it by default).  out: dense [M][N] of
+ * out_dtype.  M <= 16 runs a bandwidth-bound decode kernel, larger M the
+ * tcgen05 GEMM that unpacks the 2-bit tiles in shared memory (for K % 64 != 0
+ * it first copies the packed rows to a 16-byte pitch in the workspace, and
+ * for N * size(out) % 16 != 0 it stages the output rows there and copies
+ * them out; bq_bitlinear_w2a8_path() tells which kernels a shape runs).
+ * workspace: at least bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0)
+ * bytes, 256-byte aligned; bq_bitlinear_workspace_layout() gives where
+ * xq [M][K] int8, act_scale fp32 [M] and rowsum int32 [M] sit, so they can
+ * be read back.
  */
 bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t K,
                             const uint32_t *wpacked, const float *w_scale, int64_t N,
                             const float *bias, float eps, bq_dtype out_dtype, void *out,
                             void *workspace, size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Which kernels bq_bitlinear_w2a8 runs for a shape on the current device (for
+ * tests and profiling; the choice depends on M, N, K, the activation dtype,
+ * the 16-byte alignment of x and the device's SM count).  *path receives a
+ * bq_bitlinear_path.  Needs an sm_100 device (else BQ_ERR_UNSUPPORTED).
+ */
+typedef enum {
+    BQ_PATH_DECODE_STREAM = 1,  /* 1 token: activation quant fused, dp4a register-streaming kernel    */
+    BQ_PATH_DECODE_MMA = 2,     /* 2..16 tokens, K 2048/4096: fused, mma.sync register-streaming      */
+    BQ_PATH_DECODE_SMEM = 3,    /* other M <= 16 with K % 512 == 0: fused, shared-memory staged kernel */
+    BQ_PATH_ACT_QUANT_GEMV = 4, /* other M <= 16: activation-quant kernel, then a split GEMV kernel    */
+    BQ_PATH_TC_SINGLE = 5,      /* M > 16: activation quant, tcgen05 GEMM on single CTAs               */
+    BQ_PATH_TC_PAIR = 6         /* M > 16: activation quant, tcgen05 GEMM on CTA pairs (cta_group::2)  */
+} bq_bitlinear_path;
+bq_status bq_bitlinear_w2a8_path(const void *x, bq_dtype x_dtype, int64_t M, int64_t N, int64_t K, int *path);
 
 /*
  * Grouped affine INT4 linear with fp32 activations.
@@ -201,21 +225,24 @@ bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint3
  * would synchronize the device.  The pages have no counterpart of this entry
  * point.
  *
- * The caller passes inputs and outputs as for bq_bitlinear_w2a8.  The scratch
- * (int8 activations, per-token scales, row sums) lives in one static device
- * array of BQ_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
- * library holds until the process exits.  A call whose scratch would exceed
- * it (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) >
- * BQ_NOALLOC_SCRATCH_BYTES, i.e. M*K above about 2 MB) returns
- * BQ_ERR_WORKSPACE before launching anything.  The call never allocates
- * (no cudaMalloc / cudaFree, no allocating library routine).
+ * The caller passes inputs and outputs as for bq_bitlinear_w2a8, and the
+ * arguments are checked in the same way and order, with the same results.
+ * The scratch (int8 activations, per-token scales, row sums, and for more
+ * than 16 tokens the re-pitched weights or staged outputs of ragged shapes)
+ * lives in one static device array of BQ_NOALLOC_SCRATCH_BYTES bytes, which
+ * every GPU that loads the library holds until the process exits.  A valid
+ * call whose scratch would exceed it (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8,
+ * M, N, K, 0) > BQ_NOALLOC_SCRATCH_BYTES, i.e. M*K above about 2 MB) returns
+ * BQ_ERR_WORKSPACE before launching anything.  The call never allocates (no
+ * cudaMalloc / cudaFree, no allocating library routine).
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls on a device share the
- * array and it keeps the last call's contents; each call writes all the
- * scratch it reads, so nothing needs clearing, but calls that overlap on the
- * GPU (unordered streams) race on it.
+ * The first call on a device (and the first after its context was destroyed
+ * and re-created) looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any
+ * stream capture.  All calls on a device share the array and it keeps the
+ * last call's contents; each call writes all the scratch it reads, so nothing
+ * needs clearing, but calls that overlap on the GPU (unordered streams) race
+ * on it.
  */
 #define BQ_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
 bq_status bq_bitlinear_w2a8_noalloc(const void *x, bq_dtype x_dtype, int64_t M, int64_t K,
@@ -240,6 +267,23 @@ const char *bq_status_string(bq_status status);
  * NULL) receives the raw word (bits 0-7 status, bits 8-31 the site).
  */
 bq_status bq_device_status(bq_stream_t stream, uint32_t *detail);
+
+/*
+ * Failure-detection check (diagnostic; the pages have no counterpart).  Runs
+ * the single-CTA W8A8 tensor-core GEMM kernel on one 128 x 256 tile:
+ * x int8 [128][256], w int8 [256][256] (BQ_W_NK), deq_scale fp32 [256]
+ * (32-byte aligned), per_token_scale fp32 [128], out bf16 [128][256], with
+ * every bounded wait limited to wait_limit_ns (1e5 .. 2e9) and the producer
+ * withholding the copies of the second K block.  The MMA issuer's and the
+ * epilogue's waits on that block run out: the kernel records BQ_ERR_TIMEOUT
+ * (site: MMA issuer 2 or epilogue 3) in the device status word, waits for
+ * its own copies and MMAs in flight, frees its tensor memory and returns
+ * within a few limits; no fault, no trap, the context stays usable.  `out`
+ * is left partly unwritten.  Read the outcome with bq_device_status().
+ */
+bq_status bq_diag_gemm_withheld_arrival(const int8_t *x, const int8_t *w, const float *deq_scale,
+                                        const float *per_token_scale, void *out_bf16, uint64_t wait_limit_ns,
+                                        bq_stream_t stream);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 int bq_version(void);

@@ -55,6 +55,8 @@ def lib():
             "bq_oracle_int4_unpack": (None, [P, I64, I64, P]),
             "bq_oracle_half_to_double": (F64, [ctypes.c_uint16]),
             "bq_oracle_gemm_i8_pertoken": (I64, [P, I64, P, ctypes.c_int, I64, P, P, P, I64, I64, I64, P]),
+            "bq_oracle_gemm_i8_pertoken_batched": (I64, [P, I64, I64, ctypes.c_int, P, ctypes.c_int, I64, I64, P, I64,
+                                                          P, I64, P, I64, I64, I64, I64, P]),
             "bq_oracle_bitlinear_from_codes": (None, [P, P, P, F64, P, I64, I64, I64, P, P]),
             "bq_oracle_linear_w4_grouped": (None, [P, I64, I64, P, P, P, P, I64, I64, P]),
         }
@@ -174,6 +176,28 @@ def gemm_i8_pertoken(x, w, deq_scale, per_token_scale, bias=None, layout: int = 
     out = np.empty((M, N), np.float64)
     ovf = lib().bq_oracle_gemm_i8_pertoken(_p(x), K, _p(w), int(layout), w.shape[1], _p(deq), _p(pts),
                                            _p(b), M, N, K, _p(out))
+    return out, int(ovf)
+
+
+def gemm_i8_pertoken_batched(x, w, deq_scale, per_token_scale, bias=None, layout: int = 0, trans_a: bool = False,
+                             shared_scales: bool = True):
+    """Batched per-token W8A8 matmul.  x int8 [B,M,K] ([B,K,M] with trans_a);
+    w int8 [B,N,K] (layout 0) or [B,K,N] (layout 1); deq_scale [N] and
+    per_token_scale [M] shared by every batch (shared_scales) or [B,N] and
+    [B,M].  Returns (out f64 [B,M,N], number of accumulators outside int32)."""
+    x = _c(x, np.int8)
+    w = _c(w, np.int8)
+    B = x.shape[0]
+    M, K = (x.shape[2], x.shape[1]) if trans_a else (x.shape[1], x.shape[2])
+    N = w.shape[1] if layout == 0 else w.shape[2]
+    deq = _c(deq_scale, np.float32)
+    pts = _c(per_token_scale, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((B, M, N), np.float64)
+    ovf = lib().bq_oracle_gemm_i8_pertoken_batched(
+        _p(x), x.shape[2], x.shape[1] * x.shape[2], int(bool(trans_a)), _p(w), int(layout), w.shape[2],
+        w.shape[1] * w.shape[2], _p(deq), 0 if shared_scales else N, _p(pts), 0 if shared_scales else M, _p(b),
+        B, M, N, K, _p(out))
     return out, int(ovf)
 
 

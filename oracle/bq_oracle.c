@@ -272,6 +272,46 @@ int64_t bq_oracle_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w
 }
 
 /*
+ * Batched and transposed forms of the per-token W8A8 matmul ([ATB] Input /
+ * Output tables: x [m,k] or [batch,m,k], weight [k,n] or [batch,k,n],
+ * output [batch,m,n]; Parameters: transposeA and transposeB).  For each batch
+ * b the 2-D formula above, with
+ *
+ *   x(b,m,k)      = x[b*sx + m*ldx + k]       (trans_a = 0: x is [M,K] per batch)
+ *                 = x[b*sx + k*ldx + m]       (trans_a = 1: x is stored [K,M])
+ *   weight(b,k,n) = w[b*sw + n*ldw + k]       (layout 0, [N,K])
+ *                 = w[b*sw + k*ldw + n]       (layout 1, [K,N])
+ *   deqScale(b,n) = deq[b*sdeq + n],  perTokenScale(b,m) = pts[b*spts + m]
+ *
+ * (sdeq = spts = 0 is the tables' reading: one [n] and one [m] vector shared
+ * by every batch; the strides N and M give one per batch).  out is dense
+ * [batch,M,N].  Returns the number of accumulators outside int32.
+ */
+int64_t bq_oracle_gemm_i8_pertoken_batched(const int8_t *x, int64_t ldx, int64_t sx, int trans_a,
+                                           const int8_t *w, int layout, int64_t ldw, int64_t sw,
+                                           const float *deq, int64_t sdeq, const float *pts, int64_t spts,
+                                           const float *bias, int64_t batch, int64_t M, int64_t N,
+                                           int64_t K, double *out)
+{
+    int64_t overflow = 0;
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t n = 0; n < N; ++n) {
+                int64_t acc = 0;
+                for (int64_t k = 0; k < K; ++k) {
+                    int64_t xv = trans_a ? x[b * sx + k * ldx + m] : x[b * sx + m * ldx + k];
+                    int64_t wv = layout == 0 ? w[b * sw + n * ldw + k] : w[b * sw + k * ldw + n];
+                    acc += xv * wv;
+                }
+                if (acc > 2147483647LL || acc < -2147483648LL) ++overflow;
+                double v = ((double)acc * (double)deq[b * sdeq + n]) * (double)pts[b * spts + m];
+                if (bias) v += (double)bias[n];
+                out[(b * M + m) * N + n] = v;
+            }
+    return overflow;
+}
+
+/*
  * BitLinear steps 4-5 from the quantized operands ([BitLinear] forward:
  * F.linear(x_q, w_q) then out * act_scale * w_scale):
  *

@@ -127,9 +127,55 @@ def test_bitlinear_rejects(L):
     assert call(work=None) == bq.BQ_ERR_WORKSPACE
     assert call(nbytes=16) == bq.BQ_ERR_WORKSPACE
     assert call(work=ctypes.c_void_p(0x10040)) == bq.BQ_ERR_MISALIGNED
-    assert call(N=61) == bq.BQ_ERR_MISALIGNED     # tensor-core path stores whole 16-byte rows
-    assert call(K=144) == bq.BQ_ERR_MISALIGNED    # tensor-core path loads packed rows with TMA
+    assert call(x=ODD) == bq.BQ_ERR_MISALIGNED
+    assert call(out=ctypes.c_void_p(0x10008)) == bq.BQ_ERR_MISALIGNED
     assert call(M=0) == bq.BQ_OK
+    assert call(N=0, wp=None) == bq.BQ_OK
+    # ragged N and K % 64 != 0 are valid at any M (the tensor-core path stages
+    # them through the workspace), so validation lets them through
+    for kw in (dict(N=61), dict(K=144), dict(N=61, K=144, od=bq.BQ_F16)):
+        assert call(**kw) not in (bq.BQ_ERR_INVALID_ARG, bq.BQ_ERR_MISALIGNED, bq.BQ_ERR_WORKSPACE), kw
+
+
+def test_bitlinear_workspace_grows_for_tensor_core_tails(L):
+    base = bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, 300, 64, 128)
+    assert bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, 300, 61, 128) >= base + 300 * 64 * 4
+    assert bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, 300, 64, 144) >= base + 64 * 192 // 4
+    # up to 16 tokens (decode kernels) nothing is staged
+    xo, so, ro = bq.bq_bitlinear_workspace_layout(16, 144)
+    assert bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, 16, 61, 144) == ro + 256
+
+
+def test_noalloc_checks_arguments_like_the_workspace_entry_point(L):
+    """bq_bitlinear_w2a8_noalloc answers every invalid call exactly as
+    bq_bitlinear_w2a8 does (minus the workspace, which it does not take),
+    before it looks at its scratch limit or at the device."""
+    ok = dict(x=FAKE, xt=bq.BQ_BF16, M=32, K=128, wp=FAKE, ws_=FAKE, N=64, bias=None, eps=1e-5, od=bq.BQ_BF16,
+              out=FAKE)
+
+    def both(**kw):
+        a = dict(ok, **kw)
+        na = L.bq_bitlinear_w2a8_noalloc(a["x"], a["xt"], a["M"], a["K"], a["wp"], a["ws_"], a["N"], a["bias"],
+                                         a["eps"], a["od"], a["out"], None)
+        wa = L.bq_bitlinear_w2a8(a["x"], a["xt"], a["M"], a["K"], a["wp"], a["ws_"], a["N"], a["bias"], a["eps"],
+                                 a["od"], a["out"], FAKE, 1 << 40, None)
+        return na, wa
+    # invalid arguments, even where the scratch would also be too small
+    for kw in (dict(K=40), dict(K=131072 + 16, M=4096), dict(K=131088), dict(xt=bq.BQ_F16), dict(od=7),
+               dict(eps=float("nan")), dict(eps=-1.0), dict(M=-1), dict(x=None), dict(out=None), dict(ws_=None),
+               dict(M=4096, K=4096, x=None)):
+        na, wa = both(**kw)
+        assert na == wa == bq.BQ_ERR_INVALID_ARG, (kw, na, wa)
+    for kw in (dict(x=ODD), dict(out=ctypes.c_void_p(0x10008)), dict(bias=ODD), dict(M=4096, K=4096, x=ODD)):
+        na, wa = both(**kw)
+        assert na == wa == bq.BQ_ERR_MISALIGNED, (kw, na, wa)
+    # valid empty calls: nothing to do
+    for kw in (dict(M=0), dict(N=0), dict(M=0, x=None, out=None)):
+        na, wa = both(**kw)
+        assert na == wa == bq.BQ_OK, (kw, na, wa)
+    # only a valid call too large for the static scratch gets BQ_ERR_WORKSPACE
+    na, _ = both(M=1024, K=4096)
+    assert na == bq.BQ_ERR_WORKSPACE
 
 
 def test_linear_w4_rejects(L):

@@ -16,7 +16,8 @@ import torch
 import bit_quantized_linear_rmsnorm_b200 as bq
 import oracle
 import synth
-from gpu_helpers import assert_codes, assert_out, bf16_dev, dev, host, padded, tie_band
+from gpu_helpers import (assert_codes, assert_out, bf16_dev, bitlinear_expected, bitlinear_rel32, dev, host,
+                         padded, tie_band)
 
 pytestmark = pytest.mark.gpu
 
@@ -250,12 +251,15 @@ def test_gemm_closed_form_all_ones():
 
 # ------------------------------------------------------------- BitLinear
 
-def _bitlinear_check(x_f32, x_dev, w_f32, N, out, bias, what, rows=None):
+def _bitlinear_check(x_f32, x_dev, w_f32, N, out, bias, what, rows=None, path=None):
     """Runs the GPU pack + BitLinear, then checks the workspace codes and the
-    output against the oracle computed from the same inputs."""
+    output against the oracle computed from the same inputs (and, when given,
+    which kernels the call ran)."""
     eps = 1e-5
     M, K = x_f32.shape
     wp, ws_ = bq.bq_weight_quant_ternary_pack(dev(w_f32))
+    if path is not None:
+        assert bq.bq_bitlinear_w2a8_path(x_dev, N) == path, what
     nbytes = bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, M, N, K)
     work = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
     b = None if bias is None else dev(bias)
@@ -265,20 +269,11 @@ def _bitlinear_check(x_f32, x_dev, w_f32, N, out, bias, what, rows=None):
     g_xq = host(work[xo:xo + M * K].view(torch.int8).view(M, K))
     g_sc = host(work[so:so + 4 * M].view(torch.float32))
     sel = np.arange(M) if rows is None else rows
-    a = oracle.act_quant(x_f32[sel], eps, want_pre=True)
-    t = oracle.ternary_quant(w_f32, want_pre=True)
+    ref, extra, scale, a, t = bitlinear_expected(x_f32, w_f32, bias, eps, rows=sel)
     assert_codes(g_xq[sel], a["xq"], a["pre"], what + " xq")
     np.testing.assert_allclose(g_sc[sel], a["act_scale"], rtol=1e-5)
-    ref = oracle.bitlinear_from_codes(a["xq"], a["act_scale"], t["wq"], t["gamma"], bias)
-    # codes in the tie band may round either way: widen by what they can move
-    xband = tie_band(a["pre"]).astype(np.float64)
-    wband = tie_band(t["pre"]).astype(np.float64)
-    extra = (xband @ np.abs(t["wq"]).T.astype(np.float64) + np.abs(a["xq"]).astype(np.float64) @ wband.T) \
-        * a["act_scale"][:, None] * t["gamma"]
-    scale = None
-    if bias is not None:
-        scale = np.abs(ref - bias.astype(np.float64)) + np.abs(bias.astype(np.float64))
-    assert_out(host(o)[sel], ref, _TORCH_OUT[out], what, extra=extra, scale=scale)
+    rel32 = bitlinear_rel32(g_sc[sel], a["act_scale"], host(ws_)[0], t["gamma"])
+    assert_out(host(o)[sel], ref, _TORCH_OUT[out], what, extra=extra, scale=scale, rel32=rel32)
 
 
 def test_bitlinear_tiny_config():
@@ -289,7 +284,30 @@ def test_bitlinear_tiny_config():
 @pytest.mark.parametrize("M", [1, 4, 16])
 def test_bitlinear_decode_full_size(M):
     d = synth.bitlinear_decode(M)
-    _bitlinear_check(d["x"], bf16_dev(d["x_bf16"]), d["w"], 11008, "bf16", None, f"decode M={M}")
+    path = bq.BQ_PATH_DECODE_STREAM if M == 1 else bq.BQ_PATH_DECODE_MMA
+    _bitlinear_check(d["x"], bf16_dev(d["x_bf16"]), d["w"], 11008, "bf16", None, f"decode M={M}", path=path)
+
+
+# shapes the register-streaming kernels leave to the shared-memory decode
+# kernel: one token with K < 2048 or more rows per CTA than the stream kernel
+# keeps in flight, and 2..16 tokens with K % 512 == 0 but K not 2048 / 4096
+@pytest.mark.parametrize("M,N,K,out,bias,xin", [(1, 300, 1024, "bf16", False, "bf16"),
+                                                (1, 12800, 4096, "f32", True, "bf16"),
+                                                (4, 1000, 8192, "bf16", True, "f32"),
+                                                (2, 700, 1536, "f16", False, "bf16"),
+                                                (16, 400, 8192, "bf16", False, "bf16"),
+                                                (7, 900, 512, "f32", True, "f32")])
+def test_bitlinear_decode_shared_memory_kernel(M, N, K, out, bias, xin):
+    g = synth.rng((116, M, N, K))
+    if xin == "bf16":
+        bits, x = synth.bf16_activations(M, K, (116, M, K))
+        x_dev = bf16_dev(bits)
+    else:
+        x = synth.normal_f32(g, (M, K))
+        x_dev = dev(x)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    b = synth.normal_f32(g, (N,), 0.1) if bias else None
+    _bitlinear_check(x, x_dev, w, N, out, b, f"decode smem {M}x{N}x{K} {xin}", path=bq.BQ_PATH_DECODE_SMEM)
 
 
 @pytest.mark.parametrize("M,N,K,out,bias", [(3, 100, 48, "f16", True), (7, 64, 4096, "f32", False),
@@ -299,7 +317,8 @@ def test_bitlinear_decode_ragged(M, N, K, out, bias):
     x = synth.normal_f32(g, (M, K))
     w = synth.normal_f32(g, (N, K), 0.02)
     b = synth.normal_f32(g, (N,), 0.1) if bias else None
-    _bitlinear_check(x, dev(x), w, N, out, b, f"decode ragged {M}x{N}x{K}")
+    path = bq.BQ_PATH_ACT_QUANT_GEMV if K % 512 else None
+    _bitlinear_check(x, dev(x), w, N, out, b, f"decode ragged {M}x{N}x{K}", path=path)
 
 
 # one token: dp4a register-streaming kernel (fp32 and bf16 inputs, K = 2048 / 8192,
@@ -334,6 +353,21 @@ def test_bitlinear_prefill_ragged(M, N, K, out, bias):
     w = synth.normal_f32(g, (N, K), 0.02)
     b = synth.normal_f32(g, (N,), 0.1) if bias else None
     _bitlinear_check(xf, bf16_dev(bits), w, N, out, b, f"prefill ragged {M}x{N}x{K}")
+
+
+# more than 16 tokens with K % 64 != 0 (packed rows re-pitched in the
+# workspace) and / or N * size % 16 != 0 (output rows staged in the workspace)
+@pytest.mark.parametrize("M,N,K,out,bias", [(300, 61, 144, "f16", False), (257, 1001, 528, "bf16", True),
+                                            (17, 9, 16, "bf16", False), (40, 77, 80, "f32", True),
+                                            (130, 300, 1040, "bf16", False), (2500, 4601, 144, "f16", True)])
+def test_bitlinear_prefill_unaligned_tails(M, N, K, out, bias):
+    g = synth.rng((117, M, N, K))
+    bits, xf = synth.bf16_activations(M, K, (117, M), outlier_frac=0.01)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    b = synth.normal_f32(g, (N,), 0.1) if bias else None
+    x_dev = bf16_dev(bits)
+    path = bq.BQ_PATH_TC_PAIR if (M >= 2048 and N >= 4096) else bq.BQ_PATH_TC_SINGLE
+    _bitlinear_check(xf, x_dev, w, N, out, b, f"prefill tails {M}x{N}x{K}", path=path)
 
 
 def test_bitlinear_prefill_full_size_sampled_rows():

@@ -303,3 +303,121 @@ def test_w4_one_hot_gathers_x():
     x = synth.normal_f32(g, (2, K))
     out = oracle.linear_w4_grouped(x, oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), None, gs)
     np.testing.assert_array_equal(out, x[:, cols].astype(np.float64))
+
+
+def test_w4_one_hot_with_per_group_scale_picks_its_group():
+    # one nonzero code per weight row, at a column k_n in a known group, with a
+    # scale that differs per group and per row and no zero-point:
+    # out[m,n] = s[n, k_n // gs] * x[m, k_n]  (every value exact in binary64)
+    g = synth.rng(16)
+    N, K, gs = 12, 256, 32
+    G = K // gs
+    cols = g.integers(0, K, N)
+    cols[:G] = np.arange(G) * gs + 5  # every group is hit at least once
+    q = np.zeros((N, K), np.uint8)
+    q[np.arange(N), cols] = 1
+    z = np.zeros((N, G), np.uint8)
+    s = (0.5 * (np.arange(G)[None, :] + 1) + 0.125 * (np.arange(N)[:, None] % 4)).astype(np.float16)
+    x = synth.normal_f32(g, (3, K))
+    out = oracle.linear_w4_grouped(x, oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), None, gs)
+    want = np.empty((3, N))
+    for n in range(N):
+        want[:, n] = float(s[n, cols[n] // gs]) * x[:, cols[n]].astype(np.float64)
+    np.testing.assert_array_equal(out, want)
+    # zero-point 3 in that group only: its 31 zero codes weigh -3 and the one
+    # code weighs 1 - 3, so out = s * (x[k_n] - 3 * sum of x over the group)
+    z2 = z.copy()
+    z2[np.arange(N), cols // gs] = 3
+    out2 = oracle.linear_w4_grouped(x, oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z2), None, gs)
+    want2 = np.empty((3, N))
+    for n in range(N):
+        g0 = (cols[n] // gs) * gs
+        xg = x[:, g0:g0 + gs].astype(np.float64)
+        want2[:, n] = float(s[n, cols[n] // gs]) * (x[:, cols[n]].astype(np.float64) - 3.0 * xg.sum(axis=1))
+    np.testing.assert_allclose(out2, want2, rtol=1e-13, atol=1e-14)
+
+
+def test_w4_single_group_is_plain_int4_linear():
+    # group_size = K leaves one scale and zero-point per row: the grouped
+    # affine form reduces to s_n * (x . q_n - z_n * sum(x)), i.e. the plain
+    # unpack-on-demand INT4 dot product of the linear_4bit module, scaled and
+    # shifted; with s = 1, z = 0 it is the integer-code matmul itself
+    g = synth.rng(17)
+    M, N, K = 4, 9, 128
+    q = synth.nibbles(g, (N, K))
+    x = synth.normal_f32(g, (M, K))
+    one = np.ones((N, 1), np.float16)
+    zero = np.zeros((N, 1), np.uint8)
+    plain = oracle.linear_w4_grouped(x, oracle.int4_pack(q), one.view(np.uint16), oracle.int4_pack(zero), None, K)
+    np.testing.assert_allclose(plain, x.astype(np.float64) @ q.astype(np.float64).T, rtol=1e-13, atol=1e-12)
+    s = g.uniform(0.005, 0.02, (N, 1)).astype(np.float16)
+    z = synth.nibbles(g, (N, 1))
+    out = oracle.linear_w4_grouped(x, oracle.int4_pack(q), s.view(np.uint16), oracle.int4_pack(z), None, K)
+    xs = x.astype(np.float64).sum(axis=1, keepdims=True)
+    want = (plain - xs * z.astype(np.float64).T) * s.astype(np.float64).T
+    np.testing.assert_allclose(out, want, rtol=1e-12, atol=1e-13)
+
+
+def test_bitlinear_one_code_per_row_pins_weight_indexing():
+    # W has one nonzero per output row, +-c at column k_n: it is already
+    # ternary, so gamma = c and out[m,n] = +-xq[m,k_n] * act_scale[m] * c.
+    # M, N and K all differ, so a transposed operand or a swapped index fails.
+    g = synth.rng(18)
+    M, N, K = 5, 11, 48
+    c = np.float32(0.0625)
+    cols = g.permutation(K)[:N]
+    sign = np.where(g.integers(0, 2, N) == 1, 1.0, -1.0).astype(np.float32)
+    w = np.zeros((N, K), np.float32)
+    w[np.arange(N), cols] = sign * c
+    x = synth.normal_f32(g, (M, K))
+    out, a, t = oracle.bitlinear(x, w)
+    assert t["already_ternary"] and t["gamma"] == float(c)
+    want = a["xq"][:, cols].astype(np.float64) * sign[None, :] * a["act_scale"][:, None] * float(c)
+    np.testing.assert_array_equal(out, want)
+    # the same through the codes entry point with a bias
+    b = synth.normal_f32(g, (N,), 0.1)
+    out_b = oracle.bitlinear_from_codes(a["xq"], a["act_scale"], t["wq"], t["gamma"], b)
+    np.testing.assert_array_equal(out_b, want + b.astype(np.float64)[None, :])
+
+
+# --------------------------------------------------------- batched W8A8
+
+def test_gemm_batched_atb_example_stacked(golden_dir):
+    # the worked example twice as a batch of 2 ([batch,m,k] x [batch,k,n]),
+    # and with x stored transposed ([batch,k,m], transposeA): the printed
+    # output for every batch
+    d = _load(golden_dir, "atb_per_token_example.json")
+    x = np.array(d["x"], np.int8)
+    w = np.array(d["weight"], np.int8)  # [k, n]
+    want = np.array(d["output"], np.float64)
+    deq, pts = np.array(d["deqScale"], np.float32), np.array(d["perTokenScale"], np.float32)
+    xb, wb = np.stack([x, x]), np.stack([w, w])
+    out, ovf = oracle.gemm_i8_pertoken_batched(xb, wb, deq, pts, layout=1)
+    assert ovf == 0
+    np.testing.assert_array_equal(out, np.stack([want, want]))
+    out_t, _ = oracle.gemm_i8_pertoken_batched(np.ascontiguousarray(xb.transpose(0, 2, 1)), wb, deq, pts,
+                                                layout=1, trans_a=True)
+    np.testing.assert_array_equal(out_t, np.stack([want, want]))
+    out_nk, _ = oracle.gemm_i8_pertoken_batched(xb, np.ascontiguousarray(wb.transpose(0, 2, 1)), deq, pts,
+                                                 layout=0)
+    np.testing.assert_array_equal(out_nk, np.stack([want, want]))
+
+
+def test_gemm_batched_is_per_batch_matmul_with_its_scales():
+    # different data per batch: each batch equals the integer matmul of its
+    # own operands (numpy int64), scaled by the shared or per-batch vectors
+    g = synth.rng(19)
+    B, M, N, K = 3, 5, 7, 40
+    x, w = synth.int8_uniform(g, (B, M, K)), synth.int8_uniform(g, (B, N, K))
+    deq_b, pts_b = synth.uniform_f32(g, (B, N), 0.001, 0.01), synth.uniform_f32(g, (B, M), 0.001, 0.01)
+    out, _ = oracle.gemm_i8_pertoken_batched(x, w, deq_b, pts_b, shared_scales=False)
+    for b in range(B):
+        acc = (x[b].astype(np.int64) @ w[b].astype(np.int64).T).astype(np.float64)
+        ref = pts_b[b].astype(np.float64)[:, None] * acc * deq_b[b].astype(np.float64)[None, :]
+        np.testing.assert_allclose(out[b], ref, rtol=1e-15, atol=0)
+    # shared scales: batch b uses deq[n] and pts[m] of the one vector each
+    out_s, _ = oracle.gemm_i8_pertoken_batched(x, w, deq_b[1], pts_b[2])
+    for b in range(B):
+        acc = (x[b].astype(np.int64) @ w[b].astype(np.int64).T).astype(np.float64)
+        ref = pts_b[2].astype(np.float64)[:, None] * acc * deq_b[1].astype(np.float64)[None, :]
+        np.testing.assert_allclose(out_s[b], ref, rtol=1e-15, atol=0)
