@@ -66,8 +66,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-workloads", action="store_true", help="skip the secondary workloads")
-    p.add_argument("--workloads", default="decode,w4,prefill,tiny",
-                   help="comma list of secondary workloads: decode, w4, prefill, tiny")
+    p.add_argument("--workloads", default="decode,w4,prefill,tiny,batched",
+                   help="comma list of secondary workloads: decode, w4, prefill, tiny, batched")
     p.add_argument("--workload-steps", type=int, default=200)
     p.add_argument("--no-head", action="store_true", help="skip the headline GEMM (profiling runs only)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -452,6 +452,8 @@ def workloads(args, pk):
         _prefill(res, max(steps // 4, 1), peak_int8, hbm)
     if "tiny" in want:
         _tiny(res, steps)
+    if "batched" in want:
+        _batched(res, steps, peak_int8)
     st, detail = bq.bq_device_status()
     if st != bq.BQ_OK:
         raise RuntimeError(f"device status {detail:#x} after the workloads")
@@ -581,6 +583,51 @@ def _tiny(res, steps):
 
     ms, _, _ = graph_time(step, steps, 3)
     res["bitlinear_tiny"] = {"us_per_step": round(ms * 1e3, 3), "config": "x fp32 [8,256], W [128,256]"}
+
+
+def _batched(res, steps, peak_int8):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
+    # batched per-token W8A8: 8 x ([512,4096] x [4096,4096]) per-batch weights and scales,
+    # and the 4096^3 product with x stored [K, M] (transposeA); 4 rotating copies (> L2)
+    B, M, N, K = 8, 512, 4096, 4096
+    g = synth.rng(31)
+    x = torch.from_numpy(synth.int8_uniform(g, (B, M, K))).cuda()
+    w = torch.from_numpy(synth.int8_uniform(g, (B, N, K))).cuda()
+    deq = torch.from_numpy(synth.uniform_f32(g, (B, N), 0.001, 0.01)).cuda()
+    pts = torch.from_numpy(synth.uniform_f32(g, (B, M), 0.001, 0.01)).cuda()
+    sets = [(x.clone(), w.clone()) for _ in range(4)]
+    out = torch.empty((B, M, N), dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        a, b = sets[i % 4]
+        bq.bq_gemm_i8_pertoken_batched(a, b, deq, pts, out=out)
+
+    ms, _, _ = graph_time(step, steps, 3)
+    ops = 2.0 * B * M * N * K
+    res["gemm_batched_8x512"] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(ops / (ms * 1e-3) / 1e12, 1),
+                                 "frac_int8_peak": round(ops / (ms * 1e-3) / 1e12 / peak_int8, 4),
+                                 "config": "x int8 [8,512,4096] x w int8 [8,4096,4096] (N,K), per-batch scales, bf16 out"}
+    del sets, x, w
+    d = synth.gemm_w8a8()
+    xt = torch.from_numpy(np.ascontiguousarray(d["x"].T)).cuda()[None]
+    w1 = torch.from_numpy(d["w"]).cuda()[None]
+    sets = [(xt.clone(), w1.clone()) for _ in range(4)]
+    dq, pt = torch.from_numpy(d["deq_scale"]).cuda(), torch.from_numpy(d["per_token_scale"]).cuda()
+    out1 = torch.empty((1, 4096, 4096), dtype=torch.bfloat16, device="cuda")
+
+    def step_t(i):
+        a, b = sets[i % 4]
+        bq.bq_gemm_i8_pertoken_batched(a, b, dq, pt, trans_a=True, out=out1)
+
+    ms, _, _ = graph_time(step_t, steps, 3)
+    ops = 2.0 * 4096 ** 3
+    res["gemm_transA_4096"] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(ops / (ms * 1e-3) / 1e12, 1),
+                               "frac_int8_peak": round(ops / (ms * 1e-3) / 1e12 / peak_int8, 4),
+                               "config": "x int8 stored [4096 (K), 4096 (M)] (transposeA) x w [4096,4096] (N,K), "
+                                         "single-CTA tiles, bf16 out"}
 
 
 # ---------------------------------------------------------------------------

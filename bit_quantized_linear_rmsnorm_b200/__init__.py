@@ -26,7 +26,8 @@ BQ_W_NK, BQ_W_KN = 0, 1
 
 EXPORTED = [
     "bq_act_quant_int8", "bq_weight_quant_ternary_pack", "bq_weight_pack_int4_grouped",
-    "bq_gemm_i8_pertoken", "bq_bitlinear_w2a8", "bq_linear_w4_grouped", "bq_workspace_bytes",
+    "bq_gemm_i8_pertoken", "bq_gemm_i8_pertoken_batched", "bq_bitlinear_w2a8", "bq_act_quant_int8_layernorm",
+    "bq_bitlinear_w2a8_layernorm", "bq_linear_w4_grouped", "bq_workspace_bytes",
     "bq_bitlinear_workspace_layout", "bq_status_string", "bq_device_status", "bq_version",
     "bq_bitlinear_w2a8_noalloc", "bq_bitlinear_w2a8_path", "bq_diag_gemm_withheld_arrival",
 ]
@@ -47,7 +48,11 @@ _SIGS = {
     "bq_weight_quant_ternary_pack": (I32, [P, I32, I64, I64, P, P, P, SZ, P]),
     "bq_weight_pack_int4_grouped": (I32, [P, P, I64, I64, I64, P, P, P]),
     "bq_gemm_i8_pertoken": (I32, [P, I64, P, I32, I64, P, P, P, I64, I64, I64, I32, P, I64, P]),
+    "bq_gemm_i8_pertoken_batched": (I32, [P, I64, I64, I32, P, I32, I64, I64, P, I64, P, I64, P, I64, I64, I64, I64,
+                                          I32, P, I64, I64, P]),
     "bq_bitlinear_w2a8": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P, SZ, P]),
+    "bq_act_quant_int8_layernorm": (I32, [P, I32, I64, I64, I64, P, P, F32, P, I64, P, P, P]),
+    "bq_bitlinear_w2a8_layernorm": (I32, [P, I32, I64, I64, P, P, P, P, I64, P, F32, I32, P, P, SZ, P]),
     "bq_linear_w4_grouped": (I32, [P, I64, I64, P, P, P, P, I64, I64, P, P, SZ, P]),
     "bq_bitlinear_w2a8_noalloc": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P]),
     "bq_bitlinear_w2a8_path": (I32, [P, I32, I64, I64, I64, ctypes.POINTER(I32)]),
@@ -151,6 +156,41 @@ def bq_act_quant_int8(x: torch.Tensor, eps: float = 1e-5, xq=None, act_scale=Non
     return xq, act_scale, rowsum
 
 
+def bq_act_quant_int8_layernorm(x: torch.Tensor, eps: float = 1e-5, ln_weight=None, ln_bias=None, xq=None,
+                                act_scale=None, rowsum=None, want_rowsum: bool = True, stream=None):
+    """LayerNorm (optional affine) + per-token int8 quantization:
+    (xq int8 [M,K], act_scale fp32 [M], rowsum int32 [M] or None)."""
+    M, K = x.shape
+    if xq is None:
+        ldq = (K + 15) // 16 * 16
+        xq = torch.empty((M, ldq), dtype=torch.int8, device=x.device)[:, :K]
+    if act_scale is None:
+        act_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    if rowsum is None and want_rowsum:
+        rowsum = torch.empty(M, dtype=torch.int32, device=x.device)
+    st = lib().bq_act_quant_int8_layernorm(_ptr(x), _DTYPE[x.dtype], M, K, _ld(x), _ptr(ln_weight), _ptr(ln_bias),
+                                           float(eps), _ptr(xq), _ld(xq), _ptr(act_scale), _ptr(rowsum),
+                                           _stream(stream))
+    _check(st, "bq_act_quant_int8_layernorm")
+    return xq, act_scale, rowsum
+
+
+def bq_bitlinear_w2a8_layernorm(x: torch.Tensor, wpacked: torch.Tensor, w_scale: torch.Tensor, N: int,
+                                ln_weight=None, ln_bias=None, bias=None, eps: float = 1e-5, out_dtype=torch.bfloat16,
+                                out=None, workspace=None, stream=None):
+    """BitLinear forward with the LayerNorm normaliser."""
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    nbytes = bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().bq_bitlinear_w2a8_layernorm(_ptr(x), _DTYPE[x.dtype], M, K, _ptr(ln_weight), _ptr(ln_bias),
+                                           _ptr(wpacked), _ptr(w_scale), N, _ptr(bias), float(eps), _DTYPE[out.dtype],
+                                           _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bq_bitlinear_w2a8_layernorm")
+    return out
+
+
 def bq_weight_quant_ternary_pack(w: torch.Tensor, wpacked=None, w_scale=None, workspace=None, stream=None):
     """(wpacked uint32-as-int32 [N,K/16], w_scale fp32 [1])."""
     N, K = w.shape
@@ -195,6 +235,39 @@ def bq_gemm_i8_pertoken(x: torch.Tensor, w: torch.Tensor, deq_scale: torch.Tenso
                                    _ptr(per_token_scale), _ptr(bias), M, N, K, _DTYPE[out.dtype], _ptr(out), _ld(out),
                                    _stream(stream))
     _check(st, "bq_gemm_i8_pertoken")
+    return out
+
+
+def _ld3(t: torch.Tensor):
+    """(leading dimension, batch stride) of a [B, rows, cols] tensor with unit inner stride."""
+    if t.dim() != 3 or t.stride(2) != 1:
+        raise ValueError("expected a 3-D tensor with unit inner stride")
+    return t.stride(1), t.stride(0)
+
+
+def bq_gemm_i8_pertoken_batched(x: torch.Tensor, w: torch.Tensor, deq_scale: torch.Tensor,
+                                per_token_scale: torch.Tensor, bias=None, w_layout: int = BQ_W_NK,
+                                trans_a: bool = False, out_dtype=torch.bfloat16, out=None, stream=None):
+    """Batched per-token W8A8 matmul.  x int8 [B,M,K] ([B,K,M] with trans_a);
+    w int8 [B,N,K] (BQ_W_NK) or [B,K,N] (BQ_W_KN); deq_scale [N] / [B,N] and
+    per_token_scale [M] / [B,M] (1-D: shared by every batch)."""
+    B = x.shape[0]
+    M, K = (x.shape[2], x.shape[1]) if trans_a else (x.shape[1], x.shape[2])
+    N = w.shape[1] if w_layout == BQ_W_NK else w.shape[2]
+    if out is None:
+        esz = torch.tensor([], dtype=out_dtype).element_size()
+        pad = 16 // esz
+        ldo = (N + pad - 1) // pad * pad
+        out = torch.empty((B, M, ldo), dtype=out_dtype, device=x.device)[:, :, :N]
+    ldx, sx = _ld3(x)
+    ldw, sw = _ld3(w)
+    ldo_, so = _ld3(out)
+    sd = deq_scale.stride(0) if deq_scale.dim() == 2 else 0
+    sp = per_token_scale.stride(0) if per_token_scale.dim() == 2 else 0
+    st = lib().bq_gemm_i8_pertoken_batched(_ptr(x), ldx, sx, int(bool(trans_a)), _ptr(w), w_layout, ldw, sw,
+                                           _ptr(deq_scale), sd, _ptr(per_token_scale), sp, _ptr(bias), B, M, N, K,
+                                           _DTYPE[out.dtype], _ptr(out), ldo_, so, _stream(stream))
+    _check(st, "bq_gemm_i8_pertoken_batched")
     return out
 
 

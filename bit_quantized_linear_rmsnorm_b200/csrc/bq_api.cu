@@ -251,20 +251,34 @@ bq_status bq_weight_pack_int4_grouped(const uint8_t *q, const uint8_t *zeros, in
                                       dev));
 }
 
-bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_wlayout w_layout, int64_t ldw,
-                              const float *deq_scale, const float *per_token_scale, const float *bias, int64_t M,
-                              int64_t N, int64_t K, bq_dtype out_dtype, void *out, int64_t ldo,
-                              bq_stream_t stream) {
-    if (M < 0 || N < 0 || K < 1 || K > kMaxK || M > kMaxDim || N > kMaxDim) return BQ_ERR_INVALID_ARG;
+bq_status bq_gemm_i8_pertoken_batched(const int8_t *x, int64_t ldx, int64_t stride_x, int trans_a, const int8_t *w,
+                                      bq_wlayout w_layout, int64_t ldw, int64_t stride_w, const float *deq_scale,
+                                      int64_t stride_deq, const float *per_token_scale, int64_t stride_pts,
+                                      const float *bias, int64_t batch, int64_t M, int64_t N, int64_t K,
+                                      bq_dtype out_dtype, void *out, int64_t ldo, int64_t stride_out,
+                                      bq_stream_t stream) {
+    if (batch < 0 || M < 0 || N < 0 || K < 1 || K > kMaxK || M > kMaxDim || N > kMaxDim) return BQ_ERR_INVALID_ARG;
+    if (trans_a != 0 && trans_a != 1) return BQ_ERR_INVALID_ARG;
     if (w_layout != BQ_W_NK && w_layout != BQ_W_KN) return BQ_ERR_INVALID_ARG;
     if (!out_dtype_ok(out_dtype)) return BQ_ERR_INVALID_ARG;
-    if (ldx < K || ldw < (w_layout == BQ_W_NK ? K : N) || ldo < N) return BQ_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return BQ_OK;
+    const int64_t x_rows = trans_a ? K : M, x_cols = trans_a ? M : K;
+    const int64_t w_rows = w_layout == BQ_W_NK ? N : K, w_cols = w_layout == BQ_W_NK ? K : N;
+    if (ldx < x_cols || ldw < w_cols || ldo < N) return BQ_ERR_INVALID_ARG;
+    if (batch > 1 && (stride_x < x_rows * ldx || stride_w < w_rows * ldw || stride_out < M * ldo ||
+                      (stride_deq != 0 && stride_deq < N) || (stride_pts != 0 && stride_pts < M)))
+        return BQ_ERR_INVALID_ARG;
+    if (stride_deq < 0 || stride_pts < 0) return BQ_ERR_INVALID_ARG;
+    if (batch == 0 || M == 0 || N == 0) return BQ_OK;
+    // tile indices are 32-bit
+    if (((M + 127) / 128) * ((N + 255) / 256) * batch > kMaxDim) return BQ_ERR_INVALID_ARG;
     if (x == nullptr || w == nullptr || deq_scale == nullptr || per_token_scale == nullptr || out == nullptr)
         return BQ_ERR_INVALID_ARG;
+    const int esz = esize(out_dtype);
     if (!aligned(x, 16) || !aligned(w, 16) || !aligned(out, 16) || ldx % 16 != 0 || ldw % 16 != 0 ||
-        (ldo * esize(out_dtype)) % 16 != 0 || !aligned(deq_scale, 32) || !aligned(per_token_scale, 4) ||
-        !aligned(bias, 4))
+        (ldo * esz) % 16 != 0 || !aligned(deq_scale, 32) || !aligned(per_token_scale, 4) || !aligned(bias, 4))
+        return BQ_ERR_MISALIGNED;
+    if (batch > 1 && (stride_x % 16 != 0 || stride_w % 16 != 0 || (stride_out * esz) % 16 != 0 ||
+                      (stride_deq * 4) % 32 != 0))
         return BQ_ERR_MISALIGNED;
     DevInfo dev;
     const bq_status st = current_device(&dev);
@@ -272,6 +286,7 @@ bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_
     GemmArgs g;
     g.a = x;
     g.lda = ldx;
+    g.a_mn = trans_a != 0;
     g.b = w;
     g.ldb = ldw;
     g.b_layout = w_layout;
@@ -284,7 +299,70 @@ bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_
     g.out_dtype = out_dtype;
     g.out = out;
     g.ldo = ldo;
+    g.batch = batch;
+    g.sa = batch > 1 ? stride_x : 0;
+    g.sb = batch > 1 ? stride_w : 0;
+    g.so = batch > 1 ? stride_out : 0;
+    g.s_col = batch > 1 ? stride_deq : 0;
+    g.s_row = batch > 1 ? stride_pts : 0;
     return launch_gemm_tc(g, static_cast<cudaStream_t>(stream), dev);
+}
+
+bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_wlayout w_layout, int64_t ldw,
+                              const float *deq_scale, const float *per_token_scale, const float *bias, int64_t M,
+                              int64_t N, int64_t K, bq_dtype out_dtype, void *out, int64_t ldo,
+                              bq_stream_t stream) {
+    return bq_gemm_i8_pertoken_batched(x, ldx, 0, 0, w, w_layout, ldw, 0, deq_scale, 0, per_token_scale, 0, bias, 1,
+                                       M, N, K, out_dtype, out, ldo, 0, stream);
+}
+
+// The ternary linear and rescale of a BitLinear call whose activations are
+// already quantized into the workspace (xq [M][K], act_scale, rowsum).
+static bq_status bitlinear_linear(int path, const BitlinearLayout &l, uint8_t *ws, int64_t M, int64_t K,
+                                  const uint32_t *wpacked, const float *w_scale, int64_t N, const float *bias,
+                                  bq_dtype out_dtype, void *out, cudaStream_t s, const DevInfo &dev) {
+    const int8_t *xq = reinterpret_cast<const int8_t *>(ws + l.xq);
+    const float *act_scale = reinterpret_cast<const float *>(ws + l.scale);
+    const int32_t *rowsum = reinterpret_cast<const int32_t *>(ws + l.rowsum);
+    if (path == BQ_PATH_ACT_QUANT_GEMV)
+        return from_cuda(
+            launch_gemv_w2a8(xq, K, act_scale, rowsum, wpacked, w_scale, bias, M, N, K, out_dtype, out, s, dev));
+    // tensor-core path: its tensor copies need 16-byte row pitches, so packed
+    // rows of K % 64 != 0 codes are re-pitched into the workspace first, and
+    // output rows of N * size % 16 != 0 bytes are staged there and copied out
+    const uint32_t *wrows = wpacked;
+    int64_t ldb = K / 16;
+    if (K % 64 != 0) {
+        uint32_t *wpad = reinterpret_cast<uint32_t *>(ws + l.wpad);
+        ldb = (K + 63) / 64 * 4;
+        const cudaError_t e =
+            cudaMemcpy2DAsync(wpad, static_cast<size_t>(ldb) * 4, wpacked, static_cast<size_t>(K / 16) * 4,
+                              static_cast<size_t>(K / 16) * 4, static_cast<size_t>(N), cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return BQ_ERR_CUDA;
+        wrows = wpad;
+    }
+    const bool stage_out = (N * esize(out_dtype)) % 16 != 0;
+    GemmArgs g;
+    g.a = xq;
+    g.lda = K;
+    g.b = wrows;
+    g.ldb = ldb;
+    g.b_packed2 = true;
+    g.colscale = w_scale;
+    g.rowscale = act_scale;
+    g.rowcorr = rowsum;
+    g.bias = bias;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.out_dtype = out_dtype;
+    g.out = stage_out ? static_cast<void *>(ws + l.opad) : out;
+    g.ldo = stage_out ? (N + 7) / 8 * 8 : N;
+    const bq_status st = launch_gemm_tc(g, s, dev);
+    if (st != BQ_OK || !stage_out) return st;
+    const size_t row = static_cast<size_t>(N) * esize(out_dtype);
+    return from_cuda(cudaMemcpy2DAsync(out, row, g.out, static_cast<size_t>(g.ldo) * esize(out_dtype), row,
+                                       static_cast<size_t>(M), cudaMemcpyDeviceToDevice, s));
 }
 
 bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const uint32_t *wpacked,
@@ -308,46 +386,50 @@ bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t 
     if (path == BQ_PATH_DECODE_STREAM || path == BQ_PATH_DECODE_MMA || path == BQ_PATH_DECODE_SMEM)
         return from_cuda(launch_decode_w2a8(x, x_dtype, M, K, eps, wpacked, w_scale, bias, N, out_dtype, out, xq,
                                             act_scale, rowsum, s, dev));
-    cudaError_t e = launch_act_quant(x, x_dtype, M, K, K, eps, xq, K, act_scale, rowsum, s, dev);
-    if (e != cudaSuccess) return BQ_ERR_CUDA;
-    if (path == BQ_PATH_ACT_QUANT_GEMV)
-        return from_cuda(
-            launch_gemv_w2a8(xq, K, act_scale, rowsum, wpacked, w_scale, bias, M, N, K, out_dtype, out, s, dev));
-    // tensor-core path: its tensor copies need 16-byte row pitches, so packed
-    // rows of K % 64 != 0 codes are re-pitched into the workspace first, and
-    // output rows of N * size % 16 != 0 bytes are staged there and copied out
-    const uint32_t *wrows = wpacked;
-    int64_t ldb = K / 16;
-    if (K % 64 != 0) {
-        uint32_t *wpad = reinterpret_cast<uint32_t *>(ws + l.wpad);
-        ldb = (K + 63) / 64 * 4;
-        e = cudaMemcpy2DAsync(wpad, static_cast<size_t>(ldb) * 4, wpacked, static_cast<size_t>(K / 16) * 4,
-                              static_cast<size_t>(K / 16) * 4, static_cast<size_t>(N), cudaMemcpyDeviceToDevice, s);
-        if (e != cudaSuccess) return BQ_ERR_CUDA;
-        wrows = wpad;
-    }
-    const bool stage_out = (N * esize(out_dtype)) % 16 != 0;
-    GemmArgs g;
-    g.a = xq;
-    g.lda = K;
-    g.b = wrows;
-    g.ldb = ldb;
-    g.b_packed2 = true;
-    g.colscale = w_scale;
-    g.rowscale = act_scale;
-    g.rowcorr = rowsum;
-    g.bias = bias;
-    g.M = M;
-    g.N = N;
-    g.K = K;
-    g.out_dtype = out_dtype;
-    g.out = stage_out ? static_cast<void *>(ws + l.opad) : out;
-    g.ldo = stage_out ? (N + 7) / 8 * 8 : N;
-    st = launch_gemm_tc(g, s, dev);
-    if (st != BQ_OK || !stage_out) return st;
-    const size_t row = static_cast<size_t>(N) * esize(out_dtype);
-    return from_cuda(cudaMemcpy2DAsync(out, row, g.out, static_cast<size_t>(g.ldo) * esize(out_dtype), row,
-                                       static_cast<size_t>(M), cudaMemcpyDeviceToDevice, s));
+    if (launch_act_quant(x, x_dtype, M, K, K, eps, xq, K, act_scale, rowsum, s, dev) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    return bitlinear_linear(path, l, ws, M, K, wpacked, w_scale, N, bias, out_dtype, out, s, dev);
+}
+
+bq_status bq_act_quant_int8_layernorm(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                      const float *ln_weight, const float *ln_bias, float eps, int8_t *xq,
+                                      int64_t ldq, float *act_scale, int32_t *rowsum, bq_stream_t stream) {
+    if (!act_dtype_ok(x_dtype) || M < 0 || K < 1 || ldx < K || ldq < K || !std::isfinite(eps) || eps < 0.0f)
+        return BQ_ERR_INVALID_ARG;
+    if (M > 0 && (x == nullptr || xq == nullptr || act_scale == nullptr)) return BQ_ERR_INVALID_ARG;
+    if (M == 0) return BQ_OK;
+    if (!aligned(x, esize(x_dtype)) || !aligned(xq, 16) || ldq % 16 != 0 || !aligned(act_scale, 4) ||
+        !aligned(rowsum, 4) || !aligned(ln_weight, 4) || !aligned(ln_bias, 4))
+        return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    return from_cuda(launch_act_quant_ln(x, x_dtype, M, K, ldx, ln_weight, ln_bias, eps, xq, ldq, act_scale, rowsum,
+                                         static_cast<cudaStream_t>(stream), dev));
+}
+
+bq_status bq_bitlinear_w2a8_layernorm(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const float *ln_weight,
+                                      const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t N,
+                                      const float *bias, float eps, bq_dtype out_dtype, void *out, void *workspace,
+                                      size_t workspace_bytes, bq_stream_t stream) {
+    bool empty = false;
+    bq_status st = bitlinear_check_args(x, x_dtype, M, K, wpacked, w_scale, N, bias, eps, out_dtype, out, &empty);
+    if (st != BQ_OK || empty) return st;
+    if (!aligned(ln_weight, 4) || !aligned(ln_bias, 4)) return BQ_ERR_MISALIGNED;
+    const BitlinearLayout l = bitlinear_layout(M, N, K);
+    if (workspace == nullptr || workspace_bytes < l.total) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_act_quant_ln(x, x_dtype, M, K, K, ln_weight, ln_bias, eps, reinterpret_cast<int8_t *>(ws + l.xq), K,
+                            reinterpret_cast<float *>(ws + l.scale), reinterpret_cast<int32_t *>(ws + l.rowsum), s,
+                            dev) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    const int path = M > kGemvMaxM ? bitlinear_path(x, x_dtype, M, N, K, dev) : BQ_PATH_ACT_QUANT_GEMV;
+    return bitlinear_linear(path, l, ws, M, K, wpacked, w_scale, N, bias, out_dtype, out, s, dev);
 }
 
 bq_status bq_bitlinear_w2a8_path(const void *x, bq_dtype x_dtype, int64_t M, int64_t N, int64_t K, int *path) {

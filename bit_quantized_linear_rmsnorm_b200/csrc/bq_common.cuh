@@ -165,6 +165,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// 3-D tiled load (x innermost, z the batch), completing on mbarrier `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+// 3-D tiled store shared -> global (bulk-group completion); out-of-range
+// parts of the box are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, uint32_t src, int32_t x, int32_t y, int32_t z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z), "r"(src)
+                 : "memory");
+}
+
 // Prefetch of a 2-D tile into L2 (no shared-memory destination, nothing to
 // wait for): safe to issue before the previous grid's results are visible,
 // since no data is consumed and L2 stays coherent.
@@ -362,13 +381,14 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor_sw128(uint32_t saddr) {
 }
 
 // Instruction descriptor for kind::i8 with a 32-bit signed accumulator.
-// a_signed / b_signed pick s8 or u8 operands; b_mn_major selects an N-major B.
+// a_signed / b_signed pick s8 or u8 operands; a_mn_major / b_mn_major select
+// an M-major A / N-major B (the operand's rows run along M / N in memory).
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed, bool b_signed,
-                                                 bool b_mn_major) {
+                                                 bool b_mn_major, bool a_mn_major = false) {
     return (2u << 4)                                   // D format: s32
            | ((a_signed ? 1u : 0u) << 7)               // A format
            | ((b_signed ? 1u : 0u) << 10)              // B format
-           | (0u << 15)                                // A K-major
+           | ((a_mn_major ? 1u : 0u) << 15)            // A major
            | ((b_mn_major ? 1u : 0u) << 16)            // B major
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16

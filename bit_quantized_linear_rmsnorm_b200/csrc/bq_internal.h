@@ -65,6 +65,12 @@ cudaError_t launch_act_quant(const void *x, bq_dtype xt, int64_t M, int64_t K, i
                              int8_t *xq, int64_t ldq, float *act_scale, int32_t *rowsum, cudaStream_t s,
                              const DevInfo &dev);
 
+// LayerNorm (optional affine ln_weight / ln_bias [K]) + per-token int8
+// quantization, in binary64 (act_quant_ln.cu).
+cudaError_t launch_act_quant_ln(const void *x, bq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *ln_weight,
+                                const float *ln_bias, float eps, int8_t *xq, int64_t ldq, float *act_scale,
+                                int32_t *rowsum, cudaStream_t s, const DevInfo &dev);
+
 // Workspace of the ternary reduction (fp64 partial sums and extrema).
 size_t ternary_pack_workspace_bytes(int64_t N, int64_t K);
 cudaError_t launch_ternary_pack(const void *w, bq_dtype wt, int64_t N, int64_t K, uint32_t *wpacked,
@@ -77,7 +83,7 @@ cudaError_t launch_int4_pack(const uint8_t *q, const uint8_t *zeros, int64_t N, 
 //   W8A8: out = (float(acc) * colscale[n]) * rowscale[m] (+ bias[n])
 //   W2A8: out = (float(acc - rowcorr[m]) * rowscale[m]) * (*colscale_scalar) (+ bias[n])
 struct GemmArgs {
-    const int8_t *a = nullptr;      // [M][lda] int8, K-major
+    const int8_t *a = nullptr;      // [M][lda] int8, K-major (or [K][lda], M-major, with a_mn)
     int64_t lda = 0;
     const void *b = nullptr;        // int8 [N][ldb] / [K][ldb], or packed 2-bit u32 [N][K/16]
     int64_t ldb = 0;                // elements (bytes for int8, words for packed)
@@ -91,12 +97,16 @@ struct GemmArgs {
     bq_dtype out_dtype = BQ_BF16;
     void *out = nullptr;
     int64_t ldo = 0;
+    bool a_mn = false;              // A stored [K][lda], M contiguous (ATB transposeA = true)
+    int64_t batch = 1;              // independent products of the same shape
+    int64_t sa = 0, sb = 0, so = 0; // elements (words for packed B) between batches of a, b, out
+    int64_t s_col = 0, s_row = 0;   // elements between batches of colscale / rowscale (0: shared)
     uint64_t wait_ns = 2000000000ull;  // limit of the kernel's bounded waits
     int withhold_kb = -1;              // failure-detection check only (single-CTA kernel)
 };
 bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev);
 // Whether launch_gemm_tc runs a product of this shape on CTA pairs.
-bool gemm_uses_pair(bool packed, bq_wlayout b_layout, int64_t M, int64_t N, const DevInfo &dev);
+bool gemm_uses_pair(bool packed, bq_wlayout b_layout, int64_t M, int64_t N, const DevInfo &dev, int64_t batch = 1);
 
 // Decode path (M <= 16) of the ternary linear: reads the packed weights once.
 cudaError_t launch_gemv_w2a8(const int8_t *xq, int64_t ldq, const float *act_scale, const int32_t *rowsum,

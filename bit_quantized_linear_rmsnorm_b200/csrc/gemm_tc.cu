@@ -76,6 +76,8 @@ struct GemmDev {
     const int32_t *rowcorr;
     const float *bias;
     int M, N, K;
+    int batch;              // independent products (tile coordinate z)
+    int64_t s_col, s_row;   // colscale / rowscale elements between batches (0: shared)
     uint32_t *status;
     uint64_t wait_ns;  // limit of every bounded wait
     int withhold_kb;   // (failure-detection check only) K block of the first tile whose copies are never issued
@@ -113,22 +115,25 @@ __device__ __forceinline__ uint64_t smem_desc_mnmajor_sw128(uint32_t saddr) {
 // least half of the CTAs idle, each of its tiles as two 128 x 128 halves, so
 // the busiest CTAs end half a tile earlier.
 struct Items {
-    int num_m, big, count;
-    __device__ Items(int num_tiles, int num_m_, int G, bool allow) : num_m(num_m_) {
+    int num_m, per_batch, big, count;
+    __device__ Items(int num_tiles, int num_m_, int per_batch_, int G, bool allow)
+        : num_m(num_m_), per_batch(per_batch_) {
         const int full = (num_tiles / G) * G, left = num_tiles - full;
         const bool split = allow && left > 0 && 2 * left <= G;
         big = split ? full : num_tiles;
         count = split ? full + 2 * left : num_tiles;
     }
-    __device__ void tile(int item, int &m0, int &n0, bool &half) const {
+    __device__ void tile(int item, int &b, int &m0, int &n0, bool &half) const {
         const int t = item < big ? item : big + ((item - big) >> 1);
-        m0 = (t % num_m) * BM;
-        n0 = (t / num_m) * BN + (item < big ? 0 : ((item - big) & 1) * (BN / 2));
+        b = t / per_batch;
+        const int r = t - b * per_batch;
+        m0 = (r % num_m) * BM;
+        n0 = (r / num_m) * BN + (item < big ? 0 : ((item - big) & 1) * (BN / 2));
         half = item >= big;
     }
 };
 
-template <bool PACKED, bool B_KN, typename OutT>
+template <bool PACKED, bool A_MN, bool B_KN, typename OutT>
 __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmO,
@@ -157,10 +162,10 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int num_m = (p.M + BM - 1) / BM;
     const int num_n = (p.N + BN - 1) / BN;
-    const int num_tiles = num_m * num_n;
+    const int num_tiles = num_m * num_n * p.batch;
     const int nkb = (p.K + BK - 1) / BK;
     // (the 2-bit path keeps whole tiles: its unpack warps expand the full B tile)
-    const Items items(num_tiles, num_m, static_cast<int>(gridDim.x), !PACKED);
+    const Items items(num_tiles, num_m, num_m * num_n, static_cast<int>(gridDim.x), !PACKED);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -197,9 +202,9 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         int64_t issued = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < items.count && ok; item += gridDim.x) {
-            int m0, n0;
+            int bz, m0, n0;
             bool half;
-            items.tile(item, m0, n0, half);
+            items.tile(item, bz, m0, n0, half);
             const uint32_t b_bytes = half ? B_BYTES / 2 : B_BYTES;
             for (int kb = 0; kb < nkb; ++kb) {
                 if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, p.status, SITE_GEMM_PRODUCER, p.wait_ns)) {
@@ -211,18 +216,22 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                     // failure-detection check: this stage's barrier never completes
                 } else if constexpr (PACKED) {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + P_BYTES);
-                    tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
-                    tma_load_2d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * (BK / 16), n0, full(stage));
-                } else if constexpr (B_KN) {
-                    mbar_arrive_expect_tx(full(stage), A_BYTES + b_bytes);
-                    tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
-                    const uint32_t b_dst = sbase + C::OFF_B + stage * B_BYTES;
-                    tma_load_2d(b_dst, &tmB, n0, kb * BK, full(stage));
-                    if (!half) tma_load_2d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, full(stage));
+                    tma_load_3d(a_dst, &tmA, kb * BK, m0, bz, full(stage));
+                    tma_load_3d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * (BK / 16), n0, bz, full(stage));
                 } else {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + b_bytes);
-                    tma_load_2d(a_dst, &tmA, kb * BK, m0, full(stage));
-                    tma_load_2d(sbase + C::OFF_B + stage * B_BYTES, half ? &tmBh : &tmB, kb * BK, n0, full(stage));
+                    // A: a 128 (K) x 128 (M) box when M-major, 128 (M) x 128 (K) otherwise
+                    if constexpr (A_MN)
+                        tma_load_3d(a_dst, &tmA, m0, kb * BK, bz, full(stage));
+                    else
+                        tma_load_3d(a_dst, &tmA, kb * BK, m0, bz, full(stage));
+                    const uint32_t b_dst = sbase + C::OFF_B + stage * B_BYTES;
+                    if constexpr (B_KN) {
+                        tma_load_3d(b_dst, &tmB, n0, kb * BK, bz, full(stage));
+                        if (!half) tma_load_3d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, bz, full(stage));
+                    } else {
+                        tma_load_3d(b_dst, half ? &tmBh : &tmB, kb * BK, n0, bz, full(stage));
+                    }
                 }
                 ++issued;
                 if (++stage == S) {
@@ -238,8 +247,8 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             mbar_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1), p.wait_ns);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = idesc_i8(BM, BN, true, !PACKED, B_KN);
-        constexpr uint32_t idesc_half = idesc_i8(BM, BN / 2, true, !PACKED, B_KN);
+        constexpr uint32_t idesc = idesc_i8(BM, BN, true, !PACKED, B_KN, A_MN);
+        constexpr uint32_t idesc_half = idesc_i8(BM, BN / 2, true, !PACKED, B_KN, A_MN);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -270,7 +279,8 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                 const uint32_t b_addr = sbase + C::OFF_B + stage * B_BYTES;
 #pragma unroll
                 for (int ks = 0; ks < BK / UMMA_K; ++ks) {
-                    const uint64_t ad = smem_desc_kmajor_sw128(a_addr + ks * UMMA_K);
+                    const uint64_t ad = A_MN ? smem_desc_mnmajor_sw128(a_addr + ks * UMMA_K * 128)
+                                             : smem_desc_kmajor_sw128(a_addr + ks * UMMA_K);
                     const uint64_t bd = B_KN ? smem_desc_mnmajor_sw128(b_addr + ks * UMMA_K * 128)
                                              : smem_desc_kmajor_sw128(b_addr + ks * UMMA_K);
                     tc_mma_i8(d_tmem, ad, bd, id, (kb | ks) != 0 ? 1u : 0u);
@@ -298,9 +308,11 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         uint32_t chunk_ctr = 0;
         int t = 0;
         for (int item = blockIdx.x; item < items.count; item += gridDim.x, ++t) {
-            int m0, n0;
+            int bz, m0, n0;
             bool half;
-            items.tile(item, m0, n0, half);
+            items.tile(item, bz, m0, n0, half);
+            const float *colscale = p.colscale + bz * p.s_col;
+            const float *rowscale = p.rowscale + bz * p.s_row;
             const int nc32 = half ? BN / 64 : BN / 32;  // 32-column chunks of this item
             const int abuf = t & 1;
             const uint32_t aphase = static_cast<uint32_t>(t >> 1) & 1u;
@@ -308,7 +320,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             named_bar_sync(1, 128);  // previous tile finished reading vcol / vbias
             for (int i = et; i < BN; i += 128) {
                 const int n = n0 + i;
-                vcol[i] = (!PACKED && n < p.N) ? __ldg(p.colscale + n) : 0.0f;
+                vcol[i] = (!PACKED && n < p.N) ? __ldg(colscale + n) : 0.0f;
                 vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
             }
             named_bar_sync(1, 128);
@@ -329,7 +341,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             if (*reinterpret_cast<volatile int *>(epi_fail)) break;
             tc_fence_after();
             const int row = m0 + r;
-            const float rs = row < p.M ? __ldg(p.rowscale + row) : 0.0f;
+            const float rs = row < p.M ? __ldg(rowscale + row) : 0.0f;
             const int corr = (p.rowcorr != nullptr && row < p.M) ? __ldg(p.rowcorr + row) : 0;
 
 #pragma unroll 1
@@ -379,7 +391,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                     fence_proxy_async_smem();
                     named_bar_sync(1, 128);
                     if (et == 0) {
-                        tma_store_2d(&tmO, smem_u32(stg + sb * STG_BYTES), n0 + c32 * 32 + sc * CC, m0);
+                        tma_store_3d(&tmO, smem_u32(stg + sb * STG_BYTES), n0 + c32 * 32 + sc * CC, m0, bz);
                         bulk_commit();
                     }
                     ++chunk_ctr;
@@ -495,12 +507,12 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
 }
 // Tensor copy into this CTA's shared memory whose completion counts on the
 // barrier at cluster address `bar` (the leader's).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
-                                                 uint32_t bar) {
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                                 int32_t z, uint32_t bar) {
     asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
 __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -565,17 +577,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
     const bool leader = rank == 0;
     const int num_m = (p.M + 2 * BM - 1) / (2 * BM);  // 256-row tiles
     const int num_n = (p.N + BN - 1) / BN;
-    const int num_tiles = num_m * num_n;
+    const int num_tiles = num_m * num_n * p.batch;
     const int nkb = (p.K + BK - 1) / BK;
     const int cl = static_cast<int>(blockIdx.x >> 1), ncl = static_cast<int>(gridDim.x >> 1);
     // items as in the single-CTA schedule, over pairs and 256 x 256 tiles
     const int full_w = (num_tiles / ncl) * ncl, left = num_tiles - full_w;
     const bool split = left > 0 && 2 * left <= ncl;
     const int big = split ? full_w : num_tiles, count = split ? full_w + 2 * left : num_tiles;
-    auto tile_of = [&](int item, int &m0, int &n0, bool &half) {
+    auto tile_of = [&](int item, int &b, int &m0, int &n0, bool &half) {
         const int t = item < big ? item : big + ((item - big) >> 1);
-        m0 = (t % num_m) * 2 * BM;
-        n0 = (t / num_m) * BN + (item < big ? 0 : ((item - big) & 1) * (BN / 2));
+        b = t / (num_m * num_n);
+        const int r = t - b * num_m * num_n;
+        m0 = (r % num_m) * 2 * BM;
+        n0 = (r / num_m) * BN + (item < big ? 0 : ((item - big) & 1) * (BN / 2));
         half = item >= big;
     };
 
@@ -615,9 +629,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         int64_t issued = 0;
         bool ok = true;
         for (int item = cl; item < count && ok; item += ncl) {
-            int m0, n0;
+            int bz, m0, n0;
             bool half;
-            tile_of(item, m0, n0, half);
+            tile_of(item, bz, m0, n0, half);
             const uint32_t b_bytes = half ? PB_BYTES / 2 : PB_BYTES;
             const int nb0 = n0 + (half ? BN / 4 : BN / 2) * static_cast<int>(rank);  // this CTA's B rows
             for (int kb = 0; kb < nkb; ++kb) {
@@ -628,16 +642,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
                 if constexpr (PACKED) {  // own barrier: this CTA's unpack warps wait on it
                     const uint32_t p_bytes = half ? PP_BYTES / 2 : PP_BYTES;
                     mbar_arrive_expect_tx(full(stage), PA_BYTES + p_bytes);
-                    tma_load_2d(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
-                                full(stage));
-                    tma_load_2d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * (BK / 16), nb0,
+                    tma_load_3d(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
+                                bz, full(stage));
+                    tma_load_3d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * (BK / 16), nb0, bz,
                                 full(stage));
                 } else {  // the leader's barrier counts both CTAs' copies
                     if (leader) mbar_arrive_expect_tx(full(stage), 2u * (PA_BYTES + b_bytes));
                     const uint32_t lbar = cluster_addr(full(stage), 0);
-                    tma_load_2d_pair(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
-                                     lbar);
-                    tma_load_2d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK, nb0, lbar);
+                    tma_load_3d_pair(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
+                                     bz, lbar);
+                    tma_load_3d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK, nb0, bz, lbar);
                 }
                 ++issued;
                 if (++stage == S) {
@@ -705,9 +719,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         uint32_t chunk_ctr = 0;
         int t = 0;
         for (int item = cl; item < count; item += ncl, ++t) {
-            int m0, n0;
+            int bz, m0, n0;
             bool half;
-            tile_of(item, m0, n0, half);
+            tile_of(item, bz, m0, n0, half);
+            const float *colscale = p.colscale + bz * p.s_col;
+            const float *rowscale = p.rowscale + bz * p.s_row;
             const int mr = m0 + BM * static_cast<int>(rank);  // this CTA's first row
             const int nc32 = half ? BN / 64 : BN / 32;
             const int abuf = t & 1;
@@ -716,7 +732,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             named_bar_sync(1, 128);
             for (int i = et; i < BN; i += 128) {
                 const int n = n0 + i;
-                vcol[i] = (!PACKED && n < p.N) ? __ldg(p.colscale + n) : 0.0f;
+                vcol[i] = (!PACKED && n < p.N) ? __ldg(colscale + n) : 0.0f;
                 vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
             }
             named_bar_sync(1, 128);
@@ -732,7 +748,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             if (*reinterpret_cast<volatile int *>(epi_fail)) break;
             tc_fence_after();
             const int row = mr + r;
-            const float rs = row < p.M ? __ldg(p.rowscale + row) : 0.0f;
+            const float rs = row < p.M ? __ldg(rowscale + row) : 0.0f;
             const int corr = (PACKED && row < p.M) ? __ldg(p.rowcorr + row) : 0;
 
 #pragma unroll 1
@@ -779,7 +795,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
                     fence_proxy_async_smem();
                     named_bar_sync(1, 128);
                     if (et == 0) {
-                        tma_store_2d(&tmO, smem_u32(stg + sb * STG_BYTES), n0 + c32 * 32 + sc * CC, mr);
+                        tma_store_3d(&tmO, smem_u32(stg + sb * STG_BYTES), n0 + c32 * 32 + sc * CC, mr, bz);
                         bulk_commit();
                     }
                     ++chunk_ctr;
@@ -848,31 +864,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// 3-D tiled tensor map: {inner, outer, batch} elements with row and batch
+// strides in bytes (both multiples of 16), box {box_inner, box_outer, 1}.
 bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw, uint64_t batch = 1,
+              uint64_t batch_bytes = 0) {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+    if (batch <= 1 || batch_bytes == 0) batch_bytes = (row_bytes * outer + 15) / 16 * 16;
+    const cuuint64_t dims[3] = {inner, outer, batch < 1 ? 1 : batch};
+    const cuuint64_t strides[2] = {row_bytes, batch_bytes};
+    const cuuint32_t box[3] = {box_inner, box_outer, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <bool PACKED, bool B_KN, typename OutT>
-bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
-                   const CUtensorMap &mO,
-                   cudaStream_t s, const DevInfo &dev) {
-    using C = Cfg<PACKED>;
-    auto kern = gemm_tc_kernel<PACKED, B_KN, OutT>;
-    static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
-    if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
-        return BQ_ERR_CUDA;
-    const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
-    const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
+GemmDev dev_args(const GemmArgs &g, const DevInfo &dev) {
     GemmDev p;
     p.colscale = g.colscale;
     p.rowscale = g.rowscale;
@@ -881,10 +891,27 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
     p.M = static_cast<int>(g.M);
     p.N = static_cast<int>(g.N);
     p.K = static_cast<int>(g.K);
+    p.batch = static_cast<int>(g.batch);
+    p.s_col = g.s_col;
+    p.s_row = g.s_row;
     p.status = dev.status;
     p.wait_ns = g.wait_ns;
     p.withhold_kb = g.withhold_kb;
-    kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mBh, mO, p);
+    return p;
+}
+
+template <bool PACKED, bool A_MN, bool B_KN, typename OutT>
+bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
+                   const CUtensorMap &mO,
+                   cudaStream_t s, const DevInfo &dev) {
+    using C = Cfg<PACKED>;
+    auto kern = gemm_tc_kernel<PACKED, A_MN, B_KN, OutT>;
+    static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
+    if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN) * g.batch;
+    const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
+    kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mBh, mO, dev_args(g, dev));
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
@@ -896,85 +923,90 @@ bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMa
     static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
     if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
         return BQ_ERR_CUDA;
-    const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN);
+    const int64_t tiles = ((g.M + 2 * BM - 1) / (2 * BM)) * ((g.N + BN - 1) / BN) * g.batch;
     const int64_t pairs = std::min<int64_t>(tiles, dev.num_sms / 2);
-    GemmDev p;
-    p.colscale = g.colscale;
-    p.rowscale = g.rowscale;
-    p.rowcorr = g.rowcorr;
-    p.bias = g.bias;
-    p.M = static_cast<int>(g.M);
-    p.N = static_cast<int>(g.N);
-    p.K = static_cast<int>(g.K);
-    p.status = dev.status;
-    p.wait_ns = g.wait_ns;
-    p.withhold_kb = -1;  // (the check runs on a single CTA)
+    GemmDev p = dev_args(g, dev);
+    p.withhold_kb = -1;  // (the failure-detection check runs on a single CTA)
     kern<<<static_cast<unsigned>(2 * pairs), C::kThreads, C::SMEM, s>>>(mA, mB128, mB64, mO, p);
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-// The pair kernel takes products with K-major (or 2-bit packed) weights that
-// fill at least one wave of CTA pairs with 256 x 256 tiles.
-bool use_pair(const GemmArgs &g, const DevInfo &dev) { return gemm_uses_pair(g.b_packed2, g.b_layout, g.M, g.N, dev); }
+// The pair kernel takes products with K-major A and K-major (or 2-bit packed)
+// weights that fill at least one wave of CTA pairs with 256 x 256 tiles.
+bool use_pair(const GemmArgs &g, const DevInfo &dev) {
+    return !g.a_mn && gemm_uses_pair(g.b_packed2, g.b_layout, g.M, g.N, dev, g.batch);
+}
 
 template <typename OutT>
 bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
                    const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
+    const uint64_t nb = static_cast<uint64_t>(g.batch);
     if (g.b_packed2 && use_pair(g, dev)) {
         // per CTA of a pair: its half of the packed tile (128 rows), 64 rows for half tiles
         CUtensorMap mP128, mP64;
         if (!make_map(&mP128, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN / 2,
-                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4) ||
             !make_map(&mP64, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN / 4,
-                      CU_TENSOR_MAP_SWIZZLE_NONE))
+                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4))
             return BQ_ERR_CUDA;
         return launch_pair<true, OutT>(g, mA, mP128, mP64, mO, s, dev);
     }
-    if (g.b_packed2) return launch_t<true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    if (g.b_packed2) return launch_t<true, false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
     if (use_pair(g, dev)) {
         // per CTA of a pair: 128-row boxes of B (half of a 256-wide tile), 64-row boxes for half tiles
         CUtensorMap mBq;
         if (!make_map(&mBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 4,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
+                      CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sb))
             return BQ_ERR_CUDA;
         return launch_pair<false, OutT>(g, mA, mBh, mBq, mO, s, dev);
     }
-    if (g.b_layout == BQ_W_KN) return launch_t<false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
-    return launch_t<false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    if (g.a_mn) {
+        if (g.b_layout == BQ_W_KN) return launch_t<false, true, true, OutT>(g, mA, mB, mBh, mO, s, dev);
+        return launch_t<false, true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    }
+    if (g.b_layout == BQ_W_KN) return launch_t<false, false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
+    return launch_t<false, false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
 }
 
 }  // namespace
 
-bool gemm_uses_pair(bool packed, bq_wlayout b_layout, int64_t M, int64_t N, const DevInfo &dev) {
+bool gemm_uses_pair(bool packed, bq_wlayout b_layout, int64_t M, int64_t N, const DevInfo &dev, int64_t batch) {
     if ((!packed && b_layout == BQ_W_KN) || dev.num_sms < 2) return false;
-    const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+    const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN) * batch;
     return tiles >= dev.num_sms / 2;
 }
 
 bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) {
+    const uint64_t nb = static_cast<uint64_t>(g.batch);
     CUtensorMap mA, mB, mBh, mO;
-    if (!make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.K, g.M, g.lda, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
-        return BQ_ERR_CUDA;
+    const bool okA = g.a_mn ? make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.M, g.K, g.lda, BM, BK,
+                                       CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sa)
+                            : make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.K, g.M, g.lda, BK, BM,
+                                       CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sa);
+    if (!okA) return BQ_ERR_CUDA;
     bool okB;
     if (g.b_packed2)
         okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN,
-                       CU_TENSOR_MAP_SWIZZLE_NONE);
+                       CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4);
     else if (g.b_layout == BQ_W_KN)
-        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.N, g.K, g.ldb, 128, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.N, g.K, g.ldb, 128, BK, CU_TENSOR_MAP_SWIZZLE_128B,
+                       nb, g.sb);
     else
-        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B,
+                       nb, g.sb);
     if (!okB) return BQ_ERR_CUDA;
     // K-major weights: a 128-row box too, for the half tiles of a last partial wave
     mBh = mB;
     if (!g.b_packed2 && g.b_layout != BQ_W_KN &&
-        !make_map(&mBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map(&mBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B,
+                  nb, g.sb))
         return BQ_ERR_CUDA;
     CUtensorMapDataType odt = g.out_dtype == BQ_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                               : g.out_dtype == BQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                                       : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const int esz = g.out_dtype == BQ_F32 ? 4 : 2;
-    if (!make_map(&mO, odt, g.out, g.N, g.M, g.ldo * esz, 64 / esz, BM, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map(&mO, odt, g.out, g.N, g.M, g.ldo * esz, 64 / esz, BM, CU_TENSOR_MAP_SWIZZLE_64B, nb, g.so * esz))
         return BQ_ERR_CUDA;
     switch (g.out_dtype) {
         case BQ_F32:

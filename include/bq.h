@@ -154,6 +154,36 @@ bq_status bq_gemm_i8_pertoken(const int8_t *x, int64_t ldx, const int8_t *w, bq_
                               void *out, int64_t ldo, bq_stream_t stream);
 
 /*
+ * Batched and transposed forms of the per-token W8A8 matmul.
+ * Source: "Per-token Quantization for Matmul" (Huawei CANN ATB), Parameters
+ * (transposeA, transposeB) and Input / Output tables (x [batch,m,k],
+ * weight [batch,k,n], output [batch,m,n]).
+ *
+ * For every b in [0, batch):
+ *   acc[b,m,n] = sum_k x(b,m,k) * w(b,k,n)             (exact int32)
+ *   out[b,m,n] = (float(acc) * deq_scale[b*stride_deq + n])
+ *                * per_token_scale[b*stride_pts + m]  (+ bias[n])
+ * x(b,m,k) = x[b*stride_x + m*ldx + k]  (trans_a = 0: [batch][M][ldx])
+ *          = x[b*stride_x + k*ldx + m]  (trans_a = 1: [batch][K][ldx], M contiguous)
+ * w(b,k,n) as in bq_gemm_i8_pertoken at w + b*stride_w.  out: out_dtype
+ * [batch][M][ldo] at out + b*stride_out.  Strides count elements.
+ * stride_deq = stride_pts = 0 shares one deq_scale [N] and one
+ * per_token_scale [M] among all batches (the tables' [n] and [m]); N and M
+ * give each batch its own.  bias [N] (or NULL) is shared.  With batch > 1:
+ * stride_x >= rows(x) * ldx, stride_w >= rows(w) * ldw, stride_out >= M * ldo,
+ * each a multiple of 16 bytes, and stride_deq * 4 a multiple of 32.  The
+ * alignment rules of bq_gemm_i8_pertoken hold for each batch.  All batches
+ * run in one launch (the tile schedule spans them); transposeA runs on
+ * single-CTA tiles.  bq_gemm_i8_pertoken is this call with batch = 1.
+ */
+bq_status bq_gemm_i8_pertoken_batched(const int8_t *x, int64_t ldx, int64_t stride_x, int trans_a,
+                                      const int8_t *w, bq_wlayout w_layout, int64_t ldw, int64_t stride_w,
+                                      const float *deq_scale, int64_t stride_deq,
+                                      const float *per_token_scale, int64_t stride_pts, const float *bias,
+                                      int64_t batch, int64_t M, int64_t N, int64_t K, bq_dtype out_dtype,
+                                      void *out, int64_t ldo, int64_t stride_out, bq_stream_t stream);
+
+/*
  * BitLinear forward with ternary weights and int8 activations (W1.58A8).
  * Source: "Class BitLinear" (LLaMA-BitNet utils.py), forward steps 1-5.
  *
@@ -178,6 +208,39 @@ bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t 
                             const uint32_t *wpacked, const float *w_scale, int64_t N,
                             const float *bias, float eps, bq_dtype out_dtype, void *out,
                             void *workspace, size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Per-token int8 activation quantization after a LayerNorm (the normaliser of
+ * BitLinear and BitConv1d in "Common Attention Utilities", frankenstein-
+ * transformer: "Applies LayerNorm to inputs before quantization"):
+ *
+ *   mu[m] = mean_k x[m,k],  var[m] = mean_k (x[m,k] - mu[m])^2
+ *   y[m,k] = (x[m,k] - mu[m]) / sqrt(var[m] + eps) * g[k] + b[k]
+ *   a[m] = max(max_k |y[m,k]|, 1e-5),  xq = clamp(rne(y * 127 / a), -128, 127)
+ *   act_scale[m] = a[m] / 127,  rowsum[m] = sum_k xq[m,k]
+ *
+ * ln_weight (g) and ln_bias (b): fp32 [K] each, 4-byte aligned, or NULL for
+ * g = 1 / b = 0 (a parameter-free LayerNorm).  Computed in binary64 (the mean
+ * subtraction cancels).  Other arguments and rules as bq_act_quant_int8.
+ */
+bq_status bq_act_quant_int8_layernorm(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                      const float *ln_weight, const float *ln_bias, float eps, int8_t *xq,
+                                      int64_t ldq, float *act_scale, int32_t *rowsum, bq_stream_t stream);
+
+/*
+ * BitLinear forward with the LayerNorm normaliser ("Common Attention
+ * Utilities", BitLinear: LayerNorm, 8-bit per-token activations, absmean
+ * ternary weights, rescale): bq_act_quant_int8_layernorm into the workspace,
+ * then the ternary linear and rescale of bq_bitlinear_w2a8
+ * (out = (float(acc) * act_scale[m]) * gamma (+ bias[n])) on the split GEMV
+ * kernel (M <= 16) or the tcgen05 GEMM (M > 16).  Arguments, workspace
+ * (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) and its layout) and
+ * rules as bq_bitlinear_w2a8, plus ln_weight / ln_bias as above.
+ */
+bq_status bq_bitlinear_w2a8_layernorm(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const float *ln_weight,
+                                      const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t N,
+                                      const float *bias, float eps, bq_dtype out_dtype, void *out, void *workspace,
+                                      size_t workspace_bytes, bq_stream_t stream);
 
 /*
  * Which kernels bq_bitlinear_w2a8 runs for a shape on the current device (for

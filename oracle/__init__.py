@@ -47,6 +47,7 @@ def lib():
         sig = {
             "bq_oracle_round_half_even": (F64, [F64]),
             "bq_oracle_act_quant": (None, [P, I64, I64, F64, P, P, P, P, P]),
+            "bq_oracle_act_quant_layernorm": (None, [P, I64, I64, F64, P, P, P, P, P, P, P]),
             "bq_oracle_ternary_quant": (ctypes.c_int, [P, I64, I64, P, P, P]),
             "bq_oracle_ternary_bake": (None, [P, F64, I64, P]),
             "bq_oracle_ternary_pack": (None, [P, I64, I64, P]),
@@ -100,6 +101,37 @@ def act_quant(x, eps: float = 1e-5, want_pre: bool = False, want_y: bool = False
     if want_y:
         out["y"] = y
     return out
+
+
+def act_quant_layernorm(x, eps: float = 1e-5, ln_weight=None, ln_bias=None, want_pre: bool = False,
+                        want_y: bool = False):
+    """LayerNorm (optional affine ln_weight / ln_bias [K]) + per-token absmax
+    int8 quantization of x [M,K]; returns the same dict as act_quant."""
+    x = _c(x, np.float32)
+    M, K = x.shape
+    gw = None if ln_weight is None else _c(ln_weight, np.float32)
+    gb = None if ln_bias is None else _c(ln_bias, np.float32)
+    xq = np.empty((M, K), np.int8)
+    sc = np.empty(M, np.float64)
+    rs = np.empty(M, np.int64)
+    pre = np.empty((M, K), np.float64) if want_pre else None
+    y = np.empty((M, K), np.float64) if want_y else None
+    lib().bq_oracle_act_quant_layernorm(_p(x), M, K, float(eps), _p(gw), _p(gb), _p(xq), _p(sc), _p(rs), _p(pre),
+                                        _p(y))
+    out = {"xq": xq, "act_scale": sc, "rowsum": rs}
+    if want_pre:
+        out["pre"] = pre
+    if want_y:
+        out["y"] = y
+    return out
+
+
+def bitlinear_layernorm(x, w, eps: float = 1e-5, ln_weight=None, ln_bias=None, bias=None):
+    """BitLinear forward with the LayerNorm normaliser."""
+    a = act_quant_layernorm(x, eps, ln_weight, ln_bias)
+    t = ternary_quant(w)
+    out = bitlinear_from_codes(a["xq"], a["act_scale"], t["wq"], t["gamma"], bias)
+    return out, a, t
 
 
 def ternary_quant(w, want_pre: bool = False):

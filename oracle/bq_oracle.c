@@ -105,6 +105,63 @@ void bq_oracle_act_quant(const float *x, int64_t M, int64_t K, double eps,
 }
 
 /*
+ * Per-token activation quantization after a LayerNorm, the normaliser of the
+ * BitLinear and BitConv1d layers of [common] ("Applies LayerNorm to inputs
+ * before quantization"; BitConv1d normalises over the channel dimension),
+ * followed by the same 8-bit per-token quantization as above:
+ *
+ *   mu[m]      = (1/K) sum_k x[m,k]
+ *   var[m]     = (1/K) sum_k (x[m,k] - mu[m])^2          (biased, as LayerNorm)
+ *   y[m,k]     = (x[m,k] - mu[m]) / sqrt(var[m] + eps) * g[k] + b[k]
+ *   a[m]       = max( max_k |y[m,k]|, 1e-5 )
+ *   pre[m,k]   = y[m,k] * 127 / a[m]
+ *   xq[m,k]    = clamp( round_half_even(pre), -128, 127 )
+ *   act_scale[m] = a[m] / 127,   rowsum[m] = sum_k xq[m,k]
+ *
+ * g (ln_weight) and b (ln_bias) are the LayerNorm's elementwise affine
+ * parameters, [K] each; NULL stands for g = 1 and b = 0 (a parameter-free
+ * LayerNorm).  Optional outputs (rowsum, pre, y) may be NULL.
+ */
+void bq_oracle_act_quant_layernorm(const float *x, int64_t M, int64_t K, double eps,
+                                   const float *g, const float *b, int8_t *xq,
+                                   double *act_scale, int64_t *rowsum, double *pre,
+                                   double *y_out)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        const float *xr = x + m * K;
+        double sum = 0.0;
+        for (int64_t k = 0; k < K; ++k) sum += (double)xr[k];
+        double mu = sum / (double)K;
+        double sq = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double d = (double)xr[k] - mu;
+            sq += d * d;
+        }
+        double sd = sqrt(sq / (double)K + eps);
+
+        double amax = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double y = ((double)xr[k] - mu) / sd * (g ? (double)g[k] : 1.0) + (b ? (double)b[k] : 0.0);
+            if (y_out) y_out[m * K + k] = y;
+            if (fabs(y) > amax) amax = fabs(y);
+        }
+        double a = amax > ORACLE_ABSMAX_FLOOR ? amax : ORACLE_ABSMAX_FLOOR;
+
+        int64_t total = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            double y = ((double)xr[k] - mu) / sd * (g ? (double)g[k] : 1.0) + (b ? (double)b[k] : 0.0);
+            double v = y * ORACLE_ACT_QMAX / a;
+            if (pre) pre[m * K + k] = v;
+            double q = clampd(bq_oracle_round_half_even(v), -128.0, 127.0);
+            xq[m * K + k] = (int8_t)q;
+            total += (int64_t)q;
+        }
+        act_scale[m] = a / ORACLE_ACT_QMAX;
+        if (rowsum) rowsum[m] = total;
+    }
+}
+
+/*
  * Absmean ternary weight quantization with the bake rule.
  * [BitLinear] step 3 (ternary {-1,0,+1} via absmean); [common] weight_quant
  * (scale by the inverse mean absolute value, round to the nearest integer in

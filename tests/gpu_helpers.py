@@ -95,15 +95,19 @@ def assert_out(gpu: np.ndarray, ref: np.ndarray, dtype, what: str, extra=None, s
                            f"{float(np.max(err - tol)):.3e} over at {np.unravel_index(np.argmax(err - tol), err.shape)}")
 
 
-def bitlinear_expected(x_f32, w_f32, bias, eps=1e-5, rows=None):
+def bitlinear_expected(x_f32, w_f32, bias, eps=1e-5, rows=None, ln=None):
     """Oracle BitLinear output for rows `rows` of x (all when None) with what
     the tolerance needs: the tie-band widening `extra`, the term magnitude
     `scale` (None without bias) and the oracle's steps `a` (act quant) and `t`
-    (ternary quant).  Everything here comes from the oracle alone."""
+    (ternary quant).  `ln` = (ln_weight, ln_bias) selects the LayerNorm
+    normaliser.  Everything here comes from the oracle alone."""
     import oracle
     M = x_f32.shape[0]
     sel = np.arange(M) if rows is None else rows
-    a = oracle.act_quant(x_f32[sel], eps, want_pre=True)
+    if ln is None:
+        a = oracle.act_quant(x_f32[sel], eps, want_pre=True)
+    else:
+        a = oracle.act_quant_layernorm(x_f32[sel], eps, ln[0], ln[1], want_pre=True)
     t = oracle.ternary_quant(w_f32, want_pre=True)
     ref = oracle.bitlinear_from_codes(a["xq"], a["act_scale"], t["wq"], t["gamma"], bias)
     # codes in the tie band may round either way: widen by what they can move

@@ -190,3 +190,41 @@ def test_linear_w4_rejects(L):
     assert call(work=None) == bq.BQ_ERR_WORKSPACE
     assert call(x=ODD) == bq.BQ_ERR_MISALIGNED
     assert call(M=0) == bq.BQ_OK
+
+
+def test_gemm_batched_rejects(L):
+    f = L.bq_gemm_i8_pertoken_batched
+
+    def call(x=FAKE, ldx=64, sx=64 * 64, ta=0, w=FAKE, wl=0, ldw=64, sw=64 * 64, deq=FAKE, sd=0, pts=FAKE, sp=0,
+             bias=None, B=2, M=64, N=64, K=64, od=bq.BQ_BF16, out=FAKE, ldo=64, so=64 * 64):
+        return f(x, ldx, sx, ta, w, wl, ldw, sw, deq, sd, pts, sp, bias, B, M, N, K, od, out, ldo, so, None)
+    assert call(B=-1) == bq.BQ_ERR_INVALID_ARG
+    assert call(ta=2) == bq.BQ_ERR_INVALID_ARG
+    assert call(sx=64 * 63) == bq.BQ_ERR_INVALID_ARG          # batches would overlap
+    assert call(sw=16) == bq.BQ_ERR_INVALID_ARG
+    assert call(so=64) == bq.BQ_ERR_INVALID_ARG
+    assert call(sd=32) == bq.BQ_ERR_INVALID_ARG               # a per-batch deqScale needs N entries
+    assert call(sp=-64) == bq.BQ_ERR_INVALID_ARG
+    assert call(ta=1, ldx=32) == bq.BQ_ERR_INVALID_ARG        # transposed x is [K][ldx >= M]
+    assert call(sx=64 * 64 + 8) == bq.BQ_ERR_MISALIGNED
+    assert call(sd=66) == bq.BQ_ERR_MISALIGNED                # each batch's deqScale 32-byte aligned
+    assert call(B=0) == bq.BQ_OK
+    assert call(B=1, sx=0, sw=0, so=0, x=ODD) == bq.BQ_ERR_MISALIGNED
+    # batch 1 ignores the strides
+    assert call(B=1, sx=0, sw=0, so=0, sd=0) not in (bq.BQ_ERR_INVALID_ARG, bq.BQ_ERR_MISALIGNED)
+
+
+def test_layernorm_calls_reject(L):
+    f = L.bq_act_quant_int8_layernorm
+    assert f(FAKE, bq.BQ_F32, 4, 64, 64, None, None, 1e-5, FAKE, 64, FAKE, None, None) not in (
+        bq.BQ_ERR_INVALID_ARG, bq.BQ_ERR_MISALIGNED)
+    assert f(FAKE, bq.BQ_F16, 4, 64, 64, None, None, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_INVALID_ARG
+    assert f(FAKE, bq.BQ_F32, 4, 64, 64, ODD, None, 1e-5, FAKE, 64, FAKE, None, None) == bq.BQ_ERR_MISALIGNED
+    assert f(None, bq.BQ_F32, 0, 64, 64, None, None, 1e-5, None, 64, None, None, None) == bq.BQ_OK
+    g = L.bq_bitlinear_w2a8_layernorm
+    assert g(FAKE, bq.BQ_BF16, 32, 40, None, None, FAKE, FAKE, 64, None, 1e-5, bq.BQ_BF16, FAKE, FAKE, 1 << 24,
+             None) == bq.BQ_ERR_INVALID_ARG
+    assert g(FAKE, bq.BQ_BF16, 32, 128, None, ODD, FAKE, FAKE, 64, None, 1e-5, bq.BQ_BF16, FAKE, FAKE, 1 << 24,
+             None) == bq.BQ_ERR_MISALIGNED
+    assert g(FAKE, bq.BQ_BF16, 32, 128, None, None, FAKE, FAKE, 64, None, 1e-5, bq.BQ_BF16, FAKE, None, 0,
+             None) == bq.BQ_ERR_WORKSPACE

@@ -469,3 +469,153 @@ def test_linear_w4_zero_point_equals_code_gives_bias():
     b = synth.normal_f32(g, (N,), 0.01)
     x = synth.normal_f32(g, (3, K))
     _w4_check(3, N, K, gs, None, full=(q, z, s, b, x))
+
+
+# ------------------------------------------------- batched / transposed W8A8
+
+def _dev3(a: np.ndarray, align_elems: int = 16):
+    """Device copy of a [B, R, C] array with rows padded to align_elems (the
+    batch stride is R * padded row), sliced back to [B, R, C]."""
+    B, R, C = a.shape
+    ld = (C + align_elems - 1) // align_elems * align_elems
+    buf = np.zeros((B, R, ld), a.dtype)
+    buf[:, :, :C] = a
+    return dev(buf)[:, :, :C]
+
+
+def test_gemm_batched_atb_example(golden_dir):
+    import json
+    import os
+    with open(os.path.join(golden_dir, "atb_per_token_example.json")) as f:
+        ex = json.load(f)
+    x = np.array(ex["x"], np.int8)
+    w = np.array(ex["weight"], np.int8)  # [k, n]
+    want = np.stack([np.array(ex["output"], np.float64)] * 3)
+    deq = dev(np.array(ex["deqScale"], np.float32))
+    pts = dev(np.array(ex["perTokenScale"], np.float32))
+    for trans in (False, True):
+        xs = np.stack([x.T if trans else x] * 3)
+        for layout, ws in ((bq.BQ_W_KN, np.stack([w] * 3)), (bq.BQ_W_NK, np.stack([w.T] * 3))):
+            for out in ("bf16", "f16", "f32"):
+                o = bq.bq_gemm_i8_pertoken_batched(_dev3(np.ascontiguousarray(xs)), _dev3(np.ascontiguousarray(ws)),
+                                                   deq, pts, w_layout=layout, trans_a=trans,
+                                                   out_dtype=_TORCH_OUT[out])
+                np.testing.assert_array_equal(host(o), want, err_msg=f"trans {trans} layout {layout} {out}")
+
+
+@pytest.mark.parametrize("B,M,N,K,layout,trans,out,bias,shared", [
+    (3, 200, 300, 160, bq.BQ_W_NK, False, "bf16", False, True),
+    (2, 129, 257, 96, bq.BQ_W_KN, False, "f32", True, False),
+    (1, 300, 520, 400, bq.BQ_W_NK, True, "bf16", True, True),
+    (4, 130, 200, 64, bq.BQ_W_KN, True, "f16", False, False),
+    (2, 257, 384, 1000, bq.BQ_W_NK, True, "f32", False, True),
+    # enough 256 x 256 tiles over the batches for CTA pairs
+    (4, 1024, 2048, 128, bq.BQ_W_NK, False, "bf16", True, False),
+    (6, 700, 1300, 48, bq.BQ_W_NK, False, "f16", False, True),
+])
+def test_gemm_batched_ragged(B, M, N, K, layout, trans, out, bias, shared):
+    g = synth.rng((118, B, M, N, K))
+    x = synth.int8_uniform(g, (B, M, K))
+    w = synth.int8_uniform(g, (B, N, K))
+    deq = synth.uniform_f32(g, (N,) if shared else (B, N), 0.001, 0.01)
+    pts = synth.uniform_f32(g, (M,) if shared else (B, M), 0.001, 0.01)
+    b = synth.normal_f32(g, (N,), 0.5) if bias else None
+    xs = np.ascontiguousarray(x.transpose(0, 2, 1)) if trans else x
+    ws = w if layout == bq.BQ_W_NK else np.ascontiguousarray(w.transpose(0, 2, 1))
+    deq_d = dev(deq) if shared else _dev3(deq[:, None, :], 8)[:, 0, :]
+    o = bq.bq_gemm_i8_pertoken_batched(_dev3(xs), _dev3(ws), deq_d, dev(pts), None if b is None else dev(b),
+                                       w_layout=layout, trans_a=trans, out_dtype=_TORCH_OUT[out])
+    torch.cuda.synchronize()
+    ref, ovf = oracle.gemm_i8_pertoken_batched(xs, ws, deq, pts, b, layout=layout, trans_a=trans,
+                                               shared_scales=shared)
+    assert ovf == 0
+    scale = None
+    if b is not None:
+        scale = np.abs(ref - b.astype(np.float64)) + np.abs(b.astype(np.float64))
+    assert_out(host(o), ref, _TORCH_OUT[out], f"batched {B}x{M}x{N}x{K} layout {layout} trans {trans} {out}",
+               scale=scale)
+
+
+def test_gemm_transposed_a_full_size_sampled_rows():
+    # the 4096^3 workload with x stored [K, M] (transposeA)
+    d = synth.gemm_w8a8()
+    xt = np.ascontiguousarray(d["x"].T)
+    o = bq.bq_gemm_i8_pertoken_batched(dev(xt)[None], dev(d["w"])[None], dev(d["deq_scale"]),
+                                       dev(d["per_token_scale"]), trans_a=True)
+    torch.cuda.synchronize()
+    rows = np.sort(np.concatenate([[0, 127, 128, 4095], synth.rng(119).choice(4096, 28, replace=False)]))
+    ref, _ = oracle.gemm_i8_pertoken(d["x"][rows], d["w"], d["deq_scale"], d["per_token_scale"][rows])
+    assert_out(host(o)[0][rows], ref, torch.bfloat16, "gemm 4096^3 transposeA sampled rows")
+
+
+# ---------------------------------------------------- LayerNorm normaliser
+
+def _ln_params(g, K, affine):
+    if not affine:
+        return None, None
+    return (1.0 + 0.2 * g.standard_normal(K)).astype(np.float32), (0.1 * g.standard_normal(K)).astype(np.float32)
+
+
+@pytest.mark.parametrize("M,K,dtype,affine", [(8, 256, "f32", False), (37, 1000, "bf16", True),
+                                              (300, 4096, "bf16", True), (5, 4096, "f32", False),
+                                              (1, 7, "f32", True), (2000, 512, "bf16", False)])
+def test_act_quant_layernorm(M, K, dtype, affine):
+    g = synth.rng((121, M, K))
+    x = synth.normal_f32(g, (M, K)) + np.float32(0.75)  # a nonzero mean for the LayerNorm to remove
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(x)
+        x = synth.bf16_bits_to_f32(bits)
+        xd = bf16_dev(bits)
+    else:
+        xd = dev(x)
+    lw, lb = _ln_params(g, K, affine)
+    xq, sc, rs = bq.bq_act_quant_int8_layernorm(xd, 1e-5, None if lw is None else dev(lw),
+                                                None if lb is None else dev(lb))
+    torch.cuda.synchronize()
+    ref = oracle.act_quant_layernorm(x, 1e-5, lw, lb, want_pre=True)
+    g_xq = host(xq)
+    assert_codes(g_xq, ref["xq"], ref["pre"], f"layernorm quant {M}x{K} {dtype}")
+    np.testing.assert_allclose(host(sc), ref["act_scale"], rtol=1e-5)
+    np.testing.assert_array_equal(host(rs), g_xq.astype(np.int64).sum(axis=1))
+
+
+def test_act_quant_layernorm_special_rows():
+    K = 512
+    x = synth.normal_f32(synth.rng(122), (4, K))
+    x[0] = 3.0                   # constant row: zero after the mean is removed
+    x[1] = 0.0
+    x[1, 7] = 5.0                # one-hot row
+    x[2] += np.float32(1000.0)   # large common offset
+    xq, sc, _ = bq.bq_act_quant_int8_layernorm(dev(x), 1e-5)
+    torch.cuda.synchronize()
+    ref = oracle.act_quant_layernorm(x, 1e-5, want_pre=True)
+    assert_codes(host(xq), ref["xq"], ref["pre"], "layernorm special rows")
+    np.testing.assert_allclose(host(sc), ref["act_scale"], rtol=1e-5)
+    assert np.all(host(xq)[0] == 0)
+
+
+@pytest.mark.parametrize("M,N,K,out,bias,affine", [(4, 11008, 4096, "bf16", False, False),
+                                                   (16, 300, 2048, "f32", True, True),
+                                                   (300, 520, 512, "bf16", True, True),
+                                                   (300, 61, 144, "f16", False, True),
+                                                   (2048, 4096, 256, "bf16", False, False)])
+def test_bitlinear_layernorm(M, N, K, out, bias, affine):
+    g = synth.rng((123, M, N, K))
+    bits, xf = synth.bf16_activations(M, K, (123, M, K), outlier_frac=0.01)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    b = synth.normal_f32(g, (N,), 0.1) if bias else None
+    lw, lb = _ln_params(g, K, affine)
+    wp, ws_ = bq.bq_weight_quant_ternary_pack(dev(w))
+    work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, M, N, K), dtype=torch.uint8, device="cuda")
+    o = bq.bq_bitlinear_w2a8_layernorm(bf16_dev(bits), wp, ws_, N, None if lw is None else dev(lw),
+                                       None if lb is None else dev(lb), None if b is None else dev(b), 1e-5,
+                                       _TORCH_OUT[out], workspace=work)
+    torch.cuda.synchronize()
+    xo, so, _ = bq.bq_bitlinear_workspace_layout(M, K)
+    g_xq = host(work[xo:xo + M * K].view(torch.int8).view(M, K))
+    g_sc = host(work[so:so + 4 * M].view(torch.float32))
+    what = f"bitlinear layernorm {M}x{N}x{K}"
+    ref, extra, scale, a, t = bitlinear_expected(xf, w, b, 1e-5, ln=(lw, lb))
+    assert_codes(g_xq, a["xq"], a["pre"], what + " xq")
+    rel32 = bitlinear_rel32(g_sc, a["act_scale"], host(ws_)[0], t["gamma"])
+    assert_out(host(o), ref, _TORCH_OUT[out], what, extra=extra, scale=scale, rel32=rel32)

@@ -421,3 +421,46 @@ def test_gemm_batched_is_per_batch_matmul_with_its_scales():
         acc = (x[b].astype(np.int64) @ w[b].astype(np.int64).T).astype(np.float64)
         ref = pts_b[2].astype(np.float64)[:, None] * acc * deq_b[1].astype(np.float64)[None, :]
         np.testing.assert_allclose(out_s[b], ref, rtol=1e-15, atol=0)
+
+
+# ------------------------------------------------ LayerNorm normaliser
+
+def test_layernorm_matches_torch_layer_norm():
+    g = synth.rng(20)
+    x = synth.normal_f32(g, (12, 300)) + np.float32(3.0)
+    x[4] *= 1e-4  # eps matters
+    w = (1.0 + 0.1 * g.standard_normal(300)).astype(np.float32)
+    b = (0.05 * g.standard_normal(300)).astype(np.float32)
+    for gw, gb in ((None, None), (w, b)):
+        y = oracle.act_quant_layernorm(x, 1e-5, gw, gb, want_y=True)["y"]
+        ref = torch.nn.functional.layer_norm(torch.from_numpy(x).double(), (300,),
+                                             None if gw is None else torch.from_numpy(gw).double(),
+                                             None if gb is None else torch.from_numpy(gb).double(),
+                                             eps=1e-5).numpy()
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_layernorm_quant_shift_invariant_and_centred():
+    # without the affine part the codes ignore a constant shift of the row
+    # (RMSNorm's codes would not) and are those of x - mean(x)
+    x = synth.normal_f32(synth.rng(21), (16, 256))
+    a = oracle.act_quant_layernorm(x)
+    b = oracle.act_quant_layernorm(x + np.float32(0.5))
+    c = oracle.act_quant(x - x.astype(np.float64).mean(axis=1, keepdims=True).astype(np.float32))
+    agree = (a["xq"] == b["xq"]).mean()
+    assert agree > 0.999  # the shift is exact in fp32 only up to rounding of x + 0.5
+    assert (a["xq"] == c["xq"]).mean() > 0.999
+    r = oracle.act_quant(x + np.float32(0.5))
+    assert (r["xq"] != a["xq"]).mean() > 0.1
+
+
+def test_layernorm_quant_constant_row_and_affine_closed_forms():
+    K = 64
+    x = np.full((1, K), 2.5, np.float32)
+    r = oracle.act_quant_layernorm(x)
+    assert np.all(r["xq"] == 0) and r["act_scale"][0] == 1e-5 / 127.0
+    # constant row with an affine bias: y = b exactly, so the codes quantize b
+    b = np.linspace(-1.0, 1.0, K).astype(np.float32)
+    r = oracle.act_quant_layernorm(x, ln_bias=b, want_pre=True)
+    np.testing.assert_allclose(r["pre"][0], b.astype(np.float64) * 127.0 / np.abs(b).max(), rtol=1e-15)
+    assert r["act_scale"][0] == pytest.approx(1.0 / 127.0, rel=1e-15)
