@@ -69,6 +69,8 @@ def parse_args():
     p.add_argument("--workloads", default="decode,w4,prefill,tiny,batched",
                    help="comma list of secondary workloads: decode, w4, prefill, tiny, batched")
     p.add_argument("--workload-steps", type=int, default=200)
+    p.add_argument("--decode-ms", default="1,4,16", help="token counts of the BitLinear decode workload")
+    p.add_argument("--w4-ms", default="1,32", help="token counts of the grouped INT4 workload")
     p.add_argument("--no-head", action="store_true", help="skip the headline GEMM (profiling runs only)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=0, help="oracle sample rows of the headline (0 = calibrate)")
@@ -445,9 +447,9 @@ def workloads(args, pk):
     steps = args.workload_steps
     want = set(args.workloads.split(","))
     if "decode" in want:
-        _decode(res, steps, hbm)
+        _decode(res, steps, hbm, [int(m) for m in args.decode_ms.split(",")])
     if "w4" in want:
-        _w4(res, steps, hbm)
+        _w4(res, steps, hbm, [int(m) for m in args.w4_ms.split(",")])
     if "prefill" in want:
         _prefill(res, max(steps // 4, 1), peak_int8, hbm)
     if "tiny" in want:
@@ -460,7 +462,7 @@ def workloads(args, pk):
     return res
 
 
-def _decode(res, steps, hbm):
+def _decode(res, steps, hbm, ms=(1, 4, 16)):
     import torch
 
     import bit_quantized_linear_rmsnorm_b200 as bq
@@ -471,7 +473,7 @@ def _decode(res, steps, hbm):
     del w
     copies = 24  # 24 x 11.3 MB = 270 MB > 2x L2
     wps = [wp.clone() for _ in range(copies)]
-    for M in (1, 4, 16):
+    for M in ms:
         d = synth.bitlinear_decode(M)
         x = torch.from_numpy(d["x_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
         out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
@@ -490,7 +492,7 @@ def _decode(res, steps, hbm):
     del wps
 
 
-def _w4(res, steps, hbm):
+def _w4(res, steps, hbm, ms=(1, 32)):
     import torch
 
     import bit_quantized_linear_rmsnorm_b200 as bq
@@ -503,7 +505,7 @@ def _w4(res, steps, hbm):
     bias = torch.from_numpy(wq["bias"]).cuda()
     copies = 10  # 10 x 30.6 MB = 306 MB
     sets = [(qw.clone(), sc.clone(), qz.clone()) for _ in range(copies)]
-    for M in (1, 32):
+    for M in ms:
         x = torch.from_numpy(synth.linear_w4_activations(M)).cuda()
         out = torch.empty((M, N), dtype=torch.float32, device="cuda")
         work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4_GROUPED, M, N, K, gs), dtype=torch.uint8,

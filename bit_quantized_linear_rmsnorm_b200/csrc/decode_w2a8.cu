@@ -724,11 +724,17 @@ cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStre
     }
 }
 
-// Register-streaming variant for 2..16 tokens on the mma.sync tensor path
-// (one m16n8k32 covers 16 rows x 32 K for eight tokens at once, where dp4a
-// would repeat the whole dot product per token).  Same launch shape as the
-// one-token kernel: 256 threads at most 128 registers, two CTAs per SM, one
-// CTA per SM per call, L2 prefetch before the dependency wait.
+// 2..16 tokens: two launches chained by programmatic dependent launch.
+//
+// 1. decode_token_quant_kernel (one CTA per token) quantizes each token once
+//    into the workspace (codes, act_scale, row sum).  It waits for the work
+//    before it in the stream (griddepcontrol.wait) before it lets its
+//    dependent start (griddepcontrol.launch_dependents).
+// 2. decode_w2a8_mma_kernel therefore starts only once everything before the
+//    call is complete and visible, so it loads its packed weights into
+//    registers at once (they stream from HBM while the tokens are quantized)
+//    and waits only for the codes; it copies them into shared memory and
+//    runs mma.sync m16n8k32 (u8 fields x s8 codes) from registers.
 //
 // Work unit = (16-row block rb, 256-wide K block kb); warp w takes the K
 // blocks kb = w + 8 c (c < KBW, K = 2048 KBW) of every row block.  Lane
@@ -740,87 +746,100 @@ cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStre
 // matching B fragment of token g is bytes 4 j .. 4 j + 3 of the two 16-byte
 // activation chunks 16 kb + 4 t + 2 s and + 1.  The four fields accumulate in
 // four accumulators, combined as acc0 + acc1 / 4 + acc2 / 16 + acc3 / 64
-// (each acc_j is a multiple of 4^j, so the shifts are exact).
+// (each acc_j is a multiple of 4^j, so the shifts are exact).  Each masked
+// fragment serves both token groups (tokens 0-7 and 8-15).
 constexpr int kMmaThreads = 256;
 constexpr int kMmaWarps = kMmaThreads / 32;
 constexpr int kMmaUnits = 10;  // units per warp held in registers
+constexpr int kTokThreads = 128;
 
 // 16-byte chunk c of a token row sits at chunk c ^ (2 ((c >> 3) & 1)): the
 // B-fragment loads of lanes t = 0..3 (chunks 4 t + const) and of consecutive
 // tokens (row pitch K + 16 bytes) then fall in distinct bank groups.
 __device__ __forceinline__ int xchunk_swz(int c) { return c ^ (((c >> 3) & 1) << 1); }
 
-// One warp quantizes one token row into the swizzled shared-memory row `dst`
-// (and the workspace row `ws` when not null).  Rows of up to 512 chunks stay
-// in registers between the statistics and the codes; longer rows are read
-// twice.
+// One CTA per token: RMSNorm statistics and codes of row blockIdx.x into the
+// workspace.  Chunk c of the row is held by thread c % 128 (at most CPT
+// 16-byte chunks per thread, K <= 4096 fp32 / 8192 bf16).
 template <typename InT>
-__device__ __forceinline__ void warp_quant_token_swz(const InT *__restrict__ xr, int K, float eps, int8_t *dst,
-                                                     int8_t *ws, float &scale, int &rowsum) {
+__global__ void __launch_bounds__(kTokThreads) decode_token_quant_kernel(const DecodeArgs p) {
     constexpr int EPC = Elt<InT>::kPerChunk;
-    constexpr int CPL = 16;
-    const int lane = threadIdx.x & 31;
+    constexpr int CPT = 8;
+    __shared__ float red[2][kTokThreads / 32];
+    __shared__ int redi[kTokThreads / 32];
+    // the row may come from the previous kernel, and the previous call's
+    // linear kernel may still read the workspace: wait, then release ours
+    pdl_wait();
+    pdl_launch_dependents();
+    const int m = blockIdx.x, K = p.K;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nch = K / EPC;
-    const uint4 *xv = reinterpret_cast<const uint4 *>(xr);
-    const bool cached = nch <= 32 * CPL;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K);
+    uint4 c[CPT];
     float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
-    uint4 c[CPL];
-    auto stats = [&](const uint4 &u) {
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int ch = threadIdx.x + kTokThreads * i;
+        c[i] = ch < nch ? __ldg(xv + ch) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
         float f[EPC];
-        Elt<InT>::unpack(u, f);
+        Elt<InT>::unpack(c[i], f);
 #pragma unroll
         for (int e = 0; e < EPC; e += 2) {
             ss0 = fmaf(f[e], f[e], ss0);
             ss1 = fmaf(f[e + 1], f[e + 1], ss1);
             amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
         }
-    };
-    if (cached) {
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int ch = lane + 32 * i;
-            c[i] = ch < nch ? __ldg(xv + ch) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) stats(c[i]);
-    } else {
-        for (int ch = lane; ch < nch; ch += 32) stats(__ldg(xv + ch));
     }
-    const float ss = warp_sum_f(ss0 + ss1);
+    float ss = warp_sum_f(ss0 + ss1);
     amax = warp_max_f(amax);
-    float fac;
-    quant_row_factor(ss, amax, K, eps, fac, scale);
-    int isum = 0;
-    auto codes = [&](const uint4 &u, int ch) {
-        float e[EPC];
-        Elt<InT>::unpack(u, e);
-        uint32_t w[EPC / 4];
-#pragma unroll
-        for (int j = 0; j < EPC / 4; ++j) {
-            w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
-                               fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
-            isum = dp4a_ss(w[j], 0x01010101u, isum);
-        }
-        const int o = ch * EPC;  // code byte offset
-        int8_t *d = dst + xchunk_swz(o >> 4) * 16 + (o & 15);
-        if constexpr (EPC == 8) {
-            *reinterpret_cast<uint2 *>(d) = make_uint2(w[0], w[1]);
-            if (ws) *reinterpret_cast<uint2 *>(ws + o) = make_uint2(w[0], w[1]);
-        } else {
-            *reinterpret_cast<uint32_t *>(d) = w[0];
-            if (ws) *reinterpret_cast<uint32_t *>(ws + o) = w[0];
-        }
-    };
-    if (cached) {
-#pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int ch = lane + 32 * i;
-            if (ch < nch) codes(c[i], ch);
-        }
-    } else {
-        for (int ch = lane; ch < nch; ch += 32) codes(__ldg(xv + ch), ch);
+    if (lane == 0) {
+        red[0][warp] = ss;
+        red[1][warp] = amax;
     }
-    rowsum = warp_sum_i(isum);
+    __syncthreads();
+    ss = red[0][0];
+    amax = red[1][0];
+#pragma unroll
+    for (int w = 1; w < kTokThreads / 32; ++w) {
+        ss += red[0][w];
+        amax = fmaxf(amax, red[1][w]);
+    }
+    float fac, scale;
+    quant_row_factor(ss, amax, K, p.eps, fac, scale);
+    int isum = 0;
+    int8_t *q = p.ws_xq + static_cast<int64_t>(m) * K;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int ch = threadIdx.x + kTokThreads * i;
+        if (ch < nch) {
+            float e[EPC];
+            Elt<InT>::unpack(c[i], e);
+            uint32_t w[EPC / 4];
+#pragma unroll
+            for (int j = 0; j < EPC / 4; ++j) {
+                w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
+                                   fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
+                isum = dp4a_ss(w[j], 0x01010101u, isum);
+            }
+            if constexpr (EPC == 8)
+                *reinterpret_cast<uint2 *>(q + ch * 8) = make_uint2(w[0], w[1]);
+            else
+                *reinterpret_cast<uint32_t *>(q + ch * 4) = w[0];
+        }
+    }
+    isum = warp_sum_i(isum);
+    if (lane == 0) redi[warp] = isum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int tot = 0;
+#pragma unroll
+        for (int w = 0; w < kTokThreads / 32; ++w) tot += redi[w];
+        p.ws_scale[m] = scale;
+        p.ws_rowsum[m] = tot;
+    }
 }
 
 template <typename OutT>
@@ -838,9 +857,10 @@ struct MmaLayout {
     static __host__ __device__ int bytes(int K) { return off_rowsum(K) + MT * 4; }
 };
 
-template <int MT, int KBW, typename InT>
-__global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const DecodeArgs p) {
+template <int MT, int KBW>
+__global__ void __launch_bounds__(kMmaThreads, 1) decode_w2a8_mma_kernel(const DecodeArgs p) {
     using L = MmaLayout<MT, KBW>;
+    constexpr int NH = MT / 8;  // token groups of eight
     extern __shared__ __align__(16) uint8_t smem[];
     const int K = p.K, M = p.M;
     const int xp = L::pitch(K);
@@ -854,29 +874,9 @@ __global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const D
     const int wpr = K / 16;  // packed words per row
     const uint32_t *wrow = p.wpacked + static_cast<int64_t>(rr.begin) * wpr;
 
-    for (int l = threadIdx.x; l < rr.rows * wpr / 32; l += kMmaThreads) prefetch_l2(wrow + 32 * l);
-    for (int i = threadIdx.x; i < L::kMaxRows * MT; i += kMmaThreads) rowacc[i] = 0;
-    pdl_launch_dependents();
-    pdl_wait();
-
-    // activations: warp w quantizes tokens w, w + 8 (codes stay out of registers)
-    for (int m = warp; m < M; m += kMmaWarps) {
-        float sc;
-        int rsum;
-        warp_quant_token_swz<InT>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K, K, p.eps,
-                                  xs + m * xp, blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(m) * K : nullptr,
-                                  sc, rsum);
-        if (lane == 0) {
-            s_scale[m] = sc;
-            s_rowsum[m] = rsum;
-            if (blockIdx.x == 0) {
-                p.ws_scale[m] = sc;
-                p.ws_rowsum[m] = rsum;
-            }
-        }
-    }
-
-    // this warp's weight words (unit i: row block i / KBW, K block warp + 8 (i % KBW))
+    // this warp's weight words (unit i: row block i / KBW, K block warp + 8 (i % KBW)),
+    // read before the dependency wait: the token kernel released this grid only
+    // after everything before the call had completed
     const int nrb = (rr.rows + 15) / 16;
     uint4 wa[kMmaUnits], wb[kMmaUnits];
 #pragma unroll
@@ -889,46 +889,67 @@ __global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const D
         wb[i] = r1 < rr.rows ? __ldcs(reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(r1) * wpr))
                              : make_uint4(0u, 0u, 0u, 0u);
     }
+    for (int i = threadIdx.x; i < L::kMaxRows * MT; i += kMmaThreads) rowacc[i] = 0;
     const float gamma = __ldg(p.w_scale);
+    pdl_launch_dependents();
+    pdl_wait();  // the token codes are written and visible
+
+    // token codes -> shared memory (swizzled rows), per-token scale and row sum
+    const int cpr = K / 16;  // 16-byte chunks per token row
+    for (int i = threadIdx.x; i < M * cpr; i += kMmaThreads) {
+        const int m = i / cpr, c = i - m * cpr;
+        *reinterpret_cast<uint4 *>(xs + m * xp + xchunk_swz(c) * 16) =
+            __ldcg(reinterpret_cast<const uint4 *>(p.ws_xq + static_cast<int64_t>(m) * K) + c);
+    }
+    if (threadIdx.x < M) {
+        s_scale[threadIdx.x] = __ldcg(p.ws_scale + threadIdx.x);
+        s_rowsum[threadIdx.x] = __ldcg(p.ws_rowsum + threadIdx.x);
+    }
     __syncthreads();
 
-    // token group h (tokens 8 h .. 8 h + 7) in the outer loop: one accumulator
-    // set live, kept across the KBW K blocks of a row block
+    // per unit: the masked A fragments once, both token groups; the
+    // accumulators of a row block are kept across its KBW K blocks
+    int acc[NH][4][4];
 #pragma unroll
-    for (int h = 0; h < MT / 8; ++h) {
-        const int tok = g + 8 * h;
-        int acc[4][4];
+    for (int i = 0; i < kMmaUnits; ++i) {
+        const int rb = i / KBW, kb = warp + kMmaWarps * (i % KBW);
+        if (i % KBW == 0) {
 #pragma unroll
-        for (int i = 0; i < kMmaUnits; ++i) {
-            const int rb = i / KBW, kb = warp + kMmaWarps * (i % KBW);
-            if (i % KBW == 0) {
+            for (int h = 0; h < NH; ++h)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0;
-            }
-            if (rb < nrb) {
+                for (int j = 0; j < 4; ++j) acc[h][j][0] = acc[h][j][1] = acc[h][j][2] = acc[h][j][3] = 0;
+        }
+        if (rb < nrb) {
 #pragma unroll
-                for (int s = 0; s < 2; ++s) {
+            for (int s = 0; s < 2; ++s) {
+                const uint32_t w0 = s ? wa[i].z : wa[i].x, w1 = s ? wa[i].w : wa[i].y;
+                const uint32_t v0 = s ? wb[i].z : wb[i].x, v1 = s ? wb[i].w : wb[i].y;
+                const int c0 = 16 * kb + 4 * t + 2 * s;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const int tok = g + 8 * h;
                     uint4 bx0 = make_uint4(0u, 0u, 0u, 0u), bx1 = make_uint4(0u, 0u, 0u, 0u);
                     if (tok < M) {
-                        const int c0 = 16 * kb + 4 * t + 2 * s;
                         bx0 = *reinterpret_cast<const uint4 *>(xs + tok * xp + xchunk_swz(c0) * 16);
                         bx1 = *reinterpret_cast<const uint4 *>(xs + tok * xp + xchunk_swz(c0 + 1) * 16);
                     }
-                    const uint32_t w0 = s ? wa[i].z : wa[i].x, w1 = s ? wa[i].w : wa[i].y;
-                    const uint32_t v0 = s ? wb[i].z : wb[i].x, v1 = s ? wb[i].w : wb[i].y;
                     const uint32_t b0[4] = {bx0.x, bx0.y, bx0.z, bx0.w}, b1[4] = {bx1.x, bx1.y, bx1.z, bx1.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t mk = 0x03030303u << (2 * j);
                         const uint32_t a[4] = {w0 & mk, v0 & mk, w1 & mk, v1 & mk};
-                        mma_u8s8_16832(acc[j], a, b0[j], b1[j]);
+                        mma_u8s8_16832(acc[h][j], a, b0[j], b1[j]);
                     }
                 }
-                if (i % KBW == KBW - 1) {  // last K block of this row block: combine and flush
+            }
+            if (i % KBW == KBW - 1) {  // last K block of this row block: combine and flush
+                const int r0 = rb * 16 + g, r1 = r0 + 8;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
                     int v[4];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) v[c] = acc[0][c] + (acc[1][c] >> 2) + (acc[2][c] >> 4) + (acc[3][c] >> 6);
-                    const int r0 = rb * 16 + g, r1 = r0 + 8;
+                    for (int c = 0; c < 4; ++c)
+                        v[c] = acc[h][0][c] + (acc[h][1][c] >> 2) + (acc[h][2][c] >> 4) + (acc[h][3][c] >> 6);
                     const int m0 = 2 * t + 8 * h, m1 = m0 + 1;
                     if (r0 < rr.rows && m0 < M) atomicAdd(&rowacc[r0 * MT + m0], v[0]);
                     if (r0 < rr.rows && m1 < M) atomicAdd(&rowacc[r0 * MT + m1], v[1]);
@@ -956,16 +977,10 @@ __global__ void __launch_bounds__(kMmaThreads, 2) decode_w2a8_mma_kernel(const D
     }
 }
 
-template <int MT, int KBW, typename InT>
-cudaError_t launch_mma_t(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
-    auto kern = decode_w2a8_mma_kernel<MT, KBW, InT>;
-    const int smem = MmaLayout<MT, KBW>::bytes(a.K);
-    static SmemOptIn opt_in;
-    const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
-    if (e != cudaSuccess) return e;
+cudaError_t launch_pdl_cfg(const void *kern, const DecodeArgs &a, int grid, int threads, int smem, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(kMmaThreads);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -973,7 +988,20 @@ cudaError_t launch_mma_t(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    void *args[] = {const_cast<DecodeArgs *>(&a)};
+    return cudaLaunchKernelExC(&cfg, kern, args);
+}
+
+template <int MT, int KBW, typename InT>
+cudaError_t launch_mma_t(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
+    auto kern = decode_w2a8_mma_kernel<MT, KBW>;
+    const int smem = MmaLayout<MT, KBW>::bytes(a.K);
+    static SmemOptIn opt_in;
+    cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
+    if (e != cudaSuccess) return e;
+    e = launch_pdl_cfg(reinterpret_cast<const void *>(decode_token_quant_kernel<InT>), a, a.M, kTokThreads, 0, s);
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cfg(reinterpret_cast<const void *>(kern), a, grid, kMmaThreads, smem, s);
 }
 
 template <typename InT>
