@@ -66,8 +66,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-workloads", action="store_true", help="skip the secondary workloads")
-    p.add_argument("--workloads", default="decode,w4,prefill,tiny,batched",
-                   help="comma list of secondary workloads: decode, w4, prefill, tiny, batched")
+    p.add_argument("--workloads", default="decode,w4,prefill,tiny,batched,w4a4,layernorm,conv",
+                   help="comma list of secondary workloads: decode, w4, prefill, tiny, batched, w4a4, layernorm, conv")
     p.add_argument("--workload-steps", type=int, default=200)
     p.add_argument("--decode-ms", default="1,4,16", help="token counts of the BitLinear decode workload")
     p.add_argument("--w4-ms", default="1,32", help="token counts of the grouped INT4 workload")
@@ -456,6 +456,12 @@ def workloads(args, pk):
         _tiny(res, steps)
     if "batched" in want:
         _batched(res, steps, peak_int8)
+    if "w4a4" in want:
+        _w4a4(res, steps, peak_int8, hbm)
+    if "layernorm" in want:
+        _layernorm(res, steps, peak_int8, hbm)
+    if "conv" in want:
+        _conv(res, max(steps // 4, 1), peak_int8)
     st, detail = bq.bq_device_status()
     if st != bq.BQ_OK:
         raise RuntimeError(f"device status {detail:#x} after the workloads")
@@ -488,7 +494,8 @@ def _decode(res, steps, hbm, ms=(1, 4, 16)):
         res[f"bitlinear_decode_M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
                                          "frac_hbm": round(gbs / hbm, 4), "algorithmic_bytes": byts,
                                          "weight_GB/s": round((N * K // 4) / (ms * 1e-3) / 1e9, 1),
-                                         "launches_per_step": 1, "config": f"x bf16 [{M},4096], W 2-bit [11008,4096]"}
+                                         "launches_per_step": 1 if M == 1 else 2,
+                                         "config": f"x bf16 [{M},4096], W 2-bit [11008,4096]"}
     del wps
 
 
@@ -630,6 +637,112 @@ def _batched(res, steps, peak_int8):
                                "frac_int8_peak": round(ops / (ms * 1e-3) / 1e12 / peak_int8, 4),
                                "config": "x int8 stored [4096 (K), 4096 (M)] (transposeA) x w [4096,4096] (N,K), "
                                          "single-CTA tiles, bf16 out"}
+
+
+def _w4a4(res, steps, peak_int8, hbm):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
+    # 4-bit activations / 4-bit weights with given steps: prefill 4096^3 and one-token decode 11008 x 4096
+    eps = 1e-6
+    for (M, N, K, tag) in ((4096, 4096, 4096, "w4a4_prefill_4096"), (1, 11008, 4096, "w4a4_decode_M1")):
+        g = synth.rng((41, M, N))
+        x = torch.from_numpy(synth.f32_to_bf16_bits(synth.normal_f32(g, (M, K))).view(np.int16)).cuda().view(
+            torch.bfloat16)
+        w = torch.from_numpy(synth.normal_f32(g, (N, K), 0.02)).cuda()
+        sa = torch.tensor([0.27], dtype=torch.float32, device="cuda")
+        sw = (w.abs().amax(dim=1) / 7.5).contiguous()
+        wp = bq.bq_weight_quant_int4_pack(w, sw, eps)
+        del w
+        copies = max(1, min(24, int(300e6 // (N * K // 2))))
+        wps = [wp.clone() for _ in range(copies)]
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4A4, M, N, K), dtype=torch.uint8, device="cuda")
+
+        def step(i, x=x, sa=sa, sw=sw, out=out, work=work, wps=wps):
+            bq.bq_linear_w4a4(x, sa, wps[i % len(wps)], sw, N, eps, out=out, workspace=work)
+
+        ms, _, _ = graph_time(step, steps if M == 1 else max(steps // 4, 1), 3)
+        if M == 1:
+            byts = N * K // 2 + 4 * N + 2 * K + 2 * N
+            gbs = byts / (ms * 1e-3) / 1e9
+            res[tag] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                        "algorithmic_bytes": byts, "config": "x bf16 [1,4096], W 4-bit [11008,4096], per-channel steps; "
+                                                             "act quant + dp4a GEMV"}
+        else:
+            ops = 2.0 * M * N * K
+            tops = ops / (ms * 1e-3) / 1e12
+            res[tag] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(tops, 1),
+                        "frac_int8_peak": round(tops / peak_int8, 4),
+                        "config": "x bf16 [4096,4096], W 4-bit [4096,4096], per-channel steps; act quant + tcgen05 "
+                                  "GEMM with the nibbles sign-extended in shared memory"}
+        del wps
+
+
+def _layernorm(res, steps, peak_int8, hbm):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
+    # BitLinear with the LayerNorm normaliser: prefill 8192 x 4096 x 4096, one-token decode 11008 x 4096
+    for (M, N, K, tag) in ((8192, 4096, 4096, "bitlinear_ln_prefill"), (1, 11008, 4096, "bitlinear_ln_decode_M1")):
+        g = synth.rng((42, M, N))
+        x = torch.from_numpy(synth.f32_to_bf16_bits(synth.normal_f32(g, (M, K)) + np.float32(0.75)).view(np.int16)
+                             ).cuda().view(torch.bfloat16)
+        lw = torch.from_numpy((1.0 + 0.2 * g.standard_normal(K)).astype(np.float32)).cuda()
+        lb = torch.from_numpy((0.1 * g.standard_normal(K)).astype(np.float32)).cuda()
+        wp, wsc = bq.bq_weight_quant_ternary_pack(torch.from_numpy(synth.bitlinear_weight(N, K, 6)).cuda())
+        copies = max(1, min(24, int(300e6 // (N * K // 4))))
+        wps = [wp.clone() for _ in range(copies)]
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, M, N, K), dtype=torch.uint8, device="cuda")
+
+        def step(i, x=x, out=out, work=work, wps=wps, wsc=wsc, lw=lw, lb=lb):
+            bq.bq_bitlinear_w2a8_layernorm(x, wps[i % len(wps)], wsc, N, lw, lb, None, 1e-5, out=out, workspace=work)
+
+        ms, _, _ = graph_time(step, steps if M == 1 else max(steps // 4, 1), 3)
+        if M == 1:
+            byts = N * K // 4 + 2 * K + 8 * K + 2 * N
+            gbs = byts / (ms * 1e-3) / 1e9
+            res[tag] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                        "algorithmic_bytes": byts, "config": "x bf16 [1,4096], affine LayerNorm, W 2-bit [11008,4096]; "
+                                                             "binary64 LayerNorm quant + split GEMV"}
+        else:
+            ops = 2.0 * M * N * K
+            tops = ops / (ms * 1e-3) / 1e12
+            res[tag] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(tops, 1),
+                        "frac_int8_peak": round(tops / peak_int8, 4),
+                        "config": "x bf16 [8192,4096], affine LayerNorm, W 2-bit [4096,4096]; binary64 LayerNorm "
+                                  "quant + tcgen05 GEMM"}
+        del wps
+
+
+def _conv(res, steps, peak_int8):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
+    # BitConv1d: x (8, 1024, 1024) -> (8, 1024, 1024), kernel 3, padding 1
+    B, C_in, L, C_out, KS = 8, 1024, 1024, 1024, 3
+    g = synth.rng(43)
+    x = torch.from_numpy(synth.f32_to_bf16_bits(synth.normal_f32(g, (B, C_in, L))).view(np.int16)).cuda().view(
+        torch.bfloat16)
+    wp, wsc = bq.bq_bitconv1d_weight_pack(torch.from_numpy(synth.normal_f32(g, (C_out, C_in, KS), 0.02)).cuda())
+    out = torch.empty((B, C_out, L), dtype=torch.bfloat16, device="cuda")
+    work = torch.empty(bq.lib().bq_bitconv1d_workspace_bytes(B, C_in, L, C_out, KS, 1, 1, 1), dtype=torch.uint8,
+                       device="cuda")
+
+    def step(i):
+        bq.bq_bitconv1d(x, wp, wsc, C_out, KS, 1, 1, 1, out=out, workspace=work)
+
+    ms, _, _ = graph_time(step, steps, 3)
+    ops = 2.0 * B * L * C_out * C_in * KS
+    tops = ops / (ms * 1e-3) / 1e12
+    res["bitconv1d_8x1024x1024_k3"] = {"us_per_step": round(ms * 1e3, 2), "TOPS": round(tops, 1),
+                                       "frac_int8_peak": round(tops / peak_int8, 4),
+                                       "config": "x bf16 (8, 1024, 1024), W [1024, 1024, 3] ternary, padding 1; "
+                                                 "transpose, LayerNorm quant, 3 x (gather + tcgen05 GEMM), tap sum"}
 
 
 # ---------------------------------------------------------------------------

@@ -22,12 +22,14 @@ BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_MISALIGNED, BQ_ERR_WORKSPA
 BQ_F32, BQ_BF16, BQ_F16 = 0, 1, 2
 BQ_W_NK, BQ_W_KN = 0, 1
 (BQ_OP_ACT_QUANT_INT8, BQ_OP_WEIGHT_QUANT_TERNARY_PACK, BQ_OP_WEIGHT_PACK_INT4_GROUPED,
- BQ_OP_GEMM_I8_PERTOKEN, BQ_OP_BITLINEAR_W2A8, BQ_OP_LINEAR_W4_GROUPED) = range(6)
+ BQ_OP_GEMM_I8_PERTOKEN, BQ_OP_BITLINEAR_W2A8, BQ_OP_LINEAR_W4_GROUPED, BQ_OP_LINEAR_W4A4) = range(7)
 
 EXPORTED = [
     "bq_act_quant_int8", "bq_weight_quant_ternary_pack", "bq_weight_pack_int4_grouped",
     "bq_gemm_i8_pertoken", "bq_gemm_i8_pertoken_batched", "bq_bitlinear_w2a8", "bq_act_quant_int8_layernorm",
-    "bq_bitlinear_w2a8_layernorm", "bq_linear_w4_grouped", "bq_workspace_bytes",
+    "bq_bitlinear_w2a8_layernorm", "bq_weight_quant_int4_pack", "bq_act_quant_int4", "bq_linear_w4a4",
+    "bq_bitconv1d_weight_pack_workspace_bytes", "bq_bitconv1d_weight_pack", "bq_bitconv1d_workspace_bytes",
+    "bq_bitconv1d", "bq_linear_w4_grouped", "bq_workspace_bytes",
     "bq_bitlinear_workspace_layout", "bq_status_string", "bq_device_status", "bq_version",
     "bq_bitlinear_w2a8_noalloc", "bq_bitlinear_w2a8_path", "bq_diag_gemm_withheld_arrival",
 ]
@@ -57,6 +59,13 @@ _SIGS = {
     "bq_bitlinear_w2a8_noalloc": (I32, [P, I32, I64, I64, P, P, I64, P, F32, I32, P, P]),
     "bq_bitlinear_w2a8_path": (I32, [P, I32, I64, I64, I64, ctypes.POINTER(I32)]),
     "bq_diag_gemm_withheld_arrival": (I32, [P, P, P, P, P, ctypes.c_uint64, P]),
+    "bq_weight_quant_int4_pack": (I32, [P, I32, I64, I64, P, I32, F32, P, P]),
+    "bq_act_quant_int4": (I32, [P, I32, I64, I64, I64, P, F32, P, I64, P]),
+    "bq_linear_w4a4": (I32, [P, I32, I64, I64, P, P, P, I32, I64, P, F32, I32, P, P, SZ, P]),
+    "bq_bitconv1d_weight_pack_workspace_bytes": (SZ, [I64, I64, I64]),
+    "bq_bitconv1d_weight_pack": (I32, [P, I32, I64, I64, I64, P, P, P, SZ, P]),
+    "bq_bitconv1d_workspace_bytes": (SZ, [I64, I64, I64, I64, I64, I64, I64, I64]),
+    "bq_bitconv1d": (I32, [P, I32, I64, I64, I64, P, P, P, P, I64, I64, I64, I64, I64, P, F32, I32, P, P, SZ, P]),
     "bq_workspace_bytes": (SZ, [I32, I64, I64, I64, I64]),
     "bq_bitlinear_workspace_layout": (None, [I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     "bq_status_string": (ctypes.c_char_p, [I32]),
@@ -322,3 +331,76 @@ def bq_bitlinear_w2a8_path(x: torch.Tensor, N: int) -> int:
     st = lib().bq_bitlinear_w2a8_path(_ptr(x), _DTYPE[x.dtype], M, N, K, ctypes.byref(path))
     _check(st, "bq_bitlinear_w2a8_path")
     return path.value
+
+
+def bq_weight_quant_int4_pack(w: torch.Tensor, scale_w: torch.Tensor, eps: float, wpacked=None, stream=None):
+    """Signed 4-bit codes of w [N,K] with step max(scale_w, eps) (scale_w one
+    value or [N]), packed eight per word: int32 [N, K/8]."""
+    N, K = w.shape
+    if wpacked is None:
+        wpacked = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    per_channel = 1 if scale_w.numel() == N and N > 1 else 0
+    st = lib().bq_weight_quant_int4_pack(_ptr(w), _DTYPE[w.dtype], N, K, _ptr(scale_w), per_channel, float(eps),
+                                         _ptr(wpacked), _stream(stream))
+    _check(st, "bq_weight_quant_int4_pack")
+    return wpacked
+
+
+def bq_act_quant_int4(x: torch.Tensor, scale_a: torch.Tensor, eps: float, xq=None, stream=None):
+    """Signed 4-bit codes of x [M,K] (as int8) with step max(scale_a, eps)."""
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    st = lib().bq_act_quant_int4(_ptr(x), _DTYPE[x.dtype], M, K, _ld(x), _ptr(scale_a), float(eps), _ptr(xq), _ld(xq),
+                                 _stream(stream))
+    _check(st, "bq_act_quant_int4")
+    return xq
+
+
+def bq_linear_w4a4(x: torch.Tensor, scale_a: torch.Tensor, wpacked: torch.Tensor, scale_w: torch.Tensor, N: int,
+                   eps: float, bias=None, out_dtype=torch.bfloat16, out=None, workspace=None, stream=None):
+    """Forward of the 4-bit activation / 4-bit weight linear with given steps."""
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    per_channel = 1 if scale_w.numel() == N and N > 1 else 0
+    nbytes = bq_workspace_bytes(BQ_OP_LINEAR_W4A4, M, N, K)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().bq_linear_w4a4(_ptr(x), _DTYPE[x.dtype], M, K, _ptr(scale_a), _ptr(wpacked), _ptr(scale_w),
+                              per_channel, N, _ptr(bias), float(eps), _DTYPE[out.dtype], _ptr(out), _ptr(ws),
+                              ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bq_linear_w4a4")
+    return out
+
+
+def bq_bitconv1d_weight_pack(w: torch.Tensor, wpacked=None, w_scale=None, workspace=None, stream=None):
+    """Ternary codes of a Conv1d weight [C_out, Cg, KS] packed per tap:
+    (wpacked int32 [KS, C_out, Cgp/16], w_scale fp32 [1])."""
+    C_out, Cg, KS = w.shape
+    Cgp = (Cg + 63) // 64 * 64
+    if wpacked is None:
+        wpacked = torch.empty((KS, C_out, Cgp // 16), dtype=torch.int32, device=w.device)
+    if w_scale is None:
+        w_scale = torch.empty(1, dtype=torch.float32, device=w.device)
+    ws = _workspace(int(lib().bq_bitconv1d_weight_pack_workspace_bytes(C_out, Cg, KS)), w.device, workspace)
+    st = lib().bq_bitconv1d_weight_pack(_ptr(w.contiguous()), _DTYPE[w.dtype], C_out, Cg, KS, _ptr(wpacked),
+                                        _ptr(w_scale), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bq_bitconv1d_weight_pack")
+    return wpacked, w_scale
+
+
+def bq_bitconv1d(x: torch.Tensor, wpacked: torch.Tensor, w_scale: torch.Tensor, C_out: int, kernel_size: int,
+                 stride: int = 1, padding: int = 0, groups: int = 1, ln_weight=None, ln_bias=None, bias=None,
+                 eps: float = 1e-5, out_dtype=torch.bfloat16, out=None, workspace=None, stream=None):
+    """Ternary Conv1d forward: x (B, C_in, L) -> (B, C_out, L_out)."""
+    B, C_in, L = x.shape
+    L_out = (L + 2 * padding - kernel_size) // stride + 1
+    if out is None:
+        out = torch.empty((B, C_out, L_out), dtype=out_dtype, device=x.device)
+    nbytes = int(lib().bq_bitconv1d_workspace_bytes(B, C_in, L, C_out, kernel_size, stride, padding, groups))
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().bq_bitconv1d(_ptr(x), _DTYPE[x.dtype], B, C_in, L, _ptr(ln_weight), _ptr(ln_bias), _ptr(wpacked),
+                            _ptr(w_scale), C_out, kernel_size, stride, padding, groups, _ptr(bias), float(eps),
+                            _DTYPE[out.dtype], _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bq_bitconv1d")
+    return out

@@ -1,0 +1,234 @@
+// Ternary Conv1d ("Common Attention Utilities", frankenstein-transformer,
+// BitConv1d: the ternary weights and 8-bit activations of BitLinear; the input
+// (B, C_in, L) is LayerNorm-normalised over the channels at every position
+// before the activation quantization; output (B, C_out, L_out)).
+//
+//   out[b,co,lo] = gamma * sum_t act_scale[b,p] * sum_c wq[co,c,t] * xq[b,p,g Cg + c]  (+ bias[co])
+//   p = lo * stride + t - pad,  L_out = (L + 2 pad - KS) / stride + 1
+//
+// The activation scale belongs to the input position, so each tap is its own
+// integer contraction over the channels, scaled by the scale of the position
+// it reads.  The path:
+//   1. x (B, C_in, L) -> rows [B*L][C_in] (tiled transpose through shared memory);
+//   2. LayerNorm + per-position int8 quantization of those rows (the binary64
+//      kernel of act_quant_ln.cu): codes and scales;
+//   3. per tap t: the rows read by the tap gathered into [B*L_out][C_in]
+//      (zero rows and scale where the tap falls into the padding) with their
+//      code sums per channel group, then per group the ternary tcgen05 GEMM
+//      against the tap's packed weights [C_out/groups][C_in/groups], which
+//      computes (acc - rowsum) * scale * gamma in fp32;
+//   4. the taps summed in fp32 (+ bias), rounded once and transposed into
+//      (B, C_out, L_out).
+// Weights are packed per tap by bq_bitconv1d_weight_pack: [KS][C_out][Cgp/16]
+// words with Cgp = Cg rounded up to 64 (16-byte row pitch for the tensor copy).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <type_traits>
+
+#include "bq_internal.h"
+
+namespace bq {
+namespace {
+
+// 32 x 32 tiles: src [batch][R][C] -> dst [batch][C][R] (element type T).
+template <typename T>
+__global__ void transpose_kernel(const T *__restrict__ src, int64_t R, int64_t C, T *__restrict__ dst) {
+    __shared__ T tile[32][33];
+    const int64_t b = blockIdx.z;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+    const T *s = src + b * R * C;
+    T *d = dst + b * R * C;
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t r = r0 + i, c = c0 + threadIdx.x;
+        if (r < R && c < C) tile[i][threadIdx.x] = s[r * C + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t c = c0 + i, r = r0 + threadIdx.x;
+        if (r < R && c < C) d[c * R + r] = tile[threadIdx.x][i];
+    }
+}
+
+template <typename T>
+cudaError_t transpose(const T *src, int64_t batch, int64_t R, int64_t C, T *dst, cudaStream_t s) {
+    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32),
+                    static_cast<unsigned>(batch));
+    transpose_kernel<T><<<grid, dim3(32, 8), 0, s>>>(src, R, C, dst);
+    return cudaGetLastError();
+}
+
+// Rows of tap t: row (b, lo) of the gathered codes is row (b, p) of xq, p =
+// lo * stride + t - pad, or zeros outside [0, L); rs[row] is that position's
+// scale (0 outside) and rc[g * rows + row] the sum of its codes over the
+// channels of group g (the offset-binary correction of that group's product).
+__global__ void tap_gather_kernel(const int8_t *__restrict__ xq, const float *__restrict__ act_scale, int64_t B,
+                                  int64_t C_in, int64_t L, int64_t L_out, int64_t stride, int64_t pad, int64_t t,
+                                  int64_t groups, int8_t *__restrict__ a, float *__restrict__ rs,
+                                  int32_t *__restrict__ rc) {
+    const int64_t rows = B * L_out, chunks = C_in / 16, Cg = C_in / groups;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = tid; i < rows * chunks; i += nth) {
+        const int64_t row = i / chunks, c = i - row * chunks;
+        const int64_t b = row / L_out, lo = row - b * L_out, p = lo * stride + t - pad;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (p >= 0 && p < L) v = __ldg(reinterpret_cast<const uint4 *>(xq + (b * L + p) * C_in) + c);
+        reinterpret_cast<uint4 *>(a + row * C_in)[c] = v;
+    }
+    for (int64_t i = tid; i < rows * groups; i += nth) {
+        const int64_t g = i / rows, row = i - g * rows;
+        const int64_t b = row / L_out, lo = row - b * L_out, p = lo * stride + t - pad;
+        const bool in = p >= 0 && p < L;
+        int sum = 0;
+        if (in) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xq + (b * L + p) * C_in + g * Cg);
+            for (int64_t c = 0; c < Cg / 16; ++c) {
+                const uint4 v = __ldg(src + c);
+                sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
+                sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
+                sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
+                sum = __dp4a(static_cast<int>(v.w), 0x01010101, sum);
+            }
+        }
+        rc[g * rows + row] = sum;
+        if (g == 0) rs[row] = in ? __ldg(act_scale + b * L + p) : 0.0f;
+    }
+}
+
+// out[b, co, lo] = sum_t part[t][(b L_out + lo) * ldp + co] (+ bias[co]), through
+// 32 x 32 shared-memory tiles (reads along co, writes along lo).
+template <typename OutT>
+__global__ void tap_sum_kernel(const float *__restrict__ part, int64_t KS, int64_t B, int64_t L_out, int64_t C_out,
+                               int64_t ldp, const float *__restrict__ bias, OutT *__restrict__ out) {
+    __shared__ float tile[32][33];
+    const int64_t b = blockIdx.z;
+    const int64_t l0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+    const int64_t tap_stride = B * L_out * ldp;
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t lo = l0 + i, co = c0 + threadIdx.x;
+        float v = 0.0f;
+        if (lo < L_out && co < C_out) {
+            const float *p = part + (b * L_out + lo) * ldp + co;
+            for (int64_t t = 0; t < KS; ++t) v = __fadd_rn(v, p[t * tap_stride]);
+            if (bias != nullptr) v = __fadd_rn(v, __ldg(bias + co));
+        }
+        tile[i][threadIdx.x] = v;
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int64_t co = c0 + i, lo = l0 + threadIdx.x;
+        if (lo < L_out && co < C_out) {
+            const float v = tile[threadIdx.x][i];
+            OutT o;
+            if constexpr (sizeof(OutT) == 4)
+                o = v;
+            else if constexpr (std::is_same<OutT, __half>::value)
+                o = __float2half_rn(v);
+            else
+                o = __float2bfloat16_rn(v);
+            out[(b * C_out + co) * L_out + lo] = o;
+        }
+    }
+}
+
+inline size_t a256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+BitconvLayout bitconv_layout(int64_t B, int64_t C_in, int64_t L, int64_t C_out, int64_t KS, int64_t stride,
+                             int64_t pad, int64_t groups) {
+    BitconvLayout l;
+    l.L_out = (L + 2 * pad - KS) / stride + 1;
+    l.ldp = (C_out + 3) / 4 * 4;
+    const size_t rows = static_cast<size_t>(B * L), orows = static_cast<size_t>(B * l.L_out);
+    l.xt = 0;
+    l.xq = l.xt + a256(rows * static_cast<size_t>(C_in) * 4);
+    l.scale = l.xq + a256(rows * static_cast<size_t>(C_in));
+    l.a = l.scale + a256(rows * 4);
+    l.rs = l.a + a256(orows * static_cast<size_t>(C_in));
+    l.rc = l.rs + a256(orows * 4);
+    l.part = l.rc + a256(orows * static_cast<size_t>(groups) * 4);
+    l.total = l.part + a256(static_cast<size_t>(KS) * orows * static_cast<size_t>(l.ldp) * 4);
+    return l;
+}
+
+cudaError_t launch_bitconv_weight_transpose(const void *w, bq_dtype wt, int64_t C_out, int64_t Cg, int64_t KS,
+                                            void *dst, cudaStream_t s) {
+    // [C_out * Cg][KS] -> [KS][C_out * Cg]
+    if (wt == BQ_BF16)
+        return transpose(static_cast<const __nv_bfloat16 *>(w), 1, C_out * Cg, KS, static_cast<__nv_bfloat16 *>(dst),
+                         s);
+    return transpose(static_cast<const float *>(w), 1, C_out * Cg, KS, static_cast<float *>(dst), s);
+}
+
+bq_status launch_bitconv1d(const void *x, bq_dtype xt, int64_t B, int64_t C_in, int64_t L, const float *ln_weight,
+                           const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t C_out,
+                           int64_t KS, int64_t stride, int64_t pad, int64_t groups, const float *bias, float eps,
+                           bq_dtype out_dtype, void *out, void *workspace, cudaStream_t s, const DevInfo &dev) {
+    const BitconvLayout l = bitconv_layout(B, C_in, L, C_out, KS, stride, pad, groups);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    // 1. (B, C_in, L) -> [B*L][C_in]
+    cudaError_t e = xt == BQ_BF16 ? transpose(static_cast<const __nv_bfloat16 *>(x), B, C_in, L,
+                                              reinterpret_cast<__nv_bfloat16 *>(ws + l.xt), s)
+                                  : transpose(static_cast<const float *>(x), B, C_in, L,
+                                              reinterpret_cast<float *>(ws + l.xt), s);
+    if (e != cudaSuccess) return BQ_ERR_CUDA;
+    // 2. per-position LayerNorm + int8 codes
+    int8_t *xq = reinterpret_cast<int8_t *>(ws + l.xq);
+    float *act_scale = reinterpret_cast<float *>(ws + l.scale);
+    e = launch_act_quant_ln(ws + l.xt, xt, B * L, C_in, C_in, ln_weight, ln_bias, eps, xq, C_in, act_scale, nullptr, s,
+                            dev);
+    if (e != cudaSuccess) return BQ_ERR_CUDA;
+    // 3. per tap: gather, ternary GEMM into the tap's fp32 partial
+    const int64_t orows = B * l.L_out, Cg = C_in / groups, Cog = C_out / groups, Cgp = (Cg + 63) / 64 * 64;
+    int8_t *a = reinterpret_cast<int8_t *>(ws + l.a);
+    float *rs = reinterpret_cast<float *>(ws + l.rs);
+    int32_t *rc = reinterpret_cast<int32_t *>(ws + l.rc);  // [groups][rows]
+    float *part = reinterpret_cast<float *>(ws + l.part);
+    const int ggrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((orows * (C_in / 16) + 255) / 256,
+                                                                               dev.num_sms * 8)));
+    for (int64_t t = 0; t < KS; ++t) {
+        tap_gather_kernel<<<ggrid, 256, 0, s>>>(xq, act_scale, B, C_in, L, l.L_out, stride, pad, t, groups, a, rs, rc);
+        if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
+        for (int64_t gr = 0; gr < groups; ++gr) {  // group gr: its channels, weight rows and output columns
+            GemmArgs g;
+            g.a = a + gr * Cg;
+            g.lda = C_in;
+            g.b = wpacked + (t * C_out + gr * Cog) * (Cgp / 16);
+            g.ldb = Cgp / 16;
+            g.b_pack = 2;
+            g.colscale = w_scale;
+            g.rowscale = rs;
+            g.rowcorr = rc + gr * orows;
+            g.M = orows;
+            g.N = Cog;
+            g.K = Cg;
+            g.out_dtype = BQ_F32;
+            g.out = part + t * orows * l.ldp + gr * Cog;
+            g.ldo = l.ldp;
+            const bq_status st = launch_gemm_tc(g, s, dev);
+            if (st != BQ_OK) return st;
+        }
+    }
+    // 4. sum the taps (+ bias), transpose to (B, C_out, L_out)
+    const dim3 grid(static_cast<unsigned>((C_out + 31) / 32), static_cast<unsigned>((l.L_out + 31) / 32),
+                    static_cast<unsigned>(B));
+    switch (out_dtype) {
+        case BQ_F32:
+            tap_sum_kernel<float><<<grid, dim3(32, 8), 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
+                                                               static_cast<float *>(out));
+            break;
+        case BQ_F16:
+            tap_sum_kernel<__half><<<grid, dim3(32, 8), 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
+                                                                static_cast<__half *>(out));
+            break;
+        default:
+            tap_sum_kernel<__nv_bfloat16><<<grid, dim3(32, 8), 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
+                                                                       static_cast<__nv_bfloat16 *>(out));
+    }
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+}  // namespace bq

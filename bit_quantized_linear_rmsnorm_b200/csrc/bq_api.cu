@@ -96,6 +96,23 @@ constexpr int kGemvMaxM = 16;
 struct BitlinearLayout {
     size_t xq, scale, rowsum, wpad, opad, total;
 };
+// Workspace of bq_linear_w4a4: xq [M][K] int8, the per-row step [M] and the
+// per-channel step [N] (fp32), and for more than 16 tokens with
+// N * size(out) % 16 != 0 an output staging buffer (rows padded to 8 elements).
+struct W4a4Layout {
+    size_t xq, row, col, opad, total;
+};
+W4a4Layout w4a4_layout(int64_t M, int64_t N, int64_t K) {
+    W4a4Layout l;
+    l.xq = 0;
+    l.row = align256(static_cast<size_t>(M) * static_cast<size_t>(K));
+    l.col = l.row + align256(static_cast<size_t>(M) * 4);
+    l.opad = l.col + align256(static_cast<size_t>(N) * 4);
+    l.total = l.opad;
+    if (M > kGemvMaxM && N % 8 != 0) l.total += align256(static_cast<size_t>(M) * static_cast<size_t>((N + 7) / 8 * 8) * 4);
+    return l;
+}
+
 BitlinearLayout bitlinear_layout(int64_t M, int64_t N, int64_t K) {
     BitlinearLayout l;
     l.xq = 0;
@@ -177,6 +194,8 @@ size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t gro
         case BQ_OP_LINEAR_W4_GROUPED:
             if (group_size <= 0) return 0;
             return linear_w4_workspace_bytes(M, N, K, group_size);
+        case BQ_OP_LINEAR_W4A4:
+            return w4a4_layout(M, N, K).total;
         default:
             return 0;
     }
@@ -347,7 +366,7 @@ static bq_status bitlinear_linear(int path, const BitlinearLayout &l, uint8_t *w
     g.lda = K;
     g.b = wrows;
     g.ldb = ldb;
-    g.b_packed2 = true;
+    g.b_pack = 2;
     g.colscale = w_scale;
     g.rowscale = act_scale;
     g.rowcorr = rowsum;
@@ -473,6 +492,157 @@ bq_status bq_diag_gemm_withheld_arrival(const int8_t *x, const int8_t *w, const 
     g.withhold_kb = 1;
     if (gemm_uses_pair(false, BQ_W_NK, g.M, g.N, dev)) return BQ_ERR_UNSUPPORTED;  // (a one-tile grid never pairs)
     return launch_gemm_tc(g, static_cast<cudaStream_t>(stream), dev);
+}
+
+bq_status bq_weight_quant_int4_pack(const void *w, bq_dtype w_dtype, int64_t N, int64_t K, const float *scale_w,
+                                    int scale_w_per_channel, float eps, uint32_t *wpacked, bq_stream_t stream) {
+    if (!act_dtype_ok(w_dtype) || N < 0 || K < 1 || K % 8 != 0 || !std::isfinite(eps) || eps <= 0.0f ||
+        (scale_w_per_channel != 0 && scale_w_per_channel != 1))
+        return BQ_ERR_INVALID_ARG;
+    if (N == 0) return BQ_OK;
+    if (w == nullptr || scale_w == nullptr || wpacked == nullptr) return BQ_ERR_INVALID_ARG;
+    if (!aligned(w, esize(w_dtype)) || !aligned(scale_w, 4) || !aligned(wpacked, 4)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    return from_cuda(launch_q4_weight_pack(w, w_dtype, N, K, scale_w, scale_w_per_channel, eps, wpacked,
+                                           static_cast<cudaStream_t>(stream), dev));
+}
+
+bq_status bq_act_quant_int4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, int64_t ldx, const float *scale_a,
+                            float eps, int8_t *xq, int64_t ldq, bq_stream_t stream) {
+    if (!act_dtype_ok(x_dtype) || M < 0 || K < 1 || ldx < K || ldq < K || !std::isfinite(eps) || eps <= 0.0f)
+        return BQ_ERR_INVALID_ARG;
+    if (M == 0) return BQ_OK;
+    if (x == nullptr || scale_a == nullptr || xq == nullptr) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(scale_a, 4)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    return from_cuda(launch_q4_act_quant(x, x_dtype, M, K, ldx, scale_a, eps, xq, ldq, nullptr, nullptr, 0, 0, nullptr,
+                                         static_cast<cudaStream_t>(stream), dev));
+}
+
+bq_status bq_linear_w4a4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const float *scale_a,
+                         const uint32_t *wpacked, const float *scale_w, int scale_w_per_channel, int64_t N,
+                         const float *bias, float eps, bq_dtype out_dtype, void *out, void *workspace,
+                         size_t workspace_bytes, bq_stream_t stream) {
+    if (!act_dtype_ok(x_dtype) || !out_dtype_ok(out_dtype) || M < 0 || N < 0 || K < 1 || K % 32 != 0 ||
+        K > kMaxK || M > kMaxDim || N > kMaxDim || !std::isfinite(eps) || eps <= 0.0f ||
+        (scale_w_per_channel != 0 && scale_w_per_channel != 1))
+        return BQ_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return BQ_OK;
+    if (x == nullptr || scale_a == nullptr || wpacked == nullptr || scale_w == nullptr || out == nullptr)
+        return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(scale_a, 4) || !aligned(wpacked, 16) || !aligned(scale_w, 4) ||
+        !aligned(bias, 4) || !aligned(out, 16))
+        return BQ_ERR_MISALIGNED;
+    const W4a4Layout l = w4a4_layout(M, N, K);
+    if (workspace == nullptr || workspace_bytes < l.total) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int8_t *xq = reinterpret_cast<int8_t *>(ws + l.xq);
+    float *row_step = reinterpret_cast<float *>(ws + l.row);
+    float *col_step = reinterpret_cast<float *>(ws + l.col);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_q4_act_quant(x, x_dtype, M, K, K, scale_a, eps, xq, K, row_step, scale_w, scale_w_per_channel, N,
+                            col_step, s, dev) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (M <= kGemvMaxM)
+        return from_cuda(launch_w4a4_gemv(xq, M, K, wpacked, row_step, col_step, bias, N, out_dtype, out, s, dev));
+    const bool stage_out = (N * esize(out_dtype)) % 16 != 0;
+    GemmArgs g;
+    g.a = xq;
+    g.lda = K;
+    g.b = wpacked;
+    g.ldb = K / 8;
+    g.b_pack = 4;
+    g.colscale = col_step;
+    g.rowscale = row_step;
+    g.bias = bias;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.out_dtype = out_dtype;
+    g.out = stage_out ? static_cast<void *>(ws + l.opad) : out;
+    g.ldo = stage_out ? (N + 7) / 8 * 8 : N;
+    st = launch_gemm_tc(g, s, dev);
+    if (st != BQ_OK || !stage_out) return st;
+    const size_t row = static_cast<size_t>(N) * esize(out_dtype);
+    return from_cuda(cudaMemcpy2DAsync(out, row, g.out, static_cast<size_t>(g.ldo) * esize(out_dtype), row,
+                                       static_cast<size_t>(M), cudaMemcpyDeviceToDevice, s));
+}
+
+size_t bq_bitconv1d_weight_pack_workspace_bytes(int64_t C_out, int64_t Cg, int64_t KS) {
+    if (C_out < 0 || Cg < 0 || KS < 0) return 0;
+    const size_t n = static_cast<size_t>(C_out) * static_cast<size_t>(Cg) * static_cast<size_t>(KS);
+    return align256(n * 4) + align256(ternary_pack_workspace_bytes(KS * C_out, Cg)) + align256(n / 4 + 16);
+}
+
+size_t bq_bitconv1d_workspace_bytes(int64_t B, int64_t C_in, int64_t L, int64_t C_out, int64_t KS, int64_t stride,
+                                    int64_t pad, int64_t groups) {
+    if (B < 0 || C_in < 1 || L < 1 || C_out < 1 || KS < 1 || stride < 1 || pad < 0 || groups < 1) return 0;
+    if (L + 2 * pad < KS) return 0;
+    return bitconv_layout(B, C_in, L, C_out, KS, stride, pad, groups).total;
+}
+
+bq_status bq_bitconv1d_weight_pack(const void *w, bq_dtype w_dtype, int64_t C_out, int64_t Cg, int64_t KS,
+                                   uint32_t *wpacked, float *w_scale, void *workspace, size_t workspace_bytes,
+                                   bq_stream_t stream) {
+    if (!act_dtype_ok(w_dtype) || C_out < 0 || Cg < 16 || Cg % 16 != 0 || KS < 1) return BQ_ERR_INVALID_ARG;
+    if (C_out == 0) return BQ_OK;
+    if (w == nullptr || wpacked == nullptr || w_scale == nullptr) return BQ_ERR_INVALID_ARG;
+    if (!aligned(w, esize(w_dtype)) || !aligned(wpacked, 16) || !aligned(w_scale, 4)) return BQ_ERR_MISALIGNED;
+    const size_t need = bq_bitconv1d_weight_pack_workspace_bytes(C_out, Cg, KS);
+    if (workspace == nullptr || workspace_bytes < need) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = static_cast<size_t>(C_out) * static_cast<size_t>(Cg) * static_cast<size_t>(KS);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *wt = ws;                                   // [KS][C_out][Cg] in the weight's dtype
+    uint8_t *tws = ws + align256(n * 4);                // reduction partials of the ternary pack
+    uint32_t *dense = reinterpret_cast<uint32_t *>(tws + align256(ternary_pack_workspace_bytes(KS * C_out, Cg)));
+    if (launch_bitconv_weight_transpose(w, w_dtype, C_out, Cg, KS, wt, s) != cudaSuccess) return BQ_ERR_CUDA;
+    const int64_t Cgp = (Cg + 63) / 64 * 64;
+    uint32_t *dst = Cgp == Cg ? wpacked : dense;
+    if (launch_ternary_pack(wt, w_dtype, KS * C_out, Cg, dst, w_scale, tws, s, dev) != cudaSuccess)
+        return BQ_ERR_CUDA;
+    if (Cgp == Cg) return BQ_OK;
+    return from_cuda(cudaMemcpy2DAsync(wpacked, static_cast<size_t>(Cgp / 16) * 4, dense,
+                                       static_cast<size_t>(Cg / 16) * 4, static_cast<size_t>(Cg / 16) * 4,
+                                       static_cast<size_t>(KS * C_out), cudaMemcpyDeviceToDevice, s));
+}
+
+bq_status bq_bitconv1d(const void *x, bq_dtype x_dtype, int64_t B, int64_t C_in, int64_t L, const float *ln_weight,
+                       const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t C_out, int64_t KS,
+                       int64_t stride, int64_t pad, int64_t groups, const float *bias, float eps, bq_dtype out_dtype,
+                       void *out, void *workspace, size_t workspace_bytes, bq_stream_t stream) {
+    if (!act_dtype_ok(x_dtype) || !out_dtype_ok(out_dtype) || B < 0 || C_in < 16 || L < 1 || C_out < 1 || KS < 1 ||
+        stride < 1 || pad < 0 || groups < 1 || C_in % groups != 0 || C_out % groups != 0 || !std::isfinite(eps) ||
+        eps < 0.0f || L + 2 * pad < KS)
+        return BQ_ERR_INVALID_ARG;
+    const int64_t Cg = C_in / groups, Cog = C_out / groups;
+    if (C_in % 16 != 0 || Cg % 16 != 0 || Cg > kMaxK || (groups > 1 && Cog % 4 != 0)) return BQ_ERR_INVALID_ARG;
+    if (B * L > kMaxDim || B * ((L + 2 * pad - KS) / stride + 1) > kMaxDim) return BQ_ERR_INVALID_ARG;
+    if (B == 0) return BQ_OK;
+    if (x == nullptr || wpacked == nullptr || w_scale == nullptr || out == nullptr) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(wpacked, 16) || !aligned(w_scale, 4) || !aligned(bias, 4) ||
+        !aligned(ln_weight, 4) || !aligned(ln_bias, 4) || !aligned(out, esize(out_dtype)))
+        return BQ_ERR_MISALIGNED;
+    const size_t need = bitconv_layout(B, C_in, L, C_out, KS, stride, pad, groups).total;
+    if (workspace == nullptr || workspace_bytes < need) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    return launch_bitconv1d(x, x_dtype, B, C_in, L, ln_weight, ln_bias, wpacked, w_scale, C_out, KS, stride, pad, groups,
+                            bias, eps, out_dtype, out, workspace, static_cast<cudaStream_t>(stream), dev);
 }
 
 bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint32_t *qweight,

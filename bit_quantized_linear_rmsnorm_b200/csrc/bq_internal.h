@@ -80,15 +80,15 @@ cudaError_t launch_int4_pack(const uint8_t *q, const uint8_t *zeros, int64_t N, 
                              uint32_t *qweight, uint32_t *qzeros, cudaStream_t s, const DevInfo &dev);
 
 // Epilogue of the integer GEMMs:
-//   W8A8: out = (float(acc) * colscale[n]) * rowscale[m] (+ bias[n])
-//   W2A8: out = (float(acc - rowcorr[m]) * rowscale[m]) * (*colscale_scalar) (+ bias[n])
+//   W8A8, W4A4: out = (float(acc) * colscale[n]) * rowscale[m] (+ bias[n])
+//   W2A8:       out = (float(acc - rowcorr[m]) * rowscale[m]) * (*colscale_scalar) (+ bias[n])
 struct GemmArgs {
     const int8_t *a = nullptr;      // [M][lda] int8, K-major (or [K][lda], M-major, with a_mn)
     int64_t lda = 0;
-    const void *b = nullptr;        // int8 [N][ldb] / [K][ldb], or packed 2-bit u32 [N][K/16]
+    const void *b = nullptr;        // int8 [N][ldb] / [K][ldb], or packed u32 [N][ldb] (K * b_pack / 32 words)
     int64_t ldb = 0;                // elements (bytes for int8, words for packed)
     bq_wlayout b_layout = BQ_W_NK;
-    bool b_packed2 = false;         // ternary offset-binary codes
+    int b_pack = 0;                 // 0: int8 B; 2: ternary offset-binary codes; 4: signed 4-bit codes
     const float *colscale = nullptr;  // [N] (W8A8) or one device scalar (W2A8)
     const float *rowscale = nullptr;  // [M]
     const int32_t *rowcorr = nullptr; // [M] (W2A8) or nullptr
@@ -125,6 +125,31 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
                                const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
                                int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,
                                const DevInfo &dev);
+
+// W4A4 (4-bit activations and weights with given steps, w4a4.cu).
+cudaError_t launch_q4_weight_pack(const void *w, bq_dtype wt, int64_t N, int64_t K, const float *scale_w,
+                                  int per_channel, float eps, uint32_t *wpacked, cudaStream_t s, const DevInfo &dev);
+cudaError_t launch_q4_act_quant(const void *x, bq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *scale_a,
+                                float eps, int8_t *xq, int64_t ldq, float *row_step, const float *scale_w,
+                                int per_channel, int64_t N, float *col_step, cudaStream_t s, const DevInfo &dev);
+cudaError_t launch_w4a4_gemv(const int8_t *xq, int64_t M, int64_t K, const uint32_t *wpacked, const float *row_step,
+                             const float *col_step, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
+                             cudaStream_t s, const DevInfo &dev);
+
+// Ternary Conv1d (bitconv1d.cu): workspace layout, weight transpose to
+// [KS][C_out * Cg], and the forward.
+struct BitconvLayout {
+    int64_t L_out = 0, ldp = 0;  // output length; row pitch of the fp32 tap partials
+    size_t xt = 0, xq = 0, scale = 0, a = 0, rs = 0, rc = 0, part = 0, total = 0;
+};
+BitconvLayout bitconv_layout(int64_t B, int64_t C_in, int64_t L, int64_t C_out, int64_t KS, int64_t stride,
+                             int64_t pad, int64_t groups);
+cudaError_t launch_bitconv_weight_transpose(const void *w, bq_dtype wt, int64_t C_out, int64_t Cg, int64_t KS,
+                                            void *dst, cudaStream_t s);
+bq_status launch_bitconv1d(const void *x, bq_dtype xt, int64_t B, int64_t C_in, int64_t L, const float *ln_weight,
+                           const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t C_out,
+                           int64_t KS, int64_t stride, int64_t pad, int64_t groups, const float *bias, float eps,
+                           bq_dtype out_dtype, void *out, void *workspace, cudaStream_t s, const DevInfo &dev);
 
 // Grouped INT4 linear.
 size_t linear_w4_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group_size);

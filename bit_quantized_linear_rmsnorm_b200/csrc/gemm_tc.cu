@@ -50,13 +50,22 @@ constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t A_BYTES = BM * BK;           // 16 KB
 constexpr uint32_t B_BYTES = BN * BK;           // 32 KB
-constexpr uint32_t P_BYTES = BN * (BK / 16) * 4;  // 8 KB packed 2-bit tile
 constexpr uint32_t STG_BYTES = BM * 64;         // 8 KB epilogue staging buffer
 
-template <bool PACKED>
+// Packed weights: PK = 0 for int8 B, 2 for ternary offset-binary codes (2 bits,
+// unsigned), 4 for signed 4-bit codes.  A 128-K slab of one weight row is
+// BK * PK / 32 words.
+template <int PK>
+constexpr int slab_words() { return PK == 0 ? 0 : BK * PK / 32; }
+template <int PK>
+constexpr uint32_t p_bytes(int rows) { return static_cast<uint32_t>(rows * slab_words<PK>() * 4); }
+
+template <int PK>
 struct Cfg {
+    static constexpr bool PACKED = PK != 0;
+    static constexpr uint32_t P_BYTES = p_bytes<PK>(BN);  // 8 KB (2-bit) / 16 KB (4-bit) tile
     static constexpr int kStages = PACKED ? 3 : 4;
-    static constexpr int kUnpack = 256;  // unpack threads (W2A8)
+    static constexpr int kUnpack = 256;  // unpack threads (packed weights)
     static constexpr int kThreads = PACKED ? 256 + kUnpack : 256;
     static constexpr uint32_t OFF_A = 0;
     static constexpr uint32_t OFF_B = OFF_A + kStages * A_BYTES;
@@ -133,12 +142,38 @@ struct Items {
     }
 };
 
-template <bool PACKED, bool A_MN, bool B_KN, typename OutT>
-__global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
+// 16 weights of one 16-byte chunk from the packed slab word(s): ternary codes
+// are expanded to u8 codes (w + 1), signed 4-bit codes sign-extended to s8.
+template <int PK>
+__device__ __forceinline__ uint4 unpack_chunk(const uint32_t *words, int c) {
+    if constexpr (PK == 2) {
+        const uint32_t u = words[c];
+        return make_uint4(u & 0x03030303u, (u >> 2) & 0x03030303u, (u >> 4) & 0x03030303u, (u >> 6) & 0x03030303u);
+    } else {
+        const uint2 u = reinterpret_cast<const uint2 *>(words)[c];
+        uint32_t r[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t w = h ? u.y : u.x;
+            uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // even / odd nibbles as bytes
+            lo |= (lo & 0x08080808u) * 30u;  // sign extension: bit 3 set -> byte | 0xF0 (no carry between bytes)
+            hi |= (hi & 0x08080808u) * 30u;
+            r[2 * h] = __byte_perm(lo, hi, 0x5140);
+            r[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+        }
+        return make_uint4(r[0], r[1], r[2], r[3]);
+    }
+}
+
+template <int PK, bool A_MN, bool B_KN, typename OutT>
+__global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmO,
                    const GemmDev p) {
-    using C = Cfg<PACKED>;
+    using C = Cfg<PK>;
+    constexpr bool PACKED = PK != 0;
+    constexpr bool TERN = PK == 2;  // ternary codes: acc - rowsum, one scalar weight scale
+    constexpr uint32_t P_BYTES = C::P_BYTES;
     constexpr int S = C::kStages;
     constexpr int CC = 64 / static_cast<int>(sizeof(OutT));  // output columns per staging chunk
 
@@ -217,7 +252,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                 } else if constexpr (PACKED) {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + P_BYTES);
                     tma_load_3d(a_dst, &tmA, kb * BK, m0, bz, full(stage));
-                    tma_load_3d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * (BK / 16), n0, bz, full(stage));
+                    tma_load_3d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * slab_words<PK>(), n0, bz, full(stage));
                 } else {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + b_bytes);
                     // A: a 128 (K) x 128 (M) box when M-major, 128 (M) x 128 (K) otherwise
@@ -247,8 +282,8 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             mbar_drain(full(static_cast<int>(i % S)), static_cast<uint32_t>((i / S) & 1), p.wait_ns);
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = idesc_i8(BM, BN, true, !PACKED, B_KN, A_MN);
-        constexpr uint32_t idesc_half = idesc_i8(BM, BN / 2, true, !PACKED, B_KN, A_MN);
+        constexpr uint32_t idesc = idesc_i8(BM, BN, true, !TERN, B_KN, A_MN);
+        constexpr uint32_t idesc_half = idesc_i8(BM, BN / 2, true, !TERN, B_KN, A_MN);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -304,7 +339,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         const int r = 32 * q + lane;
         const int et = threadIdx.x - 128;  // 0..127
         uint8_t *stg = smem + C::OFF_STG;
-        const float colscale_scalar = PACKED ? __ldg(p.colscale) : 0.0f;
+        const float colscale_scalar = TERN ? __ldg(p.colscale) : 0.0f;
         uint32_t chunk_ctr = 0;
         int t = 0;
         for (int item = blockIdx.x; item < items.count; item += gridDim.x, ++t) {
@@ -320,7 +355,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             named_bar_sync(1, 128);  // previous tile finished reading vcol / vbias
             for (int i = et; i < BN; i += 128) {
                 const int n = n0 + i;
-                vcol[i] = (!PACKED && n < p.N) ? __ldg(colscale + n) : 0.0f;
+                vcol[i] = (!TERN && n < p.N) ? __ldg(colscale + n) : 0.0f;
                 vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
             }
             named_bar_sync(1, 128);
@@ -342,7 +377,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
             tc_fence_after();
             const int row = m0 + r;
             const float rs = row < p.M ? __ldg(rowscale + row) : 0.0f;
-            const int corr = (p.rowcorr != nullptr && row < p.M) ? __ldg(p.rowcorr + row) : 0;
+            const int corr = (TERN && row < p.M) ? __ldg(p.rowcorr + row) : 0;
 
 #pragma unroll 1
             for (int c32 = 0; c32 < nc32; ++c32) {
@@ -360,7 +395,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                 for (int j = 0; j < 32; ++j) {
                     const float a = static_cast<float>(static_cast<int>(v[j]) - corr);
                     float o;
-                    if constexpr (PACKED)
+                    if constexpr (TERN)
                         o = __fmul_rn(__fmul_rn(a, rs), colscale_scalar);
                     else
                         o = __fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs);
@@ -400,7 +435,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
         }
         if (et == 0) bulk_wait_all();
     } else if (PACKED && warp >= 8) {
-        // ------------------------------------------------------------ unpack 2-bit codes
+        // ------------------------------------------------------------ unpack packed codes
         const int ut = threadIdx.x - 256;  // 0 .. C::kUnpack - 1
         int stage = 0;
         uint32_t phase = 0;
@@ -419,9 +454,7 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
                 for (int i = 0; i < (BN * 8) / C::kUnpack; ++i) {
                     const int idx = ut + C::kUnpack * i;
                     const int n = idx >> 3, c = idx & 7;  // weight row, 16-element chunk of the 128-K slab
-                    const uint32_t u = pk[idx];
-                    const uint4 codes = make_uint4(u & 0x03030303u, (u >> 2) & 0x03030303u,
-                                                   (u >> 4) & 0x03030303u, (u >> 6) & 0x03030303u);
+                    const uint4 codes = unpack_chunk<PK>(pk + n * slab_words<PK>(), c);
                     *reinterpret_cast<uint4 *>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = codes;
                 }
                 fence_proxy_async_smem();
@@ -469,11 +502,12 @@ __global__ void __launch_bounds__(Cfg<PACKED>::kThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr uint32_t PA_BYTES = 128 * BK;              // own 128 rows of A
 constexpr uint32_t PB_BYTES = 128 * BK;              // own half of a 256-wide B tile
-constexpr uint32_t PP_BYTES = 128 * (BK / 16) * 4;   // its packed 2-bit form
-template <bool PACKED>
+template <int PK>
 struct PairCfg {
+    static constexpr bool PACKED = PK != 0;
+    static constexpr uint32_t PP_BYTES = p_bytes<PK>(128);  // its packed form
     static constexpr int kStages = PACKED ? 5 : 6;
-    static constexpr int kUnpack = 256;  // unpack threads (W2A8)
+    static constexpr int kUnpack = 256;  // unpack threads (packed weights)
     static constexpr int kThreads = PACKED ? 256 + kUnpack : 256;
     static constexpr uint32_t OFF_A = 0;
     static constexpr uint32_t OFF_B = OFF_A + kStages * PA_BYTES;
@@ -486,6 +520,11 @@ struct PairCfg {
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, epilogue failure
     static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;
 };
+
+static_assert(Cfg<0>::SMEM <= 232448 && Cfg<2>::SMEM <= 232448 && Cfg<4>::SMEM <= 232448,
+              "single-CTA stages exceed the 227 KB of shared memory per CTA");
+static_assert(PairCfg<0>::SMEM <= 232448 && PairCfg<2>::SMEM <= 232448 && PairCfg<4>::SMEM <= 232448,
+              "pair stages exceed the 227 KB of shared memory per CTA");
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -544,12 +583,15 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-template <bool PACKED, typename OutT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kThreads, 1)
+template <int PK, typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmBh, const __grid_constant__ CUtensorMap tmO,
                      const GemmDev p) {
-    using C = PairCfg<PACKED>;
+    using C = PairCfg<PK>;
+    constexpr bool PACKED = PK != 0;
+    constexpr bool TERN = PK == 2;
+    constexpr uint32_t PP_BYTES = C::PP_BYTES;
     constexpr int S = C::kStages;
     constexpr uint32_t OFF_A = C::OFF_A, OFF_B = C::OFF_B, OFF_P = C::OFF_P, OFF_STG = C::OFF_STG;
     constexpr uint32_t OFF_VEC = C::OFF_VEC, OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC;
@@ -644,7 +686,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
                     mbar_arrive_expect_tx(full(stage), PA_BYTES + p_bytes);
                     tma_load_3d(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
                                 bz, full(stage));
-                    tma_load_3d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * (BK / 16), nb0, bz,
+                    tma_load_3d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * slab_words<PK>(), nb0, bz,
                                 full(stage));
                 } else {  // the leader's barrier counts both CTAs' copies
                     if (leader) mbar_arrive_expect_tx(full(stage), 2u * (PA_BYTES + b_bytes));
@@ -668,8 +710,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         }
     } else if (warp == 1 && lane == 0 && leader) {
         // ------------------------------------------------------------ MMA issuer (leader)
-        constexpr uint32_t idesc = idesc_i8(2 * BM, BN, true, !PACKED, false);
-        constexpr uint32_t idesc_half = idesc_i8(2 * BM, BN / 2, true, !PACKED, false);
+        constexpr uint32_t idesc = idesc_i8(2 * BM, BN, true, !TERN, false);
+        constexpr uint32_t idesc_half = idesc_i8(2 * BM, BN / 2, true, !TERN, false);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -715,7 +757,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         const int r = 32 * q + lane;
         const int et = threadIdx.x - 128;
         uint8_t *stg = smem + OFF_STG;
-        const float colscale_scalar = PACKED ? __ldg(p.colscale) : 0.0f;
+        const float colscale_scalar = TERN ? __ldg(p.colscale) : 0.0f;
         uint32_t chunk_ctr = 0;
         int t = 0;
         for (int item = cl; item < count; item += ncl, ++t) {
@@ -732,7 +774,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             named_bar_sync(1, 128);
             for (int i = et; i < BN; i += 128) {
                 const int n = n0 + i;
-                vcol[i] = (!PACKED && n < p.N) ? __ldg(colscale + n) : 0.0f;
+                vcol[i] = (!TERN && n < p.N) ? __ldg(colscale + n) : 0.0f;
                 vbias[i] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.0f;
             }
             named_bar_sync(1, 128);
@@ -749,7 +791,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
             tc_fence_after();
             const int row = mr + r;
             const float rs = row < p.M ? __ldg(rowscale + row) : 0.0f;
-            const int corr = (PACKED && row < p.M) ? __ldg(p.rowcorr + row) : 0;
+            const int corr = (TERN && row < p.M) ? __ldg(p.rowcorr + row) : 0;
 
 #pragma unroll 1
             for (int c32 = 0; c32 < nc32; ++c32) {
@@ -766,7 +808,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const float a = static_cast<float>(static_cast<int>(v[j]) - corr);
-                    const float o = PACKED ? __fmul_rn(__fmul_rn(a, rs), colscale_scalar)
+                    const float o = TERN ? __fmul_rn(__fmul_rn(a, rs), colscale_scalar)
                                            : __fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs);
                     f[j] = __fadd_rn(o, vbias[c32 * 32 + j]);
                 }
@@ -810,7 +852,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
         uint32_t phase = 0;
         bool ok = true;
         for (int item = cl; item < count && ok; item += ncl) {
-            const int words = (item < big ? 128 : 64) * (BK / 16);  // packed words of this CTA's rows
+            const int chunks = (item < big ? 128 : 64) * 8;  // 16-weight chunks of this CTA's rows
             for (int kb = 0; kb < nkb; ++kb) {
                 bool got = true;
                 if (lane == 0) got = mbar_wait_spin(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK, p.wait_ns);
@@ -821,11 +863,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PACKED>::kTh
                 const uint32_t *pk = reinterpret_cast<const uint32_t *>(smem + OFF_P + stage * PP_BYTES);
                 uint8_t *bt = smem + OFF_B + stage * PB_BYTES;
 #pragma unroll 2
-                for (int idx = ut; idx < words; idx += C::kUnpack) {
+                for (int idx = ut; idx < chunks; idx += C::kUnpack) {
                     const int n = idx >> 3, c = idx & 7;  // weight row, 16-element chunk of the 128-K slab
-                    const uint32_t u = pk[idx];
-                    const uint4 codes = make_uint4(u & 0x03030303u, (u >> 2) & 0x03030303u,
-                                                   (u >> 4) & 0x03030303u, (u >> 6) & 0x03030303u);
+                    const uint4 codes = unpack_chunk<PK>(pk + n * slab_words<PK>(), c);
                     *reinterpret_cast<uint4 *>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = codes;
                 }
                 // every lane orders its stores before the tensor core's reads, then the
@@ -900,12 +940,12 @@ GemmDev dev_args(const GemmArgs &g, const DevInfo &dev) {
     return p;
 }
 
-template <bool PACKED, bool A_MN, bool B_KN, typename OutT>
+template <int PK, bool A_MN, bool B_KN, typename OutT>
 bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
                    const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
-    using C = Cfg<PACKED>;
-    auto kern = gemm_tc_kernel<PACKED, A_MN, B_KN, OutT>;
+    using C = Cfg<PK>;
+    auto kern = gemm_tc_kernel<PK, A_MN, B_KN, OutT>;
     static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
     if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
         return BQ_ERR_CUDA;
@@ -915,11 +955,11 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-template <bool PACKED, typename OutT>
+template <int PK, typename OutT>
 bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB128, const CUtensorMap &mB64,
                       const CUtensorMap &mO, cudaStream_t s, const DevInfo &dev) {
-    using C = PairCfg<PACKED>;
-    auto kern = gemm_pair_kernel<PACKED, OutT>;
+    using C = PairCfg<PK>;
+    auto kern = gemm_pair_kernel<PK, OutT>;
     static SmemOptIn opt_in;  // once per context (also keeps later calls capture-safe)
     if (smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(C::SMEM)) != cudaSuccess)
         return BQ_ERR_CUDA;
@@ -934,7 +974,25 @@ bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMa
 // The pair kernel takes products with K-major A and K-major (or 2-bit packed)
 // weights that fill at least one wave of CTA pairs with 256 x 256 tiles.
 bool use_pair(const GemmArgs &g, const DevInfo &dev) {
-    return !g.a_mn && gemm_uses_pair(g.b_packed2, g.b_layout, g.M, g.N, dev, g.batch);
+    return !g.a_mn && gemm_uses_pair(g.b_pack != 0, g.b_layout, g.M, g.N, dev, g.batch);
+}
+
+template <int PK, typename OutT>
+bq_status dispatch_packed(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
+                          cudaStream_t s, const DevInfo &dev) {
+    const uint64_t nb = static_cast<uint64_t>(g.batch);
+    if (use_pair(g, dev)) {
+        // per CTA of a pair: its half of the packed tile (128 rows), 64 rows for half tiles
+        CUtensorMap mP128, mP64;
+        const uint64_t words = static_cast<uint64_t>(g.K) * PK / 32;
+        if (!make_map(&mP128, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, words, g.N, g.ldb * 4, slab_words<PK>(), BN / 2,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4) ||
+            !make_map(&mP64, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, words, g.N, g.ldb * 4, slab_words<PK>(), BN / 4,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4))
+            return BQ_ERR_CUDA;
+        return launch_pair<PK, OutT>(g, mA, mP128, mP64, mO, s, dev);
+    }
+    return launch_t<PK, false, false, OutT>(g, mA, mB, mB, mO, s, dev);
 }
 
 template <typename OutT>
@@ -942,31 +1000,22 @@ bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
                    const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
     const uint64_t nb = static_cast<uint64_t>(g.batch);
-    if (g.b_packed2 && use_pair(g, dev)) {
-        // per CTA of a pair: its half of the packed tile (128 rows), 64 rows for half tiles
-        CUtensorMap mP128, mP64;
-        if (!make_map(&mP128, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN / 2,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4) ||
-            !make_map(&mP64, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN / 4,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4))
-            return BQ_ERR_CUDA;
-        return launch_pair<true, OutT>(g, mA, mP128, mP64, mO, s, dev);
-    }
-    if (g.b_packed2) return launch_t<true, false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    if (g.b_pack == 2) return dispatch_packed<2, OutT>(g, mA, mB, mO, s, dev);
+    if (g.b_pack == 4) return dispatch_packed<4, OutT>(g, mA, mB, mO, s, dev);
     if (use_pair(g, dev)) {
         // per CTA of a pair: 128-row boxes of B (half of a 256-wide tile), 64-row boxes for half tiles
         CUtensorMap mBq;
         if (!make_map(&mBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 4,
                       CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sb))
             return BQ_ERR_CUDA;
-        return launch_pair<false, OutT>(g, mA, mBh, mBq, mO, s, dev);
+        return launch_pair<0, OutT>(g, mA, mBh, mBq, mO, s, dev);
     }
     if (g.a_mn) {
-        if (g.b_layout == BQ_W_KN) return launch_t<false, true, true, OutT>(g, mA, mB, mBh, mO, s, dev);
-        return launch_t<false, true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+        if (g.b_layout == BQ_W_KN) return launch_t<0, true, true, OutT>(g, mA, mB, mBh, mO, s, dev);
+        return launch_t<0, true, false, OutT>(g, mA, mB, mBh, mO, s, dev);
     }
-    if (g.b_layout == BQ_W_KN) return launch_t<false, false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
-    return launch_t<false, false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
+    if (g.b_layout == BQ_W_KN) return launch_t<0, false, true, OutT>(g, mA, mB, mBh, mO, s, dev);
+    return launch_t<0, false, false, OutT>(g, mA, mB, mBh, mO, s, dev);
 }
 
 }  // namespace
@@ -986,9 +1035,9 @@ bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) 
                                        CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sa);
     if (!okA) return BQ_ERR_CUDA;
     bool okB;
-    if (g.b_packed2)
-        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, g.K / 16, g.N, g.ldb * 4, BK / 16, BN,
-                       CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4);
+    if (g.b_pack != 0)
+        okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, static_cast<uint64_t>(g.K) * g.b_pack / 32, g.N,
+                       g.ldb * 4, BK * g.b_pack / 32, BN, CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4);
     else if (g.b_layout == BQ_W_KN)
         okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.N, g.K, g.ldb, 128, BK, CU_TENSOR_MAP_SWIZZLE_128B,
                        nb, g.sb);
@@ -998,7 +1047,7 @@ bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) 
     if (!okB) return BQ_ERR_CUDA;
     // K-major weights: a 128-row box too, for the half tiles of a last partial wave
     mBh = mB;
-    if (!g.b_packed2 && g.b_layout != BQ_W_KN &&
+    if (g.b_pack == 0 && g.b_layout != BQ_W_KN &&
         !make_map(&mBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B,
                   nb, g.sb))
         return BQ_ERR_CUDA;

@@ -78,7 +78,8 @@ typedef enum {
     BQ_OP_WEIGHT_PACK_INT4_GROUPED = 2,
     BQ_OP_GEMM_I8_PERTOKEN = 3,
     BQ_OP_BITLINEAR_W2A8 = 4,
-    BQ_OP_LINEAR_W4_GROUPED = 5
+    BQ_OP_LINEAR_W4_GROUPED = 5,
+    BQ_OP_LINEAR_W4A4 = 6
 } bq_op;
 
 /*
@@ -279,6 +280,87 @@ bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint3
                                const uint16_t *scales_f16, const uint32_t *qzeros,
                                const float *bias, int64_t N, int64_t group_size, float *out,
                                void *workspace, size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * 4-bit activations and 4-bit weights with given step sizes (W4A4).
+ * Source: "bitorch_engine.layers.qlinear.nbit.cutlass.q4_layer.
+ * Q4LinearFunction" (bitorch-engine), forward(x, weight, scale_a, scale_w,
+ * eps, is_train): the inputs and the weights are quantized to 4 bits with the
+ * given scale factors, eps avoids a division by zero, then the linear.
+ *
+ *   s_a = max(scale_a, eps),  s_w[n] = max(scale_w[per_channel ? n : 0], eps)
+ *   xq[m,k] = clamp(rne(x[m,k] / s_a), -8, 7),  wq[n,k] = clamp(rne(w[n,k] / s_w[n]), -8, 7)
+ *   out[m,n] = (float(sum_k xq * wq) * s_w[n]) * s_a (+ bias[n])
+ *
+ * Steps are device fp32 values (read by the kernels, no host round trip):
+ * scale_a one value, scale_w one value or [N] (scale_w_per_channel = 1).
+ * eps > 0.  Quotients are correctly rounded fp32 divisions rounded to
+ * nearest even.  is_train only decides what a training framework keeps for
+ * its backward; the forward result is the same.
+ *
+ * bq_weight_quant_int4_pack: w dense [N][K] fp32 or bf16 -> wpacked uint32
+ * [N][K/8], eight signed (two's-complement) nibbles per word, element k of a
+ * row in bits [4*(k%8), 4*(k%8)+3] of word k/8.  K % 8 == 0.
+ * bq_act_quant_int4: x [M][ldx] fp32 or bf16 -> xq int8 [M][ldq] in [-8, 7].
+ * bq_linear_w4a4: x dense [M][K] (K % 32 == 0, any N), wpacked as above
+ * (16-byte aligned), bias fp32 [N] or NULL, out dense [M][N] of out_dtype.
+ * The activation codes go to the workspace
+ * (bq_workspace_bytes(BQ_OP_LINEAR_W4A4, M, N, K, 0) bytes, 256-byte aligned);
+ * up to 16 tokens run a dp4a GEMV kernel, more run the tcgen05 kind::i8 GEMM
+ * with the packed weights sign-extended to int8 in shared memory (no int8
+ * copy of the weights in global memory).
+ */
+bq_status bq_weight_quant_int4_pack(const void *w, bq_dtype w_dtype, int64_t N, int64_t K, const float *scale_w,
+                                    int scale_w_per_channel, float eps, uint32_t *wpacked, bq_stream_t stream);
+bq_status bq_act_quant_int4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, int64_t ldx, const float *scale_a,
+                            float eps, int8_t *xq, int64_t ldq, bq_stream_t stream);
+bq_status bq_linear_w4a4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, const float *scale_a,
+                         const uint32_t *wpacked, const float *scale_w, int scale_w_per_channel, int64_t N,
+                         const float *bias, float eps, bq_dtype out_dtype, void *out, void *workspace,
+                         size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Ternary Conv1d with LayerNorm-normalised 8-bit activations.
+ * Source: "Common Attention Utilities" (frankenstein-transformer), BitConv1d:
+ * the ternary weights and int8 activations of BitLinear, the input (B, C_in,
+ * L) LayerNorm-normalised over the channel dimension before the activation
+ * quantization, forward (B, C_in, L) -> (B, C_out, L_out) with kernel_size,
+ * stride, padding and groups.
+ *
+ *   per position (b, p): LayerNorm over the C_in channels (optional affine
+ *     ln_weight / ln_bias [C_in]), then bq_act_quant_int8_layernorm's codes
+ *     xq[b,p,:] and act_scale[b,p];
+ *   gamma, wq = absmean ternary quantization of all weights (bake rule);
+ *   out[b,co,lo] = gamma * sum_t act_scale[b,p] * sum_c wq[co,c,t] * xq[b,p,g*Cg+c]
+ *                  (+ bias[co]),  p = lo*stride + t - pad (padding adds nothing),
+ *   Cg = C_in / groups, g = co / (C_out / groups),
+ *   L_out = (L + 2*pad - KS) / stride + 1.
+ * Each tap is an exact integer contraction over the group's channels, scaled
+ * by the scale of the position it reads; the taps are summed in fp32 and the
+ * result rounded once to out_dtype.
+ *
+ * bq_bitconv1d_weight_pack: w dense [C_out][Cg][KS] (the Conv1d weight) fp32
+ * or bf16, Cg % 16 == 0 -> wpacked uint32 [KS][C_out][Cgp/16] (Cgp = Cg
+ * rounded up to 64; per tap the 2-bit layout of bq_weight_quant_ternary_pack
+ * along the channels, rows Cgp/16 words apart) and w_scale (one fp32 on the
+ * device).  workspace: bq_bitconv1d_weight_pack_workspace_bytes().
+ * bq_bitconv1d: x dense (B, C_in, L), C_in % 16 == 0, Cg % 16 == 0 and, with
+ * groups > 1, (C_out / groups) % 4 == 0; out dense (B, C_out, L_out).  Runs a
+ * transpose to position-major rows, the binary64 LayerNorm quantization, per
+ * tap a row gather and per group the tcgen05 ternary GEMM into fp32
+ * partials, and a tap-sum / transpose kernel.  workspace:
+ * bq_bitconv1d_workspace_bytes(), 256-byte aligned.
+ */
+size_t bq_bitconv1d_weight_pack_workspace_bytes(int64_t C_out, int64_t Cg, int64_t KS);
+bq_status bq_bitconv1d_weight_pack(const void *w, bq_dtype w_dtype, int64_t C_out, int64_t Cg, int64_t KS,
+                                   uint32_t *wpacked, float *w_scale, void *workspace, size_t workspace_bytes,
+                                   bq_stream_t stream);
+size_t bq_bitconv1d_workspace_bytes(int64_t B, int64_t C_in, int64_t L, int64_t C_out, int64_t KS, int64_t stride,
+                                    int64_t pad, int64_t groups);
+bq_status bq_bitconv1d(const void *x, bq_dtype x_dtype, int64_t B, int64_t C_in, int64_t L, const float *ln_weight,
+                       const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t C_out, int64_t KS,
+                       int64_t stride, int64_t pad, int64_t groups, const float *bias, float eps, bq_dtype out_dtype,
+                       void *out, void *workspace, size_t workspace_bytes, bq_stream_t stream);
 
 /*
  * BitLinear forward with the contract and results of bq_bitlinear_w2a8, for

@@ -60,6 +60,11 @@ def lib():
                                                           P, I64, P, I64, I64, I64, I64, P]),
             "bq_oracle_bitlinear_from_codes": (None, [P, P, P, F64, P, I64, I64, I64, P, P]),
             "bq_oracle_linear_w4_grouped": (None, [P, I64, I64, P, P, P, P, I64, I64, P]),
+            "bq_oracle_q4_quant": (None, [P, I64, I64, P, I64, F64, P, P]),
+            "bq_oracle_bitlinear_backward": (None, [P, P, P, I64, I64, I64, F64, P, P]),
+            "bq_oracle_bitconv1d_from_codes": (None, [P, P, P, F64, P, I64, I64, I64, I64, I64, I64, I64, I64, P]),
+            "bq_oracle_linear_w4a4_from_codes": (None, [P, P, P, P, I64, F64, P, I64, I64, I64, P]),
+            "bq_oracle_s4_pack": (None, [P, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(_lib, name)
@@ -265,3 +270,98 @@ def linear_w4_grouped(x, qweight, scales_f16_bits, qzeros, bias, group_size: int
     out = np.empty((M, N), np.float64)
     lib().bq_oracle_linear_w4_grouped(_p(x), M, K, _p(qw), _p(sc), _p(qz), _p(b), N, int(group_size), _p(out))
     return out
+
+
+def q4_quant(v, scale, eps: float, per_row: bool = False, want_pre: bool = False):
+    """Signed 4-bit codes of v [rows, cols] with step max(scale, eps): one
+    step (scale of one element) or one per row (scale [rows])."""
+    v = _c(v, np.float32)
+    rows, cols = v.shape
+    sc = _c(np.atleast_1d(scale), np.float32)
+    q = np.empty((rows, cols), np.int8)
+    pre = np.empty((rows, cols), np.float64) if want_pre else None
+    lib().bq_oracle_q4_quant(_p(v), rows, cols, _p(sc), 1 if per_row else 0, float(eps), _p(q), _p(pre))
+    return (q, pre) if want_pre else q
+
+
+def linear_w4a4_from_codes(xq, wq, scale_a, scale_w, eps: float, bias=None, per_channel: bool = False):
+    xq = _c(xq, np.int8)
+    wq = _c(wq, np.int8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    sa = _c(np.atleast_1d(scale_a), np.float32)
+    sw = _c(np.atleast_1d(scale_w), np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((M, N), np.float64)
+    lib().bq_oracle_linear_w4a4_from_codes(_p(xq), _p(wq), _p(sa), _p(sw), 1 if per_channel else 0, float(eps),
+                                           _p(b), M, N, K, _p(out))
+    return out
+
+
+def linear_w4a4(x, w, scale_a, scale_w, eps: float, bias=None, per_channel: bool = False):
+    """The whole W4A4 forward: 4-bit codes of x and w, integer linear, rescale."""
+    xq = q4_quant(x, scale_a, eps)
+    wq = q4_quant(w, scale_w, eps, per_row=per_channel)
+    return linear_w4a4_from_codes(xq, wq, scale_a, scale_w, eps, bias, per_channel), xq, wq
+
+
+def s4_pack(q):
+    q = _c(q, np.int8)
+    rows, cols = q.shape
+    assert cols % 8 == 0
+    out = np.empty((rows, cols // 8), np.uint32)
+    lib().bq_oracle_s4_pack(_p(q), rows, cols, _p(out))
+    return out
+
+
+def bitconv1d_act_quant(x, eps: float = 1e-5, ln_weight=None, ln_bias=None, want_pre: bool = False):
+    """Per-position LayerNorm over the channels + int8 quantization of x (B, C, L):
+    the act quant of the rows of x transposed to (B, L, C).  Returns the
+    act_quant_layernorm dict with xq [B*L, C] and act_scale [B*L]."""
+    x = _c(x, np.float32)
+    B, C, L = x.shape
+    rows = np.ascontiguousarray(x.transpose(0, 2, 1).reshape(B * L, C))
+    return act_quant_layernorm(rows, eps, ln_weight, ln_bias, want_pre=want_pre)
+
+
+def bitconv1d_from_codes(xq, act_scale, wq, gamma: float, B: int, L: int, stride: int = 1, pad: int = 0,
+                         groups: int = 1, bias=None):
+    """Ternary Conv1d from position-major codes xq [B*L, C_in], act_scale [B*L]
+    and weight codes wq [C_out, C_in/groups, KS]; returns out f64 (B, C_out, L_out)."""
+    xq = _c(xq, np.int8)
+    wq = _c(wq, np.int8)
+    sc = _c(act_scale, np.float64)
+    C_in = xq.shape[1]
+    C_out, _, KS = wq.shape
+    L_out = (L + 2 * pad - KS) // stride + 1
+    b = None if bias is None else _c(bias, np.float32)
+    out = np.empty((B, C_out, L_out), np.float64)
+    lib().bq_oracle_bitconv1d_from_codes(_p(xq), _p(sc), _p(wq), float(gamma), _p(b), B, C_in, L, C_out, KS, stride,
+                                         pad, groups, _p(out))
+    return out
+
+
+def bitconv1d(x, w, eps: float = 1e-5, stride: int = 1, pad: int = 0, groups: int = 1, ln_weight=None, ln_bias=None,
+              bias=None):
+    """Whole BitConv1d forward: per-position LayerNorm + int8 quant, ternary
+    weight quant, convolution of the dequantized values."""
+    x = _c(x, np.float32)
+    B, C, L = x.shape
+    a = bitconv1d_act_quant(x, eps, ln_weight, ln_bias)
+    t = ternary_quant(np.ascontiguousarray(w, np.float32).reshape(w.shape[0], -1))
+    wq = t["wq"].reshape(w.shape)
+    out = bitconv1d_from_codes(a["xq"], a["act_scale"], wq, t["gamma"], B, L, stride, pad, groups, bias)
+    return out, a, t
+
+
+def bitlinear_backward(x, w, dout, eps: float = 1e-5):
+    """STE backward of the BitLinear forward: (dx f64 [M,K], dw f64 [N,K])."""
+    x = _c(x, np.float32)
+    w = _c(w, np.float32)
+    dout = _c(dout, np.float32)
+    M, K = x.shape
+    N = w.shape[0]
+    dx = np.empty((M, K), np.float64)
+    dw = np.empty((N, K), np.float64)
+    lib().bq_oracle_bitlinear_backward(_p(x), _p(w), _p(dout), M, N, K, float(eps), _p(dx), _p(dw))
+    return dx, dw

@@ -20,6 +20,9 @@
  *                Input / Output tables and the Example.
  *   [linear_4bit] "vyre_libs/nn/linear/inner/linear_4bit/mod.rs" (docs.rs
  *                vyre-libs 0.7.2): module doc, QuantizedLinear4BitSpec.
+ *   [Q4Linear]   "bitorch_engine.layers.qlinear.nbit.cutlass.q4_layer.
+ *                Q4LinearFunction" (bitorch-engine docs): forward(x, weight,
+ *                scale_a, scale_w, eps, is_train).
  *
  * Readings taken where the pages are silent (each is also listed in the
  * design notes): RMSNorm puts eps inside the square root; the activation
@@ -35,6 +38,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define ORACLE_ABSMAX_FLOOR 1e-5   /* absmax / absmean lower clamp            */
@@ -159,6 +163,53 @@ void bq_oracle_act_quant_layernorm(const float *x, int64_t M, int64_t K, double 
         act_scale[m] = a / ORACLE_ACT_QMAX;
         if (rowsum) rowsum[m] = total;
     }
+}
+
+/*
+ * Ternary Conv1d ([common] BitConv1d: "the same ternary weight ({-1, 0, 1}) +
+ * int8 activation quantization as BitLinear"; "Inputs are LayerNorm-
+ * normalized over the channel dimension before activation quantization";
+ * forward maps (B, C_in, L) to (B, C_out, L_out)), from the quantized
+ * operands:
+ *
+ *   xq [B, L, C_in] and act_scale [B, L]: the per-position codes and scales
+ *       of the LayerNorm-normalised input (position-major, as act quant of
+ *       the rows of x transposed to (B, L, C_in));
+ *   wq [C_out, C_in / groups, KS] ternary codes with one scale gamma;
+ *   out[b, co, lo] = gamma * sum_t sum_c wq[co, c, t] * xq[b, p, g * Cg + c]
+ *                    * act_scale[b, p]      (+ bias[co])
+ *       with p = lo * stride + t - pad (taps outside [0, L) add nothing),
+ *       Cg = C_in / groups, g = co / (C_out / groups),
+ *       L_out = (L + 2 pad - KS) / stride + 1.
+ *
+ * Each tap's integer dot product is exact; it is scaled by the scale of the
+ * position it reads, and the taps are summed in double.
+ */
+void bq_oracle_bitconv1d_from_codes(const int8_t *xq, const double *act_scale, const int8_t *wq,
+                                    double gamma, const float *bias, int64_t B, int64_t C_in,
+                                    int64_t L, int64_t C_out, int64_t KS, int64_t stride,
+                                    int64_t pad, int64_t groups, double *out)
+{
+    int64_t L_out = (L + 2 * pad - KS) / stride + 1;
+    int64_t Cg = C_in / groups, Cog = C_out / groups;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t co = 0; co < C_out; ++co) {
+            int64_t g = co / Cog;
+            for (int64_t lo = 0; lo < L_out; ++lo) {
+                double sum = 0.0;
+                for (int64_t t = 0; t < KS; ++t) {
+                    int64_t p = lo * stride + t - pad;
+                    if (p < 0 || p >= L) continue;
+                    int64_t acc = 0;
+                    for (int64_t c = 0; c < Cg; ++c)
+                        acc += (int64_t)wq[(co * Cg + c) * KS + t] * (int64_t)xq[(b * L + p) * C_in + g * Cg + c];
+                    sum += (double)acc * act_scale[b * L + p];
+                }
+                double v = gamma * sum;
+                if (bias) v += (double)bias[co];
+                out[(b * C_out + co) * L_out + lo] = v;
+            }
+        }
 }
 
 /*
@@ -369,6 +420,71 @@ int64_t bq_oracle_gemm_i8_pertoken_batched(const int8_t *x, int64_t ldx, int64_t
 }
 
 /*
+ * 4-bit quantization with a given step size ([Q4Linear] forward: activations
+ * and weights are quantized "to 4-bits using specified scale factors"; eps
+ * "to avoid division by zero").  Row r of v [rows, cols] uses the step
+ *   s_r = max(scale[r * scale_stride], eps)       (stride 0: one step for all)
+ *   pre = v / s_r;   q = clamp(round_half_even(pre), -8, 7)
+ * pre may be NULL.
+ */
+void bq_oracle_q4_quant(const float *v, int64_t rows, int64_t cols, const float *scale,
+                        int64_t scale_stride, double eps, int8_t *q, double *pre)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        double st = (double)scale[r * scale_stride];
+        if (st < eps) st = eps;
+        for (int64_t c = 0; c < cols; ++c) {
+            double x = (double)v[r * cols + c] / st;
+            if (pre) pre[r * cols + c] = x;
+            q[r * cols + c] = (int8_t)clampd(bq_oracle_round_half_even(x), -8.0, 7.0);
+        }
+    }
+}
+
+/*
+ * The Q4Linear forward ([Q4Linear] forward: quantize x and weight to 4 bits,
+ * then the linear operation), from 4-bit codes:
+ *   out[m,n] = ((sum_k xq[m,k] * wq[n,k]) * s_w[n]) * s_a   (+ bias[n])
+ * with s_a = max(scale_a, eps) and s_w[n] = max(scale_w[n * sw_stride], eps).
+ */
+void bq_oracle_linear_w4a4_from_codes(const int8_t *xq, const int8_t *wq, const float *scale_a,
+                                      const float *scale_w, int64_t sw_stride, double eps,
+                                      const float *bias, int64_t M, int64_t N, int64_t K,
+                                      double *out)
+{
+    double sa = (double)scale_a[0];
+    if (sa < eps) sa = eps;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += (int64_t)xq[m * K + k] * (int64_t)wq[n * K + k];
+            double sw = (double)scale_w[n * sw_stride];
+            if (sw < eps) sw = eps;
+            double v = ((double)acc * sw) * sa;
+            if (bias) v += (double)bias[n];
+            out[m * N + n] = v;
+        }
+}
+
+/*
+ * Signed 4-bit codes packed eight per 32-bit word along the row, low nibble
+ * first (element c of a row in bits [4*(c%8), 4*(c%8)+3] of word c/8, as the
+ * two's-complement nibble of a value in [-8, 7]).  cols % 8 == 0.
+ */
+void bq_oracle_s4_pack(const int8_t *q, int64_t rows, int64_t cols, uint32_t *packed)
+{
+    int64_t words = cols / 8;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t wi = 0; wi < words; ++wi) {
+            uint32_t word = 0;
+            for (int j = 0; j < 8; ++j)
+                word |= ((uint32_t)q[r * cols + 8 * wi + j] & 15u) << (4 * j);
+            packed[r * words + wi] = word;
+        }
+}
+
+/*
  * BitLinear steps 4-5 from the quantized operands ([BitLinear] forward:
  * F.linear(x_q, w_q) then out * act_scale * w_scale):
  *
@@ -392,6 +508,60 @@ void bq_oracle_bitlinear_from_codes(const int8_t *xq, const double *act_scale,
             if (bias) v += (double)bias[n];
             out[m * N + n] = v;
         }
+}
+
+/*
+ * Backward of the BitLinear forward under the straight-through estimator
+ * ([BitLinear] "Quantise ... (STE)" in steps 2-3; [common] activation_quant and
+ * weight_quant: the STE "passes gradients through the rounding operation
+ * unchanged").  The forward used xt = xq * act_scale in place of the
+ * normalised y and wt = wq * gamma in place of w, with identity gradients
+ * through both, so for dout [M,N]:
+ *
+ *   dW[n,k] = sum_m dout[m,n] * xq[m,k] * act_scale[m]
+ *   dy[m,k] = sum_n dout[m,n] * wq[n,k] * gamma
+ *   dx[m,k] = (dy[m,k] - y[m,k] * (1/K) sum_j dy[m,j] * y[m,j]) / r[m]
+ *
+ * the last line being the backward of the parameter-free RMSNorm
+ * y = x / r, r = sqrt(mean(x^2) + eps).  x [M,K], w [N,K], dout [M,N].
+ */
+void bq_oracle_bitlinear_backward(const float *x, const float *w, const float *dout, int64_t M,
+                                  int64_t N, int64_t K, double eps, double *dx, double *dw)
+{
+    int8_t *xq = (int8_t *)malloc((size_t)(M * K));
+    int8_t *wq = (int8_t *)malloc((size_t)(N * K));
+    double *act = (double *)malloc((size_t)M * sizeof(double));
+    double *y = (double *)malloc((size_t)(M * K) * sizeof(double));
+    double *dy = (double *)malloc((size_t)K * sizeof(double));
+    double gamma;
+    bq_oracle_act_quant(x, M, K, eps, xq, act, NULL, NULL, y);
+    bq_oracle_ternary_quant(w, N, K, &gamma, wq, NULL);
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t m = 0; m < M; ++m)
+                s += (double)dout[m * N + n] * ((double)xq[m * K + k] * act[m]);
+            dw[n * K + k] = s;
+        }
+    for (int64_t m = 0; m < M; ++m) {
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) ss += (double)x[m * K + k] * (double)x[m * K + k];
+        double r = sqrt(ss / (double)K + eps);
+        double dot = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t n = 0; n < N; ++n) s += (double)dout[m * N + n] * ((double)wq[n * K + k] * gamma);
+            dy[k] = s;
+            dot += s * y[m * K + k];
+        }
+        for (int64_t k = 0; k < K; ++k)
+            dx[m * K + k] = (dy[k] - y[m * K + k] * (dot / (double)K)) / r;
+    }
+    free(xq);
+    free(wq);
+    free(act);
+    free(y);
+    free(dy);
 }
 
 /*

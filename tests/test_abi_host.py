@@ -228,3 +228,49 @@ def test_layernorm_calls_reject(L):
              None) == bq.BQ_ERR_MISALIGNED
     assert g(FAKE, bq.BQ_BF16, 32, 128, None, None, FAKE, FAKE, 64, None, 1e-5, bq.BQ_BF16, FAKE, None, 0,
              None) == bq.BQ_ERR_WORKSPACE
+
+
+def test_w4a4_calls_reject(L):
+    f = L.bq_linear_w4a4
+
+    def call(x=FAKE, xt=bq.BQ_BF16, M=32, K=128, sa=FAKE, wp=FAKE, sw=FAKE, pc=1, N=64, bias=None, eps=1e-6,
+             od=bq.BQ_BF16, out=FAKE, work=FAKE, nbytes=1 << 24):
+        return f(x, xt, M, K, sa, wp, sw, pc, N, bias, eps, od, out, work, nbytes, None)
+    assert call(K=48) == bq.BQ_ERR_INVALID_ARG          # K % 32
+    assert call(eps=0.0) == bq.BQ_ERR_INVALID_ARG
+    assert call(pc=2) == bq.BQ_ERR_INVALID_ARG
+    assert call(sa=None) == bq.BQ_ERR_INVALID_ARG
+    assert call(wp=ctypes.c_void_p(0x10008)) == bq.BQ_ERR_MISALIGNED
+    assert call(work=None) == bq.BQ_ERR_WORKSPACE
+    assert call(nbytes=64) == bq.BQ_ERR_WORKSPACE
+    assert call(M=0) == bq.BQ_OK
+    g = L.bq_weight_quant_int4_pack
+    assert g(FAKE, bq.BQ_F32, 8, 12, FAKE, 0, 1e-6, FAKE, None) == bq.BQ_ERR_INVALID_ARG   # K % 8
+    assert g(FAKE, bq.BQ_F32, 8, 16, None, 0, 1e-6, FAKE, None) == bq.BQ_ERR_INVALID_ARG
+    assert g(None, bq.BQ_F32, 0, 16, None, 0, 1e-6, None, None) == bq.BQ_OK
+    a = L.bq_act_quant_int4
+    assert a(FAKE, bq.BQ_F16, 4, 16, 16, FAKE, 1e-6, FAKE, 16, None) == bq.BQ_ERR_INVALID_ARG
+    assert a(FAKE, bq.BQ_F32, 4, 16, 8, FAKE, 1e-6, FAKE, 16, None) == bq.BQ_ERR_INVALID_ARG
+    ws = bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4A4, 300, 61, 256)
+    assert ws >= 300 * 256 + 300 * 4 + 61 * 4 + 300 * 64 * 4
+
+
+def test_bitconv1d_calls_reject(L):
+    f = L.bq_bitconv1d
+
+    def call(x=FAKE, xt=bq.BQ_BF16, B=2, C_in=64, Lx=32, lw=None, lb=None, wp=FAKE, ws_=FAKE, C_out=32, KS=3,
+             stride=1, pad=1, groups=1, bias=None, eps=1e-5, od=bq.BQ_BF16, out=FAKE, work=FAKE, nbytes=1 << 26):
+        return f(x, xt, B, C_in, Lx, lw, lb, wp, ws_, C_out, KS, stride, pad, groups, bias, eps, od, out, work, nbytes,
+                 None)
+    assert call(C_in=40) == bq.BQ_ERR_INVALID_ARG           # C_in % 16
+    assert call(groups=3) == bq.BQ_ERR_INVALID_ARG          # groups divides C_in and C_out
+    assert call(groups=2, C_out=36) == bq.BQ_ERR_INVALID_ARG  # (C_out / groups) % 4
+    assert call(KS=40, pad=0) == bq.BQ_ERR_INVALID_ARG      # no output position
+    assert call(stride=0) == bq.BQ_ERR_INVALID_ARG
+    assert call(work=None) == bq.BQ_ERR_WORKSPACE
+    assert call(x=ODD) == bq.BQ_ERR_MISALIGNED
+    assert call(B=0) == bq.BQ_OK
+    assert bq.lib().bq_bitconv1d_workspace_bytes(2, 64, 32, 32, 3, 1, 1, 1) > 3 * 2 * 32 * 32 * 4
+    g = L.bq_bitconv1d_weight_pack
+    assert g(FAKE, bq.BQ_F32, 32, 24, 3, FAKE, FAKE, FAKE, 1 << 24, None) == bq.BQ_ERR_INVALID_ARG  # Cg % 16
+    assert g(FAKE, bq.BQ_F32, 32, 32, 3, FAKE, FAKE, None, 0, None) == bq.BQ_ERR_WORKSPACE

@@ -619,3 +619,124 @@ def test_bitlinear_layernorm(M, N, K, out, bias, affine):
     assert_codes(g_xq, a["xq"], a["pre"], what + " xq")
     rel32 = bitlinear_rel32(g_sc, a["act_scale"], host(ws_)[0], t["gamma"])
     assert_out(host(o), ref, _TORCH_OUT[out], what, extra=extra, scale=scale, rel32=rel32)
+
+
+# ------------------------------------------------------- W4A4 (Q4Linear)
+
+def _q4_inputs(M, N, K, seed, per_channel, xin):
+    g = synth.rng((124, seed))
+    x = synth.normal_f32(g, (M, K))
+    if xin == "bf16":
+        bits = synth.f32_to_bf16_bits(x)
+        x = synth.bf16_bits_to_f32(bits)
+        xd = bf16_dev(bits)
+    else:
+        xd = dev(x)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    # steps: about a quarter of a standard deviation for x, max|w_n| / 7.5 per weight row
+    sa = np.array([0.27], np.float32)
+    sw = (np.abs(w).max(axis=1) / 7.5).astype(np.float32) if per_channel else np.array([0.006], np.float32)
+    return x, xd, w, sa, sw
+
+
+def _q4_band_extra(xq, x_pre, wq, w_pre, sa, sw_n, eps):
+    xband = tie_band(x_pre).astype(np.float64)
+    wband = tie_band(w_pre).astype(np.float64)
+    s_a = max(float(sa[0]), eps)
+    s_w = np.maximum(sw_n.astype(np.float64), eps)
+    return (xband @ np.abs(wq).T.astype(np.float64) + np.abs(xq).astype(np.float64) @ wband.T) * s_a * s_w[None, :]
+
+
+@pytest.mark.parametrize("N,K,per_channel,win", [(300, 256, True, "f32"), (64, 4096, False, "bf16"), (7, 8, True, "f32")])
+def test_q4_weight_pack(N, K, per_channel, win):
+    _, _, w, _, sw = _q4_inputs(1, N, K, (N, K), per_channel, "f32")
+    eps = 1e-6
+    if win == "bf16":
+        bits = synth.f32_to_bf16_bits(w)
+        w = synth.bf16_bits_to_f32(bits)
+        wd = bf16_dev(bits)
+    else:
+        wd = dev(w)
+    wp = bq.bq_weight_quant_int4_pack(wd, dev(sw), eps)
+    torch.cuda.synchronize()
+    wq, pre = oracle.q4_quant(w, sw, eps, per_row=per_channel, want_pre=True)
+    u = oracle.int4_unpack(host(wp).view(np.uint32), K).astype(np.int16)
+    codes = np.where(u >= 8, u - 16, u)
+    assert_codes(codes, wq, pre, f"q4 pack {N}x{K}")
+    if not tie_band(pre).any():
+        np.testing.assert_array_equal(host(wp).view(np.uint32), oracle.s4_pack(wq))
+
+
+@pytest.mark.parametrize("M,N,K,per_channel,bias,out,xin", [
+    (1, 11008, 4096, True, False, "bf16", "bf16"),
+    (5, 300, 1024, False, True, "f32", "f32"),
+    (16, 1000, 2048, True, True, "f16", "bf16"),
+    (17, 257, 256, True, False, "bf16", "f32"),
+    (300, 61, 512, False, True, "f16", "bf16"),
+    (300, 520, 1024, True, True, "bf16", "bf16"),
+    (2500, 4608, 256, True, False, "bf16", "bf16"),  # CTA pairs
+])
+def test_linear_w4a4(M, N, K, per_channel, bias, out, xin):
+    eps = 1e-6
+    x, xd, w, sa, sw = _q4_inputs(M, N, K, (M, N, K), per_channel, xin)
+    b = synth.normal_f32(synth.rng((125, N)), (N,), 0.1) if bias else None
+    wp = bq.bq_weight_quant_int4_pack(dev(w), dev(sw), eps)
+    work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4A4, M, N, K), dtype=torch.uint8, device="cuda")
+    o = bq.bq_linear_w4a4(xd, dev(sa), wp, dev(sw), N, eps, None if b is None else dev(b), _TORCH_OUT[out],
+                          workspace=work)
+    torch.cuda.synchronize()
+    xq, x_pre = oracle.q4_quant(x, sa, eps, want_pre=True)
+    wq, w_pre = oracle.q4_quant(w, sw, eps, per_row=per_channel, want_pre=True)
+    assert_codes(host(work[:M * K].view(torch.int8).view(M, K)), xq, x_pre, f"w4a4 act codes {M}x{K}")
+    ref = oracle.linear_w4a4_from_codes(xq, wq, sa, sw, eps, b, per_channel=per_channel)
+    sw_n = sw if per_channel else np.full(N, sw[0], np.float32)
+    extra = _q4_band_extra(xq, x_pre, wq, w_pre, sa, sw_n, eps)
+    scale = None
+    if b is not None:
+        scale = np.abs(ref - b.astype(np.float64)) + np.abs(b.astype(np.float64))
+    assert_out(host(o), ref, _TORCH_OUT[out], f"w4a4 {M}x{N}x{K}", extra=extra, scale=scale)
+
+
+# -------------------------------------------------------------- BitConv1d
+
+@pytest.mark.parametrize("B,C_in,L,C_out,KS,stride,pad,groups,xin,out,bias,affine", [
+    (2, 64, 37, 48, 3, 1, 1, 1, "bf16", "bf16", True, True),
+    (1, 128, 100, 96, 4, 2, 0, 2, "f32", "f32", False, False),
+    (3, 32, 9, 8, 5, 1, 2, 1, "f32", "f16", True, False),
+    (2, 80, 20, 40, 3, 1, 1, 1, "bf16", "bf16", False, True),       # channels re-pitched to 128
+    (4, 512, 256, 512, 3, 1, 1, 1, "bf16", "bf16", True, False),     # several GEMM tiles per tap
+    (2, 256, 64, 64, 1, 1, 0, 4, "bf16", "f32", False, True),
+])
+def test_bitconv1d(B, C_in, L, C_out, KS, stride, pad, groups, xin, out, bias, affine):
+    g = synth.rng((126, B, C_in, L, C_out, KS))
+    x = synth.normal_f32(g, (B, C_in, L)) + np.float32(0.3)
+    if xin == "bf16":
+        bits = synth.f32_to_bf16_bits(x)
+        x = synth.bf16_bits_to_f32(bits)
+        xd = bf16_dev(bits)
+    else:
+        xd = dev(x)
+    w = synth.normal_f32(g, (C_out, C_in // groups, KS), 0.02)
+    b = synth.normal_f32(g, (C_out,), 0.1) if bias else None
+    lw, lb = _ln_params(g, C_in, affine)
+    wp, ws_ = bq.bq_bitconv1d_weight_pack(dev(w))
+    o = bq.bq_bitconv1d(xd, wp, ws_, C_out, KS, stride, pad, groups, None if lw is None else dev(lw),
+                        None if lb is None else dev(lb), None if b is None else dev(b), 1e-5, _TORCH_OUT[out])
+    torch.cuda.synchronize()
+    a = oracle.bitconv1d_act_quant(x, 1e-5, lw, lb, want_pre=True)
+    t = oracle.ternary_quant(w.reshape(C_out, -1), want_pre=True)
+    assert float(host(ws_)[0]) == pytest.approx(t["gamma"], rel=1e-6)
+    wq = t["wq"].reshape(w.shape)
+    conv = lambda xc, wc, bb=None: oracle.bitconv1d_from_codes(xc, a["act_scale"], wc, t["gamma"], B, L, stride, pad,
+                                                               groups, bb)
+    ref = conv(a["xq"], wq, b)
+    # term magnitude and tie-band widening, from the oracle's conv of absolute codes / band indicators
+    absx, absw = np.abs(a["xq"].astype(np.int16)).astype(np.int8), np.abs(wq)
+    mag = conv(absx, absw)
+    extra = conv(tie_band(a["pre"]).astype(np.int8), absw) + \
+        conv(absx, tie_band(t["pre"]).reshape(w.shape).astype(np.int8))
+    if b is not None:
+        mag = mag + np.abs(b.astype(np.float64))[None, :, None]
+    rel32 = (KS + 7) * 2.0 ** -24  # fp32 tap products and tap sum (scales are binary64 rounded once)
+    assert_out(host(o), ref, _TORCH_OUT[out], f"bitconv1d {B}x{C_in}x{L} -> {C_out} k{KS} s{stride} p{pad} g{groups}",
+               extra=extra, scale=mag, rel32=rel32)

@@ -464,3 +464,113 @@ def test_layernorm_quant_constant_row_and_affine_closed_forms():
     r = oracle.act_quant_layernorm(x, ln_bias=b, want_pre=True)
     np.testing.assert_allclose(r["pre"][0], b.astype(np.float64) * 127.0 / np.abs(b).max(), rtol=1e-15)
     assert r["act_scale"][0] == pytest.approx(1.0 / 127.0, rel=1e-15)
+
+
+# ------------------------------------------------------- W4A4 (Q4Linear)
+
+def test_q4_quant_hand_cases():
+    # step 0.5: values on the grid, half-step ties to even, clamping at -8 / 7
+    v = np.array([[0.0, 0.5, -0.5, 0.25, 0.75, -0.25, -0.75, 1.25, 3.5, 3.75, 4.0, -4.0, -4.25, 100.0, -100.0,
+                   0.2499]], np.float32)
+    want = [0, 1, -1, 0, 2, 0, -2, 2, 7, 7, 7, -8, -8, 7, -8, 0]
+    np.testing.assert_array_equal(oracle.q4_quant(v, np.float32(0.5), 1e-8)[0], want)
+    # a step below eps is replaced by eps (no division by zero)
+    np.testing.assert_array_equal(oracle.q4_quant(np.array([[0.0, 1e-6, -3e-6]], np.float32), np.float32(0.0), 1e-6)[0],
+                                  [0, 1, -3])
+    # per-row steps
+    q = oracle.q4_quant(np.array([[1.0, 2.0], [1.0, 2.0]], np.float32), np.array([1.0, 0.5], np.float32), 1e-8,
+                        per_row=True)
+    np.testing.assert_array_equal(q, [[1, 2], [2, 4]])
+
+
+def test_w4a4_unit_steps_is_integer_matmul():
+    # integer inputs inside [-8, 7] with unit steps are their own codes, so
+    # the forward is the integer matmul (numpy int64), plus the bias
+    g = synth.rng(22)
+    x = g.integers(-8, 8, (6, 48)).astype(np.float32)
+    w = g.integers(-8, 8, (9, 48)).astype(np.float32)
+    b = synth.normal_f32(g, (9,), 0.1)
+    out, xq, wq = oracle.linear_w4a4(x, w, np.float32(1.0), np.float32(1.0), 1e-6, b)
+    np.testing.assert_array_equal(xq, x.astype(np.int8))
+    ref = x.astype(np.int64) @ w.astype(np.int64).T
+    np.testing.assert_array_equal(out, ref.astype(np.float64) + b.astype(np.float64))
+
+
+def test_w4a4_scales_pin_order_and_channel():
+    # per-channel weight steps: out[m,n] = acc * s_w[n] * s_a exactly (powers of two)
+    g = synth.rng(23)
+    xq = g.integers(-8, 8, (4, 32)).astype(np.int8)
+    wq = g.integers(-8, 8, (5, 32)).astype(np.int8)
+    sw = np.array([0.5, 0.25, 2.0, 1.0, 0.125], np.float32)
+    out = oracle.linear_w4a4_from_codes(xq, wq, np.float32(0.0625), sw, 1e-9, per_channel=True)
+    acc = xq.astype(np.int64) @ wq.astype(np.int64).T
+    np.testing.assert_array_equal(out, acc * sw.astype(np.float64)[None, :] * 0.0625)
+
+
+def test_s4_pack_golden_and_roundtrip():
+    q = np.array([[0, 1, -1, 7, -8, 2, -3, 5]], np.int8)
+    # nibbles low first: 0x0, 0x1, 0xF, 0x7, 0x8, 0x2, 0xD, 0x5
+    assert int(oracle.s4_pack(q)[0, 0]) == 0x5D287F10
+    g = synth.rng(24)
+    q = g.integers(-8, 8, (7, 64)).astype(np.int8)
+    u = oracle.int4_unpack(oracle.s4_pack(q), 64).astype(np.int16)
+    np.testing.assert_array_equal(np.where(u >= 8, u - 16, u), q)
+
+
+# ------------------------------------------------------------- BitConv1d
+
+def test_bitconv1d_matches_torch_conv1d_of_dequantized_values():
+    # the convolution of the dequantized operands (xq * act_scale, wq * gamma)
+    # by torch's conv1d in float64, for strides, padding and groups
+    g = synth.rng(25)
+    for (B, C_in, L, C_out, KS, stride, pad, groups) in [(2, 16, 11, 8, 3, 1, 1, 1), (1, 12, 9, 6, 2, 2, 0, 3),
+                                                          (3, 8, 5, 4, 5, 1, 2, 2)]:
+        x = synth.normal_f32(g, (B, C_in, L))
+        w = synth.normal_f32(g, (C_out, C_in // groups, KS), 0.02)
+        bias = synth.normal_f32(g, (C_out,), 0.1)
+        out, a, t = oracle.bitconv1d(x, w, stride=stride, pad=pad, groups=groups, bias=bias)
+        xd = (a["xq"].astype(np.float64) * a["act_scale"][:, None]).reshape(B, L, C_in).transpose(0, 2, 1)
+        wd = t["wq"].reshape(w.shape).astype(np.float64) * t["gamma"]
+        ref = torch.nn.functional.conv1d(torch.from_numpy(np.ascontiguousarray(xd)), torch.from_numpy(wd),
+                                         torch.from_numpy(bias.astype(np.float64)), stride=stride, padding=pad,
+                                         groups=groups).numpy()
+        np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-14)
+
+
+def test_bitconv1d_kernel_one_is_bitlinear_per_position():
+    # kernel size 1, stride 1, no padding: each position is a BitLinear of
+    # its LayerNorm-normalised channel vector
+    g = synth.rng(26)
+    B, C_in, L, C_out = 2, 32, 7, 5
+    x = synth.normal_f32(g, (B, C_in, L))
+    w = synth.normal_f32(g, (C_out, C_in, 1), 0.02)
+    out, _, _ = oracle.bitconv1d(x, w)
+    rows = np.ascontiguousarray(x.transpose(0, 2, 1).reshape(B * L, C_in))
+    ref, _, _ = oracle.bitlinear_layernorm(rows, w[:, :, 0])
+    np.testing.assert_allclose(out, ref.reshape(B, L, C_out).transpose(0, 2, 1), rtol=1e-14, atol=0)
+
+
+# ------------------------------------------------- BitLinear STE backward
+
+def test_bitlinear_backward_matches_autograd_of_the_ste_surrogate():
+    # torch autograd (fp64) of the straight-through forward written with
+    # detach: y + (xt - y).detach() and w + (wt - w).detach(), where xt and wt
+    # are the oracle's dequantized operands, through torch's own RMSNorm
+    g = synth.rng(27)
+    M, N, K = 6, 10, 48
+    x = synth.normal_f32(g, (M, K))
+    w = synth.normal_f32(g, (N, K), 0.02)
+    dout = synth.normal_f32(g, (M, N))
+    eps = 1e-5
+    dx, dw = oracle.bitlinear_backward(x, w, dout, eps)
+    a = oracle.act_quant(x, eps)
+    t = oracle.ternary_quant(w)
+    xt = torch.from_numpy(a["xq"].astype(np.float64) * a["act_scale"][:, None])
+    wt = torch.from_numpy(t["wq"].astype(np.float64) * t["gamma"])
+    xx = torch.from_numpy(x.astype(np.float64)).requires_grad_()
+    ww = torch.from_numpy(w.astype(np.float64)).requires_grad_()
+    y = torch.nn.functional.rms_norm(xx, (K,), eps=eps)
+    out = (y + (xt - y).detach()) @ (ww + (wt - ww).detach()).T
+    out.backward(torch.from_numpy(dout.astype(np.float64)))
+    np.testing.assert_allclose(dx, xx.grad.numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(dw, ww.grad.numpy(), rtol=1e-10, atol=1e-13)
