@@ -9,14 +9,21 @@
 // pre-rounding value of a code near +-0.5 would move by ~1e-5 (the mean's own
 // rounding, scaled by 127 / max|y|), far more than the 1e-6 relative band in
 // which a code may round either way, so codes would not be reproducible.  In
-// binary64 every pre-rounding value is within a few 2^-53 of the exact one.
+// binary64 every pre-rounding value is within a few 2^-53 of the exact one
+// (the row's 1/sqrt(var + eps) and 127/max|y| are each taken once and
+// multiplied in, a few ulp of binary64 from dividing per element).
 //
-// One CTA per row (grid-stride over rows).  Pass 1 reads the row from HBM
-// (sum), passes 2-4 (sum of squared deviations, max|y|, codes) re-read it from
-// L1/L2 (a row of 4096 bf16 is 8 KB).  HBM-bound on the first read; the fp64
-// work per element is a handful of operations.
+// One CTA per row (grid-stride over rows).  Aligned rows of up to 1024
+// 16-byte chunks are read once into registers and every pass (mean,
+// variance, max|y|, codes) works from there; other rows take the general
+// kernel, which re-reads the row from L1/L2 in each pass.  HBM-bound: one
+// read of x, one write of the codes; the fp64 work per element is a handful
+// of operations.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
+#include "bq_common.cuh"
 #include "bq_internal.h"
 
 namespace bq {
@@ -54,6 +61,8 @@ __global__ void __launch_bounds__(kLnThreads)
     auto mx = [](double p, double q) { return fmax(p, q); };
     auto addi = [](int p, int q) { return p + q; };
     const double inv_k = 1.0 / static_cast<double>(K);
+    pdl_wait();  // x may come from the previous kernel; its readers of xq are done
+    pdl_launch_dependents();
     for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
         const In *xr = x + m * ldx;
         double s = 0.0;
@@ -65,9 +74,9 @@ __global__ void __launch_bounds__(kLnThreads)
             q = fma(d, d, q);
         }
         const double var = block_reduce(q, red_d, add) * inv_k;
-        const double sd = sqrt(var + eps);
+        const double rsd = 1.0 / sqrt(var + eps);  // one division per row
         auto y_of = [&](int64_t k) {
-            const double d = (load_x(xr, k) - mu) / sd;
+            const double d = (load_x(xr, k) - mu) * rsd;
             const double gk = g != nullptr ? static_cast<double>(__ldg(g + k)) : 1.0;
             const double bk = b != nullptr ? static_cast<double>(__ldg(b + k)) : 0.0;
             return fma(d, gk, bk);
@@ -92,21 +101,165 @@ __global__ void __launch_bounds__(kLnThreads)
     }
 }
 
+// Rows with 16-byte aligned bases and K a multiple of the elements per
+// 16-byte chunk, at most 256 * CPT chunks: one read of the row from HBM into
+// registers (chunk c of a row held by thread c % 256), then the mean, the
+// variance, max|y| and the codes from registers.
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<float> {
+    static constexpr int kElts = 4;
+    __device__ static void unpack(const uint4 &v, float (&f)[4]) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int kElts = 8;
+    __device__ static void unpack(const uint4 &v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+template <typename In, int CPT>
+__global__ void __launch_bounds__(kLnThreads)
+    act_quant_ln_vec_kernel(const In *__restrict__ x, int64_t M, int64_t K, int64_t ldx, double eps,
+                            const float *__restrict__ g, const float *__restrict__ b, int8_t *__restrict__ xq,
+                            int64_t ldq, float *__restrict__ act_scale, int32_t *__restrict__ rowsum) {
+    constexpr int E = Vec16<In>::kElts;
+    __shared__ double red_d[kLnThreads / 32];
+    __shared__ int red_i[kLnThreads / 32];
+    auto add = [](double p, double q) { return p + q; };
+    auto mx = [](double p, double q) { return fmax(p, q); };
+    auto addi = [](int p, int q) { return p + q; };
+    const double inv_k = 1.0 / static_cast<double>(K);
+    const int nch = static_cast<int>(K / E);
+    pdl_wait();  // x may come from the previous kernel; its readers of xq are done
+    pdl_launch_dependents();
+    for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * ldx);
+        float v[CPT][E];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + kLnThreads * i;
+            const uint4 u = c < nch ? __ldcs(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+            Vec16<In>::unpack(u, v[i]);
+        }
+        double s = 0.0;
+#pragma unroll
+        for (int i = 0; i < CPT; ++i)
+#pragma unroll
+            for (int e = 0; e < E; ++e) s += static_cast<double>(v[i][e]);
+        const double mu = block_reduce(s, red_d, add) * inv_k;
+        double q = 0.0;
+#pragma unroll
+        for (int i = 0; i < CPT; ++i)
+            if (threadIdx.x + kLnThreads * i < nch)
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const double d = static_cast<double>(v[i][e]) - mu;
+                    q = fma(d, d, q);
+                }
+        const double rsd = 1.0 / sqrt(block_reduce(q, red_d, add) * inv_k + eps);  // one division per row
+        auto y_of = [&](int i, int e) {
+            const int64_t k = static_cast<int64_t>(threadIdx.x + kLnThreads * i) * E + e;
+            const double d = (static_cast<double>(v[i][e]) - mu) * rsd;
+            const double gk = g != nullptr ? static_cast<double>(__ldg(g + k)) : 1.0;
+            const double bk = b != nullptr ? static_cast<double>(__ldg(b + k)) : 0.0;
+            return fma(d, gk, bk);
+        };
+        double amax = 0.0;
+#pragma unroll
+        for (int i = 0; i < CPT; ++i)
+            if (threadIdx.x + kLnThreads * i < nch)
+#pragma unroll
+                for (int e = 0; e < E; ++e) amax = fmax(amax, fabs(y_of(i, e)));
+        const double a = fmax(block_reduce(amax, red_d, mx), 1e-5);
+        const double f = 127.0 / a;
+        int isum = 0;
+        int8_t *qr = xq + m * ldq;
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = threadIdx.x + kLnThreads * i;
+            if (c < nch) {
+                uint32_t w[E / 4];
+#pragma unroll
+                for (int j = 0; j < E / 4; ++j) {
+                    uint32_t word = 0;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        int code = __double2int_rn(y_of(i, 4 * j + u) * f);  // nearest, ties to even
+                        code = code < -128 ? -128 : (code > 127 ? 127 : code);
+                        isum += code;
+                        word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * u);
+                    }
+                    w[j] = word;
+                }
+                if constexpr (E == 8)
+                    *reinterpret_cast<uint2 *>(qr + static_cast<int64_t>(c) * 8) = make_uint2(w[0], w[1]);
+                else
+                    *reinterpret_cast<uint32_t *>(qr + static_cast<int64_t>(c) * 4) = w[0];
+            }
+        }
+        isum = block_reduce(isum, red_i, addi);
+        if (threadIdx.x == 0) {
+            act_scale[m] = static_cast<float>(a / 127.0);
+            if (rowsum != nullptr) rowsum[m] = isum;
+        }
+    }
+}
+
+template <typename In>
+cudaError_t launch_ln_typed(const In *x, int64_t M, int64_t K, int64_t ldx, double eps, const float *g, const float *b,
+                            int8_t *xq, int64_t ldq, float *act_scale, int32_t *rowsum, cudaStream_t s,
+                            const DevInfo &dev) {
+    constexpr int E = Vec16<In>::kElts;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(M, static_cast<int64_t>(dev.num_sms) * 8));
+    const bool vec = reinterpret_cast<uintptr_t>(x) % 16 == 0 && (ldx * static_cast<int64_t>(sizeof(In))) % 16 == 0 &&
+                     K % E == 0 && reinterpret_cast<uintptr_t>(xq) % 8 == 0 && ldq % 8 == 0;
+    const int64_t cpt = (K / E + kLnThreads - 1) / kLnThreads;
+    // launched as a programmatic dependent of the previous kernel; it waits for
+    // it before touching memory and then releases its own dependent
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kLnThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (vec && cpt <= 1)
+        return cudaLaunchKernelEx(&cfg, act_quant_ln_vec_kernel<In, 1>, x, M, K, ldx, eps, g, b, xq, ldq, act_scale,
+                                  rowsum);
+    if (vec && cpt <= 2)
+        return cudaLaunchKernelEx(&cfg, act_quant_ln_vec_kernel<In, 2>, x, M, K, ldx, eps, g, b, xq, ldq, act_scale,
+                                  rowsum);
+    if (vec && cpt <= 4)
+        return cudaLaunchKernelEx(&cfg, act_quant_ln_vec_kernel<In, 4>, x, M, K, ldx, eps, g, b, xq, ldq, act_scale,
+                                  rowsum);
+    return cudaLaunchKernelEx(&cfg, act_quant_ln_kernel<In>, x, M, K, ldx, eps, g, b, xq, ldq, act_scale, rowsum);
+}
+
 }  // namespace
 
 cudaError_t launch_act_quant_ln(const void *x, bq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *ln_weight,
                                 const float *ln_bias, float eps, int8_t *xq, int64_t ldq, float *act_scale,
                                 int32_t *rowsum, cudaStream_t s, const DevInfo &dev) {
-    const int64_t grid = std::min<int64_t>(M, static_cast<int64_t>(dev.num_sms) * 8);
     if (xt == BQ_BF16)
-        act_quant_ln_kernel<__nv_bfloat16><<<static_cast<unsigned>(grid), kLnThreads, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(x), M, K, ldx, static_cast<double>(eps), ln_weight, ln_bias, xq, ldq,
-            act_scale, rowsum);
-    else
-        act_quant_ln_kernel<float><<<static_cast<unsigned>(grid), kLnThreads, 0, s>>>(
-            static_cast<const float *>(x), M, K, ldx, static_cast<double>(eps), ln_weight, ln_bias, xq, ldq,
-            act_scale, rowsum);
-    return cudaGetLastError();
+        return launch_ln_typed(static_cast<const __nv_bfloat16 *>(x), M, K, ldx, static_cast<double>(eps), ln_weight,
+                               ln_bias, xq, ldq, act_scale, rowsum, s, dev);
+    return launch_ln_typed(static_cast<const float *>(x), M, K, ldx, static_cast<double>(eps), ln_weight, ln_bias, xq,
+                           ldq, act_scale, rowsum, s, dev);
 }
 
 }  // namespace bq

@@ -447,6 +447,11 @@ bq_status bq_bitlinear_w2a8_layernorm(const void *x, bq_dtype x_dtype, int64_t M
                             reinterpret_cast<float *>(ws + l.scale), reinterpret_cast<int32_t *>(ws + l.rowsum), s,
                             dev) != cudaSuccess)
         return BQ_ERR_CUDA;
+    if (M <= kGemvMaxM && decode_mma_from_codes_supported(M, N, K, dev))
+        return from_cuda(launch_decode_mma_from_codes(reinterpret_cast<int8_t *>(ws + l.xq),
+                                                      reinterpret_cast<float *>(ws + l.scale),
+                                                      reinterpret_cast<int32_t *>(ws + l.rowsum), M, K, wpacked,
+                                                      w_scale, bias, N, out_dtype, out, s, dev));
     const int path = M > kGemvMaxM ? bitlinear_path(x, x_dtype, M, N, K, dev) : BQ_PATH_ACT_QUANT_GEMV;
     return bitlinear_linear(path, l, ws, M, K, wpacked, w_scale, N, bias, out_dtype, out, s, dev);
 }

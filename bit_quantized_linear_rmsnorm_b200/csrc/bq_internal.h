@@ -121,6 +121,15 @@ bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const
 // Which decode kernel launch_decode_w2a8 runs for a supported shape
 // (BQ_PATH_DECODE_STREAM, BQ_PATH_DECODE_MMA or BQ_PATH_DECODE_SMEM).
 int decode_w2a8_kind(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev);
+// The weight-streaming half of the 2..16-token decode path on codes already in
+// global memory (written by a kernel launched just before it that waits for
+// its own predecessors before it releases its dependents, as every quantizer
+// of this library does).  1..16 tokens, K 2048 or 4096.
+bool decode_mma_from_codes_supported(int64_t M, int64_t N, int64_t K, const DevInfo &dev);
+cudaError_t launch_decode_mma_from_codes(const int8_t *xq, const float *act_scale, const int32_t *rowsum, int64_t M,
+                                         int64_t K, const uint32_t *wpacked, const float *w_scale, const float *bias,
+                                         int64_t N, bq_dtype out_dtype, void *out, cudaStream_t s,
+                                         const DevInfo &dev);
 cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K, float eps, const uint32_t *wpacked,
                                const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
                                int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,

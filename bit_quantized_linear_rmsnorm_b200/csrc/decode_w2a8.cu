@@ -894,17 +894,19 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_w2a8_mma_kernel(const D
     pdl_launch_dependents();
     pdl_wait();  // the token codes are written and visible
 
-    // token codes -> shared memory (swizzled rows), per-token scale and row sum
+    // token codes -> shared memory (swizzled rows) with asynchronous 16-byte
+    // copies, all of a thread's in flight at once; per-token scale and row sum
     const int cpr = K / 16;  // 16-byte chunks per token row
     for (int i = threadIdx.x; i < M * cpr; i += kMmaThreads) {
         const int m = i / cpr, c = i - m * cpr;
-        *reinterpret_cast<uint4 *>(xs + m * xp + xchunk_swz(c) * 16) =
-            __ldcg(reinterpret_cast<const uint4 *>(p.ws_xq + static_cast<int64_t>(m) * K) + c);
+        cp_async_16(smem_u32(xs + m * xp + xchunk_swz(c) * 16), p.ws_xq + static_cast<int64_t>(m) * K + 16 * c, 16);
     }
+    cp_async_commit();
     if (threadIdx.x < M) {
         s_scale[threadIdx.x] = __ldcg(p.ws_scale + threadIdx.x);
         s_rowsum[threadIdx.x] = __ldcg(p.ws_rowsum + threadIdx.x);
     }
+    cp_async_wait_all();
     __syncthreads();
 
     // per unit: the masked A fragments once, both token groups; the
@@ -1097,6 +1099,49 @@ bool decode_w2a8_supported(const void *x, int64_t M, int64_t N, int64_t K, const
     const int rb = rows_per_cta(N, dev);
     if (rb > kMaxRB || rb < 1) return false;
     return Layout(static_cast<int>(K), mt_of(M), rb).total + 1024 <= dev.max_smem_optin;
+}
+
+bool decode_mma_from_codes_supported(int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
+    return M >= 1 && mma_stream_supported(M < 2 ? 2 : M, N, K, dev);
+}
+
+cudaError_t launch_decode_mma_from_codes(const int8_t *xq, const float *act_scale, const int32_t *rowsum, int64_t M,
+                                         int64_t K, const uint32_t *wpacked, const float *w_scale, const float *bias,
+                                         int64_t N, bq_dtype out_dtype, void *out, cudaStream_t s,
+                                         const DevInfo &dev) {
+    DecodeArgs a;
+    a.x = nullptr;
+    a.M = static_cast<int>(M);
+    a.K = static_cast<int>(K);
+    a.eps = 0.0f;
+    a.wpacked = wpacked;
+    a.w_scale = w_scale;
+    a.bias = bias;
+    a.N = static_cast<int>(N);
+    a.out = out;
+    a.ws_xq = const_cast<int8_t *>(xq);
+    a.ws_scale = const_cast<float *>(act_scale);
+    a.ws_rowsum = const_cast<int32_t *>(rowsum);
+    a.rb = rows_per_cta(N, dev);
+    a.status = dev.status;
+    a.out_dtype = out_dtype;
+    const int grid = grid_of(N, dev);
+    const bool two = M > 8;
+    const void *kern;
+    int smem;
+    if (K == 2048) {
+        kern = two ? reinterpret_cast<const void *>(decode_w2a8_mma_kernel<16, 1>)
+                   : reinterpret_cast<const void *>(decode_w2a8_mma_kernel<8, 1>);
+        smem = two ? MmaLayout<16, 1>::bytes(2048) : MmaLayout<8, 1>::bytes(2048);
+    } else {
+        kern = two ? reinterpret_cast<const void *>(decode_w2a8_mma_kernel<16, 2>)
+                   : reinterpret_cast<const void *>(decode_w2a8_mma_kernel<8, 2>);
+        smem = two ? MmaLayout<16, 2>::bytes(4096) : MmaLayout<8, 2>::bytes(4096);
+    }
+    static SmemOptIn opt_in[4];
+    const cudaError_t e = smem_opt_in(opt_in[(K == 2048 ? 0 : 2) + (two ? 1 : 0)], dev, kern, static_cast<size_t>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cfg(kern, a, grid, kMmaThreads, smem, s);
 }
 
 int decode_w2a8_kind(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev) {
