@@ -196,6 +196,8 @@ size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t gro
             return linear_w4_workspace_bytes(M, N, K, group_size);
         case BQ_OP_LINEAR_W4A4:
             return w4a4_layout(M, N, K).total;
+        case BQ_OP_BITLINEAR_W2A8_BACKWARD:
+            return bitlinear_bwd_layout(M, N, K).total;
         default:
             return 0;
     }
@@ -648,6 +650,28 @@ bq_status bq_bitconv1d(const void *x, bq_dtype x_dtype, int64_t B, int64_t C_in,
     if (st != BQ_OK) return st;
     return launch_bitconv1d(x, x_dtype, B, C_in, L, ln_weight, ln_bias, wpacked, w_scale, C_out, KS, stride, pad, groups,
                             bias, eps, out_dtype, out, workspace, static_cast<cudaStream_t>(stream), dev);
+}
+
+bq_status bq_bitlinear_w2a8_backward(const void *x, bq_dtype x_dtype, const void *dout, int64_t M, int64_t K,
+                                     const uint32_t *wpacked, const float *w_scale, int64_t N, float eps, float *dx,
+                                     float *dw, void *workspace, size_t workspace_bytes, bq_stream_t stream) {
+    if (!act_dtype_ok(x_dtype) || M < 0 || N < 0 || K < 1 || K % 16 != 0 || N % 8 != 0 || K > kMaxK ||
+        M > kMaxDim / 2 || N > kMaxDim || !std::isfinite(eps) || eps < 0.0f)
+        return BQ_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return BQ_OK;
+    if (x == nullptr || dout == nullptr || wpacked == nullptr || w_scale == nullptr || dx == nullptr || dw == nullptr)
+        return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(dout, 16) || !aligned(wpacked, 16) || !aligned(w_scale, 4) || !aligned(dx, 16) ||
+        !aligned(dw, 16))
+        return BQ_ERR_MISALIGNED;
+    const size_t need = bitlinear_bwd_layout(M, N, K).total;
+    if (workspace == nullptr || workspace_bytes < need) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    return launch_bitlinear_backward(x, x_dtype, dout, M, K, wpacked, w_scale, N, eps, dx, dw, workspace,
+                                     static_cast<cudaStream_t>(stream), dev);
 }
 
 bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint32_t *qweight,

@@ -160,6 +160,34 @@ bq_status launch_bitconv1d(const void *x, bq_dtype xt, int64_t B, int64_t C_in, 
                            int64_t KS, int64_t stride, int64_t pad, int64_t groups, const float *bias, float eps,
                            bq_dtype out_dtype, void *out, void *workspace, cudaStream_t s, const DevInfo &dev);
 
+// bf16 x bf16 -> fp32 tensor-core GEMM (gemm_bf16.cu):
+//   out[m,n] = (*scale or 1) * sum_k A(m,k) * B(k,n)
+// A [M][lda] K-major or [K][lda] M-major (a_mn); B [N][ldb] K-major or
+// [K][ldb] N-major (b_mn); out fp32 [M][ldo].  lda, ldb % 8 == 0, ldo % 4 == 0.
+struct Bf16Args {
+    const void *a = nullptr;
+    int64_t lda = 0;
+    bool a_mn = false;
+    const void *b = nullptr;
+    int64_t ldb = 0;
+    bool b_mn = false;
+    int64_t M = 0, N = 0, K = 0;
+    const float *scale = nullptr;
+    float *out = nullptr;
+    int64_t ldo = 0;
+};
+bq_status launch_gemm_bf16(const Bf16Args &g, cudaStream_t s, const DevInfo &dev);
+
+// Straight-through backward of BitLinear (bitlinear_bwd.cu): workspace layout
+// (xq, act_scale, bf16 ternary weights, the dW operands, dy) and the launch.
+struct BwdLayout {
+    size_t xq = 0, scale = 0, wt = 0, a2 = 0, b2 = 0, dy = 0, total = 0;
+};
+BwdLayout bitlinear_bwd_layout(int64_t M, int64_t N, int64_t K);
+bq_status launch_bitlinear_backward(const void *x, bq_dtype xt, const void *dout, int64_t M, int64_t K,
+                                    const uint32_t *wpacked, const float *w_scale, int64_t N, float eps, float *dx,
+                                    float *dw, void *workspace, cudaStream_t s, const DevInfo &dev);
+
 // Grouped INT4 linear.
 size_t linear_w4_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t group_size);
 // Multi-token path on the tensor cores (2..32 tokens, K % 1024 == 0, groups of 128k).

@@ -143,7 +143,9 @@ struct Items {
 };
 
 // 16 weights of one 16-byte chunk from the packed slab word(s): ternary codes
-// are expanded to u8 codes (w + 1), signed 4-bit codes sign-extended to s8.
+// are expanded to u8 codes (w + 1); a signed 4-bit code n goes to the high
+// half of its byte, which read as s8 is exactly 16 n (the epilogue divides the
+// accumulator by 16, exactly).
 template <int PK>
 __device__ __forceinline__ uint4 unpack_chunk(const uint32_t *words, int c) {
     if constexpr (PK == 2) {
@@ -155,9 +157,7 @@ __device__ __forceinline__ uint4 unpack_chunk(const uint32_t *words, int c) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const uint32_t w = h ? u.y : u.x;
-            uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;  // even / odd nibbles as bytes
-            lo |= (lo & 0x08080808u) * 30u;  // sign extension: bit 3 set -> byte | 0xF0 (no carry between bytes)
-            hi |= (hi & 0x08080808u) * 30u;
+            const uint32_t lo = (w << 4) & 0xF0F0F0F0u, hi = w & 0xF0F0F0F0u;  // even / odd nibbles, 16 n as s8
             r[2 * h] = __byte_perm(lo, hi, 0x5140);
             r[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
         }
@@ -393,7 +393,8 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
                 float f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float a = static_cast<float>(static_cast<int>(v[j]) - corr);
+                    float a = static_cast<float>(static_cast<int>(v[j]) - corr);
+                    if constexpr (PK == 4) a = __fmul_rn(a, 0.0625f);  // 16 x the code products, exact
                     float o;
                     if constexpr (TERN)
                         o = __fmul_rn(__fmul_rn(a, rs), colscale_scalar);
@@ -807,7 +808,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
                 float f[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const float a = static_cast<float>(static_cast<int>(v[j]) - corr);
+                    float a = static_cast<float>(static_cast<int>(v[j]) - corr);
+                    if constexpr (PK == 4) a = __fmul_rn(a, 0.0625f);  // 16 x the code products, exact
                     const float o = TERN ? __fmul_rn(__fmul_rn(a, rs), colscale_scalar)
                                            : __fmul_rn(__fmul_rn(a, vcol[c32 * 32 + j]), rs);
                     f[j] = __fadd_rn(o, vbias[c32 * 32 + j]);

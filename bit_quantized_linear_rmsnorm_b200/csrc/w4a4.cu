@@ -80,8 +80,9 @@ __global__ void q4_act_quant_kernel(const In *__restrict__ x, int64_t M, int64_t
 
 // Up to 16 tokens: one warp per weight row at a time (grid-stride over rows),
 // lanes stride over 16-byte pieces (32 weights) of the row; the codes of all
-// tokens sit in shared memory.  A piece's nibbles are sign-extended to bytes
-// (x | ((x & 0x08080808) * 30) per byte, no carries) and dotted with dp4a.
+// tokens sit in shared memory.  Each nibble n goes to the high half of a byte,
+// which read as s8 is exactly 16 n; dp4a sums 16 x the products, and the
+// final sum is shifted down by 4 (exact).
 constexpr int kGemvWarps = 8;
 
 template <int MT, typename OutT>
@@ -108,9 +109,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
             uint32_t b[8];  // 32 sign-extended codes, k = 32 pc + 4 j + 0..3 in b[j]
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-                uint32_t lo = ws[h] & 0x0F0F0F0Fu, hi = (ws[h] >> 4) & 0x0F0F0F0Fu;
-                lo |= (lo & 0x08080808u) * 30u;
-                hi |= (hi & 0x08080808u) * 30u;
+                const uint32_t lo = (ws[h] << 4) & 0xF0F0F0F0u, hi = ws[h] & 0xF0F0F0F0u;
                 b[2 * h] = __byte_perm(lo, hi, 0x5140);
                 b[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
             }
@@ -144,6 +143,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
 #pragma unroll
             for (int m = 1; m < MT; ++m)
                 if (lane == m) v = acc[m];
+            v >>= 4;  // the sum of 16 x the products
             float o = __fmul_rn(__fmul_rn(static_cast<float>(v), __ldg(col_step + n)), __ldg(row_step + lane));
             if (bias != nullptr) o = __fadd_rn(o, __ldg(bias + n));
             if constexpr (sizeof(OutT) == 4)

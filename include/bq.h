@@ -79,7 +79,8 @@ typedef enum {
     BQ_OP_GEMM_I8_PERTOKEN = 3,
     BQ_OP_BITLINEAR_W2A8 = 4,
     BQ_OP_LINEAR_W4_GROUPED = 5,
-    BQ_OP_LINEAR_W4A4 = 6
+    BQ_OP_LINEAR_W4A4 = 6,
+    BQ_OP_BITLINEAR_W2A8_BACKWARD = 7
 } bq_op;
 
 /*
@@ -242,6 +243,32 @@ bq_status bq_bitlinear_w2a8_layernorm(const void *x, bq_dtype x_dtype, int64_t M
                                       const float *ln_bias, const uint32_t *wpacked, const float *w_scale, int64_t N,
                                       const float *bias, float eps, bq_dtype out_dtype, void *out, void *workspace,
                                       size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Backward of the BitLinear forward under the straight-through estimator.
+ * Source: "Class BitLinear" (LLaMA-BitNet utils.py), forward steps 2-3
+ * ("Quantise ... (STE)"); "Common Attention Utilities", activation_quant and
+ * weight_quant (the STE "passes gradients through the rounding operation
+ * unchanged").  With the forward's xq, act_scale (recomputed from x) and the
+ * ternary codes wq with scale gamma:
+ *
+ *   dw[n,k] = sum_m dout[m,n] * act_scale[m] * xq[m,k]
+ *   dy[m,k] = gamma * sum_n dout[m,n] * wq[n,k]
+ *   dx[m,k] = (dy[m,k] - y[m,k] * mean_j(dy[m,j] * y[m,j])) / r[m],
+ *   y = x / r, r = sqrt(mean(x^2) + eps)   (the parameter-free RMSNorm's backward)
+ *
+ * x: dense [M][K] fp32 or bf16; dout: dense bf16 [M][N] (the incoming
+ * gradient); wpacked, w_scale as bq_bitlinear_w2a8; K % 16 == 0, N % 8 == 0.
+ * dx: fp32 [M][K]; dw: fp32 [N][K] (the gradient of the master weight).  The
+ * contractions run on the bf16 tensor cores (tcgen05 kind::f16, fp32
+ * accumulation): dout and the codes are exact in bf16, and the products
+ * dout * act_scale of dw are split into two bf16 parts (16 significant bits).
+ * workspace: bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8_BACKWARD, M, N, K, 0)
+ * bytes, 256-byte aligned.
+ */
+bq_status bq_bitlinear_w2a8_backward(const void *x, bq_dtype x_dtype, const void *dout, int64_t M, int64_t K,
+                                     const uint32_t *wpacked, const float *w_scale, int64_t N, float eps, float *dx,
+                                     float *dw, void *workspace, size_t workspace_bytes, bq_stream_t stream);
 
 /*
  * Which kernels bq_bitlinear_w2a8 runs for a shape on the current device (for

@@ -274,3 +274,18 @@ def test_bitconv1d_calls_reject(L):
     g = L.bq_bitconv1d_weight_pack
     assert g(FAKE, bq.BQ_F32, 32, 24, 3, FAKE, FAKE, FAKE, 1 << 24, None) == bq.BQ_ERR_INVALID_ARG  # Cg % 16
     assert g(FAKE, bq.BQ_F32, 32, 32, 3, FAKE, FAKE, None, 0, None) == bq.BQ_ERR_WORKSPACE
+
+
+def test_backward_rejects(L):
+    f = L.bq_bitlinear_w2a8_backward
+
+    def call(x=FAKE, xt=bq.BQ_BF16, d=FAKE, M=32, K=128, wp=FAKE, ws_=FAKE, N=64, eps=1e-5, dx=FAKE, dw=FAKE,
+             work=FAKE, nbytes=1 << 26):
+        return f(x, xt, d, M, K, wp, ws_, N, eps, dx, dw, work, nbytes, None)
+    assert call(K=40) == bq.BQ_ERR_INVALID_ARG
+    assert call(N=60) == bq.BQ_ERR_INVALID_ARG     # N % 8 (bf16 rows of dout, 16-byte pitch)
+    assert call(d=None) == bq.BQ_ERR_INVALID_ARG
+    assert call(d=ODD) == bq.BQ_ERR_MISALIGNED
+    assert call(work=None) == bq.BQ_ERR_WORKSPACE
+    assert call(M=0) == bq.BQ_OK
+    assert bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8_BACKWARD, 32, 64, 128) >= 32 * 128 * 5 + 64 * 128 * 2

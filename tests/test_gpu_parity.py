@@ -740,3 +740,45 @@ def test_bitconv1d(B, C_in, L, C_out, KS, stride, pad, groups, xin, out, bias, a
     rel32 = (KS + 7) * 2.0 ** -24  # fp32 tap products and tap sum (scales are binary64 rounded once)
     assert_out(host(o), ref, _TORCH_OUT[out], f"bitconv1d {B}x{C_in}x{L} -> {C_out} k{KS} s{stride} p{pad} g{groups}",
                extra=extra, scale=mag, rel32=rel32)
+
+
+# ------------------------------------------------- BitLinear STE backward
+
+@pytest.mark.parametrize("M,N,K,xin", [(8, 128, 256, "f32"), (300, 520, 1024, "bf16"), (129, 264, 640, "f32"),
+                                       (1024, 2048, 512, "bf16"), (2, 64, 64, "bf16")])
+def test_bitlinear_backward(M, N, K, xin):
+    u = 2.0 ** -24
+    g = synth.rng((127, M, N, K))
+    if xin == "bf16":
+        bits, x = synth.bf16_activations(M, K, (127, M, K), outlier_frac=0.01)
+        xd = bf16_dev(bits)
+    else:
+        x = synth.normal_f32(g, (M, K))
+        xd = dev(x)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    dbits = synth.f32_to_bf16_bits(synth.normal_f32(g, (M, N)))
+    dout = synth.bf16_bits_to_f32(dbits)
+    wp, ws_ = bq.bq_weight_quant_ternary_pack(dev(w))
+    dx, dw = bq.bq_bitlinear_w2a8_backward(xd, bf16_dev(dbits), wp, ws_, 1e-5)
+    torch.cuda.synchronize()
+    rdx, rdw = oracle.bitlinear_backward(x, w, dout, 1e-5)
+    a = oracle.act_quant(x, 1e-5, want_pre=True, want_y=True)
+    t = oracle.ternary_quant(w, want_pre=True)
+    s, gam = a["act_scale"], t["gamma"]
+    ad = np.abs(dout.astype(np.float64))
+    # dw: hi + lo split of dout * s (2^-16 relative), fp32 accumulation over 2M terms
+    mag_dw = ad.T @ (np.abs(a["xq"]).astype(np.float64) * s[:, None])
+    ex_dw = ad.T @ (tie_band(a["pre"]).astype(np.float64) * s[:, None])
+    tol_dw = (2.0 ** -16 + (2 * M + 2) * u) * (mag_dw + ex_dw) + ex_dw + 1e-30
+    err = np.abs(host(dw).astype(np.float64) - rdw)
+    assert (err <= tol_dw).all(), f"dw {M}x{N}x{K}: worst {float((err - tol_dw).max()):.3e} over"
+    # dx: dy exact products, fp32 accumulation over N terms and the gamma scale,
+    # then the RMSNorm backward (binary64 reductions, one fp32 rounding)
+    mag_dy = gam * (ad @ np.abs(t["wq"]).astype(np.float64))
+    ex_dy = gam * (ad @ tie_band(t["pre"]).astype(np.float64))
+    tol_dy = (N + 2) * u * (mag_dy + ex_dy) + ex_dy
+    y = a["y"]
+    r = np.sqrt((x.astype(np.float64) ** 2).mean(axis=1) + 1e-5)[:, None]
+    tol_dx = (tol_dy + np.abs(y) * (tol_dy * np.abs(y)).mean(axis=1, keepdims=True)) / r + 2 * u * np.abs(rdx) + 1e-30
+    err = np.abs(host(dx).astype(np.float64) - rdx)
+    assert (err <= tol_dx).all(), f"dx {M}x{N}x{K}: worst {float((err - tol_dx).max()):.3e} over"
