@@ -66,8 +66,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-workloads", action="store_true", help="skip the secondary workloads")
-    p.add_argument("--workloads", default="decode,w4,prefill,tiny,batched,w4a4,layernorm,conv",
-                   help="comma list of secondary workloads: decode, w4, prefill, tiny, batched, w4a4, layernorm, conv")
+    p.add_argument("--workloads", default="decode,w4,prefill,tiny,batched,w4a4,layernorm,conv,backward",
+                   help="comma list of secondary workloads: decode, w4, prefill, tiny, batched, w4a4, layernorm, "
+                        "conv, backward")
     p.add_argument("--workload-steps", type=int, default=200)
     p.add_argument("--decode-ms", default="1,4,16", help="token counts of the BitLinear decode workload")
     p.add_argument("--w4-ms", default="1,32", help="token counts of the grouped INT4 workload")
@@ -462,6 +463,8 @@ def workloads(args, pk):
         _layernorm(res, steps, peak_int8, hbm)
     if "conv" in want:
         _conv(res, max(steps // 4, 1), peak_int8)
+    if "backward" in want:
+        _backward(res, max(steps // 8, 1), pk)
     st, detail = bq.bq_device_status()
     if st != bq.BQ_OK:
         raise RuntimeError(f"device status {detail:#x} after the workloads")
@@ -743,6 +746,37 @@ def _conv(res, steps, peak_int8):
                                        "frac_int8_peak": round(tops / peak_int8, 4),
                                        "config": "x bf16 (8, 1024, 1024), W [1024, 1024, 3] ternary, padding 1; "
                                                  "transpose, LayerNorm quant, 3 x (gather + tcgen05 GEMM), tap sum"}
+
+
+def _backward(res, steps, pk):
+    import torch
+
+    import bit_quantized_linear_rmsnorm_b200 as bq
+    import synth
+    # straight-through backward of BitLinear, M = N = K = 4096: dy and dW on the bf16 tensor cores
+    M = N = K = 4096
+    g = synth.rng(44)
+    x = torch.from_numpy(synth.f32_to_bf16_bits(synth.normal_f32(g, (M, K))).view(np.int16)).cuda().view(
+        torch.bfloat16)
+    dout = torch.from_numpy(synth.f32_to_bf16_bits(synth.normal_f32(g, (M, N))).view(np.int16)).cuda().view(
+        torch.bfloat16)
+    wp, wsc = bq.bq_weight_quant_ternary_pack(torch.from_numpy(synth.bitlinear_weight(N, K, 7)).cuda())
+    dx = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8_BACKWARD, M, N, K), dtype=torch.uint8,
+                       device="cuda")
+
+    def step(i):
+        bq.bq_bitlinear_w2a8_backward(x, dout, wp, wsc, 1e-5, dx=dx, dw=dw, workspace=work)
+
+    ms, _, _ = graph_time(step, steps, 3)
+    flops = 2.0 * 2.0 * M * N * K  # the two contractions (the hi / lo split of dW is overhead, not counted)
+    tf = flops / (ms * 1e-3) / 1e12
+    res["bitlinear_backward_4096"] = {"us_per_step": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1),
+                                      "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4),
+                                      "config": "x bf16 [4096,4096], dout bf16 [4096,4096], W 2-bit [4096,4096]; "
+                                                "act quant, operand prep, 2 x tcgen05 kind::f16 GEMM (dW with a "
+                                                "hi/lo split: 2M contraction), RMSNorm backward"}
 
 
 # ---------------------------------------------------------------------------

@@ -13,10 +13,12 @@
 // (the row's 1/sqrt(var + eps) and 127/max|y| are each taken once and
 // multiplied in, a few ulp of binary64 from dividing per element).
 //
-// One CTA per row (grid-stride over rows).  Aligned rows of up to 1024
-// 16-byte chunks are read once into registers and every pass (mean,
-// variance, max|y|, codes) works from there; other rows take the general
-// kernel, which re-reads the row from L1/L2 in each pass.  HBM-bound: one
+// Aligned rows are read once from HBM and every pass (mean and variance,
+// max|y|, codes) works from on-chip copies: at least eight rows of up to
+// 768 16-byte chunks take one warp per row with the row staged in shared
+// memory; fewer rows of up to 1024 chunks take one CTA per row, the row in
+// registers; other rows take the general kernel, which re-reads the row from
+// L1/L2 in each pass.  HBM-bound: one
 // read of x, one write of the codes; the fp64 work per element is a handful
 // of operations.
 #include <cuda_bf16.h>
@@ -218,6 +220,140 @@ __global__ void __launch_bounds__(kLnThreads)
     }
 }
 
+// One warp per row (aligned rows, K a multiple of the chunk's elements):
+// each lane copies its 16-byte chunks of the row into the warp's slice of
+// shared memory with cp.async (all in flight at once), then the passes read
+// the row from there; reductions by warp shuffles only (no block barrier),
+// eight rows in flight per CTA.  In the passes lane l owns the four
+// consecutive elements k = 4 l + 128 i, so one warp instruction reads 128
+// consecutive elements of the row, of g and of b, and writes 128 consecutive
+// codes (every access coalesced; g and b are L1-resident across rows).  The
+// first pass accumulates sum(x) and sum(x^2) in binary64 together
+// (var = E[x^2] - mu^2 loses about mu^2 / var * 2^-53 relative, far below
+// what a code decision can see); y = x * rsd - mu * rsd (one fused
+// multiply-add, then the affine one).
+__device__ __forceinline__ void quad_of(const uint8_t *rowb, int k0, const float *, float (&v)[4]) {
+    const float4 t = *reinterpret_cast<const float4 *>(rowb + 4 * k0);
+    v[0] = t.x;
+    v[1] = t.y;
+    v[2] = t.z;
+    v[3] = t.w;
+}
+__device__ __forceinline__ void quad_of(const uint8_t *rowb, int k0, const __nv_bfloat16 *, float (&v)[4]) {
+    const uint2 t = *reinterpret_cast<const uint2 *>(rowb + 2 * k0);
+    v[0] = __uint_as_float(t.x << 16);
+    v[1] = __uint_as_float(t.x & 0xffff0000u);
+    v[2] = __uint_as_float(t.y << 16);
+    v[3] = __uint_as_float(t.y & 0xffff0000u);
+}
+// p[k0 .. k0 + 3] (def where p is null); v16: p is 16-byte aligned
+__device__ __forceinline__ void affine_quad(const float *p, bool v16, int k0, float def, double (&o)[4]) {
+    if (p == nullptr) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = def;
+    } else if (v16) {
+        const float4 t = __ldg(reinterpret_cast<const float4 *>(p + k0));
+        o[0] = t.x;
+        o[1] = t.y;
+        o[2] = t.z;
+        o[3] = t.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = __ldg(p + k0 + j);
+    }
+}
+
+template <typename In>
+__global__ void __launch_bounds__(kLnThreads)
+    act_quant_ln_warp_kernel(const In *__restrict__ x, int64_t M, int64_t K, int64_t ldx, double eps,
+                             const float *__restrict__ g, const float *__restrict__ b, int8_t *__restrict__ xq,
+                             int64_t ldq, float *__restrict__ act_scale, int32_t *__restrict__ rowsum) {
+    constexpr int E = Vec16<In>::kElts;
+    extern __shared__ uint4 srows[];  // [8][nch]
+    const int lane = threadIdx.x & 31;
+    const int nch = static_cast<int>(K / E);
+    const int kk = static_cast<int>(K);
+    uint4 *row = srows + static_cast<int64_t>(threadIdx.x >> 5) * nch;
+    const uint8_t *rowb = reinterpret_cast<const uint8_t *>(row);
+    const int64_t warp = static_cast<int64_t>(blockIdx.x) * (kLnThreads / 32) + (threadIdx.x >> 5);
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kLnThreads / 32);
+    const double inv_k = 1.0 / static_cast<double>(K);
+    const bool g16 = reinterpret_cast<uintptr_t>(g) % 16 == 0;
+    const bool b16 = reinterpret_cast<uintptr_t>(b) % 16 == 0;
+    pdl_wait();  // x may come from the previous kernel; its readers of xq are done
+    pdl_launch_dependents();
+    for (int64_t m = warp; m < M; m += nwarps) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * ldx);
+        __syncwarp();  // the previous row's readers are done with the slice
+        for (int ch = lane; ch < nch; ch += 32) cp_async_16(smem_u32(row + ch), xr + ch, 16);
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncwarp();
+        double s = 0.0, s2 = 0.0;
+        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+            float v[4];
+            quad_of(rowb, k0, x, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const double d = static_cast<double>(v[e]);
+                s += d;
+                s2 = fma(d, d, s2);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        }
+        const double mu = s * inv_k;
+        const double var = fmax(s2 * inv_k - mu * mu, 0.0);
+        const double rsd = 1.0 / sqrt(var + eps);  // one division per row
+        const double nmr = -mu * rsd;
+        // y for the quad at k0: (x - mu) / sqrt(var + eps) * g + b
+        auto y_quad = [&](int k0, double (&y)[4]) {
+            float v[4];
+            quad_of(rowb, k0, x, v);
+            double gk[4], bk[4];
+            affine_quad(g, g16, k0, 1.0f, gk);
+            affine_quad(b, b16, k0, 0.0f, bk);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) y[e] = fma(fma(static_cast<double>(v[e]), rsd, nmr), gk[e], bk[e]);
+        };
+        double amax = 0.0;
+        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+            double y[4];
+            y_quad(k0, y);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) amax = fmax(amax, fabs(y[e]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const double a = fmax(amax, 1e-5);
+        const double f = 127.0 / a;
+        int isum = 0;
+        int8_t *qr = xq + m * ldq;
+        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+            double y[4];
+            y_quad(k0, y);
+            uint32_t word = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                int code = __double2int_rn(y[e] * f);  // nearest, ties to even
+                code = code < -128 ? -128 : (code > 127 ? 127 : code);
+                isum += code;
+                word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * e);
+            }
+            *reinterpret_cast<uint32_t *>(qr + k0) = word;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+        if (lane == 0) {
+            act_scale[m] = static_cast<float>(a / 127.0);
+            if (rowsum != nullptr) rowsum[m] = isum;
+        }
+    }
+}
+
 template <typename In>
 cudaError_t launch_ln_typed(const In *x, int64_t M, int64_t K, int64_t ldx, double eps, const float *g, const float *b,
                             int8_t *xq, int64_t ldq, float *act_scale, int32_t *rowsum, cudaStream_t s,
@@ -238,6 +374,21 @@ cudaError_t launch_ln_typed(const In *x, int64_t M, int64_t K, int64_t ldx, doub
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const int64_t nch = K / E;
+    const size_t wsmem = static_cast<size_t>(kLnThreads / 32) * static_cast<size_t>(nch) * 16;
+    if (vec && M >= 8 && wsmem <= 96 * 1024) {
+        // one warp per row, rows staged in shared memory
+        static SmemOptIn opt_in;
+        if (wsmem > 48 * 1024) {
+            const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(act_quant_ln_warp_kernel<In>),
+                                              wsmem);
+            if (e != cudaSuccess) return e;
+        }
+        cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>((M + 7) / 8, static_cast<int64_t>(dev.num_sms) * 8)));
+        cfg.dynamicSmemBytes = wsmem;
+        return cudaLaunchKernelEx(&cfg, act_quant_ln_warp_kernel<In>, x, M, K, ldx, eps, g, b, xq, ldq, act_scale,
+                                  rowsum);
+    }
     if (vec && cpt <= 1)
         return cudaLaunchKernelEx(&cfg, act_quant_ln_vec_kernel<In, 1>, x, M, K, ldx, eps, g, b, xq, ldq, act_scale,
                                   rowsum);

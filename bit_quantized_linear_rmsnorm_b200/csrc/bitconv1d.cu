@@ -63,64 +63,90 @@ cudaError_t transpose(const T *src, int64_t batch, int64_t R, int64_t C, T *dst,
 // lo * stride + t - pad, or zeros outside [0, L); rs[row] is that position's
 // scale (0 outside) and rc[g * rows + row] the sum of its codes over the
 // channels of group g (the offset-binary correction of that group's product).
-__global__ void tap_gather_kernel(const int8_t *__restrict__ xq, const float *__restrict__ act_scale, int64_t B,
-                                  int64_t C_in, int64_t L, int64_t L_out, int64_t stride, int64_t pad, int64_t t,
-                                  int64_t groups, int8_t *__restrict__ a, float *__restrict__ rs,
-                                  int32_t *__restrict__ rc) {
-    const int64_t rows = B * L_out, chunks = C_in / 16, Cg = C_in / groups;
-    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = tid; i < rows * chunks; i += nth) {
-        const int64_t row = i / chunks, c = i - row * chunks;
-        const int64_t b = row / L_out, lo = row - b * L_out, p = lo * stride + t - pad;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (p >= 0 && p < L) v = __ldg(reinterpret_cast<const uint4 *>(xq + (b * L + p) * C_in) + c);
-        reinterpret_cast<uint4 *>(a + row * C_in)[c] = v;
-    }
-    for (int64_t i = tid; i < rows * groups; i += nth) {
-        const int64_t g = i / rows, row = i - g * rows;
+// One warp per row; a 16-byte chunk lies inside one group (Cg % 16 == 0), its
+// code sum goes to the warp's group counters in shared memory.
+constexpr int kGatherWarps = 8;
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    tap_gather_kernel(const int8_t *__restrict__ xq, const float *__restrict__ act_scale, int64_t B, int64_t C_in,
+                      int64_t L, int64_t L_out, int64_t stride, int64_t pad, int64_t t, int64_t groups,
+                      int8_t *__restrict__ a, float *__restrict__ rs, int32_t *__restrict__ rc) {
+    extern __shared__ int gsum[];  // [kGatherWarps][groups]
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    int *mine = gsum + wib * groups;
+    const int64_t rows = B * L_out, chunks = C_in / 16, cpg = (C_in / groups) / 16;
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * kGatherWarps + wib; row < rows;
+         row += static_cast<int64_t>(gridDim.x) * kGatherWarps) {
         const int64_t b = row / L_out, lo = row - b * L_out, p = lo * stride + t - pad;
         const bool in = p >= 0 && p < L;
-        int sum = 0;
-        if (in) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(xq + (b * L + p) * C_in + g * Cg);
-            for (int64_t c = 0; c < Cg / 16; ++c) {
-                const uint4 v = __ldg(src + c);
-                sum = __dp4a(static_cast<int>(v.x), 0x01010101, sum);
-                sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
-                sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
-                sum = __dp4a(static_cast<int>(v.w), 0x01010101, sum);
-            }
+        for (int64_t gi = lane; gi < groups; gi += 32) mine[gi] = 0;
+        __syncwarp();
+        const uint4 *src = reinterpret_cast<const uint4 *>(xq + (b * L + (in ? p : 0)) * C_in);
+        uint4 *dst = reinterpret_cast<uint4 *>(a + row * C_in);
+        int lsum = 0;  // one group: this lane's part of the row sum
+        for (int64_t c = lane; c < chunks; c += 32) {
+            const uint4 v = in ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            dst[c] = v;
+            int sum = __dp4a(static_cast<int>(v.x), 0x01010101, 0);
+            sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
+            sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
+            sum = __dp4a(static_cast<int>(v.w), 0x01010101, sum);
+            if (groups == 1)
+                lsum += sum;
+            else
+                atomicAdd(mine + c / cpg, sum);
         }
-        rc[g * rows + row] = sum;
-        if (g == 0) rs[row] = in ? __ldg(act_scale + b * L + p) : 0.0f;
+        if (groups == 1) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+            if (lane == 0) mine[0] = lsum;
+        }
+        __syncwarp();
+        for (int64_t gi = lane; gi < groups; gi += 32) rc[gi * rows + row] = mine[gi];
+        if (lane == 0) rs[row] = in ? __ldg(act_scale + b * L + p) : 0.0f;
+        __syncwarp();
     }
 }
 
-// out[b, co, lo] = sum_t part[t][(b L_out + lo) * ldp + co] (+ bias[co]), through
-// 32 x 32 shared-memory tiles (reads along co, writes along lo).
+// out[b, co, lo] = sum_t part[t][(b L_out + lo) * ldp + co] (+ bias[co]), through a
+// 32 (lo) x 128 (co) shared-memory tile: 16-byte reads along co, writes along lo.
 template <typename OutT>
-__global__ void tap_sum_kernel(const float *__restrict__ part, int64_t KS, int64_t B, int64_t L_out, int64_t C_out,
-                               int64_t ldp, const float *__restrict__ bias, OutT *__restrict__ out) {
-    __shared__ float tile[32][33];
+__global__ void __launch_bounds__(256) tap_sum_kernel(const float *__restrict__ part, int64_t KS, int64_t B,
+                                                      int64_t L_out, int64_t C_out, int64_t ldp,
+                                                      const float *__restrict__ bias, OutT *__restrict__ out) {
+    __shared__ float tile[32][129];
     const int64_t b = blockIdx.z;
-    const int64_t l0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+    const int64_t l0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 128;
     const int64_t tap_stride = B * L_out * ldp;
-    for (int i = threadIdx.y; i < 32; i += 8) {
-        const int64_t lo = l0 + i, co = c0 + threadIdx.x;
-        float v = 0.0f;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+    const int64_t co = c0 + 4 * tx;
+    for (int i = ty; i < 32; i += 8) {
+        const int64_t lo = l0 + i;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (lo < L_out && co < C_out) {
             const float *p = part + (b * L_out + lo) * ldp + co;
-            for (int64_t t = 0; t < KS; ++t) v = __fadd_rn(v, p[t * tap_stride]);
-            if (bias != nullptr) v = __fadd_rn(v, __ldg(bias + co));
+            if (co + 4 <= ldp) {
+                for (int64_t t = 0; t < KS; ++t) {
+                    const float4 q = __ldcs(reinterpret_cast<const float4 *>(p + t * tap_stride));
+                    v.x = __fadd_rn(v.x, q.x);
+                    v.y = __fadd_rn(v.y, q.y);
+                    v.z = __fadd_rn(v.z, q.z);
+                    v.w = __fadd_rn(v.w, q.w);
+                }
+            }
         }
-        tile[i][threadIdx.x] = v;
+        const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float r = e[j];
+            if (bias != nullptr && co + j < C_out) r = __fadd_rn(r, __ldg(bias + co + j));
+            tile[i][4 * tx + j] = r;
+        }
     }
     __syncthreads();
-    for (int i = threadIdx.y; i < 32; i += 8) {
-        const int64_t co = c0 + i, lo = l0 + threadIdx.x;
-        if (lo < L_out && co < C_out) {
-            const float v = tile[threadIdx.x][i];
+    for (int cc = ty; cc < 128; cc += 8) {
+        const int64_t c = c0 + cc, lo = l0 + tx;
+        if (c < C_out && lo < L_out) {
+            const float v = tile[tx][cc];
             OutT o;
             if constexpr (sizeof(OutT) == 4)
                 o = v;
@@ -128,7 +154,7 @@ __global__ void tap_sum_kernel(const float *__restrict__ part, int64_t KS, int64
                 o = __float2half_rn(v);
             else
                 o = __float2bfloat16_rn(v);
-            out[(b * C_out + co) * L_out + lo] = o;
+            out[(b * C_out + c) * L_out + lo] = o;
         }
     }
 }
@@ -187,10 +213,12 @@ bq_status launch_bitconv1d(const void *x, bq_dtype xt, int64_t B, int64_t C_in, 
     float *rs = reinterpret_cast<float *>(ws + l.rs);
     int32_t *rc = reinterpret_cast<int32_t *>(ws + l.rc);  // [groups][rows]
     float *part = reinterpret_cast<float *>(ws + l.part);
-    const int ggrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((orows * (C_in / 16) + 255) / 256,
-                                                                               dev.num_sms * 8)));
+    const int ggrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((orows + kGatherWarps - 1) / kGatherWarps,
+                                                                               dev.num_sms * 16)));
+    const size_t gsmem = static_cast<size_t>(kGatherWarps) * static_cast<size_t>(groups) * 4;
     for (int64_t t = 0; t < KS; ++t) {
-        tap_gather_kernel<<<ggrid, 256, 0, s>>>(xq, act_scale, B, C_in, L, l.L_out, stride, pad, t, groups, a, rs, rc);
+        tap_gather_kernel<<<ggrid, kGatherWarps * 32, gsmem, s>>>(xq, act_scale, B, C_in, L, l.L_out, stride, pad, t,
+                                                                  groups, a, rs, rc);
         if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
         for (int64_t gr = 0; gr < groups; ++gr) {  // group gr: its channels, weight rows and output columns
             GemmArgs g;
@@ -213,20 +241,20 @@ bq_status launch_bitconv1d(const void *x, bq_dtype xt, int64_t B, int64_t C_in, 
         }
     }
     // 4. sum the taps (+ bias), transpose to (B, C_out, L_out)
-    const dim3 grid(static_cast<unsigned>((C_out + 31) / 32), static_cast<unsigned>((l.L_out + 31) / 32),
+    const dim3 grid(static_cast<unsigned>((C_out + 127) / 128), static_cast<unsigned>((l.L_out + 31) / 32),
                     static_cast<unsigned>(B));
     switch (out_dtype) {
         case BQ_F32:
-            tap_sum_kernel<float><<<grid, dim3(32, 8), 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
-                                                               static_cast<float *>(out));
+            tap_sum_kernel<float><<<grid, 256, 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
+                                                       static_cast<float *>(out));
             break;
         case BQ_F16:
-            tap_sum_kernel<__half><<<grid, dim3(32, 8), 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
-                                                                static_cast<__half *>(out));
+            tap_sum_kernel<__half><<<grid, 256, 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
+                                                        static_cast<__half *>(out));
             break;
         default:
-            tap_sum_kernel<__nv_bfloat16><<<grid, dim3(32, 8), 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
-                                                                       static_cast<__nv_bfloat16 *>(out));
+            tap_sum_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(part, KS, B, l.L_out, C_out, l.ldp, bias,
+                                                               static_cast<__nv_bfloat16 *>(out));
     }
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

@@ -53,29 +53,73 @@ __global__ void ternary_to_bf16_kernel(const uint32_t *__restrict__ wpacked, int
 
 // Operands of dW: a2 [2M][N] bf16 with rows m = hi(dout[m,:] * s[m]) and
 // M + m = lo(...) (hi = bf16(p), lo = bf16(p - hi), p the fp32 product), and
-// b2 [2M][K] bf16 = the codes xq[m,:] in rows m and M + m.
+// b2 [2M][K] bf16 = the codes xq[m,:] in rows m and M + m.  Eight elements
+// per thread and step (N % 8 == 0, K % 16 == 0): 16-byte loads and stores.
 __global__ void dw_operands_kernel(const __nv_bfloat16 *__restrict__ dout, const float *__restrict__ act_scale,
                                    const int8_t *__restrict__ xq, int64_t M, int64_t N, int64_t K,
                                    __nv_bfloat16 *__restrict__ a2, __nv_bfloat16 *__restrict__ b2) {
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t i = tid; i < M * N; i += nth) {
-        const int64_t m = i / N;
-        const float prod = __fmul_rn(__bfloat162float(dout[i]), __ldg(act_scale + m));
-        const __nv_bfloat16 hi = __float2bfloat16_rn(prod);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(prod, __bfloat162float(hi)));
-        a2[i] = hi;
-        a2[M * N + i] = lo;
+    const int64_t n8 = N / 8, k8 = K / 8;
+    for (int64_t i = tid; i < M * n8; i += nth) {
+        const int64_t m = i / n8;
+        const float sm = __ldg(act_scale + m);
+        const uint4 d = __ldcs(reinterpret_cast<const uint4 *>(dout) + i);
+        const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t h2 = 0, l2 = 0;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float prod = __fmul_rn(__uint_as_float(e ? (dw[j] & 0xffff0000u) : (dw[j] << 16)), sm);
+                const __nv_bfloat16 h = __float2bfloat16_rn(prod);
+                const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(prod, __bfloat162float(h)));
+                h2 |= static_cast<uint32_t>(__bfloat16_as_ushort(h)) << (16 * e);
+                l2 |= static_cast<uint32_t>(__bfloat16_as_ushort(l)) << (16 * e);
+            }
+            hi[j] = h2;
+            lo[j] = l2;
+        }
+        reinterpret_cast<uint4 *>(a2)[i] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        reinterpret_cast<uint4 *>(a2 + M * N)[i] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
-    for (int64_t i = tid; i < M * K; i += nth) {
-        const __nv_bfloat16 v = __float2bfloat16_rn(static_cast<float>(xq[i]));
-        b2[i] = v;
-        b2[M * K + i] = v;
+    for (int64_t i = tid; i < M * k8; i += nth) {
+        const uint2 q = __ldg(reinterpret_cast<const uint2 *>(xq) + i);
+        const uint32_t qw[2] = {q.x, q.y};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c0 = static_cast<int8_t>((qw[j >> 1] >> (16 * (j & 1))) & 0xffu);
+            const int c1 = static_cast<int8_t>((qw[j >> 1] >> (16 * (j & 1) + 8)) & 0xffu);
+            o[j] = static_cast<uint32_t>(__bfloat16_as_ushort(__int2bfloat16_rn(c0))) |
+                   (static_cast<uint32_t>(__bfloat16_as_ushort(__int2bfloat16_rn(c1))) << 16);
+        }
+        const uint4 v = make_uint4(o[0], o[1], o[2], o[3]);
+        reinterpret_cast<uint4 *>(b2)[i] = v;
+        reinterpret_cast<uint4 *>(b2 + M * K)[i] = v;
+    }
+}
+
+// 8 consecutive elements of x as floats
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
     }
 }
 
 // dx = (dy - y * mean(dy * y)) / r, y = x / r, r = sqrt(mean(x^2) + eps): one
-// CTA per row, row reductions in binary64.
+// CTA per row, row reductions in binary64, eight elements per thread and step
+// (K % 16 == 0).
 template <typename In>
 __global__ void __launch_bounds__(256) rms_backward_kernel(const In *__restrict__ x, const float *__restrict__ dy,
                                                            int64_t M, int64_t K, double eps, float *__restrict__ dx) {
@@ -85,10 +129,16 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const In *__restrict_
         const In *xr = x + m * K;
         const float *dr = dy + m * K;
         double ss = 0.0, dot = 0.0;
-        for (int64_t k = threadIdx.x; k < K; k += 256) {
-            const double xv = static_cast<double>(static_cast<float>(xr[k]));
-            ss = fma(xv, xv, ss);
-            dot = fma(static_cast<double>(dr[k]), xv, dot);
+        for (int64_t k = 8 * threadIdx.x; k < K; k += 8 * 256) {
+            float xv[8], dv[8];
+            load8(xr + k, xv);
+            load8(dr + k, dv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const double xd = static_cast<double>(xv[e]);
+                ss = fma(xd, xd, ss);
+                dot = fma(static_cast<double>(dv[e]), xd, dot);
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -112,9 +162,16 @@ __global__ void __launch_bounds__(256) rms_backward_kernel(const In *__restrict_
         // mean(dy * y) = dot / (r K); dx = (dy - x / r * mean(dy * y)) / r
         const double c = dot / (r * r * static_cast<double>(K));
         const double inv_r = 1.0 / r;
-        for (int64_t k = threadIdx.x; k < K; k += 256) {
-            const double xv = static_cast<double>(static_cast<float>(xr[k]));
-            dx[m * K + k] = static_cast<float>((static_cast<double>(dr[k]) - xv * c) * inv_r);
+        for (int64_t k = 8 * threadIdx.x; k < K; k += 8 * 256) {
+            float xv[8], dv[8], o[8];
+            load8(xr + k, xv);
+            load8(dr + k, dv);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                o[e] = static_cast<float>((static_cast<double>(dv[e]) - static_cast<double>(xv[e]) * c) * inv_r);
+            float4 *dst = reinterpret_cast<float4 *>(dx + m * K + k);
+            dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+            dst[1] = make_float4(o[4], o[5], o[6], o[7]);
         }
     }
 }
@@ -153,7 +210,7 @@ bq_status launch_bitlinear_backward(const void *x, bq_dtype xt, const void *dout
     // the forward's codes and scales, again from x
     if (launch_act_quant(x, xt, M, K, K, eps, xq, K, act_scale, nullptr, s, dev) != cudaSuccess) return BQ_ERR_CUDA;
     ternary_to_bf16_kernel<<<grid_of_items(N * K / 16, dev), 256, 0, s>>>(wpacked, N, K, wt);
-    dw_operands_kernel<<<grid_of_items(M * std::max(N, K), dev), 256, 0, s>>>(
+    dw_operands_kernel<<<grid_of_items(M * std::max(N, K) / 8, dev), 256, 0, s>>>(
         static_cast<const __nv_bfloat16 *>(dout), act_scale, xq, M, N, K, a2, b2);
     if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
     // dy [M][K] = gamma * dout [M][N] . wt [N][K]   (A K-major, B N-major)

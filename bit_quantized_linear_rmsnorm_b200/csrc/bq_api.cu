@@ -635,7 +635,8 @@ bq_status bq_bitconv1d(const void *x, bq_dtype x_dtype, int64_t B, int64_t C_in,
         eps < 0.0f || L + 2 * pad < KS)
         return BQ_ERR_INVALID_ARG;
     const int64_t Cg = C_in / groups, Cog = C_out / groups;
-    if (C_in % 16 != 0 || Cg % 16 != 0 || Cg > kMaxK || (groups > 1 && Cog % 4 != 0)) return BQ_ERR_INVALID_ARG;
+    if (C_in % 16 != 0 || Cg % 16 != 0 || Cg > kMaxK || (groups > 1 && Cog % 4 != 0) || groups > 1024)
+        return BQ_ERR_INVALID_ARG;
     if (B * L > kMaxDim || B * ((L + 2 * pad - KS) / stride + 1) > kMaxDim) return BQ_ERR_INVALID_ARG;
     if (B == 0) return BQ_OK;
     if (x == nullptr || wpacked == nullptr || w_scale == nullptr || out == nullptr) return BQ_ERR_INVALID_ARG;

@@ -78,6 +78,48 @@ __global__ void q4_act_quant_kernel(const In *__restrict__ x, int64_t M, int64_t
         for (int64_t n = tid; n < N; n += stride) col_step[n] = step_of(scale_w, per_channel ? n : 0, eps);
 }
 
+// The same for rows whose base is 16-byte aligned and K % 8 == 0: eight
+// elements (one or two 16-byte loads) per thread and step, eight codes stored
+// at once.
+template <typename In>
+__global__ void q4_act_quant_vec_kernel(const In *__restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                                        const float *__restrict__ scale_a, float eps, int8_t *__restrict__ xq,
+                                        int64_t ldq, float *__restrict__ row_step, const float *__restrict__ scale_w,
+                                        int per_channel, int64_t N, float *__restrict__ col_step) {
+    const float sa = step_of(scale_a, 0, eps);
+    const int64_t cpr = K / 8, total = M * cpr;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = tid; i < total; i += stride) {
+        const int64_t m = i / cpr, k0 = (i - m * cpr) * 8;
+        float v[8];
+        if constexpr (sizeof(In) == 2) {
+            const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(x + m * ldx + k0));
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[2 * j] = __uint_as_float(w[j] << 16);
+                v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+            }
+        } else {
+            const float4 a = __ldcs(reinterpret_cast<const float4 *>(x + m * ldx + k0));
+            const float4 b = __ldcs(reinterpret_cast<const float4 *>(x + m * ldx + k0 + 4));
+            v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+        }
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            lo |= (static_cast<uint32_t>(q4_code(v[j], sa)) & 0xffu) << (8 * j);
+            hi |= (static_cast<uint32_t>(q4_code(v[4 + j], sa)) & 0xffu) << (8 * j);
+        }
+        *reinterpret_cast<uint2 *>(xq + m * ldq + k0) = make_uint2(lo, hi);
+    }
+    if (row_step != nullptr)
+        for (int64_t m = tid; m < M; m += stride) row_step[m] = sa;
+    if (col_step != nullptr)
+        for (int64_t n = tid; n < N; n += stride) col_step[n] = step_of(scale_w, per_channel ? n : 0, eps);
+}
+
 // Up to 16 tokens: one warp per weight row at a time (grid-stride over rows),
 // lanes stride over 16-byte pieces (32 weights) of the row; the codes of all
 // tokens sit in shared memory.  Each nibble n goes to the high half of a byte,
@@ -103,6 +145,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
         int acc[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[m] = 0;
+#pragma unroll 4
         for (int64_t pc = lane; pc < pieces; pc += 32) {
             const uint4 u = __ldcs(wr + pc);
             const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
@@ -168,7 +211,7 @@ cudaError_t launch_gemv_mt(const int8_t *xq, int M, int64_t K, const uint32_t *w
         if (e != cudaSuccess) return e;
     }
     int64_t grid = (N + kGemvWarps - 1) / kGemvWarps;
-    const int64_t cap = static_cast<int64_t>(dev.num_sms) * (smem > 100 * 1024 ? 2 : 4);
+    const int64_t cap = static_cast<int64_t>(dev.num_sms) * (smem > 100 * 1024 ? 2 : smem > 24 * 1024 ? 4 : 8);
     if (grid > cap) grid = cap;
     kern<<<static_cast<unsigned>(grid), kGemvWarps * 32, smem, s>>>(xq, M, K, wpacked, row_step, col_step, bias, N,
                                                                      static_cast<OutT *>(out));
@@ -205,6 +248,20 @@ cudaError_t launch_q4_weight_pack(const void *w, bq_dtype wt, int64_t N, int64_t
 cudaError_t launch_q4_act_quant(const void *x, bq_dtype xt, int64_t M, int64_t K, int64_t ldx, const float *scale_a,
                                 float eps, int8_t *xq, int64_t ldq, float *row_step, const float *scale_w,
                                 int per_channel, int64_t N, float *col_step, cudaStream_t s, const DevInfo &dev) {
+    const bool vec = K % 8 == 0 && reinterpret_cast<uintptr_t>(x) % 16 == 0 &&
+                     (ldx * (xt == BQ_BF16 ? 2 : 4)) % 16 == 0 && reinterpret_cast<uintptr_t>(xq) % 8 == 0 &&
+                     ldq % 8 == 0;
+    if (vec) {
+        const int vgrid = grid_for(std::max<int64_t>(M * K / 8, N), dev);
+        if (xt == BQ_BF16)
+            q4_act_quant_vec_kernel<__nv_bfloat16><<<vgrid, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16 *>(x), M, K, ldx, scale_a, eps, xq, ldq, row_step, scale_w, per_channel,
+                N, col_step);
+        else
+            q4_act_quant_vec_kernel<float><<<vgrid, 256, 0, s>>>(static_cast<const float *>(x), M, K, ldx, scale_a, eps,
+                                                                 xq, ldq, row_step, scale_w, per_channel, N, col_step);
+        return cudaGetLastError();
+    }
     const int grid = grid_for(std::max<int64_t>(M * K, N), dev);
     if (xt == BQ_BF16)
         q4_act_quant_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), M, K, ldx,

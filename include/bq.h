@@ -371,8 +371,9 @@ bq_status bq_linear_w4a4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, 
  * rounded up to 64; per tap the 2-bit layout of bq_weight_quant_ternary_pack
  * along the channels, rows Cgp/16 words apart) and w_scale (one fp32 on the
  * device).  workspace: bq_bitconv1d_weight_pack_workspace_bytes().
- * bq_bitconv1d: x dense (B, C_in, L), C_in % 16 == 0, Cg % 16 == 0 and, with
- * groups > 1, (C_out / groups) % 4 == 0; out dense (B, C_out, L_out).  Runs a
+ * bq_bitconv1d: x dense (B, C_in, L), C_in % 16 == 0, Cg % 16 == 0, groups
+ * <= 1024 and, with groups > 1, (C_out / groups) % 4 == 0; out dense
+ * (B, C_out, L_out).  Runs a
  * transpose to position-major rows, the binary64 LayerNorm quantization, per
  * tap a row gather and per group the tcgen05 ternary GEMM into fp32
  * partials, and a tap-sum / transpose kernel.  workspace:
