@@ -67,7 +67,10 @@ struct TcLayout {
     static constexpr uint32_t NBAR = 2 * kTcStages + 2 * kTcBufs + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag
     static constexpr uint32_t OFF_GT = OFF_MISC + 16;         // per K block: group index, zero-point shift
-    static constexpr uint32_t SMEM = OFF_GT + 8 * kTcBlocks + 1024;  // + alignment slack
+    // the scales of every step, [tile][K block][row] fp16, loaded once after the dependency wait
+    static constexpr uint32_t OFF_SC = OFF_GT + 8 * kTcBlocks;
+    static constexpr uint32_t SC_BYTES = kTcMaxTiles * kTcBlocks * kTcRows * 2;
+    static constexpr uint32_t SMEM = OFF_SC + SC_BYTES + 1024;  // + alignment slack
 };
 
 __device__ __forceinline__ int tc_digit(int v) { return ((v + 128) & 255) - 128; }
@@ -339,13 +342,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
         const int th = (warp - 8) >> 2;  // tokens 16 th .. 16 th + 15
         const int r_in = 32 * q + lane;
         const int *grp_of = reinterpret_cast<const int *>(smem + TcLayout::OFF_GT);
-        // the scale of step j is loaded during step j - 1
-        auto scale_of = [&](int j) -> uint16_t {
-            const int t = j / kTcBlocks, g = j - t * kTcBlocks, r = t * kTcRows + r_in;
-            return j < nsteps && r < rows ? __ldg(p.scales + static_cast<int64_t>(n0 + r) * G + grp_of[g])
-                                          : static_cast<uint16_t>(0);
-        };
-        uint16_t sc_next = scale_of(0);
+        // every scale of this CTA's steps into shared memory at once (one
+        // memory latency for all of them, not one per step): the two warps of
+        // a lane quarter take two tiles each
+        uint16_t *sc_tab = reinterpret_cast<uint16_t *>(smem + TcLayout::OFF_SC);
+#pragma unroll
+        for (int tt = 0; tt < kTcMaxTiles / 2; ++tt) {
+            const int t = 2 * th + tt, r = t * kTcRows + r_in;
+#pragma unroll
+            for (int g = 0; g < kTcBlocks; ++g)
+                sc_tab[(t * kTcBlocks + g) * kTcRows + r_in] =
+                    t < ntiles && r < rows ? __ldg(p.scales + static_cast<int64_t>(n0 + r) * G + grp_of[g])
+                                           : static_cast<uint16_t>(0);
+        }
+        named_bar_sync(1, 256);  // the eight epilogue warps
         float acc[16];
         for (int j = 0; j < nsteps; ++j) {
             const int t = j / kTcBlocks, g = j - t * kTcBlocks, b = j % kTcBufs;
@@ -355,8 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) w4_tc_kernel(const TcArgs p) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) acc[i] = 0.f;
             }
-            const float sc = __half2float(__ushort_as_half(sc_next));
-            sc_next = scale_of(j + 1);
+            const float sc = __half2float(__ushort_as_half(sc_tab[j * kTcRows + r_in]));
             bool ok = true;
             if (lane == 0)
                 ok = mbar_wait_spin(t_full(b), static_cast<uint32_t>(j / kTcBufs) & 1u, abort_flag, p.status,
