@@ -65,6 +65,7 @@ def lib():
             "bq_oracle_bitconv1d_from_codes": (None, [P, P, P, F64, P, I64, I64, I64, I64, I64, I64, I64, I64, P]),
             "bq_oracle_linear_w4a4_from_codes": (None, [P, P, P, P, I64, F64, P, I64, I64, I64, P]),
             "bq_oracle_s4_pack": (None, [P, I64, I64, P]),
+            "bq_oracle_linear_w4a4_backward": (None, [P, P, P, P, P, I64, F64, I64, I64, I64, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(_lib, name)
@@ -303,6 +304,26 @@ def linear_w4a4(x, w, scale_a, scale_w, eps: float, bias=None, per_channel: bool
     xq = q4_quant(x, scale_a, eps)
     wq = q4_quant(w, scale_w, eps, per_row=per_channel)
     return linear_w4a4_from_codes(xq, wq, scale_a, scale_w, eps, bias, per_channel), xq, wq
+
+
+def linear_w4a4_backward(x, w, dout, scale_a, scale_w, eps: float, per_channel: bool = False):
+    """Straight-through backward of the W4A4 forward: dict of dx f64 [M,K],
+    dw f64 [N,K], dscale_a (float) and g f64 [M,K] (the gradient reaching the
+    dequantized activations, before the range mask)."""
+    x = _c(x, np.float32)
+    w = _c(w, np.float32)
+    dout = _c(dout, np.float32)
+    M, K = x.shape
+    N = w.shape[0]
+    sa = _c(np.atleast_1d(scale_a), np.float32)
+    sw = _c(np.atleast_1d(scale_w), np.float32)
+    dx = np.empty((M, K), np.float64)
+    dw = np.empty((N, K), np.float64)
+    ds = np.zeros(1, np.float64)
+    g = np.empty((M, K), np.float64)
+    lib().bq_oracle_linear_w4a4_backward(_p(x), _p(w), _p(dout), _p(sa), _p(sw), 1 if per_channel else 0,
+                                         float(eps), M, N, K, _p(dx), _p(dw), _p(ds), _p(g))
+    return {"dx": dx, "dw": dw, "dscale_a": float(ds[0]), "g": g}
 
 
 def s4_pack(q):

@@ -22,7 +22,7 @@
  *                vyre-libs 0.7.2): module doc, QuantizedLinear4BitSpec.
  *   [Q4Linear]   "bitorch_engine.layers.qlinear.nbit.cutlass.q4_layer.
  *                Q4LinearFunction" (bitorch-engine docs): forward(x, weight,
- *                scale_a, scale_w, eps, is_train).
+ *                scale_a, scale_w, eps, is_train) and backward(output_gradient).
  *
  * Readings taken where the pages are silent (each is also listed in the
  * design notes): RMSNorm puts eps inside the square root; the activation
@@ -465,6 +465,69 @@ void bq_oracle_linear_w4a4_from_codes(const int8_t *xq, const int8_t *wq, const 
             if (bias) v += (double)bias[n];
             out[m * N + n] = v;
         }
+}
+
+/*
+ * The Q4Linear backward ([Q4Linear] backward: gradients for the input, the
+ * weight and the activation scale, "adjusted based on quantization ranges";
+ * none for scale_w and eps), read as straight-through rounding passed only
+ * inside the clamp range.  With the forward's steps s_a = max(scale_a, eps),
+ * s_w[n] = max(scale_w[n * sw_stride], eps), quotients u = x / s_a,
+ * v = w / s_w[n], codes xq = clamp(rne(u), -8, 7), wq = clamp(rne(v), -8, 7),
+ * and the dequantized operands xh = s_a * xq, wh[n,:] = s_w[n] * wq[n,:]
+ * (out = xh wh^T + bias):
+ *
+ *   g[m,k]   = sum_n dout[m,n] * wh[n,k]                (gradient reaching xh)
+ *   dx[m,k]  = g[m,k]          if -8 <= u[m,k] <= 7, else 0
+ *   dw[n,k]  = sum_m dout[m,n] * xh[m,k]   if -8 <= v[n,k] <= 7, else 0
+ *   dscale_a = sum_{m,k} g[m,k] * d xh[m,k] / d s_a,
+ *              d xh / d s_a = xq - u inside the range, xq (the bound) outside,
+ *              and dscale_a = 0 when scale_a < eps (s_a is then the constant eps).
+ *
+ * g (optional) receives g[m,k].
+ */
+void bq_oracle_linear_w4a4_backward(const float *x, const float *w, const float *dout,
+                                    const float *scale_a, const float *scale_w, int64_t sw_stride,
+                                    double eps, int64_t M, int64_t N, int64_t K, double *dx,
+                                    double *dw, double *dscale_a, double *g)
+{
+    int8_t *xq = (int8_t *)malloc((size_t)(M * K));
+    int8_t *wq = (int8_t *)malloc((size_t)(N * K));
+    double *u = (double *)malloc((size_t)(M * K) * sizeof(double));
+    double *v = (double *)malloc((size_t)(N * K) * sizeof(double));
+    double sa = (double)scale_a[0];
+    int sa_clamped = sa < eps;
+    if (sa_clamped) sa = eps;
+    bq_oracle_q4_quant(x, M, K, scale_a, 0, eps, xq, u);
+    bq_oracle_q4_quant(w, N, K, scale_w, sw_stride, eps, wq, v);
+    double ds = 0.0;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            double gk = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                double sw = (double)scale_w[n * sw_stride];
+                if (sw < eps) sw = eps;
+                gk += (double)dout[m * N + n] * (sw * (double)wq[n * K + k]);
+            }
+            if (g) g[m * K + k] = gk;
+            double um = u[m * K + k];
+            int inside = um >= -8.0 && um <= 7.0;
+            dx[m * K + k] = inside ? gk : 0.0;
+            double dxh_ds = inside ? (double)xq[m * K + k] - um : (double)xq[m * K + k];
+            ds += gk * dxh_ds;
+        }
+    *dscale_a = sa_clamped ? 0.0 : ds;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double s = 0.0;
+            for (int64_t m = 0; m < M; ++m) s += (double)dout[m * N + n] * (sa * (double)xq[m * K + k]);
+            double vn = v[n * K + k];
+            dw[n * K + k] = (vn >= -8.0 && vn <= 7.0) ? s : 0.0;
+        }
+    free(xq);
+    free(wq);
+    free(u);
+    free(v);
 }
 
 /*

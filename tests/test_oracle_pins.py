@@ -574,3 +574,61 @@ def test_bitlinear_backward_matches_autograd_of_the_ste_surrogate():
     out.backward(torch.from_numpy(dout.astype(np.float64)))
     np.testing.assert_allclose(dx, xx.grad.numpy(), rtol=1e-10, atol=1e-13)
     np.testing.assert_allclose(dw, ww.grad.numpy(), rtol=1e-10, atol=1e-13)
+
+
+# ------------------------------------------------- Q4Linear straight-through backward
+
+def test_w4a4_backward_hand_worked():
+    # x = (1.375, 5), s_a = 0.5: u = (2.75, 10), codes (3, 7 clamped); w = (0.625, -0.25), s_w = 0.25:
+    # v = (2.5, -1), codes (2, -1) (2.5 ties to even), wh = (0.5, -0.25); dout = 2:
+    # g = (1, -0.5); dx = (1, 0) (the second quotient is outside [-8, 7]);
+    # dw = 2 * xh = 2 * (1.5, 3.5) = (3, 7); dscale_a = 1 * (3 - 2.75) + (-0.5) * 7 = -3.25
+    r = oracle.linear_w4a4_backward(np.array([[1.375, 5.0]], np.float32), np.array([[0.625, -0.25]], np.float32),
+                                    np.array([[2.0]], np.float32), 0.5, 0.25, 1e-6)
+    np.testing.assert_array_equal(r["g"], [[1.0, -0.5]])
+    np.testing.assert_array_equal(r["dx"], [[1.0, 0.0]])
+    np.testing.assert_array_equal(r["dw"], [[3.0, 7.0]])
+    assert r["dscale_a"] == -3.25
+    # a weight quotient outside the range masks its weight gradient: w = 2.5 at s_w = 0.25 gives v = 10
+    r = oracle.linear_w4a4_backward(np.array([[1.375]], np.float32), np.array([[2.5]], np.float32),
+                                    np.array([[2.0]], np.float32), 0.5, 0.25, 1e-6)
+    np.testing.assert_array_equal(r["dw"], [[0.0]])
+    np.testing.assert_array_equal(r["g"], [[2.0 * 0.25 * 7]])
+
+
+def _ste_dequant(v, s):
+    # s * clamp(rne(v / s), -8, 7) in value; rounding passed straight through, the clamp's
+    # gradient taken on the unrounded quotient
+    u = v / s
+    cu = torch.clamp(u, -8.0, 7.0)
+    q = torch.clamp(torch.round(u), -8.0, 7.0)
+    return s * (cu + (q - cu).detach())
+
+
+@pytest.mark.parametrize("per_channel,scale_a", [(False, 0.15), (True, 0.15), (False, 1e-9)])
+def test_w4a4_backward_matches_autograd_of_the_ste_surrogate(per_channel, scale_a):
+    g = synth.rng((29, per_channel))
+    M, N, K = 5, 9, 40
+    eps = 1e-6
+    x = synth.normal_f32(g, (M, K))
+    w = synth.normal_f32(g, (N, K), 0.02)
+    dout = synth.normal_f32(g, (M, N))
+    sw = (np.float32(0.003) * (1 + g.random(N))).astype(np.float32) if per_channel else np.float32(0.003)
+    r = oracle.linear_w4a4_backward(x, w, dout, scale_a, sw, eps, per_channel=per_channel)
+    xx = torch.from_numpy(x.astype(np.float64)).requires_grad_()
+    ww = torch.from_numpy(w.astype(np.float64)).requires_grad_()
+    sa = torch.tensor(float(np.float32(scale_a)), dtype=torch.float64, requires_grad=True)
+    swt = torch.from_numpy(np.atleast_1d(sw).astype(np.float64))
+    s_a = torch.clamp(sa, min=eps)
+    s_w = torch.clamp(swt, min=eps)[:, None] if per_channel else torch.clamp(swt, min=eps)
+    out = _ste_dequant(xx, s_a) @ _ste_dequant(ww, s_w).T
+    out.backward(torch.from_numpy(dout.astype(np.float64)))
+    # the case must exercise both sides of the range
+    u = x.astype(np.float64) / max(float(np.float32(scale_a)), eps)
+    if scale_a > eps:
+        assert ((u < -8) | (u > 7)).any() and ((u >= -8) & (u <= 7)).any()
+    np.testing.assert_allclose(r["dx"], xx.grad.numpy(), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(r["dw"], ww.grad.numpy(), rtol=1e-12, atol=1e-14)
+    assert abs(r["dscale_a"] - float(sa.grad)) <= 1e-10 * (1 + abs(float(sa.grad)))
+    if scale_a < eps:
+        assert r["dscale_a"] == 0.0
