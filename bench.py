@@ -777,6 +777,28 @@ def _backward(res, steps, pk):
                                       "config": "x bf16 [4096,4096], dout bf16 [4096,4096], W 2-bit [4096,4096]; "
                                                 "act quant, operand prep, 2 x tcgen05 kind::f16 GEMM (dW with a "
                                                 "hi/lo split: 2M contraction), RMSNorm backward"}
+    del dx, dw, work
+
+    # straight-through backward of the 4-bit activation / weight linear, one weight step, M = N = K = 4096
+    wf = torch.from_numpy(synth.normal_f32(g, (N, K), 0.02)).cuda()
+    sa = torch.tensor([0.27], dtype=torch.float32, device="cuda")
+    sw = torch.tensor([0.006], dtype=torch.float32, device="cuda")
+    dx = torch.empty((M, K), dtype=torch.float32, device="cuda")
+    dw = torch.empty((N, K), dtype=torch.float32, device="cuda")
+    ds = torch.empty(1, dtype=torch.float32, device="cuda")
+    work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4A4_BACKWARD, M, N, K), dtype=torch.uint8,
+                       device="cuda")
+
+    def step4(i):
+        bq.bq_linear_w4a4_backward(x, wf, dout, sa, sw, 1e-6, dx=dx, dw=dw, dscale_a=ds, workspace=work)
+
+    ms, _, _ = graph_time(step4, steps, 3)
+    tf = flops / (ms * 1e-3) / 1e12
+    res["w4a4_backward_4096"] = {"us_per_step": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1),
+                                 "frac_bf16_peak": round(tf / pk["bf16_tflops"], 4),
+                                 "config": "x bf16 [4096,4096], W fp32 [4096,4096] (4-bit codes, one step), dout bf16 "
+                                           "[4096,4096]; codes, 2 x tcgen05 kind::f16 GEMM, range masks, binary64 "
+                                           "dscale_a"}
 
 
 # ---------------------------------------------------------------------------

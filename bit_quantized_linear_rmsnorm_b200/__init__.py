@@ -23,14 +23,15 @@ BQ_F32, BQ_BF16, BQ_F16 = 0, 1, 2
 BQ_W_NK, BQ_W_KN = 0, 1
 (BQ_OP_ACT_QUANT_INT8, BQ_OP_WEIGHT_QUANT_TERNARY_PACK, BQ_OP_WEIGHT_PACK_INT4_GROUPED,
  BQ_OP_GEMM_I8_PERTOKEN, BQ_OP_BITLINEAR_W2A8, BQ_OP_LINEAR_W4_GROUPED, BQ_OP_LINEAR_W4A4,
- BQ_OP_BITLINEAR_W2A8_BACKWARD) = range(8)
+ BQ_OP_BITLINEAR_W2A8_BACKWARD, BQ_OP_LINEAR_W4A4_BACKWARD) = range(9)
 
 EXPORTED = [
     "bq_act_quant_int8", "bq_weight_quant_ternary_pack", "bq_weight_pack_int4_grouped",
     "bq_gemm_i8_pertoken", "bq_gemm_i8_pertoken_batched", "bq_bitlinear_w2a8", "bq_act_quant_int8_layernorm",
     "bq_bitlinear_w2a8_layernorm", "bq_weight_quant_int4_pack", "bq_act_quant_int4", "bq_linear_w4a4",
     "bq_bitconv1d_weight_pack_workspace_bytes", "bq_bitconv1d_weight_pack", "bq_bitconv1d_workspace_bytes",
-    "bq_bitconv1d", "bq_bitlinear_w2a8_backward", "bq_linear_w4_grouped", "bq_workspace_bytes",
+    "bq_bitconv1d", "bq_bitlinear_w2a8_backward", "bq_linear_w4a4_backward", "bq_linear_w4_grouped",
+    "bq_workspace_bytes",
     "bq_bitlinear_workspace_layout", "bq_status_string", "bq_device_status", "bq_version",
     "bq_bitlinear_w2a8_noalloc", "bq_bitlinear_w2a8_path", "bq_diag_gemm_withheld_arrival",
 ]
@@ -68,6 +69,7 @@ _SIGS = {
     "bq_bitconv1d_workspace_bytes": (SZ, [I64, I64, I64, I64, I64, I64, I64, I64]),
     "bq_bitconv1d": (I32, [P, I32, I64, I64, I64, P, P, P, P, I64, I64, I64, I64, I64, P, F32, I32, P, P, SZ, P]),
     "bq_bitlinear_w2a8_backward": (I32, [P, I32, P, I64, I64, P, P, I64, F32, P, P, P, SZ, P]),
+    "bq_linear_w4a4_backward": (I32, [P, I32, P, P, I64, I64, I64, P, P, I32, F32, P, P, P, P, SZ, P]),
     "bq_workspace_bytes": (SZ, [I32, I64, I64, I64, I64]),
     "bq_bitlinear_workspace_layout": (None, [I64, I64, ctypes.POINTER(SZ), ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
     "bq_status_string": (ctypes.c_char_p, [I32]),
@@ -424,3 +426,26 @@ def bq_bitlinear_w2a8_backward(x: torch.Tensor, dout: torch.Tensor, wpacked: tor
                                           _stream(stream))
     _check(st, "bq_bitlinear_w2a8_backward")
     return dx, dw
+
+
+def bq_linear_w4a4_backward(x: torch.Tensor, w: torch.Tensor, dout: torch.Tensor, scale_a: torch.Tensor,
+                            scale_w: torch.Tensor, eps: float, dx=None, dw=None, dscale_a=None, workspace=None,
+                            stream=None):
+    """Straight-through backward of the 4-bit activation / 4-bit weight linear:
+    (dx fp32 [M,K], dw fp32 [N,K], dscale_a fp32 [1])."""
+    M, K = x.shape
+    N = w.shape[0]
+    per_channel = 1 if scale_w.numel() == N and N > 1 else 0
+    if dx is None:
+        dx = torch.empty((M, K), dtype=torch.float32, device=x.device)
+    if dw is None:
+        dw = torch.empty((N, K), dtype=torch.float32, device=x.device)
+    if dscale_a is None:
+        dscale_a = torch.empty(1, dtype=torch.float32, device=x.device)
+    nbytes = bq_workspace_bytes(BQ_OP_LINEAR_W4A4_BACKWARD, M, N, K)
+    ws = _workspace(nbytes, x.device, workspace)
+    st = lib().bq_linear_w4a4_backward(_ptr(x), _DTYPE[x.dtype], _ptr(w), _ptr(dout), M, K, N, _ptr(scale_a),
+                                       _ptr(scale_w), per_channel, float(eps), _ptr(dx), _ptr(dw), _ptr(dscale_a),
+                                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check(st, "bq_linear_w4a4_backward")
+    return dx, dw, dscale_a

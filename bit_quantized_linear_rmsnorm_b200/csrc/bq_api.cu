@@ -198,6 +198,8 @@ size_t bq_workspace_bytes(bq_op op, int64_t M, int64_t N, int64_t K, int64_t gro
             return w4a4_layout(M, N, K).total;
         case BQ_OP_BITLINEAR_W2A8_BACKWARD:
             return bitlinear_bwd_layout(M, N, K).total;
+        case BQ_OP_LINEAR_W4A4_BACKWARD:
+            return w4a4_bwd_layout(M, N, K).total;
         default:
             return 0;
     }
@@ -659,7 +661,15 @@ bq_status bq_bitlinear_w2a8_backward(const void *x, bq_dtype x_dtype, const void
     if (!act_dtype_ok(x_dtype) || M < 0 || N < 0 || K < 1 || K % 16 != 0 || N % 8 != 0 || K > kMaxK ||
         M > kMaxDim / 2 || N > kMaxDim || !std::isfinite(eps) || eps < 0.0f)
         return BQ_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return BQ_OK;
+    if (M == 0 || N == 0) {  // the gradients that exist are zero
+        if ((M > 0 && dx == nullptr) || (N > 0 && dw == nullptr)) return BQ_ERR_INVALID_ARG;
+        const cudaStream_t s = static_cast<cudaStream_t>(stream);
+        if (M > 0 && cudaMemsetAsync(dx, 0, static_cast<size_t>(M) * static_cast<size_t>(K) * 4, s) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        if (N > 0 && cudaMemsetAsync(dw, 0, static_cast<size_t>(N) * static_cast<size_t>(K) * 4, s) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        return BQ_OK;
+    }
     if (x == nullptr || dout == nullptr || wpacked == nullptr || w_scale == nullptr || dx == nullptr || dw == nullptr)
         return BQ_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(dout, 16) || !aligned(wpacked, 16) || !aligned(w_scale, 4) || !aligned(dx, 16) ||
@@ -673,6 +683,40 @@ bq_status bq_bitlinear_w2a8_backward(const void *x, bq_dtype x_dtype, const void
     if (st != BQ_OK) return st;
     return launch_bitlinear_backward(x, x_dtype, dout, M, K, wpacked, w_scale, N, eps, dx, dw, workspace,
                                      static_cast<cudaStream_t>(stream), dev);
+}
+
+bq_status bq_linear_w4a4_backward(const void *x, bq_dtype x_dtype, const float *w, const void *dout, int64_t M,
+                                  int64_t K, int64_t N, const float *scale_a, const float *scale_w,
+                                  int scale_w_per_channel, float eps, float *dx, float *dw, float *dscale_a,
+                                  void *workspace, size_t workspace_bytes, bq_stream_t stream) {
+    if (!act_dtype_ok(x_dtype) || M < 0 || N < 0 || K < 1 || K % 16 != 0 || N % 8 != 0 || K > kMaxK ||
+        M > kMaxDim || N > kMaxDim / 2 || !std::isfinite(eps) || eps <= 0.0f ||
+        (scale_w_per_channel != 0 && scale_w_per_channel != 1))
+        return BQ_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) {  // the gradients are zero
+        if ((M > 0 && dx == nullptr) || (N > 0 && dw == nullptr) || dscale_a == nullptr) return BQ_ERR_INVALID_ARG;
+        const cudaStream_t s = static_cast<cudaStream_t>(stream);
+        if (M > 0 && cudaMemsetAsync(dx, 0, static_cast<size_t>(M) * static_cast<size_t>(K) * 4, s) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        if (N > 0 && cudaMemsetAsync(dw, 0, static_cast<size_t>(N) * static_cast<size_t>(K) * 4, s) != cudaSuccess)
+            return BQ_ERR_CUDA;
+        if (cudaMemsetAsync(dscale_a, 0, 4, s) != cudaSuccess) return BQ_ERR_CUDA;
+        return BQ_OK;
+    }
+    if (x == nullptr || w == nullptr || dout == nullptr || scale_a == nullptr || scale_w == nullptr || dx == nullptr ||
+        dw == nullptr || dscale_a == nullptr)
+        return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(dout, 16) || !aligned(scale_a, 4) || !aligned(scale_w, 4) ||
+        !aligned(dx, 16) || !aligned(dw, 16) || !aligned(dscale_a, 4))
+        return BQ_ERR_MISALIGNED;
+    const size_t need = w4a4_bwd_layout(M, N, K).total;
+    if (workspace == nullptr || workspace_bytes < need) return BQ_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BQ_ERR_MISALIGNED;
+    DevInfo dev;
+    const bq_status st = current_device(&dev);
+    if (st != BQ_OK) return st;
+    return launch_w4a4_backward(x, x_dtype, w, dout, M, K, N, scale_a, scale_w, scale_w_per_channel, eps, dx, dw,
+                                dscale_a, workspace, static_cast<cudaStream_t>(stream), dev);
 }
 
 bq_status bq_linear_w4_grouped(const float *x, int64_t M, int64_t K, const uint32_t *qweight,

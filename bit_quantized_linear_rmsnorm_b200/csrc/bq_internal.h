@@ -178,6 +178,18 @@ struct Bf16Args {
 };
 bq_status launch_gemm_bf16(const Bf16Args &g, cudaStream_t s, const DevInfo &dev);
 
+// Straight-through backward of the W4A4 linear (w4a4.cu): workspace layout
+// (epilogue steps, bf16 codes of x and of w (twice), the per-channel dout
+// operand, g, the dscale_a partials) and the launch.
+struct W4a4BwdLayout {
+    size_t steps, xq, wq, a2, g, part, total;
+};
+W4a4BwdLayout w4a4_bwd_layout(int64_t M, int64_t N, int64_t K);
+bq_status launch_w4a4_backward(const void *x, bq_dtype xt, const float *w, const void *dout, int64_t M, int64_t K,
+                               int64_t N, const float *scale_a, const float *scale_w, int per_channel, float eps,
+                               float *dx, float *dw, float *dscale_a, void *workspace, cudaStream_t s,
+                               const DevInfo &dev);
+
 // Straight-through backward of BitLinear (bitlinear_bwd.cu): workspace layout
 // (xq, act_scale, bf16 ternary weights, the dW operands, dy) and the launch.
 struct BwdLayout {

@@ -227,6 +227,175 @@ cudaError_t launch_gemv_out(const int8_t *xq, int M, int64_t K, const uint32_t *
     return launch_gemv_mt<16, OutT>(xq, M, K, wpacked, row_step, col_step, bias, N, out, s, dev);
 }
 
+// ---------------------------------------------------------------------------
+// Straight-through backward (gradients for x, w and scale_a; none for scale_w
+// and eps): the reading of Q4LinearFunction.backward ("adjusts gradients
+// based on quantization ranges").  With the forward's quotients u = x / s_a
+// and v = w / s_w[n]:
+//   g  = dout . wh,  wh[n,:] = s_w[n] * wq[n,:]     (bf16 tensor cores)
+//   dx = g where -8 <= u <= 7, else 0
+//   dw = s_a * (dout^T . xq) where -8 <= v <= 7, else 0
+//   dscale_a = sum g * (inside ? xq - u : xq); 0 when scale_a < eps
+// The codes are exact in bf16.  Per-channel weight steps run along the
+// contraction of g, so they are folded into dout as hi + lo bf16 parts
+// stacked along it (2N), each pair carrying the fp32 product to 16
+// significant bits; one step for all weights is applied in the epilogue.
+// ---------------------------------------------------------------------------
+constexpr int kBwdPartMax = 1024;  // CTAs of the dx kernel = binary64 partials of dscale_a
+
+__device__ __forceinline__ void load8v(const float *p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(p)), b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    v[0] = a.x;
+    v[1] = a.y;
+    v[2] = a.z;
+    v[3] = a.w;
+    v[4] = b.x;
+    v[5] = b.y;
+    v[6] = b.z;
+    v[7] = b.w;
+}
+__device__ __forceinline__ void load8v(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
+}
+
+// the steps the GEMM epilogues multiply by: max(scale_a, eps), max(scale_w[0], eps)
+__global__ void w4a4_bwd_steps_kernel(const float *__restrict__ scale_a, const float *__restrict__ scale_w, float eps,
+                                      float *__restrict__ steps) {
+    steps[0] = fmaxf(__ldg(scale_a), eps);
+    steps[1] = fmaxf(__ldg(scale_w), eps);
+}
+
+// codes clamp(rne(v / s_r), -8, 7) of v [rows][cols] as bf16, s_r = max(scale[r * stride], eps),
+// eight per thread (cols % 8 == 0); copies == 2 writes the matrix a second time below itself
+template <typename In>
+__global__ void q4_codes_bf16_kernel(const In *__restrict__ v, int64_t rows, int64_t cols,
+                                     const float *__restrict__ scale, int64_t stride, float eps,
+                                     __nv_bfloat16 *__restrict__ out, int copies) {
+    const int64_t c8 = cols / 8, total = rows * c8;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / c8;
+        const float st = fmaxf(__ldg(scale + r * stride), eps);
+        float e[8];
+        load8v(v + i * 8, e);
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            o[j] = bf16x2_bits(static_cast<float>(q4_code(e[2 * j], st)), static_cast<float>(q4_code(e[2 * j + 1], st)));
+        const uint4 val = make_uint4(o[0], o[1], o[2], o[3]);
+        reinterpret_cast<uint4 *>(out)[i] = val;
+        if (copies > 1) reinterpret_cast<uint4 *>(out + rows * cols)[i] = val;
+    }
+}
+
+// per-channel weight steps folded into dout: a2 [M][2N], column n = hi(p), N + n = lo(p),
+// p = dout[m,n] * s_w[n] (fp32), hi = bf16(p), lo = bf16(p - hi); eight per thread (N % 8 == 0)
+__global__ void dout_steps_kernel(const __nv_bfloat16 *__restrict__ dout, int64_t M, int64_t N,
+                                  const float *__restrict__ scale_w, float eps, __nv_bfloat16 *__restrict__ a2) {
+    const int64_t n8 = N / 8, total = M * n8;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = i / n8, c = i - m * n8;
+        float d[8];
+        load8v(dout + i * 8, d);
+        float hi[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float p = __fmul_rn(d[j], fmaxf(__ldg(scale_w + c * 8 + j), eps));
+            hi[j] = __bfloat162float(__float2bfloat16_rn(p));
+            lo[j] = __fsub_rn(p, hi[j]);
+        }
+        uint4 *row = reinterpret_cast<uint4 *>(a2 + m * 2 * N);
+        row[c] = make_uint4(bf16x2_bits(hi[0], hi[1]), bf16x2_bits(hi[2], hi[3]), bf16x2_bits(hi[4], hi[5]),
+                            bf16x2_bits(hi[6], hi[7]));
+        row[n8 + c] = make_uint4(bf16x2_bits(lo[0], lo[1]), bf16x2_bits(lo[2], lo[3]), bf16x2_bits(lo[4], lo[5]),
+                                 bf16x2_bits(lo[6], lo[7]));
+    }
+}
+
+// dx = g inside the range, 0 outside; this CTA's binary64 sum of
+// g * (inside ? q - u : q) into part[blockIdx.x] (q - u is exact in fp32:
+// an integer minus a quotient within half a unit of it)
+template <typename In>
+__global__ void __launch_bounds__(256) w4a4_dx_kernel(const In *__restrict__ x, const float *__restrict__ g,
+                                                     int64_t M, int64_t K, const float *__restrict__ steps,
+                                                     float *__restrict__ dx, double *__restrict__ part) {
+    __shared__ double red[8];
+    const float sa = steps[0];
+    const int64_t total = M * K / 8;
+    double acc = 0.0;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        float e[8], gv[8], o[8];
+        load8v(x + i * 8, e);
+        load8v(g + i * 8, gv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float u = __fdiv_rn(e[j], sa);  // the forward's quotient
+            const float q = fminf(fmaxf(rintf(u), -8.0f), 7.0f);
+            const bool in = u >= -8.0f && u <= 7.0f;
+            o[j] = in ? gv[j] : 0.0f;
+            acc += static_cast<double>(gv[j]) * static_cast<double>(in ? __fsub_rn(q, u) : q);
+        }
+        float4 *dst = reinterpret_cast<float4 *>(dx + i * 8);
+        dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += red[w];
+        part[blockIdx.x] = t;
+    }
+}
+
+// dscale_a = the partials summed in a fixed order (one warp), 0 when scale_a < eps
+__global__ void w4a4_dscale_kernel(const double *__restrict__ part, int n, const float *__restrict__ scale_a,
+                                   float eps, float *__restrict__ dscale) {
+    double t = 0.0;
+    for (int i = threadIdx.x; i < n; i += 32) t += part[i];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (threadIdx.x == 0) *dscale = __ldg(scale_a) < eps ? 0.0f : static_cast<float>(t);
+}
+
+// dw = 0 where the weight quotient lies outside [-8, 7]; eight per thread (K % 8 == 0)
+__global__ void w4a4_dw_mask_kernel(const float *__restrict__ w, int64_t N, int64_t K,
+                                    const float *__restrict__ scale_w, int64_t stride, float eps,
+                                    float *__restrict__ dw) {
+    const int64_t k8 = K / 8, total = N * k8;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float st = fmaxf(__ldg(scale_w + (i / k8) * stride), eps);
+        float e[8];
+        load8v(w + i * 8, e);
+        float4 *d = reinterpret_cast<float4 *>(dw + i * 8);
+        float4 a = d[0], b = d[1];
+        float o[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float u = __fdiv_rn(e[j], st);
+            if (!(u >= -8.0f && u <= 7.0f)) o[j] = 0.0f;
+        }
+        d[0] = make_float4(o[0], o[1], o[2], o[3]);
+        d[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+}
+
 int grid_for(int64_t items, const DevInfo &dev) {
     return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, dev.num_sms * 16)));
 }
@@ -285,6 +454,86 @@ cudaError_t launch_w4a4_gemv(const int8_t *xq, int64_t M, int64_t K, const uint3
         default:
             return launch_gemv_out<__nv_bfloat16>(xq, m, K, wpacked, row_step, col_step, bias, N, out, s, dev);
     }
+}
+
+W4a4BwdLayout w4a4_bwd_layout(int64_t M, int64_t N, int64_t K) {
+    auto a256 = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+    const size_t m = static_cast<size_t>(M), n = static_cast<size_t>(N), k = static_cast<size_t>(K);
+    W4a4BwdLayout l;
+    l.steps = 0;
+    l.xq = 256;
+    l.wq = l.xq + a256(m * k * 2);
+    l.a2 = l.wq + a256(2 * n * k * 2);
+    l.g = l.a2 + a256(m * 2 * n * 2);
+    l.part = l.g + a256(m * k * 4);
+    l.total = l.part + a256(static_cast<size_t>(kBwdPartMax) * 8);
+    return l;
+}
+
+bq_status launch_w4a4_backward(const void *x, bq_dtype xt, const float *w, const void *dout, int64_t M, int64_t K,
+                               int64_t N, const float *scale_a, const float *scale_w, int per_channel, float eps,
+                               float *dx, float *dw, float *dscale_a, void *workspace, cudaStream_t s,
+                               const DevInfo &dev) {
+    const W4a4BwdLayout l = w4a4_bwd_layout(M, N, K);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *steps = reinterpret_cast<float *>(ws + l.steps);
+    __nv_bfloat16 *xqb = reinterpret_cast<__nv_bfloat16 *>(ws + l.xq);
+    __nv_bfloat16 *wqb = reinterpret_cast<__nv_bfloat16 *>(ws + l.wq);
+    __nv_bfloat16 *a2 = reinterpret_cast<__nv_bfloat16 *>(ws + l.a2);
+    float *g = reinterpret_cast<float *>(ws + l.g);
+    double *part = reinterpret_cast<double *>(ws + l.part);
+    const __nv_bfloat16 *db = static_cast<const __nv_bfloat16 *>(dout);
+    w4a4_bwd_steps_kernel<<<1, 1, 0, s>>>(scale_a, scale_w, eps, steps);
+    if (xt == BQ_BF16)
+        q4_codes_bf16_kernel<__nv_bfloat16><<<grid_for(M * K / 8, dev), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), M, K, scale_a, 0, eps, xqb, 1);
+    else
+        q4_codes_bf16_kernel<float><<<grid_for(M * K / 8, dev), 256, 0, s>>>(static_cast<const float *>(x), M, K,
+                                                                             scale_a, 0, eps, xqb, 1);
+    q4_codes_bf16_kernel<float><<<grid_for(N * K / 8, dev), 256, 0, s>>>(w, N, K, scale_w, per_channel ? 1 : 0, eps,
+                                                                         wqb, per_channel ? 2 : 1);
+    if (per_channel) dout_steps_kernel<<<grid_for(M * N / 8, dev), 256, 0, s>>>(db, M, N, scale_w, eps, a2);
+    if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
+    // g [M][K] = dout [M][N] . wh [N][K]   (A K-major, B N-major)
+    Bf16Args gg;
+    gg.a = per_channel ? static_cast<const void *>(a2) : dout;
+    gg.lda = per_channel ? 2 * N : N;
+    gg.a_mn = false;
+    gg.b = wqb;
+    gg.ldb = K;
+    gg.b_mn = true;
+    gg.M = M;
+    gg.N = K;
+    gg.K = per_channel ? 2 * N : N;
+    gg.scale = per_channel ? nullptr : steps + 1;
+    gg.out = g;
+    gg.ldo = K;
+    bq_status st = launch_gemm_bf16(gg, s, dev);
+    if (st != BQ_OK) return st;
+    // dw [N][K] = s_a * dout^T [N][M] . xq [M][K]   (A M-major, B N-major)
+    Bf16Args h;
+    h.a = dout;
+    h.lda = N;
+    h.a_mn = true;
+    h.b = xqb;
+    h.ldb = K;
+    h.b_mn = true;
+    h.M = N;
+    h.N = K;
+    h.K = M;
+    h.scale = steps;
+    h.out = dw;
+    h.ldo = K;
+    st = launch_gemm_bf16(h, s, dev);
+    if (st != BQ_OK) return st;
+    const int pg = std::min(grid_for(M * K / 8, dev), kBwdPartMax);
+    if (xt == BQ_BF16)
+        w4a4_dx_kernel<__nv_bfloat16><<<pg, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(x), g, M, K, steps, dx, part);
+    else
+        w4a4_dx_kernel<float><<<pg, 256, 0, s>>>(static_cast<const float *>(x), g, M, K, steps, dx, part);
+    w4a4_dscale_kernel<<<1, 32, 0, s>>>(part, pg, scale_a, eps, dscale_a);
+    w4a4_dw_mask_kernel<<<grid_for(N * K / 8, dev), 256, 0, s>>>(w, N, K, scale_w, per_channel ? 1 : 0, eps, dw);
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
 }  // namespace bq

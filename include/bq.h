@@ -80,7 +80,8 @@ typedef enum {
     BQ_OP_BITLINEAR_W2A8 = 4,
     BQ_OP_LINEAR_W4_GROUPED = 5,
     BQ_OP_LINEAR_W4A4 = 6,
-    BQ_OP_BITLINEAR_W2A8_BACKWARD = 7
+    BQ_OP_BITLINEAR_W2A8_BACKWARD = 7,
+    BQ_OP_LINEAR_W4A4_BACKWARD = 8
 } bq_op;
 
 /*
@@ -264,7 +265,8 @@ bq_status bq_bitlinear_w2a8_layernorm(const void *x, bq_dtype x_dtype, int64_t M
  * accumulation): dout and the codes are exact in bf16, and the products
  * dout * act_scale of dw are split into two bf16 parts (16 significant bits).
  * workspace: bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8_BACKWARD, M, N, K, 0)
- * bytes, 256-byte aligned.
+ * bytes, 256-byte aligned.  M == 0 or N == 0: the gradients that exist are
+ * written as zeros (dw when M == 0, dx when N == 0) and nothing else runs.
  */
 bq_status bq_bitlinear_w2a8_backward(const void *x, bq_dtype x_dtype, const void *dout, int64_t M, int64_t K,
                                      const uint32_t *wpacked, const float *w_scale, int64_t N, float eps, float *dx,
@@ -345,6 +347,39 @@ bq_status bq_linear_w4a4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, 
                          const uint32_t *wpacked, const float *scale_w, int scale_w_per_channel, int64_t N,
                          const float *bias, float eps, bq_dtype out_dtype, void *out, void *workspace,
                          size_t workspace_bytes, bq_stream_t stream);
+
+/*
+ * Straight-through backward of the 4-bit activation and weight linear.
+ * Source: "bitorch_engine.layers.qlinear.nbit.cutlass.q4_layer.
+ * Q4LinearFunction", backward(output_gradient): gradients for the input, the
+ * weight and the activation scale, adjusted by the quantization ranges; none
+ * for scale_w and eps.  Read as rounding passed straight through inside the
+ * clamp range of the unrounded quotient.  With the forward's s_a, s_w[n],
+ * u = x / s_a, v = w / s_w[n], xq, wq (bq_linear_w4a4):
+ *
+ *   g[m,k]   = sum_n dout[m,n] * s_w[n] * wq[n,k]
+ *   dx[m,k]  = g[m,k] where -8 <= u[m,k] <= 7, else 0
+ *   dw[n,k]  = s_a * sum_m dout[m,n] * xq[m,k] where -8 <= v[n,k] <= 7, else 0
+ *   dscale_a = sum_{m,k} g[m,k] * (inside ? xq[m,k] - u[m,k] : xq[m,k]),
+ *              0 when scale_a < eps
+ *
+ * x: dense [M][K] fp32 or bf16; w: dense fp32 [N][K] (the master weights the
+ * forward quantized); dout: dense bf16 [M][N]; scale_a: one fp32, scale_w: one
+ * fp32 or [N] (scale_w_per_channel), both on the device; K % 16 == 0,
+ * N % 8 == 0, eps > 0.  dx fp32 [M][K], dw fp32 [N][K], dscale_a one fp32, all
+ * on the device (16-byte aligned; dscale_a 4-byte).  The quotients are the
+ * forward's correctly rounded fp32 divisions.  The two contractions run on the
+ * bf16 tensor cores (fp32 accumulation; codes and dout exact in bf16, per-channel
+ * steps folded into dout as two bf16 parts, 16 significant bits); dscale_a is a
+ * binary64 sum in a fixed order (deterministic).  M == 0 or N == 0: the
+ * gradients are written as zeros.  workspace:
+ * bq_workspace_bytes(BQ_OP_LINEAR_W4A4_BACKWARD, M, N, K, 0) bytes, 256-byte
+ * aligned.
+ */
+bq_status bq_linear_w4a4_backward(const void *x, bq_dtype x_dtype, const float *w, const void *dout, int64_t M,
+                                  int64_t K, int64_t N, const float *scale_a, const float *scale_w,
+                                  int scale_w_per_channel, float eps, float *dx, float *dw, float *dscale_a,
+                                  void *workspace, size_t workspace_bytes, bq_stream_t stream);
 
 /*
  * Ternary Conv1d with LayerNorm-normalised 8-bit activations.

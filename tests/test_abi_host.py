@@ -287,5 +287,27 @@ def test_backward_rejects(L):
     assert call(d=None) == bq.BQ_ERR_INVALID_ARG
     assert call(d=ODD) == bq.BQ_ERR_MISALIGNED
     assert call(work=None) == bq.BQ_ERR_WORKSPACE
-    assert call(M=0) == bq.BQ_OK
+    assert call(M=0, dw=None) == bq.BQ_ERR_INVALID_ARG  # M == 0 writes dw as zeros: it must exist
+    assert call(M=0, N=0) == bq.BQ_OK                    # no gradient to write
     assert bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8_BACKWARD, 32, 64, 128) >= 32 * 128 * 5 + 64 * 128 * 2
+
+
+def test_w4a4_backward_rejects(L):
+    f = L.bq_linear_w4a4_backward
+
+    def call(x=FAKE, xt=bq.BQ_BF16, w=FAKE, d=FAKE, M=32, K=128, N=64, sa=FAKE, sw=FAKE, pc=0, eps=1e-6, dx=FAKE,
+             dw=FAKE, ds=FAKE, work=FAKE, nbytes=1 << 26):
+        return f(x, xt, w, d, M, K, N, sa, sw, pc, eps, dx, dw, ds, work, nbytes, None)
+    assert call(K=40) == bq.BQ_ERR_INVALID_ARG     # K % 16
+    assert call(N=60) == bq.BQ_ERR_INVALID_ARG     # N % 8
+    assert call(eps=0.0) == bq.BQ_ERR_INVALID_ARG  # the steps need eps > 0
+    assert call(pc=2) == bq.BQ_ERR_INVALID_ARG
+    assert call(xt=bq.BQ_F16) == bq.BQ_ERR_INVALID_ARG
+    assert call(ds=None) == bq.BQ_ERR_INVALID_ARG
+    assert call(w=ODD) == bq.BQ_ERR_MISALIGNED
+    assert call(dx=ODD) == bq.BQ_ERR_MISALIGNED
+    assert call(work=None) == bq.BQ_ERR_WORKSPACE
+    assert call(nbytes=16) == bq.BQ_ERR_WORKSPACE
+    assert call(M=0, dw=None) == bq.BQ_ERR_INVALID_ARG
+    need = bq.bq_workspace_bytes(bq.BQ_OP_LINEAR_W4A4_BACKWARD, 32, 64, 128)
+    assert need >= 32 * 128 * (2 + 4) + 2 * 64 * 128 * 2 + 32 * 2 * 64 * 2

@@ -782,3 +782,87 @@ def test_bitlinear_backward(M, N, K, xin):
     tol_dx = (tol_dy + np.abs(y) * (tol_dy * np.abs(y)).mean(axis=1, keepdims=True)) / r + 2 * u * np.abs(rdx) + 1e-30
     err = np.abs(host(dx).astype(np.float64) - rdx)
     assert (err <= tol_dx).all(), f"dx {M}x{N}x{K}: worst {float((err - tol_dx).max()):.3e} over"
+
+
+# ------------------------------------------------- W4A4 straight-through backward
+
+def _range_band(pre):
+    """Quotients within TIE_REL (relative) of the clamp-range ends -8 and 7."""
+    return (np.abs(pre + 8.0) <= 8e-6) | (np.abs(pre - 7.0) <= 7e-6)
+
+
+@pytest.mark.parametrize("M,N,K,xin,per_channel", [(8, 64, 128, "f32", False), (300, 520, 1024, "bf16", True),
+                                                   (129, 264, 640, "f32", True), (1024, 2048, 512, "bf16", False),
+                                                   (2, 8, 64, "bf16", True)])
+def test_w4a4_backward(M, N, K, xin, per_channel):
+    u = 2.0 ** -24
+    eps = 1e-6
+    g = synth.rng((131, M, N, K))
+    x = synth.normal_f32(g, (M, K))
+    if xin == "bf16":
+        bits = synth.f32_to_bf16_bits(x)
+        x = synth.bf16_bits_to_f32(bits)
+        xd = bf16_dev(bits)
+    else:
+        xd = dev(x)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    # steps that leave some quotients outside [-8, 7] on both operands
+    sa = np.array([0.15], np.float32)
+    sw = (np.abs(w).max(axis=1) / 9.0).astype(np.float32) if per_channel else np.array([0.003], np.float32)
+    dbits = synth.f32_to_bf16_bits(synth.normal_f32(g, (M, N)))
+    dout = synth.bf16_bits_to_f32(dbits)
+    dx, dw, ds = bq.bq_linear_w4a4_backward(xd, dev(w), bf16_dev(dbits), dev(sa), dev(sw), eps)
+    torch.cuda.synchronize()
+    r = oracle.linear_w4a4_backward(x, w, dout, sa, sw, eps, per_channel=per_channel)
+    xq, xpre = oracle.q4_quant(x, sa, eps, want_pre=True)
+    wq, wpre = oracle.q4_quant(w, sw, eps, per_row=per_channel, want_pre=True)
+    s_a = float(sa[0])
+    s_w = sw.astype(np.float64) if per_channel else np.full(N, float(sw[0]))
+    ad = np.abs(dout.astype(np.float64))
+    # g: exact products accumulated in fp32 over N terms (per-channel steps: hi + lo parts, 2^-16)
+    mag_g = ad @ (np.abs(wq).astype(np.float64) * s_w[:, None])
+    ex_g = ad @ (tie_band(wpre).astype(np.float64) * s_w[:, None])
+    rel_g = (2.0 ** -16 + (2 * N + 2) * u) if per_channel else (N + 2) * u
+    tol_g = rel_g * (mag_g + ex_g) + ex_g
+    xin_band = _range_band(xpre)
+    tol_dx = tol_g + np.where(xin_band, np.abs(r["g"]) + tol_g, 0.0) + 1e-30
+    err = np.abs(host(dx).astype(np.float64) - r["dx"])
+    assert (err <= tol_dx).all(), f"dx {M}x{N}x{K}: worst {float((err - tol_dx).max()):.3e} over"
+    # dw: exact products accumulated in fp32 over M terms, then the step
+    mag_dw = s_a * (ad.T @ np.abs(xq).astype(np.float64))
+    ex_dw = s_a * (ad.T @ tie_band(xpre).astype(np.float64))
+    tol_dw = (M + 2) * u * (mag_dw + ex_dw) + ex_dw
+    tol_dw = tol_dw + np.where(_range_band(wpre), np.abs(r["dw"]) + tol_dw, 0.0) + 1e-30
+    err = np.abs(host(dw).astype(np.float64) - r["dw"])
+    assert (err <= tol_dw).all(), f"dw {M}x{N}x{K}: worst {float((err - tol_dw).max()):.3e} over"
+    # dscale_a: g's error times |term|, the fp32 quotient (2^-24 |u|) and code or mask flips times |g|
+    inside = (xpre >= -8) & (xpre <= 7)
+    term = np.where(inside, xq - xpre, xq.astype(np.float64))
+    ag = np.abs(r["g"])
+    tol_ds = float((tol_g * np.abs(term)).sum() + (ag * (u * np.abs(xpre) + tie_band(xpre) + 8.0 * xin_band)).sum()
+                   + u * abs(r["dscale_a"]) + 1e-30)
+    got = float(host(ds)[0])
+    assert abs(got - r["dscale_a"]) <= tol_ds + 2 * u * abs(r["dscale_a"]), (got, r["dscale_a"], tol_ds)
+    assert (~inside).any() and inside.any()  # both sides of the range were exercised
+
+
+def test_w4a4_backward_scale_below_eps_and_empty():
+    g = synth.rng(133)
+    M, N, K = 16, 32, 64
+    x = synth.normal_f32(g, (M, K))
+    w = synth.normal_f32(g, (N, K), 0.02)
+    dbits = synth.f32_to_bf16_bits(synth.normal_f32(g, (M, N)))
+    sa, sw = np.array([1e-9], np.float32), np.array([0.003], np.float32)
+    dx, dw, ds = bq.bq_linear_w4a4_backward(dev(x), dev(w), bf16_dev(dbits), dev(sa), dev(sw), 1e-6)
+    torch.cuda.synchronize()
+    r = oracle.linear_w4a4_backward(x, w, synth.bf16_bits_to_f32(dbits), sa, sw, 1e-6)
+    assert float(host(ds)[0]) == 0.0 and r["dscale_a"] == 0.0
+    np.testing.assert_array_equal(host(dx), r["dx"].astype(np.float32))  # every quotient is outside: all zero
+    # empty shapes write zero gradients
+    dx0 = torch.full((M, K), 7.0, device="cuda")
+    ds0 = torch.full((1,), 7.0, device="cuda")
+    bq.bq_linear_w4a4_backward(dev(x), dev(w[:0]), torch.empty((M, 0), dtype=torch.bfloat16, device="cuda"),
+                               dev(sa), dev(np.array([0.003], np.float32)), 1e-6, dx=dx0,
+                               dw=torch.empty((0, K), device="cuda"), dscale_a=ds0)
+    torch.cuda.synchronize()
+    assert float(dx0.abs().max()) == 0.0 and float(ds0[0]) == 0.0
