@@ -496,9 +496,10 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
 //               an accumulator on the leader's barrier.
 // A short last wave runs as 256 x 128 halves (each CTA 64 rows of B).
 // W2A8 (PACKED): each CTA loads A and its half of the packed 2-bit codes with
-// plain tensor copies on its own full barrier; its unpack warps (8-15)
-// expand only that half into the B stage and arrive on the leader's bready
-// barrier, which is what the MMA waits for (both CTAs' stages complete).
+// plain tensor copies on its own full barrier; its unpack warps (8-15, two
+// groups of four taking the k-blocks in turn) expand only that half into the B
+// stage and arrive on the leader's bready barrier, which is what the MMA waits
+// for (both CTAs' stages complete).
 // Every wait is bounded; both CTAs always reach the closing cluster barrier.
 // ---------------------------------------------------------------------------
 constexpr uint32_t PA_BYTES = 128 * BK;              // own 128 rows of A
@@ -506,6 +507,7 @@ constexpr uint32_t PB_BYTES = 128 * BK;              // own half of a 256-wide B
 template <int PK>
 struct PairCfg {
     static constexpr bool PACKED = PK != 0;
+    static constexpr int kUnpackGroups = 2;  // unpack warp groups, taking k-blocks in turn
     static constexpr uint32_t PP_BYTES = p_bytes<PK>(128);  // its packed form
     static constexpr int kStages = PACKED ? 5 : 6;
     static constexpr int kUnpack = 256;  // unpack threads (packed weights)
@@ -640,7 +642,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
         for (int s = 0; s < S; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 1);
-            mbar_init(bready(s), 2 * C::kUnpack / 32);  // the unpack warps of both CTAs (leader's barrier)
+            mbar_init(bready(s), 2 * (C::kUnpack / 32) / C::kUnpackGroups);  // one unpack group per CTA (leader's)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull(b), 1);
@@ -849,13 +851,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
         if (et == 0) bulk_wait_all();
     } else if (PACKED && warp >= 8) {
         // ------------------------------------------------------------ unpack own half of B (both CTAs)
+        // The unpack warps form kUnpackGroups groups that take the k-blocks in
+        // turn, each expanding a whole stage: the wait -> expand -> fence ->
+        // arrive chains of consecutive stages overlap, instead of all eight warps
+        // walking every stage's chain together.  Every warp follows the same
+        // stage / phase sequence, so the barrier parities stay in step.
+        constexpr int kGroup = C::kUnpack / C::kUnpackGroups;  // threads per group
         const int ut = threadIdx.x - 256;
-        int stage = 0;
+        const int grp = ut / kGroup, gt = ut - grp * kGroup;
+        int stage = 0, step = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int item = cl; item < count && ok; item += ncl) {
             const int chunks = (item < big ? 128 : 64) * 8;  // 16-weight chunks of this CTA's rows
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = 0; kb < nkb; ++kb, ++step) {
+                if (step % C::kUnpackGroups != grp) {  // another group's k-block
+                    if (++stage == S) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    continue;
+                }
                 bool got = true;
                 if (lane == 0) got = mbar_wait_spin(full(stage), phase, abort_flag, p.status, SITE_GEMM_UNPACK, p.wait_ns);
                 if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
@@ -864,8 +880,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
                 }
                 const uint32_t *pk = reinterpret_cast<const uint32_t *>(smem + OFF_P + stage * PP_BYTES);
                 uint8_t *bt = smem + OFF_B + stage * PB_BYTES;
-#pragma unroll 2
-                for (int idx = ut; idx < chunks; idx += C::kUnpack) {
+#pragma unroll 4
+                for (int idx = gt; idx < chunks; idx += kGroup) {
                     const int n = idx >> 3, c = idx & 7;  // weight row, 16-element chunk of the 128-K slab
                     const uint4 codes = unpack_chunk<PK>(pk + n * slab_words<PK>(), c);
                     *reinterpret_cast<uint4 *>(bt + n * 128 + ((c ^ (n & 7)) << 4)) = codes;
