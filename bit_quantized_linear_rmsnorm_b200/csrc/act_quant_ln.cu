@@ -228,10 +228,8 @@ __global__ void __launch_bounds__(kLnThreads)
 // consecutive elements k = 4 l + 128 i, so one warp instruction reads 128
 // consecutive elements of the row, of g and of b, and writes 128 consecutive
 // codes (every access coalesced; g and b are L1-resident across rows).  The
-// first pass accumulates sum(x) and sum(x^2) in binary64 together
-// (var = E[x^2] - mu^2 loses about mu^2 / var * 2^-53 relative, far below
-// what a code decision can see); y = x * rsd - mu * rsd (one fused
-// multiply-add, then the affine one).
+// first pass accumulates the sum and the sum of squares of x - x[0] in
+// binary64 together.
 __device__ __forceinline__ void quad_of(const uint8_t *rowb, int k0, const float *, float (&v)[4]) {
     const float4 t = *reinterpret_cast<const float4 *>(rowb + 4 * k0);
     v[0] = t.x;
@@ -248,6 +246,22 @@ __device__ __forceinline__ void quad_of(const uint8_t *rowb, int k0, const __nv_
 }
 // p[k0 .. k0 + 3] (def where p is null); v16: p is 16-byte aligned
 __device__ __forceinline__ void affine_quad(const float *p, bool v16, int k0, float def, double (&o)[4]) {
+    if (p == nullptr) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = def;
+    } else if (v16) {
+        const float4 t = __ldg(reinterpret_cast<const float4 *>(p + k0));
+        o[0] = t.x;
+        o[1] = t.y;
+        o[2] = t.z;
+        o[3] = t.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = __ldg(p + k0 + j);
+    }
+}
+
+__device__ __forceinline__ void affine_quad_f(const float *p, bool v16, int k0, float def, float (&o)[4]) {
     if (p == nullptr) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) o[j] = def;
@@ -282,6 +296,18 @@ __global__ void __launch_bounds__(kLnThreads)
     const bool b16 = reinterpret_cast<uintptr_t>(b) % 16 == 0;
     pdl_wait();  // x may come from the previous kernel; its readers of xq are done
     pdl_launch_dependents();
+    float gmax = 1.0f;  // max |g| over the row (the same for every row)
+    if (g != nullptr) {
+        gmax = 0.0f;
+        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+            float gk[4];
+            affine_quad_f(g, g16, k0, 1.0f, gk);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) gmax = fmaxf(gmax, fabsf(gk[e]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+    }
     for (int64_t m = warp; m < M; m += nwarps) {
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * ldx);
         __syncwarp();  // the previous row's readers are done with the slice
@@ -289,13 +315,22 @@ __global__ void __launch_bounds__(kLnThreads)
         cp_async_commit();
         cp_async_wait_all();
         __syncwarp();
+        // sums of d = x - c and d^2 with c the row's first element (x - c is
+        // exact in binary64), so the variance E[d^2] - E[d]^2 cancels only by
+        // (mu - c)^2 / var, a few units for any row, not by mu^2 / var
+        double c;
+        {
+            float v0[4];
+            quad_of(rowb, 0, x, v0);
+            c = static_cast<double>(v0[0]);
+        }
         double s = 0.0, s2 = 0.0;
         for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
             float v[4];
             quad_of(rowb, k0, x, v);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const double d = static_cast<double>(v[e]);
+                const double d = static_cast<double>(v[e]) - c;
                 s += d;
                 s2 = fma(d, d, s2);
             }
@@ -305,50 +340,105 @@ __global__ void __launch_bounds__(kLnThreads)
             s += __shfl_xor_sync(0xffffffffu, s, o);
             s2 += __shfl_xor_sync(0xffffffffu, s2, o);
         }
-        const double mu = s * inv_k;
-        const double var = fmax(s2 * inv_k - mu * mu, 0.0);
+        const double md = s * inv_k;
+        const double mu = c + md;
+        const double var = fmax(s2 * inv_k - md * md, 0.0);
         const double rsd = 1.0 / sqrt(var + eps);  // one division per row
         const double nmr = -mu * rsd;
-        // y for the quad at k0: (x - mu) / sqrt(var + eps) * g + b
-        auto y_quad = [&](int k0, double (&y)[4]) {
-            float v[4];
-            quad_of(rowb, k0, x, v);
-            double gk[4], bk[4];
-            affine_quad(g, g16, k0, 1.0f, gk);
-            affine_quad(b, b16, k0, 0.0f, bk);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) y[e] = fma(fma(static_cast<double>(v[e]), rsd, nmr), gk[e], bk[e]);
-        };
-        double amax = 0.0;
-        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
-            double y[4];
-            y_quad(k0, y);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) amax = fmax(amax, fabs(y[e]));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const double a = fmax(amax, 1e-5);
-        const double f = 127.0 / a;
-        int isum = 0;
         int8_t *qr = xq + m * ldq;
-        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
-            double y[4];
-            y_quad(k0, y);
-            uint32_t word = 0;
+        int isum = 0;
+        float scale;
+
+        // Passes 2 and 3 in fp32 with the row constants split into two fp32
+        // parts: x * rsd_h + nmr_h is formed exactly inside one FMA (the mean
+        // cancels before the only rounding) and corrected by the low parts, so
+        // y is within about three fp32 roundings of itself plus an absolute
+        // 6 u^2 |nmr| |g| (u = 2^-24).  Scaled by f = 127 / max|y|, that term
+        // stays below 4.3e-8 when |nmr| * max|g| * f < 2^21, far inside the
+        // 1e-6 band around a rounding tie (5e-7 at the smallest tie, 0.5), so
+        // the codes agree with binary64 ones outside it.  Rows that fail the
+        // check (a near-constant row far from zero, say) take the binary64 passes.
+        const float rsd_h = static_cast<float>(rsd), rsd_l = static_cast<float>(rsd - static_cast<double>(rsd_h));
+        const float nmr_h = static_cast<float>(nmr), nmr_l = static_cast<float>(nmr - static_cast<double>(nmr_h));
+        auto y_quad_f = [&](int k0, float (&y)[4]) {
+            float v[4], gk[4], bk[4];
+            quad_of(rowb, k0, x, v);
+            affine_quad_f(g, g16, k0, 1.0f, gk);
+            affine_quad_f(b, b16, k0, 0.0f, bk);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                int code = __double2int_rn(y[e] * f);  // nearest, ties to even
-                code = code < -128 ? -128 : (code > 127 ? 127 : code);
-                isum += code;
-                word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * e);
+                const float yn = __fadd_rn(__fmaf_rn(v[e], rsd_h, nmr_h), __fmaf_rn(v[e], rsd_l, nmr_l));
+                y[e] = __fmaf_rn(yn, gk[e], bk[e]);
             }
-            *reinterpret_cast<uint32_t *>(qr + k0) = word;
+        };
+        float amax_f = 0.0f;
+        for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+            float y[4];
+            y_quad_f(k0, y);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) amax_f = fmaxf(amax_f, fabsf(y[e]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax_f = fmaxf(amax_f, __shfl_xor_sync(0xffffffffu, amax_f, o));
+        const float a_f = fmaxf(amax_f, 1e-5f);
+        const float f_f = __fdiv_rn(127.0f, a_f);
+        if (fabs(nmr) * static_cast<double>(gmax) * static_cast<double>(f_f) < 2097152.0) {
+            for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+                float y[4];
+                y_quad_f(k0, y);
+                uint32_t word = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // nearest, ties to even: y * f added to 1.5 * 2^23 in one rounding
+                    int code = __float_as_int(__fmaf_rn(y[e], f_f, 12582912.0f)) - 0x4B400000;
+                    code = code < -128 ? -128 : (code > 127 ? 127 : code);
+                    isum += code;
+                    word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * e);
+                }
+                *reinterpret_cast<uint32_t *>(qr + k0) = word;
+            }
+            scale = __fdiv_rn(a_f, 127.0f);
+        } else {
+            // binary64 passes: y for the quad at k0 = (x - mu) / sqrt(var + eps) * g + b
+            auto y_quad = [&](int k0, double (&y)[4]) {
+                float v[4];
+                quad_of(rowb, k0, x, v);
+                double gk[4], bk[4];
+                affine_quad(g, g16, k0, 1.0f, gk);
+                affine_quad(b, b16, k0, 0.0f, bk);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) y[e] = fma(fma(static_cast<double>(v[e]), rsd, nmr), gk[e], bk[e]);
+            };
+            double amax = 0.0;
+            for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+                double y[4];
+                y_quad(k0, y);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) amax = fmax(amax, fabs(y[e]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmax(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const double a = fmax(amax, 1e-5);
+            const double f = 127.0 / a;
+            for (int k0 = 4 * lane; k0 < kk; k0 += 128) {
+                double y[4];
+                y_quad(k0, y);
+                uint32_t word = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int code = __double2int_rn(y[e] * f);  // nearest, ties to even
+                    code = code < -128 ? -128 : (code > 127 ? 127 : code);
+                    isum += code;
+                    word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * e);
+                }
+                *reinterpret_cast<uint32_t *>(qr + k0) = word;
+            }
+            scale = static_cast<float>(a / 127.0);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
         if (lane == 0) {
-            act_scale[m] = static_cast<float>(a / 127.0);
+            act_scale[m] = scale;
             if (rowsum != nullptr) rowsum[m] = isum;
         }
     }

@@ -579,6 +579,31 @@ def test_act_quant_layernorm(M, K, dtype, affine):
     np.testing.assert_array_equal(host(rs), g_xq.astype(np.int64).sum(axis=1))
 
 
+@pytest.mark.parametrize("affine", [False, True])
+def test_act_quant_layernorm_degenerate_rows_many(affine):
+    # sixteen rows (the warp-per-row kernel): rows whose mean is far from zero relative to their
+    # spread take its binary64 passes, ordinary rows its fp32 passes; all are compared alike
+    M, K = 16, 512
+    g = synth.rng((123, affine))
+    x = synth.normal_f32(g, (M, K))
+    x[0] = 1e5                                                       # constant, large
+    x[1] = 3.0                                                       # constant, small
+    x[2] = np.float32(1e4) + np.float32(1e-3) * synth.normal_f32(g, (K,))  # tiny spread, large offset
+    x[3] = np.float32(-250.0) + synth.normal_f32(g, (K,))            # offset 250 sigma
+    x[4] = 0.0
+    x[4, 9] = -7.0                                                   # one-hot
+    lw, lb = _ln_params(g, K, affine)
+    xq, sc, rs = bq.bq_act_quant_int8_layernorm(dev(x), 1e-5, None if lw is None else dev(lw),
+                                                None if lb is None else dev(lb))
+    torch.cuda.synchronize()
+    ref = oracle.act_quant_layernorm(x, 1e-5, lw, lb, want_pre=True)
+    assert_codes(host(xq), ref["xq"], ref["pre"], f"layernorm degenerate rows affine={affine}")
+    np.testing.assert_allclose(host(sc), ref["act_scale"], rtol=1e-5)
+    np.testing.assert_array_equal(host(rs), host(xq).astype(np.int64).sum(axis=1))
+    if not affine:
+        assert np.all(host(xq)[0] == 0) and np.all(host(xq)[1] == 0)
+
+
 def test_act_quant_layernorm_special_rows():
     K = 512
     x = synth.normal_f32(synth.rng(122), (4, K))
