@@ -5,22 +5,24 @@
 //   mu = mean(x), var = mean((x - mu)^2), y = (x - mu) / sqrt(var + eps) * g + b,
 //   a = max(max|y|, 1e-5), xq = clamp(rne(y * 127 / a), -128, 127), act_scale = a / 127.
 //
-// The arithmetic is binary64.  Subtracting the mean cancels: in fp32 the
+// Subtracting the mean cancels: with the mean rounded to fp32 first, the
 // pre-rounding value of a code near +-0.5 would move by ~1e-5 (the mean's own
 // rounding, scaled by 127 / max|y|), far more than the 1e-6 relative band in
-// which a code may round either way, so codes would not be reproducible.  In
-// binary64 every pre-rounding value is within a few 2^-53 of the exact one
-// (the row's 1/sqrt(var + eps) and 127/max|y| are each taken once and
-// multiplied in, a few ulp of binary64 from dividing per element).
+// which a code may round either way.  So the mean and variance are taken in
+// binary64, and y is formed either in binary64 or, in the warp-per-row kernel,
+// in fp32 with the row constants 1/sqrt(var + eps) and -mean/sqrt(var + eps)
+// split into two fp32 parts: the mean then cancels exactly inside one fused
+// multiply-add before its only rounding, and y stays within a few fp32
+// roundings of itself (the bound and the per-row check that sends other rows
+// to binary64 are at the kernel).  Either way every pre-rounding value is well
+// inside the tie band of the exact one.
 //
 // Aligned rows are read once from HBM and every pass (mean and variance,
 // max|y|, codes) works from on-chip copies: at least eight rows of up to
 // 768 16-byte chunks take one warp per row with the row staged in shared
 // memory; fewer rows of up to 1024 chunks take one CTA per row, the row in
 // registers; other rows take the general kernel, which re-reads the row from
-// L1/L2 in each pass.  HBM-bound: one
-// read of x, one write of the codes; the fp64 work per element is a handful
-// of operations.
+// L1/L2 in each pass.  HBM-bound: one read of x, one write of the codes.
 #include <cuda_bf16.h>
 
 #include <algorithm>
