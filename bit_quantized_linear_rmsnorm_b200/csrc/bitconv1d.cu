@@ -32,30 +32,94 @@
 namespace bq {
 namespace {
 
-// 32 x 32 tiles: src [batch][R][C] -> dst [batch][C][R] (element type T).
+// 64 x 64 tiles: src [batch][R][C] -> dst [batch][C][R] (element type T,
+// 2 or 4 bytes).  A thread loads 4 consecutive elements of a source row as
+// one vector and, after the tile is in shared memory, writes 4 consecutive
+// elements of a destination row as one vector (8 or 16 bytes per access on
+// both sides); the tile rows are padded by one element, which leaves at most
+// a 2-way bank conflict on the column reads.  Ragged or unaligned edges fall
+// back to element accesses.
 template <typename T>
-__global__ void transpose_kernel(const T *__restrict__ src, int64_t R, int64_t C, T *__restrict__ dst) {
-    __shared__ T tile[32][33];
+struct Vec4;
+template <>
+struct Vec4<float> {
+    using V = float4;
+    __device__ static void split(const V &v, float (&e)[4]) {
+        e[0] = v.x;
+        e[1] = v.y;
+        e[2] = v.z;
+        e[3] = v.w;
+    }
+    __device__ static V join(const float (&e)[4]) { return make_float4(e[0], e[1], e[2], e[3]); }
+};
+template <>
+struct Vec4<__nv_bfloat16> {
+    using V = uint2;
+    __device__ static void split(const V &v, __nv_bfloat16 (&e)[4]) {
+        e[0] = __ushort_as_bfloat16(static_cast<unsigned short>(v.x & 0xffffu));
+        e[1] = __ushort_as_bfloat16(static_cast<unsigned short>(v.x >> 16));
+        e[2] = __ushort_as_bfloat16(static_cast<unsigned short>(v.y & 0xffffu));
+        e[3] = __ushort_as_bfloat16(static_cast<unsigned short>(v.y >> 16));
+    }
+    __device__ static V join(const __nv_bfloat16 (&e)[4]) {
+        return make_uint2(static_cast<uint32_t>(__bfloat16_as_ushort(e[0])) |
+                              (static_cast<uint32_t>(__bfloat16_as_ushort(e[1])) << 16),
+                          static_cast<uint32_t>(__bfloat16_as_ushort(e[2])) |
+                              (static_cast<uint32_t>(__bfloat16_as_ushort(e[3])) << 16));
+    }
+};
+
+constexpr int kTr = 64;  // tile edge
+template <typename T>
+__global__ void __launch_bounds__(256) transpose_kernel(const T *__restrict__ src, int64_t R, int64_t C,
+                                                       T *__restrict__ dst) {
+    using V = typename Vec4<T>::V;
+    __shared__ T tile[kTr][kTr + 1];
     const int64_t b = blockIdx.z;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32, c0 = static_cast<int64_t>(blockIdx.x) * 32;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kTr, c0 = static_cast<int64_t>(blockIdx.x) * kTr;
     const T *s = src + b * R * C;
     T *d = dst + b * R * C;
-    for (int i = threadIdx.y; i < 32; i += 8) {
-        const int64_t r = r0 + i, c = c0 + threadIdx.x;
-        if (r < R && c < C) tile[i][threadIdx.x] = s[r * C + c];
+    const int q = threadIdx.x & 15, h = threadIdx.x >> 4;  // 4-element group q of a line, line h (+ 16 i)
+    const bool cvec = C % 4 == 0 && reinterpret_cast<uintptr_t>(src) % sizeof(V) == 0;
+    const bool rvec = R % 4 == 0 && reinterpret_cast<uintptr_t>(dst) % sizeof(V) == 0;
+#pragma unroll
+    for (int i = 0; i < kTr / 16; ++i) {
+        const int tr = h + 16 * i;
+        const int64_t r = r0 + tr, c = c0 + 4 * q;
+        T e[4];
+        if (r < R && cvec && c + 3 < C) {
+            Vec4<T>::split(__ldg(reinterpret_cast<const V *>(s + r * C + c)), e);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) e[j] = (r < R && c + j < C) ? s[r * C + c + j] : T{};
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tile[tr][4 * q + j] = e[j];
     }
     __syncthreads();
-    for (int i = threadIdx.y; i < 32; i += 8) {
-        const int64_t c = c0 + i, r = r0 + threadIdx.x;
-        if (r < R && c < C) d[c * R + r] = tile[threadIdx.x][i];
+#pragma unroll
+    for (int i = 0; i < kTr / 16; ++i) {
+        const int tc = h + 16 * i;
+        const int64_t c = c0 + tc, r = r0 + 4 * q;
+        if (c >= C) continue;
+        T e[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) e[j] = tile[4 * q + j][tc];
+        if (rvec && r + 3 < R) {
+            *reinterpret_cast<V *>(d + c * R + r) = Vec4<T>::join(e);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (r + j < R) d[c * R + r + j] = e[j];
+        }
     }
 }
 
 template <typename T>
 cudaError_t transpose(const T *src, int64_t batch, int64_t R, int64_t C, T *dst, cudaStream_t s) {
-    const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32),
+    const dim3 grid(static_cast<unsigned>((C + kTr - 1) / kTr), static_cast<unsigned>((R + kTr - 1) / kTr),
                     static_cast<unsigned>(batch));
-    transpose_kernel<T><<<grid, dim3(32, 8), 0, s>>>(src, R, C, dst);
+    transpose_kernel<T><<<grid, 256, 0, s>>>(src, R, C, dst);
     return cudaGetLastError();
 }
 
