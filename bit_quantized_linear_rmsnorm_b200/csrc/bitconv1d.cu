@@ -127,6 +127,8 @@ cudaError_t transpose(const T *src, int64_t batch, int64_t R, int64_t C, T *dst,
 // lo * stride + t - pad, or zeros outside [0, L); rs[row] is that position's
 // scale (0 outside) and rc[g * rows + row] the sum of its codes over the
 // channels of group g (the offset-binary correction of that group's product).
+// With a == nullptr only rs and rc are written (stride 1: the padded scale and
+// code-sum arrays, L_out = L + 2 pad rows per batch, t = 0).
 // One warp per row; a 16-byte chunk lies inside one group (Cg % 16 == 0), its
 // code sum goes to the warp's group counters in shared memory.
 constexpr int kGatherWarps = 8;
@@ -145,11 +147,11 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
         for (int64_t gi = lane; gi < groups; gi += 32) mine[gi] = 0;
         __syncwarp();
         const uint4 *src = reinterpret_cast<const uint4 *>(xq + (b * L + (in ? p : 0)) * C_in);
-        uint4 *dst = reinterpret_cast<uint4 *>(a + row * C_in);
+        uint4 *dst = a != nullptr ? reinterpret_cast<uint4 *>(a + row * C_in) : nullptr;
         int lsum = 0;  // one group: this lane's part of the row sum
         for (int64_t c = lane; c < chunks; c += 32) {
             const uint4 v = in ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            dst[c] = v;
+            if (dst != nullptr) dst[c] = v;
             int sum = __dp4a(static_cast<int>(v.x), 0x01010101, 0);
             sum = __dp4a(static_cast<int>(v.y), 0x01010101, sum);
             sum = __dp4a(static_cast<int>(v.z), 0x01010101, sum);
@@ -237,7 +239,12 @@ BitconvLayout bitconv_layout(int64_t B, int64_t C_in, int64_t L, int64_t C_out, 
     l.xq = l.xt + a256(rows * static_cast<size_t>(C_in) * 4);
     l.scale = l.xq + a256(rows * static_cast<size_t>(C_in));
     l.a = l.scale + a256(rows * 4);
-    l.rs = l.a + a256(orows * static_cast<size_t>(C_in));
+    size_t a_bytes = orows * static_cast<size_t>(C_in);  // gathered codes, or (stride 1) the padded arrays
+    if (stride == 1) {
+        const size_t lp = static_cast<size_t>(B * (L + 2 * pad));
+        a_bytes = std::max(a_bytes, a256(lp * 4) + static_cast<size_t>(groups) * lp * 4);
+    }
+    l.rs = l.a + a256(a_bytes);
     l.rc = l.rs + a256(orows * 4);
     l.part = l.rc + a256(orows * static_cast<size_t>(groups) * 4);
     l.total = l.part + a256(static_cast<size_t>(KS) * orows * static_cast<size_t>(l.ldp) * 4);
@@ -277,31 +284,72 @@ bq_status launch_bitconv1d(const void *x, bq_dtype xt, int64_t B, int64_t C_in, 
     float *rs = reinterpret_cast<float *>(ws + l.rs);
     int32_t *rc = reinterpret_cast<int32_t *>(ws + l.rc);  // [groups][rows]
     float *part = reinterpret_cast<float *>(ws + l.part);
-    const int ggrid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>((orows + kGatherWarps - 1) / kGatherWarps,
-                                                                               dev.num_sms * 16)));
     const size_t gsmem = static_cast<size_t>(kGatherWarps) * static_cast<size_t>(groups) * 4;
-    for (int64_t t = 0; t < KS; ++t) {
-        tap_gather_kernel<<<ggrid, kGatherWarps * 32, gsmem, s>>>(xq, act_scale, B, C_in, L, l.L_out, stride, pad, t,
-                                                                  groups, a, rs, rc);
+    auto gather_grid = [&](int64_t nrows) {
+        return static_cast<int>(
+            std::max<int64_t>(1, std::min<int64_t>((nrows + kGatherWarps - 1) / kGatherWarps, dev.num_sms * 16)));
+    };
+    if (stride == 1) {
+        // Tap t of output row (b, lo) reads codes row (b, lo + t - pad): the GEMM reads
+        // the codes in place as [B][L][C_in] at a row offset, the tensor copies
+        // filling rows outside [0, L) with zeros (the padding); the scale and the code
+        // sums come from per-batch arrays padded with zeros, L + 2 pad long, built once.
+        const int64_t Lp = L + 2 * pad;
+        float *rsp = reinterpret_cast<float *>(a);
+        int32_t *rcp = reinterpret_cast<int32_t *>(a + a256(static_cast<size_t>(B * Lp) * 4));  // [groups][B][Lp]
+        tap_gather_kernel<<<gather_grid(B * Lp), kGatherWarps * 32, gsmem, s>>>(xq, act_scale, B, C_in, L, Lp, 1, pad,
+                                                                               0, groups, nullptr, rsp, rcp);
         if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
-        for (int64_t gr = 0; gr < groups; ++gr) {  // group gr: its channels, weight rows and output columns
-            GemmArgs g;
-            g.a = a + gr * Cg;
-            g.lda = C_in;
-            g.b = wpacked + (t * C_out + gr * Cog) * (Cgp / 16);
-            g.ldb = Cgp / 16;
-            g.b_pack = 2;
-            g.colscale = w_scale;
-            g.rowscale = rs;
-            g.rowcorr = rc + gr * orows;
-            g.M = orows;
-            g.N = Cog;
-            g.K = Cg;
-            g.out_dtype = BQ_F32;
-            g.out = part + t * orows * l.ldp + gr * Cog;
-            g.ldo = l.ldp;
-            const bq_status st = launch_gemm_tc(g, s, dev);
-            if (st != BQ_OK) return st;
+        for (int64_t t = 0; t < KS; ++t)
+            for (int64_t gr = 0; gr < groups; ++gr) {
+                GemmArgs g;
+                g.a = xq + gr * Cg;
+                g.lda = C_in;
+                g.batch = B;
+                g.sa = L * C_in;
+                g.a_rows = L;
+                g.a_row_off = t - pad;
+                g.b = wpacked + (t * C_out + gr * Cog) * (Cgp / 16);
+                g.ldb = Cgp / 16;
+                g.b_pack = 2;
+                g.colscale = w_scale;
+                g.rowscale = rsp + t;
+                g.rowcorr = rcp + gr * B * Lp + t;
+                g.s_row = Lp;
+                g.M = l.L_out;
+                g.N = Cog;
+                g.K = Cg;
+                g.out_dtype = BQ_F32;
+                g.out = part + t * orows * l.ldp + gr * Cog;
+                g.ldo = l.ldp;
+                g.so = l.L_out * l.ldp;
+                const bq_status st = launch_gemm_tc(g, s, dev);
+                if (st != BQ_OK) return st;
+            }
+    } else {
+        for (int64_t t = 0; t < KS; ++t) {
+            tap_gather_kernel<<<gather_grid(orows), kGatherWarps * 32, gsmem, s>>>(xq, act_scale, B, C_in, L, l.L_out,
+                                                                                 stride, pad, t, groups, a, rs, rc);
+            if (cudaGetLastError() != cudaSuccess) return BQ_ERR_CUDA;
+            for (int64_t gr = 0; gr < groups; ++gr) {  // group gr: its channels, weight rows and output columns
+                GemmArgs g;
+                g.a = a + gr * Cg;
+                g.lda = C_in;
+                g.b = wpacked + (t * C_out + gr * Cog) * (Cgp / 16);
+                g.ldb = Cgp / 16;
+                g.b_pack = 2;
+                g.colscale = w_scale;
+                g.rowscale = rs;
+                g.rowcorr = rc + gr * orows;
+                g.M = orows;
+                g.N = Cog;
+                g.K = Cg;
+                g.out_dtype = BQ_F32;
+                g.out = part + t * orows * l.ldp + gr * Cog;
+                g.ldo = l.ldp;
+                const bq_status st = launch_gemm_tc(g, s, dev);
+                if (st != BQ_OK) return st;
+            }
         }
     }
     // 4. sum the taps (+ bias), transpose to (B, C_out, L_out)

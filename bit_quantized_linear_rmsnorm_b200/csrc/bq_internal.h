@@ -100,7 +100,10 @@ struct GemmArgs {
     bool a_mn = false;              // A stored [K][lda], M contiguous (ATB transposeA = true)
     int64_t batch = 1;              // independent products of the same shape
     int64_t sa = 0, sb = 0, so = 0; // elements (words for packed B) between batches of a, b, out
-    int64_t s_col = 0, s_row = 0;   // elements between batches of colscale / rowscale (0: shared)
+    int64_t s_col = 0, s_row = 0;   // elements between batches of colscale / rowscale and rowcorr (0: shared)
+    // (packed B, K-major A) rows of A per batch (0: M); output row m reads A row
+    // m + a_row_off, and rows outside [0, a_rows) read as zeros
+    int64_t a_rows = 0, a_row_off = 0;
     uint64_t wait_ns = 2000000000ull;  // limit of the kernel's bounded waits
     int withhold_kb = -1;              // failure-detection check only (single-CTA kernel)
 };

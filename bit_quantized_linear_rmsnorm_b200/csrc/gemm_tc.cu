@@ -86,7 +86,9 @@ struct GemmDev {
     const float *bias;
     int M, N, K;
     int batch;              // independent products (tile coordinate z)
-    int64_t s_col, s_row;   // colscale / rowscale elements between batches (0: shared)
+    int64_t s_col, s_row;   // colscale / rowscale (and rowcorr) elements between batches (0: shared)
+    int a_row_off;          // (packed B) A row of output row m: m + a_row_off
+    int b_shared;           // one B for all batches (batch > 1 with a zero B stride): B tiles at batch 0
     uint32_t *status;
     uint64_t wait_ns;  // limit of every bounded wait
     int withhold_kb;   // (failure-detection check only) K block of the first tile whose copies are never issued
@@ -251,8 +253,9 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
                     // failure-detection check: this stage's barrier never completes
                 } else if constexpr (PACKED) {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + P_BYTES);
-                    tma_load_3d(a_dst, &tmA, kb * BK, m0, bz, full(stage));
-                    tma_load_3d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * slab_words<PK>(), n0, bz, full(stage));
+                    tma_load_3d(a_dst, &tmA, kb * BK, m0 + p.a_row_off, bz, full(stage));
+                    tma_load_3d(sbase + C::OFF_P + stage * P_BYTES, &tmB, kb * slab_words<PK>(), n0, p.b_shared ? 0 : bz,
+                                full(stage));
                 } else {
                     mbar_arrive_expect_tx(full(stage), A_BYTES + b_bytes);
                     // A: a 128 (K) x 128 (M) box when M-major, 128 (M) x 128 (K) otherwise
@@ -262,10 +265,11 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
                         tma_load_3d(a_dst, &tmA, kb * BK, m0, bz, full(stage));
                     const uint32_t b_dst = sbase + C::OFF_B + stage * B_BYTES;
                     if constexpr (B_KN) {
-                        tma_load_3d(b_dst, &tmB, n0, kb * BK, bz, full(stage));
-                        if (!half) tma_load_3d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, bz, full(stage));
+                        tma_load_3d(b_dst, &tmB, n0, kb * BK, p.b_shared ? 0 : bz, full(stage));
+                        if (!half)
+                            tma_load_3d(b_dst + B_BYTES / 2, &tmB, n0 + 128, kb * BK, p.b_shared ? 0 : bz, full(stage));
                     } else {
-                        tma_load_3d(b_dst, half ? &tmBh : &tmB, kb * BK, n0, bz, full(stage));
+                        tma_load_3d(b_dst, half ? &tmBh : &tmB, kb * BK, n0, p.b_shared ? 0 : bz, full(stage));
                     }
                 }
                 ++issued;
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
             tc_fence_after();
             const int row = m0 + r;
             const float rs = row < p.M ? __ldg(rowscale + row) : 0.0f;
-            const int corr = (TERN && row < p.M) ? __ldg(p.rowcorr + row) : 0;
+            const int corr = (TERN && row < p.M) ? __ldg(p.rowcorr + bz * p.s_row + row) : 0;
 
 #pragma unroll 1
             for (int c32 = 0; c32 < nc32; ++c32) {
@@ -687,16 +691,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
                 if constexpr (PACKED) {  // own barrier: this CTA's unpack warps wait on it
                     const uint32_t p_bytes = half ? PP_BYTES / 2 : PP_BYTES;
                     mbar_arrive_expect_tx(full(stage), PA_BYTES + p_bytes);
-                    tma_load_3d(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
-                                bz, full(stage));
-                    tma_load_3d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * slab_words<PK>(), nb0, bz,
+                    tma_load_3d(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK,
+                                m0 + BM * static_cast<int>(rank) + p.a_row_off, bz, full(stage));
+                    tma_load_3d(sbase + OFF_P + stage * PP_BYTES, half ? &tmBh : &tmB, kb * slab_words<PK>(), nb0,
+                                p.b_shared ? 0 : bz,
                                 full(stage));
                 } else {  // the leader's barrier counts both CTAs' copies
                     if (leader) mbar_arrive_expect_tx(full(stage), 2u * (PA_BYTES + b_bytes));
                     const uint32_t lbar = cluster_addr(full(stage), 0);
                     tma_load_3d_pair(sbase + OFF_A + stage * PA_BYTES, &tmA, kb * BK, m0 + BM * static_cast<int>(rank),
                                      bz, lbar);
-                    tma_load_3d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK, nb0, bz, lbar);
+                    tma_load_3d_pair(sbase + OFF_B + stage * PB_BYTES, half ? &tmBh : &tmB, kb * BK, nb0,
+                                     p.b_shared ? 0 : bz, lbar);
                 }
                 ++issued;
                 if (++stage == S) {
@@ -794,7 +800,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
             tc_fence_after();
             const int row = mr + r;
             const float rs = row < p.M ? __ldg(rowscale + row) : 0.0f;
-            const int corr = (TERN && row < p.M) ? __ldg(p.rowcorr + row) : 0;
+            const int corr = (TERN && row < p.M) ? __ldg(p.rowcorr + bz * p.s_row + row) : 0;
 
 #pragma unroll 1
             for (int c32 = 0; c32 < nc32; ++c32) {
@@ -924,6 +930,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 3-D tiled tensor map: {inner, outer, batch} elements with row and batch
 // strides in bytes (both multiples of 16), box {box_inner, box_outer, 1}.
+// batches of the B tensor maps: one when all batches share B (zero B stride)
+uint64_t b_batches(const GemmArgs &g) { return g.batch > 1 && g.sb == 0 ? 1 : static_cast<uint64_t>(g.batch); }
+
 bool make_map(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw, uint64_t batch = 1,
               uint64_t batch_bytes = 0) {
@@ -952,6 +961,8 @@ GemmDev dev_args(const GemmArgs &g, const DevInfo &dev) {
     p.batch = static_cast<int>(g.batch);
     p.s_col = g.s_col;
     p.s_row = g.s_row;
+    p.a_row_off = static_cast<int>(g.a_row_off);
+    p.b_shared = g.batch > 1 && g.sb == 0 ? 1 : 0;
     p.status = dev.status;
     p.wait_ns = g.wait_ns;
     p.withhold_kb = g.withhold_kb;
@@ -1004,9 +1015,9 @@ bq_status dispatch_packed(const GemmArgs &g, const CUtensorMap &mA, const CUtens
         CUtensorMap mP128, mP64;
         const uint64_t words = static_cast<uint64_t>(g.K) * PK / 32;
         if (!make_map(&mP128, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, words, g.N, g.ldb * 4, slab_words<PK>(), BN / 2,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4) ||
+                      CU_TENSOR_MAP_SWIZZLE_NONE, b_batches(g), g.sb * 4) ||
             !make_map(&mP64, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, words, g.N, g.ldb * 4, slab_words<PK>(), BN / 4,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4))
+                      CU_TENSOR_MAP_SWIZZLE_NONE, b_batches(g), g.sb * 4))
             return BQ_ERR_CUDA;
         return launch_pair<PK, OutT>(g, mA, mP128, mP64, mO, s, dev);
     }
@@ -1024,7 +1035,7 @@ bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
         // per CTA of a pair: 128-row boxes of B (half of a 256-wide tile), 64-row boxes for half tiles
         CUtensorMap mBq;
         if (!make_map(&mBq, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 4,
-                      CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sb))
+                      CU_TENSOR_MAP_SWIZZLE_128B, b_batches(g), g.sb))
             return BQ_ERR_CUDA;
         return launch_pair<0, OutT>(g, mA, mBh, mBq, mO, s, dev);
     }
@@ -1049,25 +1060,25 @@ bq_status launch_gemm_tc(const GemmArgs &g, cudaStream_t s, const DevInfo &dev) 
     CUtensorMap mA, mB, mBh, mO;
     const bool okA = g.a_mn ? make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.M, g.K, g.lda, BM, BK,
                                        CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sa)
-                            : make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.K, g.M, g.lda, BK, BM,
-                                       CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sa);
+                            : make_map(&mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a, g.K, g.a_rows > 0 ? g.a_rows : g.M,
+                                       g.lda, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, nb, g.sa);
     if (!okA) return BQ_ERR_CUDA;
     bool okB;
     if (g.b_pack != 0)
         okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b, static_cast<uint64_t>(g.K) * g.b_pack / 32, g.N,
-                       g.ldb * 4, BK * g.b_pack / 32, BN, CU_TENSOR_MAP_SWIZZLE_NONE, nb, g.sb * 4);
+                       g.ldb * 4, BK * g.b_pack / 32, BN, CU_TENSOR_MAP_SWIZZLE_NONE, b_batches(g), g.sb * 4);
     else if (g.b_layout == BQ_W_KN)
         okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.N, g.K, g.ldb, 128, BK, CU_TENSOR_MAP_SWIZZLE_128B,
-                       nb, g.sb);
+                       b_batches(g), g.sb);
     else
         okB = make_map(&mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN, CU_TENSOR_MAP_SWIZZLE_128B,
-                       nb, g.sb);
+                       b_batches(g), g.sb);
     if (!okB) return BQ_ERR_CUDA;
     // K-major weights: a 128-row box too, for the half tiles of a last partial wave
     mBh = mB;
     if (g.b_pack == 0 && g.b_layout != BQ_W_KN &&
         !make_map(&mBh, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b, g.K, g.N, g.ldb, BK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B,
-                  nb, g.sb))
+                  b_batches(g), g.sb))
         return BQ_ERR_CUDA;
     CUtensorMapDataType odt = g.out_dtype == BQ_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                               : g.out_dtype == BQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16

@@ -731,6 +731,9 @@ def test_linear_w4a4(M, N, K, per_channel, bias, out, xin):
     (2, 80, 20, 40, 3, 1, 1, 1, "bf16", "bf16", False, True),       # channels re-pitched to 128
     (4, 512, 256, 512, 3, 1, 1, 1, "bf16", "bf16", True, False),     # several GEMM tiles per tap
     (2, 256, 64, 64, 1, 1, 0, 4, "bf16", "f32", False, True),
+    (2, 128, 50, 64, 3, 1, 1, 2, "bf16", "bf16", True, True),       # groups with padding at stride 1
+    (1, 64, 5, 32, 7, 1, 3, 1, "f32", "f32", False, False),          # padding wide against L
+    (2, 32, 4, 16, 6, 1, 1, 1, "f32", "bf16", False, False),         # one output position
 ])
 def test_bitconv1d(B, C_in, L, C_out, KS, stride, pad, groups, xin, out, bias, affine):
     g = synth.rng((126, B, C_in, L, C_out, KS))
