@@ -447,6 +447,11 @@ bq_status bq_bitlinear_w2a8_layernorm(const void *x, bq_dtype x_dtype, int64_t M
     if (st != BQ_OK) return st;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (decode_ln1_supported(x, M, N, K, x_dtype, dev))  // one token: normaliser fused into the weight stream
+        return from_cuda(launch_decode_ln1(x, x_dtype, K, ln_weight, ln_bias, eps, wpacked, w_scale, bias, N, out_dtype,
+                                           out, reinterpret_cast<int8_t *>(ws + l.xq),
+                                           reinterpret_cast<float *>(ws + l.scale),
+                                           reinterpret_cast<int32_t *>(ws + l.rowsum), s, dev));
     if (launch_act_quant_ln(x, x_dtype, M, K, K, ln_weight, ln_bias, eps, reinterpret_cast<int8_t *>(ws + l.xq), K,
                             reinterpret_cast<float *>(ws + l.scale), reinterpret_cast<int32_t *>(ws + l.rowsum), s,
                             dev) != cudaSuccess)

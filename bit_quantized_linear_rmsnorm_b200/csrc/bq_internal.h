@@ -137,6 +137,14 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
                                const float *w_scale, const float *bias, int64_t N, bq_dtype out_dtype, void *out,
                                int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum, cudaStream_t s,
                                const DevInfo &dev);
+// One-token BitLinear with the LayerNorm normaliser fused into the
+// weight-streaming kernel (one launch; codes, act_scale and rowsum also go to
+// the workspace, as in launch_decode_w2a8).
+bool decode_ln1_supported(const void *x, int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev);
+cudaError_t launch_decode_ln1(const void *x, bq_dtype xt, int64_t K, const float *ln_w, const float *ln_b, float eps,
+                              const uint32_t *wpacked, const float *w_scale, const float *bias, int64_t N,
+                              bq_dtype out_dtype, void *out, int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum,
+                              cudaStream_t s, const DevInfo &dev);
 
 // W4A4 (4-bit activations and weights with given steps, w4a4.cu).
 cudaError_t launch_q4_weight_pack(const void *w, bq_dtype wt, int64_t N, int64_t K, const float *scale_w,

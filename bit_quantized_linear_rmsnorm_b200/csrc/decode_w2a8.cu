@@ -64,6 +64,7 @@ struct DecodeArgs {
     int rb;  // rows per CTA
     uint32_t *status;
     bq_dtype out_dtype;
+    const float *ln_w = nullptr, *ln_b = nullptr;  // LayerNorm normaliser (one-token stream kernel): affine or NULL
 };
 
 struct Layout {
@@ -549,13 +550,46 @@ __device__ __forceinline__ int chunk_dot(const uint4 &w, const uint4 (&x)[4]) {
     return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
 }
 
-template <int MT, typename InT, typename OutT>
+// eight affine parameters of chunk c (k = 8 c .. 8 c + 7 for bf16, 4 c .. for fp32) as floats
+template <int EPC>
+__device__ __forceinline__ void ln_param8(const float *p, int c, float def, float (&o)[EPC]) {
+    if (p == nullptr) {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) o[e] = def;
+    } else if (reinterpret_cast<uintptr_t>(p) % 16 == 0) {
+#pragma unroll
+        for (int h = 0; h < EPC / 4; ++h) {
+            const float4 t = __ldg(reinterpret_cast<const float4 *>(p + c * EPC) + h);
+            o[4 * h] = t.x;
+            o[4 * h + 1] = t.y;
+            o[4 * h + 2] = t.z;
+            o[4 * h + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) o[e] = __ldg(p + c * EPC + e);
+    }
+}
+
+// LN = true (one token): the LayerNorm normaliser instead of the RMSNorm one.
+// Mean and variance from binary64 sums of x - x[0] (the shifted form cancels
+// only by (mean - x[0])^2 / var); y = x * rsd + nmr with rsd = 1/sqrt(var +
+// eps) and nmr = -mean * rsd split into two fp32 parts each, so the mean
+// cancels inside one fused multiply-add before its only rounding, then the
+// affine step in fp32.  y is then within about three fp32 roundings of itself
+// plus an absolute 6 u^2 |nmr| max|g| (u = 2^-24), which, scaled by
+// f = 127 / max|y|, stays below 4.3e-8 when |nmr| max|g| f < 2^21: far inside
+// the 1e-6 band around a rounding tie.  A row that fails the check takes
+// binary64 passes (the decision is the same for the whole CTA).
+template <int MT, typename InT, typename OutT, bool LN>
 __global__ void __launch_bounds__(kStreamThreads, 2) decode_w2a8_stream_kernel(const DecodeArgs p) {
     constexpr int EPC = Elt<InT>::kPerChunk;
     constexpr int XC = StreamX<MT>::kChunks;
+    static_assert(!LN || MT == 1, "the LayerNorm form streams one token");
     __shared__ __align__(16) int8_t xs[MT][kStreamXPitch];
     __shared__ int rowacc[kStreamMaxRows][MT];
     __shared__ float q_ss[MT][kStreamWarps], q_mx[MT][kStreamWarps];
+    __shared__ double q_d[2][kStreamWarps];  // LN: sums of x - x[0] and of its square
     __shared__ int q_rs[MT][kStreamWarps];
     const int K = p.K;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -583,24 +617,53 @@ __global__ void __launch_bounds__(kStreamThreads, 2) decode_w2a8_stream_kernel(c
             xc[m][i] = c < nch ? __ldg(xv + c) : make_uint4(0u, 0u, 0u, 0u);
         }
     }
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+    double ln_c = 0.0;  // LN: the row's first element
+    if constexpr (LN) {
+        ln_c = static_cast<double>(static_cast<float>(static_cast<const InT *>(p.x)[0]));
+        double s = 0.0, s2 = 0.0;
 #pragma unroll
         for (int i = 0; i < XC; ++i) {
-            float f[EPC];
-            Elt<InT>::unpack(xc[m][i], f);
+            const int c = threadIdx.x + kStreamThreads * i;
+            if (c < nch) {
+                float f[EPC];
+                Elt<InT>::unpack(xc[0][i], f);
 #pragma unroll
-            for (int e = 0; e < EPC; e += 2) {
-                ss0 = fmaf(f[e], f[e], ss0);
-                ss1 = fmaf(f[e + 1], f[e + 1], ss1);
-                amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+                for (int e = 0; e < EPC; ++e) {
+                    const double d = static_cast<double>(f[e]) - ln_c;
+                    s += d;
+                    s2 = fma(d, d, s2);
+                }
             }
         }
-        const float ss = warp_sum_f(ss0 + ss1), mx = warp_max_f(amax);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+            s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        }
         if (lane == 0) {
-            q_ss[m][warp] = ss;
-            q_mx[m][warp] = mx;
+            q_d[0][warp] = s;
+            q_d[1][warp] = s2;
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < XC; ++i) {
+                float f[EPC];
+                Elt<InT>::unpack(xc[m][i], f);
+#pragma unroll
+                for (int e = 0; e < EPC; e += 2) {
+                    ss0 = fmaf(f[e], f[e], ss0);
+                    ss1 = fmaf(f[e + 1], f[e + 1], ss1);
+                    amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+                }
+            }
+            const float ss = warp_sum_f(ss0 + ss1), mx = warp_max_f(amax);
+            if (lane == 0) {
+                q_ss[m][warp] = ss;
+                q_mx[m][warp] = mx;
+            }
         }
     }
 
@@ -616,6 +679,139 @@ __global__ void __launch_bounds__(kStreamThreads, 2) decode_w2a8_stream_kernel(c
 
     // code factor of each token (every thread derives the same one), codes
     float sc[MT];
+    if constexpr (LN) {
+        double S = 0.0, S2 = 0.0;
+#pragma unroll
+        for (int w2 = 0; w2 < kStreamWarps; ++w2) {
+            S += q_d[0][w2];
+            S2 += q_d[1][w2];
+        }
+        const double md = S / static_cast<double>(K);
+        const double mu = ln_c + md;
+        const double var = fmax(S2 / static_cast<double>(K) - md * md, 0.0);
+        const double rsd = 1.0 / sqrt(var + static_cast<double>(p.eps));
+        const double nmr = -mu * rsd;
+        const float rsd_h = static_cast<float>(rsd), rsd_l = static_cast<float>(rsd - static_cast<double>(rsd_h));
+        const float nmr_h = static_cast<float>(nmr), nmr_l = static_cast<float>(nmr - static_cast<double>(nmr_h));
+        float gmax = 0.0f;  // max |g| (for the error check), gathered with max|y|
+        auto y_f = [&](int i, float (&y)[EPC]) {
+            const int c = threadIdx.x + kStreamThreads * i;
+            float f[EPC], gk[EPC], bk[EPC];
+            Elt<InT>::unpack(xc[0][i], f);
+            ln_param8<EPC>(p.ln_w, c, 1.0f, gk);
+            ln_param8<EPC>(p.ln_b, c, 0.0f, bk);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+                y[e] = __fmaf_rn(__fadd_rn(__fmaf_rn(f[e], rsd_h, nmr_h), __fmaf_rn(f[e], rsd_l, nmr_l)), gk[e], bk[e]);
+                gmax = fmaxf(gmax, fabsf(gk[e]));
+            }
+        };
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < XC; ++i)
+            if (threadIdx.x + kStreamThreads * i < nch) {
+                float y[EPC];
+                y_f(i, y);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) amax = fmaxf(amax, fabsf(y[e]));
+            }
+        amax = warp_max_f(amax);
+        gmax = warp_max_f(gmax);
+        if (lane == 0) {
+            q_ss[0][warp] = amax;
+            q_mx[0][warp] = gmax;
+        }
+        __syncthreads();
+        amax = 0.0f;
+        gmax = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < kStreamWarps; ++w2) {
+            amax = fmaxf(amax, q_ss[0][w2]);
+            gmax = fmaxf(gmax, q_mx[0][w2]);
+        }
+        const float a_f = fmaxf(amax, 1e-5f);
+        const float fac = __fdiv_rn(127.0f, a_f);
+        const bool fast = fabs(nmr) * static_cast<double>(gmax) * static_cast<double>(fac) < 2097152.0;
+        double fd = 0.0;
+        if (fast) {
+            sc[0] = __fdiv_rn(a_f, 127.0f);
+        } else {  // binary64 passes (uniform over the CTA)
+            double ad = 0.0;
+#pragma unroll
+            for (int i = 0; i < XC; ++i) {
+                const int c = threadIdx.x + kStreamThreads * i;
+                if (c < nch) {
+                    float f[EPC], gk[EPC], bk[EPC];
+                    Elt<InT>::unpack(xc[0][i], f);
+                    ln_param8<EPC>(p.ln_w, c, 1.0f, gk);
+                    ln_param8<EPC>(p.ln_b, c, 0.0f, bk);
+#pragma unroll
+                    for (int e = 0; e < EPC; ++e)
+                        ad = fmax(ad, fabs(fma(fma(static_cast<double>(f[e]), rsd, nmr), static_cast<double>(gk[e]),
+                                               static_cast<double>(bk[e]))));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) ad = fmax(ad, __shfl_xor_sync(0xffffffffu, ad, o));
+            if (lane == 0) q_d[0][warp] = ad;
+            __syncthreads();
+            ad = 0.0;
+#pragma unroll
+            for (int w2 = 0; w2 < kStreamWarps; ++w2) ad = fmax(ad, q_d[0][w2]);
+            ad = fmax(ad, 1e-5);
+            fd = 127.0 / ad;
+            sc[0] = static_cast<float>(ad / 127.0);
+        }
+        int isum = 0;
+#pragma unroll
+        for (int i = 0; i < XC; ++i) {
+            const int c = threadIdx.x + kStreamThreads * i;
+            if (c < nch) {
+                uint32_t wq[EPC / 4];
+                if (fast) {
+                    float y[EPC];
+                    y_f(i, y);
+#pragma unroll
+                    for (int j = 0; j < EPC / 4; ++j)
+                        wq[j] = pack_codes4(__fmaf_rn(y[4 * j], fac, kRoundMagic), __fmaf_rn(y[4 * j + 1], fac, kRoundMagic),
+                                            __fmaf_rn(y[4 * j + 2], fac, kRoundMagic),
+                                            __fmaf_rn(y[4 * j + 3], fac, kRoundMagic));
+                } else {
+                    float f[EPC], gk[EPC], bk[EPC];
+                    Elt<InT>::unpack(xc[0][i], f);
+                    ln_param8<EPC>(p.ln_w, c, 1.0f, gk);
+                    ln_param8<EPC>(p.ln_b, c, 0.0f, bk);
+#pragma unroll
+                    for (int j = 0; j < EPC / 4; ++j) {
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int e = 4 * j + u;
+                            const double y = fma(fma(static_cast<double>(f[e]), rsd, nmr), static_cast<double>(gk[e]),
+                                                 static_cast<double>(bk[e]));
+                            int code = __double2int_rn(y * fd);
+                            code = code < -128 ? -128 : (code > 127 ? 127 : code);
+                            word |= (static_cast<uint32_t>(code) & 0xffu) << (8 * u);
+                        }
+                        wq[j] = word;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < EPC / 4; ++j) isum = dp4a_ss(wq[j], 0x01010101u, isum);
+                int8_t *ws = blockIdx.x == 0 ? p.ws_xq + c * EPC : nullptr;
+                if constexpr (EPC == 8) {
+                    *reinterpret_cast<uint2 *>(&xs[0][c * 8]) = make_uint2(wq[0], wq[1]);
+                    if (ws) *reinterpret_cast<uint2 *>(ws) = make_uint2(wq[0], wq[1]);
+                } else {
+                    *reinterpret_cast<uint32_t *>(&xs[0][c * 4]) = wq[0];
+                    if (ws) *reinterpret_cast<uint32_t *>(ws) = wq[0];
+                }
+            }
+        }
+        isum = warp_sum_i(isum);
+        if (lane == 0) q_rs[0][warp] = isum;
+        if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_scale[0] = sc[0];
+    } else {
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         float ss = 0.f, mx = 0.f;
@@ -653,6 +849,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) decode_w2a8_stream_kernel(c
         isum = warp_sum_i(isum);
         if (lane == 0) q_rs[m][warp] = isum;
         if (blockIdx.x == 0 && threadIdx.x == 0) p.ws_scale[m] = sc[m];
+    }
     }
     __syncthreads();
 
@@ -696,7 +893,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) decode_w2a8_stream_kernel(c
     }
 }
 
-template <typename InT, typename OutT>
+template <typename InT, typename OutT, bool LN = false>
 cudaError_t launch_stream(const DecodeArgs &a, int MT, cudaStream_t s, int grid) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -709,18 +906,18 @@ cudaError_t launch_stream(const DecodeArgs &a, int MT, cudaStream_t s, int grid)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     (void)MT;  // one token (two would not fit the register budget)
-    return cudaLaunchKernelEx(&cfg, decode_w2a8_stream_kernel<1, InT, OutT>, a);
+    return cudaLaunchKernelEx(&cfg, decode_w2a8_stream_kernel<1, InT, OutT, LN>, a);
 }
 
-template <typename InT>
+template <typename InT, bool LN = false>
 cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStream_t s, int grid) {
     switch (ot) {
         case BQ_F32:
-            return launch_stream<InT, float>(a, MT, s, grid);
+            return launch_stream<InT, float, LN>(a, MT, s, grid);
         case BQ_F16:
-            return launch_stream<InT, __half>(a, MT, s, grid);
+            return launch_stream<InT, __half, LN>(a, MT, s, grid);
         default:
-            return launch_stream<InT, __nv_bfloat16>(a, MT, s, grid);
+            return launch_stream<InT, __nv_bfloat16, LN>(a, MT, s, grid);
     }
 }
 
@@ -1185,6 +1382,37 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     const int smem = static_cast<int>(Layout(static_cast<int>(K), MT, rb).total) + 1024;
     if (xt == BQ_BF16) return dispatch_out<__nv_bfloat16>(a, out_dtype, MT, smem, dev, s, grid);
     return dispatch_out<float>(a, out_dtype, MT, smem, dev, s, grid);
+}
+
+bool decode_ln1_supported(const void *x, int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev) {
+    return M == 1 && reinterpret_cast<uintptr_t>(x) % 16 == 0 && stream_supported(M, N, K, xt, dev);
+}
+
+cudaError_t launch_decode_ln1(const void *x, bq_dtype xt, int64_t K, const float *ln_w, const float *ln_b, float eps,
+                              const uint32_t *wpacked, const float *w_scale, const float *bias, int64_t N,
+                              bq_dtype out_dtype, void *out, int8_t *ws_xq, float *ws_scale, int32_t *ws_rowsum,
+                              cudaStream_t s, const DevInfo &dev) {
+    DecodeArgs a;
+    a.x = x;
+    a.M = 1;
+    a.K = static_cast<int>(K);
+    a.eps = eps;
+    a.wpacked = wpacked;
+    a.w_scale = w_scale;
+    a.bias = bias;
+    a.N = static_cast<int>(N);
+    a.out = out;
+    a.ws_xq = ws_xq;
+    a.ws_scale = ws_scale;
+    a.ws_rowsum = ws_rowsum;
+    a.rb = rows_per_cta(N, dev);
+    a.status = dev.status;
+    a.out_dtype = out_dtype;
+    a.ln_w = ln_w;
+    a.ln_b = ln_b;
+    const int grid = grid_of(N, dev);
+    if (xt == BQ_BF16) return launch_stream_out<__nv_bfloat16, true>(a, out_dtype, 1, s, grid);
+    return launch_stream_out<float, true>(a, out_dtype, 1, s, grid);
 }
 
 }  // namespace bq

@@ -623,7 +623,10 @@ def test_act_quant_layernorm_special_rows():
                                                    (16, 300, 2048, "f32", True, True),
                                                    (300, 520, 512, "bf16", True, True),
                                                    (300, 61, 144, "f16", False, True),
-                                                   (2048, 4096, 256, "bf16", False, False)])
+                                                   (2048, 4096, 256, "bf16", False, False),
+                                                   (1, 11008, 4096, "bf16", True, True),     # one token: fused
+                                                   (1, 300, 2048, "f32", False, False),
+                                                   (1, 5000, 8192, "bf16", False, True)])
 def test_bitlinear_layernorm(M, N, K, out, bias, affine):
     g = synth.rng((123, M, N, K))
     bits, xf = synth.bf16_activations(M, K, (123, M, K), outlier_frac=0.01)
@@ -644,6 +647,39 @@ def test_bitlinear_layernorm(M, N, K, out, bias, affine):
     assert_codes(g_xq, a["xq"], a["pre"], what + " xq")
     rel32 = bitlinear_rel32(g_sc, a["act_scale"], host(ws_)[0], t["gamma"])
     assert_out(host(o), ref, _TORCH_OUT[out], what, extra=extra, scale=scale, rel32=rel32)
+
+
+@pytest.mark.parametrize("row,affine", [("constant", False), ("constant", True), ("offset", True), ("tiny", False)])
+def test_bitlinear_layernorm_one_token_degenerate(row, affine):
+    # one token through the fused kernel: a constant row far from zero and a tiny spread on a large
+    # offset take its binary64 passes, a 250-sigma offset its fp32 ones
+    N, K = 2000, 4096
+    g = synth.rng((125, ["constant", "offset", "tiny"].index(row), int(affine)))
+    xf = synth.normal_f32(g, (1, K))
+    if row == "constant":
+        xf[:] = 1e5
+    elif row == "offset":
+        xf += np.float32(250.0)
+    else:
+        xf = np.float32(1e4) + np.float32(1e-2) * xf
+    bits = synth.f32_to_bf16_bits(xf)
+    xf = synth.bf16_bits_to_f32(bits)
+    w = synth.normal_f32(g, (N, K), 0.02)
+    lw, lb = _ln_params(g, K, affine)
+    wp, ws_ = bq.bq_weight_quant_ternary_pack(dev(w))
+    work = torch.empty(bq.bq_workspace_bytes(bq.BQ_OP_BITLINEAR_W2A8, 1, N, K), dtype=torch.uint8, device="cuda")
+    o = bq.bq_bitlinear_w2a8_layernorm(bf16_dev(bits), wp, ws_, N, None if lw is None else dev(lw),
+                                       None if lb is None else dev(lb), None, 1e-5, torch.float32, workspace=work)
+    torch.cuda.synchronize()
+    xo, so, _ = bq.bq_bitlinear_workspace_layout(1, K)
+    g_xq = host(work[xo:xo + K].view(torch.int8).view(1, K))
+    g_sc = host(work[so:so + 4].view(torch.float32))
+    what = f"bitlinear layernorm one token {row} affine={affine}"
+    ref, extra, scale, a, t = bitlinear_expected(xf, w, None, 1e-5, ln=(lw, lb))
+    assert_codes(g_xq, a["xq"], a["pre"], what + " xq")
+    np.testing.assert_allclose(g_sc, a["act_scale"], rtol=1e-5)
+    rel32 = bitlinear_rel32(g_sc, a["act_scale"], host(ws_)[0], t["gamma"])
+    assert_out(host(o), ref, torch.float32, what, extra=extra, scale=scale, rel32=rel32)
 
 
 # ------------------------------------------------------- W4A4 (Q4Linear)
