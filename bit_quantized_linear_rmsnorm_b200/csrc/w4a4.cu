@@ -145,32 +145,42 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
         int acc[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) acc[m] = 0;
-#pragma unroll 4
-        for (int64_t pc = lane; pc < pieces; pc += 32) {
-            const uint4 u = __ldcs(wr + pc);
-            const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
-            uint32_t b[8];  // 32 sign-extended codes, k = 32 pc + 4 j + 0..3 in b[j]
+        // four pieces per lane in flight before any of them is used
+        for (int64_t base = lane; base < pieces; base += 32 * 4) {
+            uint4 u4[4];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const uint32_t lo = (ws[h] << 4) & 0xF0F0F0F0u, hi = ws[h] & 0xF0F0F0F0u;
-                b[2 * h] = __byte_perm(lo, hi, 0x5140);
-                b[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+            for (int j = 0; j < 4; ++j) {
+                const int64_t pc = base + 32 * j;
+                u4[j] = pc < pieces ? __ldcs(wr + pc) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                if (m < M) {
-                    const uint4 *xr = reinterpret_cast<const uint4 *>(xs + static_cast<int64_t>(m) * K + 32 * pc);
-                    const uint4 a0 = xr[0], a1 = xr[1];
-                    int s = acc[m];
-                    s = dp4a_ss(a0.x, b[0], s);
-                    s = dp4a_ss(a0.y, b[1], s);
-                    s = dp4a_ss(a0.z, b[2], s);
-                    s = dp4a_ss(a0.w, b[3], s);
-                    s = dp4a_ss(a1.x, b[4], s);
-                    s = dp4a_ss(a1.y, b[5], s);
-                    s = dp4a_ss(a1.z, b[6], s);
-                    s = dp4a_ss(a1.w, b[7], s);
-                    acc[m] = s;
+            for (int j = 0; j < 4; ++j) {
+                const int64_t pc = base + 32 * j;
+                if (pc >= pieces) break;
+                const uint32_t ws[4] = {u4[j].x, u4[j].y, u4[j].z, u4[j].w};
+                uint32_t b[8];  // 32 sign-extended codes, k = 32 pc + 4 i + 0..3 in b[i]
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint32_t lo = (ws[h] << 4) & 0xF0F0F0F0u, hi = ws[h] & 0xF0F0F0F0u;
+                    b[2 * h] = __byte_perm(lo, hi, 0x5140);
+                    b[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+                }
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    if (m < M) {
+                        const uint4 *xr = reinterpret_cast<const uint4 *>(xs + static_cast<int64_t>(m) * K + 32 * pc);
+                        const uint4 a0 = xr[0], a1 = xr[1];
+                        int s = acc[m];
+                        s = dp4a_ss(a0.x, b[0], s);
+                        s = dp4a_ss(a0.y, b[1], s);
+                        s = dp4a_ss(a0.z, b[2], s);
+                        s = dp4a_ss(a0.w, b[3], s);
+                        s = dp4a_ss(a1.x, b[4], s);
+                        s = dp4a_ss(a1.y, b[5], s);
+                        s = dp4a_ss(a1.z, b[6], s);
+                        s = dp4a_ss(a1.w, b[7], s);
+                        acc[m] = s;
+                    }
                 }
             }
         }
