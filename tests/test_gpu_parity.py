@@ -592,6 +592,8 @@ def test_act_quant_layernorm_degenerate_rows_many(affine):
     x[3] = np.float32(-250.0) + synth.normal_f32(g, (K,))            # offset 250 sigma
     x[4] = 0.0
     x[4, 9] = -7.0                                                   # one-hot
+    x[5, ::7] = np.float32(1e-40)                                    # subnormal and zero elements
+    x[5, 3::11] = 0.0
     lw, lb = _ln_params(g, K, affine)
     xq, sc, rs = bq.bq_act_quant_int8_layernorm(dev(x), 1e-5, None if lw is None else dev(lw),
                                                 None if lb is None else dev(lb))
