@@ -32,9 +32,11 @@
  * first along the reduction axis; the INT4 affine form is s*(q - z).
  *
  * Pins: every function here is checked by the CPU test-suite against values
- * the pages print (the ATB example), closed forms, invariants and library
- * routines on special cases.  The BitLinear composition is pinned only
- * through its steps plus closed-form special cases.
+ * the pages print (the ATB example), closed forms, invariants, library
+ * routines on special cases, and (for the backward passes) autograd of the
+ * straight-through forward.  The BitLinear composition is pinned through its
+ * steps, closed-form special cases and a one-code-per-row case that fixes
+ * the weight indexing.
  */
 #include <math.h>
 #include <stdint.h>
