@@ -64,6 +64,7 @@ __global__ void q4_act_quant_kernel(const In *__restrict__ x, int64_t M, int64_t
                                     const float *__restrict__ scale_a, float eps, int8_t *__restrict__ xq,
                                     int64_t ldq, float *__restrict__ row_step, const float *__restrict__ scale_w,
                                     int per_channel, int64_t N, float *__restrict__ col_step) {
+    pdl_launch_dependents();  // the GEMV may be scheduled (it reads the codes only after its wait)
     const float sa = step_of(scale_a, 0, eps);
     const int64_t total = M * K;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -86,6 +87,7 @@ __global__ void q4_act_quant_vec_kernel(const In *__restrict__ x, int64_t M, int
                                         const float *__restrict__ scale_a, float eps, int8_t *__restrict__ xq,
                                         int64_t ldq, float *__restrict__ row_step, const float *__restrict__ scale_w,
                                         int per_channel, int64_t N, float *__restrict__ col_step) {
+    pdl_launch_dependents();  // the GEMV may be scheduled (it reads the codes only after its wait)
     const float sa = step_of(scale_a, 0, eps);
     const int64_t cpr = K / 8, total = M * cpr;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -134,6 +136,17 @@ __global__ void __launch_bounds__(kGemvWarps * 32)
                      const float *__restrict__ bias, int64_t N, OutT *__restrict__ out) {
     extern __shared__ __align__(16) int8_t xs[];  // [MT][K]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // launched as a programmatic dependent of the act-quant kernel: before the
+    // dependency wait a warp only prefetches its first weight row into L2
+    // (which consumes nothing); everything is read after it
+    {
+        const int64_t n = static_cast<int64_t>(blockIdx.x) * kGemvWarps + warp;
+        if (n < N)
+            for (int64_t l = lane; l < (K / 2 + 127) / 128; l += 32)
+                prefetch_l2(reinterpret_cast<const uint8_t *>(wpacked + n * (K / 8)) + l * 128);
+    }
+    pdl_launch_dependents();
+    pdl_wait();
     const int64_t chunks = static_cast<int64_t>(M) * K / 16;
     for (int64_t i = threadIdx.x; i < chunks; i += blockDim.x)
         reinterpret_cast<uint4 *>(xs)[i] = __ldg(reinterpret_cast<const uint4 *>(xq) + i);
@@ -223,9 +236,17 @@ cudaError_t launch_gemv_mt(const int8_t *xq, int M, int64_t K, const uint32_t *w
     int64_t grid = (N + kGemvWarps - 1) / kGemvWarps;
     const int64_t cap = static_cast<int64_t>(dev.num_sms) * (smem > 100 * 1024 ? 2 : smem > 24 * 1024 ? 4 : 8);
     if (grid > cap) grid = cap;
-    kern<<<static_cast<unsigned>(grid), kGemvWarps * 32, smem, s>>>(xq, M, K, wpacked, row_step, col_step, bias, N,
-                                                                     static_cast<OutT *>(out));
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kGemvWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, xq, M, K, wpacked, row_step, col_step, bias, N, static_cast<OutT *>(out));
 }
 
 template <typename OutT>

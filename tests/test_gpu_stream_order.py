@@ -72,3 +72,31 @@ def test_weights_packed_just_before_the_call(M, ln):
         assert torch.equal(o.view(torch.int16), r.view(torch.int16)), f"call {i}: output differs from the synchronised call"
     # and consecutive references really differ, so a stale read could not pass
     assert not torch.equal(refs[0], refs[1]) and not torch.equal(refs[1], refs[2])
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_w4a4_weights_packed_just_before_the_call(M):
+    # the 4-bit path: act-quant kernel, then the GEMV launched as its programmatic dependent
+    dev = "cuda"
+    K4, N4 = 4096, 11008
+    g = synth.rng((78, M))
+    ws_f32 = [torch.from_numpy(synth.normal_f32(g, (N4, K4), 0.02 * (i + 1))).to(dev) for i in range(3)]
+    x = torch.from_numpy(synth.normal_f32(g, (M, K4))).to(dev)
+    sa = torch.tensor([0.27], dtype=torch.float32, device=dev)
+    sw = torch.tensor([0.006], dtype=torch.float32, device=dev)
+    wp = torch.empty((N4, K4 // 8), dtype=torch.int32, device=dev)
+    refs = []
+    for w in ws_f32:
+        bq.bq_weight_quant_int4_pack(w, sw, 1e-6, wpacked=wp)
+        torch.cuda.synchronize()
+        refs.append(bq.bq_linear_w4a4(x, sa, wp, sw, N4, 1e-6, out_dtype=torch.float32))
+        torch.cuda.synchronize()
+    outs = []
+    for _ in range(2):
+        for w in ws_f32:
+            bq.bq_weight_quant_int4_pack(w, sw, 1e-6, wpacked=wp)
+            outs.append(bq.bq_linear_w4a4(x, sa, wp, sw, N4, 1e-6, out_dtype=torch.float32))
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        assert torch.equal(o, refs[i % 3]), f"call {i}: output differs from the synchronised call"
+    assert not torch.equal(refs[0], refs[1])
