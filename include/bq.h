@@ -223,8 +223,12 @@ bq_status bq_bitlinear_w2a8(const void *x, bq_dtype x_dtype, int64_t M, int64_t 
  *   act_scale[m] = a[m] / 127,  rowsum[m] = sum_k xq[m,k]
  *
  * ln_weight (g) and ln_bias (b): fp32 [K] each, 4-byte aligned, or NULL for
- * g = 1 / b = 0 (a parameter-free LayerNorm).  Computed in binary64 (the mean
- * subtraction cancels).  Other arguments and rules as bq_act_quant_int8.
+ * g = 1 / b = 0 (a parameter-free LayerNorm).  The mean and variance are taken
+ * in binary64 (the mean subtraction cancels); y in binary64 or, for at least
+ * eight aligned rows, in fp32 with the row constants split into two fp32 parts
+ * under a per-row error check (rows that fail it take binary64), so every code
+ * agrees with the binary64 one except within 1e-6 (relative) of a rounding
+ * tie.  Other arguments and rules as bq_act_quant_int8.
  */
 bq_status bq_act_quant_int8_layernorm(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, int64_t ldx,
                                       const float *ln_weight, const float *ln_bias, float eps, int8_t *xq,
@@ -235,8 +239,12 @@ bq_status bq_act_quant_int8_layernorm(const void *x, bq_dtype x_dtype, int64_t M
  * Utilities", BitLinear: LayerNorm, 8-bit per-token activations, absmean
  * ternary weights, rescale): bq_act_quant_int8_layernorm into the workspace,
  * then the ternary linear and rescale of bq_bitlinear_w2a8
- * (out = (float(acc) * act_scale[m]) * gamma (+ bias[n])) on the split GEMV
- * kernel (M <= 16) or the tcgen05 GEMM (M > 16).  Arguments, workspace
+ * (out = (float(acc) * act_scale[m]) * gamma (+ bias[n])) on the mma.sync
+ * weight-streaming kernel or the split GEMV kernel (M <= 16) or the tcgen05
+ * GEMM (M > 16); one token with K in {2048, 4096, 8192} (fp32: up to 4096) and a
+ * 16-byte aligned x runs the normaliser inside the weight-streaming kernel,
+ * one launch, which also writes the codes, act_scale and rowsum to the
+ * workspace.  Arguments, workspace
  * (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) and its layout) and
  * rules as bq_bitlinear_w2a8, plus ln_weight / ln_bias as above.
  */
