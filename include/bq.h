@@ -241,10 +241,11 @@ bq_status bq_act_quant_int8_layernorm(const void *x, bq_dtype x_dtype, int64_t M
  * then the ternary linear and rescale of bq_bitlinear_w2a8
  * (out = (float(acc) * act_scale[m]) * gamma (+ bias[n])) on the mma.sync
  * weight-streaming kernel or the split GEMV kernel (M <= 16) or the tcgen05
- * GEMM (M > 16); one token with K in {2048, 4096, 8192} (fp32: up to 4096) and a
- * 16-byte aligned x runs the normaliser inside the weight-streaming kernel,
- * one launch, which also writes the codes, act_scale and rowsum to the
- * workspace.  Arguments, workspace
+ * GEMM (M > 16); one token with K in {2048, 4096, 8192} (fp32: up to 4096),
+ * a 16-byte aligned x and at most 5120 * 64 / K weight rows per SM (N up to
+ * 11840 at K = 4096 on 148 SMs) runs the normaliser inside the
+ * weight-streaming kernel, one launch, which also writes the codes, act_scale
+ * and rowsum to the workspace.  Arguments, workspace
  * (bq_workspace_bytes(BQ_OP_BITLINEAR_W2A8, M, N, K, 0) and its layout) and
  * rules as bq_bitlinear_w2a8, plus ln_weight / ln_bias as above.
  */
