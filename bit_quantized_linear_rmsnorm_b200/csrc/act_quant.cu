@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                          int8_t *__restrict__ xq, int64_t ldq, float *__restrict__ act_scale,
                          int32_t *__restrict__ rowsum) {
     constexpr int EPC = Elt<In>::kPerChunk;
+    pdl_launch_dependents();  // a dependent GEMM reads the codes only after its wait
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(kRowThreads)
                          int8_t *__restrict__ xq, int64_t ldq, float *__restrict__ act_scale,
                          int32_t *__restrict__ rowsum) {
     constexpr int EPC = Elt<In>::kPerChunk;
+    pdl_launch_dependents();  // a dependent GEMM reads the codes only after its wait
     __shared__ float s_ss[kRowThreads / 32], s_mx[kRowThreads / 32];
     __shared__ int s_rs[kRowThreads / 32];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -233,6 +235,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     act_quant_scalar_kernel(const In *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float eps,
                             int8_t *__restrict__ xq, int64_t ldq, float *__restrict__ act_scale,
                             int32_t *__restrict__ rowsum) {
+    pdl_launch_dependents();  // a dependent GEMM reads the codes only after its wait
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kWarpsPerBlock) + (threadIdx.x >> 5);
     const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarpsPerBlock;

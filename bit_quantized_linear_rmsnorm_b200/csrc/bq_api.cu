@@ -375,6 +375,7 @@ static bq_status bitlinear_linear(int path, const BitlinearLayout &l, uint8_t *w
     g.rowscale = act_scale;
     g.rowcorr = rowsum;
     g.bias = bias;
+    g.pdl = K % 64 == 0;  // straight after the quantizer (no re-pitch copy in between)
     g.M = M;
     g.N = N;
     g.K = K;
@@ -577,6 +578,7 @@ bq_status bq_linear_w4a4(const void *x, bq_dtype x_dtype, int64_t M, int64_t K, 
     g.colscale = col_step;
     g.rowscale = row_step;
     g.bias = bias;
+    g.pdl = true;  // straight after the quantizer
     g.M = M;
     g.N = N;
     g.K = K;

@@ -104,6 +104,9 @@ struct GemmArgs {
     // (packed B, K-major A) rows of A per batch (0: M); output row m reads A row
     // m + a_row_off, and rows outside [0, a_rows) read as zeros
     int64_t a_rows = 0, a_row_off = 0;
+    // launched as a programmatic dependent of the kernel just before it (the
+    // kernel's producer and epilogue wait for it before reading anything)
+    bool pdl = false;
     uint64_t wait_ns = 2000000000ull;  // limit of the kernel's bounded waits
     int withhold_kb = -1;              // failure-detection check only (single-CTA kernel)
 };

@@ -234,6 +234,7 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------------ producer
+        pdl_wait();  // (a programmatic dependent of the act-quant kernel: its codes are ready)
         int stage = 0;
         uint32_t phase = 0;
         int64_t issued = 0;
@@ -339,6 +340,7 @@ __global__ void __launch_bounds__(Cfg<PK>::kThreads, 1)
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ epilogue
+        pdl_wait();  // the row scales and sums come from the kernel before
         const int q = warp - 4;  // TMEM lane quarter
         const int r = 32 * q + lane;
         const int et = threadIdx.x - 128;  // 0..127
@@ -673,6 +675,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
+        pdl_wait();  // (a programmatic dependent of the act-quant kernel: its codes are ready)
         int stage = 0;
         uint32_t phase = 0;
         int64_t issued = 0;
@@ -762,6 +765,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<PK>::kThread
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ epilogue (both CTAs)
+        pdl_wait();  // the row scales and sums come from the kernel before
         const int q = warp - 4;
         const int r = 32 * q + lane;
         const int et = threadIdx.x - 128;
@@ -980,6 +984,19 @@ bq_status launch_t(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &
         return BQ_ERR_CUDA;
     const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN) * g.batch;
     const int grid = static_cast<int>(tiles < dev.num_sms ? tiles : dev.num_sms);
+    if (g.pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = C::SMEM;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, mA, mB, mBh, mO, dev_args(g, dev)) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+    }
     kern<<<grid, C::kThreads, C::SMEM, s>>>(mA, mB, mBh, mO, dev_args(g, dev));
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
@@ -996,6 +1013,19 @@ bq_status launch_pair(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMa
     const int64_t pairs = std::min<int64_t>(tiles, dev.num_sms / 2);
     GemmDev p = dev_args(g, dev);
     p.withhold_kb = -1;  // (the failure-detection check runs on a single CTA)
+    if (g.pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = C::SMEM;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, mA, mB128, mB64, mO, p) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+    }
     kern<<<static_cast<unsigned>(2 * pairs), C::kThreads, C::SMEM, s>>>(mA, mB128, mB64, mO, p);
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
@@ -1009,7 +1039,6 @@ bool use_pair(const GemmArgs &g, const DevInfo &dev) {
 template <int PK, typename OutT>
 bq_status dispatch_packed(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mO,
                           cudaStream_t s, const DevInfo &dev) {
-    const uint64_t nb = static_cast<uint64_t>(g.batch);
     if (use_pair(g, dev)) {
         // per CTA of a pair: its half of the packed tile (128 rows), 64 rows for half tiles
         CUtensorMap mP128, mP64;
@@ -1028,7 +1057,6 @@ template <typename OutT>
 bq_status dispatch(const GemmArgs &g, const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mBh,
                    const CUtensorMap &mO,
                    cudaStream_t s, const DevInfo &dev) {
-    const uint64_t nb = static_cast<uint64_t>(g.batch);
     if (g.b_pack == 2) return dispatch_packed<2, OutT>(g, mA, mB, mO, s, dev);
     if (g.b_pack == 4) return dispatch_packed<4, OutT>(g, mA, mB, mO, s, dev);
     if (use_pair(g, dev)) {
