@@ -523,7 +523,7 @@ def _decode(res, steps, hbm, ms=(1, 4, 16)):
         res[f"bitlinear_decode_M{M}"] = {"us_per_step": round(ms * 1e3, 3), "GB/s": round(gbs, 1),
                                          "frac_hbm": round(gbs / hbm, 4), "algorithmic_bytes": byts,
                                          "weight_GB/s": round((N * K // 4) / (ms * 1e-3) / 1e9, 1),
-                                         "launches_per_step": 1 if M == 1 else 2,
+                                         "launches_per_step": 1,
                                          "config": f"x bf16 [{M},4096], W 2-bit [11008,4096]"}
     del wps
 

@@ -5,7 +5,14 @@
 //   xq, act_scale = per-token int8 quantization of RMSNorm(x)
 //   acc[m,n] = sum_k xq[m,k] * w_q[n,k],   out = (float(acc) * act_scale[m]) * gamma (+ bias)
 //
-// Bandwidth-bound on the 2-bit weights.  One CTA owns RB consecutive output
+// Kernels, each one launch per call with the tokens quantized inside it:
+// decode_w2a8_stream_kernel (one token, K a multiple of 2048, dp4a from
+// registers), decode_w2a8_fused_kernel (2..16 tokens, K = 2048 or 4096,
+// masked mma.sync from registers), and decode_w2a8_kernel below for the other
+// shapes with K % 512 == 0.  decode_w2a8_mma_kernel serves the LayerNorm
+// BitLinear, whose quantizer has already written the codes.
+//
+// decode_w2a8_kernel: bandwidth-bound on the 2-bit weights.  One CTA owns RB consecutive output
 // rows and copies them into shared memory with 16-byte cp.async (many copies
 // in flight per SM through the load/store path -- measured faster than 2-D
 // TMA boxes for this short HBM stream), laid out in 128-byte K slices of
@@ -921,17 +928,15 @@ cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStre
     }
 }
 
-// 2..16 tokens: two launches chained by programmatic dependent launch.
-//
-// 1. decode_token_quant_kernel (one CTA per token) quantizes each token once
-//    into the workspace (codes, act_scale, row sum).  It waits for the work
-//    before it in the stream (griddepcontrol.wait) before it lets its
-//    dependent start (griddepcontrol.launch_dependents).
-// 2. decode_w2a8_mma_kernel therefore starts only once everything before the
-//    call is complete and visible, so it loads its packed weights into
-//    registers at once (they stream from HBM while the tokens are quantized)
-//    and waits only for the codes; it copies them into shared memory and
-//    runs mma.sync m16n8k32 (u8 fields x s8 codes) from registers.
+// 2..16 tokens whose codes are already in the workspace (the LayerNorm
+// BitLinear, after its quantizer): decode_w2a8_mma_kernel, launched as a
+// programmatic dependent of the quantizer.  The quantizer waits for the work
+// before it in the stream (griddepcontrol.wait) before it lets its dependent
+// start (griddepcontrol.launch_dependents), so this kernel starts only once
+// everything before the call is complete and visible: it loads its packed
+// weights into registers at once (they stream from HBM while the tokens are
+// quantized) and waits only for the codes; it copies them into shared memory
+// and runs mma.sync m16n8k32 (u8 fields x s8 codes) from registers.
 //
 // Work unit = (16-row block rb, 256-wide K block kb); warp w takes the K
 // blocks kb = w + 8 c (c < KBW, K = 2048 KBW) of every row block.  Lane
@@ -948,96 +953,11 @@ cudaError_t launch_stream_out(const DecodeArgs &a, bq_dtype ot, int MT, cudaStre
 constexpr int kMmaThreads = 256;
 constexpr int kMmaWarps = kMmaThreads / 32;
 constexpr int kMmaUnits = 10;  // units per warp held in registers
-constexpr int kTokThreads = 128;
 
 // 16-byte chunk c of a token row sits at chunk c ^ (2 ((c >> 3) & 1)): the
 // B-fragment loads of lanes t = 0..3 (chunks 4 t + const) and of consecutive
 // tokens (row pitch K + 16 bytes) then fall in distinct bank groups.
 __device__ __forceinline__ int xchunk_swz(int c) { return c ^ (((c >> 3) & 1) << 1); }
-
-// One CTA per token: RMSNorm statistics and codes of row blockIdx.x into the
-// workspace.  Chunk c of the row is held by thread c % 128 (at most CPT
-// 16-byte chunks per thread, K <= 4096 fp32 / 8192 bf16).
-template <typename InT>
-__global__ void __launch_bounds__(kTokThreads) decode_token_quant_kernel(const DecodeArgs p) {
-    constexpr int EPC = Elt<InT>::kPerChunk;
-    constexpr int CPT = 8;
-    __shared__ float red[2][kTokThreads / 32];
-    __shared__ int redi[kTokThreads / 32];
-    // the row may come from the previous kernel, and the previous call's
-    // linear kernel may still read the workspace: wait, then release ours
-    pdl_wait();
-    pdl_launch_dependents();
-    const int m = blockIdx.x, K = p.K;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nch = K / EPC;
-    const uint4 *xv = reinterpret_cast<const uint4 *>(static_cast<const InT *>(p.x) + static_cast<int64_t>(m) * K);
-    uint4 c[CPT];
-    float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int ch = threadIdx.x + kTokThreads * i;
-        c[i] = ch < nch ? __ldg(xv + ch) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        float f[EPC];
-        Elt<InT>::unpack(c[i], f);
-#pragma unroll
-        for (int e = 0; e < EPC; e += 2) {
-            ss0 = fmaf(f[e], f[e], ss0);
-            ss1 = fmaf(f[e + 1], f[e + 1], ss1);
-            amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
-        }
-    }
-    float ss = warp_sum_f(ss0 + ss1);
-    amax = warp_max_f(amax);
-    if (lane == 0) {
-        red[0][warp] = ss;
-        red[1][warp] = amax;
-    }
-    __syncthreads();
-    ss = red[0][0];
-    amax = red[1][0];
-#pragma unroll
-    for (int w = 1; w < kTokThreads / 32; ++w) {
-        ss += red[0][w];
-        amax = fmaxf(amax, red[1][w]);
-    }
-    float fac, scale;
-    quant_row_factor(ss, amax, K, p.eps, fac, scale);
-    int isum = 0;
-    int8_t *q = p.ws_xq + static_cast<int64_t>(m) * K;
-#pragma unroll
-    for (int i = 0; i < CPT; ++i) {
-        const int ch = threadIdx.x + kTokThreads * i;
-        if (ch < nch) {
-            float e[EPC];
-            Elt<InT>::unpack(c[i], e);
-            uint32_t w[EPC / 4];
-#pragma unroll
-            for (int j = 0; j < EPC / 4; ++j) {
-                w[j] = pack_codes4(fmaf(e[4 * j], fac, kRoundMagic), fmaf(e[4 * j + 1], fac, kRoundMagic),
-                                   fmaf(e[4 * j + 2], fac, kRoundMagic), fmaf(e[4 * j + 3], fac, kRoundMagic));
-                isum = dp4a_ss(w[j], 0x01010101u, isum);
-            }
-            if constexpr (EPC == 8)
-                *reinterpret_cast<uint2 *>(q + ch * 8) = make_uint2(w[0], w[1]);
-            else
-                *reinterpret_cast<uint32_t *>(q + ch * 4) = w[0];
-        }
-    }
-    isum = warp_sum_i(isum);
-    if (lane == 0) redi[warp] = isum;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int tot = 0;
-#pragma unroll
-        for (int w = 0; w < kTokThreads / 32; ++w) tot += redi[w];
-        p.ws_scale[m] = scale;
-        p.ws_rowsum[m] = tot;
-    }
-}
 
 template <typename OutT>
 __device__ __forceinline__ void store_out(void *out, int64_t i, float v) {
@@ -1176,6 +1096,251 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_w2a8_mma_kernel(const D
     }
 }
 
+// 2..16 tokens in one launch.  One CTA per SM over a range of output rows (as
+// decode_w2a8_mma_kernel), 16 warps; the tokens are quantized inside the
+// launch, every CTA quantizing all of them (M x K activations, read from L2):
+// with TOK = 4, 8 or 16 token slots, warp w takes part w % (16 / TOK) of
+// token w / (16 / TOK); the partial statistics of a token's warps meet in
+// shared memory and are added in part order, so every CTA derives the same
+// code factor.  Weights: before the dependency wait only L2 prefetches of
+// this CTA's lines; after it, each warp loads its units (16 rows x 256 K)
+// into registers, all in flight while the tokens are quantized.  Warp w takes
+// the 256-wide K block w % G (G = K / 256) of row blocks w / G, w / G +
+// 16 / G, ..., so its token fragments are loaded from shared memory once;
+// masked mma.sync as decode_w2a8_mma_kernel (one or two token groups, tokens
+// >= M read as zero), partial row sums added in shared memory, then the
+// epilogue.
+constexpr int kF4Threads = 512;
+constexpr int kF4Warps = kF4Threads / 32;
+constexpr int kF4Units = 5;  // 16-row units per warp held in registers
+
+template <int KK, int TOK>
+struct F4Layout {
+    static constexpr int kG = KK / 256;                     // 256-wide K blocks
+    static constexpr int kRBS = kF4Warps / kG;              // row-block stride of a warp
+    static constexpr int kMaxRows = 16 * kF4Units * kRBS;   // rows per CTA
+    static constexpr int kPitch = KK + 16;                  // padded token rows
+    static constexpr int kOffAcc = TOK * kPitch;            // [rows][TOK] partial row sums
+    static constexpr int kOffStat = kOffAcc + kMaxRows * TOK * 4;     // [warp] (sum x^2, max|x|)
+    static constexpr int kOffRs = kOffStat + kF4Warps * 8;            // [warp] code sums
+    static constexpr int kOffScale = kOffRs + kF4Warps * 4;           // [token] act_scale
+    static constexpr int kBytes = kOffScale + TOK * 4;
+};
+
+template <int KK, int TOK, typename InT>
+__global__ void __launch_bounds__(kF4Threads, 1) decode_w2a8_fused_kernel(const DecodeArgs p) {
+    using L = F4Layout<KK, TOK>;
+    constexpr int EPC = Elt<InT>::kPerChunk;
+    constexpr int NH = TOK > 8 ? 2 : 1;        // token groups of eight
+    constexpr int WPT = kF4Warps / TOK;        // warps per token
+    constexpr int KP = KK / WPT;               // a warp's part of a token
+    constexpr int XC = KP / EPC / 32;          // 16-byte activation chunks per lane
+    constexpr int XR = XC <= 8 ? XC : 8;       // of them held in registers at once (more: read twice)
+    constexpr int G = L::kG, RBS = L::kRBS;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int M = p.M;
+    int8_t *xs = reinterpret_cast<int8_t *>(smem);
+    int *rowacc = reinterpret_cast<int *>(smem + L::kOffAcc);
+    float *s_stat = reinterpret_cast<float *>(smem + L::kOffStat);
+    int *s_rs = reinterpret_cast<int *>(smem + L::kOffRs);
+    float *s_scale = reinterpret_cast<float *>(smem + L::kOffScale);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const RowRange rr = row_range(p.N);
+    const int R = rr.rows, nrb = (R + 15) / 16;
+    constexpr int wpr = KK / 16;  // packed words per row
+    const uint32_t *wrow = p.wpacked + static_cast<int64_t>(rr.begin) * wpr;
+    const int kb = warp % G, rb0 = warp / G;
+
+    // before the dependency wait: L2 prefetches of this CTA's weight lines
+    // (nothing is consumed) and shared-memory set-up
+    for (int l = threadIdx.x; l < R * (wpr / 32); l += kF4Threads) prefetch_l2(wrow + 32 * l);
+    for (int i = threadIdx.x; i < R * TOK; i += kF4Threads) rowacc[i] = 0;
+    pdl_wait();  // x, the weights and w_scale may come from the kernels before
+    pdl_launch_dependents();
+
+    // this warp's part of its token, then its weight units
+    const int tok = warp / WPT, part = warp % WPT;
+    const bool tokw = tok < M;
+    const uint4 *xv =
+        reinterpret_cast<const uint4 *>(static_cast<const InT *>(p.x) + static_cast<int64_t>(tok) * KK + part * KP);
+    uint4 xc[XR];
+    if (tokw) {
+#pragma unroll
+        for (int j = 0; j < XR; ++j) xc[j] = __ldg(xv + lane + 32 * j);
+    }
+    uint4 wa[kF4Units], wb[kF4Units];
+#pragma unroll
+    for (int i = 0; i < kF4Units; ++i) {
+        const int r0 = (rb0 + RBS * i) * 16 + g, r1 = r0 + 8;
+        const uint32_t *base = wrow + 16 * kb + 4 * t;
+        wa[i] = r0 < R ? __ldcs(reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(r0) * wpr))
+                       : make_uint4(0u, 0u, 0u, 0u);
+        wb[i] = r1 < R ? __ldcs(reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(r1) * wpr))
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const float gamma = __ldg(p.w_scale);
+
+    // partial statistics of the part
+    if (tokw) {
+        float ss0 = 0.f, ss1 = 0.f, amax = 0.f;
+#pragma unroll
+        for (int b = 0; b < XC; b += XR) {
+            if (b > 0) {
+#pragma unroll
+                for (int j = 0; j < XR; ++j) xc[j] = __ldg(xv + lane + 32 * (b + j));
+            }
+#pragma unroll
+            for (int j = 0; j < XR; ++j) {
+                float f[EPC];
+                Elt<InT>::unpack(xc[j], f);
+#pragma unroll
+                for (int e = 0; e < EPC; e += 2) {
+                    ss0 = fmaf(f[e], f[e], ss0);
+                    ss1 = fmaf(f[e + 1], f[e + 1], ss1);
+                    amax = fmaxf(amax, fmaxf(fabsf(f[e]), fabsf(f[e + 1])));
+                }
+            }
+        }
+        const float ss = warp_sum_f(ss0 + ss1);
+        amax = warp_max_f(amax);
+        if (lane == 0) {
+            s_stat[2 * warp] = ss;
+            s_stat[2 * warp + 1] = amax;
+        }
+    }
+    __syncthreads();
+
+    // the token's statistics (parts added in order), codes of the part into
+    // shared memory (and the workspace, CTA 0)
+    if (tokw) {
+        float ss = 0.f, amax = 0.f;
+#pragma unroll
+        for (int c = 0; c < WPT; ++c) {
+            ss += s_stat[2 * (WPT * tok + c)];
+            amax = fmaxf(amax, s_stat[2 * (WPT * tok + c) + 1]);
+        }
+        float fac, scale;
+        quant_row_factor(ss, amax, KK, p.eps, fac, scale);
+        int8_t *xrow = xs + tok * L::kPitch;
+        int8_t *wsrow = blockIdx.x == 0 ? p.ws_xq + static_cast<int64_t>(tok) * KK : nullptr;
+        int isum = 0;
+#pragma unroll
+        for (int j = 0; j < XC; ++j) {
+            const int c = part * (KP / EPC) + lane + 32 * j;  // chunk of EPC activations in the token
+            if (XC > XR && j % XR == 0) {                     // read again (from L1)
+#pragma unroll
+                for (int i = 0; i < XR; ++i) xc[i] = __ldg(xv + lane + 32 * (j + i));
+            }
+            float e[EPC];
+            Elt<InT>::unpack(xc[j % XR], e);
+            uint32_t w[EPC / 4];
+#pragma unroll
+            for (int i = 0; i < EPC / 4; ++i) {
+                w[i] = pack_codes4(fmaf(e[4 * i], fac, kRoundMagic), fmaf(e[4 * i + 1], fac, kRoundMagic),
+                                   fmaf(e[4 * i + 2], fac, kRoundMagic), fmaf(e[4 * i + 3], fac, kRoundMagic));
+                isum = dp4a_ss(w[i], 0x01010101u, isum);
+            }
+            if constexpr (EPC == 8) {
+                *reinterpret_cast<uint2 *>(xrow + xchunk_swz(c >> 1) * 16 + (c & 1) * 8) = make_uint2(w[0], w[1]);
+                if (wsrow) *reinterpret_cast<uint2 *>(wsrow + 8 * c) = make_uint2(w[0], w[1]);
+            } else {
+                *reinterpret_cast<uint32_t *>(xrow + xchunk_swz(c >> 2) * 16 + (c & 3) * 4) = w[0];
+                if (wsrow) *reinterpret_cast<uint32_t *>(wsrow + 4 * c) = w[0];
+            }
+        }
+        isum = warp_sum_i(isum);
+        if (lane == 0) {
+            s_rs[warp] = isum;
+            if (part == 0) s_scale[tok] = scale;
+        }
+    }
+    __syncthreads();  // the codes are in shared memory
+
+    // this warp's B fragments (K block kb; tokens >= M read as zero)
+    uint4 bx[2][NH][2];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+        const int c0 = 16 * kb + 4 * t + 2 * s;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+            const int tb = g + 8 * h;
+            bx[s][h][0] = bx[s][h][1] = make_uint4(0u, 0u, 0u, 0u);
+            if (tb < M) {
+                bx[s][h][0] = *reinterpret_cast<const uint4 *>(xs + tb * L::kPitch + xchunk_swz(c0) * 16);
+                bx[s][h][1] = *reinterpret_cast<const uint4 *>(xs + tb * L::kPitch + xchunk_swz(c0 + 1) * 16);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kF4Units; ++i) {
+        const int rb = rb0 + RBS * i;
+        if (rb < nrb) {
+            int acc[NH][4][4];
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[h][j][0] = acc[h][j][1] = acc[h][j][2] = acc[h][j][3] = 0;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const uint32_t w0 = s ? wa[i].z : wa[i].x, w1 = s ? wa[i].w : wa[i].y;
+                const uint32_t v0 = s ? wb[i].z : wb[i].x, v1 = s ? wb[i].w : wb[i].y;
+#pragma unroll
+                for (int h = 0; h < NH; ++h) {
+                    const uint32_t b0[4] = {bx[s][h][0].x, bx[s][h][0].y, bx[s][h][0].z, bx[s][h][0].w};
+                    const uint32_t b1[4] = {bx[s][h][1].x, bx[s][h][1].y, bx[s][h][1].z, bx[s][h][1].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t mk = 0x03030303u << (2 * j);
+                        const uint32_t a[4] = {w0 & mk, v0 & mk, w1 & mk, v1 & mk};
+                        mma_u8s8_16832(acc[h][j], a, b0[j], b1[j]);
+                    }
+                }
+            }
+            const int r0 = rb * 16 + g, r1 = r0 + 8;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                int v[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    v[c] = acc[h][0][c] + (acc[h][1][c] >> 2) + (acc[h][2][c] >> 4) + (acc[h][3][c] >> 6);
+                const int m0 = 2 * t + 8 * h, m1 = m0 + 1;
+                if (r0 < R && m0 < M) atomicAdd(&rowacc[r0 * TOK + m0], v[0]);
+                if (r0 < R && m1 < M) atomicAdd(&rowacc[r0 * TOK + m1], v[1]);
+                if (r1 < R && m0 < M) atomicAdd(&rowacc[r1 * TOK + m0], v[2]);
+                if (r1 < R && m1 < M) atomicAdd(&rowacc[r1 * TOK + m1], v[3]);
+            }
+        }
+    }
+    __syncthreads();
+
+    // epilogue: out = ((acc - rowsum) * act_scale) * gamma (+ bias), rows fastest
+    for (int e = threadIdx.x; e < R * M; e += kF4Threads) {
+        const int m = e / R, r = e - m * R;
+        int rs = 0;
+#pragma unroll
+        for (int c = 0; c < WPT; ++c) rs += s_rs[WPT * m + c];
+        const int n = rr.begin + r;
+        float o = __fmul_rn(__fmul_rn(static_cast<float>(rowacc[r * TOK + m] - rs), s_scale[m]), gamma);
+        if (p.bias) o = __fadd_rn(o, __ldg(p.bias + n));
+        const int64_t oi = static_cast<int64_t>(m) * p.N + n;
+        if (p.out_dtype == BQ_F32)
+            store_out<float>(p.out, oi, o);
+        else if (p.out_dtype == BQ_F16)
+            store_out<__half>(p.out, oi, o);
+        else
+            store_out<__nv_bfloat16>(p.out, oi, o);
+    }
+    if (blockIdx.x == 0 && threadIdx.x < M) {
+        const int m = threadIdx.x;
+        int rs = 0;
+#pragma unroll
+        for (int c = 0; c < WPT; ++c) rs += s_rs[WPT * m + c];
+        p.ws_scale[m] = s_scale[m];
+        p.ws_rowsum[m] = rs;
+    }
+}
+
 cudaError_t launch_pdl_cfg(const void *kern, const DecodeArgs &a, int grid, int threads, int smem, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -1189,25 +1354,6 @@ cudaError_t launch_pdl_cfg(const void *kern, const DecodeArgs &a, int grid, int 
     cfg.numAttrs = 1;
     void *args[] = {const_cast<DecodeArgs *>(&a)};
     return cudaLaunchKernelExC(&cfg, kern, args);
-}
-
-template <int MT, int KBW, typename InT>
-cudaError_t launch_mma_t(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
-    auto kern = decode_w2a8_mma_kernel<MT, KBW>;
-    const int smem = MmaLayout<MT, KBW>::bytes(a.K);
-    static SmemOptIn opt_in;
-    cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
-    if (e != cudaSuccess) return e;
-    e = launch_pdl_cfg(reinterpret_cast<const void *>(decode_token_quant_kernel<InT>), a, a.M, kTokThreads, 0, s);
-    if (e != cudaSuccess) return e;
-    return launch_pdl_cfg(reinterpret_cast<const void *>(kern), a, grid, kMmaThreads, smem, s);
-}
-
-template <typename InT>
-cudaError_t launch_mma(const DecodeArgs &a, const DevInfo &dev, cudaStream_t s, int grid) {
-    const bool two = a.M > 8;
-    if (a.K == 2048) return two ? launch_mma_t<16, 1, InT>(a, dev, s, grid) : launch_mma_t<8, 1, InT>(a, dev, s, grid);
-    return two ? launch_mma_t<16, 2, InT>(a, dev, s, grid) : launch_mma_t<8, 2, InT>(a, dev, s, grid);
 }
 
 template <int MT, bool MMA, typename InT, typename OutT>
@@ -1261,6 +1407,37 @@ int grid_of(int64_t N, const DevInfo &dev) { return static_cast<int>(std::min<in
 int rows_per_cta(int64_t N, const DevInfo &dev) {
     const int64_t G = grid_of(N, dev);
     return static_cast<int>((N + G - 1) / G);
+}
+
+template <int KK, int TOK, typename InT>
+cudaError_t launch_fused_t(const DecodeArgs &a, const DevInfo &dev, int grid, cudaStream_t s) {
+    auto kern = decode_w2a8_fused_kernel<KK, TOK, InT>;
+    constexpr int smem = F4Layout<KK, TOK>::kBytes;
+    static SmemOptIn opt_in;
+    const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_pdl_cfg(reinterpret_cast<const void *>(kern), a, grid, kF4Threads, smem, s);
+}
+
+// Shapes of the one-launch kernel: 2..16 tokens, K = 2048 or 4096, every
+// unit of a warp in registers.
+bool fused_supported(int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
+    if (M < 2 || M > 16 || (K != 2048 && K != 4096)) return false;
+    const int64_t max_rows = K == 2048 ? F4Layout<2048, 4>::kMaxRows : F4Layout<4096, 4>::kMaxRows;
+    return rows_per_cta(N, dev) <= max_rows;
+}
+
+template <int KK, typename InT>
+cudaError_t launch_fused_k(const DecodeArgs &a, const DevInfo &dev, int grid, cudaStream_t s) {
+    if (a.M <= 4) return launch_fused_t<KK, 4, InT>(a, dev, grid, s);
+    if (a.M <= 8) return launch_fused_t<KK, 8, InT>(a, dev, grid, s);
+    return launch_fused_t<KK, 16, InT>(a, dev, grid, s);
+}
+
+template <typename InT>
+cudaError_t launch_fused(const DecodeArgs &a, const DevInfo &dev, int grid, cudaStream_t s) {
+    if (a.K == 2048) return launch_fused_k<2048, InT>(a, dev, grid, s);
+    return launch_fused_k<4096, InT>(a, dev, grid, s);
 }
 
 // Shapes of the register-streaming kernel: one token, 256 % (K/64) == 0
@@ -1342,7 +1519,7 @@ cudaError_t launch_decode_mma_from_codes(const int8_t *xq, const float *act_scal
 }
 
 int decode_w2a8_kind(int64_t M, int64_t N, int64_t K, bq_dtype xt, const DevInfo &dev) {
-    if (mma_stream_supported(M, N, K, dev)) return BQ_PATH_DECODE_MMA;
+    if (fused_supported(M, N, K, dev)) return BQ_PATH_DECODE_MMA;
     if (stream_supported(M, N, K, xt, dev)) return BQ_PATH_DECODE_STREAM;
     return BQ_PATH_DECODE_SMEM;
 }
@@ -1372,8 +1549,8 @@ cudaError_t launch_decode_w2a8(const void *x, bq_dtype xt, int64_t M, int64_t K,
     a.out_dtype = out_dtype;
     const int kind = decode_w2a8_kind(M, N, K, xt, dev);
     if (kind == BQ_PATH_DECODE_MMA) {
-        if (xt == BQ_BF16) return launch_mma<__nv_bfloat16>(a, dev, s, grid);
-        return launch_mma<float>(a, dev, s, grid);
+        if (xt == BQ_BF16) return launch_fused<__nv_bfloat16>(a, dev, grid, s);
+        return launch_fused<float>(a, dev, grid, s);
     }
     if (kind == BQ_PATH_DECODE_STREAM) {
         if (xt == BQ_BF16) return launch_stream_out<__nv_bfloat16>(a, out_dtype, static_cast<int>(M), s, grid);

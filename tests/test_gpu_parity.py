@@ -322,9 +322,10 @@ def test_bitlinear_decode_ragged(M, N, K, out, bias):
 
 
 # one token: dp4a register-streaming kernel (fp32 and bf16 inputs, K = 2048 / 8192,
-# fewer rows than SMs); 2..16 tokens: mma.sync register-streaming kernel
-# (K = 2048 / 4096, one or two token groups, up to 80 rows per CTA, fewer rows
-# than SMs) and, past its row limit, the shared-memory kernel
+# fewer rows than SMs); 2..4 tokens: the one-launch mma.sync kernel; 5..16
+# tokens: the two-launch mma.sync kernel (K = 2048 / 4096, one or two token
+# groups, up to 80 rows per CTA, fewer rows than SMs) and, past its row limit,
+# the shared-memory kernel
 @pytest.mark.parametrize("M,N,K,out,bias,xin", [(1, 300, 2048, "f32", True, "f32"), (1, 100, 4096, "f16", True, "bf16"),
                                                 (1, 5000, 8192, "bf16", False, "bf16"),
                                                 (2, 1000, 4096, "bf16", True, "bf16"),
@@ -333,7 +334,8 @@ def test_bitlinear_decode_ragged(M, N, K, out, bias):
                                                 (9, 150, 2048, "bf16", False, "bf16"), (16, 11900, 4096, "bf16", True, "f32"),
                                                 (16, 11008, 4096, "bf16", True, "f32"), (8, 4096, 4096, "f16", False, "f32"),
                                                 (3, 40, 4096, "bf16", True, "bf16"), (16, 11840, 4096, "f32", False, "bf16"),
-                                                (7, 8000, 2048, "bf16", True, "bf16")])
+                                                (7, 8000, 2048, "bf16", True, "bf16"), (4, 3000, 2048, "f16", True, "f32"),
+                                                (2, 11840, 4096, "bf16", False, "f32")])
 def test_bitlinear_decode_stream_shapes(M, N, K, out, bias, xin):
     g = synth.rng((110, M, N, K))
     if xin == "bf16":

@@ -1,10 +1,11 @@
 """Stream order of the weight-streaming decode kernels.
 
-The decode kernels (one to sixteen tokens, RMSNorm or LayerNorm normaliser)
-issue their weight loads before their dependency wait.  That is correct only
-because the kernel launched ahead of them in the same call (the token or
-LayerNorm quantizer) waits for everything earlier in the stream before it
-releases them.  Here the packed weights are rewritten in place by the packing
+The one-launch decode kernels (RMSNorm at one to sixteen tokens, LayerNorm at
+one token) read nothing before their dependency wait but prefetch their
+weights into L2 there; the LayerNorm decode at 2..16 tokens issues its weight
+loads before its wait, which is correct only because the LayerNorm quantizer
+launched ahead of it in the same call waits for everything earlier in the
+stream before it releases it.  Here the packed weights are rewritten in place by the packing
 kernel on the same stream directly before each call, with a different weight
 matrix each time and no host synchronisation in between; every output must be
 bit-identical to the same call made after a full synchronisation (the same
@@ -40,7 +41,7 @@ def _call(ln, x, wp, ws, lw, lb, out):
     return bq.bq_bitlinear_w2a8(x, wp, ws, N, None, 1e-5, torch.bfloat16, out=out)
 
 
-@pytest.mark.parametrize("M,ln", [(1, False), (4, False), (16, False), (1, True), (4, True)])
+@pytest.mark.parametrize("M,ln", [(1, False), (4, False), (16, False), (1, True), (4, True), (16, True)])
 def test_weights_packed_just_before_the_call(M, ln):
     dev = "cuda"
     # three different weight matrices, each scaled differently so that a stale read changes every output
