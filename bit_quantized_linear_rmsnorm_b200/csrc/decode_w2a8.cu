@@ -1110,29 +1110,29 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_w2a8_mma_kernel(const D
 // masked mma.sync as decode_w2a8_mma_kernel (one or two token groups, tokens
 // >= M read as zero), partial row sums added in shared memory, then the
 // epilogue.
-constexpr int kF4Threads = 512;
-constexpr int kF4Warps = kF4Threads / 32;
-constexpr int kF4Units = 5;  // 16-row units per warp held in registers
+constexpr int kFusedThreads = 512;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kFusedUnits = 5;  // 16-row units per warp held in registers
 
 template <int KK, int TOK>
-struct F4Layout {
+struct FusedLayout {
     static constexpr int kG = KK / 256;                     // 256-wide K blocks
-    static constexpr int kRBS = kF4Warps / kG;              // row-block stride of a warp
-    static constexpr int kMaxRows = 16 * kF4Units * kRBS;   // rows per CTA
+    static constexpr int kRBS = kFusedWarps / kG;              // row-block stride of a warp
+    static constexpr int kMaxRows = 16 * kFusedUnits * kRBS;   // rows per CTA
     static constexpr int kPitch = KK + 16;                  // padded token rows
     static constexpr int kOffAcc = TOK * kPitch;            // [rows][TOK] partial row sums
     static constexpr int kOffStat = kOffAcc + kMaxRows * TOK * 4;     // [warp] (sum x^2, max|x|)
-    static constexpr int kOffRs = kOffStat + kF4Warps * 8;            // [warp] code sums
-    static constexpr int kOffScale = kOffRs + kF4Warps * 4;           // [token] act_scale
+    static constexpr int kOffRs = kOffStat + kFusedWarps * 8;            // [warp] code sums
+    static constexpr int kOffScale = kOffRs + kFusedWarps * 4;           // [token] act_scale
     static constexpr int kBytes = kOffScale + TOK * 4;
 };
 
 template <int KK, int TOK, typename InT>
-__global__ void __launch_bounds__(kF4Threads, 1) decode_w2a8_fused_kernel(const DecodeArgs p) {
-    using L = F4Layout<KK, TOK>;
+__global__ void __launch_bounds__(kFusedThreads, 1) decode_w2a8_fused_kernel(const DecodeArgs p) {
+    using L = FusedLayout<KK, TOK>;
     constexpr int EPC = Elt<InT>::kPerChunk;
     constexpr int NH = TOK > 8 ? 2 : 1;        // token groups of eight
-    constexpr int WPT = kF4Warps / TOK;        // warps per token
+    constexpr int WPT = kFusedWarps / TOK;        // warps per token
     constexpr int KP = KK / WPT;               // a warp's part of a token
     constexpr int XC = KP / EPC / 32;          // 16-byte activation chunks per lane
     constexpr int XR = XC <= 8 ? XC : 8;       // of them held in registers at once (more: read twice)
@@ -1154,8 +1154,8 @@ __global__ void __launch_bounds__(kF4Threads, 1) decode_w2a8_fused_kernel(const 
 
     // before the dependency wait: L2 prefetches of this CTA's weight lines
     // (nothing is consumed) and shared-memory set-up
-    for (int l = threadIdx.x; l < R * (wpr / 32); l += kF4Threads) prefetch_l2(wrow + 32 * l);
-    for (int i = threadIdx.x; i < R * TOK; i += kF4Threads) rowacc[i] = 0;
+    for (int l = threadIdx.x; l < R * (wpr / 32); l += kFusedThreads) prefetch_l2(wrow + 32 * l);
+    for (int i = threadIdx.x; i < R * TOK; i += kFusedThreads) rowacc[i] = 0;
     pdl_wait();  // x, the weights and w_scale may come from the kernels before
     pdl_launch_dependents();
 
@@ -1169,9 +1169,9 @@ __global__ void __launch_bounds__(kF4Threads, 1) decode_w2a8_fused_kernel(const 
 #pragma unroll
         for (int j = 0; j < XR; ++j) xc[j] = __ldg(xv + lane + 32 * j);
     }
-    uint4 wa[kF4Units], wb[kF4Units];
+    uint4 wa[kFusedUnits], wb[kFusedUnits];
 #pragma unroll
-    for (int i = 0; i < kF4Units; ++i) {
+    for (int i = 0; i < kFusedUnits; ++i) {
         const int r0 = (rb0 + RBS * i) * 16 + g, r1 = r0 + 8;
         const uint32_t *base = wrow + 16 * kb + 4 * t;
         wa[i] = r0 < R ? __ldcs(reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(r0) * wpr))
@@ -1273,7 +1273,7 @@ __global__ void __launch_bounds__(kF4Threads, 1) decode_w2a8_fused_kernel(const 
         }
     }
 #pragma unroll
-    for (int i = 0; i < kF4Units; ++i) {
+    for (int i = 0; i < kFusedUnits; ++i) {
         const int rb = rb0 + RBS * i;
         if (rb < nrb) {
             int acc[NH][4][4];
@@ -1315,7 +1315,7 @@ __global__ void __launch_bounds__(kF4Threads, 1) decode_w2a8_fused_kernel(const 
     __syncthreads();
 
     // epilogue: out = ((acc - rowsum) * act_scale) * gamma (+ bias), rows fastest
-    for (int e = threadIdx.x; e < R * M; e += kF4Threads) {
+    for (int e = threadIdx.x; e < R * M; e += kFusedThreads) {
         const int m = e / R, r = e - m * R;
         int rs = 0;
 #pragma unroll
@@ -1412,18 +1412,18 @@ int rows_per_cta(int64_t N, const DevInfo &dev) {
 template <int KK, int TOK, typename InT>
 cudaError_t launch_fused_t(const DecodeArgs &a, const DevInfo &dev, int grid, cudaStream_t s) {
     auto kern = decode_w2a8_fused_kernel<KK, TOK, InT>;
-    constexpr int smem = F4Layout<KK, TOK>::kBytes;
+    constexpr int smem = FusedLayout<KK, TOK>::kBytes;
     static SmemOptIn opt_in;
     const cudaError_t e = smem_opt_in(opt_in, dev, reinterpret_cast<const void *>(kern), static_cast<size_t>(smem));
     if (e != cudaSuccess) return e;
-    return launch_pdl_cfg(reinterpret_cast<const void *>(kern), a, grid, kF4Threads, smem, s);
+    return launch_pdl_cfg(reinterpret_cast<const void *>(kern), a, grid, kFusedThreads, smem, s);
 }
 
 // Shapes of the one-launch kernel: 2..16 tokens, K = 2048 or 4096, every
 // unit of a warp in registers.
 bool fused_supported(int64_t M, int64_t N, int64_t K, const DevInfo &dev) {
     if (M < 2 || M > 16 || (K != 2048 && K != 4096)) return false;
-    const int64_t max_rows = K == 2048 ? F4Layout<2048, 4>::kMaxRows : F4Layout<4096, 4>::kMaxRows;
+    const int64_t max_rows = K == 2048 ? FusedLayout<2048, 4>::kMaxRows : FusedLayout<4096, 4>::kMaxRows;
     return rows_per_cta(N, dev) <= max_rows;
 }
 
